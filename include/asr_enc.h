@@ -1,0 +1,199 @@
+/*
+ * asr_enc.h -- C ABI of the B200 (sm_100a) ASR audio-encoder forward pass.
+ *
+ * The operation: 16 kHz mono PCM -> log-mel -> conv stem -> pre-LN
+ * transformer tower with windowed (block-diagonal) or full attention ->
+ * encoder head -> SwiGLU adapter, as described by
+ *   "MOSS-Transcribe-preview-2B-GGUF", Architecture table (rows "Audio
+ *   encoder", "Conv front-end", "Encoder head", "Adapter", "Audio") and
+ *   Non-obvious gotchas (trailing STFT frame dropped: n_samples/hop frames);
+ * and, for the full-attention variant with a Conv1D stem, by
+ *   "CrisperWhisper -> ONNX (with cross-attentions)", What this exports
+ *   instead (whisper-small geometry) and Results (1500 encoder frames per
+ *   30 s window).
+ *
+ * Conventions for every entry point:
+ *   - Plain C types only.  Device pointers are CUDA device addresses on the
+ *     current device; `stream` is a cudaStream_t passed as void* (NULL = the
+ *     legacy default stream).
+ *   - Nothing is thrown across the ABI; each call returns an asr_status.
+ *     On failure, asr_enc_last_error() returns a message (per handle, or the
+ *     process-wide one when the handle is NULL).
+ *   - Calls are asynchronous with respect to the host unless stated; the
+ *     library synchronises only where a call says it reads device memory
+ *     back (asr_enc_sync_status, asr_enc_forward_host).
+ *   - The caller owns every buffer it passes.  The handle owns the repacked
+ *     weights it obtained through the caller's allocator at create time.
+ */
+#ifndef ASR_ENC_H
+#define ASR_ENC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+#if defined(__GNUC__)
+#pragma GCC visibility push(default)
+#endif
+
+typedef struct asr_enc asr_enc; /* opaque, library-owned */
+
+typedef enum {
+  ASR_OK = 0,
+  ASR_E_INVAL = 1,          /* bad argument: NULL pointer, bad geometry or size */
+  ASR_E_UNSUPPORTED = 2,    /* well-formed but outside what this build implements */
+  ASR_E_NOMEM = 3,          /* the allocator callback returned NULL */
+  ASR_E_CUDA = 4,           /* a CUDA runtime/driver call failed (message has the name) */
+  ASR_E_WORKSPACE = 5,      /* workspace NULL or smaller than asr_enc_workspace_size() */
+  ASR_E_DEVICE_TIMEOUT = 6  /* a bounded device-side wait gave up (see asr_enc_sync_status) */
+} asr_status;
+
+enum { ASR_STEM_CONV2D_CHUNKED = 0, ASR_STEM_CONV1D = 1 };
+enum { ASR_POS_PER_CHUNK = 0, ASR_POS_GLOBAL = 1 };
+enum { ASR_DTYPE_BF16 = 0, ASR_DTYPE_F32 = 1 };
+
+/* Encoder geometry.  Field meanings:
+ *  stem           ASR_STEM_CONV2D_CHUNKED: 3 x Conv2D k3 s2 p1 (1->C->C->C) + GELU
+ *                 applied per chunk of chunk_frames mel frames, then conv_out
+ *                 (C*n_mels/8 -> d_model, no bias) ("Conv front-end" row).
+ *                 ASR_STEM_CONV1D: Conv1D k3 s1 p1 (n_mels->d) + GELU, Conv1D
+ *                 k3 s2 p1 (d->d) + GELU (whisper-small geometry).
+ *  n_mels, n_fft, hop   128|80, 400, 160 ("Audio" row).  Only n_fft 400 / hop 160.
+ *  chunk_frames   100 (conv2d stem only; 0 otherwise).
+ *  conv_ch        Conv2D channels C (480); ignored by the Conv1D stem.
+ *  d_model, n_heads, head_dim, d_ffn, n_layers   tower shape; head_dim must be 64.
+ *  window_tokens  attention window in tokens (104); 0 = full attention per clip.
+ *  pos_mode       ASR_POS_PER_CHUNK (positions restart each chunk) or ASR_POS_GLOBAL.
+ *  proj1_out, proj2_out        encoder head widths; 0 = absent (final LN only).
+ *  adapter_hidden, adapter_out SwiGLU adapter widths; 0 = absent.
+ *  ln_eps         LayerNorm epsilon.
+ *  dtype          ASR_DTYPE_BF16 (bf16 weights) or ASR_DTYPE_F32 (fp32 weights).
+ */
+typedef struct {
+  int stem;
+  int n_mels, n_fft, hop, chunk_frames;
+  int conv_ch, d_model, n_heads, head_dim, d_ffn, n_layers;
+  int window_tokens;
+  int pos_mode;
+  int proj1_out, proj2_out, adapter_hidden, adapter_out;
+  float ln_eps;
+  int dtype;
+} asr_geometry;
+
+/* Device allocator supplied by the caller (e.g. a PyTorch caching allocator).
+ * alloc returns a device pointer aligned to >= 256 bytes or NULL. */
+typedef void* (*asr_alloc_fn)(void* ctx, size_t bytes);
+typedef void (*asr_free_fn)(void* ctx, void* ptr);
+
+/* ---- weights ------------------------------------------------------------
+ * Weights are passed as an array of device pointers in a fixed name order.
+ * asr_enc_weight_count() gives the count; asr_enc_weight_info() the name,
+ * rank and shape of entry i.  Matrices are [out, in] row-major (torch Linear
+ * layout); Conv2D kernels [out, in, kh(freq), kw(time)]; Conv1D kernels
+ * [out, in, k]; biases and LayerNorm gain/shift are vectors.  Every tensor
+ * is of the geometry's dtype.  Order: conv1.w conv1.b conv2.w conv2.b
+ * [conv3.w conv3.b conv_out.w] then per layer l: ln1.g ln1.b q.w q.b k.w k.b
+ * v.w v.b o.w o.b ln2.g ln2.b fc1.w fc1.b fc2.w fc2.b, then ln_post.g
+ * ln_post.b [proj1.w proj1.b proj2.w proj2.b] [adapter.gate.w adapter.up.w
+ * adapter.down.w].  Returns -1 for an invalid geometry. */
+int asr_enc_weight_count(const asr_geometry* g);
+/* name: static string owned by the library; shape: up to 4 extents. */
+asr_status asr_enc_weight_info(const asr_geometry* g, int i, const char** name, int* ndim,
+                               int64_t shape[4]);
+
+/* ---- geometry queries (host only, bit-exact) ----------------------------- */
+
+/* Tokens per clip of n_samples: frames = n_samples/hop (trailing STFT frame
+ * dropped); conv2d stem: (frames/chunk_frames) * L3 with L3 the length of a
+ * chunk after three k3 s2 p1 convolutions (13 for 100 frames); conv1d stem:
+ * frames after k3 s1 p1 then k3 s2 p1 (n/320).  Returns -1 when n_samples is
+ * not a whole number of hops (conv2d: of chunks) or the geometry is invalid. */
+int64_t asr_enc_tokens(const asr_geometry* g, int64_t n_samples);
+
+/* Attention-window partition of a batch of `batch` clips of n_samples each,
+ * as cumulative token offsets cu[0..n] (int32, cu[0]=0, cu[n]=batch*tokens).
+ * Windows tile each clip from its first token in steps of window_tokens, the
+ * last one short; window_tokens==0 gives one window per clip.  *n is in/out:
+ * capacity of cu in entries on input (n+1 needed), window count on output.
+ * With cu==NULL only the count is returned. */
+asr_status asr_enc_windows(const asr_geometry* g, int64_t n_samples, int batch, int32_t* cu,
+                           int* n);
+
+/* ---- handle lifecycle ---------------------------------------------------- */
+
+/* Validate the geometry, then copy and repack the weights (fused QKV rows,
+ * permuted conv_out columns, conv kernels in tap-major/channel-minor order,
+ * fp32 bias and LayerNorm vectors) into device buffers obtained from
+ * `alloc` (cudaMalloc when alloc is NULL), and build the weight TMA
+ * descriptors.  `weights` points to asr_enc_weight_count(g) device pointers.
+ * Work is enqueued on `stream` and completed before return.
+ * Limits: n_fft 400, hop 160, head_dim 64, d_model % 64 == 0, d_ffn % 64 == 0,
+ * conv_ch % 8 == 0; otherwise ASR_E_UNSUPPORTED. */
+asr_status asr_enc_create(const asr_geometry* g, const void* const* weights, int n_weights,
+                          asr_alloc_fn alloc, asr_free_fn free_fn, void* alloc_ctx, void* stream,
+                          asr_enc** out);
+
+/* Release everything the handle owns (through free_fn).  NULL is a no-op.
+ * The caller must ensure no forward using the handle is still running. */
+void asr_enc_destroy(asr_enc* e);
+
+/* Bytes of workspace a forward of `batch` clips of n_samples needs
+ * (0 on invalid sizes). */
+size_t asr_enc_workspace_size(const asr_enc* e, int64_t n_samples, int batch);
+
+/* ---- forward ------------------------------------------------------------- */
+
+/* Run the whole forward on `stream`.
+ *  pcm         device float32 [batch, n_samples], row-major.
+ *  n_samples   per clip; must be a multiple of 16000 for the conv2d stem and
+ *              of 320 for the conv1d stem (ASR_E_UNSUPPORTED otherwise).
+ *  out         device float32 [batch, T, D_out], T = asr_enc_tokens(),
+ *              D_out = adapter_out, else proj2_out, else d_model.
+ *  out_tokens  optional host pointer; receives T.
+ *  workspace   device buffer of >= asr_enc_workspace_size() bytes,
+ *              256-byte aligned; the forward may overwrite all of it.
+ * Asynchronous.  Bounded device waits that give up set the handle's device
+ * status word; read it with asr_enc_sync_status(). */
+asr_status asr_enc_forward(asr_enc* e, const float* pcm, int64_t n_samples, int batch, float* out,
+                           int64_t* out_tokens, void* workspace, size_t ws_bytes, void* stream);
+
+/* Same as asr_enc_forward but with HOST buffers: copies pcm (host float32
+ * [batch, n_samples]; page-locked for full speed) into the workspace, runs
+ * the forward and copies the result back into host `out` ([batch, T,
+ * D_out]).  Synchronises `stream` and returns the device status. */
+asr_status asr_enc_forward_host(asr_enc* e, const float* pcm_host, int64_t n_samples, int batch,
+                                float* out_host, int64_t* out_tokens, void* workspace,
+                                size_t ws_bytes, void* stream);
+
+/* Synchronise the stream of the last forward and read the device status
+ * word: ASR_OK, or ASR_E_DEVICE_TIMEOUT if a bounded wait gave up. */
+asr_status asr_enc_sync_status(asr_enc* e);
+
+/* ---- per-stage taps (debug / parity) --------------------------------------
+ * With taps enabled (mask of 1<<stage), the forward also copies the listed
+ * stage tensors into the workspace (asr_enc_workspace_size grows
+ * accordingly), and asr_enc_tap copies the last forward's tensor to `dst`
+ * (device, float32) after checking dst_bytes.  Stages and shapes:
+ *  ASR_TAP_MEL      [batch, n_mels, n_samples/hop]  normalised log-mel
+ *  ASR_TAP_STEM     [batch*T, d_model]  after the stem and positions
+ *  ASR_TAP_LAYER0   [batch*T, d_model]  residual stream after layer 0
+ *  ASR_TAP_ENCODER  [batch*T, d_model]  after the last layer (before ln_post)
+ *  ASR_TAP_HEAD     [batch*T, proj2_out] head output (adapter input)
+ * The workspace must not be reused between the forward and the tap call. */
+enum { ASR_TAP_MEL = 0, ASR_TAP_STEM = 1, ASR_TAP_LAYER0 = 2, ASR_TAP_ENCODER = 3, ASR_TAP_HEAD = 4,
+       ASR_TAP_COUNT = 5 };
+asr_status asr_enc_set_taps(asr_enc* e, unsigned mask);
+asr_status asr_enc_tap(asr_enc* e, int stage, float* dst, size_t dst_bytes, void* stream);
+
+/* Message of the last failure on `e` (or process-wide when e is NULL). */
+const char* asr_enc_last_error(const asr_enc* e);
+
+#if defined(__GNUC__)
+#pragma GCC visibility pop
+#endif
+#ifdef __cplusplus
+}
+#endif
+#endif /* ASR_ENC_H */

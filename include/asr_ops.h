@@ -1,0 +1,80 @@
+/*
+ * asr_ops.h -- kernel-level entry points of the ASR encoder library.
+ *
+ * Each call runs one stage of the forward pass with exactly the kernel that
+ * asr_enc_forward launches for it, on caller-owned device buffers, so that
+ * every stage can be checked on its own.  Conventions as in asr_enc.h
+ * (device pointers, stream as void*, asr_status return, asynchronous).
+ */
+#ifndef ASR_OPS_H
+#define ASR_OPS_H
+
+#include "asr_enc.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+#if defined(__GNUC__)
+#pragma GCC visibility push(default)
+#endif
+
+/* Log-mel front-end of a batch of clips ("MOSS-Transcribe-preview-2B-GGUF",
+ * Architecture "Audio" row; Non-obvious gotchas on the trailing frame):
+ * periodic Hann(400), centred reflect-padded frames every 160 samples,
+ * |DFT|^2 of 201 bins, trailing frame dropped, Slaney mel filterbank (0-8 kHz),
+ * log10(max(., 1e-10)), clamp at (clip max - 8), then (x + 4) / 4.
+ *  pcm   device float32 [batch, n_samples]; n_samples % 160 == 0, > 200.
+ *  mel   device float32 [batch, n_mels, n_samples/160] (normalised).
+ *  ws    device scratch of >= asr_op_log_mel_ws_size(batch) bytes.
+ * n_mels: 1..128. */
+size_t asr_op_log_mel_ws_size(int batch);
+asr_status asr_op_log_mel(const float* pcm, int64_t n_samples, int batch, int n_mels, float* mel,
+                          void* ws, size_t ws_bytes, void* stream);
+
+/* Dense layer on the tcgen05 GEMM engine: acc = X W^T (fp32 accumulate in
+ * tensor memory), then the epilogue.
+ *  x     device bf16 [M, K] row-major;  w  device bf16 [N, K] row-major.
+ *  bias  device float32 [N] or NULL.
+ *  epi   ASR_EPI_BF16       y bf16 [M, N] = acc + bias
+ *        ASR_EPI_BF16_GELU  y bf16 [M, N] = GELU(acc + bias)      (exact erf)
+ *        ASR_EPI_F32_RESID  y f32  [M, N] += acc + bias           (in place)
+ *        ASR_EPI_F32        y f32  [M, N] = acc + bias
+ *        ASR_EPI_SWIGLU     y bf16 [M, N/2]: W rows interleaved in blocks of
+ *                           16 (gate rows 16j..16j+15, then the matching up
+ *                           rows), y[:, 16j+i] = SiLU(gate) * up
+ * Limits: K % 8 == 0, N % 16 == 0, M >= 1.  ws: device scratch of
+ * >= asr_op_linear_ws_size() bytes (device status word). */
+enum { ASR_EPI_BF16 = 0, ASR_EPI_BF16_GELU = 1, ASR_EPI_F32_RESID = 2, ASR_EPI_F32 = 3,
+       ASR_EPI_SWIGLU = 4 };
+size_t asr_op_linear_ws_size(void);
+asr_status asr_op_linear(const void* x, const void* w, const float* bias, int64_t M, int N, int K,
+                         int epi, void* y, void* ws, size_t ws_bytes, void* stream);
+
+/* LayerNorm over the last axis: y = (x - mean) / sqrt(var + eps) * g + b,
+ * x device float32 [M, D], g/b device float32 [D], y device bf16 [M, D]
+ * (out_f32 == 0) or float32 (out_f32 != 0).  D % 4 == 0, D <= 4096. */
+asr_status asr_op_layer_norm(const float* x, const float* g, const float* b, int64_t M, int D,
+                             float eps, void* y, int out_f32, void* stream);
+
+/* Windowed / full attention over segments: for each segment [cu[j], cu[j+1])
+ * and head h, softmax(Q K^T / 8) V, with Q, K, V read from
+ * qkv device bf16 [T, 3*H*64] (columns: q heads, k heads, v heads) and the
+ * result written to out device bf16 [T, H*64].  cu: device int32 [n_seg+1].
+ * max_seg: the longest segment (sizes the launch grid).  head_dim 64. */
+asr_status asr_op_attention(const void* qkv, const int32_t* cu, int n_seg, int max_seg, int64_t T,
+                            int H, void* out, void* stream);
+
+/* Bounded-wait self-check: launches one kernel that waits on a shared-memory
+ * barrier that nothing ever completes, gives up after limit_ns nanoseconds
+ * of device time, writes 1 to *status_dev (device int32) and returns
+ * normally.  It shows that a stalled device wait ends with a status the host
+ * can read while the CUDA context stays usable. */
+asr_status asr_op_wait_probe(int64_t limit_ns, int* status_dev, void* stream);
+
+#if defined(__GNUC__)
+#pragma GCC visibility pop
+#endif
+#ifdef __cplusplus
+}
+#endif
+#endif /* ASR_OPS_H */

@@ -38,7 +38,7 @@ from scipy.special import erf
 __all__ = [
     "hann_periodic", "frame_signal", "power_spectrum", "hz_to_mel_slaney", "mel_to_hz_slaney",
     "mel_filterbank", "log_mel", "conv2d", "conv1d", "gelu", "silu", "layer_norm", "sinusoids",
-    "token_count", "window_partition", "attention_windows", "attention_masked", "window_mask",
+    "linear", "token_count", "window_partition", "attention_windows", "attention_masked", "window_mask",
     "encoder_layer", "stem_conv2d_chunked", "stem_conv1d", "encode_tokens", "encode_clip", "forward",
     "as64",
 ]
@@ -355,11 +355,16 @@ def attention_masked(q, k, v, mask, n_heads: int) -> np.ndarray:
 # Layers.
 # --------------------------------------------------------------------------
 
-def _lin(x, W, name, bias=True):
-    y = x @ as64(W[name + ".w"]).T
-    if bias:
-        y = y + as64(W[name + ".b"])
+def linear(x, w, b=None):
+    """y = x W^T + b with W [out, in] (torch Linear layout), in float64."""
+    y = np.asarray(x, np.float64) @ as64(w).T
+    if b is not None:
+        y = y + as64(b)
     return y
+
+
+def _lin(x, W, name, bias=True):
+    return linear(x, W[name + ".w"], W[name + ".b"] if bias else None)
 
 
 def encoder_layer(x: np.ndarray, W, l: int, geom, cu) -> np.ndarray:

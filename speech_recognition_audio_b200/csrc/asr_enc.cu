@@ -1,0 +1,937 @@
+// C ABI of the encoder library: geometry queries, weight repacking, the
+// workspace plan and the forward launch sequence.
+//
+// Forward of one batch (conv2d stem; "MOSS-Transcribe-preview-2B-GGUF",
+// Architecture table):
+//   log-mel -> conv1 (CUDA cores) -> conv2, conv3 (implicit GEMM, bias+GELU)
+//   -> conv_out (+ per-chunk sinusoidal positions) -> 32 x [LN1 -> QKV ->
+//   windowed attention -> out-proj + residual -> LN2 -> fc1 + GELU -> fc2 +
+//   residual] -> ln_post -> proj1 + GELU -> proj2 -> gate/up + SwiGLU -> down.
+// Conv1D stem (whisper-small geometry, "CrisperWhisper -> ONNX", What this
+// exports instead / Results): log-mel -> transpose -> conv1 (k3 s1) + GELU ->
+// conv2 (k3 s2) + GELU + global positions -> 12 layers with full attention
+// -> final LayerNorm.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/asr_enc.h"
+#include "../../include/asr_ops.h"
+#include "kernels.h"
+
+using namespace asr;
+
+namespace {
+
+std::mutex g_err_mu;
+std::string g_err = "";
+
+constexpr unsigned long long kWaitLimitNs = 2000ull * 1000 * 1000;  // 2 s per device wait
+
+struct LayerW {
+  GemmB qkv, o, fc1, fc2;
+  float *bqkv, *bo, *b1, *b2, *ln1g, *ln1b, *ln2g, *ln2b;
+};
+
+struct ActMaps {
+  const void* ws = nullptr;
+  int64_t n = 0;
+  int batch = 0;
+  unsigned taps = 0;
+  CUtensorMap h, att, ff, c3, p1, p2, gu;
+};
+
+struct Plan {
+  int64_t n = 0, Tc = 0, T = 0;
+  int B = 0, F = 0, nwin_clip = 0, nwin = 0, max_win = 0, chunks = 0;
+  int T1 = 0, F1 = 0, T2 = 0, F2 = 0, T3 = 0, F3 = 0;
+  size_t off_clipmax = 0, off_cu = 0, off_mel = 0, off_c1 = 0, off_c2 = 0, off_c3 = 0, off_melT = 0, off_x = 0,
+         off_h = 0, off_qkv = 0, off_att = 0, off_ff = 0, off_p1 = 0, off_p2 = 0, off_gu = 0, off_pcm = 0, off_out = 0;
+  size_t off_tap[ASR_TAP_COUNT] = {0, 0, 0, 0, 0};
+  size_t tap_bytes[ASR_TAP_COUNT] = {0, 0, 0, 0, 0};
+  size_t total = 0;
+};
+
+int64_t conv_len(int64_t n, int k, int s, int p) { return (n + 2 * p - k) / s + 1; }
+
+bool geom_valid(const asr_geometry* g, std::string* why) {
+  auto fail = [&](const char* m) {
+    if (why) *why = m;
+    return false;
+  };
+  if (!g) return fail("geometry is NULL");
+  if (g->stem != ASR_STEM_CONV2D_CHUNKED && g->stem != ASR_STEM_CONV1D) return fail("unknown stem");
+  if (g->n_mels <= 0 || g->n_mels > 128) return fail("n_mels must be 1..128");
+  if (g->n_fft != 400 || g->hop != 160) return fail("only n_fft 400 / hop 160 are implemented");
+  if (g->stem == ASR_STEM_CONV2D_CHUNKED) {
+    if (g->chunk_frames <= 0) return fail("chunk_frames must be > 0");
+    if (g->conv_ch <= 0 || g->conv_ch % 8 || g->conv_ch > 512) return fail("conv_ch must be a multiple of 8, <= 512");
+  }
+  if (g->d_model <= 0 || g->d_model % 128 || g->d_model > 2048) return fail("d_model must be a multiple of 128, <= 2048");
+  if (g->head_dim != 64 || g->n_heads * g->head_dim != g->d_model) return fail("head_dim must be 64 and n_heads*64 == d_model");
+  if (g->d_ffn <= 0 || g->d_ffn % 64) return fail("d_ffn must be a positive multiple of 64");
+  if (g->n_layers < 0) return fail("n_layers < 0");
+  if (g->window_tokens < 0) return fail("window_tokens < 0");
+  if (g->pos_mode != ASR_POS_PER_CHUNK && g->pos_mode != ASR_POS_GLOBAL) return fail("unknown pos_mode");
+  if (g->pos_mode == ASR_POS_PER_CHUNK && g->stem != ASR_STEM_CONV2D_CHUNKED) return fail("per-chunk positions need the chunked stem");
+  if ((g->proj1_out == 0) != (g->proj2_out == 0)) return fail("proj1_out and proj2_out must both be set or both 0");
+  if (g->proj1_out && (g->proj1_out % 64 || g->proj2_out % 128 || g->proj2_out > 2048)) return fail("head widths: proj1 % 64, proj2 % 128, <= 2048");
+  if ((g->adapter_hidden == 0) != (g->adapter_out == 0)) return fail("adapter_hidden and adapter_out must both be set or both 0");
+  if (g->adapter_hidden && (g->adapter_hidden % 16 || g->adapter_out % 16)) return fail("adapter widths must be multiples of 16");
+  if (g->adapter_hidden && !g->proj1_out) return fail("the adapter needs the head projections");
+  if (!(g->ln_eps > 0.f)) return fail("ln_eps must be > 0");
+  if (g->dtype != ASR_DTYPE_BF16 && g->dtype != ASR_DTYPE_F32) return fail("unknown dtype");
+  return true;
+}
+
+int d_out(const asr_geometry* g) {
+  if (g->adapter_hidden) return g->adapter_out;
+  if (g->proj2_out) return g->proj2_out;
+  return g->d_model;
+}
+
+struct WSpec {
+  std::string name;
+  int ndim;
+  int64_t shape[4];
+};
+
+std::vector<WSpec> weight_specs(const asr_geometry* g) {
+  std::vector<WSpec> s;
+  const int64_t d = g->d_model, C = g->conv_ch;
+  auto add = [&](const std::string& n, std::initializer_list<int64_t> sh) {
+    WSpec w;
+    w.name = n;
+    w.ndim = static_cast<int>(sh.size());
+    int i = 0;
+    for (int64_t v : sh) w.shape[i++] = v;
+    for (; i < 4; ++i) w.shape[i] = 1;
+    s.push_back(w);
+  };
+  if (g->stem == ASR_STEM_CONV2D_CHUNKED) {
+    const int64_t f3 = conv_len(conv_len(conv_len(g->n_mels, 3, 2, 1), 3, 2, 1), 3, 2, 1);
+    add("conv1.w", {C, 1, 3, 3}); add("conv1.b", {C});
+    add("conv2.w", {C, C, 3, 3}); add("conv2.b", {C});
+    add("conv3.w", {C, C, 3, 3}); add("conv3.b", {C});
+    add("conv_out.w", {d, C * f3});
+  } else {
+    add("conv1.w", {d, g->n_mels, 3}); add("conv1.b", {d});
+    add("conv2.w", {d, d, 3}); add("conv2.b", {d});
+  }
+  for (int l = 0; l < g->n_layers; ++l) {
+    const std::string p = "layers." + std::to_string(l) + ".";
+    add(p + "ln1.g", {d}); add(p + "ln1.b", {d});
+    add(p + "q.w", {d, d}); add(p + "q.b", {d});
+    add(p + "k.w", {d, d}); add(p + "k.b", {d});
+    add(p + "v.w", {d, d}); add(p + "v.b", {d});
+    add(p + "o.w", {d, d}); add(p + "o.b", {d});
+    add(p + "ln2.g", {d}); add(p + "ln2.b", {d});
+    add(p + "fc1.w", {g->d_ffn, d}); add(p + "fc1.b", {g->d_ffn});
+    add(p + "fc2.w", {d, g->d_ffn}); add(p + "fc2.b", {d});
+  }
+  add("ln_post.g", {d}); add("ln_post.b", {d});
+  if (g->proj1_out) {
+    add("proj1.w", {g->proj1_out, d}); add("proj1.b", {g->proj1_out});
+    add("proj2.w", {g->proj2_out, g->proj1_out}); add("proj2.b", {g->proj2_out});
+  }
+  if (g->adapter_hidden) {
+    add("adapter.gate.w", {g->adapter_hidden, g->proj2_out});
+    add("adapter.up.w", {g->adapter_hidden, g->proj2_out});
+    add("adapter.down.w", {g->adapter_out, g->adapter_hidden});
+  }
+  return s;
+}
+
+int64_t numel(const WSpec& w) {
+  int64_t n = 1;
+  for (int i = 0; i < w.ndim; ++i) n *= w.shape[i];
+  return n;
+}
+
+// Tokens per clip, or -1.
+int64_t tokens_per_clip(const asr_geometry* g, int64_t n) {
+  if (!geom_valid(g, nullptr) || n <= 0 || n % g->hop) return -1;
+  const int64_t frames = n / g->hop;
+  if (g->stem == ASR_STEM_CONV2D_CHUNKED) {
+    if (frames % g->chunk_frames) return -1;
+    const int64_t t3 = conv_len(conv_len(conv_len(g->chunk_frames, 3, 2, 1), 3, 2, 1), 3, 2, 1);
+    return (frames / g->chunk_frames) * t3;
+  }
+  return conv_len(conv_len(frames, 3, 1, 1), 3, 2, 1);
+}
+
+// Host tables in double precision, rounded once to float.
+void build_mel_tables(int n_mels, MelTables* t) {
+  memset(t, 0, sizeof *t);
+  const double PI = 3.14159265358979323846;
+  for (int j = 0; j < 200; ++j) t->w200[j] = make_float2((float)cos(2 * PI * j / 200), (float)-sin(2 * PI * j / 200));
+  for (int k = 0; k <= 200; ++k) t->w400[k] = make_float2((float)cos(2 * PI * k / 400), (float)-sin(2 * PI * k / 400));
+  for (int n = 0; n < 400; ++n) t->hann[n] = (float)(0.5 - 0.5 * cos(2 * PI * n / 400));
+  // Slaney mel scale: 3 f / 200 below 1 kHz, 15 + 27 ln(f / 1000) / ln 6.4 above.
+  auto hz2mel = [](double f) { return f < 1000.0 ? 3.0 * f / 200.0 : 15.0 + 27.0 * log(f / 1000.0) / log(6.4); };
+  auto mel2hz = [](double m) { return m < 15.0 ? 200.0 * m / 3.0 : 1000.0 * exp((m - 15.0) * log(6.4) / 27.0); };
+  const double mmax = hz2mel(8000.0);
+  std::vector<double> fpts(n_mels + 2);
+  for (int i = 0; i < n_mels + 2; ++i) fpts[i] = mel2hz(mmax * i / (n_mels + 1));
+  int off = 0;
+  for (int m = 0; m < n_mels; ++m) {
+    const double lo = fpts[m], ce = fpts[m + 1], hi = fpts[m + 2];
+    const double norm = 2.0 / (hi - lo);
+    int first = -1, cnt = 0;
+    for (int k = 0; k <= 200; ++k) {
+      const double f = 40.0 * k;
+      const double w = std::max(0.0, std::min((f - lo) / (ce - lo), (hi - f) / (hi - ce))) * norm;
+      if (w > 0.0) {
+        if (first < 0) first = k;
+        t->fw[off + cnt] = (float)w;
+        ++cnt;
+      } else if (first >= 0) {
+        break;
+      }
+    }
+    t->fstart[m] = first < 0 ? 0 : first;
+    t->fcount[m] = cnt;
+    t->foff[m] = off;
+    off += cnt;
+  }
+}
+
+// Sinusoidal positions [rows, d]: d/2 frequencies exp(-ln(1e4) i / (d/2 - 1)),
+// [sin(p w_i) | cos(p w_i)].
+std::vector<float> build_pe(int rows, int d) {
+  std::vector<float> pe((size_t)rows * d);
+  const int half = d / 2;
+  const double inc = log(10000.0) / (half - 1);
+  for (int p = 0; p < rows; ++p)
+    for (int i = 0; i < half; ++i) {
+      const double a = p * exp(-inc * i);
+      pe[(size_t)p * d + i] = (float)sin(a);
+      pe[(size_t)p * d + half + i] = (float)cos(a);
+    }
+  return pe;
+}
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+}  // namespace
+
+struct asr_enc {
+  asr_geometry g;
+  asr_alloc_fn alloc = nullptr;
+  asr_free_fn free_fn = nullptr;
+  void* ctx = nullptr;
+  int device = 0, num_sms = 148;
+  void* slab = nullptr;
+  size_t slab_bytes = 0, slab_used = 0;
+  std::string err;
+  // stem
+  float *c1w = nullptr, *c1b = nullptr, *c2b = nullptr, *c3b = nullptr;
+  GemmB c2, c3, cout;
+  float* pe = nullptr;
+  int pe_rows = 0;
+  std::vector<LayerW> layers;
+  float *lnpg = nullptr, *lnpb = nullptr, *bp1 = nullptr, *bp2 = nullptr;
+  GemmB p1, p2, gu, down;
+  MelTables* mel_tab = nullptr;
+  int* status = nullptr;
+  unsigned taps = 0;
+  cudaStream_t last_stream = nullptr;
+  bool have_last = false;
+  Plan last_plan;
+  void* last_ws = nullptr;
+  ActMaps maps;
+};
+
+namespace {
+
+asr_status fail(asr_enc* e, asr_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  if (e) e->err = buf;
+  std::lock_guard<std::mutex> lk(g_err_mu);
+  g_err = buf;
+  return st;
+}
+
+#define ASR_CUDA(e, call)                                                                                   \
+  do {                                                                                                      \
+    cudaError_t _r = (call);                                                                                \
+    if (_r != cudaSuccess) return fail((e), ASR_E_CUDA, "%s failed: %s", #call, cudaGetErrorString(_r));   \
+  } while (0)
+
+void* slab_take(asr_enc* e, size_t bytes) {
+  const size_t off = align_up(e->slab_used, 1024);
+  if (off + bytes > e->slab_bytes) return nullptr;
+  e->slab_used = off + bytes;
+  return static_cast<char*>(e->slab) + off;
+}
+
+std::vector<float> fetch(const void* dptr, int64_t n, int dtype) {
+  std::vector<float> out((size_t)n);
+  if (dtype == ASR_DTYPE_F32) {
+    cudaMemcpy(out.data(), dptr, n * 4, cudaMemcpyDeviceToHost);
+  } else {
+    std::vector<uint16_t> tmp((size_t)n);
+    cudaMemcpy(tmp.data(), dptr, n * 2, cudaMemcpyDeviceToHost);
+    for (int64_t i = 0; i < n; ++i) {
+      uint32_t u = static_cast<uint32_t>(tmp[i]) << 16;
+      float f;
+      memcpy(&f, &u, 4);
+      out[i] = f;
+    }
+  }
+  return out;
+}
+
+uint16_t f2bf(float f) {
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  if ((u & 0x7F800000u) == 0x7F800000u) return static_cast<uint16_t>((u >> 16) | ((u & 0xFFFF) ? 0x40 : 0));
+  const uint32_t rounding = 0x7FFFu + ((u >> 16) & 1u);
+  return static_cast<uint16_t>((u + rounding) >> 16);
+}
+
+}  // namespace
+
+// ====================================================================== ABI
+
+extern "C" {
+
+int asr_enc_weight_count(const asr_geometry* g) {
+  if (!geom_valid(g, nullptr)) return -1;
+  return static_cast<int>(weight_specs(g).size());
+}
+
+asr_status asr_enc_weight_info(const asr_geometry* g, int i, const char** name, int* ndim, int64_t shape[4]) {
+  std::string why;
+  if (!geom_valid(g, &why)) return fail(nullptr, ASR_E_INVAL, "invalid geometry: %s", why.c_str());
+  static std::mutex mu;
+  static std::map<std::string, std::string> names;  // interned names
+  auto s = weight_specs(g);
+  if (i < 0 || i >= (int)s.size()) return fail(nullptr, ASR_E_INVAL, "weight index %d out of range", i);
+  if (name) {
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = names.emplace(s[i].name, s[i].name).first;
+    *name = it->second.c_str();
+  }
+  if (ndim) *ndim = s[i].ndim;
+  if (shape)
+    for (int k = 0; k < 4; ++k) shape[k] = s[i].shape[k];
+  return ASR_OK;
+}
+
+int64_t asr_enc_tokens(const asr_geometry* g, int64_t n_samples) { return tokens_per_clip(g, n_samples); }
+
+asr_status asr_enc_windows(const asr_geometry* g, int64_t n_samples, int batch, int32_t* cu, int* n) {
+  if (!n) return fail(nullptr, ASR_E_INVAL, "n is NULL");
+  const int64_t t = tokens_per_clip(g, n_samples);
+  if (t < 0 || batch <= 0) return fail(nullptr, ASR_E_INVAL, "invalid geometry, n_samples or batch");
+  const int64_t w = g->window_tokens ? g->window_tokens : t;
+  const int64_t per = (t + w - 1) / w;
+  const int64_t count = per * batch;
+  if (count > 0x7FFFFFFF || t * batch > 0x7FFFFFFF) return fail(nullptr, ASR_E_UNSUPPORTED, "partition too large");
+  if (cu) {
+    if (*n < count + 1) return fail(nullptr, ASR_E_INVAL, "cu capacity %d < %lld", *n, (long long)(count + 1));
+    int idx = 0;
+    cu[idx++] = 0;
+    for (int b = 0; b < batch; ++b)
+      for (int64_t j = 0; j < per; ++j) cu[idx++] = static_cast<int32_t>(b * t + std::min((j + 1) * w, t));
+  }
+  *n = static_cast<int>(count);
+  return ASR_OK;
+}
+
+const char* asr_enc_last_error(const asr_enc* e) {
+  if (e) return e->err.c_str();
+  std::lock_guard<std::mutex> lk(g_err_mu);
+  static thread_local std::string copy;
+  copy = g_err;
+  return copy.c_str();
+}
+
+void asr_enc_destroy(asr_enc* e) {
+  if (!e) return;
+  if (e->slab) {
+    if (e->free_fn)
+      e->free_fn(e->ctx, e->slab);
+    else if (!e->alloc)
+      cudaFree(e->slab);
+  }
+  delete e;
+}
+
+asr_status asr_enc_create(const asr_geometry* g, const void* const* weights, int n_weights, asr_alloc_fn alloc,
+                          asr_free_fn free_fn, void* alloc_ctx, void* stream, asr_enc** out) {
+  if (!out) return fail(nullptr, ASR_E_INVAL, "out is NULL");
+  *out = nullptr;
+  std::string why;
+  if (!geom_valid(g, &why)) return fail(nullptr, ASR_E_UNSUPPORTED, "geometry not supported: %s", why.c_str());
+  auto specs = weight_specs(g);
+  if (!weights || n_weights != (int)specs.size())
+    return fail(nullptr, ASR_E_INVAL, "expected %d weight pointers, got %d", (int)specs.size(), n_weights);
+  for (int i = 0; i < n_weights; ++i)
+    if (!weights[i]) return fail(nullptr, ASR_E_INVAL, "weight %d (%s) is NULL", i, specs[i].name.c_str());
+
+  asr_enc* e = new asr_enc();
+  e->g = *g;
+  e->alloc = alloc;
+  e->free_fn = free_fn;
+  e->ctx = alloc_ctx;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto bad = [&](asr_status s) {
+    std::string m = e->err;
+    asr_enc_destroy(e);
+    fail(nullptr, s, "%s", m.c_str());
+    return s;
+  };
+  if (cudaGetDevice(&e->device) != cudaSuccess) return bad(fail(e, ASR_E_CUDA, "cudaGetDevice failed"));
+  if (cudaDeviceGetAttribute(&e->num_sms, cudaDevAttrMultiProcessorCount, e->device) != cudaSuccess)
+    return bad(fail(e, ASR_E_CUDA, "cudaDeviceGetAttribute failed"));
+  int major = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, e->device);
+  if (major != 10) return bad(fail(e, ASR_E_UNSUPPORTED, "this library runs on sm_100 (B200) only; device has sm_%d", major * 10));
+
+  const int d = g->d_model, C = g->conv_ch, L = g->n_layers;
+  // ---- slab size
+  size_t need = 0;
+  auto acc = [&](size_t bytes) { need = align_up(need, 1024) + bytes; };
+  for (auto& w : specs) acc((size_t)numel(w) * 4);  // generous: every tensor at 4 bytes/element
+  const int pe_rows = g->stem == ASR_STEM_CONV2D_CHUNKED
+                          ? (int)conv_len(conv_len(conv_len(g->chunk_frames, 3, 2, 1), 3, 2, 1), 3, 2, 1)
+                          : 1500;
+  acc((size_t)pe_rows * d * 4);
+  acc(sizeof(MelTables));
+  acc(256);  // status
+  e->slab_bytes = align_up(need, 1024) + 4096;
+  e->slab = alloc ? alloc(alloc_ctx, e->slab_bytes) : nullptr;
+  if (!alloc && cudaMalloc(&e->slab, e->slab_bytes) != cudaSuccess) e->slab = nullptr;
+  if (!e->slab) return bad(fail(e, ASR_E_NOMEM, "allocation of %zu bytes failed", e->slab_bytes));
+
+  std::vector<void*> host_keep;
+  auto up_f32 = [&](const std::vector<float>& v) -> float* {
+    float* p = static_cast<float*>(slab_take(e, v.size() * 4));
+    if (p) cudaMemcpy(p, v.data(), v.size() * 4, cudaMemcpyHostToDevice);
+    return p;
+  };
+  auto up_bf16 = [&](const std::vector<float>& v) -> bf16* {
+    std::vector<uint16_t> h(v.size());
+    for (size_t i = 0; i < v.size(); ++i) h[i] = f2bf(v[i]);
+    bf16* p = static_cast<bf16*>(slab_take(e, h.size() * 2));
+    if (p) cudaMemcpy(p, h.data(), h.size() * 2, cudaMemcpyHostToDevice);
+    return p;
+  };
+  int wi = 0;
+  auto next = [&]() {
+    const WSpec& s = specs[wi];
+    return fetch(weights[wi++], numel(s), g->dtype);
+  };
+  auto gemm_w = [&](GemmB& gb, const std::vector<float>& v, int N, int K) -> bool {
+    gb.ptr = up_bf16(v);
+    gb.N = N;
+    gb.K = K;
+    return gb.ptr && make_weight_maps(gb);
+  };
+  cudaStreamSynchronize(st);
+  if (g->stem == ASR_STEM_CONV2D_CHUNKED) {
+    const int f3 = (int)conv_len(conv_len(conv_len(g->n_mels, 3, 2, 1), 3, 2, 1), 3, 2, 1);
+    auto w1 = next();
+    e->c1w = up_f32(w1);  // [C][kh*3+kw]
+    e->c1b = up_f32(next());
+    for (int layer = 0; layer < 2; ++layer) {
+      auto w = next();  // [o][c][kh][kw] -> [o][(kw*3+kh)*C + c]
+      std::vector<float> r((size_t)C * 9 * C);
+      for (int o = 0; o < C; ++o)
+        for (int c = 0; c < C; ++c)
+          for (int kh = 0; kh < 3; ++kh)
+            for (int kw = 0; kw < 3; ++kw)
+              r[(size_t)o * 9 * C + (kw * 3 + kh) * C + c] = w[(((size_t)o * C + c) * 3 + kh) * 3 + kw];
+      if (!gemm_w(layer == 0 ? e->c2 : e->c3, r, C, 9 * C)) return bad(fail(e, ASR_E_CUDA, "conv weight upload / TMA map failed"));
+      auto b = next();
+      (layer == 0 ? e->c2b : e->c3b) = up_f32(b);
+    }
+    auto wo = next();  // [d][c*f3 + f] -> [d][f*C + c]
+    std::vector<float> r((size_t)d * C * f3);
+    for (int o = 0; o < d; ++o)
+      for (int c = 0; c < C; ++c)
+        for (int f = 0; f < f3; ++f) r[(size_t)o * C * f3 + f * C + c] = wo[(size_t)o * C * f3 + c * f3 + f];
+    if (!gemm_w(e->cout, r, d, C * f3)) return bad(fail(e, ASR_E_CUDA, "conv_out upload / TMA map failed"));
+  } else {
+    const int M = g->n_mels;
+    auto w1 = next();  // [d][c][k] -> [d][k*M + c]
+    std::vector<float> r1((size_t)d * 3 * M);
+    for (int o = 0; o < d; ++o)
+      for (int c = 0; c < M; ++c)
+        for (int k = 0; k < 3; ++k) r1[(size_t)o * 3 * M + k * M + c] = w1[((size_t)o * M + c) * 3 + k];
+    if (!gemm_w(e->c2, r1, d, 3 * M)) return bad(fail(e, ASR_E_CUDA, "conv1 upload failed"));
+    e->c2b = up_f32(next());
+    auto w2 = next();
+    std::vector<float> r2((size_t)d * 3 * d);
+    for (int o = 0; o < d; ++o)
+      for (int c = 0; c < d; ++c)
+        for (int k = 0; k < 3; ++k) r2[(size_t)o * 3 * d + k * d + c] = w2[((size_t)o * d + c) * 3 + k];
+    if (!gemm_w(e->c3, r2, d, 3 * d)) return bad(fail(e, ASR_E_CUDA, "conv2 upload failed"));
+    e->c3b = up_f32(next());
+  }
+  e->layers.resize(L);
+  for (int l = 0; l < L; ++l) {
+    LayerW& lw = e->layers[l];
+    lw.ln1g = up_f32(next());
+    lw.ln1b = up_f32(next());
+    std::vector<float> wqkv, bqkv;
+    for (int j = 0; j < 3; ++j) {
+      auto w = next();
+      auto b = next();
+      wqkv.insert(wqkv.end(), w.begin(), w.end());
+      bqkv.insert(bqkv.end(), b.begin(), b.end());
+    }
+    if (!gemm_w(lw.qkv, wqkv, 3 * d, d)) return bad(fail(e, ASR_E_CUDA, "qkv upload failed"));
+    lw.bqkv = up_f32(bqkv);
+    if (!gemm_w(lw.o, next(), d, d)) return bad(fail(e, ASR_E_CUDA, "o upload failed"));
+    lw.bo = up_f32(next());
+    lw.ln2g = up_f32(next());
+    lw.ln2b = up_f32(next());
+    if (!gemm_w(lw.fc1, next(), g->d_ffn, d)) return bad(fail(e, ASR_E_CUDA, "fc1 upload failed"));
+    lw.b1 = up_f32(next());
+    if (!gemm_w(lw.fc2, next(), d, g->d_ffn)) return bad(fail(e, ASR_E_CUDA, "fc2 upload failed"));
+    lw.b2 = up_f32(next());
+  }
+  e->lnpg = up_f32(next());
+  e->lnpb = up_f32(next());
+  if (g->proj1_out) {
+    if (!gemm_w(e->p1, next(), g->proj1_out, d)) return bad(fail(e, ASR_E_CUDA, "proj1 upload failed"));
+    e->bp1 = up_f32(next());
+    if (!gemm_w(e->p2, next(), g->proj2_out, g->proj1_out)) return bad(fail(e, ASR_E_CUDA, "proj2 upload failed"));
+    e->bp2 = up_f32(next());
+  }
+  if (g->adapter_hidden) {
+    const int H = g->adapter_hidden, K = g->proj2_out;
+    auto wg = next();
+    auto wu = next();
+    std::vector<float> r((size_t)2 * H * K);
+    for (int j = 0; j < H / 16; ++j)
+      for (int i = 0; i < 16; ++i) {
+        memcpy(&r[((size_t)32 * j + i) * K], &wg[((size_t)16 * j + i) * K], K * 4);
+        memcpy(&r[((size_t)32 * j + 16 + i) * K], &wu[((size_t)16 * j + i) * K], K * 4);
+      }
+    if (!gemm_w(e->gu, r, 2 * H, K)) return bad(fail(e, ASR_E_CUDA, "adapter gate/up upload failed"));
+    if (!gemm_w(e->down, next(), g->adapter_out, H)) return bad(fail(e, ASR_E_CUDA, "adapter down upload failed"));
+  }
+  e->pe_rows = pe_rows;
+  e->pe = up_f32(build_pe(pe_rows, d));
+  MelTables mt;
+  build_mel_tables(g->n_mels, &mt);
+  e->mel_tab = static_cast<MelTables*>(slab_take(e, sizeof(MelTables)));
+  if (!e->mel_tab) return bad(fail(e, ASR_E_NOMEM, "slab exhausted"));
+  cudaMemcpy(e->mel_tab, &mt, sizeof mt, cudaMemcpyHostToDevice);
+  e->status = static_cast<int*>(slab_take(e, 256));
+  if (!e->status) return bad(fail(e, ASR_E_NOMEM, "slab exhausted"));
+  cudaMemset(e->status, 0, 256);
+  cudaError_t r = cudaDeviceSynchronize();
+  if (r != cudaSuccess) return bad(fail(e, ASR_E_CUDA, "weight repack failed: %s", cudaGetErrorString(r)));
+  if (!e->pe || !e->c2.ptr) return bad(fail(e, ASR_E_NOMEM, "slab exhausted"));
+  *out = e;
+  return ASR_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+bool make_plan(const asr_enc* e, int64_t n, int B, Plan* p) {
+  const asr_geometry* g = &e->g;
+  const int64_t tc = tokens_per_clip(g, n);
+  if (tc <= 0 || B <= 0) return false;
+  p->n = n;
+  p->B = B;
+  p->Tc = tc;
+  p->T = tc * B;
+  p->F = (int)(n / g->hop);
+  const int64_t w = g->window_tokens ? g->window_tokens : tc;
+  p->nwin_clip = (int)((tc + w - 1) / w);
+  p->nwin = p->nwin_clip * B;
+  p->max_win = (int)std::min<int64_t>(w, tc);
+  const int d = g->d_model;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    off = align_up(off, 1024);
+    size_t r = off;
+    off += bytes;
+    return r;
+  };
+  p->off_clipmax = take((size_t)B * 4);
+  p->off_cu = take((size_t)(p->nwin + 1) * 4);
+  p->off_mel = take((size_t)B * g->n_mels * p->F * 4);
+  if (g->stem == ASR_STEM_CONV2D_CHUNKED) {
+    p->chunks = (int)(B * (p->F / g->chunk_frames));
+    p->T1 = (int)conv_len(g->chunk_frames, 3, 2, 1); p->F1 = (int)conv_len(g->n_mels, 3, 2, 1);
+    p->T2 = (int)conv_len(p->T1, 3, 2, 1); p->F2 = (int)conv_len(p->F1, 3, 2, 1);
+    p->T3 = (int)conv_len(p->T2, 3, 2, 1); p->F3 = (int)conv_len(p->F2, 3, 2, 1);
+    const size_t C = g->conv_ch;
+    p->off_c1 = take((size_t)p->chunks * p->T1 * p->F1 * C * 2);
+    p->off_c2 = take((size_t)p->chunks * p->T2 * p->F2 * C * 2);
+    p->off_c3 = take((size_t)p->T * p->F3 * C * 2);
+  } else {
+    p->off_melT = take((size_t)B * p->F * g->n_mels * 2);
+    p->off_c1 = take((size_t)B * p->F * d * 2);
+  }
+  p->off_x = take((size_t)p->T * d * 4);
+  p->off_h = take((size_t)p->T * d * 2);
+  p->off_qkv = take((size_t)p->T * 3 * d * 2);
+  p->off_att = take((size_t)p->T * d * 2);
+  p->off_ff = take((size_t)p->T * g->d_ffn * 2);
+  if (g->proj1_out) {
+    p->off_p1 = take((size_t)p->T * g->proj1_out * 2);
+    p->off_p2 = take((size_t)p->T * g->proj2_out * 2);
+  }
+  if (g->adapter_hidden) p->off_gu = take((size_t)p->T * g->adapter_hidden * 2);
+  p->tap_bytes[ASR_TAP_MEL] = (size_t)B * g->n_mels * p->F * 4;
+  p->tap_bytes[ASR_TAP_STEM] = p->tap_bytes[ASR_TAP_LAYER0] = p->tap_bytes[ASR_TAP_ENCODER] = (size_t)p->T * d * 4;
+  p->tap_bytes[ASR_TAP_HEAD] = g->proj2_out ? (size_t)p->T * g->proj2_out * 4 : 0;
+  for (int t = 0; t < ASR_TAP_COUNT; ++t)
+    if ((e->taps >> t) & 1u) p->off_tap[t] = take(p->tap_bytes[t]);
+  p->off_pcm = take((size_t)B * n * 4);
+  p->off_out = take((size_t)p->T * d_out(g) * 4);
+  p->total = align_up(off, 1024);
+  return true;
+}
+
+asr_status gemm(asr_enc* e, const CUtensorMap* amap, const ConvGather* cg, const GemmB& w, long long M, void* out,
+                long long ldo, const float* bias, const float* pe, int period, int epi, cudaStream_t st) {
+  GemmParams p;
+  memset(&p, 0, sizeof p);
+  p.M = (int)M;
+  p.out = out;
+  p.ldo = ldo;
+  p.bias = bias;
+  p.pe = pe;
+  p.pe_period = period;
+  if (cg) p.g = *cg;
+  p.status = e->status;
+  p.limit_ns = kWaitLimitNs;
+  const int bn = gemm_pick_bn((int)M, w.N, e->num_sms, cg != nullptr);
+  cudaError_t r = launch_gemm(amap, w, p, epi, bn, e->num_sms, st);
+  if (r != cudaSuccess) return fail(e, ASR_E_CUDA, "gemm launch (N=%d K=%d M=%lld epi=%d bn=%d): %s", w.N, w.K, M, epi, bn, cudaGetErrorString(r));
+  return ASR_OK;
+}
+
+#define ASR_TRY(x)                 \
+  do {                             \
+    asr_status _s = (x);           \
+    if (_s != ASR_OK) return _s;   \
+  } while (0)
+#define ASR_LAUNCH(e, x)                                                                                     \
+  do {                                                                                                       \
+    cudaError_t _r = (x);                                                                                    \
+    if (_r != cudaSuccess) return fail((e), ASR_E_CUDA, "%s: %s", #x, cudaGetErrorString(_r));               \
+  } while (0)
+
+asr_status ensure_maps(asr_enc* e, const Plan& p, char* ws) {
+  ActMaps& m = e->maps;
+  if (m.ws == ws && m.n == p.n && m.batch == p.B && m.taps == e->taps) return ASR_OK;
+  const asr_geometry* g = &e->g;
+  const int d = g->d_model;
+  bool ok = make_tmap_bf16(&m.h, ws + p.off_h, p.T, d, d, 128) &&
+            make_tmap_bf16(&m.att, ws + p.off_att, p.T, d, d, 128) &&
+            make_tmap_bf16(&m.ff, ws + p.off_ff, p.T, g->d_ffn, g->d_ffn, 128);
+  if (ok && g->stem == ASR_STEM_CONV2D_CHUNKED)
+    ok = make_tmap_bf16(&m.c3, ws + p.off_c3, p.T, (size_t)p.F3 * g->conv_ch, (size_t)p.F3 * g->conv_ch, 128);
+  if (ok && g->proj1_out)
+    ok = make_tmap_bf16(&m.p1, ws + p.off_p1, p.T, g->proj1_out, g->proj1_out, 128) &&
+         make_tmap_bf16(&m.p2, ws + p.off_p2, p.T, g->proj2_out, g->proj2_out, 128);
+  if (ok && g->adapter_hidden) ok = make_tmap_bf16(&m.gu, ws + p.off_gu, p.T, g->adapter_hidden, g->adapter_hidden, 128);
+  if (!ok) {
+    m.ws = nullptr;
+    return fail(e, ASR_E_CUDA, "TMA descriptor encoding failed (workspace alignment?)");
+  }
+  m.ws = ws;
+  m.n = p.n;
+  m.batch = p.B;
+  m.taps = e->taps;
+  return ASR_OK;
+}
+
+asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, char* ws, cudaStream_t st) {
+  const asr_geometry* g = &e->g;
+  const int d = g->d_model;
+  ASR_TRY(ensure_maps(e, p, ws));
+  unsigned* clip_max = reinterpret_cast<unsigned*>(ws + p.off_clipmax);
+  int* cu = reinterpret_cast<int*>(ws + p.off_cu);
+  float* mel = reinterpret_cast<float*>(ws + p.off_mel);
+  float* x = reinterpret_cast<float*>(ws + p.off_x);
+  bf16* h = reinterpret_cast<bf16*>(ws + p.off_h);
+  bf16* qkv = reinterpret_cast<bf16*>(ws + p.off_qkv);
+  bf16* att = reinterpret_cast<bf16*>(ws + p.off_att);
+  bf16* ff = reinterpret_cast<bf16*>(ws + p.off_ff);
+  auto tap = [&](int t) -> float* { return ((e->taps >> t) & 1u) ? reinterpret_cast<float*>(ws + p.off_tap[t]) : nullptr; };
+
+  ASR_LAUNCH(e, cudaMemsetAsync(e->status, 0, 4, st));
+  ASR_LAUNCH(e, cudaMemsetAsync(clip_max, 0, (size_t)p.B * 4, st));
+  const int w = g->window_tokens ? g->window_tokens : (int)p.Tc;
+  ASR_LAUNCH(e, launch_fill_windows(cu, p.B, (int)p.Tc, w, p.nwin_clip, st));
+  ASR_LAUNCH(e, launch_log_mel(pcm, p.n, p.B, g->n_mels, e->mel_tab, mel, clip_max, st));
+  if (float* t = tap(ASR_TAP_MEL)) ASR_LAUNCH(e, launch_mel_normalize(mel, clip_max, (long long)g->n_mels * p.F, p.B, t, st));
+
+  if (g->stem == ASR_STEM_CONV2D_CHUNKED) {
+    const int C = g->conv_ch;
+    bf16* c1 = reinterpret_cast<bf16*>(ws + p.off_c1);
+    bf16* c2 = reinterpret_cast<bf16*>(ws + p.off_c2);
+    bf16* c3 = reinterpret_cast<bf16*>(ws + p.off_c3);
+    ASR_LAUNCH(e, launch_conv1_chunked(mel, clip_max, p.B, g->n_mels, p.F, g->chunk_frames, e->c1w, e->c1b, C, c1, st));
+    ConvGather cg2 = {c1, p.T1, p.F1, C, p.T2, p.F2, 2, 2, 3, 3, 1, 1};
+    ASR_TRY(gemm(e, nullptr, &cg2, e->c2, (long long)p.chunks * p.T2 * p.F2, c2, C, e->c2b, nullptr, 1, EPI_GELU, st));
+    ConvGather cg3 = {c2, p.T2, p.F2, C, p.T3, p.F3, 2, 2, 3, 3, 1, 1};
+    ASR_TRY(gemm(e, nullptr, &cg3, e->c3, (long long)p.chunks * p.T3 * p.F3, c3, C, e->c3b, nullptr, 1, EPI_GELU, st));
+    ASR_TRY(gemm(e, &e->maps.c3, nullptr, e->cout, p.T, x, d, nullptr, e->pe, p.T3, EPI_OUT_F32 | EPI_PE, st));
+  } else {
+    if (p.Tc > e->pe_rows) return fail(e, ASR_E_UNSUPPORTED, "conv1d stem: %lld positions > %d", (long long)p.Tc, e->pe_rows);
+    bf16* melT = reinterpret_cast<bf16*>(ws + p.off_melT);
+    bf16* c1 = reinterpret_cast<bf16*>(ws + p.off_c1);
+    ASR_LAUNCH(e, launch_mel_normalize_transpose(mel, clip_max, p.B, g->n_mels, p.F, melT, st));
+    ConvGather cg1 = {melT, p.F, 1, g->n_mels, p.F, 1, 1, 1, 3, 1, 1, 0};
+    ASR_TRY(gemm(e, nullptr, &cg1, e->c2, (long long)p.B * p.F, c1, d, e->c2b, nullptr, 1, EPI_GELU, st));
+    ConvGather cg2 = {c1, p.F, 1, d, (int)p.Tc, 1, 2, 1, 3, 1, 1, 0};
+    ASR_TRY(gemm(e, nullptr, &cg2, e->c3, p.T, x, d, e->c3b, e->pe, (int)p.Tc, EPI_GELU | EPI_OUT_F32 | EPI_PE, st));
+  }
+  if (float* t = tap(ASR_TAP_STEM)) ASR_LAUNCH(e, cudaMemcpyAsync(t, x, (size_t)p.T * d * 4, cudaMemcpyDeviceToDevice, st));
+
+  for (int l = 0; l < g->n_layers; ++l) {
+    const LayerW& lw = e->layers[l];
+    ASR_LAUNCH(e, launch_layer_norm(x, lw.ln1g, lw.ln1b, p.T, d, g->ln_eps, h, false, st));
+    ASR_TRY(gemm(e, &e->maps.h, nullptr, lw.qkv, p.T, qkv, 3 * d, lw.bqkv, nullptr, 1, 0, st));
+    ASR_LAUNCH(e, launch_attention(qkv, cu, p.nwin, p.max_win, g->n_heads, att, st));
+    ASR_TRY(gemm(e, &e->maps.att, nullptr, lw.o, p.T, x, d, lw.bo, nullptr, 1, EPI_RESID, st));
+    ASR_LAUNCH(e, launch_layer_norm(x, lw.ln2g, lw.ln2b, p.T, d, g->ln_eps, h, false, st));
+    ASR_TRY(gemm(e, &e->maps.h, nullptr, lw.fc1, p.T, ff, g->d_ffn, lw.b1, nullptr, 1, EPI_GELU, st));
+    ASR_TRY(gemm(e, &e->maps.ff, nullptr, lw.fc2, p.T, x, d, lw.b2, nullptr, 1, EPI_RESID, st));
+    if (l == 0)
+      if (float* t = tap(ASR_TAP_LAYER0)) ASR_LAUNCH(e, cudaMemcpyAsync(t, x, (size_t)p.T * d * 4, cudaMemcpyDeviceToDevice, st));
+  }
+  if (float* t = tap(ASR_TAP_ENCODER)) ASR_LAUNCH(e, cudaMemcpyAsync(t, x, (size_t)p.T * d * 4, cudaMemcpyDeviceToDevice, st));
+
+  if (!g->proj1_out) {
+    ASR_LAUNCH(e, launch_layer_norm(x, e->lnpg, e->lnpb, p.T, d, g->ln_eps, out, true, st));
+    return ASR_OK;
+  }
+  bf16* p1 = reinterpret_cast<bf16*>(ws + p.off_p1);
+  bf16* p2 = reinterpret_cast<bf16*>(ws + p.off_p2);
+  ASR_LAUNCH(e, launch_layer_norm(x, e->lnpg, e->lnpb, p.T, d, g->ln_eps, h, false, st));
+  ASR_TRY(gemm(e, &e->maps.h, nullptr, e->p1, p.T, p1, g->proj1_out, e->bp1, nullptr, 1, EPI_GELU, st));
+  if (!g->adapter_hidden) {
+    ASR_TRY(gemm(e, &e->maps.p1, nullptr, e->p2, p.T, out, g->proj2_out, e->bp2, nullptr, 1, EPI_OUT_F32, st));
+    if (float* t = tap(ASR_TAP_HEAD)) ASR_LAUNCH(e, cudaMemcpyAsync(t, out, (size_t)p.T * g->proj2_out * 4, cudaMemcpyDeviceToDevice, st));
+    return ASR_OK;
+  }
+  ASR_TRY(gemm(e, &e->maps.p1, nullptr, e->p2, p.T, p2, g->proj2_out, e->bp2, nullptr, 1, 0, st));
+  if (float* t = tap(ASR_TAP_HEAD)) ASR_LAUNCH(e, launch_bf16_to_f32(p2, t, (long long)p.T * g->proj2_out, st));
+  bf16* gu = reinterpret_cast<bf16*>(ws + p.off_gu);
+  ASR_TRY(gemm(e, &e->maps.p2, nullptr, e->gu, p.T, gu, g->adapter_hidden, nullptr, nullptr, 1, EPI_SWIGLU, st));
+  ASR_TRY(gemm(e, &e->maps.gu, nullptr, e->down, p.T, out, g->adapter_out, nullptr, nullptr, 1, EPI_OUT_F32, st));
+  return ASR_OK;
+}
+
+asr_status check_forward_args(asr_enc* e, int64_t n, int B, const void* pcm, const void* out, void* ws, size_t ws_bytes,
+                              Plan* p) {
+  if (!e) return fail(nullptr, ASR_E_INVAL, "handle is NULL");
+  if (!pcm || !out) return fail(e, ASR_E_INVAL, "pcm or out is NULL");
+  if (B <= 0) return fail(e, ASR_E_INVAL, "batch must be > 0");
+  if (n <= e->g.n_fft / 2) return fail(e, ASR_E_INVAL, "n_samples must exceed n_fft/2 (reflect padding)");
+  if (tokens_per_clip(&e->g, n) <= 0)
+    return fail(e, ASR_E_UNSUPPORTED, e->g.stem == ASR_STEM_CONV2D_CHUNKED
+                                          ? "n_samples must be a whole number of %d-frame chunks"
+                                          : "n_samples must be a multiple of the hop (%d frames ok)",
+                e->g.chunk_frames);
+  if (e->g.stem == ASR_STEM_CONV1D && (n / e->g.hop) % 2)
+    return fail(e, ASR_E_UNSUPPORTED, "conv1d stem: an even number of frames is required");
+  const int64_t T = tokens_per_clip(&e->g, n) * B;
+  if (T > 0x7FFFFFFFLL / 8 || (int64_t)B * n > (1LL << 40)) return fail(e, ASR_E_UNSUPPORTED, "batch too large");
+  if (!make_plan(e, n, B, p)) return fail(e, ASR_E_INVAL, "plan failed");
+  if (!ws || ws_bytes < p->total) return fail(e, ASR_E_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, p->total);
+  if (reinterpret_cast<uintptr_t>(ws) & 255) return fail(e, ASR_E_WORKSPACE, "workspace must be 256-byte aligned");
+  return ASR_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t asr_enc_workspace_size(const asr_enc* e, int64_t n_samples, int batch) {
+  Plan p;
+  if (!e || !make_plan(e, n_samples, batch, &p)) return 0;
+  return p.total;
+}
+
+asr_status asr_enc_forward(asr_enc* e, const float* pcm, int64_t n_samples, int batch, float* out, int64_t* out_tokens,
+                           void* workspace, size_t ws_bytes, void* stream) {
+  Plan p;
+  ASR_TRY(check_forward_args(e, n_samples, batch, pcm, out, workspace, ws_bytes, &p));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ASR_TRY(run_forward(e, pcm, p, out, static_cast<char*>(workspace), st));
+  e->last_stream = st;
+  e->have_last = true;
+  e->last_plan = p;
+  e->last_ws = workspace;
+  if (out_tokens) *out_tokens = p.Tc;
+  return ASR_OK;
+}
+
+asr_status asr_enc_sync_status(asr_enc* e) {
+  if (!e) return fail(nullptr, ASR_E_INVAL, "handle is NULL");
+  cudaStream_t st = e->have_last ? e->last_stream : nullptr;
+  ASR_CUDA(e, cudaStreamSynchronize(st));
+  int s = 0;
+  ASR_CUDA(e, cudaMemcpy(&s, e->status, 4, cudaMemcpyDeviceToHost));
+  if (s != 0) return fail(e, ASR_E_DEVICE_TIMEOUT, "a bounded device wait gave up (code %d)", s);
+  return ASR_OK;
+}
+
+asr_status asr_enc_forward_host(asr_enc* e, const float* pcm_host, int64_t n_samples, int batch, float* out_host,
+                                int64_t* out_tokens, void* workspace, size_t ws_bytes, void* stream) {
+  Plan p;
+  ASR_TRY(check_forward_args(e, n_samples, batch, pcm_host, out_host, workspace, ws_bytes, &p));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  float* dpcm = reinterpret_cast<float*>(ws + p.off_pcm);
+  ASR_CUDA(e, cudaMemcpyAsync(dpcm, pcm_host, (size_t)batch * n_samples * 4, cudaMemcpyHostToDevice, st));
+  const size_t out_bytes = (size_t)p.T * d_out(&e->g) * 4;
+  float* dout = reinterpret_cast<float*>(ws + p.off_out);
+  ASR_TRY(run_forward(e, dpcm, p, dout, ws, st));
+  ASR_CUDA(e, cudaMemcpyAsync(out_host, dout, out_bytes, cudaMemcpyDeviceToHost, st));
+  e->last_stream = st;
+  e->have_last = true;
+  e->last_plan = p;
+  e->last_ws = workspace;
+  if (out_tokens) *out_tokens = p.Tc;
+  return asr_enc_sync_status(e);
+}
+
+asr_status asr_enc_set_taps(asr_enc* e, unsigned mask) {
+  if (!e) return fail(nullptr, ASR_E_INVAL, "handle is NULL");
+  if (mask >> ASR_TAP_COUNT) return fail(e, ASR_E_INVAL, "unknown tap bits");
+  e->taps = mask;
+  e->maps.ws = nullptr;
+  return ASR_OK;
+}
+
+asr_status asr_enc_tap(asr_enc* e, int stage, float* dst, size_t dst_bytes, void* stream) {
+  if (!e) return fail(nullptr, ASR_E_INVAL, "handle is NULL");
+  if (stage < 0 || stage >= ASR_TAP_COUNT) return fail(e, ASR_E_INVAL, "unknown tap stage %d", stage);
+  if (!((e->taps >> stage) & 1u) || !e->have_last) return fail(e, ASR_E_INVAL, "tap %d not recorded", stage);
+  const size_t bytes = e->last_plan.tap_bytes[stage];
+  if (!dst || dst_bytes < bytes) return fail(e, ASR_E_INVAL, "tap needs %zu bytes", bytes);
+  ASR_CUDA(e, cudaMemcpyAsync(dst, static_cast<char*>(e->last_ws) + e->last_plan.off_tap[stage], bytes,
+                              cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream)));
+  return ASR_OK;
+}
+
+// ==================================================================== ops
+
+size_t asr_op_log_mel_ws_size(int batch) { return batch > 0 ? align_up((size_t)batch * 4, 256) : 0; }
+
+asr_status asr_op_log_mel(const float* pcm, int64_t n_samples, int batch, int n_mels, float* mel, void* ws,
+                          size_t ws_bytes, void* stream) {
+  if (!pcm || !mel || batch <= 0 || n_mels <= 0 || n_mels > 128 || n_samples <= 200 || n_samples % 160)
+    return fail(nullptr, ASR_E_INVAL, "log_mel: bad arguments");
+  if (!ws || ws_bytes < asr_op_log_mel_ws_size(batch)) return fail(nullptr, ASR_E_WORKSPACE, "log_mel: workspace too small");
+  static std::mutex mu;
+  static std::map<std::pair<int, int>, MelTables*> cache;  // (device, n_mels) -> device tables
+  int dev = 0;
+  cudaGetDevice(&dev);
+  MelTables* tab = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = cache.find({dev, n_mels});
+    if (it == cache.end()) {
+      MelTables h;
+      build_mel_tables(n_mels, &h);
+      if (cudaMalloc(&tab, sizeof h) != cudaSuccess) return fail(nullptr, ASR_E_NOMEM, "log_mel: table allocation");
+      cudaMemcpy(tab, &h, sizeof h, cudaMemcpyHostToDevice);
+      cache[{dev, n_mels}] = tab;
+    } else {
+      tab = it->second;
+    }
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned* cm = static_cast<unsigned*>(ws);
+  ASR_CUDA(nullptr, cudaMemsetAsync(cm, 0, (size_t)batch * 4, st));
+  ASR_CUDA(nullptr, launch_log_mel(pcm, n_samples, batch, n_mels, tab, mel, cm, st));
+  ASR_CUDA(nullptr, launch_mel_normalize(mel, cm, (long long)n_mels * (n_samples / 160), batch, mel, st));
+  return ASR_OK;
+}
+
+size_t asr_op_linear_ws_size(void) { return 256; }
+
+asr_status asr_op_linear(const void* x, const void* w, const float* bias, int64_t M, int N, int K, int epi, void* y,
+                         void* ws, size_t ws_bytes, void* stream) {
+  if (!x || !w || !y || M <= 0 || N <= 0 || K <= 0 || K % 8 || N % 16)
+    return fail(nullptr, ASR_E_INVAL, "linear: bad arguments (K %% 8, N %% 16)");
+  if (!ws || ws_bytes < 256) return fail(nullptr, ASR_E_WORKSPACE, "linear: workspace too small");
+  int e_bits;
+  switch (epi) {
+    case ASR_EPI_BF16: e_bits = 0; break;
+    case ASR_EPI_BF16_GELU: e_bits = EPI_GELU; break;
+    case ASR_EPI_F32_RESID: e_bits = EPI_RESID; break;
+    case ASR_EPI_F32: e_bits = EPI_OUT_F32; break;
+    case ASR_EPI_SWIGLU:
+      if (N % 32) return fail(nullptr, ASR_E_INVAL, "linear: SwiGLU needs N %% 32 == 0");
+      e_bits = EPI_SWIGLU;
+      break;
+    default: return fail(nullptr, ASR_E_INVAL, "linear: unknown epilogue %d", epi);
+  }
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  GemmB wb;
+  wb.ptr = static_cast<const bf16*>(w);
+  wb.N = N;
+  wb.K = K;
+  CUtensorMap amap;
+  if (!make_weight_maps(wb) || !make_tmap_bf16(&amap, x, M, K, K, 128))
+    return fail(nullptr, ASR_E_INVAL, "linear: TMA descriptor encoding failed (16-byte alignment?)");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ASR_CUDA(nullptr, cudaMemsetAsync(ws, 0, 4, st));
+  GemmParams p;
+  memset(&p, 0, sizeof p);
+  p.M = (int)M;
+  p.out = y;
+  p.ldo = (e_bits & EPI_SWIGLU) ? N / 2 : N;
+  p.bias = bias;
+  p.pe_period = 1;
+  p.status = static_cast<int*>(ws);
+  p.limit_ns = kWaitLimitNs;
+  const int bn = gemm_pick_bn((int)M, N, sms, false);
+  ASR_CUDA(nullptr, launch_gemm(&amap, wb, p, e_bits, bn, sms, st));
+  return ASR_OK;
+}
+
+asr_status asr_op_layer_norm(const float* x, const float* g, const float* b, int64_t M, int D, float eps, void* y,
+                             int out_f32, void* stream) {
+  if (!x || !g || !b || !y || M <= 0 || D % 128 || D > 2048) return fail(nullptr, ASR_E_INVAL, "layer_norm: bad arguments");
+  ASR_CUDA(nullptr, launch_layer_norm(x, g, b, M, D, eps, y, out_f32 != 0, static_cast<cudaStream_t>(stream)));
+  return ASR_OK;
+}
+
+asr_status asr_op_attention(const void* qkv, const int32_t* cu, int n_seg, int max_seg, int64_t T, int H, void* out,
+                            void* stream) {
+  if (!qkv || !cu || !out || n_seg <= 0 || max_seg <= 0 || H <= 0 || T <= 0)
+    return fail(nullptr, ASR_E_INVAL, "attention: bad arguments");
+  ASR_CUDA(nullptr, launch_attention(static_cast<const bf16*>(qkv), cu, n_seg, max_seg, H, static_cast<bf16*>(out),
+                                     static_cast<cudaStream_t>(stream)));
+  return ASR_OK;
+}
+
+asr_status asr_op_wait_probe(int64_t limit_ns, int* status_dev, void* stream) {
+  if (!status_dev || limit_ns <= 0 || limit_ns > 10LL * 1000 * 1000 * 1000)
+    return fail(nullptr, ASR_E_INVAL, "wait_probe: bad arguments (limit 1 ns .. 10 s)");
+  ASR_CUDA(nullptr, launch_wait_probe((unsigned long long)limit_ns, status_dev, static_cast<cudaStream_t>(stream)));
+  return ASR_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,147 @@
+// Host side of the tcgen05 GEMM engine: TMA descriptor encoding, tile-width
+// choice and dispatch to the kernel instantiations.
+#include <mutex>
+
+#include "kernels.h"
+
+namespace asr {
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+constexpr int kSlotRows[4] = {256, 128, 240, 64};
+
+template <int BN>
+constexpr int stages_for() {
+  return BN >= 192 ? 4 : (BN >= 128 ? 6 : 8);
+}
+
+template <int BN, bool G, int EPI>
+cudaError_t run(const CUtensorMap* a, const CUtensorMap& b, const GemmParams& p, int grid, cudaStream_t st) {
+  using S = GemmShape<BN, stages_for<BN>(), G>;
+  auto k = gemm_bf16_tc_kernel<BN, S::STAGES, G, EPI>;
+  cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_BYTES);
+  if (err != cudaSuccess) return err;
+  k<<<grid, S::THREADS, S::SMEM_BYTES, st>>>(a ? *a : b, b, p);
+  return cudaGetLastError();
+}
+
+template <int BN>
+cudaError_t run_tma(int epi, const CUtensorMap* a, const CUtensorMap& b, const GemmParams& p, int grid,
+                    cudaStream_t st) {
+  switch (epi) {
+    case 0: return run<BN, false, 0>(a, b, p, grid, st);
+    case EPI_GELU: return run<BN, false, EPI_GELU>(a, b, p, grid, st);
+    case EPI_OUT_F32: return run<BN, false, EPI_OUT_F32>(a, b, p, grid, st);
+    case EPI_RESID: return run<BN, false, EPI_RESID>(a, b, p, grid, st);
+    case EPI_OUT_F32 | EPI_PE: return run<BN, false, EPI_OUT_F32 | EPI_PE>(a, b, p, grid, st);
+    case EPI_SWIGLU: return run<BN, false, EPI_SWIGLU>(a, b, p, grid, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int BN>
+cudaError_t run_gather(int epi, const CUtensorMap& b, const GemmParams& p, int grid, cudaStream_t st) {
+  switch (epi) {
+    case EPI_GELU: return run<BN, true, EPI_GELU>(nullptr, b, p, grid, st);
+    case EPI_GELU | EPI_OUT_F32 | EPI_PE: return run<BN, true, EPI_GELU | EPI_OUT_F32 | EPI_PE>(nullptr, b, p, grid, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+int gemm_bn_slot(int bn) {
+  for (int i = 0; i < 4; ++i)
+    if (kSlotRows[i] == bn) return i;
+  return -1;
+}
+
+bool make_tmap_bf16(CUtensorMap* map, const void* ptr, unsigned long long rows, unsigned long long cols,
+                    unsigned long long row_stride_elems, unsigned int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || !ptr || (reinterpret_cast<uintptr_t>(ptr) & 15) || (row_stride_elems * 2) % 16 || rows == 0 ||
+      cols == 0 || box_rows == 0 || box_rows > 256)
+    return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {row_stride_elems * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_weight_maps(GemmB& w) {
+  for (int i = 0; i < 4; ++i)
+    if (!make_tmap_bf16(&w.map[i], w.ptr, w.N, w.K, w.K, kSlotRows[i])) return false;
+  return true;
+}
+
+int gemm_pick_bn(int M, int N, int num_sms, bool gather) {
+  if (N % 240 == 0 && N % 256 != 0 && N <= 480) return 240;
+  if (N <= 64) return 64;
+  const long long mb = (M + 127) / 128;
+  long long best_cost = -1;
+  int best = 256;
+  for (int bn : {256, 128}) {
+    const long long tiles = mb * ((N + bn - 1) / bn);
+    const long long waves = (tiles + num_sms - 1) / num_sms;
+    // per-tile cost ~ columns + fixed overhead (epilogue drain, pipeline fill)
+    const long long cost = waves * (bn + 24);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = bn;
+    }
+  }
+  (void)gather;
+  return best;
+}
+
+cudaError_t launch_gemm(const CUtensorMap* a_map, const GemmB& w, GemmParams p, int epi, int bn, int num_sms,
+                        cudaStream_t st) {
+  const int slot = gemm_bn_slot(bn);
+  if (slot < 0 || p.M <= 0) return cudaErrorInvalidValue;
+  p.N = w.N;
+  p.K = w.K;
+  p.m_blocks = (p.M + 127) / 128;
+  p.n_blocks = (p.N + bn - 1) / bn;
+  p.k_blocks = (p.K + 63) / 64;
+  p.num_tiles = p.m_blocks * p.n_blocks;
+  const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
+  const CUtensorMap& b = w.map[slot];
+  const bool gather = (a_map == nullptr);
+  if (gather) {
+    switch (bn) {
+      case 256: return run_gather<256>(epi, b, p, grid, st);
+      case 240: return run_gather<240>(epi, b, p, grid, st);
+      case 128: return run_gather<128>(epi, b, p, grid, st);
+      case 64: return run_gather<64>(epi, b, p, grid, st);
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  switch (bn) {
+    case 256: return run_tma<256>(epi, a_map, b, p, grid, st);
+    case 128: return run_tma<128>(epi, a_map, b, p, grid, st);
+    case 64: return run_tma<64>(epi, a_map, b, p, grid, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace asr

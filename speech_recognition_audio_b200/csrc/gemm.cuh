@@ -1,0 +1,376 @@
+// tcgen05 GEMM engine for sm_100a: D[M,N] = A[M,K] * B[N,K]^T, bf16 inputs,
+// fp32 accumulation in tensor memory, fused epilogues.
+//
+// Every dense contraction of the encoder runs here: the conv stem as an
+// implicit GEMM (A gathered from the NHWC activation by cp.async warps), the
+// conv_out projection with the sinusoidal positions, the QKV / output / FFN
+// projections of each pre-LN layer with bias, GELU and residual epilogues,
+// and the head and SwiGLU adapter projections ("MOSS-Transcribe-preview-2B-
+// GGUF", Architecture table: "Audio encoder", "Conv front-end", "Encoder
+// head", "Adapter" rows).
+//
+// Structure (one persistent CTA per SM, static round-robin over 128 x BN
+// output tiles):
+//   warp 0      TMA producer: B tiles (and A tiles when A is a plain matrix)
+//               into a STAGES-deep ring of 128-byte-swizzled smem buffers.
+//   warp 1      allocates tensor memory; lane 0 issues tcgen05.mma
+//               (M=128, N=BN, K=16) and commits to the ring's "empty"
+//               barriers and, per tile, to an accumulator "full" barrier.
+//   warps 2-5   epilogue: tcgen05.ld the accumulator (each warp owns the 32
+//               TMEM lanes of its quarter), apply bias / GELU / positions /
+//               residual / SwiGLU, store to global memory, release the
+//               accumulator.  Two accumulators in TMEM let the epilogue of
+//               tile i overlap the MMAs of tile i+1.
+//   warps 6-9   (implicit-GEMM mode only) gather the A tile with 16-byte
+//               cp.async (zero fill for padding and tails) into the same
+//               swizzled layout, then fence the async proxy and arrive.
+// All waits are bounded (globaltimer); a role that gives up records a status
+// code, and the CTA drains its in-flight copies and MMAs before freeing
+// tensor memory and exiting.
+#pragma once
+
+#include "common.cuh"
+
+namespace asr {
+
+enum : int { EPI_GELU = 1, EPI_OUT_F32 = 2, EPI_RESID = 4, EPI_PE = 8, EPI_SWIGLU = 16 };
+
+struct ConvGather {
+  const bf16* x;  // activation [n_img, T_in, F_in, C] (C innermost)
+  int T_in, F_in, C;
+  int T_out, F_out;
+  int st, sf;     // strides along T and F
+  int kt, kf;     // kernel extents
+  int pt, pf;     // zero padding
+};
+
+struct GemmParams {
+  int M, N, K;
+  int m_blocks, n_blocks, k_blocks, num_tiles;
+  void* out;
+  long long ldo;          // output row stride in elements
+  const float* bias;      // [N] or null
+  const float* pe;        // [pe_period, N] or null
+  int pe_period;
+  ConvGather g;
+  int* status;
+  unsigned long long limit_ns;
+};
+
+static constexpr unsigned long long kDrainLimitNs = 200ull * 1000 * 1000;
+
+template <int BN_, int STAGES_, bool GATHER_>
+struct GemmShape {
+  static constexpr int BM = 128, BN = BN_, BK = 64, STAGES = STAGES_;
+  static constexpr bool GATHER = GATHER_;
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int ACC_COLS = (BN + 31) / 32 * 32;
+  static constexpr int TMEM_COLS =
+      2 * ACC_COLS <= 32 ? 32 : 2 * ACC_COLS <= 64 ? 64 : 2 * ACC_COLS <= 128 ? 128 : 2 * ACC_COLS <= 256 ? 256 : 512;
+  static constexpr int EPI_WARPS = 4;
+  static constexpr int GATHER_WARPS = GATHER ? 4 : 0;
+  static constexpr int GATHER_LAG = 2;
+  static constexpr int THREADS = 32 * (2 + EPI_WARPS + GATHER_WARPS);
+  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5) + 16;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
+  static_assert(2 * ACC_COLS <= 512, "two accumulators must fit in TMEM");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+};
+
+template <int EPI>
+__device__ __forceinline__ void epilogue_store16(const GemmParams& p, int row, int n, float* v, float* u) {
+  if (p.bias) {
+    const float4* b4 = reinterpret_cast<const float4*>(p.bias + n);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float4 b = __ldg(b4 + i);
+      v[4 * i] += b.x; v[4 * i + 1] += b.y; v[4 * i + 2] += b.z; v[4 * i + 3] += b.w;
+    }
+    if (EPI & EPI_SWIGLU) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float4 b = __ldg(b4 + 4 + i);
+        u[4 * i] += b.x; u[4 * i + 1] += b.y; u[4 * i + 2] += b.z; u[4 * i + 3] += b.w;
+      }
+    }
+  }
+  if (EPI & EPI_SWIGLU) {
+    // gate = v (columns n..n+15), up = u (n+16..n+31) -> 16 outputs at n/2.
+    bf16* o = reinterpret_cast<bf16*>(p.out) + (long long)row * p.ldo + (n >> 1);
+    alignas(16) __nv_bfloat162 r[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      r[i] = __floats2bfloat162_rn(silu(v[2 * i]) * u[2 * i], silu(v[2 * i + 1]) * u[2 * i + 1]);
+    uint4* o4 = reinterpret_cast<uint4*>(o);
+    o4[0] = reinterpret_cast<uint4*>(r)[0];
+    o4[1] = reinterpret_cast<uint4*>(r)[1];
+    return;
+  }
+  if (EPI & EPI_GELU) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = gelu_erf(v[i]);
+  }
+  if (EPI & EPI_PE) {
+    const float4* pe4 = reinterpret_cast<const float4*>(p.pe + (long long)(row % p.pe_period) * p.N + n);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float4 e = __ldg(pe4 + i);
+      v[4 * i] += e.x; v[4 * i + 1] += e.y; v[4 * i + 2] += e.z; v[4 * i + 3] += e.w;
+    }
+  }
+  if (EPI & (EPI_OUT_F32 | EPI_RESID)) {
+    float4* o4 = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (long long)row * p.ldo + n);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float4 r = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      if (EPI & EPI_RESID) {
+        float4 x = o4[i];
+        r.x += x.x; r.y += x.y; r.z += x.z; r.w += x.w;
+      }
+      o4[i] = r;
+    }
+  } else {
+    bf16* o = reinterpret_cast<bf16*>(p.out) + (long long)row * p.ldo + n;
+    alignas(16) __nv_bfloat162 r[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) r[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+    uint4* o4 = reinterpret_cast<uint4*>(o);
+    o4[0] = reinterpret_cast<uint4*>(r)[0];
+    o4[1] = reinterpret_cast<uint4*>(r)[1];
+  }
+}
+
+template <int BN, int STAGES, bool GATHER, int EPI>
+__global__ void __launch_bounds__(GemmShape<BN, STAGES, GATHER>::THREADS, 1)
+    gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const GemmParams p) {
+  using S = GemmShape<BN, STAGES, GATHER>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * S::A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * S::STAGE_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], GATHER ? 1 + 32 * S::GATHER_WARPS : 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], S::EPI_WARPS);
+    }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmB);
+    if (!GATHER) tma_prefetch_desc(&tmA);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, S::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+        const int m0 = (t % p.m_blocks) * S::BM;
+        const int n0 = (t / p.m_blocks) * BN;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait_bounded(&empty[s], ph ^ 1, p.limit_ns, p.status, DEV_TIMEOUT_PRODUCER)) {
+            ok = false;
+            break;
+          }
+          if (GATHER) {
+            mbar_arrive_expect_tx(&full[s], S::B_BYTES);
+          } else {
+            mbar_arrive_expect_tx(&full[s], S::A_BYTES + S::B_BYTES);
+            tma_load_2d(sA + s * S::A_BYTES, &tmA, &full[s], kb * S::BK, m0);
+          }
+          tma_load_2d(sB + s * S::B_BYTES, &tmB, &full[s], kb * S::BK, n0);
+          ++it;
+        }
+      }
+      // Drain: every issued load must have landed before the CTA exits.
+      if (!GATHER) {
+        for (int s = 0; s < STAGES; ++s) {
+          if (it > s) {
+            const int last = s + ((it - 1 - s) / STAGES) * STAGES;
+            mbar_wait_bounded(&full[s], (last / STAGES) & 1, kDrainLimitNs, nullptr, 0);
+          }
+        }
+      } else {
+        // Gather mode: full[] also needs the gather warps' arrivals, which
+        // may be missing after a failure; the bound covers that case.
+        for (int s = 0; s < STAGES; ++s) {
+          if (it > s) {
+            const int last = s + ((it - 1 - s) / STAGES) * STAGES;
+            if (!ok || *reinterpret_cast<volatile int*>(p.status) != 0)
+              mbar_wait_bounded(&full[s], (last / STAGES) & 1, kDrainLimitNs / 20, nullptr, 0);
+            else
+              mbar_wait_bounded(&full[s], (last / STAGES) & 1, kDrainLimitNs, nullptr, 0);
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(S::BM, BN);
+      int it = 0, tl = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++tl) {
+        const int a = tl & 1;
+        const uint32_t aph = (tl >> 1) & 1;
+        if (!mbar_wait_bounded(&tempty[a], aph ^ 1, p.limit_ns, p.status, DEV_TIMEOUT_MMA)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + a * S::ACC_COLS;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait_bounded(&full[s], ph, p.limit_ns, p.status, DEV_TIMEOUT_MMA)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + s * S::A_BYTES));
+          const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + s * S::B_BYTES));
+#pragma unroll
+          for (int k = 0; k < S::BK / 16; ++k)
+            tc_mma_bf16(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+          tc_commit(&empty[s]);
+          ++it;
+        }
+        if (!ok) break;
+        tc_commit(&tfull[a]);
+      }
+      // Drain: all issued MMAs complete before tensor memory is released.
+      tc_commit(drain);
+      mbar_wait_bounded(drain, 0, kDrainLimitNs, nullptr, 0);
+    }
+  } else if (warp < 2 + S::EPI_WARPS) {
+    // ------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    int tl = 0;
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++tl) {
+      const int a = tl & 1;
+      const uint32_t aph = (tl >> 1) & 1;
+      if (!mbar_wait_bounded(&tfull[a], aph, p.limit_ns, p.status, DEV_TIMEOUT_EPILOGUE)) break;
+      tc_fence_after();
+      const int m0 = (t % p.m_blocks) * S::BM;
+      const int n0 = (t / p.m_blocks) * BN;
+      const int row = m0 + 32 * q + lane;
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + a * S::ACC_COLS;
+      constexpr int STEP = (EPI & EPI_SWIGLU) ? 32 : 16;
+#pragma unroll 1
+      for (int c = 0; c < BN; c += STEP) {
+        float v[16], u[16];
+        tmem_ld16(tb + c, v);
+        if (EPI & EPI_SWIGLU) tmem_ld16(tb + c + 16, u);
+        tmem_ld_wait();
+        const int n = n0 + c;
+        if (row < p.M && n < p.N) epilogue_store16<EPI>(p, row, n, v, u);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[a]);
+    }
+  } else if (GATHER) {
+    // ------------------------------------------------ implicit-GEMM gather
+    const int gt = threadIdx.x - 32 * (2 + S::EPI_WARPS);  // 0..127
+    const int chunk = gt & 7;                               // 16-byte chunk of a 128-byte row
+    const int rsub = gt >> 3;                               // rows rsub + 16 i
+    const ConvGather& g = p.g;
+    const int per_img = g.T_out * g.F_out;
+    int it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+      const int m0 = (t % p.m_blocks) * S::BM;
+      const bf16* rbase[8];
+      int tb[8], fb[8];
+      bool rv[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int m = m0 + rsub + 16 * i;
+        rv[i] = m < p.M;
+        const int mm = rv[i] ? m : 0;
+        const int img = mm / per_img;
+        const int rem = mm - img * per_img;
+        const int to = rem / g.F_out;
+        const int fo = rem - to * g.F_out;
+        tb[i] = to * g.st - g.pt;
+        fb[i] = fo * g.sf - g.pf;
+        rbase[i] = g.x + (long long)img * g.T_in * g.F_in * g.C;
+      }
+      for (int kb = 0; kb < p.k_blocks; ++kb) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (!mbar_wait_bounded(&empty[s], ph ^ 1, p.limit_ns, p.status, DEV_TIMEOUT_GATHER)) {
+          ok = false;
+          break;
+        }
+        const int k = kb * S::BK + chunk * 8;
+        const bool kv = k < p.K;
+        const int tap = kv ? k / g.C : 0;
+        const int c = k - tap * g.C;
+        const int dt = tap / g.kf;
+        const int df = tap - dt * g.kf;
+        uint8_t* dst_stage = sA + s * S::A_BYTES;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int row = rsub + 16 * i;
+          const int ti = tb[i] + dt;
+          const int fi = fb[i] + df;
+          const bool valid = kv && rv[i] && ti >= 0 && ti < g.T_in && fi >= 0 && fi < g.F_in;
+          const bf16* src = valid ? rbase[i] + ((long long)(ti * g.F_in + fi) * g.C + c) : g.x;
+          uint8_t* dst = dst_stage + row * 128 + ((chunk ^ (row & 7)) << 4);
+          cp_async_16_zfill(dst, src, valid);
+        }
+        cp_async_commit();
+        if (it >= S::GATHER_LAG) {
+          cp_async_wait<S::GATHER_LAG>();
+          fence_proxy_async_smem();
+          mbar_arrive(&full[(it - S::GATHER_LAG) % STAGES]);
+        }
+        ++it;
+      }
+    }
+    cp_async_wait<0>();
+    if (ok) {
+      fence_proxy_async_smem();
+      for (int j = (it > S::GATHER_LAG ? it - S::GATHER_LAG : 0); j < it; ++j) mbar_arrive(&full[j % STAGES]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, S::TMEM_COLS);
+}
+
+}  // namespace asr

@@ -1,0 +1,61 @@
+// Host-side declarations of the kernel launchers (one definition each, in
+// mel.cu, stem.cu, layer.cu, gemm.cu).
+#pragma once
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "gemm.cuh"
+
+namespace asr {
+
+// Tables of the log-mel kernel, computed on the host in double precision.
+struct MelTables {
+  float2 w200[200];   // exp(-2 pi i j / 200)
+  float2 w400[201];   // exp(-2 pi i k / 400)
+  float hann[400];    // periodic Hann
+  int fstart[128], fcount[128], foff[128];
+  float fw[2048];     // non-zero filter weights, filter-major
+};
+
+cudaError_t launch_log_mel(const float* pcm, long long n_samples, int batch, int n_mels, const MelTables* tab,
+                           float* mel_raw, unsigned int* clip_max, cudaStream_t st);
+cudaError_t launch_mel_normalize(const float* raw, const unsigned int* clip_max, long long per_clip, int batch,
+                                 float* out, cudaStream_t st);
+cudaError_t launch_mel_normalize_transpose(const float* raw, const unsigned int* clip_max, int batch, int n_mels,
+                                           int n_frames, bf16* out, cudaStream_t st);
+
+// Conv2D 1 -> C, k3 s2 p1, + bias + GELU over each chunk of chunk_frames
+// frames of the (normalised on the fly) log-mel.  Output [chunks, T1, F1, C].
+cudaError_t launch_conv1_chunked(const float* mel_raw, const unsigned int* clip_max, int batch, int n_mels,
+                                 int n_frames, int chunk_frames, const float* w /*[C][9] (kh,kw)*/,
+                                 const float* b, int C, bf16* out, cudaStream_t st);
+
+cudaError_t launch_layer_norm(const float* x, const float* g, const float* b, long long M, int D, float eps,
+                              void* y, bool out_f32, cudaStream_t st);
+
+cudaError_t launch_attention(const bf16* qkv, const int* cu, int n_seg, int max_seg, int H, bf16* out,
+                             cudaStream_t st);
+
+cudaError_t launch_fill_windows(int* cu, int batch, int tokens_per_clip, int window, int n_win_per_clip,
+                                cudaStream_t st);
+cudaError_t launch_bf16_to_f32(const bf16* in, float* out, long long n, cudaStream_t st);
+cudaError_t launch_wait_probe(unsigned long long limit_ns, int* status, cudaStream_t st);
+
+// GEMM engine launch (gemm.cu).
+struct GemmB {              // weight operand [N, K] bf16 + its TMA maps
+  const bf16* ptr = nullptr;
+  int N = 0, K = 0;
+  CUtensorMap map[4];       // box rows 256, 128, 240, 64 (index by gemm_bn_slot)
+};
+int gemm_bn_slot(int bn);
+bool make_tmap_bf16(CUtensorMap* map, const void* ptr, unsigned long long rows, unsigned long long cols,
+                    unsigned long long row_stride_elems, unsigned int box_rows);
+bool make_weight_maps(GemmB& w);
+// Picks the tile width for an N x M problem on num_sms SMs.
+int gemm_pick_bn(int M, int N, int num_sms, bool gather);
+// a_map: TMA map of A (box 128 x 64), or null with p.g set for the implicit-GEMM mode.
+cudaError_t launch_gemm(const CUtensorMap* a_map, const GemmB& w, GemmParams p, int epi, int bn, int num_sms,
+                        cudaStream_t st);
+
+}  // namespace asr

@@ -1,0 +1,96 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+that include/*.h declares, and its host-only queries (token counts, window
+partitions, weight order) agree bit-exactly with the oracle and the seeded
+generators."""
+import ctypes
+import glob
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+import speech_recognition_audio_b200 as sra
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names |= set(re.findall(r"\b(asr_(?:enc|op)_\w+)\s*\(", text))
+    return names
+
+
+def test_library_exports_every_declared_function():
+    declared = _declared()
+    assert len(declared) >= 20
+    lib = ctypes.CDLL(sra.LIB_PATH)
+    missing = [n for n in sorted(declared) if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+@pytest.mark.parametrize("gname,secs", [("tiny", 1), ("moss", 1), ("moss", 30), ("moss", 600),
+                                        ("whisper_small", 30), ("whisper_small", 1)])
+def test_tokens_match_oracle(gname, secs):
+    g = synth.GEOMETRIES[gname]
+    n = 16000 * secs
+    assert sra.tokens(g, n) == oracle.token_count(g, n)
+
+
+def test_tokens_reject_partial_chunks():
+    g = synth.GEOMETRIES["moss"]
+    assert sra.tokens(g, 16000 + 160) == -1
+    assert sra.tokens(g, 16000 + 1) == -1
+    assert sra.tokens(synth.GEOMETRIES["whisper_small"], 16000 + 1) == -1
+
+
+@pytest.mark.parametrize("wname", list(synth.WORKLOADS))
+def test_windows_match_oracle(wname):
+    w = synth.WORKLOADS[wname]
+    g = synth.GEOMETRIES[w.geometry]
+    cu = sra.windows(g, w.n_samples, w.batch)
+    ref = oracle.window_partition(g, w.n_samples, w.batch)
+    assert cu == ref.tolist()
+
+
+def test_windows_capacity_error():
+    g = synth.GEOMETRIES["moss"]
+    cu = (ctypes.c_int32 * 2)()
+    n = ctypes.c_int(2)
+    geo = sra.Geometry.of(g)
+    rc = sra.lib.asr_enc_windows(ctypes.byref(geo), 480000, 1, cu, ctypes.byref(n))
+    assert rc == 1
+    assert b"capacity" in sra.lib.asr_enc_last_error(None)
+
+
+@pytest.mark.parametrize("gname", list(synth.GEOMETRIES))
+def test_weight_order_matches_generator(gname):
+    g = synth.GEOMETRIES[gname]
+    names = sra.weight_names(g)
+    specs = [(n, tuple(s)) for n, s, _ in synth.weight_specs(g)]
+    assert names == specs
+
+
+def test_invalid_geometry_rejected():
+    bad = synth.GEOMETRIES["moss"].as_dict()
+    bad["head_dim"] = 80
+    assert sra.lib.asr_enc_weight_count(ctypes.byref(sra.Geometry.of(bad))) == -1
+    assert sra.tokens(bad, 16000) == -1
+    bad2 = synth.GEOMETRIES["moss"].as_dict()
+    bad2["n_fft"] = 512
+    with pytest.raises(sra.AsrError):
+        sra.windows(bad2, 16000, 1)
+
+
+def test_null_handle_calls_fail_cleanly():
+    assert sra.lib.asr_enc_sync_status(None) == 1
+    assert sra.lib.asr_enc_set_taps(None, 1) == 1
+    assert sra.lib.asr_enc_workspace_size(None, 16000, 1) == 0
+    sra.lib.asr_enc_destroy(None)
+    rc = sra.lib.asr_enc_forward(None, None, 16000, 1, None, None, None, 0, None)
+    assert rc == 1

@@ -1,0 +1,150 @@
+"""End-to-end parity of the encoder forward pass (GPU) against the oracle.
+
+Every workload runs through the C ABI (asr_enc_create / asr_enc_forward) on
+its seeded synthetic audio and random-init weights:
+  tiny 1 x 1 s (fp32 weights)    whole output + every stage tap
+  moss 1 x 30 s                  whole output
+  moss 16 x 30 s (the benchmark launch configuration)
+                                 sampled windows of several clips, exact by
+                                 window independence (oracle.encode_clip)
+  moss 1 x 600 s speech-like     sampled windows, including silent stretches
+  whisper-small 32 x 30 s        two whole clips (full attention)
+Tolerances: per-row cosine >= 0.999 and max row relative L2 <= 2e-2 for the
+encoder/adapter output; log-mel max abs <= 1e-3; token counts bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from parity import assert_encoder_parity, MEL_ABS_MAX
+
+pytestmark = pytest.mark.gpu
+
+sra = pytest.importorskip("speech_recognition_audio_b200")
+
+_CACHE = {}
+
+
+def _encoder(wname, affine=False, geometry=None, seed=None):
+    key = (wname, affine, geometry, seed)
+    if key not in _CACHE:
+        w = synth.WORKLOADS[wname]
+        g = geometry or synth.GEOMETRIES[w.geometry]
+        W = synth.make_weights(g, seed if seed is not None else w.weight_seed, affine=affine)
+        enc = sra.Encoder(g, {k: v.cuda() for k, v in W.items()})
+        _CACHE.clear()  # keep one large encoder resident at a time
+        torch.cuda.empty_cache()
+        _CACHE[key] = (enc, W, g)
+    return _CACHE[key]
+
+
+def _run(enc, pcm):
+    out = enc.forward(torch.from_numpy(pcm).cuda())
+    enc.sync_status()
+    return out.cpu().numpy()
+
+
+def test_tiny_full_with_taps():
+    enc, W, g = _encoder("tiny_1x1s")
+    w = synth.WORKLOADS["tiny_1x1s"]
+    pcm = synth.pcm_batch(w)
+    enc.set_taps(0b11111)
+    out = _run(enc, pcm)
+    taps = {}
+    ref = oracle.forward(pcm, W, g, taps=taps)
+    t = taps["clips"][0]
+    T = out.shape[1]
+    assert T == 13 == oracle.token_count(g, w.n_samples)
+    mel = enc.tap(sra.TAP_MEL, (1, g.n_mels, w.n_samples // 160)).cpu().numpy()[0]
+    assert np.abs(mel - t["mel"]).max() <= MEL_ABS_MAX
+    assert_encoder_parity(enc.tap(sra.TAP_STEM, (T, g.d_model)).cpu().numpy(), t["stem"], "stem")
+    assert_encoder_parity(enc.tap(sra.TAP_LAYER0, (T, g.d_model)).cpu().numpy(), t["layer0"], "layer0")
+    assert_encoder_parity(enc.tap(sra.TAP_ENCODER, (T, g.d_model)).cpu().numpy(), t["encoder"], "encoder")
+    assert_encoder_parity(enc.tap(sra.TAP_HEAD, (T, g.proj2_out)).cpu().numpy(), t["head"], "head")
+    assert_encoder_parity(out, ref, "adapter output")
+    enc.set_taps(0)
+
+
+def test_affine_biases_small_batch():
+    # Non-zero biases and LayerNorm affine parameters exercise every epilogue's
+    # bias path and the LN gain/shift; 2 clips x 3 s, windows of 104 > 39 tokens.
+    w = synth.WORKLOADS["tiny_1x1s"]
+    g = synth.GEOMETRIES["tiny"]
+    enc, W, _ = _encoder("tiny_1x1s", affine=True, seed=77)
+    pcm = np.stack([synth.pcm_clip(48000, 500), synth.pcm_clip(48000, 501)])
+    out = _run(enc, pcm)
+    ref = oracle.forward(pcm, W, g)
+    assert out.shape == (2, 39, g.adapter_out)
+    assert_encoder_parity(out, ref, "affine tiny")
+
+
+def test_moss_1x30s_full():
+    enc, W, g = _encoder("moss_1x30s")
+    pcm = synth.pcm_batch(synth.WORKLOADS["moss_1x30s"])
+    out = _run(enc, pcm)
+    assert out.shape == (1, 390, 2048)
+    ref = oracle.forward(pcm, W, g)
+    assert_encoder_parity(out, ref, "moss 1x30s")
+
+
+def _sampled(wname, picks):
+    w = synth.WORKLOADS[wname]
+    enc, W, g = _encoder(wname)
+    pcm = synth.pcm_batch(w)
+    enc.set_taps(1 << sra.TAP_MEL)
+    out = _run(enc, pcm)
+    mel = enc.tap(sra.TAP_MEL, (w.batch, g.n_mels, w.n_samples // 160)).cpu().numpy()
+    enc.set_taps(0)
+    T = oracle.token_count(g, w.n_samples)
+    assert out.shape == (w.batch, T, g.d_out)
+    cu = oracle.window_partition(g, w.n_samples, 1)
+    for b, j in picks:
+        ref_mel = oracle.log_mel(pcm[b], g.n_mels)
+        assert np.abs(mel[b] - ref_mel).max() <= MEL_ABS_MAX
+        ref = oracle.encode_clip(pcm[b], W, g, windows=[j] if j is not None else None)
+        rows = slice(int(cu[j]), int(cu[j + 1])) if j is not None else slice(0, T)
+        assert_encoder_parity(out[b, rows], ref, f"{wname} clip {b} window {j}")
+    return out
+
+
+def test_moss_16x30s_sampled():
+    _sampled("moss_16x30s", [(0, 0), (7, 3), (15, 2)])
+
+
+def test_moss_1x600s_sampled():
+    _sampled("moss_1x600s", [(0, 0), (0, 37), (0, 74)])
+
+
+def test_whisper_small_32x30s_sampled():
+    _sampled("whisper_small_32x30s", [(0, None), (31, None)])
+
+
+def test_host_forward_matches_device_forward():
+    enc, W, g = _encoder("tiny_1x1s")
+    pcm = np.stack([synth.pcm_clip(32000, 900 + b) for b in range(3)])
+    dev = _run(enc, pcm)
+    host = enc.forward_host(torch.from_numpy(pcm).pin_memory()).numpy()
+    np.testing.assert_array_equal(dev, host)
+
+
+def test_forward_rejects_bad_sizes():
+    enc, W, g = _encoder("tiny_1x1s")
+    pcm = torch.zeros((1, 16000 + 160), device="cuda")
+    with pytest.raises(sra.AsrError) as ei:
+        enc.forward(pcm)
+    assert ei.value.code == 2
+    pcm = torch.zeros((1, 16000), device="cuda")
+    small = torch.empty(1024, dtype=torch.uint8, device="cuda")
+    with pytest.raises(sra.AsrError) as ei:
+        enc.forward(pcm, workspace=small)
+    assert ei.value.code == 5
+
+
+def test_repeat_forward_deterministic():
+    enc, W, g = _encoder("tiny_1x1s")
+    pcm = synth.pcm_batch(synth.WORKLOADS["tiny_1x1s"], batch=2)
+    a = _run(enc, pcm)
+    b = _run(enc, pcm)
+    np.testing.assert_array_equal(a, b)

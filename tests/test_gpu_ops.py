@@ -1,0 +1,134 @@
+"""Kernel-level parity of the CUDA library against the oracle (GPU).
+
+Each op is called through the C ABI (include/asr_ops.h) on seeded inputs and
+compared element by element with the oracle's float64 definition of the same
+step, at sizes that span several tiles and a ragged tail.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+sra = pytest.importorskip("speech_recognition_audio_b200")
+
+
+def _bf16(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16)
+
+
+# ------------------------------------------------------------------ GEMM
+@pytest.mark.parametrize("M,N,K", [(1, 256, 64), (13, 64, 576), (100, 128, 72), (300, 512, 1280),
+                                   (1000, 1280, 1280), (777, 480, 4320), (6240, 3840, 1280),
+                                   (200, 768, 2304), (129, 2048, 8192)])
+def test_linear_bf16_bias(M, N, K):
+    rng = np.random.default_rng(M * 7 + N + K)
+    x = _bf16(rng.normal(size=(M, K)))
+    w = _bf16(rng.normal(size=(N, K)) * 0.05)
+    b = torch.from_numpy(rng.normal(size=N).astype(np.float32))
+    y = sra.linear(x.cuda(), w.cuda(), b.cuda(), sra.EPI_BF16)
+    torch.cuda.synchronize()
+    ref = oracle.linear(x.float().numpy(), w, b.numpy())
+    got = y.float().cpu().numpy()
+    err = np.abs(got - ref)
+    tol = 2.0 ** -8 * np.abs(ref) + 1e-3 * np.sqrt(K / 64) * 0.05
+    assert (err <= tol).all(), f"max err {err.max()} (M={M} N={N} K={K})"
+
+
+@pytest.mark.parametrize("epi", ["gelu", "f32", "resid", "swiglu"])
+def test_linear_epilogues(epi):
+    M, N, K = 333, 1024, 768
+    rng = np.random.default_rng(11)
+    x = _bf16(rng.normal(size=(M, K)))
+    w = _bf16(rng.normal(size=(N, K)) * 0.04)
+    b = torch.from_numpy(rng.normal(size=N).astype(np.float32) * 0.1)
+    acc = oracle.linear(x.float().numpy(), w, b.numpy())
+    if epi == "gelu":
+        got = sra.linear(x.cuda(), w.cuda(), b.cuda(), sra.EPI_BF16_GELU).float().cpu().numpy()
+        ref = oracle.gelu(acc)
+        assert np.abs(got - ref).max() <= 2.0 ** -8 * np.abs(ref).max() + 1e-3
+    elif epi == "f32":
+        got = sra.linear(x.cuda(), w.cuda(), b.cuda(), sra.EPI_F32).cpu().numpy()
+        np.testing.assert_allclose(got, acc, rtol=1e-4, atol=1e-4)
+    elif epi == "resid":
+        r0 = rng.normal(size=(M, N)).astype(np.float32)
+        out = torch.from_numpy(r0).cuda()
+        sra.linear(x.cuda(), w.cuda(), b.cuda(), sra.EPI_F32_RESID, out=out)
+        np.testing.assert_allclose(out.cpu().numpy(), r0 + acc, rtol=1e-4, atol=1e-4)
+    else:
+        # rows interleaved in blocks of 16: gate block j then up block j
+        wg, wu = w[: N // 2], w[N // 2:]
+        wi = torch.stack([wg.view(-1, 16, K), wu.view(-1, 16, K)], 1).reshape(N, K).contiguous()
+        got = sra.linear(x.cuda(), wi.cuda(), None, sra.EPI_SWIGLU).float().cpu().numpy()
+        xf = x.float().numpy()
+        ref = oracle.silu(oracle.linear(xf, wg)) * oracle.linear(xf, wu)
+        assert got.shape == (M, N // 2)
+        assert np.abs(got - ref).max() <= 2.0 ** -8 * np.abs(ref).max() + 2e-3
+
+
+# ------------------------------------------------------------------ mel
+@pytest.mark.parametrize("n_mels,secs,batch,speech", [(128, 1, 1, False), (128, 3, 2, False),
+                                                      (80, 2, 3, False), (128, 20, 1, True)])
+def test_log_mel(n_mels, secs, batch, speech):
+    pcm = np.stack([synth.pcm_clip(16000 * secs, 100 + b, speech) for b in range(batch)])
+    got = sra.log_mel(torch.from_numpy(pcm).cuda(), n_mels).cpu().numpy()
+    for b in range(batch):
+        ref = oracle.log_mel(pcm[b], n_mels)
+        assert np.abs(got[b] - ref).max() <= 1e-3
+
+
+def test_log_mel_ragged_frames():
+    # n/160 not a multiple of the kernel's frame group
+    pcm = synth.pcm_clip(160 * 123, 7)[None]
+    got = sra.log_mel(torch.from_numpy(pcm).cuda(), 128).cpu().numpy()[0]
+    ref = oracle.log_mel(pcm[0], 128)
+    assert got.shape == ref.shape == (128, 123)
+    assert np.abs(got - ref).max() <= 1e-3
+
+
+# ------------------------------------------------------------------ LN
+@pytest.mark.parametrize("M,D", [(1, 256), (77, 768), (6240, 1280), (5, 2048)])
+def test_layer_norm(M, D):
+    rng = np.random.default_rng(D + M)
+    x = (rng.normal(size=(M, D)) * 3 + 0.5).astype(np.float32)
+    g = (1 + 0.1 * rng.normal(size=D)).astype(np.float32)
+    b = (0.02 * rng.normal(size=D)).astype(np.float32)
+    ref = oracle.layer_norm(x.astype(np.float64), g, b, 1e-5)
+    y16 = sra.layer_norm(torch.from_numpy(x).cuda(), torch.from_numpy(g).cuda(), torch.from_numpy(b).cuda())
+    y32 = sra.layer_norm(torch.from_numpy(x).cuda(), torch.from_numpy(g).cuda(), torch.from_numpy(b).cuda(),
+                         out_f32=True)
+    np.testing.assert_allclose(y32.cpu().numpy(), ref, rtol=1e-4, atol=1e-4)
+    assert np.abs(y16.float().cpu().numpy() - ref).max() <= 2.0 ** -8 * np.abs(ref).max()
+
+
+# ------------------------------------------------------------------ attention
+@pytest.mark.parametrize("lens,H", [([13], 4), ([104, 104, 104, 78], 20), ([1, 5, 64, 65, 100, 128, 129], 3),
+                                    ([1500, 1500], 12)])
+def test_attention(lens, H):
+    rng = np.random.default_rng(sum(lens) + H)
+    T = sum(lens)
+    qkv = _bf16(rng.normal(size=(T, 3 * H * 64)))
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    got = sra.attention(qkv.cuda(), torch.from_numpy(cu).cuda(), H).float().cpu().numpy()
+    q = qkv.float().numpy()
+    d = H * 64
+    ref = oracle.attention_windows(q[:, :d], q[:, d:2 * d], q[:, 2 * d:], cu, H)
+    err = np.abs(got - ref).max()
+    assert err <= 2e-2, err
+    # rows of a one-token window copy the value row
+    if lens[0] == 1:
+        np.testing.assert_allclose(got[0], q[0, 2 * d:], atol=1e-2)
+
+
+# ------------------------------------------------------------------ bounded waits
+def test_wait_probe_times_out_and_context_survives():
+    st = sra.wait_probe(50_000_000)  # 50 ms
+    assert st == 6
+    # the context is still usable afterwards
+    x = torch.ones(1000, device="cuda")
+    assert float(x.sum().item()) == 1000.0
+    m = sra.log_mel(torch.from_numpy(synth.pcm_clip(16000, 1)[None]).cuda(), 128)
+    assert torch.isfinite(m).all()
