@@ -95,7 +95,7 @@ bool make_weight_maps(GemmB& w) {
 }
 
 int gemm_pick_bn(int M, int N, int num_sms, bool gather) {
-  if (N % 240 == 0 && N % 256 != 0 && N <= 480) return 240;
+  if (gather && N % 240 == 0 && N % 256 != 0 && N <= 480) return 240;
   if (N <= 64) return 64;
   const long long mb = (M + 127) / 128;
   long long best_cost = -1;
@@ -110,7 +110,6 @@ int gemm_pick_bn(int M, int N, int num_sms, bool gather) {
       best = bn;
     }
   }
-  (void)gather;
   return best;
 }
 
