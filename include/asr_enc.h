@@ -187,6 +187,18 @@ enum { ASR_TAP_MEL = 0, ASR_TAP_STEM = 1, ASR_TAP_LAYER0 = 2, ASR_TAP_ENCODER = 
 asr_status asr_enc_set_taps(asr_enc* e, unsigned mask);
 asr_status asr_enc_tap(asr_enc* e, int stage, float* dst, size_t dst_bytes, void* stream);
 
+/* ---- kernel timing (profiling) --------------------------------------------
+ * asr_enc_profile(e, 1) makes every later forward bracket each of its kernel
+ * launches with CUDA events on the forward's stream (small extra cost; do not
+ * enable inside CUDA-graph capture).  asr_enc_profile_read synchronises the
+ * last forward's stream and returns per-stage totals: up to max entries of
+ * (static name, milliseconds, launches); the return value is the number of
+ * stages written, or -1 on error.  asr_enc_last_launches returns how many
+ * kernels the last forward launched (always counted). */
+asr_status asr_enc_profile(asr_enc* e, int enable);
+int asr_enc_profile_read(asr_enc* e, int max, const char** names, double* ms, int* launches);
+int asr_enc_last_launches(const asr_enc* e);
+
 /* Message of the last failure on `e` (or process-wide when e is NULL). */
 const char* asr_enc_last_error(const asr_enc* e);
 

@@ -43,12 +43,16 @@ asr_status asr_op_log_mel(const float* pcm, int64_t n_samples, int batch, int n_
  *                           16 (gate rows 16j..16j+15, then the matching up
  *                           rows), y[:, 16j+i] = SiLU(gate) * up
  * Limits: K % 8 == 0, N % 16 == 0, M >= 1.  ws: device scratch of
- * >= asr_op_linear_ws_size() bytes (device status word). */
+ * >= asr_op_linear_ws_size() bytes (device status word).
+ * tile_n: output tile of one SM, 128 x tile_n (256, 160, 128 or 64; 160 needs
+ * N % 160 == 0), or of a CTA pair (two SMs, tcgen05 cta_group::2),
+ * 256 x -tile_n (-256 or -128); 0 = chosen from M, N and the SM count as in
+ * the forward pass. */
 enum { ASR_EPI_BF16 = 0, ASR_EPI_BF16_GELU = 1, ASR_EPI_F32_RESID = 2, ASR_EPI_F32 = 3,
        ASR_EPI_SWIGLU = 4 };
 size_t asr_op_linear_ws_size(void);
 asr_status asr_op_linear(const void* x, const void* w, const float* bias, int64_t M, int N, int K,
-                         int epi, void* y, void* ws, size_t ws_bytes, void* stream);
+                         int epi, int tile_n, void* y, void* ws, size_t ws_bytes, void* stream);
 
 /* LayerNorm over the last axis: y = (x - mean) / sqrt(var + eps) * g + b,
  * x device float32 [M, D], g/b device float32 [D], y device bf16 [M, D]
@@ -63,6 +67,11 @@ asr_status asr_op_layer_norm(const float* x, const float* g, const float* b, int
  * max_seg: the longest segment (sizes the launch grid).  head_dim 64. */
 asr_status asr_op_attention(const void* qkv, const int32_t* cu, int n_seg, int max_seg, int64_t T,
                             int H, void* out, void* stream);
+
+/* The GELU every kernel applies (bias-free): y[i] = x[i] Phi(x[i]), with
+ * Phi from the Abramowitz & Stegun 7.1.26 approximation of erf (absolute
+ * error <= 1.5e-7).  x, y: device float32 [n]. */
+asr_status asr_op_gelu(const float* x, float* y, int64_t n, void* stream);
 
 /* Bounded-wait self-check: launches one kernel that waits on a shared-memory
  * barrier that nothing ever completes, gives up after limit_ns nanoseconds

@@ -20,7 +20,7 @@ import ctypes
 import os
 
 __all__ = ["lib", "LIB_PATH", "AsrError", "Geometry", "tokens", "windows", "weight_names", "Encoder",
-           "log_mel", "linear", "layer_norm", "attention", "wait_probe", "TAP_MEL", "TAP_STEM",
+           "log_mel", "linear", "layer_norm", "attention", "gelu", "wait_probe", "TAP_MEL", "TAP_STEM",
            "TAP_LAYER0", "TAP_ENCODER", "TAP_HEAD", "EPI_BF16", "EPI_BF16_GELU", "EPI_F32_RESID",
            "EPI_F32", "EPI_SWIGLU"]
 
@@ -57,7 +57,7 @@ class Geometry(ctypes.Structure):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m speech_recognition_audio_b200.build` "
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python speech_recognition_audio_b200/build.py` "
                           "(there is no CPU fallback)")
     L = ctypes.CDLL(LIB_PATH)
     P, I, I64, SZ, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
@@ -76,12 +76,17 @@ def _load():
         "asr_enc_set_taps": (I, [P, ctypes.c_uint]),
         "asr_enc_tap": (I, [P, I, P, SZ, P]),
         "asr_enc_last_error": (ctypes.c_char_p, [P]),
+        "asr_enc_profile": (I, [P, I]),
+        "asr_enc_profile_read": (I, [P, I, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_double),
+                                     ctypes.POINTER(I)]),
+        "asr_enc_last_launches": (I, [P]),
         "asr_op_log_mel_ws_size": (SZ, [I]),
         "asr_op_log_mel": (I, [P, I64, I, I, P, P, SZ, P]),
         "asr_op_linear_ws_size": (SZ, []),
-        "asr_op_linear": (I, [P, P, P, I64, I, I, I, P, P, SZ, P]),
+        "asr_op_linear": (I, [P, P, P, I64, I, I, I, I, P, P, SZ, P]),
         "asr_op_layer_norm": (I, [P, P, P, I64, I, F, P, I, P]),
         "asr_op_attention": (I, [P, P, I, I, I64, I, P, P]),
+        "asr_op_gelu": (I, [P, P, I64, P]),
         "asr_op_wait_probe": (I, [I64, P, P]),
     }
     for name, (res, args) in sig.items():
@@ -291,7 +296,7 @@ def log_mel(pcm, n_mels: int, stream=None):
     return mel
 
 
-def linear(x, w, bias=None, epi: int = EPI_BF16, out=None, stream=None):
+def linear(x, w, bias=None, epi: int = EPI_BF16, out=None, tile_n: int = 0, stream=None):
     """x bf16 [M, K], w bf16 [N, K], bias f32 [N] -> epilogue(x w^T + bias) (see asr_ops.h)."""
     import torch
     M, K = x.shape
@@ -306,8 +311,8 @@ def linear(x, w, bias=None, epi: int = EPI_BF16, out=None, stream=None):
         else:
             raise ValueError("EPI_F32_RESID needs `out` (updated in place)")
     ws = torch.empty(int(lib.asr_op_linear_ws_size()), dtype=torch.uint8, device=x.device)
-    _check(lib.asr_op_linear(_ptr(x), _ptr(w), _ptr(bias), M, N, K, epi, _ptr(out), _ptr(ws), ws.numel(),
-                             _stream(stream)))
+    _check(lib.asr_op_linear(_ptr(x), _ptr(w), _ptr(bias), M, N, K, epi, int(tile_n), _ptr(out), _ptr(ws),
+                             ws.numel(), _stream(stream)))
     return out
 
 
@@ -329,6 +334,14 @@ def attention(qkv, cu, n_heads: int, stream=None):
     _check(lib.asr_op_attention(_ptr(qkv), _ptr(cu), len(cu_host) - 1, max_seg, T, n_heads, _ptr(out),
                                 _stream(stream)))
     return out
+
+
+def gelu(x, stream=None):
+    """The device GELU: x CUDA float32 -> float32 of the same shape."""
+    import torch
+    y = torch.empty_like(x)
+    _check(lib.asr_op_gelu(_ptr(x), _ptr(y), x.numel(), _stream(stream)))
+    return y
 
 
 def wait_probe(limit_ns: int, stream=None) -> int:

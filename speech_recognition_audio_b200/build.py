@@ -1,6 +1,7 @@
 """Build the in-tree shared library ``libasr_enc.so`` for sm_100a with nvcc.
 
-Usage: ``python -m speech_recognition_audio_b200.build`` (or ``build()``).
+Usage: ``python speech_recognition_audio_b200/build.py [--force]`` (run by path: importing
+the package itself loads the library).
 Objects go to ``_build/`` at the repository root; the library is written next
 to this file so that it travels with the source tree.  A rebuild happens only
 when a source or header is newer than the library (or ``force=True``).

@@ -245,6 +245,12 @@ struct asr_enc {
   Plan last_plan;
   void* last_ws = nullptr;
   ActMaps maps;
+  // kernel timing
+  bool prof = false;
+  std::vector<cudaEvent_t> ev_pool;
+  size_t ev_used = 0;
+  std::vector<std::pair<int, size_t>> prof_recs;  // (stage class, index of the first of two events)
+  int launches = 0;
 };
 
 namespace {
@@ -359,6 +365,7 @@ const char* asr_enc_last_error(const asr_enc* e) {
 
 void asr_enc_destroy(asr_enc* e) {
   if (!e) return;
+  for (cudaEvent_t ev : e->ev_pool) cudaEventDestroy(ev);
   if (e->slab) {
     if (e->free_fn)
       e->free_fn(e->ctx, e->slab);
@@ -616,6 +623,7 @@ asr_status gemm(asr_enc* e, const CUtensorMap* amap, const ConvGather* cg, const
   if (cg) p.g = *cg;
   p.status = e->status;
   p.limit_ns = kWaitLimitNs;
+  p.n_fast = cg != nullptr;
   const int bn = gemm_pick_bn((int)M, w.N, e->num_sms, cg != nullptr);
   cudaError_t r = launch_gemm(amap, w, p, epi, bn, e->num_sms, st);
   if (r != cudaSuccess) return fail(e, ASR_E_CUDA, "gemm launch (N=%d K=%d M=%lld epi=%d bn=%d): %s", w.N, w.K, M, epi, bn, cudaGetErrorString(r));
@@ -631,6 +639,35 @@ asr_status gemm(asr_enc* e, const CUtensorMap* amap, const ConvGather* cg, const
   do {                                                                                                       \
     cudaError_t _r = (x);                                                                                    \
     if (_r != cudaSuccess) return fail((e), ASR_E_CUDA, "%s: %s", #x, cudaGetErrorString(_r));               \
+  } while (0)
+
+enum ProfClass { PC_MEL, PC_CONV1, PC_GEMM_CONV, PC_GEMM_CONVOUT, PC_GEMM_QKV, PC_GEMM_O, PC_GEMM_FC1, PC_GEMM_FC2,
+                 PC_GEMM_HEAD, PC_GEMM_ADAPTER, PC_LN, PC_ATTN, PC_MISC, PC_COUNT };
+const char* const kProfNames[PC_COUNT] = {"log_mel", "conv1", "gemm_conv", "gemm_conv_out", "gemm_qkv", "gemm_o",
+                                          "gemm_fc1", "gemm_fc2", "gemm_head", "gemm_adapter", "layer_norm",
+                                          "attention", "misc"};
+
+void prof_begin(asr_enc* e, int cls, cudaStream_t st) {
+  ++e->launches;
+  if (!e->prof) return;
+  while (e->ev_used + 2 > e->ev_pool.size()) {
+    cudaEvent_t ev;
+    if (cudaEventCreate(&ev) != cudaSuccess) return;
+    e->ev_pool.push_back(ev);
+  }
+  e->prof_recs.push_back({cls, e->ev_used});
+  cudaEventRecord(e->ev_pool[e->ev_used], st);
+  e->ev_used += 2;
+}
+void prof_end(asr_enc* e, cudaStream_t st) {
+  if (!e->prof || e->prof_recs.empty()) return;
+  cudaEventRecord(e->ev_pool[e->prof_recs.back().second + 1], st);
+}
+#define ASR_K(cls, stmt)          \
+  do {                            \
+    prof_begin(e, (cls), st);     \
+    stmt;                         \
+    prof_end(e, st);              \
   } while (0)
 
 asr_status ensure_maps(asr_enc* e, const Plan& p, char* ws) {
@@ -672,68 +709,71 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
   bf16* ff = reinterpret_cast<bf16*>(ws + p.off_ff);
   auto tap = [&](int t) -> float* { return ((e->taps >> t) & 1u) ? reinterpret_cast<float*>(ws + p.off_tap[t]) : nullptr; };
 
+  e->launches = 0;
+  e->ev_used = 0;
+  e->prof_recs.clear();
   ASR_LAUNCH(e, cudaMemsetAsync(e->status, 0, 4, st));
   ASR_LAUNCH(e, cudaMemsetAsync(clip_max, 0, (size_t)p.B * 4, st));
   const int w = g->window_tokens ? g->window_tokens : (int)p.Tc;
-  ASR_LAUNCH(e, launch_fill_windows(cu, p.B, (int)p.Tc, w, p.nwin_clip, st));
-  ASR_LAUNCH(e, launch_log_mel(pcm, p.n, p.B, g->n_mels, e->mel_tab, mel, clip_max, st));
-  if (float* t = tap(ASR_TAP_MEL)) ASR_LAUNCH(e, launch_mel_normalize(mel, clip_max, (long long)g->n_mels * p.F, p.B, t, st));
+  ASR_K(PC_MISC, ASR_LAUNCH(e, launch_fill_windows(cu, p.B, (int)p.Tc, w, p.nwin_clip, st)));
+  ASR_K(PC_MEL, ASR_LAUNCH(e, launch_log_mel(pcm, p.n, p.B, g->n_mels, e->mel_tab, mel, clip_max, st)));
+  if (float* t = tap(ASR_TAP_MEL)) ASR_K(PC_MISC, ASR_LAUNCH(e, launch_mel_normalize(mel, clip_max, (long long)g->n_mels * p.F, p.B, t, st)));
 
   if (g->stem == ASR_STEM_CONV2D_CHUNKED) {
     const int C = g->conv_ch;
     bf16* c1 = reinterpret_cast<bf16*>(ws + p.off_c1);
     bf16* c2 = reinterpret_cast<bf16*>(ws + p.off_c2);
     bf16* c3 = reinterpret_cast<bf16*>(ws + p.off_c3);
-    ASR_LAUNCH(e, launch_conv1_chunked(mel, clip_max, p.B, g->n_mels, p.F, g->chunk_frames, e->c1w, e->c1b, C, c1, st));
+    ASR_K(PC_CONV1, ASR_LAUNCH(e, launch_conv1_chunked(mel, clip_max, p.B, g->n_mels, p.F, g->chunk_frames, e->c1w, e->c1b, C, c1, st)));
     ConvGather cg2 = {c1, p.T1, p.F1, C, p.T2, p.F2, 2, 2, 3, 3, 1, 1};
-    ASR_TRY(gemm(e, nullptr, &cg2, e->c2, (long long)p.chunks * p.T2 * p.F2, c2, C, e->c2b, nullptr, 1, EPI_GELU, st));
+    ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, nullptr, &cg2, e->c2, (long long)p.chunks * p.T2 * p.F2, c2, C, e->c2b, nullptr, 1, EPI_GELU, st)));
     ConvGather cg3 = {c2, p.T2, p.F2, C, p.T3, p.F3, 2, 2, 3, 3, 1, 1};
-    ASR_TRY(gemm(e, nullptr, &cg3, e->c3, (long long)p.chunks * p.T3 * p.F3, c3, C, e->c3b, nullptr, 1, EPI_GELU, st));
-    ASR_TRY(gemm(e, &e->maps.c3, nullptr, e->cout, p.T, x, d, nullptr, e->pe, p.T3, EPI_OUT_F32 | EPI_PE, st));
+    ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, nullptr, &cg3, e->c3, (long long)p.chunks * p.T3 * p.F3, c3, C, e->c3b, nullptr, 1, EPI_GELU, st)));
+    ASR_K(PC_GEMM_CONVOUT, ASR_TRY(gemm(e, &e->maps.c3, nullptr, e->cout, p.T, x, d, nullptr, e->pe, p.T3, EPI_OUT_F32 | EPI_PE, st)));
   } else {
     if (p.Tc > e->pe_rows) return fail(e, ASR_E_UNSUPPORTED, "conv1d stem: %lld positions > %d", (long long)p.Tc, e->pe_rows);
     bf16* melT = reinterpret_cast<bf16*>(ws + p.off_melT);
     bf16* c1 = reinterpret_cast<bf16*>(ws + p.off_c1);
-    ASR_LAUNCH(e, launch_mel_normalize_transpose(mel, clip_max, p.B, g->n_mels, p.F, melT, st));
+    ASR_K(PC_MISC, ASR_LAUNCH(e, launch_mel_normalize_transpose(mel, clip_max, p.B, g->n_mels, p.F, melT, st)));
     ConvGather cg1 = {melT, p.F, 1, g->n_mels, p.F, 1, 1, 1, 3, 1, 1, 0};
-    ASR_TRY(gemm(e, nullptr, &cg1, e->c2, (long long)p.B * p.F, c1, d, e->c2b, nullptr, 1, EPI_GELU, st));
+    ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, nullptr, &cg1, e->c2, (long long)p.B * p.F, c1, d, e->c2b, nullptr, 1, EPI_GELU, st)));
     ConvGather cg2 = {c1, p.F, 1, d, (int)p.Tc, 1, 2, 1, 3, 1, 1, 0};
-    ASR_TRY(gemm(e, nullptr, &cg2, e->c3, p.T, x, d, e->c3b, e->pe, (int)p.Tc, EPI_GELU | EPI_OUT_F32 | EPI_PE, st));
+    ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, nullptr, &cg2, e->c3, p.T, x, d, e->c3b, e->pe, (int)p.Tc, EPI_GELU | EPI_OUT_F32 | EPI_PE, st)));
   }
   if (float* t = tap(ASR_TAP_STEM)) ASR_LAUNCH(e, cudaMemcpyAsync(t, x, (size_t)p.T * d * 4, cudaMemcpyDeviceToDevice, st));
 
   for (int l = 0; l < g->n_layers; ++l) {
     const LayerW& lw = e->layers[l];
-    ASR_LAUNCH(e, launch_layer_norm(x, lw.ln1g, lw.ln1b, p.T, d, g->ln_eps, h, false, st));
-    ASR_TRY(gemm(e, &e->maps.h, nullptr, lw.qkv, p.T, qkv, 3 * d, lw.bqkv, nullptr, 1, 0, st));
-    ASR_LAUNCH(e, launch_attention(qkv, cu, p.nwin, p.max_win, g->n_heads, att, st));
-    ASR_TRY(gemm(e, &e->maps.att, nullptr, lw.o, p.T, x, d, lw.bo, nullptr, 1, EPI_RESID, st));
-    ASR_LAUNCH(e, launch_layer_norm(x, lw.ln2g, lw.ln2b, p.T, d, g->ln_eps, h, false, st));
-    ASR_TRY(gemm(e, &e->maps.h, nullptr, lw.fc1, p.T, ff, g->d_ffn, lw.b1, nullptr, 1, EPI_GELU, st));
-    ASR_TRY(gemm(e, &e->maps.ff, nullptr, lw.fc2, p.T, x, d, lw.b2, nullptr, 1, EPI_RESID, st));
+    ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, lw.ln1g, lw.ln1b, p.T, d, g->ln_eps, h, false, st)));
+    ASR_K(PC_GEMM_QKV, ASR_TRY(gemm(e, &e->maps.h, nullptr, lw.qkv, p.T, qkv, 3 * d, lw.bqkv, nullptr, 1, 0, st)));
+    ASR_K(PC_ATTN, ASR_LAUNCH(e, launch_attention(qkv, cu, p.nwin, p.max_win, g->n_heads, att, st)));
+    ASR_K(PC_GEMM_O, ASR_TRY(gemm(e, &e->maps.att, nullptr, lw.o, p.T, x, d, lw.bo, nullptr, 1, EPI_RESID, st)));
+    ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, lw.ln2g, lw.ln2b, p.T, d, g->ln_eps, h, false, st)));
+    ASR_K(PC_GEMM_FC1, ASR_TRY(gemm(e, &e->maps.h, nullptr, lw.fc1, p.T, ff, g->d_ffn, lw.b1, nullptr, 1, EPI_GELU, st)));
+    ASR_K(PC_GEMM_FC2, ASR_TRY(gemm(e, &e->maps.ff, nullptr, lw.fc2, p.T, x, d, lw.b2, nullptr, 1, EPI_RESID, st)));
     if (l == 0)
       if (float* t = tap(ASR_TAP_LAYER0)) ASR_LAUNCH(e, cudaMemcpyAsync(t, x, (size_t)p.T * d * 4, cudaMemcpyDeviceToDevice, st));
   }
   if (float* t = tap(ASR_TAP_ENCODER)) ASR_LAUNCH(e, cudaMemcpyAsync(t, x, (size_t)p.T * d * 4, cudaMemcpyDeviceToDevice, st));
 
   if (!g->proj1_out) {
-    ASR_LAUNCH(e, launch_layer_norm(x, e->lnpg, e->lnpb, p.T, d, g->ln_eps, out, true, st));
+    ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, e->lnpg, e->lnpb, p.T, d, g->ln_eps, out, true, st)));
     return ASR_OK;
   }
   bf16* p1 = reinterpret_cast<bf16*>(ws + p.off_p1);
   bf16* p2 = reinterpret_cast<bf16*>(ws + p.off_p2);
-  ASR_LAUNCH(e, launch_layer_norm(x, e->lnpg, e->lnpb, p.T, d, g->ln_eps, h, false, st));
-  ASR_TRY(gemm(e, &e->maps.h, nullptr, e->p1, p.T, p1, g->proj1_out, e->bp1, nullptr, 1, EPI_GELU, st));
+  ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, e->lnpg, e->lnpb, p.T, d, g->ln_eps, h, false, st)));
+  ASR_K(PC_GEMM_HEAD, ASR_TRY(gemm(e, &e->maps.h, nullptr, e->p1, p.T, p1, g->proj1_out, e->bp1, nullptr, 1, EPI_GELU, st)));
   if (!g->adapter_hidden) {
-    ASR_TRY(gemm(e, &e->maps.p1, nullptr, e->p2, p.T, out, g->proj2_out, e->bp2, nullptr, 1, EPI_OUT_F32, st));
+    ASR_K(PC_GEMM_HEAD, ASR_TRY(gemm(e, &e->maps.p1, nullptr, e->p2, p.T, out, g->proj2_out, e->bp2, nullptr, 1, EPI_OUT_F32, st)));
     if (float* t = tap(ASR_TAP_HEAD)) ASR_LAUNCH(e, cudaMemcpyAsync(t, out, (size_t)p.T * g->proj2_out * 4, cudaMemcpyDeviceToDevice, st));
     return ASR_OK;
   }
-  ASR_TRY(gemm(e, &e->maps.p1, nullptr, e->p2, p.T, p2, g->proj2_out, e->bp2, nullptr, 1, 0, st));
-  if (float* t = tap(ASR_TAP_HEAD)) ASR_LAUNCH(e, launch_bf16_to_f32(p2, t, (long long)p.T * g->proj2_out, st));
+  ASR_K(PC_GEMM_HEAD, ASR_TRY(gemm(e, &e->maps.p1, nullptr, e->p2, p.T, p2, g->proj2_out, e->bp2, nullptr, 1, 0, st)));
+  if (float* t = tap(ASR_TAP_HEAD)) ASR_K(PC_MISC, ASR_LAUNCH(e, launch_bf16_to_f32(p2, t, (long long)p.T * g->proj2_out, st)));
   bf16* gu = reinterpret_cast<bf16*>(ws + p.off_gu);
-  ASR_TRY(gemm(e, &e->maps.p2, nullptr, e->gu, p.T, gu, g->adapter_hidden, nullptr, nullptr, 1, EPI_SWIGLU, st));
-  ASR_TRY(gemm(e, &e->maps.gu, nullptr, e->down, p.T, out, g->adapter_out, nullptr, nullptr, 1, EPI_OUT_F32, st));
+  ASR_K(PC_GEMM_ADAPTER, ASR_TRY(gemm(e, &e->maps.p2, nullptr, e->gu, p.T, gu, g->adapter_hidden, nullptr, nullptr, 1, EPI_SWIGLU, st)));
+  ASR_K(PC_GEMM_ADAPTER, ASR_TRY(gemm(e, &e->maps.gu, nullptr, e->down, p.T, out, g->adapter_out, nullptr, nullptr, 1, EPI_OUT_F32, st)));
   return ASR_OK;
 }
 
@@ -831,6 +871,37 @@ asr_status asr_enc_tap(asr_enc* e, int stage, float* dst, size_t dst_bytes, void
   return ASR_OK;
 }
 
+asr_status asr_enc_profile(asr_enc* e, int enable) {
+  if (!e) return fail(nullptr, ASR_E_INVAL, "handle is NULL");
+  e->prof = enable != 0;
+  return ASR_OK;
+}
+
+int asr_enc_profile_read(asr_enc* e, int max, const char** names, double* ms, int* launches) {
+  if (!e || max < 0) return -1;
+  if (!e->have_last) return 0;
+  if (cudaStreamSynchronize(e->last_stream) != cudaSuccess) return -1;
+  double tot[PC_COUNT] = {0};
+  int cnt[PC_COUNT] = {0};
+  for (auto& r : e->prof_recs) {
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, e->ev_pool[r.second], e->ev_pool[r.second + 1]) != cudaSuccess) return -1;
+    tot[r.first] += t;
+    cnt[r.first] += 1;
+  }
+  int k = 0;
+  for (int c = 0; c < PC_COUNT && k < max; ++c) {
+    if (!cnt[c]) continue;
+    if (names) names[k] = kProfNames[c];
+    if (ms) ms[k] = tot[c];
+    if (launches) launches[k] = cnt[c];
+    ++k;
+  }
+  return k;
+}
+
+int asr_enc_last_launches(const asr_enc* e) { return e ? e->launches : -1; }
+
 // ==================================================================== ops
 
 size_t asr_op_log_mel_ws_size(int batch) { return batch > 0 ? align_up((size_t)batch * 4, 256) : 0; }
@@ -868,8 +939,8 @@ asr_status asr_op_log_mel(const float* pcm, int64_t n_samples, int batch, int n_
 
 size_t asr_op_linear_ws_size(void) { return 256; }
 
-asr_status asr_op_linear(const void* x, const void* w, const float* bias, int64_t M, int N, int K, int epi, void* y,
-                         void* ws, size_t ws_bytes, void* stream) {
+asr_status asr_op_linear(const void* x, const void* w, const float* bias, int64_t M, int N, int K, int epi,
+                         int tile_n, void* y, void* ws, size_t ws_bytes, void* stream) {
   if (!x || !w || !y || M <= 0 || N <= 0 || K <= 0 || K % 8 || N % 16)
     return fail(nullptr, ASR_E_INVAL, "linear: bad arguments (K %% 8, N %% 16)");
   if (!ws || ws_bytes < 256) return fail(nullptr, ASR_E_WORKSPACE, "linear: workspace too small");
@@ -906,7 +977,10 @@ asr_status asr_op_linear(const void* x, const void* w, const float* bias, int64_
   p.pe_period = 1;
   p.status = static_cast<int*>(ws);
   p.limit_ns = kWaitLimitNs;
-  const int bn = gemm_pick_bn((int)M, N, sms, false);
+  if (tile_n && tile_n != 256 && tile_n != 160 && tile_n != 128 && tile_n != 64 && tile_n != -256 && tile_n != -128)
+    return fail(nullptr, ASR_E_INVAL, "linear: tile_n must be 0, 256, 160, 128, 64, -256 or -128");
+  if (tile_n == 160 && N % 160) return fail(nullptr, ASR_E_INVAL, "linear: tile_n 160 needs N %% 160 == 0");
+  const int bn = tile_n ? tile_n : gemm_pick_bn((int)M, N, sms, false);
   ASR_CUDA(nullptr, launch_gemm(&amap, wb, p, e_bits, bn, sms, st));
   return ASR_OK;
 }
@@ -924,6 +998,12 @@ asr_status asr_op_attention(const void* qkv, const int32_t* cu, int n_seg, int m
     return fail(nullptr, ASR_E_INVAL, "attention: bad arguments");
   ASR_CUDA(nullptr, launch_attention(static_cast<const bf16*>(qkv), cu, n_seg, max_seg, H, static_cast<bf16*>(out),
                                      static_cast<cudaStream_t>(stream)));
+  return ASR_OK;
+}
+
+asr_status asr_op_gelu(const float* x, float* y, int64_t n, void* stream) {
+  if (!x || !y || n <= 0) return fail(nullptr, ASR_E_INVAL, "gelu: bad arguments");
+  ASR_CUDA(nullptr, launch_gelu(x, y, n, static_cast<cudaStream_t>(stream)));
   return ASR_OK;
 }
 

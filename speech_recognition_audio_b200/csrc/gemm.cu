@@ -2,6 +2,7 @@
 // choice and dispatch to the kernel instantiations.
 #include <mutex>
 
+#include "gemm2.cuh"
 #include "kernels.h"
 
 namespace asr {
@@ -25,11 +26,11 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-constexpr int kSlotRows[4] = {256, 128, 240, 64};
+constexpr int kSlotRows[kGemmSlots] = {256, 128, 240, 64, 160};
 
 template <int BN>
 constexpr int stages_for() {
-  return BN >= 192 ? 4 : (BN >= 128 ? 6 : 8);
+  return BN >= 192 ? 4 : (BN > 128 ? 5 : (BN == 128 ? 6 : 8));
 }
 
 template <int BN, bool G, int EPI>
@@ -65,10 +66,45 @@ cudaError_t run_gather(int epi, const CUtensorMap& b, const GemmParams& p, int g
   }
 }
 
+template <int BN, int EPI>
+cudaError_t run2(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p, int grid, cudaStream_t st) {
+  using S = Gemm2Shape<BN, (BN >= 256 ? 6 : 8)>;
+  auto k = gemm_bf16_tc2_kernel<BN, S::STAGES, EPI>;
+  cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_BYTES);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(S::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = S::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, a, b, p);
+}
+
+template <int BN>
+cudaError_t run2_epi(int epi, const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p, int grid,
+                     cudaStream_t st) {
+  switch (epi) {
+    case 0: return run2<BN, 0>(a, b, p, grid, st);
+    case EPI_GELU: return run2<BN, EPI_GELU>(a, b, p, grid, st);
+    case EPI_OUT_F32: return run2<BN, EPI_OUT_F32>(a, b, p, grid, st);
+    case EPI_RESID: return run2<BN, EPI_RESID>(a, b, p, grid, st);
+    case EPI_OUT_F32 | EPI_PE: return run2<BN, EPI_OUT_F32 | EPI_PE>(a, b, p, grid, st);
+    case EPI_SWIGLU: return run2<BN, EPI_SWIGLU>(a, b, p, grid, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 }  // namespace
 
 int gemm_bn_slot(int bn) {
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < kGemmSlots; ++i)
     if (kSlotRows[i] == bn) return i;
   return -1;
 }
@@ -89,7 +125,7 @@ bool make_tmap_bf16(CUtensorMap* map, const void* ptr, unsigned long long rows, 
 }
 
 bool make_weight_maps(GemmB& w) {
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < kGemmSlots; ++i)
     if (!make_tmap_bf16(&w.map[i], w.ptr, w.N, w.K, w.K, kSlotRows[i])) return false;
   return true;
 }
@@ -97,24 +133,50 @@ bool make_weight_maps(GemmB& w) {
 int gemm_pick_bn(int M, int N, int num_sms, bool gather) {
   if (gather && N % 240 == 0 && N % 256 != 0 && N <= 480) return 240;
   if (N <= 64) return 64;
-  const long long mb = (M + 127) / 128;
+  // Estimated cost = waves x per-tile time.  A CTA pair computes a 256 x bn
+  // tile in about the time one SM needs for 128 x bn (the same per-SM MMA
+  // rate), slightly faster on long K thanks to its deeper pipeline.
   long long best_cost = -1;
   int best = 256;
-  for (int bn : {256, 128}) {
+  auto consider = [&](int bn, bool pair) {
+    const long long mb = pair ? (M + 255) / 256 : (M + 127) / 128;
+    const long long units = pair ? num_sms / 2 : num_sms;
     const long long tiles = mb * ((N + bn - 1) / bn);
-    const long long waves = (tiles + num_sms - 1) / num_sms;
-    // per-tile cost ~ columns + fixed overhead (epilogue drain, pipeline fill)
-    const long long cost = waves * (bn + 24);
+    const long long waves = (tiles + units - 1) / units;
+    const long long cost = waves * (bn + 32) * (pair ? 93 : 100);
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
-      best = bn;
+      best = pair ? -bn : bn;
     }
+  };
+  consider(256, false);
+  if (!gather && N % 160 == 0) consider(160, false);
+  consider(128, false);
+  if (!gather && M > 128) {
+    consider(256, true);
+    consider(128, true);
   }
   return best;
 }
 
 cudaError_t launch_gemm(const CUtensorMap* a_map, const GemmB& w, GemmParams p, int epi, int bn, int num_sms,
                         cudaStream_t st) {
+  if (bn < 0) {
+    // CTA-pair kernel: 256 x |bn| tiles, each CTA stages |bn|/2 rows of B.
+    const int w2 = -bn;
+    const int slot2 = gemm_bn_slot(w2 / 2);
+    if (!a_map || slot2 < 0 || p.M <= 0 || (w2 != 256 && w2 != 128)) return cudaErrorInvalidValue;
+    p.N = w.N;
+    p.K = w.K;
+    p.m_blocks = (p.M + 255) / 256;
+    p.n_blocks = (p.N + w2 - 1) / w2;
+    p.k_blocks = (p.K + 63) / 64;
+    p.num_tiles = p.m_blocks * p.n_blocks;
+    const int pairs = std::min(p.num_tiles, num_sms / 2);
+    const int grid = 2 * pairs;
+    return w2 == 256 ? run2_epi<256>(epi, *a_map, w.map[slot2], p, grid, st)
+                     : run2_epi<128>(epi, *a_map, w.map[slot2], p, grid, st);
+  }
   const int slot = gemm_bn_slot(bn);
   if (slot < 0 || p.M <= 0) return cudaErrorInvalidValue;
   p.N = w.N;
@@ -137,6 +199,7 @@ cudaError_t launch_gemm(const CUtensorMap* a_map, const GemmB& w, GemmParams p, 
   }
   switch (bn) {
     case 256: return run_tma<256>(epi, a_map, b, p, grid, st);
+    case 160: return run_tma<160>(epi, a_map, b, p, grid, st);
     case 128: return run_tma<128>(epi, a_map, b, p, grid, st);
     case 64: return run_tma<64>(epi, a_map, b, p, grid, st);
     default: return cudaErrorInvalidValue;

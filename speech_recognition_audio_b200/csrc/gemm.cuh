@@ -16,14 +16,19 @@
 //   warp 1      allocates tensor memory; lane 0 issues tcgen05.mma
 //               (M=128, N=BN, K=16) and commits to the ring's "empty"
 //               barriers and, per tile, to an accumulator "full" barrier.
-//   warps 2-5   epilogue: tcgen05.ld the accumulator (each warp owns the 32
-//               TMEM lanes of its quarter), apply bias / GELU / positions /
-//               residual / SwiGLU, store to global memory, release the
-//               accumulator.  Two accumulators in TMEM let the epilogue of
-//               tile i overlap the MMAs of tile i+1.
-//   warps 6-9   (implicit-GEMM mode only) gather the A tile with 16-byte
+//   warps 2-9   epilogue: tcgen05.ld the accumulator (a warp may only read
+//               the 32 TMEM lanes of its quarter, warp % 4; two warps share
+//               each quarter and take alternate 32-column groups), apply
+//               bias / GELU / SwiGLU, transpose through a per-warp shared
+//               buffer, add positions / the residual and store with
+//               coalesced accesses, release the accumulator.  Two
+//               accumulators in TMEM let the epilogue of tile i overlap the
+//               MMAs of tile i+1.
+//   warps 10-17 (implicit-GEMM mode only) gather the A tile with 16-byte
 //               cp.async (zero fill for padding and tails) into the same
-//               swizzled layout, then fence the async proxy and arrive.
+//               swizzled layout; each thread's copies arrive on the stage's
+//               full barrier when they land (cp.async.mbarrier.arrive.noinc),
+//               and the MMA thread fences the async proxy before reading.
 // All waits are bounded (globaltimer); a role that gives up records a status
 // code, and the CTA drains its in-flight copies and MMAs before freeing
 // tensor memory and exiting.
@@ -55,7 +60,21 @@ struct GemmParams {
   ConvGather g;
   int* status;
   unsigned long long limit_ns;
+  int n_fast;             // tile order: 1 = the n-blocks of an m-block run back to back
 };
+
+// Tile t -> (m block, n block).  With n_fast the tiles that share A rows run
+// on neighbouring CTAs at the same time, so A (the gathered activation of a
+// convolution) is fetched from DRAM once and re-read from L2.
+__device__ __forceinline__ void tile_coords(const GemmParams& p, int t, int& mb, int& nb) {
+  if (p.n_fast) {
+    nb = t % p.n_blocks;
+    mb = t / p.n_blocks;
+  } else {
+    mb = t % p.m_blocks;
+    nb = t / p.m_blocks;
+  }
+}
 
 static constexpr unsigned long long kDrainLimitNs = 200ull * 1000 * 1000;
 
@@ -69,77 +88,153 @@ struct GemmShape {
   static constexpr int ACC_COLS = (BN + 31) / 32 * 32;
   static constexpr int TMEM_COLS =
       2 * ACC_COLS <= 32 ? 32 : 2 * ACC_COLS <= 64 ? 64 : 2 * ACC_COLS <= 128 ? 128 : 2 * ACC_COLS <= 256 ? 256 : 512;
-  static constexpr int EPI_WARPS = 4;
-  static constexpr int GATHER_WARPS = GATHER ? 4 : 0;
-  static constexpr int GATHER_LAG = 2;
+  static constexpr int EPI_WARPS = 8;   // two per TMEM lane quarter, columns split between them
+  static constexpr int GATHER_WARPS = GATHER ? 8 : 0;
   static constexpr int THREADS = 32 * (2 + EPI_WARPS + GATHER_WARPS);
+  static constexpr int EPI_BUF_BYTES = EPI_WARPS * 4096;   // per-warp transpose buffers
   static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5) + 16;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BUF_BYTES + BAR_BYTES;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
   static_assert(2 * ACC_COLS <= 512, "two accumulators must fit in TMEM");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
+// Residual epilogues read 128 x BN fp32 values per tile; issuing L2
+// prefetches for the tile's rows before waiting for the accumulator moves that
+// DRAM latency under the tile's MMAs.  Each thread prefetches the 128-byte
+// lines of its own row in the 32-column groups its warp will handle.
+__device__ __forceinline__ void epilogue_prefetch_l2(const GemmParams& p, int t, int half, int q, int lane, int BN,
+                                                     int BM, int rank_rows) {
+  int mb, nb;
+  tile_coords(p, t, mb, nb);
+  const int m0 = mb * BM + rank_rows;
+  const int n0 = nb * BN;
+  const int row = m0 + 32 * q + lane;
+  if (row >= p.M) return;
+  const float* base = reinterpret_cast<const float*>(p.out) + (long long)row * p.ldo + n0;
+  for (int c = half * 32; c < BN && n0 + c < p.N; c += 64)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(base + c) : "memory");
+}
+
+// Epilogue of one warp: its 32 TMEM lanes (tile rows row0..row0+31) over the
+// 32-column groups g = half, half + 2, ... of a BN-wide accumulator.
+//   phase A (one thread per row): tcgen05.ld 32 columns, add the bias, apply
+//     GELU or SwiGLU, and write the row into the warp's 4 KB shared buffer
+//     (fp32, or bf16 for bf16 outputs; 16-byte chunks XOR-swizzled by row so
+//     that both phases are free of bank conflicts);
+//   phase B (threads along columns): read the buffer back so that a warp
+//     instruction covers whole 128-byte (fp32) or 64-byte (bf16) row
+//     segments, add positions / the residual with coalesced loads, and store
+//     with coalesced 16-byte (fp32) or 8-byte (bf16) stores.
 template <int EPI>
-__device__ __forceinline__ void epilogue_store16(const GemmParams& p, int row, int n, float* v, float* u) {
-  if (p.bias) {
-    const float4* b4 = reinterpret_cast<const float4*>(p.bias + n);
+__device__ __forceinline__ void epilogue_warp(const GemmParams& p, uint32_t tb, int row0, int n0, int BN, int half,
+                                              int lane, uint8_t* wbuf) {
+  constexpr bool F32 = (EPI & (EPI_OUT_F32 | EPI_RESID)) != 0;
+  constexpr bool SWI = (EPI & EPI_SWIGLU) != 0;
+#pragma unroll 1
+  for (int c = half * 32; c < BN; c += 64) {
+    const int n = n0 + c;
+    if (n >= p.N) break;                                  // warp-uniform
+    const int w = (BN - c < 32 || p.N - n < 32) ? 16 : 32;  // valid columns in this group (N % 16 == 0)
+    float v[32];
+    tmem_ld16(tb + c, v);
+    if (BN - c >= 32) tmem_ld16(tb + c + 16, v + 16);
+    tmem_ld_wait();
+    // ---- phase A
+    if (p.bias) {
+      const float4* b4 = reinterpret_cast<const float4*>(p.bias + n);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float4 b = __ldg(b4 + i);
-      v[4 * i] += b.x; v[4 * i + 1] += b.y; v[4 * i + 2] += b.z; v[4 * i + 3] += b.w;
-    }
-    if (EPI & EPI_SWIGLU) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float4 b = __ldg(b4 + 4 + i);
-        u[4 * i] += b.x; u[4 * i + 1] += b.y; u[4 * i + 2] += b.z; u[4 * i + 3] += b.w;
+      for (int i = 0; i < 8; ++i) {
+        if (i < 4 || w == 32) {
+          const float4 b = __ldg(b4 + i);
+          v[4 * i] += b.x; v[4 * i + 1] += b.y; v[4 * i + 2] += b.z; v[4 * i + 3] += b.w;
+        }
       }
     }
-  }
-  if (EPI & EPI_SWIGLU) {
-    // gate = v (columns n..n+15), up = u (n+16..n+31) -> 16 outputs at n/2.
-    bf16* o = reinterpret_cast<bf16*>(p.out) + (long long)row * p.ldo + (n >> 1);
-    alignas(16) __nv_bfloat162 r[8];
+    if (SWI) {
+      // gate = columns c..c+15, up = c+16..c+31 -> 16 bf16 outputs (2 chunks).
+      uint4* row = reinterpret_cast<uint4*>(wbuf + lane * 64);
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      r[i] = __floats2bfloat162_rn(silu(v[2 * i]) * u[2 * i], silu(v[2 * i + 1]) * u[2 * i + 1]);
-    uint4* o4 = reinterpret_cast<uint4*>(o);
-    o4[0] = reinterpret_cast<uint4*>(r)[0];
-    o4[1] = reinterpret_cast<uint4*>(r)[1];
-    return;
-  }
-  if (EPI & EPI_GELU) {
+      for (int k = 0; k < 2; ++k) {
+        alignas(16) __nv_bfloat162 r[4];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = gelu_erf(v[i]);
-  }
-  if (EPI & EPI_PE) {
-    const float4* pe4 = reinterpret_cast<const float4*>(p.pe + (long long)(row % p.pe_period) * p.N + n);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float4 e = __ldg(pe4 + i);
-      v[4 * i] += e.x; v[4 * i + 1] += e.y; v[4 * i + 2] += e.z; v[4 * i + 3] += e.w;
-    }
-  }
-  if (EPI & (EPI_OUT_F32 | EPI_RESID)) {
-    float4* o4 = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (long long)row * p.ldo + n);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float4 r = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-      if (EPI & EPI_RESID) {
-        float4 x = o4[i];
-        r.x += x.x; r.y += x.y; r.z += x.z; r.w += x.w;
+        for (int i = 0; i < 4; ++i) {
+          const int j = 8 * k + 2 * i;
+          r[i] = __floats2bfloat162_rn(silu(v[j]) * v[16 + j], silu(v[j + 1]) * v[17 + j]);
+        }
+        row[k ^ ((lane >> 1) & 3)] = *reinterpret_cast<uint4*>(r);
       }
-      o4[i] = r;
-    }
-  } else {
-    bf16* o = reinterpret_cast<bf16*>(p.out) + (long long)row * p.ldo + n;
-    alignas(16) __nv_bfloat162 r[8];
+    } else {
+      if (EPI & EPI_GELU) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) r[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-    uint4* o4 = reinterpret_cast<uint4*>(o);
-    o4[0] = reinterpret_cast<uint4*>(r)[0];
-    o4[1] = reinterpret_cast<uint4*>(r)[1];
+        for (int i = 0; i < 32; ++i) v[i] = gelu_erf(v[i]);
+      }
+      if (F32) {
+        float4* row = reinterpret_cast<float4*>(wbuf + lane * 128);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) row[k ^ (lane & 7)] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+      } else {
+        uint4* row = reinterpret_cast<uint4*>(wbuf + lane * 64);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          alignas(16) __nv_bfloat162 r[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) r[i] = __floats2bfloat162_rn(v[8 * k + 2 * i], v[8 * k + 2 * i + 1]);
+          row[k ^ ((lane >> 1) & 3)] = *reinterpret_cast<uint4*>(r);
+        }
+      }
+    }
+    __syncwarp();
+    // ---- phase B
+    if (F32) {
+      // 8 threads per row (float4 each), 4 rows per instruction, 8 passes.
+      const int k = lane & 7;
+      const int nc = n + 4 * k;
+      const bool col_ok = 4 * k < w;
+      float4 pre[8];
+      if (EPI & (EPI_RESID | EPI_PE)) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = (lane >> 3) + 4 * i;
+          const int row = row0 + r;
+          if (col_ok && row < p.M) {
+            if (EPI & EPI_RESID)
+              pre[i] = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.out) + (long long)row * p.ldo + nc);
+            else
+              pre[i] = __ldg(reinterpret_cast<const float4*>(p.pe + (long long)(row % p.pe_period) * p.N + nc));
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = (lane >> 3) + 4 * i;
+        const int row = row0 + r;
+        float4 x = reinterpret_cast<const float4*>(wbuf + r * 128)[k ^ (r & 7)];
+        if (col_ok && row < p.M) {
+          if (EPI & (EPI_RESID | EPI_PE)) {
+            x.x += pre[i].x; x.y += pre[i].y; x.z += pre[i].z; x.w += pre[i].w;
+          }
+          *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (long long)row * p.ldo + nc) = x;
+        }
+      }
+    } else {
+      // bf16: outputs per row = w (or w/2 for SwiGLU); 4 per thread (8 bytes).
+      const int wo = SWI ? w / 2 : w;
+      const int tpr = wo / 4;           // threads per row: 8 or 4 (or 2)
+      const int rpi = 32 / tpr;         // rows per pass
+      const int k4 = lane % tpr;        // which 4-column piece
+      const int rr = lane / tpr;
+      const long long ncol = SWI ? (n >> 1) + 4 * k4 : n + 4 * k4;
+#pragma unroll 1
+      for (int r = rr; r < 32; r += rpi) {
+        const int row = row0 + r;
+        const uint2* src = reinterpret_cast<const uint2*>(wbuf + r * 64);
+        const int chunk = (k4 >> 1) ^ ((r >> 1) & 3);
+        const uint2 val = src[2 * chunk + (k4 & 1)];
+        if (row < p.M) *reinterpret_cast<uint2*>(reinterpret_cast<bf16*>(p.out) + (long long)row * p.ldo + ncol) = val;
+      }
+    }
+    __syncwarp();
   }
 }
 
@@ -152,7 +247,8 @@ __global__ void __launch_bounds__(GemmShape<BN, STAGES, GATHER>::THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * S::A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * S::STAGE_BYTES);
+  uint8_t* sEpi = smem + STAGES * S::STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + S::EPI_BUF_BYTES);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   uint64_t* tfull = bars + 2 * STAGES;
@@ -194,8 +290,10 @@ __global__ void __launch_bounds__(GemmShape<BN, STAGES, GATHER>::THREADS, 1)
       int it = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
-        const int m0 = (t % p.m_blocks) * S::BM;
-        const int n0 = (t / p.m_blocks) * BN;
+        int mb, nb;
+        tile_coords(p, t, mb, nb);
+        const int m0 = mb * S::BM;
+        const int n0 = nb * BN;
         for (int kb = 0; kb < p.k_blocks; ++kb) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
@@ -257,6 +355,9 @@ __global__ void __launch_bounds__(GemmShape<BN, STAGES, GATHER>::THREADS, 1)
             ok = false;
             break;
           }
+          // cp.async wrote the A tile through the generic proxy; order those
+          // writes (observed through the barrier) before the MMA's reads.
+          if (GATHER) fence_proxy_async_smem();
           tc_fence_after();
           const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + s * S::A_BYTES));
           const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + s * S::B_BYTES));
@@ -275,48 +376,47 @@ __global__ void __launch_bounds__(GemmShape<BN, STAGES, GATHER>::THREADS, 1)
     }
   } else if (warp < 2 + S::EPI_WARPS) {
     // ------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int q = warp & 3;                   // TMEM lane quarter this warp may access
+    const int half = (warp - 2) / 4;          // which alternate column chunks it takes
+    const int rank_rows = 0;
     int tl = 0;
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++tl) {
       const int a = tl & 1;
       const uint32_t aph = (tl >> 1) & 1;
+      if (EPI & EPI_RESID) epilogue_prefetch_l2(p, t, half, q, lane, BN, S::BM, rank_rows);
       if (!mbar_wait_bounded(&tfull[a], aph, p.limit_ns, p.status, DEV_TIMEOUT_EPILOGUE)) break;
       tc_fence_after();
-      const int m0 = (t % p.m_blocks) * S::BM;
-      const int n0 = (t / p.m_blocks) * BN;
-      const int row = m0 + 32 * q + lane;
+      int mb, nb;
+      tile_coords(p, t, mb, nb);
+      const int m0 = mb * S::BM;
+      const int n0 = nb * BN;
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + a * S::ACC_COLS;
-      constexpr int STEP = (EPI & EPI_SWIGLU) ? 32 : 16;
-#pragma unroll 1
-      for (int c = 0; c < BN; c += STEP) {
-        float v[16], u[16];
-        tmem_ld16(tb + c, v);
-        if (EPI & EPI_SWIGLU) tmem_ld16(tb + c + 16, u);
-        tmem_ld_wait();
-        const int n = n0 + c;
-        if (row < p.M && n < p.N) epilogue_store16<EPI>(p, row, n, v, u);
-      }
+      epilogue_warp<EPI>(p, tb, m0 + 32 * q, n0, BN, half, lane, sEpi + (warp - 2) * 4096);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[a]);
     }
   } else if (GATHER) {
     // ------------------------------------------------ implicit-GEMM gather
-    const int gt = threadIdx.x - 32 * (2 + S::EPI_WARPS);  // 0..127
+    constexpr int RSTEP = (S::GATHER_WARPS > 0 ? S::GATHER_WARPS : 1) * 4;  // rows per pass (8 threads per row)
+    constexpr int NR = 128 / RSTEP;                         // passes over the 128-row tile
+    const int gt = threadIdx.x - 32 * (2 + S::EPI_WARPS);
     const int chunk = gt & 7;                               // 16-byte chunk of a 128-byte row
-    const int rsub = gt >> 3;                               // rows rsub + 16 i
+    const int rsub = gt >> 3;                               // rows rsub + RSTEP * i
     const ConvGather& g = p.g;
     const int per_img = g.T_out * g.F_out;
     int it = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
-      const int m0 = (t % p.m_blocks) * S::BM;
-      const bf16* rbase[8];
-      int tb[8], fb[8];
-      bool rv[8];
+      int mb, nb;
+      tile_coords(p, t, mb, nb);
+      const int m0 = mb * S::BM;
+      const bf16* rbase[NR];
+      int tb[NR], fb[NR];
+      bool rv[NR];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int m = m0 + rsub + 16 * i;
+      for (int i = 0; i < NR; ++i) {
+        const int m = m0 + rsub + RSTEP * i;
         rv[i] = m < p.M;
         const int mm = rv[i] ? m : 0;
         const int img = mm / per_img;
@@ -342,8 +442,8 @@ __global__ void __launch_bounds__(GemmShape<BN, STAGES, GATHER>::THREADS, 1)
         const int df = tap - dt * g.kf;
         uint8_t* dst_stage = sA + s * S::A_BYTES;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int row = rsub + 16 * i;
+        for (int i = 0; i < NR; ++i) {
+          const int row = rsub + RSTEP * i;
           const int ti = tb[i] + dt;
           const int fi = fb[i] + df;
           const bool valid = kv && rv[i] && ti >= 0 && ti < g.T_in && fi >= 0 && fi < g.F_in;
@@ -351,20 +451,12 @@ __global__ void __launch_bounds__(GemmShape<BN, STAGES, GATHER>::THREADS, 1)
           uint8_t* dst = dst_stage + row * 128 + ((chunk ^ (row & 7)) << 4);
           cp_async_16_zfill(dst, src, valid);
         }
-        cp_async_commit();
-        if (it >= S::GATHER_LAG) {
-          cp_async_wait<S::GATHER_LAG>();
-          fence_proxy_async_smem();
-          mbar_arrive(&full[(it - S::GATHER_LAG) % STAGES]);
-        }
+        // The barrier completes this thread's share when its copies land.
+        cp_async_arrive_noinc(&full[s]);
         ++it;
       }
     }
-    cp_async_wait<0>();
-    if (ok) {
-      fence_proxy_async_smem();
-      for (int j = (it > S::GATHER_LAG ? it - S::GATHER_LAG : 0); j < it; ++j) mbar_arrive(&full[j % STAGES]);
-    }
+    cp_async_wait_all();
   }
 
   tc_fence_before();

@@ -1,0 +1,255 @@
+// Two-SM variant of the tcgen05 GEMM engine: a CTA pair (cluster of 2)
+// computes 256 x BN output tiles with tcgen05.mma.cta_group::2 (M = 256).
+//
+// Each CTA of the pair stages its own 128 rows of A and its own BN/2 rows of
+// B (plain TMA loads, no multicast); the tensor cores of the pair exchange
+// the B halves, so every SM fetches a third less operand data per FLOP than
+// the one-SM 128 x BN tile, and each 32 KB stage covers twice the FLOPs of a
+// one-SM 48 KB stage, which is what hides L2 / HBM latency.  Accumulators:
+// each CTA's tensor memory holds its 128 rows x BN columns, twice (double
+// buffered).
+//
+// Roles (per CTA, 320 threads):
+//   warp 0  lane 0: TMA producer.  Both CTAs load into their own smem and
+//           signal the LEADER's full barrier (mapa to CTA rank 0); the leader
+//           arms it with the byte count of both halves.
+//   warp 1  allocates tensor memory (cta_group::2, both CTAs); in the leader,
+//           lane 0 issues the MMAs and commits, multicast to both CTAs, to
+//           the stage's empty barriers and the accumulator full barriers.
+//   warps 2-9  epilogue on the CTA's own TMEM rows; releases the accumulator
+//           with a remote arrive on the leader's accumulator-empty barrier.
+// Every wait is bounded; both CTAs meet at a cluster barrier before tensor
+// memory is freed.
+#pragma once
+
+#include "gemm.cuh"
+
+namespace asr {
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// TMA load into this CTA's smem, completion (bytes) reported to the barrier
+// at `bar_cluster_addr` (a shared::cluster address, here the leader's).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster_addr, int x,
+                                                 int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+      "[%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive (once each) on the barrier at the same offset in every CTA of `mask`
+// when the pair's previously issued MMAs complete.
+__device__ __forceinline__ void tc_commit_pair_mc(uint64_t* bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(mask)
+      : "memory");
+}
+
+template <int BN_, int STAGES_>
+struct Gemm2Shape {
+  static constexpr int BM = 256, BN = BN_, BK = 64, STAGES = STAGES_;
+  static constexpr int A_BYTES = 128 * BK * 2;        // this CTA's half of A
+  static constexpr int B_BYTES = (BN / 2) * BK * 2;   // this CTA's half of B
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TX_BYTES = 2 * STAGE_BYTES;    // both CTAs, counted on the leader
+  static constexpr int ACC_COLS = (BN + 31) / 32 * 32;
+  static constexpr int TMEM_COLS = 2 * ACC_COLS <= 64 ? 64 : 2 * ACC_COLS <= 128 ? 128 : 2 * ACC_COLS <= 256 ? 256 : 512;
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int THREADS = 32 * (2 + EPI_WARPS);
+  static constexpr int EPI_BUF_BYTES = EPI_WARPS * 4096;
+  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5) + 16;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BUF_BYTES + BAR_BYTES;
+  static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "UMMA N for M=256 (B halves of 16-row multiples)");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+};
+
+template <int BN, int STAGES, int EPI>
+__global__ void __launch_bounds__(Gemm2Shape<BN, STAGES>::THREADS, 1)
+    gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                         const GemmParams p) {
+  using S = Gemm2Shape<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * S::A_BYTES;
+  uint8_t* sEpi = smem + STAGES * S::STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + S::EPI_BUF_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0 = leader
+  const int pair = blockIdx.x >> 1;
+  const int n_pairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);   // leader: its own arrive.expect_tx (+ both CTAs' bytes)
+      mbar_init(&empty[s], 1);  // one multicast commit per stage use
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * S::EPI_WARPS);  // leader: epilogue warps of both CTAs
+    }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, S::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // barriers of both CTAs initialised before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint32_t full_leader0 = mapa_shared(smem_u32(&full[0]), 0);
+      int it = 0;
+      bool ok = true;
+      for (int t = pair; t < p.num_tiles && ok; t += n_pairs) {
+        int mb, nb;
+        tile_coords(p, t, mb, nb);
+        const int m0 = mb * S::BM + static_cast<int>(rank) * 128;
+        const int n0 = nb * BN + static_cast<int>(rank) * (BN / 2);
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait_bounded(&empty[s], ph ^ 1, p.limit_ns, p.status, DEV_TIMEOUT_PRODUCER)) {
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], S::TX_BYTES);
+          const uint32_t fb = full_leader0 + 8u * s;
+          tma_load_2d_pair(sA + s * S::A_BYTES, &tmA, fb, kb * S::BK, m0);
+          tma_load_2d_pair(sB + s * S::B_BYTES, &tmB, fb, kb * S::BK, n0);
+          ++it;
+        }
+      }
+      // Drain (leader sees both CTAs' bytes on its full barriers).
+      if (rank == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+          if (it > s) {
+            const int last = s + ((it - 1 - s) / STAGES) * STAGES;
+            mbar_wait_bounded(&full[s], (last / STAGES) & 1, kDrainLimitNs, nullptr, 0);
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc = idesc_bf16_f32(S::BM, BN);
+      int it = 0, tl = 0;
+      bool ok = true;
+      for (int t = pair; t < p.num_tiles && ok; t += n_pairs, ++tl) {
+        const int a = tl & 1;
+        const uint32_t aph = (tl >> 1) & 1;
+        if (!mbar_wait_bounded(&tempty[a], aph ^ 1, p.limit_ns, p.status, DEV_TIMEOUT_MMA)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + a * S::ACC_COLS;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait_bounded(&full[s], ph, p.limit_ns, p.status, DEV_TIMEOUT_MMA)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + s * S::A_BYTES));
+          const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + s * S::B_BYTES));
+#pragma unroll
+          for (int k = 0; k < S::BK / 16; ++k)
+            tc_mma_bf16_pair(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+          tc_commit_pair_mc(&empty[s], 0x3);
+          ++it;
+        }
+        if (!ok) break;
+        tc_commit_pair_mc(&tfull[a], 0x3);
+      }
+      tc_commit_pair_mc(drain, 0x1);
+      mbar_wait_bounded(drain, 0, kDrainLimitNs, nullptr, 0);
+    }
+  } else {
+    // epilogue: this CTA's 128 rows of the 256-row tile
+    const int q = warp & 3;
+    const int half = (warp - 2) / 4;
+    const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
+    const int rank_rows = static_cast<int>(rank) * 128;
+    int tl = 0;
+    for (int t = pair; t < p.num_tiles; t += n_pairs, ++tl) {
+      const int a = tl & 1;
+      const uint32_t aph = (tl >> 1) & 1;
+      if (EPI & EPI_RESID) epilogue_prefetch_l2(p, t, half, q, lane, BN, S::BM, rank_rows);
+      if (!mbar_wait_bounded(&tfull[a], aph, p.limit_ns, p.status, DEV_TIMEOUT_EPILOGUE)) break;
+      tc_fence_after();
+      int mb, nb;
+      tile_coords(p, t, mb, nb);
+      const int m0 = mb * S::BM + static_cast<int>(rank) * 128;
+      const int n0 = nb * BN;
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + a * S::ACC_COLS;
+      epilogue_warp<EPI>(p, tb, m0 + 32 * q, n0, BN, half, lane, sEpi + (warp - 2) * 4096);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8u * a);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the pair's MMAs are drained before either CTA frees TMEM
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, S::TMEM_COLS);
+}
+
+}  // namespace asr

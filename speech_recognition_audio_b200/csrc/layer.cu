@@ -298,6 +298,17 @@ cudaError_t launch_bf16_to_f32(const bf16* in, float* out, long long n, cudaStre
   return cudaGetLastError();
 }
 
+__global__ void gelu_kernel(const float* __restrict__ x, float* __restrict__ y, long long n) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+    y[i] = gelu_erf(x[i]);
+}
+
+cudaError_t launch_gelu(const float* x, float* y, long long n, cudaStream_t st) {
+  const int blocks = static_cast<int>(std::min<long long>((n + 255) / 256, 148LL * 32));
+  gelu_kernel<<<blocks, 256, 0, st>>>(x, y, n);
+  return cudaGetLastError();
+}
+
 // A barrier that nothing ever completes, waited on with the same bounded wait
 // as the GEMM pipeline: the wait gives up after limit_ns and records a status.
 __global__ void wait_probe_kernel(unsigned long long limit_ns, int* status) {

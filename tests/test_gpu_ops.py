@@ -38,6 +38,27 @@ def test_linear_bf16_bias(M, N, K):
     assert (err <= tol).all(), f"max err {err.max()} (M={M} N={N} K={K})"
 
 
+@pytest.mark.parametrize("tile_n", [256, 160, 128, 64, -256, -128])
+@pytest.mark.parametrize("M,N,K", [(6240, 1280, 1280), (300, 480, 4320), (257, 2560, 96)])
+def test_linear_tile_modes(tile_n, M, N, K):
+    """Every tile shape of the engine (one SM 128 x tile_n, or a CTA pair
+    256 x -tile_n) gives the same result, including ragged M and N tails."""
+    if tile_n == 160 and N % 160:
+        pytest.skip("160-wide tiles need N % 160 == 0")
+    rng = np.random.default_rng(M + N + K + tile_n)
+    x = _bf16(rng.normal(size=(M, K)))
+    w = _bf16(rng.normal(size=(N, K)) * 0.05)
+    b = torch.from_numpy(rng.normal(size=N).astype(np.float32))
+    r0 = rng.normal(size=(M, N)).astype(np.float32)
+    out = torch.from_numpy(r0).cuda()
+    sra.linear(x.cuda(), w.cuda(), b.cuda(), sra.EPI_F32_RESID, out=out, tile_n=tile_n)
+    ref = r0 + oracle.linear(x.float().numpy(), w, b.numpy())
+    np.testing.assert_allclose(out.cpu().numpy(), ref, rtol=1e-4, atol=2e-4 * np.sqrt(K / 64))
+    y = sra.linear(x.cuda(), w.cuda(), b.cuda(), sra.EPI_BF16_GELU, tile_n=tile_n).float().cpu().numpy()
+    g = oracle.gelu(ref - r0)
+    assert np.abs(y - g).max() <= 2.0 ** -8 * np.abs(g).max() + 1e-3
+
+
 @pytest.mark.parametrize("epi", ["gelu", "f32", "resid", "swiglu"])
 def test_linear_epilogues(epi):
     M, N, K = 333, 1024, 768
@@ -121,6 +142,19 @@ def test_attention(lens, H):
     # rows of a one-token window copy the value row
     if lens[0] == 1:
         np.testing.assert_allclose(got[0], q[0, 2 * d:], atol=1e-2)
+
+
+# ------------------------------------------------------------------ GELU
+def test_gelu_within_published_bound():
+    # The device GELU uses Abramowitz & Stegun 7.1.26 for erf (|error| <= 1.5e-7):
+    # |GELU - exact| <= |x| * 0.5 * 1.5e-7 plus fp32 rounding of the steps.
+    x = np.concatenate([np.linspace(-12, 12, 2_000_001), [0.0, -0.0, 1e-30, -1e-30, 40.0, -40.0]]).astype(np.float32)
+    got = sra.gelu(torch.from_numpy(x).cuda()).cpu().numpy().astype(np.float64)
+    ref = oracle.gelu(x.astype(np.float64))
+    err = np.abs(got - ref)
+    assert (err <= 1.2e-7 * np.abs(x) + 4e-7 * np.maximum(np.abs(ref), 1e-30)).all(), err.max()
+    assert got[-2] == 40.0 and abs(got[-1]) == 0.0
+    assert np.all(np.isfinite(got))
 
 
 # ------------------------------------------------------------------ bounded waits
