@@ -44,6 +44,7 @@ struct ActMaps {
   int batch = 0;
   unsigned taps = 0;
   CUtensorMap h, att, ff, c3, p1, p2, gu;
+  CUtensorMap cin2, cin3;  // conv-box A maps of the two stem GEMMs
 };
 
 struct Plan {
@@ -232,6 +233,7 @@ struct asr_enc {
   // stem
   float *c1w = nullptr, *c1b = nullptr, *c2b = nullptr, *c3b = nullptr;
   GemmB c2, c3, cout;
+  bool box2 = false, box3 = false;  // conv GEMMs read A as strided TMA boxes (else cp.async gather)
   float* pe = nullptr;
   int pe_rows = 0;
   std::vector<LayerW> layers;
@@ -452,15 +454,22 @@ asr_status asr_enc_create(const asr_geometry* g, const void* const* weights, int
     auto w1 = next();
     e->c1w = up_f32(w1);  // [C][kh*3+kw]
     e->c1b = up_f32(next());
+    // Conv-box mode needs F_out | 128 (a 128-row tile = whole output rows).
+    const int f1 = (int)conv_len(g->n_mels, 3, 2, 1), f2 = (int)conv_len(f1, 3, 2, 1);
+    e->box2 = f2 > 0 && 128 % f2 == 0 && (128 / f2) * 2 <= 256 && f2 * 2 <= 256;
+    e->box3 = f3 > 0 && 128 % f3 == 0 && (128 / f3) * 2 <= 256 && f3 * 2 <= 256;
     for (int layer = 0; layer < 2; ++layer) {
-      auto w = next();  // [o][c][kh][kw] -> [o][(kw*3+kh)*C + c]
-      std::vector<float> r((size_t)C * 9 * C);
+      // [o][c][kh][kw] -> [o][tap = kw*3+kh][c], channels padded to 64 per tap in box mode
+      auto w = next();
+      const bool box = layer == 0 ? e->box2 : e->box3;
+      const int cp = box ? (C + 63) / 64 * 64 : C;
+      std::vector<float> r((size_t)C * 9 * cp, 0.0f);
       for (int o = 0; o < C; ++o)
         for (int c = 0; c < C; ++c)
           for (int kh = 0; kh < 3; ++kh)
             for (int kw = 0; kw < 3; ++kw)
-              r[(size_t)o * 9 * C + (kw * 3 + kh) * C + c] = w[(((size_t)o * C + c) * 3 + kh) * 3 + kw];
-      if (!gemm_w(layer == 0 ? e->c2 : e->c3, r, C, 9 * C)) return bad(fail(e, ASR_E_CUDA, "conv weight upload / TMA map failed"));
+              r[(size_t)o * 9 * cp + (kw * 3 + kh) * cp + c] = w[(((size_t)o * C + c) * 3 + kh) * 3 + kw];
+      if (!gemm_w(layer == 0 ? e->c2 : e->c3, r, C, 9 * cp)) return bad(fail(e, ASR_E_CUDA, "conv weight upload / TMA map failed"));
       auto b = next();
       (layer == 0 ? e->c2b : e->c3b) = up_f32(b);
     }
@@ -471,20 +480,23 @@ asr_status asr_enc_create(const asr_geometry* g, const void* const* weights, int
         for (int f = 0; f < f3; ++f) r[(size_t)o * C * f3 + f * C + c] = wo[(size_t)o * C * f3 + c * f3 + f];
     if (!gemm_w(e->cout, r, d, C * f3)) return bad(fail(e, ASR_E_CUDA, "conv_out upload / TMA map failed"));
   } else {
+    // Conv1D stem: always conv-box mode (F_out = 1, 128 output frames per tile).
+    e->box2 = e->box3 = true;
     const int M = g->n_mels;
-    auto w1 = next();  // [d][c][k] -> [d][k*M + c]
-    std::vector<float> r1((size_t)d * 3 * M);
+    const int mp = (M + 63) / 64 * 64, dp = (d + 63) / 64 * 64;
+    auto w1 = next();  // [d][c][k] -> [d][k][c] with channels padded to 64
+    std::vector<float> r1((size_t)d * 3 * mp, 0.0f);
     for (int o = 0; o < d; ++o)
       for (int c = 0; c < M; ++c)
-        for (int k = 0; k < 3; ++k) r1[(size_t)o * 3 * M + k * M + c] = w1[((size_t)o * M + c) * 3 + k];
-    if (!gemm_w(e->c2, r1, d, 3 * M)) return bad(fail(e, ASR_E_CUDA, "conv1 upload failed"));
+        for (int k = 0; k < 3; ++k) r1[(size_t)o * 3 * mp + k * mp + c] = w1[((size_t)o * M + c) * 3 + k];
+    if (!gemm_w(e->c2, r1, d, 3 * mp)) return bad(fail(e, ASR_E_CUDA, "conv1 upload failed"));
     e->c2b = up_f32(next());
     auto w2 = next();
-    std::vector<float> r2((size_t)d * 3 * d);
+    std::vector<float> r2((size_t)d * 3 * dp, 0.0f);
     for (int o = 0; o < d; ++o)
       for (int c = 0; c < d; ++c)
-        for (int k = 0; k < 3; ++k) r2[(size_t)o * 3 * d + k * d + c] = w2[((size_t)o * d + c) * 3 + k];
-    if (!gemm_w(e->c3, r2, d, 3 * d)) return bad(fail(e, ASR_E_CUDA, "conv2 upload failed"));
+        for (int k = 0; k < 3; ++k) r2[(size_t)o * 3 * dp + k * dp + c] = w2[((size_t)o * d + c) * 3 + k];
+    if (!gemm_w(e->c3, r2, d, 3 * dp)) return bad(fail(e, ASR_E_CUDA, "conv2 upload failed"));
     e->c3b = up_f32(next());
   }
   e->layers.resize(L);
@@ -611,7 +623,8 @@ bool make_plan(const asr_enc* e, int64_t n, int B, Plan* p) {
 }
 
 asr_status gemm(asr_enc* e, const CUtensorMap* amap, const ConvGather* cg, const GemmB& w, long long M, void* out,
-                long long ldo, const float* bias, const float* pe, int period, int epi, cudaStream_t st) {
+                long long ldo, const float* bias, const float* pe, int period, int epi, cudaStream_t st,
+                const ConvBox* box = nullptr) {
   GemmParams p;
   memset(&p, 0, sizeof p);
   p.M = (int)M;
@@ -623,8 +636,15 @@ asr_status gemm(asr_enc* e, const CUtensorMap* amap, const ConvGather* cg, const
   if (cg) p.g = *cg;
   p.status = e->status;
   p.limit_ns = kWaitLimitNs;
-  p.n_fast = cg != nullptr;
-  const int bn = gemm_pick_bn((int)M, w.N, e->num_sms, cg != nullptr);
+  p.n_fast = cg != nullptr || box != nullptr;
+  int bn;
+  if (box) {
+    p.conv_box = 1;
+    p.cb = *box;
+    bn = gemm_pick_bn_conv(box->n_sub, w.N, e->num_sms);
+  } else {
+    bn = gemm_pick_bn((int)M, w.N, e->num_sms, cg != nullptr);
+  }
   cudaError_t r = launch_gemm(amap, w, p, epi, bn, e->num_sms, st);
   if (r != cudaSuccess) return fail(e, ASR_E_CUDA, "gemm launch (N=%d K=%d M=%lld epi=%d bn=%d): %s", w.N, w.K, M, epi, bn, cudaGetErrorString(r));
   return ASR_OK;
@@ -678,8 +698,15 @@ asr_status ensure_maps(asr_enc* e, const Plan& p, char* ws) {
   bool ok = make_tmap_bf16(&m.h, ws + p.off_h, p.T, d, d, 128) &&
             make_tmap_bf16(&m.att, ws + p.off_att, p.T, d, d, 128) &&
             make_tmap_bf16(&m.ff, ws + p.off_ff, p.T, g->d_ffn, g->d_ffn, 128);
-  if (ok && g->stem == ASR_STEM_CONV2D_CHUNKED)
-    ok = make_tmap_bf16(&m.c3, ws + p.off_c3, p.T, (size_t)p.F3 * g->conv_ch, (size_t)p.F3 * g->conv_ch, 128);
+  if (ok && g->stem == ASR_STEM_CONV2D_CHUNKED) {
+    const int C = g->conv_ch;
+    ok = make_tmap_bf16(&m.c3, ws + p.off_c3, p.T, (size_t)p.F3 * C, (size_t)p.F3 * C, 128);
+    if (ok && e->box2) ok = make_tmap_convbox(&m.cin2, ws + p.off_c1, C, p.F1, p.T1, p.chunks, p.F2, 2, 128 / p.F2, 2);
+    if (ok && e->box3) ok = make_tmap_convbox(&m.cin3, ws + p.off_c2, C, p.F2, p.T2, p.chunks, p.F3, 2, 128 / p.F3, 2);
+  } else if (ok) {
+    ok = make_tmap_convbox(&m.cin2, ws + p.off_melT, g->n_mels, 1, p.F, p.B, 1, 1, 128, 1) &&
+         make_tmap_convbox(&m.cin3, ws + p.off_c1, d, 1, p.F, p.B, 1, 1, 128, 2);
+  }
   if (ok && g->proj1_out)
     ok = make_tmap_bf16(&m.p1, ws + p.off_p1, p.T, g->proj1_out, g->proj1_out, 128) &&
          make_tmap_bf16(&m.p2, ws + p.off_p2, p.T, g->proj2_out, g->proj2_out, 128);
@@ -725,20 +752,34 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
     bf16* c2 = reinterpret_cast<bf16*>(ws + p.off_c2);
     bf16* c3 = reinterpret_cast<bf16*>(ws + p.off_c3);
     ASR_K(PC_CONV1, ASR_LAUNCH(e, launch_conv1_chunked(mel, clip_max, p.B, g->n_mels, p.F, g->chunk_frames, e->c1w, e->c1b, C, c1, st)));
-    ConvGather cg2 = {c1, p.T1, p.F1, C, p.T2, p.F2, 2, 2, 3, 3, 1, 1};
-    ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, nullptr, &cg2, e->c2, (long long)p.chunks * p.T2 * p.F2, c2, C, e->c2b, nullptr, 1, EPI_GELU, st)));
-    ConvGather cg3 = {c2, p.T2, p.F2, C, p.T3, p.F3, 2, 2, 3, 3, 1, 1};
-    ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, nullptr, &cg3, e->c3, (long long)p.chunks * p.T3 * p.F3, c3, C, e->c3b, nullptr, 1, EPI_GELU, st)));
+    const int CB = (C + 63) / 64;
+    if (e->box2) {
+      const int TR = 128 / p.F2, tpi = (p.T2 + TR - 1) / TR;
+      ConvBox b2 = {TR, p.F2, p.T2, tpi, p.chunks * tpi, 2, 2, 1, 1, 3, CB};
+      ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, &e->maps.cin2, nullptr, e->c2, (long long)p.chunks * p.T2 * p.F2, c2, C, e->c2b, nullptr, 1, EPI_GELU, st, &b2)));
+    } else {
+      ConvGather cg2 = {c1, p.T1, p.F1, C, p.T2, p.F2, 2, 2, 3, 3, 1, 1};
+      ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, nullptr, &cg2, e->c2, (long long)p.chunks * p.T2 * p.F2, c2, C, e->c2b, nullptr, 1, EPI_GELU, st)));
+    }
+    if (e->box3) {
+      const int TR = 128 / p.F3, tpi = (p.T3 + TR - 1) / TR;
+      ConvBox b3 = {TR, p.F3, p.T3, tpi, p.chunks * tpi, 2, 2, 1, 1, 3, CB};
+      ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, &e->maps.cin3, nullptr, e->c3, (long long)p.chunks * p.T3 * p.F3, c3, C, e->c3b, nullptr, 1, EPI_GELU, st, &b3)));
+    } else {
+      ConvGather cg3 = {c2, p.T2, p.F2, C, p.T3, p.F3, 2, 2, 3, 3, 1, 1};
+      ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, nullptr, &cg3, e->c3, (long long)p.chunks * p.T3 * p.F3, c3, C, e->c3b, nullptr, 1, EPI_GELU, st)));
+    }
     ASR_K(PC_GEMM_CONVOUT, ASR_TRY(gemm(e, &e->maps.c3, nullptr, e->cout, p.T, x, d, nullptr, e->pe, p.T3, EPI_OUT_F32 | EPI_PE, st)));
   } else {
     if (p.Tc > e->pe_rows) return fail(e, ASR_E_UNSUPPORTED, "conv1d stem: %lld positions > %d", (long long)p.Tc, e->pe_rows);
     bf16* melT = reinterpret_cast<bf16*>(ws + p.off_melT);
     bf16* c1 = reinterpret_cast<bf16*>(ws + p.off_c1);
     ASR_K(PC_MISC, ASR_LAUNCH(e, launch_mel_normalize_transpose(mel, clip_max, p.B, g->n_mels, p.F, melT, st)));
-    ConvGather cg1 = {melT, p.F, 1, g->n_mels, p.F, 1, 1, 1, 3, 1, 1, 0};
-    ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, nullptr, &cg1, e->c2, (long long)p.B * p.F, c1, d, e->c2b, nullptr, 1, EPI_GELU, st)));
-    ConvGather cg2 = {c1, p.F, 1, d, (int)p.Tc, 1, 2, 1, 3, 1, 1, 0};
-    ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, nullptr, &cg2, e->c3, p.T, x, d, e->c3b, e->pe, (int)p.Tc, EPI_GELU | EPI_OUT_F32 | EPI_PE, st)));
+    const int tpi1 = (p.F + 127) / 128, tpi2 = (int)((p.Tc + 127) / 128);
+    ConvBox b1 = {128, 1, p.F, tpi1, p.B * tpi1, 1, 1, 1, 0, 1, (g->n_mels + 63) / 64};
+    ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, &e->maps.cin2, nullptr, e->c2, (long long)p.B * p.F, c1, d, e->c2b, nullptr, 1, EPI_GELU, st, &b1)));
+    ConvBox b2 = {128, 1, (int)p.Tc, tpi2, p.B * tpi2, 2, 1, 1, 0, 1, (d + 63) / 64};
+    ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, &e->maps.cin3, nullptr, e->c3, p.T, x, d, e->c3b, e->pe, (int)p.Tc, EPI_GELU | EPI_OUT_F32 | EPI_PE, st, &b2)));
   }
   if (float* t = tap(ASR_TAP_STEM)) ASR_LAUNCH(e, cudaMemcpyAsync(t, x, (size_t)p.T * d * 4, cudaMemcpyDeviceToDevice, st));
 

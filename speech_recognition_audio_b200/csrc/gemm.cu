@@ -26,7 +26,7 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-constexpr int kSlotRows[kGemmSlots] = {256, 128, 240, 64, 160};
+constexpr int kSlotRows[kGemmSlots] = {256, 128, 240, 64, 160, 120};
 
 template <int BN>
 constexpr int stages_for() {
@@ -53,6 +53,17 @@ cudaError_t run_tma(int epi, const CUtensorMap* a, const CUtensorMap& b, const G
     case EPI_RESID: return run<BN, false, EPI_RESID>(a, b, p, grid, st);
     case EPI_OUT_F32 | EPI_PE: return run<BN, false, EPI_OUT_F32 | EPI_PE>(a, b, p, grid, st);
     case EPI_SWIGLU: return run<BN, false, EPI_SWIGLU>(a, b, p, grid, st);
+    case EPI_GELU | EPI_OUT_F32 | EPI_PE: return run<BN, false, EPI_GELU | EPI_OUT_F32 | EPI_PE>(a, b, p, grid, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// 240-wide tiles only serve the convolutions (N = 480).
+cudaError_t run_tma240(int epi, const CUtensorMap* a, const CUtensorMap& b, const GemmParams& p, int grid,
+                       cudaStream_t st) {
+  switch (epi) {
+    case EPI_GELU: return run<240, false, EPI_GELU>(a, b, p, grid, st);
+    case EPI_GELU | EPI_OUT_F32 | EPI_PE: return run<240, false, EPI_GELU | EPI_OUT_F32 | EPI_PE>(a, b, p, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -68,7 +79,7 @@ cudaError_t run_gather(int epi, const CUtensorMap& b, const GemmParams& p, int g
 
 template <int BN, int EPI>
 cudaError_t run2(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p, int grid, cudaStream_t st) {
-  using S = Gemm2Shape<BN, (BN >= 256 ? 6 : 8)>;
+  using S = Gemm2Shape<BN, (BN >= 192 ? 6 : 8)>;
   auto k = gemm_bf16_tc2_kernel<BN, S::STAGES, EPI>;
   cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_BYTES);
   if (err != cudaSuccess) return err;
@@ -97,6 +108,16 @@ cudaError_t run2_epi(int epi, const CUtensorMap& a, const CUtensorMap& b, const 
     case EPI_RESID: return run2<BN, EPI_RESID>(a, b, p, grid, st);
     case EPI_OUT_F32 | EPI_PE: return run2<BN, EPI_OUT_F32 | EPI_PE>(a, b, p, grid, st);
     case EPI_SWIGLU: return run2<BN, EPI_SWIGLU>(a, b, p, grid, st);
+    case EPI_GELU | EPI_OUT_F32 | EPI_PE: return run2<BN, EPI_GELU | EPI_OUT_F32 | EPI_PE>(a, b, p, grid, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t run2_240(int epi, const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p, int grid,
+                     cudaStream_t st) {
+  switch (epi) {
+    case EPI_GELU: return run2<240, EPI_GELU>(a, b, p, grid, st);
+    case EPI_GELU | EPI_OUT_F32 | EPI_PE: return run2<240, EPI_GELU | EPI_OUT_F32 | EPI_PE>(a, b, p, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -120,6 +141,21 @@ bool make_tmap_bf16(CUtensorMap* map, const void* ptr, unsigned long long rows, 
   cuuint32_t box[2] = {64, box_rows};
   cuuint32_t es[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tmap_convbox(CUtensorMap* map, const void* ptr, int C, int F_in, int T_in, int n_img, int F_out, int sf,
+                       int TR, int st) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || !ptr || (reinterpret_cast<uintptr_t>(ptr) & 15) || C % 8 || F_out * sf > 256 || TR * st > 256 ||
+      F_out * TR != 128 || sf < 1 || sf > 8 || st < 1 || st > 8)
+    return false;
+  cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)F_in, (cuuint64_t)T_in, (cuuint64_t)n_img};
+  cuuint64_t strides[3] = {(cuuint64_t)C * 2, (cuuint64_t)F_in * C * 2, (cuuint64_t)T_in * F_in * C * 2};
+  cuuint32_t box[4] = {64, (cuuint32_t)(F_out * sf), (cuuint32_t)(TR * st), 1};
+  cuuint32_t es[4] = {1, (cuuint32_t)sf, (cuuint32_t)st, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -159,21 +195,33 @@ int gemm_pick_bn(int M, int N, int num_sms, bool gather) {
   return best;
 }
 
+int gemm_pick_bn_conv(int n_sub, int N, int num_sms) {
+  // Convolution N is 480 (two 240-wide tiles) or d_model; pairs take two
+  // 128-row sub-tiles at once.
+  const int bn = (N % 240 == 0 && N % 256 != 0 && N <= 480) ? 240 : (N <= 64 ? 64 : (N % 256 == 0 ? 256 : 128));
+  if (bn == 64) return 64;
+  const long long nb = (N + bn - 1) / bn;
+  const long long w1 = ((long long)n_sub * nb + num_sms - 1) / num_sms;
+  const long long w2 = (((long long)n_sub + 1) / 2 * nb + num_sms / 2 - 1) / (num_sms / 2);
+  return (w2 * 93 <= w1 * 100) ? -bn : bn;
+}
+
 cudaError_t launch_gemm(const CUtensorMap* a_map, const GemmB& w, GemmParams p, int epi, int bn, int num_sms,
                         cudaStream_t st) {
   if (bn < 0) {
     // CTA-pair kernel: 256 x |bn| tiles, each CTA stages |bn|/2 rows of B.
     const int w2 = -bn;
     const int slot2 = gemm_bn_slot(w2 / 2);
-    if (!a_map || slot2 < 0 || p.M <= 0 || (w2 != 256 && w2 != 128)) return cudaErrorInvalidValue;
+    if (!a_map || slot2 < 0 || p.M <= 0 || (w2 != 256 && w2 != 128 && w2 != 240)) return cudaErrorInvalidValue;
     p.N = w.N;
     p.K = w.K;
-    p.m_blocks = (p.M + 255) / 256;
+    p.m_blocks = p.conv_box ? (p.cb.n_sub + 1) / 2 : (p.M + 255) / 256;
     p.n_blocks = (p.N + w2 - 1) / w2;
     p.k_blocks = (p.K + 63) / 64;
     p.num_tiles = p.m_blocks * p.n_blocks;
     const int pairs = std::min(p.num_tiles, num_sms / 2);
     const int grid = 2 * pairs;
+    if (w2 == 240) return run2_240(epi, *a_map, w.map[slot2], p, grid, st);
     return w2 == 256 ? run2_epi<256>(epi, *a_map, w.map[slot2], p, grid, st)
                      : run2_epi<128>(epi, *a_map, w.map[slot2], p, grid, st);
   }
@@ -181,7 +229,7 @@ cudaError_t launch_gemm(const CUtensorMap* a_map, const GemmB& w, GemmParams p, 
   if (slot < 0 || p.M <= 0) return cudaErrorInvalidValue;
   p.N = w.N;
   p.K = w.K;
-  p.m_blocks = (p.M + 127) / 128;
+  p.m_blocks = p.conv_box ? p.cb.n_sub : (p.M + 127) / 128;
   p.n_blocks = (p.N + bn - 1) / bn;
   p.k_blocks = (p.K + 63) / 64;
   p.num_tiles = p.m_blocks * p.n_blocks;
@@ -199,6 +247,7 @@ cudaError_t launch_gemm(const CUtensorMap* a_map, const GemmB& w, GemmParams p, 
   }
   switch (bn) {
     case 256: return run_tma<256>(epi, a_map, b, p, grid, st);
+    case 240: return run_tma240(epi, a_map, b, p, grid, st);
     case 160: return run_tma<160>(epi, a_map, b, p, grid, st);
     case 128: return run_tma<128>(epi, a_map, b, p, grid, st);
     case 64: return run_tma<64>(epi, a_map, b, p, grid, st);

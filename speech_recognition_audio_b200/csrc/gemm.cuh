@@ -49,6 +49,19 @@ struct ConvGather {
   int pt, pf;     // zero padding
 };
 
+// Convolution A operand read by TMA as strided boxes: the activation is
+// [n_img, T_in, F_in, C] (C innermost) and a 128-row tile is TR output
+// t-rows x all F_out columns of one image; for each tap and 64-channel block
+// one 4-D box {64, F_out * sf, TR * st, 1} with element strides {1, sf, st, 1}
+// lands the 128 x 64 A tile (zero fill outside the image = the padding).
+struct ConvBox {
+  int TR, F_out, T_out;   // output rows per tile, output geometry
+  int tiles_per_img;      // ceil(T_out / TR)
+  int n_sub;              // n_img * tiles_per_img 128-row sub-tiles
+  int st, sf, pt, pf;     // strides and padding along T and F
+  int kf, CB;             // taps along F, 64-channel blocks per tap
+};
+
 struct GemmParams {
   int M, N, K;
   int m_blocks, n_blocks, k_blocks, num_tiles;
@@ -61,7 +74,53 @@ struct GemmParams {
   int* status;
   unsigned long long limit_ns;
   int n_fast;             // tile order: 1 = the n-blocks of an m-block run back to back
+  int conv_box;           // 1 = A is a ConvBox (4-D strided TMA), rows mapped per image
+  ConvBox cb;
 };
+
+// Output rows covered by 128-row sub-tile u: [first, last) (conv-box mode
+// maps a sub-tile to TR output t-rows of one image; rows past the image end
+// are padding).  Plain mode: rows u*128 .. u*128+127 clipped at M.
+__device__ __forceinline__ void subtile_rows(const GemmParams& p, int u, int& first, int& last) {
+  if (p.conv_box) {
+    const ConvBox& c = p.cb;
+    if (u >= c.n_sub) {
+      first = last = 0;
+      return;
+    }
+    const int img = u / c.tiles_per_img, tb = u - img * c.tiles_per_img;
+    const int rows = min(c.TR, c.T_out - tb * c.TR) * c.F_out;
+    first = img * c.T_out * c.F_out + tb * c.TR * c.F_out;
+    last = first + rows;
+  } else {
+    first = u * 128;
+    last = min(first + 128, p.M);
+  }
+}
+
+// TMA coordinates of the A tile of sub-tile u at k-block kb (conv-box mode).
+__device__ __forceinline__ void convbox_coords(const GemmParams& p, int u, int kb, int& c0, int& f0, int& t0, int& img) {
+  const ConvBox& c = p.cb;
+  const int uu = u < c.n_sub ? u : c.n_sub - 1;  // past the end: any valid box, rows are masked
+  img = uu / c.tiles_per_img;
+  const int tb = uu - img * c.tiles_per_img;
+  const int tap = kb / c.CB;
+  const int cbk = kb - tap * c.CB;
+  const int dt = tap / c.kf, df = tap - dt * c.kf;
+  c0 = cbk * 64;
+  f0 = df - c.pf;
+  t0 = tb * c.TR * c.st + dt - c.pt;
+  if (u >= c.n_sub) t0 = 1 << 20;  // entirely outside: zero tile
+}
+
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1, int c2,
+                                            int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
 
 // Tile t -> (m block, n block).  With n_fast the tiles that share A rows run
 // on neighbouring CTAs at the same time, so A (the gathered activation of a
@@ -127,8 +186,8 @@ __device__ __forceinline__ void epilogue_prefetch_l2(const GemmParams& p, int t,
 //     segments, add positions / the residual with coalesced loads, and store
 //     with coalesced 16-byte (fp32) or 8-byte (bf16) stores.
 template <int EPI>
-__device__ __forceinline__ void epilogue_warp(const GemmParams& p, uint32_t tb, int row0, int n0, int BN, int half,
-                                              int lane, uint8_t* wbuf) {
+__device__ __forceinline__ void epilogue_warp(const GemmParams& p, uint32_t tb, int row0, int mlimit, int n0, int BN,
+                                              int half, int lane, uint8_t* wbuf) {
   constexpr bool F32 = (EPI & (EPI_OUT_F32 | EPI_RESID)) != 0;
   constexpr bool SWI = (EPI & EPI_SWIGLU) != 0;
 #pragma unroll 1
@@ -197,7 +256,7 @@ __device__ __forceinline__ void epilogue_warp(const GemmParams& p, uint32_t tb, 
         for (int i = 0; i < 8; ++i) {
           const int r = (lane >> 3) + 4 * i;
           const int row = row0 + r;
-          if (col_ok && row < p.M) {
+          if (col_ok && row < mlimit) {
             if (EPI & EPI_RESID)
               pre[i] = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.out) + (long long)row * p.ldo + nc);
             else
@@ -210,7 +269,7 @@ __device__ __forceinline__ void epilogue_warp(const GemmParams& p, uint32_t tb, 
         const int r = (lane >> 3) + 4 * i;
         const int row = row0 + r;
         float4 x = reinterpret_cast<const float4*>(wbuf + r * 128)[k ^ (r & 7)];
-        if (col_ok && row < p.M) {
+        if (col_ok && row < mlimit) {
           if (EPI & (EPI_RESID | EPI_PE)) {
             x.x += pre[i].x; x.y += pre[i].y; x.z += pre[i].z; x.w += pre[i].w;
           }
@@ -231,7 +290,7 @@ __device__ __forceinline__ void epilogue_warp(const GemmParams& p, uint32_t tb, 
         const uint2* src = reinterpret_cast<const uint2*>(wbuf + r * 64);
         const int chunk = (k4 >> 1) ^ ((r >> 1) & 3);
         const uint2 val = src[2 * chunk + (k4 & 1)];
-        if (row < p.M) *reinterpret_cast<uint2*>(reinterpret_cast<bf16*>(p.out) + (long long)row * p.ldo + ncol) = val;
+        if (row < mlimit) *reinterpret_cast<uint2*>(reinterpret_cast<bf16*>(p.out) + (long long)row * p.ldo + ncol) = val;
       }
     }
     __syncwarp();
@@ -305,7 +364,13 @@ __global__ void __launch_bounds__(GemmShape<BN, STAGES, GATHER>::THREADS, 1)
             mbar_arrive_expect_tx(&full[s], S::B_BYTES);
           } else {
             mbar_arrive_expect_tx(&full[s], S::A_BYTES + S::B_BYTES);
-            tma_load_2d(sA + s * S::A_BYTES, &tmA, &full[s], kb * S::BK, m0);
+            if (p.conv_box) {
+              int c0, f0, t0, img;
+              convbox_coords(p, mb, kb, c0, f0, t0, img);
+              tma_load_4d(sA + s * S::A_BYTES, &tmA, &full[s], c0, f0, t0, img);
+            } else {
+              tma_load_2d(sA + s * S::A_BYTES, &tmA, &full[s], kb * S::BK, m0);
+            }
           }
           tma_load_2d(sB + s * S::B_BYTES, &tmB, &full[s], kb * S::BK, n0);
           ++it;
@@ -388,10 +453,11 @@ __global__ void __launch_bounds__(GemmShape<BN, STAGES, GATHER>::THREADS, 1)
       tc_fence_after();
       int mb, nb;
       tile_coords(p, t, mb, nb);
-      const int m0 = mb * S::BM;
+      int r_first, r_last;
+      subtile_rows(p, mb, r_first, r_last);
       const int n0 = nb * BN;
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + a * S::ACC_COLS;
-      epilogue_warp<EPI>(p, tb, m0 + 32 * q, n0, BN, half, lane, sEpi + (warp - 2) * 4096);
+      epilogue_warp<EPI>(p, tb, r_first + 32 * q, r_last, n0, BN, half, lane, sEpi + (warp - 2) * 4096);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[a]);

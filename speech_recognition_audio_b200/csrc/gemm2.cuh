@@ -53,6 +53,14 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(x), "r"(y)
       : "memory");
 }
+__device__ __forceinline__ void tma_load_4d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster_addr, int c0,
+                                                 int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, "
+      "%6}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
                "r"(ncols)
@@ -96,7 +104,7 @@ struct Gemm2Shape {
   static constexpr int EPI_BUF_BYTES = EPI_WARPS * 4096;
   static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5) + 16;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BUF_BYTES + BAR_BYTES;
-  static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "UMMA N for M=256 (B halves of 16-row multiples)");
+  static_assert(BN % 16 == 0 && (BN / 2) % 8 == 0 && BN >= 64 && BN <= 256, "UMMA N for M=256; B halves of 8-row atoms");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
@@ -158,7 +166,8 @@ __global__ void __launch_bounds__(Gemm2Shape<BN, STAGES>::THREADS, 1)
       for (int t = pair; t < p.num_tiles && ok; t += n_pairs) {
         int mb, nb;
         tile_coords(p, t, mb, nb);
-        const int m0 = mb * S::BM + static_cast<int>(rank) * 128;
+        const int u = 2 * mb + static_cast<int>(rank);  // this CTA's 128-row sub-tile
+        const int m0 = u * 128;
         const int n0 = nb * BN + static_cast<int>(rank) * (BN / 2);
         for (int kb = 0; kb < p.k_blocks; ++kb) {
           const int s = it % STAGES;
@@ -169,7 +178,13 @@ __global__ void __launch_bounds__(Gemm2Shape<BN, STAGES>::THREADS, 1)
           }
           if (rank == 0) mbar_arrive_expect_tx(&full[s], S::TX_BYTES);
           const uint32_t fb = full_leader0 + 8u * s;
-          tma_load_2d_pair(sA + s * S::A_BYTES, &tmA, fb, kb * S::BK, m0);
+          if (p.conv_box) {
+            int c0, f0, t0, img;
+            convbox_coords(p, u, kb, c0, f0, t0, img);
+            tma_load_4d_pair(sA + s * S::A_BYTES, &tmA, fb, c0, f0, t0, img);
+          } else {
+            tma_load_2d_pair(sA + s * S::A_BYTES, &tmA, fb, kb * S::BK, m0);
+          }
           tma_load_2d_pair(sB + s * S::B_BYTES, &tmB, fb, kb * S::BK, n0);
           ++it;
         }
@@ -235,10 +250,11 @@ __global__ void __launch_bounds__(Gemm2Shape<BN, STAGES>::THREADS, 1)
       tc_fence_after();
       int mb, nb;
       tile_coords(p, t, mb, nb);
-      const int m0 = mb * S::BM + static_cast<int>(rank) * 128;
+      int r_first, r_last;
+      subtile_rows(p, 2 * mb + static_cast<int>(rank), r_first, r_last);
       const int n0 = nb * BN;
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + a * S::ACC_COLS;
-      epilogue_warp<EPI>(p, tb, m0 + 32 * q, n0, BN, half, lane, sEpi + (warp - 2) * 4096);
+      epilogue_warp<EPI>(p, tb, r_first + 32 * q, r_last, n0, BN, half, lane, sEpi + (warp - 2) * 4096);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8u * a);

@@ -44,19 +44,24 @@ cudaError_t launch_gelu(const float* x, float* y, long long n, cudaStream_t st);
 cudaError_t launch_wait_probe(unsigned long long limit_ns, int* status, cudaStream_t st);
 
 // GEMM engine launch (gemm.cu).
-constexpr int kGemmSlots = 5;
+constexpr int kGemmSlots = 6;
 struct GemmB {              // weight operand [N, K] bf16 + its TMA maps
   const bf16* ptr = nullptr;
   int N = 0, K = 0;
-  CUtensorMap map[kGemmSlots];  // box rows 256, 128, 240, 64, 160 (index by gemm_bn_slot)
+  CUtensorMap map[kGemmSlots];  // box rows 256, 128, 240, 64, 160, 120 (index by gemm_bn_slot)
 };
 int gemm_bn_slot(int bn);
 bool make_tmap_bf16(CUtensorMap* map, const void* ptr, unsigned long long rows, unsigned long long cols,
                     unsigned long long row_stride_elems, unsigned int box_rows);
 bool make_weight_maps(GemmB& w);
+// 4-D strided-box map over a conv activation [n_img, T_in, F_in, C] (see ConvBox).
+bool make_tmap_convbox(CUtensorMap* map, const void* ptr, int C, int F_in, int T_in, int n_img, int F_out, int sf,
+                       int TR, int st);
 // Picks the tile for an M x N problem on num_sms SMs: a positive width is a
 // one-SM 128 x bn tile, a negative one a CTA-pair 256 x |bn| tile.
 int gemm_pick_bn(int M, int N, int num_sms, bool gather);
+// Tile choice for a conv-box GEMM with n_sub 128-row sub-tiles.
+int gemm_pick_bn_conv(int n_sub, int N, int num_sms);
 // a_map: TMA map of A (box 128 x 64), or null with p.g set for the implicit-GEMM mode.
 cudaError_t launch_gemm(const CUtensorMap* a_map, const GemmB& w, GemmParams p, int epi, int bn, int num_sms,
                         cudaStream_t st);
