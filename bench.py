@@ -9,6 +9,7 @@ ranks) with TFLOP/s beside it.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --impl reference ...   # the CPU oracle on the host cores
+  python bench.py --kernel gemm_fc1 ...  # one op of the workload's shape (for ncu captures)
 
 Under torchrun (N > 1) every rank runs an independent replica of the
 workload (clips are independent: weak scaling, no collective on the data
@@ -147,6 +148,40 @@ class ClockSampler:
                 "samples_under_load": len(load), "reasons": sorted(reasons)}
 
 
+# ------------------------------------------------------- committed ncu summaries
+GEMM_SOURCES = ["speech_recognition_audio_b200/csrc/gemm.cuh", "speech_recognition_audio_b200/csrc/gemm2.cuh",
+                "speech_recognition_audio_b200/csrc/common.cuh"]
+
+
+def gemm_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for f in GEMM_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(name):
+    """DRAM bytes per launch recorded in profiles/<name>.md, or None when the
+    summary is missing or the GEMM sources changed since the capture."""
+    p = os.path.join(ROOT, "profiles", name + ".md")
+    if not os.path.exists(p):
+        return None
+    vals = {}
+    with open(p) as f:
+        for line in f:
+            if ":" in line and line.strip().startswith("- `"):
+                k, _, v = line.strip()[3:].partition("`:")
+                vals[k.strip()] = v.strip().strip("`")
+    if vals.get("source_sha256") != gemm_source_hash():
+        return None
+    try:
+        return int(float(vals["dram_bytes_per_launch"]))
+    except (KeyError, ValueError):
+        return None
+
+
 # ---------------------------------------------------------------- oracle arm
 def oracle_sample(w, g, W, pcm0):
     """One bounded sample of the workload on the CPU oracle: the log-mel of a
@@ -214,6 +249,43 @@ def run_reference(args, w, g, rank):
     return 0
 
 
+# ---------------------------------------------------------------- one op
+def run_kernel(args, w, g):
+    """Times one op of the workload's shape (warmup + steps launches)."""
+    import torch
+    import speech_recognition_audio_b200 as sra
+    T = sra.tokens(g, w.n_samples) * w.batch
+    d, f = g.d_model, g.d_ffn
+    gen = torch.Generator().manual_seed(7)
+    dev = torch.device("cuda", 0)
+    if args.kernel == "log_mel":
+        pcm = torch.from_numpy(synth.pcm_batch(w)).to(dev)
+        run = lambda: sra.log_mel(pcm, g.n_mels)
+        flops, unit = 4 * pcm.numel() + 4 * w.batch * g.n_mels * (w.n_samples // g.hop), "bytes"
+    else:
+        N, K, epi = {"gemm_fc1": (f, d, sra.EPI_BF16_GELU), "gemm_fc2": (d, f, sra.EPI_F32_RESID),
+                     "gemm_qkv": (3 * d, d, sra.EPI_BF16), "gemm_o": (d, d, sra.EPI_F32_RESID)}[args.kernel]
+        x = (torch.randn(T, K, generator=gen) * 0.5).to(torch.bfloat16).to(dev)
+        wt = (torch.randn(N, K, generator=gen) * 0.02).to(torch.bfloat16).to(dev)
+        b = torch.zeros(N, device=dev)
+        out = torch.zeros(T, N, device=dev) if epi == sra.EPI_F32_RESID else None
+        run = lambda: sra.linear(x, wt, b, epi, out=out)
+        flops, unit = 2 * T * N * K, "flop"
+    for _ in range(args.warmup):
+        run()
+    torch.cuda.synchronize()
+    s_, e_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s_.record()
+    for _ in range(args.steps):
+        run()
+    e_.record()
+    torch.cuda.synchronize()
+    ms = s_.elapsed_time(e_) / args.steps
+    print(json.dumps({"kernel": args.kernel, "workload": w.name, "ms_per_launch": ms, "work_per_launch": flops,
+                      "unit": unit, "rate": flops / (ms / 1000.0)}), flush=True)
+    return 0
+
+
 # ---------------------------------------------------------------- GPU arm
 def main():
     ap = argparse.ArgumentParser()
@@ -224,6 +296,8 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-steps", type=int, default=3)
+    ap.add_argument("--kernel", default=None, choices=["gemm_fc1", "gemm_fc2", "gemm_qkv", "gemm_o", "log_mel"],
+                    help="run one op of the workload's shape through the C ABI (for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -236,6 +310,8 @@ def main():
 
     if args.impl == "reference":
         return run_reference(args, w, g, rank)
+    if args.kernel:
+        return run_kernel(args, w, g)
 
     import torch
     import torch.distributed as dist
@@ -327,15 +403,22 @@ def main():
     gemm_keys = [k for k in per_step if k.startswith("gemm")]
     gemm_ms = sum(per_step[k] for k in gemm_keys)
     gemm_flops = sum(fl.get(k, 0) for k in gemm_keys)
-    gemm_launches = sum(launches_prof[k] for k in gemm_keys)
     peak_t = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
-    achieved = gemm_flops / (gemm_ms / 1000.0) / 1e12 if gemm_ms else None
-    roofline = {"bound": "tensor", "kernel": "gemm_bf16_tc_kernel (all tcgen05 GEMM launches of a step)",
-                "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
-                "frac": (achieved / peak_t) if achieved else None, "traffic": None,
-                "peak_kind": f"{peak_kind} sustained bf16",
-                "flops_per_launch": gemm_flops / max(gemm_launches, 1),
-                "avg_launch_ms": gemm_ms / max(gemm_launches, 1)}
+    # Dominant kernel: the largest GEMM stage of the step (one shape, one kernel).
+    top = max(gemm_keys, key=lambda k: per_step[k]) if gemm_keys else None
+    roofline = None
+    if top:
+        n_l = max(launches_prof[top], 1)
+        avg_ms = per_step[top] / n_l
+        per_launch = fl.get(top, 0) / n_l
+        achieved = per_launch / (avg_ms / 1000.0) / 1e12 if avg_ms else None
+        roofline = {"bound": "tensor", "kernel": f"tcgen05 GEMM, stage {top}", "achieved": achieved, "peak": peak_t,
+                    "unit": "TFLOP/s", "frac": (achieved / peak_t) if achieved else None,
+                    "traffic": profile_traffic(f"{top}_{w.name}"),
+                    "flops_per_launch": per_launch, "avg_launch_ms": avg_ms, "launches_per_step": n_l,
+                    "peak_kind": f"{peak_kind} sustained bf16 (MEASURED_PEAKS.json)"}
+    engine = {"achieved": gemm_flops / (gemm_ms / 1000.0) / 1e12 if gemm_ms else None, "unit": "TFLOP/s",
+              "ms_per_step": gemm_ms, "share_of_step": gemm_ms / sum(per_step.values()) if per_step else None}
     mel_ms = per_step.get("log_mel")
     mel_bytes = 4 * w.batch * w.n_samples + 4 * w.batch * g.n_mels * (w.n_samples // g.hop)
     mel_roof = None
@@ -397,6 +480,7 @@ def main():
         "e2e": e2e,
         "gpu_launches": int(launches_per_step * args.steps),
         "roofline": roofline,
+        "gemm_engine": engine,
         "mel_roofline": mel_roof,
         "kernels_ms_per_step": kernels,
         "clocks": clocks,

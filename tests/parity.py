@@ -27,5 +27,7 @@ def row_metrics(gpu, ref):
 def assert_encoder_parity(gpu, ref, what=""):
     cmin, rmax = row_metrics(gpu, ref)
     assert np.isfinite(np.asarray(gpu)).all(), f"{what}: non-finite output"
+    print(f"[parity] {what}: rows {np.shape(gpu)[0] if np.ndim(gpu) == 2 else int(np.prod(np.shape(gpu)[:-1]))}, "
+          f"min row cosine {cmin:.6f}, max row rel L2 {rmax:.3e}")
     assert cmin >= COS_MIN and rmax <= REL_L2_MAX, f"{what}: min row cosine {cmin:.6f}, max rel L2 {rmax:.3e}"
     return cmin, rmax

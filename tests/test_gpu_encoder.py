@@ -58,6 +58,7 @@ def test_tiny_full_with_taps():
     T = out.shape[1]
     assert T == 13 == oracle.token_count(g, w.n_samples)
     mel = enc.tap(sra.TAP_MEL, (1, g.n_mels, w.n_samples // 160)).cpu().numpy()[0]
+    print(f"[parity] tiny log-mel max abs {np.abs(mel - t['mel']).max():.3e}")
     assert np.abs(mel - t["mel"]).max() <= MEL_ABS_MAX
     assert_encoder_parity(enc.tap(sra.TAP_STEM, (T, g.d_model)).cpu().numpy(), t["stem"], "stem")
     assert_encoder_parity(enc.tap(sra.TAP_LAYER0, (T, g.d_model)).cpu().numpy(), t["layer0"], "layer0")
@@ -102,6 +103,7 @@ def _sampled(wname, picks):
     cu = oracle.window_partition(g, w.n_samples, 1)
     for b, j in picks:
         ref_mel = oracle.log_mel(pcm[b], g.n_mels)
+        print(f"[parity] {wname} clip {b} log-mel max abs {np.abs(mel[b] - ref_mel).max():.3e}")
         assert np.abs(mel[b] - ref_mel).max() <= MEL_ABS_MAX
         ref = oracle.encode_clip(pcm[b], W, g, windows=[j] if j is not None else None)
         rows = slice(int(cu[j]), int(cu[j + 1])) if j is not None else slice(0, T)

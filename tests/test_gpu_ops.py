@@ -126,8 +126,8 @@ def test_layer_norm(M, D):
 
 
 # ------------------------------------------------------------------ attention
-@pytest.mark.parametrize("lens,H", [([13], 4), ([104, 104, 104, 78], 20), ([1, 5, 64, 65, 100, 128, 129], 3),
-                                    ([1500, 1500], 12)])
+@pytest.mark.parametrize("lens,H", [([13], 4), ([104, 104, 104, 78], 20), ([1, 5, 64, 65, 100, 128], 3),
+                                    ([1, 5, 64, 65, 100, 128, 129], 3), ([17, 32, 33], 2), ([1500, 1500], 12)])
 def test_attention(lens, H):
     rng = np.random.default_rng(sum(lens) + H)
     T = sum(lens)
