@@ -31,6 +31,26 @@ size_t asr_op_log_mel_ws_size(int batch);
 asr_status asr_op_log_mel(const float* pcm, int64_t n_samples, int batch, int n_mels, float* mel,
                           void* ws, size_t ws_bytes, void* stream);
 
+/* Log-mel front-end that allocates no memory.  The pages have no
+ * counterpart: this entry point exists for callers that must not call
+ * cudaMalloc -- for example a plugin inside a host application that owns all
+ * device memory, or a real-time audio thread, where an allocation would
+ * stall on an implicit device synchronisation.  It computes exactly what
+ * asr_op_log_mel computes, but its scratch (the per-clip maxima and the
+ * FFT / filterbank tables, about 25 KB) is a fixed array inside the library:
+ * every GPU that loads the library holds it until the process exits.
+ *  pcm, n_samples, n_mels, mel: as for asr_op_log_mel.
+ *  batch: 1 .. 4096 clips; larger batches return ASR_E_UNSUPPORTED.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  Each call uploads the tables and clears the
+ * maxima on `stream` (a plain copy and memset, no allocation).  All calls
+ * share the one array and it keeps the last call's contents, so calls whose
+ * GPU work overlaps (different streams, not ordered) race and must not be
+ * issued. */
+asr_status asr_op_log_mel_noalloc(const float* pcm, int64_t n_samples, int batch, int n_mels, float* mel,
+                                  void* stream);
+
 /* Dense layer on the tcgen05 GEMM engine: acc = X W^T (fp32 accumulate in
  * tensor memory), then the epilogue.
  *  x     device bf16 [M, K] row-major;  w  device bf16 [N, K] row-major.

@@ -82,6 +82,7 @@ def _load():
         "asr_enc_last_launches": (I, [P]),
         "asr_op_log_mel_ws_size": (SZ, [I]),
         "asr_op_log_mel": (I, [P, I64, I, I, P, P, SZ, P]),
+        "asr_op_log_mel_noalloc": (I, [P, I64, I, I, P, P]),
         "asr_op_linear_ws_size": (SZ, []),
         "asr_op_linear": (I, [P, P, P, I64, I, I, I, I, P, P, SZ, P]),
         "asr_op_layer_norm": (I, [P, P, P, I64, I, F, P, I, P]),

@@ -1042,6 +1042,68 @@ asr_status asr_op_attention(const void* qkv, const int32_t* cu, int n_seg, int m
   return ASR_OK;
 }
 
+}  // extern "C"
+
+// ---- log-mel entry point that allocates nothing --------------------------
+// Its scratch (the per-clip maxima and the FFT / filterbank tables) lives in
+// file-scope device arrays that every GPU loading this library holds until
+// the process exits.  Host code must not pass these names to a kernel: on
+// the host they are stand-ins, not device addresses.  The device addresses
+// are looked up once per device (cudaGetSymbolAddress, with that device
+// current) and cached here.
+namespace {
+constexpr int kNoAllocMaxBatch = 4096;  // clips per call
+static __device__ __align__(256) unsigned int g_noalloc_clip_max[kNoAllocMaxBatch];
+static __device__ __align__(256) MelTables g_noalloc_tables;
+
+struct NoAllocScratch {
+  bool ready = false;
+  unsigned int* clip_max = nullptr;
+  MelTables* tables = nullptr;
+};
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+NoAllocScratch g_noalloc[kNoAllocMaxDevices];
+}  // namespace
+
+extern "C" {
+
+asr_status asr_op_log_mel_noalloc(const float* pcm, int64_t n_samples, int batch, int n_mels, float* mel,
+                                  void* stream) {
+  if (!pcm || !mel || batch <= 0 || n_mels <= 0 || n_mels > 128 || n_samples <= 200 || n_samples % 160)
+    return fail(nullptr, ASR_E_INVAL, "log_mel_noalloc: bad arguments");
+  if (batch > kNoAllocMaxBatch)
+    return fail(nullptr, ASR_E_UNSUPPORTED, "log_mel_noalloc: batch %d exceeds the static scratch limit of %d clips",
+                batch, kNoAllocMaxBatch);
+  int dev = 0;
+  ASR_CUDA(nullptr, cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(nullptr, ASR_E_UNSUPPORTED, "log_mel_noalloc: device %d", dev);
+  NoAllocScratch sc;
+  {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc[dev].ready) {
+      void* cm = nullptr;
+      void* tab = nullptr;
+      cudaError_t r = cudaGetSymbolAddress(&cm, g_noalloc_clip_max);
+      if (r == cudaSuccess) r = cudaGetSymbolAddress(&tab, g_noalloc_tables);
+      if (r != cudaSuccess)
+        return fail(nullptr, ASR_E_CUDA, "log_mel_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(r));
+      g_noalloc[dev].clip_max = static_cast<unsigned int*>(cm);
+      g_noalloc[dev].tables = static_cast<MelTables*>(tab);
+      g_noalloc[dev].ready = true;
+    }
+    sc = g_noalloc[dev];
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  MelTables h;
+  build_mel_tables(n_mels, &h);
+  ASR_CUDA(nullptr, cudaMemcpyAsync(sc.tables, &h, sizeof h, cudaMemcpyHostToDevice, st));
+  ASR_CUDA(nullptr, cudaMemsetAsync(sc.clip_max, 0, (size_t)batch * 4, st));  // the maxima start at zero
+  ASR_CUDA(nullptr, launch_log_mel(pcm, n_samples, batch, n_mels, sc.tables, mel, sc.clip_max, st));
+  ASR_CUDA(nullptr, launch_mel_normalize(mel, sc.clip_max, (long long)n_mels * (n_samples / 160), batch, mel, st));
+  return ASR_OK;
+}
+
 asr_status asr_op_gelu(const float* x, float* y, int64_t n, void* stream) {
   if (!x || !y || n <= 0) return fail(nullptr, ASR_E_INVAL, "gelu: bad arguments");
   ASR_CUDA(nullptr, launch_gelu(x, y, n, static_cast<cudaStream_t>(stream)));
