@@ -148,6 +148,29 @@ class ClockSampler:
                 "samples_under_load": len(load), "reasons": sorted(reasons)}
 
 
+# ------------------------------------------------------------ multi-GPU logic
+def rank_clip_seeds(w, rank):
+    """PCM seeds of the clips rank `rank` processes: every rank runs its own
+    replica of the workload (weak scaling), with disjoint seeds."""
+    return [w.pcm_seed_base + rank * w.batch + b for b in range(w.batch)]
+
+
+def reduce_max(value, device=None):
+    """Maximum of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(audio_s_per_rank, world, ms_max):
+    """Whole-job audio-seconds per second: all ranks' audio over the slowest rank's time."""
+    return audio_s_per_rank * world / (ms_max / 1000.0)
+
+
 # ------------------------------------------------------- committed ncu summaries
 GEMM_SOURCES = ["speech_recognition_audio_b200/csrc/gemm.cuh", "speech_recognition_audio_b200/csrc/gemm2.cuh",
                 "speech_recognition_audio_b200/csrc/common.cuh"]
@@ -331,8 +354,7 @@ def main():
     enc = sra.Encoder(g, {k: v.to(dev) for k, v in W.items()})
     del W
     # every rank processes its own replica of the workload (different seeds)
-    pcm_np = np.stack([synth.pcm_clip(w.n_samples, w.pcm_seed_base + rank * w.batch + b, w.speech_like)
-                       for b in range(w.batch)])
+    pcm_np = np.stack([synth.pcm_clip(w.n_samples, sd, w.speech_like) for sd in rank_clip_seeds(w, rank)])
     pcm = torch.from_numpy(pcm_np).to(dev)
     T = enc.tokens(w.n_samples)
     out = torch.empty((w.batch, T, enc.d_out), dtype=torch.float32, device=dev)
@@ -368,14 +390,10 @@ def main():
     enc.sync_status()
     launches_per_step = sra.lib.asr_enc_last_launches(enc.handle)
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    ms = statistics.mean(step_ms)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = reduce_max(statistics.mean(step_ms), dev)
 
     audio_per_step = w.batch * w.seconds * world
-    value = audio_per_step / (ms / 1000.0)
+    value = job_throughput(w.batch * w.seconds, world, ms)
     fl = flop_breakdown(g, w.n_samples, w.batch)
     flops = sum(fl.values())
     tflops = flops * world / (ms / 1000.0) / 1e12
@@ -445,11 +463,7 @@ def main():
         enc.forward_host(pcm_host, out_host=out_host, workspace=ws)
         e_e[i].record(stream)
     torch.cuda.synchronize()
-    e2e_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(e_s, e_e))
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = reduce_max(statistics.mean(s.elapsed_time(e) for s, e in zip(e_s, e_e)), dev)
     e2e = {"value": audio_per_step / (e2e_ms / 1000.0), "unit": "audio-s/s",
            "h2d_bytes_per_step": int(pcm_host.numel() * 4), "d2h_bytes_per_step": int(out_host.numel() * 4),
            "ms_per_step": e2e_ms}
