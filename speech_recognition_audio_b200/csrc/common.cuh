@@ -25,6 +25,16 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// ------------------------------------------------- programmatic dependent launch
+// Kernels are launched with programmatic stream serialisation: a kernel may
+// start (prologue: barrier init, tensor-memory allocation, descriptor
+// prefetch) while its predecessor is still finishing.  pdl_wait() blocks
+// until the predecessor grid has completed and its memory is visible; every
+// kernel calls it before its first global-memory access.  pdl_trigger() lets
+// the successor begin launching; it still waits for this grid to complete.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");

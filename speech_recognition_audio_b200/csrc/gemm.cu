@@ -39,8 +39,7 @@ cudaError_t run(const CUtensorMap* a, const CUtensorMap& b, const GemmParams& p,
   auto k = gemm_bf16_tc_kernel<BN, S::STAGES, G, EPI>;
   cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_BYTES);
   if (err != cudaSuccess) return err;
-  k<<<grid, S::THREADS, S::SMEM_BYTES, st>>>(a ? *a : b, b, p);
-  return cudaGetLastError();
+  return launch_pdl(k, dim3(grid), dim3(S::THREADS), S::SMEM_BYTES, st, a ? *a : b, b, p);
 }
 
 template <int BN>
@@ -88,13 +87,15 @@ cudaError_t run2(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p
   cfg.blockDim = dim3(S::THREADS, 1, 1);
   cfg.dynamicSmemBytes = S::SMEM_BYTES;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, k, a, b, p);
 }
 

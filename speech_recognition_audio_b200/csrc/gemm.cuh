@@ -342,6 +342,8 @@ __global__ void __launch_bounds__(GemmShape<BN, STAGES, GATHER>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer

@@ -157,6 +157,8 @@ __global__ void __launch_bounds__(Gemm2Shape<BN, STAGES>::THREADS, 1)
   cluster_sync();  // barriers of both CTAs initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {

@@ -22,6 +22,8 @@ template <int V, bool OUT_F32>
 __global__ void __launch_bounds__(256) layer_norm_kernel(const float* __restrict__ x, const float* __restrict__ g,
                                                          const float* __restrict__ b, long long M, float eps,
                                                          void* __restrict__ y) {
+  pdl_wait();
+  pdl_trigger();
   const long long row = blockIdx.x * 8LL + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= M) return;
@@ -74,7 +76,11 @@ static cudaError_t ln_dispatch(int V, const float* x, const float* g, const floa
   const unsigned blocks = static_cast<unsigned>((M + 7) / 8);
   switch (V) {
 #define ASR_LN_CASE(n) \
-  case n: layer_norm_kernel<n, F32><<<blocks, 256, 0, st>>>(x, g, b, M, eps, y); break;
+  case n: {                                                                                  \
+    cudaError_t e_ = launch_pdl(layer_norm_kernel<n, F32>, dim3(blocks), dim3(256), 0, st, x, g, b, M, eps, y); \
+    if (e_ != cudaSuccess) return e_;                                                        \
+    break;                                                                                   \
+  }
     ASR_LN_CASE(1) ASR_LN_CASE(2) ASR_LN_CASE(3) ASR_LN_CASE(4) ASR_LN_CASE(5) ASR_LN_CASE(6) ASR_LN_CASE(7)
     ASR_LN_CASE(8) ASR_LN_CASE(9) ASR_LN_CASE(10) ASR_LN_CASE(11) ASR_LN_CASE(12) ASR_LN_CASE(13)
     ASR_LN_CASE(14) ASR_LN_CASE(15) ASR_LN_CASE(16)
@@ -132,6 +138,8 @@ __global__ void __launch_bounds__(128) attention_kernel(const bf16* __restrict__
   __shared__ __align__(16) bf16 Qs[BQ * LDS];
   __shared__ __align__(16) bf16 Ks[2][BKV * LDS];
   __shared__ __align__(16) bf16 Vs[2][BKV * LDS];
+  pdl_wait();
+  pdl_trigger();
   const int seg = blockIdx.y, h = blockIdx.z;
   const int s0 = cu[seg], L = cu[seg + 1] - s0;
   const int q0 = blockIdx.x * BQ;
@@ -274,6 +282,8 @@ __global__ void __launch_bounds__(256) attention_window_kernel(const bf16* __res
   bf16* Qs = reinterpret_cast<bf16*>(smem_att);
   bf16* Ks = Qs + 128 * LDS;
   bf16* Vs = Ks + 128 * LDS;
+  pdl_wait();
+  pdl_trigger();
   const int seg = blockIdx.x, h = blockIdx.y;
   const int s0 = cu[seg], L = cu[seg + 1] - s0;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -375,8 +385,7 @@ static cudaError_t launch_window(const bf16* qkv, const int* cu, int n_seg, int 
   auto k = attention_window_kernel<NK>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  k<<<dim3(n_seg, H), 256, smem, st>>>(qkv, cu, H, out);
-  return cudaGetLastError();
+  return launch_pdl(k, dim3(n_seg, H), dim3(256), smem, st, qkv, cu, H, out);
 }
 
 cudaError_t launch_attention(const bf16* qkv, const int* cu, int n_seg, int max_seg, int H, bf16* out,
@@ -395,12 +404,13 @@ cudaError_t launch_attention(const bf16* qkv, const int* cu, int n_seg, int max_
     }
   }
   dim3 grid((max_seg + BQ - 1) / BQ, n_seg, H);
-  attention_kernel<<<grid, 128, 0, st>>>(qkv, cu, H, out);
-  return cudaGetLastError();
+  return launch_pdl(attention_kernel, grid, dim3(128), 0, st, qkv, cu, H, out);
 }
 
 // ------------------------------------------------------------ helpers
 __global__ void fill_windows_kernel(int* cu, int batch, int tpc, int window, int nw) {
+  pdl_wait();
+  pdl_trigger();
   const int total = batch * nw;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i <= total; i += gridDim.x * blockDim.x) {
     if (i == total) {
@@ -415,30 +425,32 @@ __global__ void fill_windows_kernel(int* cu, int batch, int tpc, int window, int
 cudaError_t launch_fill_windows(int* cu, int batch, int tokens_per_clip, int window, int n_win_per_clip,
                                 cudaStream_t st) {
   const int total = batch * n_win_per_clip + 1;
-  fill_windows_kernel<<<(total + 255) / 256, 256, 0, st>>>(cu, batch, tokens_per_clip, window, n_win_per_clip);
-  return cudaGetLastError();
+  return launch_pdl(fill_windows_kernel, dim3((total + 255) / 256), dim3(256), 0, st, cu, batch, tokens_per_clip, window,
+                    n_win_per_clip);
 }
 
 __global__ void bf16_to_f32_kernel(const bf16* __restrict__ in, float* __restrict__ out, long long n) {
+  pdl_wait();
+  pdl_trigger();
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
     out[i] = __bfloat162float(in[i]);
 }
 
 cudaError_t launch_bf16_to_f32(const bf16* in, float* out, long long n, cudaStream_t st) {
   const int blocks = static_cast<int>(std::min<long long>((n + 255) / 256, 148LL * 32));
-  bf16_to_f32_kernel<<<blocks, 256, 0, st>>>(in, out, n);
-  return cudaGetLastError();
+  return launch_pdl(bf16_to_f32_kernel, dim3(blocks), dim3(256), 0, st, in, out, n);
 }
 
 __global__ void gelu_kernel(const float* __restrict__ x, float* __restrict__ y, long long n) {
+  pdl_wait();
+  pdl_trigger();
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
     y[i] = gelu_erf(x[i]);
 }
 
 cudaError_t launch_gelu(const float* x, float* y, long long n, cudaStream_t st) {
   const int blocks = static_cast<int>(std::min<long long>((n + 255) / 256, 148LL * 32));
-  gelu_kernel<<<blocks, 256, 0, st>>>(x, y, n);
-  return cudaGetLastError();
+  return launch_pdl(gelu_kernel, dim3(blocks), dim3(256), 0, st, x, y, n);
 }
 
 // A barrier that nothing ever completes, waited on with the same bounded wait

@@ -86,6 +86,8 @@ __global__ void __launch_bounds__(THREADS) log_mel_kernel(const float* __restric
   __shared__ float hann[NFFT];
   __shared__ float red[THREADS / 32];
 
+  pdl_wait();
+  pdl_trigger();
   const int groups_per_clip = (n_frames + FB - 1) / FB;
   const int b = blockIdx.x / groups_per_clip;
   const int f0 = (blockIdx.x - b * groups_per_clip) * FB;
@@ -192,6 +194,8 @@ __global__ void __launch_bounds__(THREADS) log_mel_kernel(const float* __restric
 // Normalised log-mel in [B, n_mels, F] fp32: (max(L, m - 8) + 4) / 4.
 __global__ void mel_normalize_kernel(const float* __restrict__ raw, const unsigned int* __restrict__ clip_max,
                                      long long per_clip, int batch, float* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
   const long long total = per_clip * batch;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
        i += (long long)gridDim.x * blockDim.x) {
@@ -206,6 +210,8 @@ __global__ void mel_normalize_kernel(const float* __restrict__ raw, const unsign
 __global__ void mel_normalize_transpose_kernel(const float* __restrict__ raw, const unsigned int* __restrict__ clip_max,
                                                int n_mels, int n_frames, bf16* __restrict__ out) {
   __shared__ float tile[32][33];
+  pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.z;
   const int f0 = blockIdx.x * 32, m0 = blockIdx.y * 32;
   const float mx = ordered_to_float(clip_max[b]) - 8.0f;
@@ -226,23 +232,21 @@ cudaError_t launch_log_mel(const float* pcm, long long n_samples, int batch, int
                            float* mel_raw, unsigned int* clip_max, cudaStream_t st) {
   const int n_frames = static_cast<int>(n_samples / HOP);
   const int groups = (n_frames + FB - 1) / FB;
-  log_mel_kernel<<<groups * batch, THREADS, 0, st>>>(pcm, n_samples, n_frames, n_mels, tab, mel_raw, clip_max);
-  return cudaGetLastError();
+  return launch_pdl(log_mel_kernel, dim3(groups * batch), dim3(THREADS), 0, st, pcm, n_samples, n_frames, n_mels, tab,
+                    mel_raw, clip_max);
 }
 
 cudaError_t launch_mel_normalize(const float* raw, const unsigned int* clip_max, long long per_clip, int batch,
                                  float* out, cudaStream_t st) {
   const long long total = per_clip * batch;
   const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 148LL * 16));
-  mel_normalize_kernel<<<blocks, 256, 0, st>>>(raw, clip_max, per_clip, batch, out);
-  return cudaGetLastError();
+  return launch_pdl(mel_normalize_kernel, dim3(blocks), dim3(256), 0, st, raw, clip_max, per_clip, batch, out);
 }
 
 cudaError_t launch_mel_normalize_transpose(const float* raw, const unsigned int* clip_max, int batch, int n_mels,
                                            int n_frames, bf16* out, cudaStream_t st) {
   dim3 grid((n_frames + 31) / 32, (n_mels + 31) / 32, batch);
-  mel_normalize_transpose_kernel<<<grid, dim3(32, 8), 0, st>>>(raw, clip_max, n_mels, n_frames, out);
-  return cudaGetLastError();
+  return launch_pdl(mel_normalize_transpose_kernel, grid, dim3(32, 8), 0, st, raw, clip_max, n_mels, n_frames, out);
 }
 
 }  // namespace asr

@@ -26,6 +26,8 @@ __global__ void __launch_bounds__(THREADS)
                          int n_frames, int chunk_frames, int chunks_per_clip, const float* __restrict__ w,
                          const float* __restrict__ bias, int C, bf16* __restrict__ out) {
   __shared__ float patch[(2 * TB + 1) * (MAXM + 2)];
+  pdl_wait();
+  pdl_trigger();
   const int chunk = blockIdx.x;
   const int b = chunk / chunks_per_clip;
   const int q = chunk - b * chunks_per_clip;
@@ -94,9 +96,8 @@ cudaError_t launch_conv1_chunked(const float* mel_raw, const unsigned int* clip_
   dim3 grid(batch * chunks_per_clip, (T1 + TB - 1) / TB);
   const int groups = C / 8;
   const int threads = groups * std::max(1, THREADS / groups);
-  conv1_chunked_kernel<<<grid, threads, 0, st>>>(mel_raw, clip_max, n_mels, n_frames, chunk_frames, chunks_per_clip,
-                                                 w, b, C, out);
-  return cudaGetLastError();
+  return launch_pdl(conv1_chunked_kernel, grid, dim3(threads), 0, st, mel_raw, clip_max, n_mels, n_frames, chunk_frames,
+                    chunks_per_clip, w, b, C, out);
 }
 
 }  // namespace asr
