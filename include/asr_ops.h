@@ -84,9 +84,13 @@ asr_status asr_op_layer_norm(const float* x, const float* g, const float* b, int
  * and head h, softmax(Q K^T / 8) V, with Q, K, V read from
  * qkv device bf16 [T, 3*H*64] (columns: q heads, k heads, v heads) and the
  * result written to out device bf16 [T, H*64].  cu: device int32 [n_seg+1].
- * max_seg: the longest segment (sizes the launch grid).  head_dim 64. */
+ * max_seg: the longest segment.  head_dim 64.  Segments of at most 128
+ * tokens run on the tcgen05 kernel (one block per segment and head), longer
+ * ones on a flash-style kernel.  ws: device scratch of
+ * >= asr_op_attention_ws_size() bytes (device status word). */
+size_t asr_op_attention_ws_size(void);
 asr_status asr_op_attention(const void* qkv, const int32_t* cu, int n_seg, int max_seg, int64_t T,
-                            int H, void* out, void* stream);
+                            int H, void* out, void* ws, size_t ws_bytes, void* stream);
 
 /* The GELU every kernel applies (bias-free): y[i] = x[i] Phi(x[i]), with
  * Phi from the Abramowitz & Stegun 7.1.26 approximation of erf (absolute

@@ -86,7 +86,8 @@ def _load():
         "asr_op_linear_ws_size": (SZ, []),
         "asr_op_linear": (I, [P, P, P, I64, I, I, I, I, P, P, SZ, P]),
         "asr_op_layer_norm": (I, [P, P, P, I64, I, F, P, I, P]),
-        "asr_op_attention": (I, [P, P, I, I, I64, I, P, P]),
+        "asr_op_attention_ws_size": (SZ, []),
+        "asr_op_attention": (I, [P, P, I, I, I64, I, P, P, SZ, P]),
         "asr_op_gelu": (I, [P, P, I64, P]),
         "asr_op_wait_probe": (I, [I64, P, P]),
     }
@@ -332,8 +333,11 @@ def attention(qkv, cu, n_heads: int, stream=None):
     cu_host = cu.cpu().tolist()
     max_seg = max(b - a for a, b in zip(cu_host[:-1], cu_host[1:]))
     out = torch.empty((T, n_heads * 64), dtype=torch.bfloat16, device=qkv.device)
-    _check(lib.asr_op_attention(_ptr(qkv), _ptr(cu), len(cu_host) - 1, max_seg, T, n_heads, _ptr(out),
-                                _stream(stream)))
+    ws = torch.zeros(int(lib.asr_op_attention_ws_size()), dtype=torch.uint8, device=qkv.device)
+    _check(lib.asr_op_attention(_ptr(qkv), _ptr(cu), len(cu_host) - 1, max_seg, T, n_heads, _ptr(out), _ptr(ws),
+                                ws.numel(), _stream(stream)))
+    if int(ws[:4].view(torch.int32).item()) != 0:
+        raise AsrError(6, "attention: a bounded device wait gave up")
     return out
 
 

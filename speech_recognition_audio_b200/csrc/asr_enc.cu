@@ -45,6 +45,7 @@ struct ActMaps {
   unsigned taps = 0;
   CUtensorMap h, att, ff, c3, p1, p2, gu;
   CUtensorMap cin2, cin3;  // conv-box A maps of the two stem GEMMs
+  CUtensorMap qkv;         // 128-row boxes of the QKV buffer (tcgen05 attention)
 };
 
 struct Plan {
@@ -695,7 +696,8 @@ asr_status ensure_maps(asr_enc* e, const Plan& p, char* ws) {
   if (m.ws == ws && m.n == p.n && m.batch == p.B && m.taps == e->taps) return ASR_OK;
   const asr_geometry* g = &e->g;
   const int d = g->d_model;
-  bool ok = make_tmap_bf16(&m.h, ws + p.off_h, p.T, d, d, 128) &&
+  bool ok = make_tmap_qkv(&m.qkv, ws + p.off_qkv, p.T, g->n_heads) &&
+            make_tmap_bf16(&m.h, ws + p.off_h, p.T, d, d, 128) &&
             make_tmap_bf16(&m.att, ws + p.off_att, p.T, d, d, 128) &&
             make_tmap_bf16(&m.ff, ws + p.off_ff, p.T, g->d_ffn, g->d_ffn, 128);
   if (ok && g->stem == ASR_STEM_CONV2D_CHUNKED) {
@@ -787,7 +789,11 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
     const LayerW& lw = e->layers[l];
     ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, lw.ln1g, lw.ln1b, p.T, d, g->ln_eps, h, false, st)));
     ASR_K(PC_GEMM_QKV, ASR_TRY(gemm(e, &e->maps.h, nullptr, lw.qkv, p.T, qkv, 3 * d, lw.bqkv, nullptr, 1, 0, st)));
-    ASR_K(PC_ATTN, ASR_LAUNCH(e, launch_attention(qkv, cu, p.nwin, p.max_win, g->n_heads, att, st)));
+    if (p.max_win <= 128)
+      ASR_K(PC_ATTN, ASR_LAUNCH(e, launch_attention_tc(e->maps.qkv, qkv, cu, p.nwin, g->n_heads, att, e->status,
+                                                       kWaitLimitNs, st)));
+    else
+      ASR_K(PC_ATTN, ASR_LAUNCH(e, launch_attention(qkv, cu, p.nwin, p.max_win, g->n_heads, att, st)));
     ASR_K(PC_GEMM_O, ASR_TRY(gemm(e, &e->maps.att, nullptr, lw.o, p.T, x, d, lw.bo, nullptr, 1, EPI_RESID, st)));
     ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, lw.ln2g, lw.ln2b, p.T, d, g->ln_eps, h, false, st)));
     ASR_K(PC_GEMM_FC1, ASR_TRY(gemm(e, &e->maps.h, nullptr, lw.fc1, p.T, ff, g->d_ffn, lw.b1, nullptr, 1, EPI_GELU, st)));
@@ -1033,12 +1039,23 @@ asr_status asr_op_layer_norm(const float* x, const float* g, const float* b, int
   return ASR_OK;
 }
 
+size_t asr_op_attention_ws_size(void) { return 256; }
+
 asr_status asr_op_attention(const void* qkv, const int32_t* cu, int n_seg, int max_seg, int64_t T, int H, void* out,
-                            void* stream) {
+                            void* ws, size_t ws_bytes, void* stream) {
   if (!qkv || !cu || !out || n_seg <= 0 || max_seg <= 0 || H <= 0 || T <= 0)
     return fail(nullptr, ASR_E_INVAL, "attention: bad arguments");
-  ASR_CUDA(nullptr, launch_attention(static_cast<const bf16*>(qkv), cu, n_seg, max_seg, H, static_cast<bf16*>(out),
-                                     static_cast<cudaStream_t>(stream)));
+  if (!ws || ws_bytes < 256) return fail(nullptr, ASR_E_WORKSPACE, "attention: workspace too small");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (max_seg <= 128) {
+    CUtensorMap m;
+    if (!make_tmap_qkv(&m, qkv, T, H)) return fail(nullptr, ASR_E_INVAL, "attention: TMA descriptor encoding failed");
+    ASR_CUDA(nullptr, cudaMemsetAsync(ws, 0, 4, st));
+    ASR_CUDA(nullptr, launch_attention_tc(m, static_cast<const bf16*>(qkv), cu, n_seg, H, static_cast<bf16*>(out),
+                                          static_cast<int*>(ws), kWaitLimitNs, st));
+  } else {
+    ASR_CUDA(nullptr, launch_attention(static_cast<const bf16*>(qkv), cu, n_seg, max_seg, H, static_cast<bf16*>(out), st));
+  }
   return ASR_OK;
 }
 

@@ -53,6 +53,10 @@ cudaError_t launch_layer_norm(const float* x, const float* g, const float* b, lo
 
 cudaError_t launch_attention(const bf16* qkv, const int* cu, int n_seg, int max_seg, int H, bf16* out,
                              cudaStream_t st);
+// tcgen05 attention for segments of at most 128 tokens (attn_tc.cu).
+bool make_tmap_qkv(CUtensorMap* map, const void* qkv, long long T, int H);
+cudaError_t launch_attention_tc(const CUtensorMap& tm_qkv, const bf16* qkv, const int* cu, int n_seg, int H, bf16* out,
+                                int* status, unsigned long long limit_ns, cudaStream_t st);
 
 cudaError_t launch_fill_windows(int* cu, int batch, int tokens_per_clip, int window, int n_win_per_clip,
                                 cudaStream_t st);
