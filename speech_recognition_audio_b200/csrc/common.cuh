@@ -203,21 +203,95 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
 }
 
 // ---------------------------------------------------------------- math
-// GELU(x) = x Phi(x) with Phi(x) = (1 + erf(x / sqrt 2)) / 2, erf from the
-// Abramowitz & Stegun rational-exponential approximation 7.1.26:
-//   erf(z) = 1 - t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-z^2),
-//   t = 1 / (1 + p z), z >= 0, |error| <= 1.5e-7,
-// evaluated with the hardware reciprocal and exp2.  For x < 0 the symmetry
-// erf(-z) = -erf(z) gives Phi(x) = q with q = (1 - erf(|x| / sqrt 2)) / 2.
+// Packed fp32 pair arithmetic (the f32x2 instructions of sm_100): one
+// instruction issues two IEEE fp32 operations with the usual rounding.
+__device__ __forceinline__ unsigned long long f2_bits(float2 v) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(v.x), "f"(v.y));
+  return r;
+}
+__device__ __forceinline__ float2 bits_f2(unsigned long long r) {
+  float2 v;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
+  return v;
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
+  return bits_f2(d);
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return bits_f2(d);
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return bits_f2(d);
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+// GELU(x) = x Phi(x) with Phi(x) = (1 + erf(x / sqrt 2)) / 2 and erf from
+// Abramowitz & Stegun 7.1.28:
+//   erf(z) = 1 - (1 + a1 z + a2 z^2 + ... + a6 z^6)^-16,  z >= 0,
+//   |error| <= 3e-7  (one reciprocal, no exponential).
+// With u = |x| and h = (1 - erf(u / sqrt 2)) / 2, x Phi(x) equals x - u h
+// for x >= 0 and -u h for x < 0, i.e. (x + u) / 2 - u h in both cases (no
+// cancellation: x + u is 0 or 2u).  The 1/sqrt2 scaling and the factor 1/2
+// go into the coefficients: h = Q(u)^-16 with
+//   Q(u) = c (1 + sum_k a_k 2^(-k/2) u^k),  c = 2^(1/16),
+// evaluated by Horner in v = -u (odd coefficients negated) so that u h is
+// the product -v h.  fp32 rounding of Q is amplified 16-fold by the power:
+// the result is within 1.5e-7 |x| (approximation) + 6e-6 |x| (evaluation)
+// of the exact GELU.
+namespace gelu_as28 {
+constexpr double kC = 1.0442737824274138;  // 2^(1/16)
+constexpr float b0 = static_cast<float>(kC);
+constexpr float b1 = static_cast<float>(-kC * 0.0705230784 / 1.4142135623730951);
+constexpr float b2 = static_cast<float>(kC * 0.0422820123 / 2.0);
+constexpr float b3 = static_cast<float>(-kC * 0.0092705272 / 2.8284271247461903);
+constexpr float b4 = static_cast<float>(kC * 0.0001520143 / 4.0);
+constexpr float b5 = static_cast<float>(-kC * 0.0002765672 / 5.6568542494923806);
+constexpr float b6 = static_cast<float>(kC * 0.0000430638 / 8.0);
+}  // namespace gelu_as28
+
+__device__ __forceinline__ float2 gelu_erf2(float2 x) {
+  using namespace gelu_as28;
+  const float2 v = make_float2(-fabsf(x.x), -fabsf(x.y));
+  float2 q = fma2(v, make_float2(b6, b6), make_float2(b5, b5));
+  q = fma2(q, v, make_float2(b4, b4));
+  q = fma2(q, v, make_float2(b3, b3));
+  q = fma2(q, v, make_float2(b2, b2));
+  q = fma2(q, v, make_float2(b1, b1));
+  q = fma2(q, v, make_float2(b0, b0));
+  q = mul2(q, q);
+  q = mul2(q, q);
+  q = mul2(q, q);
+  q = mul2(q, q);
+  const float2 h = make_float2(rcp_approx(q.x), rcp_approx(q.y));
+  const float2 xu = add2(x, make_float2(-v.x, -v.y));  // x + u
+  return fma2(xu, make_float2(0.5f, 0.5f), mul2(v, h));
+}
+
 __device__ __forceinline__ float gelu_erf(float x) {
-  const float z = fabsf(x) * 0.70710678118654752f;
-  const float t = __fdividef(1.0f, fmaf(0.3275911f, z, 1.0f));
-  float poly = fmaf(t, 1.061405429f, -1.453152027f);
-  poly = fmaf(t, poly, 1.421413741f);
-  poly = fmaf(t, poly, -0.284496736f);
-  poly = fmaf(t, poly, 0.254829592f);
-  const float q = 0.5f * t * poly * __expf(-z * z);
-  return x * (x >= 0.f ? 1.0f - q : q);
+  using namespace gelu_as28;
+  const float v = -fabsf(x);
+  float q = fmaf(v, b6, b5);
+  q = fmaf(q, v, b4);
+  q = fmaf(q, v, b3);
+  q = fmaf(q, v, b2);
+  q = fmaf(q, v, b1);
+  q = fmaf(q, v, b0);
+  q *= q;
+  q *= q;
+  q *= q;
+  q *= q;
+  return fmaf(x - v, 0.5f, v * rcp_approx(q));
 }
 __device__ __forceinline__ float silu(float x) { return x / (1.0f + __expf(-x)); }
 

@@ -226,7 +226,11 @@ __device__ __forceinline__ void epilogue_warp(const GemmParams& p, uint32_t tb, 
     } else {
       if (EPI & EPI_GELU) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = gelu_erf(v[i]);
+        for (int i = 0; i < 32; i += 2) {
+          const float2 g = gelu_erf2(make_float2(v[i], v[i + 1]));
+          v[i] = g.x;
+          v[i + 1] = g.y;
+        }
       }
       if (F32) {
         float4* row = reinterpret_cast<float4*>(wbuf + lane * 128);

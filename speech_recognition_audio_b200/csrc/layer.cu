@@ -444,8 +444,15 @@ cudaError_t launch_bf16_to_f32(const bf16* in, float* out, long long n, cudaStre
 __global__ void gelu_kernel(const float* __restrict__ x, float* __restrict__ y, long long n) {
   pdl_wait();
   pdl_trigger();
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
-    y[i] = gelu_erf(x[i]);
+  // pairs through the packed form used by the GEMM epilogues and the stem; an
+  // odd last element through the scalar form
+  const long long np = n / 2;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < np; i += (long long)gridDim.x * blockDim.x) {
+    const float2 g = gelu_erf2(make_float2(x[2 * i], x[2 * i + 1]));
+    y[2 * i] = g.x;
+    y[2 * i + 1] = g.y;
+  }
+  if ((n & 1) && blockIdx.x == 0 && threadIdx.x == 0) y[n - 1] = gelu_erf(x[n - 1]);
 }
 
 cudaError_t launch_gelu(const float* x, float* y, long long n, cudaStream_t st) {

@@ -146,13 +146,18 @@ def test_attention(lens, H):
 
 # ------------------------------------------------------------------ GELU
 def test_gelu_within_published_bound():
-    # The device GELU uses Abramowitz & Stegun 7.1.26 for erf (|error| <= 1.5e-7):
-    # |GELU - exact| <= |x| * 0.5 * 1.5e-7 plus fp32 rounding of the steps.
+    # The device GELU takes erf from Abramowitz & Stegun 7.1.28 (|error| <= 3e-7),
+    # i.e. |GELU - exact| <= |x| * 0.5 * 3e-7, plus the fp32 evaluation of the
+    # 16th power: <= 111 roundings of 2^-24 relative on h <= 1/2, and the final
+    # rounding of the result.  An odd length sends the last element through the
+    # scalar form, the rest through the packed pair form.
     x = np.concatenate([np.linspace(-12, 12, 2_000_001), [0.0, -0.0, 1e-30, -1e-30, 40.0, -40.0]]).astype(np.float32)
+    assert len(x) % 2 == 1
     got = sra.gelu(torch.from_numpy(x).cuda()).cpu().numpy().astype(np.float64)
     ref = oracle.gelu(x.astype(np.float64))
     err = np.abs(got - ref)
-    assert (err <= 1.2e-7 * np.abs(x) + 4e-7 * np.maximum(np.abs(ref), 1e-30)).all(), err.max()
+    bound = (1.5e-7 + 0.5 * 111 * 2.0**-24 + 2.0**-23) * np.abs(x) + 2.0**-23 * np.abs(ref)
+    assert (err <= bound).all(), (err.max(), (err / np.maximum(bound, 1e-300)).max())
     assert got[-2] == 40.0 and abs(got[-1]) == 0.0
     assert np.all(np.isfinite(got))
 
