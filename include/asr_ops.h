@@ -62,8 +62,13 @@ asr_status asr_op_log_mel_noalloc(const float* pcm, int64_t n_samples, int batch
  *        ASR_EPI_SWIGLU     y bf16 [M, N/2]: W rows interleaved in blocks of
  *                           16 (gate rows 16j..16j+15, then the matching up
  *                           rows), y[:, 16j+i] = SiLU(gate) * up
- * Limits: K % 8 == 0, N % 16 == 0, M >= 1.  ws: device scratch of
- * >= asr_op_linear_ws_size() bytes (device status word).
+ * Limits: K % 8 == 0, N % 16 == 0, M >= 1.  ws: device scratch, caller-owned,
+ * at least 256 bytes (device status word).  With asr_op_linear_ws_size()
+ * bytes (status word and one flag per SM and epilogue warp of the current
+ * device) the residual epilogue on CTA-pair tiles runs stream-K: the
+ * (tile, k-block) work is split evenly over the SM pairs, and of a tile cut
+ * in two the trailing part's sum reaches y before the leading part's, so
+ * results are deterministic.  Smaller scratch runs whole tiles.
  * tile_n: output tile of one SM, 128 x tile_n (256, 160, 128 or 64; 160 needs
  * N % 160 == 0), or of a CTA pair (two SMs, tcgen05 cta_group::2),
  * 256 x -tile_n (-256 or -128); 0 = chosen from M, N and the SM count as in
@@ -93,8 +98,8 @@ asr_status asr_op_attention(const void* qkv, const int32_t* cu, int n_seg, int m
                             int H, void* out, void* ws, size_t ws_bytes, void* stream);
 
 /* The GELU every kernel applies (bias-free): y[i] = x[i] Phi(x[i]), with
- * Phi from the Abramowitz & Stegun 7.1.26 approximation of erf (absolute
- * error <= 1.5e-7).  x, y: device float32 [n]. */
+ * Phi from the Abramowitz & Stegun 7.1.28 approximation of erf (absolute
+ * error <= 3e-7; fp32 evaluation adds at most ~6e-6 |x|).  x, y: device float32 [n]. */
 asr_status asr_op_gelu(const float* x, float* y, int64_t n, void* stream);
 
 /* Bounded-wait self-check: launches one kernel that waits on a shared-memory

@@ -46,6 +46,9 @@ struct ActMaps {
   CUtensorMap h, att, ff, c3, p1, p2, gu;
   CUtensorMap cin2, cin3;  // conv-box A maps of the two stem GEMMs
   CUtensorMap qkv;         // 128-row boxes of the QKV buffer (tcgen05 attention)
+  // Store maps of the GEMM outputs (32 x 32 boxes): residual stream, QKV,
+  // FFN hidden, head, adapter hidden, conv outputs.
+  CUtensorMap o_x, o_qkv, o_ff, o_p1, o_p2, o_c2, o_c3, o_c1;
 };
 
 struct Plan {
@@ -53,7 +56,10 @@ struct Plan {
   int B = 0, F = 0, nwin_clip = 0, nwin = 0, max_win = 0, chunks = 0;
   int T1 = 0, F1 = 0, T2 = 0, F2 = 0, T3 = 0, F3 = 0;
   size_t off_clipmax = 0, off_cu = 0, off_mel = 0, off_c1 = 0, off_c2 = 0, off_c3 = 0, off_melT = 0, off_x = 0,
-         off_h = 0, off_qkv = 0, off_att = 0, off_ff = 0, off_p1 = 0, off_p2 = 0, off_gu = 0, off_pcm = 0, off_out = 0;
+         off_h = 0, off_qkv = 0, off_att = 0, off_ff = 0, off_p1 = 0, off_p2 = 0, off_gu = 0, off_pcm = 0, off_out = 0,
+         off_skflags = 0;
+  int sk_regions = 0;      // stream-K flag regions (one per eligible GEMM launch of a forward)
+  size_t sk_flag_ints = 0; // ints per region
   size_t off_tap[ASR_TAP_COUNT] = {0, 0, 0, 0, 0};
   size_t tap_bytes[ASR_TAP_COUNT] = {0, 0, 0, 0, 0};
   size_t total = 0;
@@ -254,6 +260,9 @@ struct asr_enc {
   size_t ev_used = 0;
   std::vector<std::pair<int, size_t>> prof_recs;  // (stage class, index of the first of two events)
   int launches = 0;
+  int sk_next = 0;  // next stream-K flag region of the running forward
+  char* sk_ws = nullptr;         // workspace of the running forward (stream-K scratch)
+  const Plan* sk_plan = nullptr;
 };
 
 namespace {
@@ -612,6 +621,11 @@ bool make_plan(const asr_enc* e, int64_t n, int B, Plan* p) {
     p->off_p2 = take((size_t)p->T * g->proj2_out * 2);
   }
   if (g->adapter_hidden) p->off_gu = take((size_t)p->T * g->adapter_hidden * 2);
+  // Stream-K flags of the residual GEMMs: per launch one flag per (CTA,
+  // epilogue warp).
+  p->sk_regions = 2 * g->n_layers + 2;
+  p->sk_flag_ints = (size_t)e->num_sms * 8;
+  p->off_skflags = take((size_t)p->sk_regions * p->sk_flag_ints * 4);
   p->tap_bytes[ASR_TAP_MEL] = (size_t)B * g->n_mels * p->F * 4;
   p->tap_bytes[ASR_TAP_STEM] = p->tap_bytes[ASR_TAP_LAYER0] = p->tap_bytes[ASR_TAP_ENCODER] = (size_t)p->T * d * 4;
   p->tap_bytes[ASR_TAP_HEAD] = g->proj2_out ? (size_t)p->T * g->proj2_out * 4 : 0;
@@ -625,7 +639,7 @@ bool make_plan(const asr_enc* e, int64_t n, int B, Plan* p) {
 
 asr_status gemm(asr_enc* e, const CUtensorMap* amap, const ConvGather* cg, const GemmB& w, long long M, void* out,
                 long long ldo, const float* bias, const float* pe, int period, int epi, cudaStream_t st,
-                const ConvBox* box = nullptr) {
+                const CUtensorMap* omap, const ConvBox* box = nullptr) {
   GemmParams p;
   memset(&p, 0, sizeof p);
   p.M = (int)M;
@@ -638,6 +652,10 @@ asr_status gemm(asr_enc* e, const CUtensorMap* amap, const ConvGather* cg, const
   p.status = e->status;
   p.limit_ns = kWaitLimitNs;
   p.n_fast = cg != nullptr || box != nullptr;
+  if (epi == EPI_RESID && e->sk_ws && e->sk_next < e->sk_plan->sk_regions) {
+    p.sk_flags = reinterpret_cast<int*>(e->sk_ws + e->sk_plan->off_skflags) + (size_t)e->sk_next * e->sk_plan->sk_flag_ints;
+    ++e->sk_next;
+  }
   int bn;
   if (box) {
     p.conv_box = 1;
@@ -646,7 +664,7 @@ asr_status gemm(asr_enc* e, const CUtensorMap* amap, const ConvGather* cg, const
   } else {
     bn = gemm_pick_bn((int)M, w.N, e->num_sms, cg != nullptr);
   }
-  cudaError_t r = launch_gemm(amap, w, p, epi, bn, e->num_sms, st);
+  cudaError_t r = launch_gemm(amap, w, p, epi, bn, e->num_sms, st, omap);
   if (r != cudaSuccess) return fail(e, ASR_E_CUDA, "gemm launch (N=%d K=%d M=%lld epi=%d bn=%d): %s", w.N, w.K, M, epi, bn, cudaGetErrorString(r));
   return ASR_OK;
 }
@@ -711,7 +729,18 @@ asr_status ensure_maps(asr_enc* e, const Plan& p, char* ws) {
   }
   if (ok && g->proj1_out)
     ok = make_tmap_bf16(&m.p1, ws + p.off_p1, p.T, g->proj1_out, g->proj1_out, 128) &&
-         make_tmap_bf16(&m.p2, ws + p.off_p2, p.T, g->proj2_out, g->proj2_out, 128);
+         make_tmap_bf16(&m.p2, ws + p.off_p2, p.T, g->proj2_out, g->proj2_out, 128) &&
+         make_tmap_out(&m.o_p1, ws + p.off_p1, p.T, g->proj1_out, g->proj1_out, false) &&
+         make_tmap_out(&m.o_p2, ws + p.off_p2, p.T, g->proj2_out, g->proj2_out, false);
+  if (ok)
+    ok = make_tmap_out(&m.o_x, ws + p.off_x, p.T, d, d, true) &&
+         make_tmap_out(&m.o_qkv, ws + p.off_qkv, p.T, 3 * d, 3 * d, false) &&
+         make_tmap_out(&m.o_ff, ws + p.off_ff, p.T, g->d_ffn, g->d_ffn, false);
+  if (ok && g->stem == ASR_STEM_CONV2D_CHUNKED)
+    ok = make_tmap_out(&m.o_c2, ws + p.off_c2, (unsigned long long)p.chunks * p.T2 * p.F2, g->conv_ch, g->conv_ch, false) &&
+         make_tmap_out(&m.o_c3, ws + p.off_c3, (unsigned long long)p.chunks * p.T3 * p.F3, g->conv_ch, g->conv_ch, false);
+  else if (ok)
+    ok = make_tmap_out(&m.o_c1, ws + p.off_c1, (unsigned long long)p.B * p.F, d, d, false);
   if (ok && g->adapter_hidden) ok = make_tmap_bf16(&m.gu, ws + p.off_gu, p.T, g->adapter_hidden, g->adapter_hidden, 128);
   if (!ok) {
     m.ws = nullptr;
@@ -741,7 +770,11 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
   e->launches = 0;
   e->ev_used = 0;
   e->prof_recs.clear();
+  e->sk_ws = ws;
+  e->sk_plan = &p;
+  e->sk_next = 0;
   ASR_LAUNCH(e, cudaMemsetAsync(e->status, 0, 4, st));
+  ASR_LAUNCH(e, cudaMemsetAsync(ws + p.off_skflags, 0, (size_t)p.sk_regions * p.sk_flag_ints * 4, st));
   ASR_LAUNCH(e, cudaMemsetAsync(clip_max, 0, (size_t)p.B * 4, st));
   const int w = g->window_tokens ? g->window_tokens : (int)p.Tc;
   ASR_K(PC_MISC, ASR_LAUNCH(e, launch_fill_windows(cu, p.B, (int)p.Tc, w, p.nwin_clip, st)));
@@ -758,20 +791,20 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
     if (e->box2) {
       const int TR = 128 / p.F2, tpi = (p.T2 + TR - 1) / TR;
       ConvBox b2 = {TR, p.F2, p.T2, tpi, p.chunks * tpi, 2, 2, 1, 1, 3, CB};
-      ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, &e->maps.cin2, nullptr, e->c2, (long long)p.chunks * p.T2 * p.F2, c2, C, e->c2b, nullptr, 1, EPI_GELU, st, &b2)));
+      ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, &e->maps.cin2, nullptr, e->c2, (long long)p.chunks * p.T2 * p.F2, c2, C, e->c2b, nullptr, 1, EPI_GELU, st, &e->maps.o_c2, &b2)));
     } else {
       ConvGather cg2 = {c1, p.T1, p.F1, C, p.T2, p.F2, 2, 2, 3, 3, 1, 1};
-      ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, nullptr, &cg2, e->c2, (long long)p.chunks * p.T2 * p.F2, c2, C, e->c2b, nullptr, 1, EPI_GELU, st)));
+      ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, nullptr, &cg2, e->c2, (long long)p.chunks * p.T2 * p.F2, c2, C, e->c2b, nullptr, 1, EPI_GELU, st, &e->maps.o_c2)));
     }
     if (e->box3) {
       const int TR = 128 / p.F3, tpi = (p.T3 + TR - 1) / TR;
       ConvBox b3 = {TR, p.F3, p.T3, tpi, p.chunks * tpi, 2, 2, 1, 1, 3, CB};
-      ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, &e->maps.cin3, nullptr, e->c3, (long long)p.chunks * p.T3 * p.F3, c3, C, e->c3b, nullptr, 1, EPI_GELU, st, &b3)));
+      ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, &e->maps.cin3, nullptr, e->c3, (long long)p.chunks * p.T3 * p.F3, c3, C, e->c3b, nullptr, 1, EPI_GELU, st, &e->maps.o_c3, &b3)));
     } else {
       ConvGather cg3 = {c2, p.T2, p.F2, C, p.T3, p.F3, 2, 2, 3, 3, 1, 1};
-      ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, nullptr, &cg3, e->c3, (long long)p.chunks * p.T3 * p.F3, c3, C, e->c3b, nullptr, 1, EPI_GELU, st)));
+      ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, nullptr, &cg3, e->c3, (long long)p.chunks * p.T3 * p.F3, c3, C, e->c3b, nullptr, 1, EPI_GELU, st, &e->maps.o_c3)));
     }
-    ASR_K(PC_GEMM_CONVOUT, ASR_TRY(gemm(e, &e->maps.c3, nullptr, e->cout, p.T, x, d, nullptr, e->pe, p.T3, EPI_OUT_F32 | EPI_PE, st)));
+    ASR_K(PC_GEMM_CONVOUT, ASR_TRY(gemm(e, &e->maps.c3, nullptr, e->cout, p.T, x, d, nullptr, e->pe, p.T3, EPI_OUT_F32 | EPI_PE, st, nullptr)));
   } else {
     if (p.Tc > e->pe_rows) return fail(e, ASR_E_UNSUPPORTED, "conv1d stem: %lld positions > %d", (long long)p.Tc, e->pe_rows);
     bf16* melT = reinterpret_cast<bf16*>(ws + p.off_melT);
@@ -779,25 +812,25 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
     ASR_K(PC_MISC, ASR_LAUNCH(e, launch_mel_normalize_transpose(mel, clip_max, p.B, g->n_mels, p.F, melT, st)));
     const int tpi1 = (p.F + 127) / 128, tpi2 = (int)((p.Tc + 127) / 128);
     ConvBox b1 = {128, 1, p.F, tpi1, p.B * tpi1, 1, 1, 1, 0, 1, (g->n_mels + 63) / 64};
-    ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, &e->maps.cin2, nullptr, e->c2, (long long)p.B * p.F, c1, d, e->c2b, nullptr, 1, EPI_GELU, st, &b1)));
+    ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, &e->maps.cin2, nullptr, e->c2, (long long)p.B * p.F, c1, d, e->c2b, nullptr, 1, EPI_GELU, st, &e->maps.o_c1, &b1)));
     ConvBox b2 = {128, 1, (int)p.Tc, tpi2, p.B * tpi2, 2, 1, 1, 0, 1, (d + 63) / 64};
-    ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, &e->maps.cin3, nullptr, e->c3, p.T, x, d, e->c3b, e->pe, (int)p.Tc, EPI_GELU | EPI_OUT_F32 | EPI_PE, st, &b2)));
+    ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, &e->maps.cin3, nullptr, e->c3, p.T, x, d, e->c3b, e->pe, (int)p.Tc, EPI_GELU | EPI_OUT_F32 | EPI_PE, st, nullptr, &b2)));
   }
   if (float* t = tap(ASR_TAP_STEM)) ASR_LAUNCH(e, cudaMemcpyAsync(t, x, (size_t)p.T * d * 4, cudaMemcpyDeviceToDevice, st));
 
   for (int l = 0; l < g->n_layers; ++l) {
     const LayerW& lw = e->layers[l];
     ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, lw.ln1g, lw.ln1b, p.T, d, g->ln_eps, h, false, st)));
-    ASR_K(PC_GEMM_QKV, ASR_TRY(gemm(e, &e->maps.h, nullptr, lw.qkv, p.T, qkv, 3 * d, lw.bqkv, nullptr, 1, 0, st)));
+    ASR_K(PC_GEMM_QKV, ASR_TRY(gemm(e, &e->maps.h, nullptr, lw.qkv, p.T, qkv, 3 * d, lw.bqkv, nullptr, 1, 0, st, &e->maps.o_qkv)));
     if (p.max_win <= 128)
       ASR_K(PC_ATTN, ASR_LAUNCH(e, launch_attention_tc(e->maps.qkv, qkv, cu, p.nwin, g->n_heads, att, e->status,
                                                        kWaitLimitNs, st)));
     else
       ASR_K(PC_ATTN, ASR_LAUNCH(e, launch_attention(qkv, cu, p.nwin, p.max_win, g->n_heads, att, st)));
-    ASR_K(PC_GEMM_O, ASR_TRY(gemm(e, &e->maps.att, nullptr, lw.o, p.T, x, d, lw.bo, nullptr, 1, EPI_RESID, st)));
+    ASR_K(PC_GEMM_O, ASR_TRY(gemm(e, &e->maps.att, nullptr, lw.o, p.T, x, d, lw.bo, nullptr, 1, EPI_RESID, st, &e->maps.o_x)));
     ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, lw.ln2g, lw.ln2b, p.T, d, g->ln_eps, h, false, st)));
-    ASR_K(PC_GEMM_FC1, ASR_TRY(gemm(e, &e->maps.h, nullptr, lw.fc1, p.T, ff, g->d_ffn, lw.b1, nullptr, 1, EPI_GELU, st)));
-    ASR_K(PC_GEMM_FC2, ASR_TRY(gemm(e, &e->maps.ff, nullptr, lw.fc2, p.T, x, d, lw.b2, nullptr, 1, EPI_RESID, st)));
+    ASR_K(PC_GEMM_FC1, ASR_TRY(gemm(e, &e->maps.h, nullptr, lw.fc1, p.T, ff, g->d_ffn, lw.b1, nullptr, 1, EPI_GELU, st, &e->maps.o_ff)));
+    ASR_K(PC_GEMM_FC2, ASR_TRY(gemm(e, &e->maps.ff, nullptr, lw.fc2, p.T, x, d, lw.b2, nullptr, 1, EPI_RESID, st, &e->maps.o_x)));
     if (l == 0)
       if (float* t = tap(ASR_TAP_LAYER0)) ASR_LAUNCH(e, cudaMemcpyAsync(t, x, (size_t)p.T * d * 4, cudaMemcpyDeviceToDevice, st));
   }
@@ -809,18 +842,21 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
   }
   bf16* p1 = reinterpret_cast<bf16*>(ws + p.off_p1);
   bf16* p2 = reinterpret_cast<bf16*>(ws + p.off_p2);
+  // Store map of the caller's output (plain stores if it is not 16-byte aligned).
+  CUtensorMap o_out_map;
+  const CUtensorMap* o_out = make_tmap_out(&o_out_map, out, p.T, d_out(g), d_out(g), true) ? &o_out_map : nullptr;
   ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, e->lnpg, e->lnpb, p.T, d, g->ln_eps, h, false, st)));
-  ASR_K(PC_GEMM_HEAD, ASR_TRY(gemm(e, &e->maps.h, nullptr, e->p1, p.T, p1, g->proj1_out, e->bp1, nullptr, 1, EPI_GELU, st)));
+  ASR_K(PC_GEMM_HEAD, ASR_TRY(gemm(e, &e->maps.h, nullptr, e->p1, p.T, p1, g->proj1_out, e->bp1, nullptr, 1, EPI_GELU, st, &e->maps.o_p1)));
   if (!g->adapter_hidden) {
-    ASR_K(PC_GEMM_HEAD, ASR_TRY(gemm(e, &e->maps.p1, nullptr, e->p2, p.T, out, g->proj2_out, e->bp2, nullptr, 1, EPI_OUT_F32, st)));
+    ASR_K(PC_GEMM_HEAD, ASR_TRY(gemm(e, &e->maps.p1, nullptr, e->p2, p.T, out, g->proj2_out, e->bp2, nullptr, 1, EPI_OUT_F32, st, o_out)));
     if (float* t = tap(ASR_TAP_HEAD)) ASR_LAUNCH(e, cudaMemcpyAsync(t, out, (size_t)p.T * g->proj2_out * 4, cudaMemcpyDeviceToDevice, st));
     return ASR_OK;
   }
-  ASR_K(PC_GEMM_HEAD, ASR_TRY(gemm(e, &e->maps.p1, nullptr, e->p2, p.T, p2, g->proj2_out, e->bp2, nullptr, 1, 0, st)));
+  ASR_K(PC_GEMM_HEAD, ASR_TRY(gemm(e, &e->maps.p1, nullptr, e->p2, p.T, p2, g->proj2_out, e->bp2, nullptr, 1, 0, st, &e->maps.o_p2)));
   if (float* t = tap(ASR_TAP_HEAD)) ASR_K(PC_MISC, ASR_LAUNCH(e, launch_bf16_to_f32(p2, t, (long long)p.T * g->proj2_out, st)));
   bf16* gu = reinterpret_cast<bf16*>(ws + p.off_gu);
-  ASR_K(PC_GEMM_ADAPTER, ASR_TRY(gemm(e, &e->maps.p2, nullptr, e->gu, p.T, gu, g->adapter_hidden, nullptr, nullptr, 1, EPI_SWIGLU, st)));
-  ASR_K(PC_GEMM_ADAPTER, ASR_TRY(gemm(e, &e->maps.gu, nullptr, e->down, p.T, out, g->adapter_out, nullptr, nullptr, 1, EPI_OUT_F32, st)));
+  ASR_K(PC_GEMM_ADAPTER, ASR_TRY(gemm(e, &e->maps.p2, nullptr, e->gu, p.T, gu, g->adapter_hidden, nullptr, nullptr, 1, EPI_SWIGLU, st, nullptr)));
+  ASR_K(PC_GEMM_ADAPTER, ASR_TRY(gemm(e, &e->maps.gu, nullptr, e->down, p.T, out, g->adapter_out, nullptr, nullptr, 1, EPI_OUT_F32, st, o_out)));
   return ASR_OK;
 }
 
@@ -984,7 +1020,16 @@ asr_status asr_op_log_mel(const float* pcm, int64_t n_samples, int batch, int n_
   return ASR_OK;
 }
 
-size_t asr_op_linear_ws_size(void) { return 256; }
+// Device SM count of the current device (the GEMM grid and stream-K scratch size).
+static int current_sm_count() {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+// Linear-op workspace: [status word, 256 B][stream-K flags].
+static size_t linear_flags_bytes(int sms) { return ((size_t)sms * 8 * 4 + 255) / 256 * 256; }
+size_t asr_op_linear_ws_size(void) { return 256 + linear_flags_bytes(current_sm_count()); }
 
 asr_status asr_op_linear(const void* x, const void* w, const float* bias, int64_t M, int N, int K, int epi,
                          int tile_n, void* y, void* ws, size_t ws_bytes, void* stream) {
@@ -1003,9 +1048,7 @@ asr_status asr_op_linear(const void* x, const void* w, const float* bias, int64_
       break;
     default: return fail(nullptr, ASR_E_INVAL, "linear: unknown epilogue %d", epi);
   }
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = current_sm_count();
   GemmB wb;
   wb.ptr = static_cast<const bf16*>(w);
   wb.N = N;
@@ -1014,7 +1057,6 @@ asr_status asr_op_linear(const void* x, const void* w, const float* bias, int64_
   if (!make_weight_maps(wb) || !make_tmap_bf16(&amap, x, M, K, K, 128))
     return fail(nullptr, ASR_E_INVAL, "linear: TMA descriptor encoding failed (16-byte alignment?)");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  ASR_CUDA(nullptr, cudaMemsetAsync(ws, 0, 4, st));
   GemmParams p;
   memset(&p, 0, sizeof p);
   p.M = (int)M;
@@ -1024,11 +1066,22 @@ asr_status asr_op_linear(const void* x, const void* w, const float* bias, int64_
   p.pe_period = 1;
   p.status = static_cast<int*>(ws);
   p.limit_ns = kWaitLimitNs;
+  const size_t fb = linear_flags_bytes(sms);
+  if (ws_bytes >= 256 + fb) {
+    // Enough scratch for stream-K: flags zeroed together with the status word.
+    p.sk_flags = reinterpret_cast<int*>(static_cast<char*>(ws) + 256);
+    ASR_CUDA(nullptr, cudaMemsetAsync(ws, 0, 256 + fb, st));
+  } else {
+    ASR_CUDA(nullptr, cudaMemsetAsync(ws, 0, 4, st));
+  }
   if (tile_n && tile_n != 256 && tile_n != 160 && tile_n != 128 && tile_n != 64 && tile_n != -256 && tile_n != -128)
     return fail(nullptr, ASR_E_INVAL, "linear: tile_n must be 0, 256, 160, 128, 64, -256 or -128");
   if (tile_n == 160 && N % 160) return fail(nullptr, ASR_E_INVAL, "linear: tile_n 160 needs N %% 160 == 0");
   const int bn = tile_n ? tile_n : gemm_pick_bn((int)M, N, sms, false);
-  ASR_CUDA(nullptr, launch_gemm(&amap, wb, p, e_bits, bn, sms, st));
+  CUtensorMap omap;
+  const bool f32_out = (e_bits & (EPI_OUT_F32 | EPI_RESID)) != 0;
+  const bool have_omap = !(e_bits & EPI_SWIGLU) && make_tmap_out(&omap, y, M, N, N, f32_out);
+  ASR_CUDA(nullptr, launch_gemm(&amap, wb, p, e_bits, bn, sms, st, have_omap ? &omap : nullptr));
   return ASR_OK;
 }
 

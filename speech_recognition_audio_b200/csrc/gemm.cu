@@ -34,50 +34,50 @@ constexpr int stages_for() {
 }
 
 template <int BN, bool G, int EPI>
-cudaError_t run(const CUtensorMap* a, const CUtensorMap& b, const GemmParams& p, int grid, cudaStream_t st) {
+cudaError_t run(const CUtensorMap* a, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& p, int grid, cudaStream_t st) {
   using S = GemmShape<BN, stages_for<BN>(), G>;
   auto k = gemm_bf16_tc_kernel<BN, S::STAGES, G, EPI>;
   cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_BYTES);
   if (err != cudaSuccess) return err;
-  return launch_pdl(k, dim3(grid), dim3(S::THREADS), S::SMEM_BYTES, st, a ? *a : b, b, p);
+  return launch_pdl(k, dim3(grid), dim3(S::THREADS), S::SMEM_BYTES, st, a ? *a : b, b, o, p);
 }
 
 template <int BN>
-cudaError_t run_tma(int epi, const CUtensorMap* a, const CUtensorMap& b, const GemmParams& p, int grid,
+cudaError_t run_tma(int epi, const CUtensorMap* a, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& p, int grid,
                     cudaStream_t st) {
   switch (epi) {
-    case 0: return run<BN, false, 0>(a, b, p, grid, st);
-    case EPI_GELU: return run<BN, false, EPI_GELU>(a, b, p, grid, st);
-    case EPI_OUT_F32: return run<BN, false, EPI_OUT_F32>(a, b, p, grid, st);
-    case EPI_RESID: return run<BN, false, EPI_RESID>(a, b, p, grid, st);
-    case EPI_OUT_F32 | EPI_PE: return run<BN, false, EPI_OUT_F32 | EPI_PE>(a, b, p, grid, st);
-    case EPI_SWIGLU: return run<BN, false, EPI_SWIGLU>(a, b, p, grid, st);
-    case EPI_GELU | EPI_OUT_F32 | EPI_PE: return run<BN, false, EPI_GELU | EPI_OUT_F32 | EPI_PE>(a, b, p, grid, st);
+    case 0: return run<BN, false, 0>(a, b, o, p, grid, st);
+    case EPI_GELU: return run<BN, false, EPI_GELU>(a, b, o, p, grid, st);
+    case EPI_OUT_F32: return run<BN, false, EPI_OUT_F32>(a, b, o, p, grid, st);
+    case EPI_RESID: return run<BN, false, EPI_RESID>(a, b, o, p, grid, st);
+    case EPI_OUT_F32 | EPI_PE: return run<BN, false, EPI_OUT_F32 | EPI_PE>(a, b, o, p, grid, st);
+    case EPI_SWIGLU: return run<BN, false, EPI_SWIGLU>(a, b, o, p, grid, st);
+    case EPI_GELU | EPI_OUT_F32 | EPI_PE: return run<BN, false, EPI_GELU | EPI_OUT_F32 | EPI_PE>(a, b, o, p, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
 // 240-wide tiles only serve the convolutions (N = 480).
-cudaError_t run_tma240(int epi, const CUtensorMap* a, const CUtensorMap& b, const GemmParams& p, int grid,
+cudaError_t run_tma240(int epi, const CUtensorMap* a, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& p, int grid,
                        cudaStream_t st) {
   switch (epi) {
-    case EPI_GELU: return run<240, false, EPI_GELU>(a, b, p, grid, st);
-    case EPI_GELU | EPI_OUT_F32 | EPI_PE: return run<240, false, EPI_GELU | EPI_OUT_F32 | EPI_PE>(a, b, p, grid, st);
+    case EPI_GELU: return run<240, false, EPI_GELU>(a, b, o, p, grid, st);
+    case EPI_GELU | EPI_OUT_F32 | EPI_PE: return run<240, false, EPI_GELU | EPI_OUT_F32 | EPI_PE>(a, b, o, p, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
 template <int BN>
-cudaError_t run_gather(int epi, const CUtensorMap& b, const GemmParams& p, int grid, cudaStream_t st) {
+cudaError_t run_gather(int epi, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& p, int grid, cudaStream_t st) {
   switch (epi) {
-    case EPI_GELU: return run<BN, true, EPI_GELU>(nullptr, b, p, grid, st);
-    case EPI_GELU | EPI_OUT_F32 | EPI_PE: return run<BN, true, EPI_GELU | EPI_OUT_F32 | EPI_PE>(nullptr, b, p, grid, st);
+    case EPI_GELU: return run<BN, true, EPI_GELU>(nullptr, b, o, p, grid, st);
+    case EPI_GELU | EPI_OUT_F32 | EPI_PE: return run<BN, true, EPI_GELU | EPI_OUT_F32 | EPI_PE>(nullptr, b, o, p, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
 template <int BN, int EPI>
-cudaError_t run2(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p, int grid, cudaStream_t st) {
+cudaError_t run2(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& p, int grid, cudaStream_t st) {
   using S = Gemm2Shape<BN, (BN >= 192 ? 6 : 8)>;
   auto k = gemm_bf16_tc2_kernel<BN, S::STAGES, EPI>;
   cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_BYTES);
@@ -96,31 +96,65 @@ cudaError_t run2(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, k, a, b, p);
+  return cudaLaunchKernelEx(&cfg, k, a, b, o, p);
 }
 
 template <int BN>
-cudaError_t run2_epi(int epi, const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p, int grid,
+cudaError_t run2_epi(int epi, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& p, int grid,
                      cudaStream_t st) {
   switch (epi) {
-    case 0: return run2<BN, 0>(a, b, p, grid, st);
-    case EPI_GELU: return run2<BN, EPI_GELU>(a, b, p, grid, st);
-    case EPI_OUT_F32: return run2<BN, EPI_OUT_F32>(a, b, p, grid, st);
-    case EPI_RESID: return run2<BN, EPI_RESID>(a, b, p, grid, st);
-    case EPI_OUT_F32 | EPI_PE: return run2<BN, EPI_OUT_F32 | EPI_PE>(a, b, p, grid, st);
-    case EPI_SWIGLU: return run2<BN, EPI_SWIGLU>(a, b, p, grid, st);
-    case EPI_GELU | EPI_OUT_F32 | EPI_PE: return run2<BN, EPI_GELU | EPI_OUT_F32 | EPI_PE>(a, b, p, grid, st);
+    case 0: return run2<BN, 0>(a, b, o, p, grid, st);
+    case EPI_GELU: return run2<BN, EPI_GELU>(a, b, o, p, grid, st);
+    case EPI_OUT_F32: return run2<BN, EPI_OUT_F32>(a, b, o, p, grid, st);
+    case EPI_RESID: return run2<BN, EPI_RESID>(a, b, o, p, grid, st);
+    case EPI_OUT_F32 | EPI_PE: return run2<BN, EPI_OUT_F32 | EPI_PE>(a, b, o, p, grid, st);
+    case EPI_SWIGLU: return run2<BN, EPI_SWIGLU>(a, b, o, p, grid, st);
+    case EPI_GELU | EPI_OUT_F32 | EPI_PE: return run2<BN, EPI_GELU | EPI_OUT_F32 | EPI_PE>(a, b, o, p, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
-cudaError_t run2_240(int epi, const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p, int grid,
+cudaError_t run2_240(int epi, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& p, int grid,
                      cudaStream_t st) {
   switch (epi) {
-    case EPI_GELU: return run2<240, EPI_GELU>(a, b, p, grid, st);
-    case EPI_GELU | EPI_OUT_F32 | EPI_PE: return run2<240, EPI_GELU | EPI_OUT_F32 | EPI_PE>(a, b, p, grid, st);
+    case EPI_GELU: return run2<240, EPI_GELU>(a, b, o, p, grid, st);
+    case EPI_GELU | EPI_OUT_F32 | EPI_PE: return run2<240, EPI_GELU | EPI_OUT_F32 | EPI_PE>(a, b, o, p, grid, st);
     default: return cudaErrorInvalidValue;
   }
+}
+
+// CTA pairs that can be resident at once: 148 SMs do not always pair up
+// into 74 clusters of two, and stream-K needs every pair of its grid
+// resident (an owner waits for the next pair's first piece).  Queried once
+// per device for the largest pair configuration (one CTA per SM).
+int resident_pairs(int num_sms) {
+  static std::mutex mu;
+  static int cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  using S = Gemm2Shape<256, 6>;
+  auto k = gemm_bf16_tc2_kernel<256, 6, EPI_RESID>;
+  int n = 0;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_BYTES) == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(num_sms, 1, 1);
+    cfg.blockDim = dim3(S::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = S::SMEM_BYTES;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void*>(k), &cfg) != cudaSuccess) n = 0;
+  }
+  cudaGetLastError();
+  if (n <= 0 || n > num_sms / 2) n = num_sms / 2;
+  if (dev >= 0 && dev < 64) cache[dev] = n;
+  return n;
 }
 
 }  // namespace
@@ -158,6 +192,22 @@ bool make_tmap_convbox(CUtensorMap* map, const void* ptr, int C, int F_in, int T
   cuuint32_t es[4] = {1, (cuuint32_t)sf, (cuuint32_t)st, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tmap_out(CUtensorMap* map, const void* ptr, unsigned long long rows, unsigned long long cols,
+                   unsigned long long row_stride_elems, bool f32) {
+  EncodeTiledFn fn = encode_fn();
+  const unsigned long long es = f32 ? 4 : 2;
+  if (!fn || !ptr || (reinterpret_cast<uintptr_t>(ptr) & 15) || (row_stride_elems * es) % 16 || rows == 0 || cols == 0)
+    return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {row_stride_elems * es};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr),
+            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -208,7 +258,8 @@ int gemm_pick_bn_conv(int n_sub, int N, int num_sms) {
 }
 
 cudaError_t launch_gemm(const CUtensorMap* a_map, const GemmB& w, GemmParams p, int epi, int bn, int num_sms,
-                        cudaStream_t st) {
+                        cudaStream_t st, const CUtensorMap* out_map) {
+  p.out_tma = (out_map != nullptr && !(epi & (EPI_PE | EPI_SWIGLU))) ? 1 : 0;
   if (bn < 0) {
     // CTA-pair kernel: 256 x |bn| tiles, each CTA stages |bn|/2 rows of B.
     const int w2 = -bn;
@@ -220,14 +271,25 @@ cudaError_t launch_gemm(const CUtensorMap* a_map, const GemmB& w, GemmParams p, 
     p.n_blocks = (p.N + w2 - 1) / w2;
     p.k_blocks = (p.K + 63) / 64;
     p.num_tiles = p.m_blocks * p.n_blocks;
-    const int pairs = std::min(p.num_tiles, num_sms / 2);
+    const int pairs = std::min(p.num_tiles, resident_pairs(num_sms));
     const int grid = 2 * pairs;
-    if (w2 == 240) return run2_240(epi, *a_map, w.map[slot2], p, grid, st);
-    return w2 == 256 ? run2_epi<256>(epi, *a_map, w.map[slot2], p, grid, st)
-                     : run2_epi<128>(epi, *a_map, w.map[slot2], p, grid, st);
+    // Stream-K when the caller gave the flags, the epilogue is the residual
+    // add, whole tiles would leave a ragged last wave, and K is long enough
+    // (>= 40 k-blocks) for a split piece to outlast an epilogue (about 3 us):
+    // with short K the extra epilogues of the split tiles cost more than the
+    // balanced last wave saves.
+    p.sk = (p.sk_flags && epi == EPI_RESID && !p.conv_box && p.k_blocks >= 40 && p.num_tiles > pairs &&
+            p.num_tiles % pairs != 0)
+               ? 1
+               : 0;
+    if (w2 == 240) return run2_240(epi, *a_map, w.map[slot2], p.out_tma ? *out_map : w.map[slot2], p, grid, st);
+    const CUtensorMap& o2 = p.out_tma ? *out_map : w.map[slot2];
+    return w2 == 256 ? run2_epi<256>(epi, *a_map, w.map[slot2], o2, p, grid, st)
+                     : run2_epi<128>(epi, *a_map, w.map[slot2], o2, p, grid, st);
   }
   const int slot = gemm_bn_slot(bn);
   if (slot < 0 || p.M <= 0) return cudaErrorInvalidValue;
+  p.sk = 0;  // the one-SM kernel runs whole tiles
   p.N = w.N;
   p.K = w.K;
   p.m_blocks = p.conv_box ? p.cb.n_sub : (p.M + 127) / 128;
@@ -236,22 +298,23 @@ cudaError_t launch_gemm(const CUtensorMap* a_map, const GemmB& w, GemmParams p, 
   p.num_tiles = p.m_blocks * p.n_blocks;
   const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
   const CUtensorMap& b = w.map[slot];
+  const CUtensorMap& o = p.out_tma ? *out_map : b;
   const bool gather = (a_map == nullptr);
   if (gather) {
     switch (bn) {
-      case 256: return run_gather<256>(epi, b, p, grid, st);
-      case 240: return run_gather<240>(epi, b, p, grid, st);
-      case 128: return run_gather<128>(epi, b, p, grid, st);
-      case 64: return run_gather<64>(epi, b, p, grid, st);
+      case 256: return run_gather<256>(epi, b, o, p, grid, st);
+      case 240: return run_gather<240>(epi, b, o, p, grid, st);
+      case 128: return run_gather<128>(epi, b, o, p, grid, st);
+      case 64: return run_gather<64>(epi, b, o, p, grid, st);
       default: return cudaErrorInvalidValue;
     }
   }
   switch (bn) {
-    case 256: return run_tma<256>(epi, a_map, b, p, grid, st);
-    case 240: return run_tma240(epi, a_map, b, p, grid, st);
-    case 160: return run_tma<160>(epi, a_map, b, p, grid, st);
-    case 128: return run_tma<128>(epi, a_map, b, p, grid, st);
-    case 64: return run_tma<64>(epi, a_map, b, p, grid, st);
+    case 256: return run_tma<256>(epi, a_map, b, o, p, grid, st);
+    case 240: return run_tma240(epi, a_map, b, o, p, grid, st);
+    case 160: return run_tma<160>(epi, a_map, b, o, p, grid, st);
+    case 128: return run_tma<128>(epi, a_map, b, o, p, grid, st);
+    case 64: return run_tma<64>(epi, a_map, b, o, p, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -76,7 +76,93 @@ struct GemmParams {
   int n_fast;             // tile order: 1 = the n-blocks of an m-block run back to back
   int conv_box;           // 1 = A is a ConvBox (4-D strided TMA), rows mapped per image
   ConvBox cb;
+  int out_tma;            // 1 = the kernel's output tensor map is valid (TMA store epilogue)
+  // Stream-K (CTA-pair kernel, residual epilogue): the num_tiles x k_blocks
+  // (tile, k-block) units are cut into equal contiguous ranges, one per CTA
+  // pair, so that no pair idles in a partial last wave.  A tile split
+  // between two pairs is a trailing piece (the first piece of the later
+  // pair: its partial sum goes into the residual stream, then one flag per
+  // epilogue warp is raised) and a leading piece (the owner, which adds the
+  // bias: it waits for the flag before its own residual update), so every
+  // element sees the same additions in the same order on every run.
+  int sk;
+  int* sk_flags;          // [pairs][2 CTAs][8 warps], zero before the launch
 };
+
+// Kinds of work piece: a whole tile, the trailing k-blocks of a split tile
+// (partial sum added to the residual stream first, without bias), or the
+// leading k-blocks of a split tile (adds bias and its sum once the trailing
+// piece's update has landed).
+enum : int { PIECE_FULL = 0, PIECE_PARTIAL = 1, PIECE_OWNER = 2 };
+
+// The sequence of (tile, k-block range) pieces of one scheduling unit (a CTA
+// pair): tiles unit, unit + n_units, ... whole, or under stream-K the unit
+// range [total * unit / n_units, total * (unit + 1) / n_units) of the
+// row-major (tile, k-block) order.  With num_tiles >= n_units every range
+// spans at least one tile's k-blocks, so a tile is split at most once:
+// its trailing part is the first piece of unit + 1.
+struct PieceIter {
+  long long u, u_end;
+  int t, step;
+  __device__ __forceinline__ PieceIter(const GemmParams& p, int unit, int n_units) : u(0), u_end(0), t(unit), step(n_units) {
+    if (p.sk) {
+      const long long total = (long long)p.num_tiles * p.k_blocks;
+      u = total * unit / n_units;
+      u_end = total * (unit + 1) / n_units;
+    }
+  }
+  __device__ __forceinline__ bool next(const GemmParams& p, int& tile, int& kb0, int& kb1) {
+    if (!p.sk) {
+      if (t >= p.num_tiles) return false;
+      tile = t;
+      kb0 = 0;
+      kb1 = p.k_blocks;
+      t += step;
+      return true;
+    }
+    if (u >= u_end) return false;
+    tile = static_cast<int>(u / p.k_blocks);
+    kb0 = static_cast<int>(u - (long long)tile * p.k_blocks);
+    const long long left = u_end - u;
+    kb1 = left < p.k_blocks - kb0 ? kb0 + static_cast<int>(left) : p.k_blocks;
+    u += kb1 - kb0;
+    return true;
+  }
+};
+__device__ __forceinline__ int piece_kind(const GemmParams& p, int kb0, int kb1) {
+  return kb0 > 0 ? PIECE_PARTIAL : (kb1 < p.k_blocks ? PIECE_OWNER : PIECE_FULL);
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Orders this thread's global accesses of the async proxy (bulk tensor
+// copies) with its generic-proxy accesses, in both directions.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+// Wait (one thread) until *flag != 0, for at most limit_ns; gives up early
+// when the status word already holds an error.
+static __device__ __noinline__ bool flag_wait_bounded(const int* flag, uint64_t limit_ns, int* status, int code) {
+  if (ld_acquire_gpu(flag) != 0) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 0;; ++it) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(flag) != 0) return true;
+    if ((it & 15) == 15) {
+      if (globaltimer_ns() - t0 > limit_ns) {
+        if (status) atomicCAS(status, 0, code);
+        return false;
+      }
+      if (status && *reinterpret_cast<volatile int*>(status) != 0) return false;
+    }
+  }
+}
 
 // Output rows covered by 128-row sub-tile u: [first, last) (conv-box mode
 // maps a sub-tile to TR output t-rows of one image; rows past the image end
@@ -175,41 +261,91 @@ __device__ __forceinline__ void epilogue_prefetch_l2(const GemmParams& p, int t,
     asm volatile("prefetch.global.L2 [%0];" ::"l"(base + c) : "memory");
 }
 
+// TMA stores from shared memory (bulk-group completion).  The tensor map
+// covers the output [rows, cols]; the box is 32 x 32 with the 128-byte
+// (fp32) or 64-byte (bf16) swizzle that the epilogue buffer is written in.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+// out[box] += smem (fp32 add performed at L2): the residual update.
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, const void* src, int x, int y) {
+  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Shared-memory sources of this thread's bulk stores may be overwritten.
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// This thread's bulk stores have completed (written to global memory).
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Bias of the tile's columns for one epilogue warp, loaded before the
+// accumulator is ready: lane l holds bias[n0 + c_j + l] for the warp's
+// column groups c_j = 32 half + 64 j (the epilogue broadcasts it by shuffle).
+__device__ __forceinline__ void load_bias(const GemmParams& p, int n0, int BN, int half, int lane, float* breg) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int c = half * 32 + 64 * j;
+    const int n = n0 + c + lane;
+    breg[j] = (p.bias && c < BN && c + lane < BN && n < p.N) ? __ldg(p.bias + n) : 0.0f;
+  }
+}
+
 // Epilogue of one warp: its 32 TMEM lanes (tile rows row0..row0+31) over the
 // 32-column groups g = half, half + 2, ... of a BN-wide accumulator.
 //   phase A (one thread per row): tcgen05.ld 32 columns, add the bias, apply
 //     GELU or SwiGLU, and write the row into the warp's 4 KB shared buffer
-//     (fp32, or bf16 for bf16 outputs; 16-byte chunks XOR-swizzled by row so
-//     that both phases are free of bank conflicts);
-//   phase B (threads along columns): read the buffer back so that a warp
-//     instruction covers whole 128-byte (fp32) or 64-byte (bf16) row
-//     segments, add positions / the residual with coalesced loads, and store
-//     with coalesced 16-byte (fp32) or 8-byte (bf16) stores.
+//     (fp32, or bf16 for bf16 outputs; 16-byte chunks XOR-swizzled by row:
+//     the 128-byte / 64-byte swizzle of the TMA store, which also keeps
+//     the row-wise writes free of bank conflicts);
+//   store: one lane issues a TMA store of the 32 x 32 box (plain outputs) or
+//     a TMA reduce-add into the fp32 residual stream, so the warp never
+//     waits on global memory; the buffer is reused once the bulk copy has
+//     read it.
+//   phase B (fallback, threads along columns) for positions, SwiGLU, conv
+//     sub-tiles whose 32 rows are not all valid, and 16-column tails: read
+//     the buffer back so that a warp instruction covers whole 128-byte
+//     (fp32) or 64-byte (bf16) row segments, add positions with coalesced
+//     loads, and store with coalesced 16-byte (fp32) or 8-byte (bf16)
+//     stores.
+//   Stream-K pieces (residual epilogue only): PIECE_PARTIAL adds its raw
+//     accumulator (no bias) to the residual stream; the caller orders the
+//     owner's update after it.
 template <int EPI>
-__device__ __forceinline__ void epilogue_warp(const GemmParams& p, uint32_t tb, int row0, int mlimit, int n0, int BN,
-                                              int half, int lane, uint8_t* wbuf) {
+__device__ __forceinline__ void epilogue_warp(const GemmParams& p, const CUtensorMap* tm_out, uint32_t tb, int row0,
+                                              int mlimit, int n0, int BN, int half, int lane, uint8_t* wbuf,
+                                              const float* breg, int kind = PIECE_FULL) {
   constexpr bool F32 = (EPI & (EPI_OUT_F32 | EPI_RESID)) != 0;
   constexpr bool SWI = (EPI & EPI_SWIGLU) != 0;
+  constexpr bool TMA_OK = (EPI & (EPI_PE | EPI_SWIGLU)) == 0;
+  if (row0 >= mlimit) return;  // no valid row in this quarter (warp-uniform)
+  // A 32-row box may be stored whole when all its rows belong to this
+  // sub-tile, or when the rows past the end lie past M (the TMA clips them).
+  const bool rows_ok = TMA_OK && p.out_tma && (mlimit - row0 >= 32 || mlimit >= p.M);
+  int j = 0;
 #pragma unroll 1
-  for (int c = half * 32; c < BN; c += 64) {
+  for (int c = half * 32; c < BN; c += 64, ++j) {
     const int n = n0 + c;
     if (n >= p.N) break;                                  // warp-uniform
     const int w = (BN - c < 32 || p.N - n < 32) ? 16 : 32;  // valid columns in this group (N % 16 == 0)
+    const bool use_tma = rows_ok && BN - c >= 32;
     float v[32];
     tmem_ld16(tb + c, v);
     if (BN - c >= 32) tmem_ld16(tb + c + 16, v + 16);
     tmem_ld_wait();
     // ---- phase A
-    if (p.bias) {
-      const float4* b4 = reinterpret_cast<const float4*>(p.bias + n);
+    if (p.bias && kind != PIECE_PARTIAL) {
+      const float bj = breg[j];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if (i < 4 || w == 32) {
-          const float4 b = __ldg(b4 + i);
-          v[4 * i] += b.x; v[4 * i + 1] += b.y; v[4 * i + 2] += b.z; v[4 * i + 3] += b.w;
-        }
-      }
+      for (int i = 0; i < 32; ++i) v[i] += __shfl_sync(0xffffffffu, bj, i);
     }
+    // The buffer may still be the source of the previous group's bulk store.
+    if (lane == 0) bulk_wait_read0();
+    __syncwarp();
     if (SWI) {
       // gate = columns c..c+15, up = c+16..c+31 -> 16 bf16 outputs (2 chunks).
       uint4* row = reinterpret_cast<uint4*>(wbuf + lane * 64);
@@ -218,8 +354,8 @@ __device__ __forceinline__ void epilogue_warp(const GemmParams& p, uint32_t tb, 
         alignas(16) __nv_bfloat162 r[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int j = 8 * k + 2 * i;
-          r[i] = __floats2bfloat162_rn(silu(v[j]) * v[16 + j], silu(v[j + 1]) * v[17 + j]);
+          const int jj = 8 * k + 2 * i;
+          r[i] = __floats2bfloat162_rn(silu(v[jj]) * v[16 + jj], silu(v[jj + 1]) * v[17 + jj]);
         }
         row[k ^ ((lane >> 1) & 3)] = *reinterpret_cast<uint4*>(r);
       }
@@ -246,6 +382,18 @@ __device__ __forceinline__ void epilogue_warp(const GemmParams& p, uint32_t tb, 
           row[k ^ ((lane >> 1) & 3)] = *reinterpret_cast<uint4*>(r);
         }
       }
+    }
+    if (use_tma) {
+      fence_proxy_async_smem();  // make this lane's smem writes visible to the bulk copy
+      __syncwarp();
+      if (lane == 0) {
+        if (EPI & EPI_RESID)
+          tma_reduce_add_2d(tm_out, wbuf, n, row0);
+        else
+          tma_store_2d(tm_out, wbuf, n, row0);
+        bulk_commit();
+      }
+      continue;
     }
     __syncwarp();
     // ---- phase B
@@ -304,7 +452,7 @@ __device__ __forceinline__ void epilogue_warp(const GemmParams& p, uint32_t tb, 
 template <int BN, int STAGES, bool GATHER, int EPI>
 __global__ void __launch_bounds__(GemmShape<BN, STAGES, GATHER>::THREADS, 1)
     gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const GemmParams p) {
+                        const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
   using S = GemmShape<BN, STAGES, GATHER>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -454,20 +602,23 @@ __global__ void __launch_bounds__(GemmShape<BN, STAGES, GATHER>::THREADS, 1)
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++tl) {
       const int a = tl & 1;
       const uint32_t aph = (tl >> 1) & 1;
-      if (EPI & EPI_RESID) epilogue_prefetch_l2(p, t, half, q, lane, BN, S::BM, rank_rows);
-      if (!mbar_wait_bounded(&tfull[a], aph, p.limit_ns, p.status, DEV_TIMEOUT_EPILOGUE)) break;
-      tc_fence_after();
       int mb, nb;
       tile_coords(p, t, mb, nb);
+      const int n0 = nb * BN;
+      if (EPI & EPI_RESID) epilogue_prefetch_l2(p, t, half, q, lane, BN, S::BM, rank_rows);
+      float breg[4];
+      load_bias(p, n0, BN, half, lane, breg);
+      if (!mbar_wait_bounded(&tfull[a], aph, p.limit_ns, p.status, DEV_TIMEOUT_EPILOGUE)) break;
+      tc_fence_after();
       int r_first, r_last;
       subtile_rows(p, mb, r_first, r_last);
-      const int n0 = nb * BN;
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + a * S::ACC_COLS;
-      epilogue_warp<EPI>(p, tb, r_first + 32 * q, r_last, n0, BN, half, lane, sEpi + (warp - 2) * 4096);
+      epilogue_warp<EPI>(p, &tmOut, tb, r_first + 32 * q, r_last, n0, BN, half, lane, sEpi + (warp - 2) * 4096, breg);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[a]);
     }
+    if (lane == 0) bulk_wait0();  // bulk stores complete before the CTA exits
   } else if (GATHER) {
     // ------------------------------------------------ implicit-GEMM gather
     constexpr int RSTEP = (S::GATHER_WARPS > 0 ? S::GATHER_WARPS : 1) * 4;  // rows per pass (8 threads per row)

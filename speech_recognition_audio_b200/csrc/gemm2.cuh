@@ -111,7 +111,7 @@ struct Gemm2Shape {
 template <int BN, int STAGES, int EPI>
 __global__ void __launch_bounds__(Gemm2Shape<BN, STAGES>::THREADS, 1)
     gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                         const GemmParams p) {
+                         const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
   using S = Gemm2Shape<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -165,13 +165,15 @@ __global__ void __launch_bounds__(Gemm2Shape<BN, STAGES>::THREADS, 1)
       const uint32_t full_leader0 = mapa_shared(smem_u32(&full[0]), 0);
       int it = 0;
       bool ok = true;
-      for (int t = pair; t < p.num_tiles && ok; t += n_pairs) {
+      PieceIter pi(p, pair, n_pairs);
+      int t, kb0, kb1;
+      while (ok && pi.next(p, t, kb0, kb1)) {
         int mb, nb;
         tile_coords(p, t, mb, nb);
         const int u = 2 * mb + static_cast<int>(rank);  // this CTA's 128-row sub-tile
         const int m0 = u * 128;
         const int n0 = nb * BN + static_cast<int>(rank) * (BN / 2);
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
           if (!mbar_wait_bounded(&empty[s], ph ^ 1, p.limit_ns, p.status, DEV_TIMEOUT_PRODUCER)) {
@@ -206,7 +208,9 @@ __global__ void __launch_bounds__(Gemm2Shape<BN, STAGES>::THREADS, 1)
       const uint32_t idesc = idesc_bf16_f32(S::BM, BN);
       int it = 0, tl = 0;
       bool ok = true;
-      for (int t = pair; t < p.num_tiles && ok; t += n_pairs, ++tl) {
+      PieceIter pi(p, pair, n_pairs);
+      int t, kb0, kb1;
+      for (; ok && pi.next(p, t, kb0, kb1); ++tl) {
         const int a = tl & 1;
         const uint32_t aph = (tl >> 1) & 1;
         if (!mbar_wait_bounded(&tempty[a], aph ^ 1, p.limit_ns, p.status, DEV_TIMEOUT_MMA)) {
@@ -215,7 +219,7 @@ __global__ void __launch_bounds__(Gemm2Shape<BN, STAGES>::THREADS, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + a * S::ACC_COLS;
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
           if (!mbar_wait_bounded(&full[s], ph, p.limit_ns, p.status, DEV_TIMEOUT_MMA)) {
@@ -227,7 +231,7 @@ __global__ void __launch_bounds__(Gemm2Shape<BN, STAGES>::THREADS, 1)
           const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + s * S::B_BYTES));
 #pragma unroll
           for (int k = 0; k < S::BK / 16; ++k)
-            tc_mma_bf16_pair(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+            tc_mma_bf16_pair(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
           tc_commit_pair_mc(&empty[s], 0x3);
           ++it;
         }
@@ -243,24 +247,50 @@ __global__ void __launch_bounds__(Gemm2Shape<BN, STAGES>::THREADS, 1)
     const int half = (warp - 2) / 4;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
     const int rank_rows = static_cast<int>(rank) * 128;
+    const int ew = warp - 2;
     int tl = 0;
-    for (int t = pair; t < p.num_tiles; t += n_pairs, ++tl) {
+    PieceIter pi(p, pair, n_pairs);
+    int t, kb0, kb1;
+    for (; pi.next(p, t, kb0, kb1); ++tl) {
       const int a = tl & 1;
       const uint32_t aph = (tl >> 1) & 1;
-      if (EPI & EPI_RESID) epilogue_prefetch_l2(p, t, half, q, lane, BN, S::BM, rank_rows);
-      if (!mbar_wait_bounded(&tfull[a], aph, p.limit_ns, p.status, DEV_TIMEOUT_EPILOGUE)) break;
-      tc_fence_after();
+      const int kind = piece_kind(p, kb0, kb1);
       int mb, nb;
       tile_coords(p, t, mb, nb);
+      const int n0 = nb * BN;
+      if ((EPI & EPI_RESID) && kind != PIECE_PARTIAL) epilogue_prefetch_l2(p, t, half, q, lane, BN, S::BM, rank_rows);
+      float breg[4];
+      load_bias(p, n0, BN, half, lane, breg);
+      if (!mbar_wait_bounded(&tfull[a], aph, p.limit_ns, p.status, DEV_TIMEOUT_EPILOGUE)) break;
+      tc_fence_after();
       int r_first, r_last;
       subtile_rows(p, 2 * mb + static_cast<int>(rank), r_first, r_last);
-      const int n0 = nb * BN;
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + a * S::ACC_COLS;
-      epilogue_warp<EPI>(p, tb, r_first + 32 * q, r_last, n0, BN, half, lane, sEpi + (warp - 2) * 4096);
+      // Flag of this warp's rows and columns: the trailing piece of a split
+      // tile is the first piece of the next pair, so it uses that pair's slot.
+      const int slot = kind == PIECE_PARTIAL ? pair : pair + 1;
+      int* flag = kind == PIECE_FULL ? nullptr : p.sk_flags + (slot * 2 + static_cast<int>(rank)) * S::EPI_WARPS + ew;
+      bool have = true;
+      if (kind == PIECE_OWNER) {
+        if (lane == 0) {
+          have = flag_wait_bounded(flag, p.limit_ns, p.status, DEV_TIMEOUT_EPILOGUE);
+          fence_proxy_async_global();  // the bulk reduces below come after the trailing piece's
+        }
+        have = __shfl_sync(0xffffffffu, have, 0);
+      }
+      if (have)
+        epilogue_warp<EPI>(p, &tmOut, tb, r_first + 32 * q, r_last, n0, BN, half, lane, sEpi + ew * 4096, breg, kind);
       tc_fence_before();
       __syncwarp();
+      if (kind == PIECE_PARTIAL && lane == 0) {
+        bulk_wait0();                 // this warp's bulk reduces have been performed
+        fence_proxy_async_global();
+        __threadfence();
+        st_release_gpu(flag, 1);
+      }
       if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8u * a);
     }
+    if (lane == 0) bulk_wait0();  // bulk stores complete before the CTA exits
   }
 
   tc_fence_before();

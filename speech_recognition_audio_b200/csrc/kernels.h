@@ -83,8 +83,14 @@ bool make_tmap_convbox(CUtensorMap* map, const void* ptr, int C, int F_in, int T
 int gemm_pick_bn(int M, int N, int num_sms, bool gather);
 // Tile choice for a conv-box GEMM with n_sub 128-row sub-tiles.
 int gemm_pick_bn_conv(int n_sub, int N, int num_sms);
+// TMA map of a GEMM output [rows, cols] (row stride in elements), box 32 x 32,
+// fp32 (128-byte swizzle) or bf16 (64-byte swizzle): the epilogue's store map.
+bool make_tmap_out(CUtensorMap* map, const void* ptr, unsigned long long rows, unsigned long long cols,
+                   unsigned long long row_stride_elems, bool f32);
 // a_map: TMA map of A (box 128 x 64), or null with p.g set for the implicit-GEMM mode.
+// out_map: store map of the output (make_tmap_out), or null for plain stores;
+// ignored for the position and SwiGLU epilogues.
 cudaError_t launch_gemm(const CUtensorMap* a_map, const GemmB& w, GemmParams p, int epi, int bn, int num_sms,
-                        cudaStream_t st);
+                        cudaStream_t st, const CUtensorMap* out_map);
 
 }  // namespace asr

@@ -59,6 +59,34 @@ def test_linear_tile_modes(tile_n, M, N, K):
     assert np.abs(y - g).max() <= 2.0 ** -8 * np.abs(g).max() + 1e-3
 
 
+@pytest.mark.parametrize("M,N,K,epi", [(6240, 1280, 5120, "resid"), (6240, 1280, 2560, "resid"),
+                                       (3000, 2048, 4096, "resid"), (600, 1280, 5120, "resid"),
+                                       (3000, 2048, 4096, "f32")])
+def test_linear_stream_k(M, N, K, epi):
+    """The residual epilogue on CTA-pair tiles runs stream-K when the tile
+    count leaves a ragged last wave: parity with the oracle, and two runs
+    agree bit for bit (a split tile's two updates land in a fixed order)."""
+    rng = np.random.default_rng(M + N + K)
+    x = _bf16(rng.normal(size=(M, K)))
+    w = _bf16(rng.normal(size=(N, K)) * 0.03)
+    b = torch.from_numpy(rng.normal(size=N).astype(np.float32))
+    acc = oracle.linear(x.float().numpy(), w, b.numpy())
+    xc, wc, bc = x.cuda(), w.cuda(), b.cuda()
+    runs = []
+    for _ in range(2):
+        if epi == "resid":
+            r0 = np.random.default_rng(5).normal(size=(M, N)).astype(np.float32)
+            out = torch.from_numpy(r0).cuda()
+            sra.linear(xc, wc, bc, sra.EPI_F32_RESID, out=out, tile_n=-256)
+            ref = r0 + acc
+        else:
+            out = sra.linear(xc, wc, bc, sra.EPI_F32, tile_n=-256)
+            ref = acc
+        runs.append(out.cpu().numpy())
+    np.testing.assert_allclose(runs[0], ref, rtol=1e-4, atol=2e-4 * np.sqrt(K / 64) * 0.6)
+    assert np.array_equal(runs[0], runs[1])
+
+
 @pytest.mark.parametrize("epi", ["gelu", "f32", "resid", "swiglu"])
 def test_linear_epilogues(epi):
     M, N, K = 333, 1024, 768
