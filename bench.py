@@ -421,7 +421,11 @@ def main():
     gemm_keys = [k for k in per_step if k.startswith("gemm")]
     gemm_ms = sum(per_step[k] for k in gemm_keys)
     gemm_flops = sum(fl.get(k, 0) for k in gemm_keys)
-    peak_t = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    # Burst peak: the timed steps last well under a second and the clocks
+    # sampled under load stay near boost, above the power-capped clock of
+    # the seconds-long sustained measurement (its ratio is reported beside).
+    peak_t = peaks.get("bf16_tflops", peaks.get("bf16_tflops_sustained"))
+    peak_sus = peaks.get("bf16_tflops_sustained")
     # Dominant kernel: the largest GEMM stage of the step (one shape, one kernel).
     top = max(gemm_keys, key=lambda k: per_step[k]) if gemm_keys else None
     roofline = None
@@ -434,7 +438,8 @@ def main():
                     "unit": "TFLOP/s", "frac": (achieved / peak_t) if achieved else None,
                     "traffic": profile_traffic(f"{top}_{w.name}"),
                     "flops_per_launch": per_launch, "avg_launch_ms": avg_ms, "launches_per_step": n_l,
-                    "peak_kind": f"{peak_kind} sustained bf16 (MEASURED_PEAKS.json)"}
+                    "peak_kind": f"{peak_kind} burst bf16 (MEASURED_PEAKS.json)",
+                    "frac_of_sustained": (achieved / peak_sus) if achieved and peak_sus else None}
     engine = {"achieved": gemm_flops / (gemm_ms / 1000.0) / 1e12 if gemm_ms else None, "unit": "TFLOP/s",
               "ms_per_step": gemm_ms, "share_of_step": gemm_ms / sum(per_step.values()) if per_step else None}
     mel_ms = per_step.get("log_mel")

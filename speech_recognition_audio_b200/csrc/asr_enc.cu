@@ -241,6 +241,7 @@ struct asr_enc {
   float *c1w = nullptr, *c1b = nullptr, *c2b = nullptr, *c3b = nullptr;
   GemmB c2, c3, cout;
   bool box2 = false, box3 = false;  // conv GEMMs read A as strided TMA boxes (else cp.async gather)
+  bool phase2 = false;              // conv1 writes parity planes, conv2 reads dense boxes
   float* pe = nullptr;
   int pe_rows = 0;
   std::vector<LayerW> layers;
@@ -468,6 +469,8 @@ asr_status asr_enc_create(const asr_geometry* g, const void* const* weights, int
     const int f1 = (int)conv_len(g->n_mels, 3, 2, 1), f2 = (int)conv_len(f1, 3, 2, 1);
     e->box2 = f2 > 0 && 128 % f2 == 0 && (128 / f2) * 2 <= 256 && f2 * 2 <= 256;
     e->box3 = f3 > 0 && 128 % f3 == 0 && (128 / f3) * 2 <= 256 && f3 * 2 <= 256;
+    const int t1 = (int)conv_len(g->chunk_frames, 3, 2, 1);
+    e->phase2 = e->box2 && t1 % 2 == 0 && f1 % 2 == 0 && f2 == f1 / 2;
     for (int layer = 0; layer < 2; ++layer) {
       // [o][c][kh][kw] -> [o][tap = kw*3+kh][c], channels padded to 64 per tap in box mode
       auto w = next();
@@ -721,7 +724,9 @@ asr_status ensure_maps(asr_enc* e, const Plan& p, char* ws) {
   if (ok && g->stem == ASR_STEM_CONV2D_CHUNKED) {
     const int C = g->conv_ch;
     ok = make_tmap_bf16(&m.c3, ws + p.off_c3, p.T, (size_t)p.F3 * C, (size_t)p.F3 * C, 128);
-    if (ok && e->box2) ok = make_tmap_convbox(&m.cin2, ws + p.off_c1, C, p.F1, p.T1, p.chunks, p.F2, 2, 128 / p.F2, 2);
+    if (ok && e->box2)
+      ok = e->phase2 ? make_tmap_convphase(&m.cin2, ws + p.off_c1, C, p.F1 / 2, p.T1 / 2, 4 * p.chunks, p.F2, 128 / p.F2)
+                     : make_tmap_convbox(&m.cin2, ws + p.off_c1, C, p.F1, p.T1, p.chunks, p.F2, 2, 128 / p.F2, 2);
     if (ok && e->box3) ok = make_tmap_convbox(&m.cin3, ws + p.off_c2, C, p.F2, p.T2, p.chunks, p.F3, 2, 128 / p.F3, 2);
   } else if (ok) {
     ok = make_tmap_convbox(&m.cin2, ws + p.off_melT, g->n_mels, 1, p.F, p.B, 1, 1, 128, 1) &&
@@ -786,11 +791,12 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
     bf16* c1 = reinterpret_cast<bf16*>(ws + p.off_c1);
     bf16* c2 = reinterpret_cast<bf16*>(ws + p.off_c2);
     bf16* c3 = reinterpret_cast<bf16*>(ws + p.off_c3);
-    ASR_K(PC_CONV1, ASR_LAUNCH(e, launch_conv1_chunked(mel, clip_max, p.B, g->n_mels, p.F, g->chunk_frames, e->c1w, e->c1b, C, c1, st)));
+    ASR_K(PC_CONV1, ASR_LAUNCH(e, launch_conv1_chunked(mel, clip_max, p.B, g->n_mels, p.F, g->chunk_frames, e->c1w, e->c1b, C, c1,
+                                                           e->phase2 ? 1 : 0, st)));
     const int CB = (C + 63) / 64;
     if (e->box2) {
       const int TR = 128 / p.F2, tpi = (p.T2 + TR - 1) / TR;
-      ConvBox b2 = {TR, p.F2, p.T2, tpi, p.chunks * tpi, 2, 2, 1, 1, 3, CB};
+      ConvBox b2 = {TR, p.F2, p.T2, tpi, p.chunks * tpi, 2, 2, 1, 1, 3, CB, e->phase2 ? 1 : 0};
       ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, &e->maps.cin2, nullptr, e->c2, (long long)p.chunks * p.T2 * p.F2, c2, C, e->c2b, nullptr, 1, EPI_GELU, st, &e->maps.o_c2, &b2)));
     } else {
       ConvGather cg2 = {c1, p.T1, p.F1, C, p.T2, p.F2, 2, 2, 3, 3, 1, 1};
@@ -798,7 +804,7 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
     }
     if (e->box3) {
       const int TR = 128 / p.F3, tpi = (p.T3 + TR - 1) / TR;
-      ConvBox b3 = {TR, p.F3, p.T3, tpi, p.chunks * tpi, 2, 2, 1, 1, 3, CB};
+      ConvBox b3 = {TR, p.F3, p.T3, tpi, p.chunks * tpi, 2, 2, 1, 1, 3, CB, 0};
       ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, &e->maps.cin3, nullptr, e->c3, (long long)p.chunks * p.T3 * p.F3, c3, C, e->c3b, nullptr, 1, EPI_GELU, st, &e->maps.o_c3, &b3)));
     } else {
       ConvGather cg3 = {c2, p.T2, p.F2, C, p.T3, p.F3, 2, 2, 3, 3, 1, 1};
@@ -811,9 +817,9 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
     bf16* c1 = reinterpret_cast<bf16*>(ws + p.off_c1);
     ASR_K(PC_MISC, ASR_LAUNCH(e, launch_mel_normalize_transpose(mel, clip_max, p.B, g->n_mels, p.F, melT, st)));
     const int tpi1 = (p.F + 127) / 128, tpi2 = (int)((p.Tc + 127) / 128);
-    ConvBox b1 = {128, 1, p.F, tpi1, p.B * tpi1, 1, 1, 1, 0, 1, (g->n_mels + 63) / 64};
+    ConvBox b1 = {128, 1, p.F, tpi1, p.B * tpi1, 1, 1, 1, 0, 1, (g->n_mels + 63) / 64, 0};
     ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, &e->maps.cin2, nullptr, e->c2, (long long)p.B * p.F, c1, d, e->c2b, nullptr, 1, EPI_GELU, st, &e->maps.o_c1, &b1)));
-    ConvBox b2 = {128, 1, (int)p.Tc, tpi2, p.B * tpi2, 2, 1, 1, 0, 1, (d + 63) / 64};
+    ConvBox b2 = {128, 1, (int)p.Tc, tpi2, p.B * tpi2, 2, 1, 1, 0, 1, (d + 63) / 64, 0};
     ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, &e->maps.cin3, nullptr, e->c3, p.T, x, d, e->c3b, e->pe, (int)p.Tc, EPI_GELU | EPI_OUT_F32 | EPI_PE, st, nullptr, &b2)));
   }
   if (float* t = tap(ASR_TAP_STEM)) ASR_LAUNCH(e, cudaMemcpyAsync(t, x, (size_t)p.T * d * 4, cudaMemcpyDeviceToDevice, st));

@@ -11,8 +11,9 @@
 //     of P V (rows past the segment meet zero probabilities);
 //   - S = Q K^T: tcgen05.mma M=128 N=128 K=64 into tensor memory;
 //   - each thread owns one query row: tcgen05.ld of its 128 scores, scale
-//     1/8, mask keys >= L, max, exp2, sum; P (bf16) is written row-major,
-//     swizzled, over the Q and K tiles as the A operand of the next MMA;
+//     1/8, mask keys >= L, max, exp2 (over the 16-key chunks below L), sum;
+//     P (bf16) is written row-major, swizzled, over the Q and K tiles as the
+//     A operand of the next MMA;
 //   - O = P V: tcgen05.mma M=128 N=64 K=128 into S's tensor-memory columns;
 //   48 KB of shared memory and 128 TMEM columns per block: 4 blocks per SM.
 //   - each thread scales its output row by 1 / sum and stores 128 bytes.
@@ -105,9 +106,17 @@ __global__ void __launch_bounds__(AT_THREADS) attention_tc_kernel(const __grid_c
     if (mx == -INFINITY) mx = 0.f;  // only when the wait failed
     float s = 0.f;
 #pragma unroll
-    for (int j = 0; j < 128; ++j) {
-      sv[j] = exp2f(sv[j] - mx);
-      s += sv[j];
+    for (int c = 0; c < 128; c += 16) {
+      if (c < L) {  // uniform: 16-key chunks wholly past the segment stay zero
+#pragma unroll
+        for (int j = c; j < c + 16; ++j) {
+          sv[j] = exp2f(sv[j] - mx);
+          s += sv[j];
+        }
+      } else {
+#pragma unroll
+        for (int j = c; j < c + 16; ++j) sv[j] = 0.f;
+      }
     }
     rsum = s > 0.f ? 1.f / s : 0.f;
     // P overwrites Q and K: every thread has passed bar_s, so the MMA that

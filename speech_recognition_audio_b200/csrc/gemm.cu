@@ -211,6 +211,19 @@ bool make_tmap_out(CUtensorMap* map, const void* ptr, unsigned long long rows, u
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_tmap_convphase(CUtensorMap* map, const void* ptr, int C, int F_h, int T_h, int n_planes, int F_out, int TR) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || !ptr || (reinterpret_cast<uintptr_t>(ptr) & 15) || C % 8 || F_out > 256 || TR > 256 || F_out * TR != 128)
+    return false;
+  cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)F_h, (cuuint64_t)T_h, (cuuint64_t)n_planes};
+  cuuint64_t strides[3] = {(cuuint64_t)C * 2, (cuuint64_t)F_h * C * 2, (cuuint64_t)T_h * F_h * C * 2};
+  cuuint32_t box[4] = {64, (cuuint32_t)F_out, (cuuint32_t)TR, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_weight_maps(GemmB& w) {
   for (int i = 0; i < kGemmSlots; ++i)
     if (!make_tmap_bf16(&w.map[i], w.ptr, w.N, w.K, w.K, kSlotRows[i])) return false;

@@ -54,12 +54,18 @@ struct ConvGather {
 // t-rows x all F_out columns of one image; for each tap and 64-channel block
 // one 4-D box {64, F_out * sf, TR * st, 1} with element strides {1, sf, st, 1}
 // lands the 128 x 64 A tile (zero fill outside the image = the padding).
+//
+// Phase mode (phase = 1, strides 2 along T and F): the activation is stored
+// as its four parity planes [n_img][t % 2][f % 2][T_in / 2][F_in / 2][C], so
+// the input rows a tap reads for consecutive outputs are consecutive in
+// one plane and each box is dense ({64, F_out, TR, 1}, no element strides).
 struct ConvBox {
   int TR, F_out, T_out;   // output rows per tile, output geometry
   int tiles_per_img;      // ceil(T_out / TR)
   int n_sub;              // n_img * tiles_per_img 128-row sub-tiles
   int st, sf, pt, pf;     // strides and padding along T and F
   int kf, CB;             // taps along F, 64-channel blocks per tap
+  int phase;              // 1 = parity-plane input (see above)
 };
 
 struct GemmParams {
@@ -194,8 +200,16 @@ __device__ __forceinline__ void convbox_coords(const GemmParams& p, int u, int k
   const int cbk = kb - tap * c.CB;
   const int dt = tap / c.kf, df = tap - dt * c.kf;
   c0 = cbk * 64;
-  f0 = df - c.pf;
-  t0 = tb * c.TR * c.st + dt - c.pt;
+  if (c.phase) {
+    // input index 2 o + d - p lies in plane (d - p) & 1 at o + ((d - p) >> 1)
+    const int at = dt - c.pt, af = df - c.pf;
+    f0 = af >> 1;
+    t0 = tb * c.TR + (at >> 1);
+    img = img * 4 + (at & 1) * 2 + (af & 1);
+  } else {
+    f0 = df - c.pf;
+    t0 = tb * c.TR * c.st + dt - c.pt;
+  }
   if (u >= c.n_sub) t0 = 1 << 20;  // entirely outside: zero tile
 }
 

@@ -43,10 +43,12 @@ cudaError_t launch_mel_normalize_transpose(const float* raw, const unsigned int*
                                            int n_frames, bf16* out, cudaStream_t st);
 
 // Conv2D 1 -> C, k3 s2 p1, + bias + GELU over each chunk of chunk_frames
-// frames of the (normalised on the fly) log-mel.  Output [chunks, T1, F1, C].
+// frames of the (normalised on the fly) log-mel.  Output [chunks, T1, F1, C],
+// or with phase != 0 (T1, F1 even) the parity planes
+// [chunks][t % 2][f % 2][T1 / 2][F1 / 2][C] read by the phase-mode conv2.
 cudaError_t launch_conv1_chunked(const float* mel_raw, const unsigned int* clip_max, int batch, int n_mels,
                                  int n_frames, int chunk_frames, const float* w /*[C][9] (kh,kw)*/,
-                                 const float* b, int C, bf16* out, cudaStream_t st);
+                                 const float* b, int C, bf16* out, int phase, cudaStream_t st);
 
 cudaError_t launch_layer_norm(const float* x, const float* g, const float* b, long long M, int D, float eps,
                               void* y, bool out_f32, cudaStream_t st);
@@ -78,6 +80,9 @@ bool make_weight_maps(GemmB& w);
 // 4-D strided-box map over a conv activation [n_img, T_in, F_in, C] (see ConvBox).
 bool make_tmap_convbox(CUtensorMap* map, const void* ptr, int C, int F_in, int T_in, int n_img, int F_out, int sf,
                        int TR, int st);
+// 4-D dense-box map over a parity-plane activation [n_planes][T_h][F_h][C]
+// (ConvBox phase mode): box {64, F_out, TR, 1}.
+bool make_tmap_convphase(CUtensorMap* map, const void* ptr, int C, int F_h, int T_h, int n_planes, int F_out, int TR);
 // Picks the tile for an M x N problem on num_sms SMs: a positive width is a
 // one-SM 128 x bn tile, a negative one a CTA-pair 256 x |bn| tile.
 int gemm_pick_bn(int M, int N, int num_sms, bool gather);

@@ -16,56 +16,84 @@
 namespace asr {
 
 // ------------------------------------------------------------ LayerNorm
-// One warp per row, the row held in registers (V float4 per lane, D = 128 V);
-// two-pass mean / variance with warp-shuffle reductions.
+// One warp per row, V float4 per lane (D = 128 V).  The statistics take one
+// pass over the row in shifted form: with K = x[row][0],
+//   mean = K + S1 / D,  var = S2 / D - (S1 / D)^2,
+//   S1 = sum (x - K),   S2 = sum (x - K)^2,
+// which keeps the cancellation at the scale of the row's spread (|x - K|
+// is a few standard deviations), not of its mean.  The second pass re-reads
+// the row (L1 / L2 hits) to normalise and store, so no thread holds a whole
+// row and every row of a 6240 x 1280 residual stream is in flight at once
+// (one wave of warps instead of two).
+// Read-only 16-byte load that the compiler may not merge with another load
+// of the same address (the second pass must re-read, not keep the row).
+__device__ __forceinline__ float4 ldg_f4_nomerge(const float4* p) {
+  float4 v;
+  asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(p));
+  return v;
+}
+
 template <int V, bool OUT_F32>
-__global__ void __launch_bounds__(256) layer_norm_kernel(const float* __restrict__ x, const float* __restrict__ g,
-                                                         const float* __restrict__ b, long long M, float eps,
-                                                         void* __restrict__ y) {
+__global__ void __launch_bounds__(256, 6) layer_norm_kernel(const float* __restrict__ x, const float* __restrict__ g,
+                                                            const float* __restrict__ b, long long M, float eps,
+                                                            void* __restrict__ y) {
   pdl_wait();
   pdl_trigger();
   const long long row = blockIdx.x * 8LL + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= M) return;
   constexpr int D = V * 128;
+  constexpr int U = V % 2 == 0 ? 2 : 1;  // 16-byte loads in flight per lane
+  // (at most 6 blocks of 256 threads per SM fit 42 registers per thread:
+  // 48 row-warps per SM, 7104 rows in flight on 148 SMs)
   const float4* xr = reinterpret_cast<const float4*>(x + row * D);
-  float4 v[V];
-  float s = 0.f;
+  const float K = __ldg(x + row * D);
+  float s1 = 0.f, s2 = 0.f;
+#pragma unroll 1
+  for (int i0 = 0; i0 < V; i0 += U) {
+    float4 v[U];
 #pragma unroll
-  for (int i = 0; i < V; ++i) {
-    v[i] = xr[lane + 32 * i];
-    s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
+    for (int u = 0; u < U; ++u) v[u] = ldg_f4_nomerge(xr + lane + 32 * (i0 + u));
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const float a = v[u].x - K, bb = v[u].y - K, c = v[u].z - K, d = v[u].w - K;
+      s1 += (a + bb) + (c + d);
+      s2 += (a * a + bb * bb) + (c * c + d * d);
+    }
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  const float mean = s * (1.0f / D);
-  float ss = 0.f;
-#pragma unroll
-  for (int i = 0; i < V; ++i) {
-    const float a = v[i].x - mean, bb = v[i].y - mean, c = v[i].z - mean, d = v[i].w - mean;
-    ss += (a * a + bb * bb) + (c * c + d * d);
+  for (int o = 16; o > 0; o >>= 1) {
+    s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+    s2 += __shfl_xor_sync(0xffffffffu, s2, o);
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  const float rstd = rsqrtf(ss * (1.0f / D) + eps);
+  const float m1 = s1 * (1.0f / D);
+  const float mean = K + m1;
+  const float var = fmaxf(s2 * (1.0f / D) - m1 * m1, 0.0f);
+  const float rstd = rsqrtf(var + eps);
   const float4* g4 = reinterpret_cast<const float4*>(g);
   const float4* b4 = reinterpret_cast<const float4*>(b);
+#pragma unroll 1
+  for (int i0 = 0; i0 < V; i0 += U) {
+    float4 v[U];
 #pragma unroll
-  for (int i = 0; i < V; ++i) {
-    const int c4 = lane + 32 * i;
-    const float4 gg = __ldg(g4 + c4), bv = __ldg(b4 + c4);
-    const float o0 = (v[i].x - mean) * rstd * gg.x + bv.x;
-    const float o1 = (v[i].y - mean) * rstd * gg.y + bv.y;
-    const float o2 = (v[i].z - mean) * rstd * gg.z + bv.z;
-    const float o3 = (v[i].w - mean) * rstd * gg.w + bv.w;
-    if (OUT_F32) {
-      reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + row * D)[c4] = make_float4(o0, o1, o2, o3);
-    } else {
-      __nv_bfloat162 p0 = __floats2bfloat162_rn(o0, o1), p1 = __floats2bfloat162_rn(o2, o3);
-      uint2 u;
-      u.x = *reinterpret_cast<uint32_t*>(&p0);
-      u.y = *reinterpret_cast<uint32_t*>(&p1);
-      reinterpret_cast<uint2*>(reinterpret_cast<bf16*>(y) + row * D)[c4] = u;
+    for (int u = 0; u < U; ++u) v[u] = ldg_f4_nomerge(xr + lane + 32 * (i0 + u));
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c4 = lane + 32 * (i0 + u);
+      const float4 gg = __ldg(g4 + c4), bv = __ldg(b4 + c4);
+      const float o0 = (v[u].x - mean) * rstd * gg.x + bv.x;
+      const float o1 = (v[u].y - mean) * rstd * gg.y + bv.y;
+      const float o2 = (v[u].z - mean) * rstd * gg.z + bv.z;
+      const float o3 = (v[u].w - mean) * rstd * gg.w + bv.w;
+      if (OUT_F32) {
+        reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + row * D)[c4] = make_float4(o0, o1, o2, o3);
+      } else {
+        __nv_bfloat162 p0 = __floats2bfloat162_rn(o0, o1), p1 = __floats2bfloat162_rn(o2, o3);
+        uint2 w2;
+        w2.x = *reinterpret_cast<uint32_t*>(&p0);
+        w2.y = *reinterpret_cast<uint32_t*>(&p1);
+        reinterpret_cast<uint2*>(reinterpret_cast<bf16*>(y) + row * D)[c4] = w2;
+      }
     }
   }
 }

@@ -13,8 +13,11 @@
 // operand; the next unit's patch is fetched into registers while the current
 // one is computed (two patch buffers, one barrier per unit).  The log-mel
 // normalisation (clamp at clip max - 8, then (x + 4) / 4) is applied while
-// staging.  Output layout: [chunk, T1, F1, C] bf16 (channels innermost), the
-// input layout of the implicit-GEMM conv2; each thread stores 16 bytes.
+// staging.  Output layout: [chunk, T1, F1, C] bf16 (channels innermost), or
+// (phase mode, T1 and F1 even) the chunk's four parity planes
+// [chunk][t % 2][f % 2][T1 / 2][F1 / 2][C], so that every tap of the stride-2
+// conv2 reads consecutive rows of one plane as a dense TMA box; each thread
+// stores 16 bytes.
 #include "kernels.h"
 
 namespace asr {
@@ -36,6 +39,7 @@ struct Conv1Args {
   const float* w;
   const float* bias;
   int C;
+  int phase;  // 1 = parity-plane output
   bf16* out;
 };
 
@@ -117,6 +121,7 @@ __global__ void __launch_bounds__(C1_THREADS, 1) conv1_chunked_kernel(const Conv
     const int npos = min(C1_TB, a.T1 - t0) * a.F1;
     const float2* buf = patch[cur];
     bf16* obase = a.out + ((long long)chunk * a.T1 + t0) * a.F1 * a.C + cg * 8;
+    bf16* pbase = a.out + (long long)chunk * a.T1 * a.F1 * a.C + cg * 8;  // the chunk's four parity planes
     if (lane_p < PL) {
       for (int pos = lane_p; pos < npos; pos += PL) {
         const int tl = pos / a.F1, fo = pos - tl * a.F1;
@@ -136,7 +141,15 @@ __global__ void __launch_bounds__(C1_THREADS, 1) conv1_chunked_kernel(const Conv
           const float2 g = gelu_erf2(acc[i]);
           r[i] = __floats2bfloat162_rn(g.x, g.y);
         }
-        *reinterpret_cast<uint4*>(obase + (long long)pos * a.C) = *reinterpret_cast<uint4*>(r);
+        bf16* dst;
+        if (a.phase) {
+          const int t = t0 + tl;
+          const int plane = (t & 1) * 2 + (fo & 1);
+          dst = pbase + (((long long)plane * (a.T1 >> 1) + (t >> 1)) * (a.F1 >> 1) + (fo >> 1)) * a.C;
+        } else {
+          dst = obase + (long long)pos * a.C;
+        }
+        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<uint4*>(r);
       }
     }
     if (un < a.n_units) conv1_stage(a, un, pf, patch[cur ^ 1]);
@@ -147,7 +160,7 @@ __global__ void __launch_bounds__(C1_THREADS, 1) conv1_chunked_kernel(const Conv
 
 cudaError_t launch_conv1_chunked(const float* mel_raw, const unsigned int* clip_max, int batch, int n_mels,
                                  int n_frames, int chunk_frames, const float* w, const float* b, int C, bf16* out,
-                                 cudaStream_t st) {
+                                 int phase, cudaStream_t st) {
   if (n_mels > C1_MAXM || C % 8 || C / 8 > C1_THREADS) return cudaErrorInvalidValue;
   Conv1Args a;
   a.mel_raw = mel_raw;
@@ -164,6 +177,8 @@ cudaError_t launch_conv1_chunked(const float* mel_raw, const unsigned int* clip_
   a.bias = b;
   a.C = C;
   a.out = out;
+  a.phase = phase ? 1 : 0;
+  if (a.phase && (a.T1 % 2 || a.F1 % 2)) return cudaErrorInvalidValue;
   const int groups = C / 8;
   const int threads = groups * (C1_THREADS / groups);
   // every patch value of a unit has an owner: threads * C1_PF >= rows * pitch
