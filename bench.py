@@ -173,7 +173,7 @@ def job_throughput(audio_s_per_rank, world, ms_max):
 
 # ------------------------------------------------------- committed ncu summaries
 GEMM_SOURCES = ["speech_recognition_audio_b200/csrc/gemm.cuh", "speech_recognition_audio_b200/csrc/gemm2.cuh",
-                "speech_recognition_audio_b200/csrc/common.cuh"]
+                "speech_recognition_audio_b200/csrc/common.cuh", "speech_recognition_audio_b200/csrc/gemm.cu"]
 
 
 def gemm_source_hash():

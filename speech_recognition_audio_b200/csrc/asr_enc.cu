@@ -44,6 +44,7 @@ struct ActMaps {
   int batch = 0;
   unsigned taps = 0;
   CUtensorMap h, att, ff, c3, p1, p2, gu;
+  CUtensorMap a1;          // conv1 taps [positions, 16] (box 128 x 64: columns 16..63 read as zeros)
   CUtensorMap cin2, cin3;  // conv-box A maps of the two stem GEMMs
   CUtensorMap qkv;         // 128-row boxes of the QKV buffer (tcgen05 attention)
   // Store maps of the GEMM outputs (32 x 32 boxes): residual stream, QKV,
@@ -55,11 +56,8 @@ struct Plan {
   int64_t n = 0, Tc = 0, T = 0;
   int B = 0, F = 0, nwin_clip = 0, nwin = 0, max_win = 0, chunks = 0;
   int T1 = 0, F1 = 0, T2 = 0, F2 = 0, T3 = 0, F3 = 0;
-  size_t off_clipmax = 0, off_cu = 0, off_mel = 0, off_c1 = 0, off_c2 = 0, off_c3 = 0, off_melT = 0, off_x = 0,
-         off_h = 0, off_qkv = 0, off_att = 0, off_ff = 0, off_p1 = 0, off_p2 = 0, off_gu = 0, off_pcm = 0, off_out = 0,
-         off_skflags = 0;
-  int sk_regions = 0;      // stream-K flag regions (one per eligible GEMM launch of a forward)
-  size_t sk_flag_ints = 0; // ints per region
+  size_t off_clipmax = 0, off_cu = 0, off_mel = 0, off_a1 = 0, off_c1 = 0, off_c2 = 0, off_c3 = 0, off_melT = 0, off_x = 0,
+         off_h = 0, off_qkv = 0, off_att = 0, off_ff = 0, off_p1 = 0, off_p2 = 0, off_gu = 0, off_pcm = 0, off_out = 0;
   size_t off_tap[ASR_TAP_COUNT] = {0, 0, 0, 0, 0};
   size_t tap_bytes[ASR_TAP_COUNT] = {0, 0, 0, 0, 0};
   size_t total = 0;
@@ -238,8 +236,8 @@ struct asr_enc {
   size_t slab_bytes = 0, slab_used = 0;
   std::string err;
   // stem
-  float *c1w = nullptr, *c1b = nullptr, *c2b = nullptr, *c3b = nullptr;
-  GemmB c2, c3, cout;
+  float *c1b = nullptr, *c2b = nullptr, *c3b = nullptr;
+  GemmB c1, c2, c3, cout;  // conv stem GEMMs (conv1: [C][16] taps kh*3+kw, 9..15 zero)
   bool box2 = false, box3 = false;  // conv GEMMs read A as strided TMA boxes (else cp.async gather)
   bool phase2 = false;              // conv1 writes parity planes, conv2 reads dense boxes
   float* pe = nullptr;
@@ -261,9 +259,6 @@ struct asr_enc {
   size_t ev_used = 0;
   std::vector<std::pair<int, size_t>> prof_recs;  // (stage class, index of the first of two events)
   int launches = 0;
-  int sk_next = 0;  // next stream-K flag region of the running forward
-  char* sk_ws = nullptr;         // workspace of the running forward (stream-K scratch)
-  const Plan* sk_plan = nullptr;
 };
 
 namespace {
@@ -462,8 +457,11 @@ asr_status asr_enc_create(const asr_geometry* g, const void* const* weights, int
   cudaStreamSynchronize(st);
   if (g->stem == ASR_STEM_CONV2D_CHUNKED) {
     const int f3 = (int)conv_len(conv_len(conv_len(g->n_mels, 3, 2, 1), 3, 2, 1), 3, 2, 1);
-    auto w1 = next();
-    e->c1w = up_f32(w1);  // [C][kh*3+kw]
+    auto w1 = next();  // [C][kh*3+kw] -> rows of 16
+    std::vector<float> r1((size_t)C * 16, 0.0f);
+    for (int o = 0; o < C; ++o)
+      for (int k = 0; k < 9; ++k) r1[(size_t)o * 16 + k] = w1[(size_t)o * 9 + k];
+    if (!gemm_w(e->c1, r1, C, 16)) return bad(fail(e, ASR_E_CUDA, "conv1 weight upload / TMA map failed"));
     e->c1b = up_f32(next());
     // Conv-box mode needs F_out | 128 (a 128-row tile = whole output rows).
     const int f1 = (int)conv_len(g->n_mels, 3, 2, 1), f2 = (int)conv_len(f1, 3, 2, 1);
@@ -607,6 +605,7 @@ bool make_plan(const asr_enc* e, int64_t n, int B, Plan* p) {
     p->T2 = (int)conv_len(p->T1, 3, 2, 1); p->F2 = (int)conv_len(p->F1, 3, 2, 1);
     p->T3 = (int)conv_len(p->T2, 3, 2, 1); p->F3 = (int)conv_len(p->F2, 3, 2, 1);
     const size_t C = g->conv_ch;
+    p->off_a1 = take((size_t)p->chunks * p->T1 * p->F1 * 16 * 2);
     p->off_c1 = take((size_t)p->chunks * p->T1 * p->F1 * C * 2);
     p->off_c2 = take((size_t)p->chunks * p->T2 * p->F2 * C * 2);
     p->off_c3 = take((size_t)p->T * p->F3 * C * 2);
@@ -624,11 +623,6 @@ bool make_plan(const asr_enc* e, int64_t n, int B, Plan* p) {
     p->off_p2 = take((size_t)p->T * g->proj2_out * 2);
   }
   if (g->adapter_hidden) p->off_gu = take((size_t)p->T * g->adapter_hidden * 2);
-  // Stream-K flags of the residual GEMMs: per launch one flag per (CTA,
-  // epilogue warp).
-  p->sk_regions = 2 * g->n_layers + 2;
-  p->sk_flag_ints = (size_t)e->num_sms * 8;
-  p->off_skflags = take((size_t)p->sk_regions * p->sk_flag_ints * 4);
   p->tap_bytes[ASR_TAP_MEL] = (size_t)B * g->n_mels * p->F * 4;
   p->tap_bytes[ASR_TAP_STEM] = p->tap_bytes[ASR_TAP_LAYER0] = p->tap_bytes[ASR_TAP_ENCODER] = (size_t)p->T * d * 4;
   p->tap_bytes[ASR_TAP_HEAD] = g->proj2_out ? (size_t)p->T * g->proj2_out * 4 : 0;
@@ -654,11 +648,6 @@ asr_status gemm(asr_enc* e, const CUtensorMap* amap, const ConvGather* cg, const
   if (cg) p.g = *cg;
   p.status = e->status;
   p.limit_ns = kWaitLimitNs;
-  p.n_fast = cg != nullptr || box != nullptr;
-  if (epi == EPI_RESID && e->sk_ws && e->sk_next < e->sk_plan->sk_regions) {
-    p.sk_flags = reinterpret_cast<int*>(e->sk_ws + e->sk_plan->off_skflags) + (size_t)e->sk_next * e->sk_plan->sk_flag_ints;
-    ++e->sk_next;
-  }
   int bn;
   if (box) {
     p.conv_box = 1;
@@ -723,7 +712,8 @@ asr_status ensure_maps(asr_enc* e, const Plan& p, char* ws) {
             make_tmap_bf16(&m.ff, ws + p.off_ff, p.T, g->d_ffn, g->d_ffn, 128);
   if (ok && g->stem == ASR_STEM_CONV2D_CHUNKED) {
     const int C = g->conv_ch;
-    ok = make_tmap_bf16(&m.c3, ws + p.off_c3, p.T, (size_t)p.F3 * C, (size_t)p.F3 * C, 128);
+    ok = make_tmap_bf16(&m.c3, ws + p.off_c3, p.T, (size_t)p.F3 * C, (size_t)p.F3 * C, 128) &&
+         make_tmap_bf16(&m.a1, ws + p.off_a1, (size_t)p.chunks * p.T1 * p.F1, 16, 16, 128);
     if (ok && e->box2)
       ok = e->phase2 ? make_tmap_convphase(&m.cin2, ws + p.off_c1, C, p.F1 / 2, p.T1 / 2, 4 * p.chunks, p.F2, 128 / p.F2)
                      : make_tmap_convbox(&m.cin2, ws + p.off_c1, C, p.F1, p.T1, p.chunks, p.F2, 2, 128 / p.F2, 2);
@@ -742,7 +732,8 @@ asr_status ensure_maps(asr_enc* e, const Plan& p, char* ws) {
          make_tmap_out(&m.o_qkv, ws + p.off_qkv, p.T, 3 * d, 3 * d, false) &&
          make_tmap_out(&m.o_ff, ws + p.off_ff, p.T, g->d_ffn, g->d_ffn, false);
   if (ok && g->stem == ASR_STEM_CONV2D_CHUNKED)
-    ok = make_tmap_out(&m.o_c2, ws + p.off_c2, (unsigned long long)p.chunks * p.T2 * p.F2, g->conv_ch, g->conv_ch, false) &&
+    ok = make_tmap_out(&m.o_c1, ws + p.off_c1, (unsigned long long)p.chunks * p.T1 * p.F1, g->conv_ch, g->conv_ch, false) &&
+         make_tmap_out(&m.o_c2, ws + p.off_c2, (unsigned long long)p.chunks * p.T2 * p.F2, g->conv_ch, g->conv_ch, false) &&
          make_tmap_out(&m.o_c3, ws + p.off_c3, (unsigned long long)p.chunks * p.T3 * p.F3, g->conv_ch, g->conv_ch, false);
   else if (ok)
     ok = make_tmap_out(&m.o_c1, ws + p.off_c1, (unsigned long long)p.B * p.F, d, d, false);
@@ -775,11 +766,7 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
   e->launches = 0;
   e->ev_used = 0;
   e->prof_recs.clear();
-  e->sk_ws = ws;
-  e->sk_plan = &p;
-  e->sk_next = 0;
   ASR_LAUNCH(e, cudaMemsetAsync(e->status, 0, 4, st));
-  ASR_LAUNCH(e, cudaMemsetAsync(ws + p.off_skflags, 0, (size_t)p.sk_regions * p.sk_flag_ints * 4, st));
   ASR_LAUNCH(e, cudaMemsetAsync(clip_max, 0, (size_t)p.B * 4, st));
   const int w = g->window_tokens ? g->window_tokens : (int)p.Tc;
   ASR_K(PC_MISC, ASR_LAUNCH(e, launch_fill_windows(cu, p.B, (int)p.Tc, w, p.nwin_clip, st)));
@@ -791,8 +778,11 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
     bf16* c1 = reinterpret_cast<bf16*>(ws + p.off_c1);
     bf16* c2 = reinterpret_cast<bf16*>(ws + p.off_c2);
     bf16* c3 = reinterpret_cast<bf16*>(ws + p.off_c3);
-    ASR_K(PC_CONV1, ASR_LAUNCH(e, launch_conv1_chunked(mel, clip_max, p.B, g->n_mels, p.F, g->chunk_frames, e->c1w, e->c1b, C, c1,
-                                                           e->phase2 ? 1 : 0, st)));
+    bf16* a1 = reinterpret_cast<bf16*>(ws + p.off_a1);
+    ASR_K(PC_CONV1, ASR_LAUNCH(e, launch_conv1_im2col(mel, clip_max, p.B, g->n_mels, p.F, g->chunk_frames,
+                                                      e->phase2 ? 1 : 0, a1, st)));
+    ASR_K(PC_CONV1, ASR_TRY(gemm(e, &e->maps.a1, nullptr, e->c1, (long long)p.chunks * p.T1 * p.F1, c1, C, e->c1b,
+                                 nullptr, 1, EPI_GELU, st, &e->maps.o_c1)));
     const int CB = (C + 63) / 64;
     if (e->box2) {
       const int TR = 128 / p.F2, tpi = (p.T2 + TR - 1) / TR;

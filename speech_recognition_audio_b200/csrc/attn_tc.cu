@@ -65,7 +65,6 @@ __global__ void __launch_bounds__(AT_THREADS) attention_tc_kernel(const __grid_c
   pdl_trigger();
 
   const int s0 = cu[seg], L = cu[seg + 1] - s0;
-  const long long ld = 3LL * H * 64;
   bool ok = true;
   if (tid == 0) {
     mbar_arrive_expect_tx(bar_qk, 3 * 16384);

@@ -273,6 +273,11 @@ int gemm_pick_bn_conv(int n_sub, int N, int num_sms) {
 cudaError_t launch_gemm(const CUtensorMap* a_map, const GemmB& w, GemmParams p, int epi, int bn, int num_sms,
                         cudaStream_t st, const CUtensorMap* out_map) {
   p.out_tma = (out_map != nullptr && !(epi & (EPI_PE | EPI_SWIGLU))) ? 1 : 0;
+  // Tile order: the tiles running at once share the larger operand, so it
+  // crosses from DRAM once and is re-read from L2 (and the TMA latency the
+  // stage ring has to cover is the L2's, not the DRAM's).  A (M x K) is the
+  // larger when M > N; convolutions always re-read their gathered A.
+  p.n_fast = (p.conv_box || a_map == nullptr || p.M > w.N) ? 1 : 0;
   if (bn < 0) {
     // CTA-pair kernel: 256 x |bn| tiles, each CTA stages |bn|/2 rows of B.
     const int w2 = -bn;

@@ -42,13 +42,13 @@ cudaError_t launch_mel_normalize(const float* raw, const unsigned int* clip_max,
 cudaError_t launch_mel_normalize_transpose(const float* raw, const unsigned int* clip_max, int batch, int n_mels,
                                            int n_frames, bf16* out, cudaStream_t st);
 
-// Conv2D 1 -> C, k3 s2 p1, + bias + GELU over each chunk of chunk_frames
-// frames of the (normalised on the fly) log-mel.  Output [chunks, T1, F1, C],
-// or with phase != 0 (T1, F1 even) the parity planes
-// [chunks][t % 2][f % 2][T1 / 2][F1 / 2][C] read by the phase-mode conv2.
-cudaError_t launch_conv1_chunked(const float* mel_raw, const unsigned int* clip_max, int batch, int n_mels,
-                                 int n_frames, int chunk_frames, const float* w /*[C][9] (kh,kw)*/,
-                                 const float* b, int C, bf16* out, int phase, cudaStream_t st);
+// A operand of the first Conv2D (1 -> C, k3 s2 p1) as a GEMM: per output
+// position of each chunk of chunk_frames frames, its 9 normalised log-mel
+// taps (kh * 3 + kw) as bf16 in a row of 16 (taps 9..15 zero).  Rows
+// [chunks][T1][F1], or with phase != 0 (T1, F1 even) the parity planes
+// [chunks][t % 2][f % 2][T1 / 2][F1 / 2] read by the phase-mode conv2.
+cudaError_t launch_conv1_im2col(const float* mel_raw, const unsigned int* clip_max, int batch, int n_mels,
+                                int n_frames, int chunk_frames, int phase, bf16* a, cudaStream_t st);
 
 cudaError_t launch_layer_norm(const float* x, const float* g, const float* b, long long M, int D, float eps,
                               void* y, bool out_f32, cudaStream_t st);
