@@ -193,6 +193,11 @@ bool make_tmap_qkv(CUtensorMap* map, const void* qkv, long long T, int H) {
 cudaError_t launch_attention_tc(const CUtensorMap& tm_qkv, const bf16* qkv, const int* cu, int n_seg, int H, bf16* out,
                                 int* status, unsigned long long limit_ns, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM);
+  // Ask for the whole shared-memory carveout: without it the driver picked a
+  // 164 KB configuration (3 blocks per SM, 2.7 waves for 1200 blocks).
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   return launch_pdl(attention_tc_kernel, dim3(n_seg, H), dim3(AT_THREADS), AT_SMEM, st, tm_qkv, qkv, cu, H, out, status,
                     limit_ns);
