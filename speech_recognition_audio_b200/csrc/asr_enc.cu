@@ -786,7 +786,7 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
     const int CB = (C + 63) / 64;
     if (e->box2) {
       const int TR = 128 / p.F2, tpi = (p.T2 + TR - 1) / TR;
-      ConvBox b2 = {TR, p.F2, p.T2, tpi, p.chunks * tpi, 2, 2, 1, 1, 3, CB, e->phase2 ? 1 : 0};
+      ConvBox b2 = {TR, p.F2, p.T2, tpi, p.chunks * tpi, 2, 2, 1, 1, 3, CB, e->phase2 ? 1 : 0, (C - 64 * (CB - 1) + 15) / 16};
       ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, &e->maps.cin2, nullptr, e->c2, (long long)p.chunks * p.T2 * p.F2, c2, C, e->c2b, nullptr, 1, EPI_GELU, st, &e->maps.o_c2, &b2)));
     } else {
       ConvGather cg2 = {c1, p.T1, p.F1, C, p.T2, p.F2, 2, 2, 3, 3, 1, 1};
@@ -794,7 +794,7 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
     }
     if (e->box3) {
       const int TR = 128 / p.F3, tpi = (p.T3 + TR - 1) / TR;
-      ConvBox b3 = {TR, p.F3, p.T3, tpi, p.chunks * tpi, 2, 2, 1, 1, 3, CB, 0};
+      ConvBox b3 = {TR, p.F3, p.T3, tpi, p.chunks * tpi, 2, 2, 1, 1, 3, CB, 0, (C - 64 * (CB - 1) + 15) / 16};
       ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, &e->maps.cin3, nullptr, e->c3, (long long)p.chunks * p.T3 * p.F3, c3, C, e->c3b, nullptr, 1, EPI_GELU, st, &e->maps.o_c3, &b3)));
     } else {
       ConvGather cg3 = {c2, p.T2, p.F2, C, p.T3, p.F3, 2, 2, 3, 3, 1, 1};
@@ -807,9 +807,10 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
     bf16* c1 = reinterpret_cast<bf16*>(ws + p.off_c1);
     ASR_K(PC_MISC, ASR_LAUNCH(e, launch_mel_normalize_transpose(mel, clip_max, p.B, g->n_mels, p.F, melT, st)));
     const int tpi1 = (p.F + 127) / 128, tpi2 = (int)((p.Tc + 127) / 128);
-    ConvBox b1 = {128, 1, p.F, tpi1, p.B * tpi1, 1, 1, 1, 0, 1, (g->n_mels + 63) / 64, 0};
+    const int CB1 = (g->n_mels + 63) / 64, CBd = (d + 63) / 64;
+    ConvBox b1 = {128, 1, p.F, tpi1, p.B * tpi1, 1, 1, 1, 0, 1, CB1, 0, (g->n_mels - 64 * (CB1 - 1) + 15) / 16};
     ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, &e->maps.cin2, nullptr, e->c2, (long long)p.B * p.F, c1, d, e->c2b, nullptr, 1, EPI_GELU, st, &e->maps.o_c1, &b1)));
-    ConvBox b2 = {128, 1, (int)p.Tc, tpi2, p.B * tpi2, 2, 1, 1, 0, 1, (d + 63) / 64, 0};
+    ConvBox b2 = {128, 1, (int)p.Tc, tpi2, p.B * tpi2, 2, 1, 1, 0, 1, CBd, 0, (d - 64 * (CBd - 1) + 15) / 16};
     ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, &e->maps.cin3, nullptr, e->c3, p.T, x, d, e->c3b, e->pe, (int)p.Tc, EPI_GELU | EPI_OUT_F32 | EPI_PE, st, nullptr, &b2)));
   }
   if (float* t = tap(ASR_TAP_STEM)) ASR_LAUNCH(e, cudaMemcpyAsync(t, x, (size_t)p.T * d * 4, cudaMemcpyDeviceToDevice, st));

@@ -66,6 +66,7 @@ struct ConvBox {
   int st, sf, pt, pf;     // strides and padding along T and F
   int kf, CB;             // taps along F, 64-channel blocks per tap
   int phase;              // 1 = parity-plane input (see above)
+  int k16_last;           // K=16 MMA steps holding channels in a tap's last 64-channel block
 };
 
 struct GemmParams {
@@ -236,6 +237,16 @@ __device__ __forceinline__ void tile_coords(const GemmParams& p, int t, int& mb,
 }
 
 static constexpr unsigned long long kDrainLimitNs = 200ull * 1000 * 1000;
+
+// K=16 MMA steps of k-block kb that hold non-zero operands: 4, except in a
+// k-block past the end of K (plain mode) or in the last channel block of a
+// tap when the channel count is not a multiple of 64 (conv-box mode), whose
+// zero-padded tail the MMA can skip.
+__device__ __forceinline__ int k16_steps(const GemmParams& p, int kb) {
+  if (p.conv_box) return (kb % p.cb.CB == p.cb.CB - 1) ? p.cb.k16_last : 4;
+  const int rem = p.K - kb * 64;
+  return rem >= 64 ? 4 : (rem + 15) / 16;
+}
 
 template <int BN_, int STAGES_, bool GATHER_>
 struct GemmShape {
@@ -594,9 +605,10 @@ __global__ void __launch_bounds__(GemmShape<BN, STAGES, GATHER>::THREADS, 1)
           tc_fence_after();
           const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + s * S::A_BYTES));
           const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + s * S::B_BYTES));
+          const int ks = k16_steps(p, kb);
 #pragma unroll
           for (int k = 0; k < S::BK / 16; ++k)
-            tc_mma_bf16(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+            if (k < ks) tc_mma_bf16(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
           tc_commit(&empty[s]);
           ++it;
         }

@@ -229,9 +229,10 @@ __global__ void __launch_bounds__(Gemm2Shape<BN, STAGES>::THREADS, 1)
           tc_fence_after();
           const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + s * S::A_BYTES));
           const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + s * S::B_BYTES));
+          const int ks = k16_steps(p, kb);
 #pragma unroll
           for (int k = 0; k < S::BK / 16; ++k)
-            tc_mma_bf16_pair(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+            if (k < ks) tc_mma_bf16_pair(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
           tc_commit_pair_mc(&empty[s], 0x3);
           ++it;
         }
