@@ -43,19 +43,23 @@ __global__ void __launch_bounds__(256, 6) layer_norm_kernel(const float* __restr
   const int lane = threadIdx.x & 31;
   if (row >= M) return;
   constexpr int D = V * 128;
-  constexpr int U = V % 2 == 0 ? 2 : 1;  // 16-byte loads in flight per lane
+  // 16-byte loads in flight per lane: the statistics pass keeps up to 5 in
+  // flight (the row arrives in two round trips), the normalising pass 2
+  // (its re-reads hit L1, and it also holds gamma and beta).
+  constexpr int U1 = V % 5 == 0 ? 5 : (V % 4 == 0 ? 4 : (V % 3 == 0 ? 3 : (V % 2 == 0 ? 2 : 1)));
+  constexpr int U = V % 2 == 0 ? 2 : 1;
   // (at most 6 blocks of 256 threads per SM fit 42 registers per thread:
   // 48 row-warps per SM, 7104 rows in flight on 148 SMs)
   const float4* xr = reinterpret_cast<const float4*>(x + row * D);
   const float K = __ldg(x + row * D);
   float s1 = 0.f, s2 = 0.f;
 #pragma unroll 1
-  for (int i0 = 0; i0 < V; i0 += U) {
-    float4 v[U];
+  for (int i0 = 0; i0 < V; i0 += U1) {
+    float4 v[U1];
 #pragma unroll
-    for (int u = 0; u < U; ++u) v[u] = ldg_f4_nomerge(xr + lane + 32 * (i0 + u));
+    for (int u = 0; u < U1; ++u) v[u] = ldg_f4_nomerge(xr + lane + 32 * (i0 + u));
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
+    for (int u = 0; u < U1; ++u) {
       const float a = v[u].x - K, bb = v[u].y - K, c = v[u].z - K, d = v[u].w - K;
       s1 += (a + bb) + (c + d);
       s2 += (a * a + bb * bb) + (c * c + d * d);
