@@ -78,7 +78,7 @@ cudaError_t run_gather(int epi, const CUtensorMap& b, const CUtensorMap& o, cons
 
 template <int BN, int EPI>
 cudaError_t run2(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& p, int grid, cudaStream_t st) {
-  using S = Gemm2Shape<BN, (BN >= 192 ? 6 : 8)>;
+  using S = Gemm2Shape<BN, (BN >= 192 ? 6 : 8), gemm2_epi_warps<EPI>()>;
   auto k = gemm_bf16_tc2_kernel<BN, S::STAGES, EPI>;
   cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_BYTES);
   if (err != cudaSuccess) return err;

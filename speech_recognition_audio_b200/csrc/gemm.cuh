@@ -269,12 +269,16 @@ struct GemmShape {
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
+// Epilogue warps: four per TMEM lane quarter share the accumulator columns
+// with 8 warps as two column parts (32-column groups part, part + 2, ...),
+// with 16 warps as four (part, part + 4, ...); `cstride` = 32 x parts.
+//
 // Residual epilogues read 128 x BN fp32 values per tile; issuing L2
 // prefetches for the tile's rows before waiting for the accumulator moves that
 // DRAM latency under the tile's MMAs.  Each thread prefetches the 128-byte
 // lines of its own row in the 32-column groups its warp will handle.
 __device__ __forceinline__ void epilogue_prefetch_l2(const GemmParams& p, int t, int half, int q, int lane, int BN,
-                                                     int BM, int rank_rows) {
+                                                     int BM, int rank_rows, int cstride = 64) {
   int mb, nb;
   tile_coords(p, t, mb, nb);
   const int m0 = mb * BM + rank_rows;
@@ -282,7 +286,7 @@ __device__ __forceinline__ void epilogue_prefetch_l2(const GemmParams& p, int t,
   const int row = m0 + 32 * q + lane;
   if (row >= p.M) return;
   const float* base = reinterpret_cast<const float*>(p.out) + (long long)row * p.ldo + n0;
-  for (int c = half * 32; c < BN && n0 + c < p.N; c += 64)
+  for (int c = half * 32; c < BN && n0 + c < p.N; c += cstride)
     asm volatile("prefetch.global.L2 [%0];" ::"l"(base + c) : "memory");
 }
 
@@ -310,11 +314,13 @@ __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_
 
 // Bias of the tile's columns for one epilogue warp, loaded before the
 // accumulator is ready: lane l holds bias[n0 + c_j + l] for the warp's
-// column groups c_j = 32 half + 64 j (the epilogue broadcasts it by shuffle).
-__device__ __forceinline__ void load_bias(const GemmParams& p, int n0, int BN, int half, int lane, float* breg) {
+// column groups c_j = 32 half + cstride j (the epilogue broadcasts it by
+// shuffle).
+__device__ __forceinline__ void load_bias(const GemmParams& p, int n0, int BN, int half, int lane, float* breg,
+                                          int cstride = 64) {
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const int c = half * 32 + 64 * j;
+    const int c = half * 32 + cstride * j;
     const int n = n0 + c + lane;
     breg[j] = (p.bias && c < BN && c + lane < BN && n < p.N) ? __ldg(p.bias + n) : 0.0f;
   }
@@ -343,7 +349,7 @@ __device__ __forceinline__ void load_bias(const GemmParams& p, int n0, int BN, i
 template <int EPI>
 __device__ __forceinline__ void epilogue_warp(const GemmParams& p, const CUtensorMap* tm_out, uint32_t tb, int row0,
                                               int mlimit, int n0, int BN, int half, int lane, uint8_t* wbuf,
-                                              const float* breg, int kind = PIECE_FULL) {
+                                              const float* breg, int kind = PIECE_FULL, int cstride = 64) {
   constexpr bool F32 = (EPI & (EPI_OUT_F32 | EPI_RESID)) != 0;
   constexpr bool SWI = (EPI & EPI_SWIGLU) != 0;
   constexpr bool TMA_OK = (EPI & (EPI_PE | EPI_SWIGLU)) == 0;
@@ -353,7 +359,7 @@ __device__ __forceinline__ void epilogue_warp(const GemmParams& p, const CUtenso
   const bool rows_ok = TMA_OK && p.out_tma && (mlimit - row0 >= 32 || mlimit >= p.M);
   int j = 0;
 #pragma unroll 1
-  for (int c = half * 32; c < BN; c += 64, ++j) {
+  for (int c = half * 32; c < BN; c += cstride, ++j) {
     const int n = n0 + c;
     if (n >= p.N) break;                                  // warp-uniform
     const int w = (BN - c < 32 || p.N - n < 32) ? 16 : 32;  // valid columns in this group (N % 16 == 0)

@@ -90,7 +90,9 @@ __device__ __forceinline__ void tc_commit_pair_mc(uint64_t* bar, uint16_t mask) 
       : "memory");
 }
 
-template <int BN_, int STAGES_>
+// EPIW_: epilogue warps, 8 or 16 (16 only for bf16 outputs, whose 32 x 32
+// staging box takes 2 KB, so the staging area stays 32 KB).
+template <int BN_, int STAGES_, int EPIW_ = 8>
 struct Gemm2Shape {
   static constexpr int BM = 256, BN = BN_, BK = 64, STAGES = STAGES_;
   static constexpr int A_BYTES = 128 * BK * 2;        // this CTA's half of A
@@ -99,20 +101,31 @@ struct Gemm2Shape {
   static constexpr int TX_BYTES = 2 * STAGE_BYTES;    // both CTAs, counted on the leader
   static constexpr int ACC_COLS = (BN + 31) / 32 * 32;
   static constexpr int TMEM_COLS = 2 * ACC_COLS <= 64 ? 64 : 2 * ACC_COLS <= 128 ? 128 : 2 * ACC_COLS <= 256 ? 256 : 512;
-  static constexpr int EPI_WARPS = 8;
+  static constexpr int EPI_WARPS = EPIW_;
   static constexpr int THREADS = 32 * (2 + EPI_WARPS);
-  static constexpr int EPI_BUF_BYTES = EPI_WARPS * 4096;
+  static constexpr int WBUF = EPI_WARPS == 16 ? 2048 : 4096;  // staging bytes per epilogue warp
+  static constexpr int CSTRIDE = 32 * (EPI_WARPS / 4);       // column stride of a warp's groups
+  static constexpr int EPI_BUF_BYTES = EPI_WARPS * WBUF;
   static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5) + 16;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BUF_BYTES + BAR_BYTES;
   static_assert(BN % 16 == 0 && (BN / 2) % 8 == 0 && BN >= 64 && BN <= 256, "UMMA N for M=256; B halves of 8-row atoms");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+  static_assert(EPI_WARPS == 8 || EPI_WARPS == 16, "two or four column parts per lane quarter");
 };
 
+// Epilogue warps of an instance: 16 for the bias + GELU bf16 epilogue (the
+// GELU's arithmetic is the epilogue's cost; with 8 warps it is latency-bound,
+// and it is the whole cost of the K = 16 conv1 GEMM), 8 otherwise.
+template <int EPI>
+constexpr int gemm2_epi_warps() {
+  return EPI == EPI_GELU ? 16 : 8;
+}
+
 template <int BN, int STAGES, int EPI>
-__global__ void __launch_bounds__(Gemm2Shape<BN, STAGES>::THREADS, 1)
+__global__ void __launch_bounds__(Gemm2Shape<BN, STAGES, gemm2_epi_warps<EPI>()>::THREADS, 1)
     gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
-  using S = Gemm2Shape<BN, STAGES>;
+  using S = Gemm2Shape<BN, STAGES, gemm2_epi_warps<EPI>()>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -245,7 +258,7 @@ __global__ void __launch_bounds__(Gemm2Shape<BN, STAGES>::THREADS, 1)
   } else {
     // epilogue: this CTA's 128 rows of the 256-row tile
     const int q = warp & 3;
-    const int half = (warp - 2) / 4;
+    const int half = (warp - 2) / 4;  // column part (0..EPI_WARPS/4 - 1)
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
     const int rank_rows = static_cast<int>(rank) * 128;
     const int ew = warp - 2;
@@ -259,9 +272,10 @@ __global__ void __launch_bounds__(Gemm2Shape<BN, STAGES>::THREADS, 1)
       int mb, nb;
       tile_coords(p, t, mb, nb);
       const int n0 = nb * BN;
-      if ((EPI & EPI_RESID) && kind != PIECE_PARTIAL) epilogue_prefetch_l2(p, t, half, q, lane, BN, S::BM, rank_rows);
+      if ((EPI & EPI_RESID) && kind != PIECE_PARTIAL)
+        epilogue_prefetch_l2(p, t, half, q, lane, BN, S::BM, rank_rows, S::CSTRIDE);
       float breg[4];
-      load_bias(p, n0, BN, half, lane, breg);
+      load_bias(p, n0, BN, half, lane, breg, S::CSTRIDE);
       if (!mbar_wait_bounded(&tfull[a], aph, p.limit_ns, p.status, DEV_TIMEOUT_EPILOGUE)) break;
       tc_fence_after();
       int r_first, r_last;
@@ -280,7 +294,8 @@ __global__ void __launch_bounds__(Gemm2Shape<BN, STAGES>::THREADS, 1)
         have = __shfl_sync(0xffffffffu, have, 0);
       }
       if (have)
-        epilogue_warp<EPI>(p, &tmOut, tb, r_first + 32 * q, r_last, n0, BN, half, lane, sEpi + ew * 4096, breg, kind);
+        epilogue_warp<EPI>(p, &tmOut, tb, r_first + 32 * q, r_last, n0, BN, half, lane, sEpi + ew * S::WBUF, breg, kind,
+                           S::CSTRIDE);
       tc_fence_before();
       __syncwarp();
       if (kind == PIECE_PARTIAL && lane == 0) {
