@@ -5,12 +5,12 @@
 // windowed, block-diagonal attention; the whisper-small variant attends over
 // the whole clip): segments are given by cumulative offsets and only a
 // segment's own keys are visited, so the block-diagonal structure costs
-// nothing.  QK^T and PV run on bf16 tensor cores (mma.sync m16n8k16, fp32
-// accumulate), softmax in fp32 registers, keys past the segment end masked
-// to -inf, scale 1/sqrt(64).  Segments of at most 128 tokens use one block
-// per (segment, head) with a one-pass softmax; longer ones a flash-style
-// kernel with one block per (64-query tile, segment, head) and an online
-// softmax over 64-key tiles.
+// nothing.  Segments of at most 128 tokens run on the tcgen05 kernel of
+// attn_tc.cu.  Longer ones (the whisper-small variant's 1500-frame clips) run
+// here: QK^T and PV on bf16 tensor cores (mma.sync m16n8k16, fp32
+// accumulate), a flash-style kernel with one block per (64-query tile,
+// segment, head) and an online softmax over 64-key tiles in fp32 registers,
+// keys past the segment end masked to -inf, scale 1/sqrt(64).
 #include "kernels.h"
 
 namespace asr {
@@ -25,6 +25,7 @@ namespace asr {
 // the row (L1 / L2 hits) to normalise and store, so no thread holds a whole
 // row and every row of a 6240 x 1280 residual stream is in flight at once
 // (one wave of warps instead of two).
+
 // Read-only 16-byte load that the compiler may not merge with another load
 // of the same address (the second pass must re-read, not keep the row).
 __device__ __forceinline__ float4 ldg_f4_nomerge(const float4* p) {
@@ -301,140 +302,9 @@ __global__ void __launch_bounds__(128) attention_kernel(const bf16* __restrict__
   }
 }
 
-// Attention for segments of at most 128 tokens (the 104-token windows): one
-// CTA per (segment, head) holds the whole window's Q, K and V in shared
-// memory; each of 8 warps owns 16 query rows and computes its full score row
-// block (keys rounded up to 16, masked past the segment end), a one-pass
-// softmax in registers and P V.  Warps whose rows all lie past the segment
-// end do nothing.
-template <int NK>  // key blocks of 16 (segment length <= 16 * NK <= 128)
-__global__ void __launch_bounds__(256) attention_window_kernel(const bf16* __restrict__ qkv, const int* __restrict__ cu,
-                                                               int H, bf16* __restrict__ out) {
-  extern __shared__ __align__(16) uint8_t smem_att[];
-  bf16* Qs = reinterpret_cast<bf16*>(smem_att);
-  bf16* Ks = Qs + 128 * LDS;
-  bf16* Vs = Ks + 128 * LDS;
-  pdl_wait();
-  pdl_trigger();
-  const int seg = blockIdx.x, h = blockIdx.y;
-  const int s0 = cu[seg], L = cu[seg + 1] - s0;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const long long ld = 3LL * H * HD;
-  const bf16* base = qkv + (long long)s0 * ld;
-  const int rows = 16 * NK;  // rows staged (queries and keys)
-  for (int c = tid; c < rows * 8; c += 256) {
-    const int r = c >> 3, k = (c & 7) * 8;
-    const bool v = r < L;
-    const bf16* src = base + (long long)(v ? r : 0) * ld + k;
-    cp_async_16_zfill(Qs + r * LDS + k, src + h * HD, v);
-    cp_async_16_zfill(Ks + r * LDS + k, src + (H + h) * HD, v);
-    cp_async_16_zfill(Vs + r * LDS + k, src + (2 * H + h) * HD, v);
-  }
-  cp_async_commit();
-  cp_async_wait<0>();
-  __syncthreads();
-  if (warp * 16 >= L || warp >= NK) return;
-
-  const int g = lane >> 2, t4 = lane & 3;
-  uint32_t qf[4][4];
-#pragma unroll
-  for (int ks = 0; ks < 4; ++ks) ldsm_x4(qf[ks], Qs + (warp * 16 + (lane & 15)) * LDS + ks * 16 + (lane >> 4) * 8);
-  float s[2 * NK][4];
-#pragma unroll
-  for (int i = 0; i < 2 * NK; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
-#pragma unroll
-  for (int ks = 0; ks < 4; ++ks) {
-#pragma unroll
-    for (int p = 0; p < NK; ++p) {
-      uint32_t kb[4];
-      ldsm_x4(kb, Ks + (16 * p + (lane & 7) + (lane >> 4) * 8) * LDS + ks * 16 + ((lane >> 3) & 1) * 8);
-      mma_bf16_16816(s[2 * p], qf[ks], kb[0], kb[1]);
-      mma_bf16_16816(s[2 * p + 1], qf[ks], kb[2], kb[3]);
-    }
-  }
-  const float sl2 = 0.125f * 1.4426950408889634f;  // (1/sqrt(64)) * log2(e)
-  float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-  for (int nt = 0; nt < 2 * NK; ++nt) {
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int key = nt * 8 + 2 * t4 + (e & 1);
-      const float v = key < L ? s[nt][e] * sl2 : -INFINITY;
-      s[nt][e] = v;
-      mx[e >> 1] = fmaxf(mx[e >> 1], v);
-    }
-  }
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
-    mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
-  }
-  float sum[2] = {0.f, 0.f};
-  uint32_t pf[NK][4];
-#pragma unroll
-  for (int nt = 0; nt < 2 * NK; ++nt) {
-    const float p0 = exp2f(s[nt][0] - mx[0]), p1 = exp2f(s[nt][1] - mx[0]);
-    const float p2 = exp2f(s[nt][2] - mx[1]), p3 = exp2f(s[nt][3] - mx[1]);
-    sum[0] += p0 + p1;
-    sum[1] += p2 + p3;
-    pf[nt >> 1][(nt & 1) * 2 + 0] = pack_bf16(p0, p1);
-    pf[nt >> 1][(nt & 1) * 2 + 1] = pack_bf16(p2, p3);
-  }
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    sum[r] += __shfl_xor_sync(0xffffffffu, sum[r], 1);
-    sum[r] += __shfl_xor_sync(0xffffffffu, sum[r], 2);
-  }
-  float o[8][4];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-#pragma unroll
-  for (int ks = 0; ks < NK; ++ks) {
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      uint32_t vb[4];
-      ldsm_x4_t(vb, Vs + (16 * ks + (lane & 7) + ((lane >> 3) & 1) * 8) * LDS + 16 * p + (lane >> 4) * 8);
-      mma_bf16_16816(o[2 * p], pf[ks], vb[0], vb[1]);
-      mma_bf16_16816(o[2 * p + 1], pf[ks], vb[2], vb[3]);
-    }
-  }
-  const float inv0 = 1.f / sum[0], inv1 = 1.f / sum[1];
-  const int r0 = warp * 16 + g, r1 = r0 + 8;
-  bf16* ob = out + (long long)s0 * (H * HD) + h * HD;
-#pragma unroll
-  for (int nt = 0; nt < 8; ++nt) {
-    const int col = nt * 8 + 2 * t4;
-    if (r0 < L)
-      *reinterpret_cast<uint32_t*>(ob + (long long)r0 * (H * HD) + col) = pack_bf16(o[nt][0] * inv0, o[nt][1] * inv0);
-    if (r1 < L)
-      *reinterpret_cast<uint32_t*>(ob + (long long)r1 * (H * HD) + col) = pack_bf16(o[nt][2] * inv1, o[nt][3] * inv1);
-  }
-}
-
-template <int NK>
-static cudaError_t launch_window(const bf16* qkv, const int* cu, int n_seg, int H, bf16* out, cudaStream_t st) {
-  const int smem = 3 * 128 * LDS * 2;
-  auto k = attention_window_kernel<NK>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(k, dim3(n_seg, H), dim3(256), smem, st, qkv, cu, H, out);
-}
-
 cudaError_t launch_attention(const bf16* qkv, const int* cu, int n_seg, int max_seg, int H, bf16* out,
                              cudaStream_t st) {
   if (n_seg <= 0 || max_seg <= 0 || H <= 0) return cudaErrorInvalidValue;
-  if (max_seg <= 128) {
-    switch ((max_seg + 15) / 16) {
-      case 1: return launch_window<1>(qkv, cu, n_seg, H, out, st);
-      case 2: return launch_window<2>(qkv, cu, n_seg, H, out, st);
-      case 3: return launch_window<3>(qkv, cu, n_seg, H, out, st);
-      case 4: return launch_window<4>(qkv, cu, n_seg, H, out, st);
-      case 5: return launch_window<5>(qkv, cu, n_seg, H, out, st);
-      case 6: return launch_window<6>(qkv, cu, n_seg, H, out, st);
-      case 7: return launch_window<7>(qkv, cu, n_seg, H, out, st);
-      default: return launch_window<8>(qkv, cu, n_seg, H, out, st);
-    }
-  }
   dim3 grid((max_seg + BQ - 1) / BQ, n_seg, H);
   return launch_pdl(attention_kernel, grid, dim3(128), 0, st, qkv, cu, H, out);
 }
