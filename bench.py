@@ -264,7 +264,8 @@ def run_reference(args, w, g, rank):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "audio-s/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": bench_config(w, T),
+            "config": dict(bench_config(w, T), l2="n/a (host CPU)",
+                           timing="host wall clock (perf_counter) per sample, mean of steps"),
             "cpu_baseline": {"value": value, "unit": "audio-s/s", "cores": blas_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "audio-s/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
