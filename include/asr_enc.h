@@ -129,8 +129,12 @@ asr_status asr_enc_windows(const asr_geometry* g, int64_t n_samples, int batch, 
  * `alloc` (cudaMalloc when alloc is NULL), and build the weight TMA
  * descriptors.  `weights` points to asr_enc_weight_count(g) device pointers.
  * Work is enqueued on `stream` and completed before return.
- * Limits: n_fft 400, hop 160, head_dim 64, d_model % 64 == 0, d_ffn % 64 == 0,
- * conv_ch % 8 == 0; otherwise ASR_E_UNSUPPORTED. */
+ * Limits: n_mels 1..128, n_fft 400, hop 160, head_dim 64 with n_heads * 64 ==
+ * d_model, d_model a multiple of 128 and <= 2048, d_ffn a multiple of 64,
+ * conv_ch a multiple of 8 and <= 512, proj1_out % 64 == 0, proj2_out % 128 == 0
+ * and <= 2048, adapter widths multiples of 16; otherwise ASR_E_UNSUPPORTED.
+ * Every CUDA runtime call made here is checked: a failed copy or launch
+ * returns ASR_E_CUDA naming the call, and nothing is left allocated. */
 asr_status asr_enc_create(const asr_geometry* g, const void* const* weights, int n_weights,
                           asr_alloc_fn alloc, asr_free_fn free_fn, void* alloc_ctx, void* stream,
                           asr_enc** out);

@@ -25,7 +25,9 @@ extern "C" {
  * log10(max(., 1e-10)), clamp at (clip max - 8), then (x + 4) / 4.
  *  pcm   device float32 [batch, n_samples]; n_samples % 160 == 0, > 200.
  *  mel   device float32 [batch, n_mels, n_samples/160] (normalised).
- *  ws    device scratch of >= asr_op_log_mel_ws_size(batch) bytes.
+ *  ws    device scratch of >= asr_op_log_mel_ws_size(batch) bytes, 256-byte
+ *        aligned: the per-clip maxima and the FFT / filterbank tables, which
+ *        every call rebuilds on the device (one small kernel, no host copy).
  * n_mels: 1..128. */
 size_t asr_op_log_mel_ws_size(int batch);
 asr_status asr_op_log_mel(const float* pcm, int64_t n_samples, int batch, int n_mels, float* mel,
@@ -36,18 +38,21 @@ asr_status asr_op_log_mel(const float* pcm, int64_t n_samples, int batch, int n_
  * cudaMalloc -- for example a plugin inside a host application that owns all
  * device memory, or a real-time audio thread, where an allocation would
  * stall on an implicit device synchronisation.  It computes exactly what
- * asr_op_log_mel computes, but its scratch (the per-clip maxima and the
- * FFT / filterbank tables, about 25 KB) is a fixed array inside the library:
- * every GPU that loads the library holds it until the process exits.
+ * asr_op_log_mel computes (same kernels, same tables, bit-identical output),
+ * but its scratch (the per-clip maxima and the FFT / filterbank tables,
+ * about 31 KB) is a fixed array inside the library: every GPU that loads the
+ * library holds it until the process exits.
  *  pcm, n_samples, n_mels, mel: as for asr_op_log_mel.
  *  batch: 1 .. 4096 clips; larger batches return ASR_E_UNSUPPORTED.
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  Each call uploads the tables and clears the
- * maxima on `stream` (a plain copy and memset, no allocation).  All calls
- * share the one array and it keeps the last call's contents, so calls whose
- * GPU work overlaps (different streams, not ordered) race and must not be
- * issued. */
+ * before any stream capture.  Each call then enqueues on `stream` a kernel
+ * that rebuilds the tables for its n_mels, a memset that clears the maxima,
+ * and the log-mel kernels; nothing is copied from the host and the calling
+ * thread does not wait for the device.  All calls share the one array and it
+ * keeps the last call's contents, so calls whose GPU work overlaps
+ * (different streams, not ordered) race and must not be issued; calls on
+ * one stream are ordered and may use different n_mels. */
 asr_status asr_op_log_mel_noalloc(const float* pcm, int64_t n_samples, int batch, int n_mels, float* mel,
                                   void* stream);
 
@@ -56,7 +61,8 @@ asr_status asr_op_log_mel_noalloc(const float* pcm, int64_t n_samples, int batch
  *  x     device bf16 [M, K] row-major;  w  device bf16 [N, K] row-major.
  *  bias  device float32 [N] or NULL.
  *  epi   ASR_EPI_BF16       y bf16 [M, N] = acc + bias
- *        ASR_EPI_BF16_GELU  y bf16 [M, N] = GELU(acc + bias)      (exact erf)
+ *        ASR_EPI_BF16_GELU  y bf16 [M, N] = GELU(acc + bias), the GELU of asr_op_gelu
+ *                           (erf from Abramowitz & Stegun 7.1.28, |error| <= 3e-7)
  *        ASR_EPI_F32_RESID  y f32  [M, N] += acc + bias           (in place)
  *        ASR_EPI_F32        y f32  [M, N] = acc + bias
  *        ASR_EPI_SWIGLU     y bf16 [M, N/2]: W rows interleaved in blocks of
@@ -81,7 +87,8 @@ asr_status asr_op_linear(const void* x, const void* w, const float* bias, int64_
 
 /* LayerNorm over the last axis: y = (x - mean) / sqrt(var + eps) * g + b,
  * x device float32 [M, D], g/b device float32 [D], y device bf16 [M, D]
- * (out_f32 == 0) or float32 (out_f32 != 0).  D % 4 == 0, D <= 4096. */
+ * (out_f32 == 0) or float32 (out_f32 != 0).  D must be a multiple of 128 and
+ * at most 2048 (ASR_E_INVAL otherwise); M >= 1. */
 asr_status asr_op_layer_norm(const float* x, const float* g, const float* b, int64_t M, int D,
                              float eps, void* y, int out_f32, void* stream);
 

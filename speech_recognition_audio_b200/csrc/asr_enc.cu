@@ -171,42 +171,6 @@ int64_t tokens_per_clip(const asr_geometry* g, int64_t n) {
   return conv_len(conv_len(frames, 3, 1, 1), 3, 2, 1);
 }
 
-// Host tables in double precision, rounded once to float.
-void build_mel_tables(int n_mels, MelTables* t) {
-  memset(t, 0, sizeof *t);
-  const double PI = 3.14159265358979323846;
-  for (int j = 0; j < 200; ++j) t->w200[j] = make_float2((float)cos(2 * PI * j / 200), (float)-sin(2 * PI * j / 200));
-  for (int k = 0; k <= 200; ++k) t->w400[k] = make_float2((float)cos(2 * PI * k / 400), (float)-sin(2 * PI * k / 400));
-  for (int n = 0; n < 400; ++n) t->hann[n] = (float)(0.5 - 0.5 * cos(2 * PI * n / 400));
-  // Slaney mel scale: 3 f / 200 below 1 kHz, 15 + 27 ln(f / 1000) / ln 6.4 above.
-  auto hz2mel = [](double f) { return f < 1000.0 ? 3.0 * f / 200.0 : 15.0 + 27.0 * log(f / 1000.0) / log(6.4); };
-  auto mel2hz = [](double m) { return m < 15.0 ? 200.0 * m / 3.0 : 1000.0 * exp((m - 15.0) * log(6.4) / 27.0); };
-  const double mmax = hz2mel(8000.0);
-  std::vector<double> fpts(n_mels + 2);
-  for (int i = 0; i < n_mels + 2; ++i) fpts[i] = mel2hz(mmax * i / (n_mels + 1));
-  int off = 0;
-  for (int m = 0; m < n_mels; ++m) {
-    const double lo = fpts[m], ce = fpts[m + 1], hi = fpts[m + 2];
-    const double norm = 2.0 / (hi - lo);
-    int first = -1, cnt = 0;
-    for (int k = 0; k <= 200; ++k) {
-      const double f = 40.0 * k;
-      const double w = std::max(0.0, std::min((f - lo) / (ce - lo), (hi - f) / (hi - ce))) * norm;
-      if (w > 0.0) {
-        if (first < 0) first = k;
-        t->fw[off + cnt] = (float)w;
-        ++cnt;
-      } else if (first >= 0) {
-        break;
-      }
-    }
-    t->fstart[m] = first < 0 ? 0 : first;
-    t->fcount[m] = cnt;
-    t->foff[m] = off;
-    off += cnt;
-  }
-}
-
 // Sinusoidal positions [rows, d]: d/2 frequencies exp(-ln(1e4) i / (d/2 - 1)),
 // [sin(p w_i) | cos(p w_i)].
 std::vector<float> build_pe(int rows, int d) {
@@ -288,21 +252,23 @@ void* slab_take(asr_enc* e, size_t bytes) {
   return static_cast<char*>(e->slab) + off;
 }
 
-std::vector<float> fetch(const void* dptr, int64_t n, int dtype) {
-  std::vector<float> out((size_t)n);
+// Copies a weight tensor to the host as float; false if the copy failed.
+bool fetch(const void* dptr, int64_t n, int dtype, std::vector<float>* out, cudaError_t* err) {
+  out->assign((size_t)n, 0.0f);
   if (dtype == ASR_DTYPE_F32) {
-    cudaMemcpy(out.data(), dptr, n * 4, cudaMemcpyDeviceToHost);
-  } else {
-    std::vector<uint16_t> tmp((size_t)n);
-    cudaMemcpy(tmp.data(), dptr, n * 2, cudaMemcpyDeviceToHost);
-    for (int64_t i = 0; i < n; ++i) {
-      uint32_t u = static_cast<uint32_t>(tmp[i]) << 16;
-      float f;
-      memcpy(&f, &u, 4);
-      out[i] = f;
-    }
+    *err = cudaMemcpy(out->data(), dptr, n * 4, cudaMemcpyDeviceToHost);
+    return *err == cudaSuccess;
   }
-  return out;
+  std::vector<uint16_t> tmp((size_t)n);
+  *err = cudaMemcpy(tmp.data(), dptr, n * 2, cudaMemcpyDeviceToHost);
+  if (*err != cudaSuccess) return false;
+  for (int64_t i = 0; i < n; ++i) {
+    uint32_t u = static_cast<uint32_t>(tmp[i]) << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    (*out)[i] = f;
+  }
+  return true;
 }
 
 uint16_t f2bf(float f) {
@@ -411,7 +377,8 @@ asr_status asr_enc_create(const asr_geometry* g, const void* const* weights, int
   if (cudaDeviceGetAttribute(&e->num_sms, cudaDevAttrMultiProcessorCount, e->device) != cudaSuccess)
     return bad(fail(e, ASR_E_CUDA, "cudaDeviceGetAttribute failed"));
   int major = 0;
-  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, e->device);
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, e->device) != cudaSuccess)
+    return bad(fail(e, ASR_E_CUDA, "cudaDeviceGetAttribute failed"));
   if (major != 10) return bad(fail(e, ASR_E_UNSUPPORTED, "this library runs on sm_100 (B200) only; device has sm_%d", major * 10));
 
   const int d = g->d_model, C = g->conv_ch, L = g->n_layers;
@@ -430,38 +397,54 @@ asr_status asr_enc_create(const asr_geometry* g, const void* const* weights, int
   if (!alloc && cudaMalloc(&e->slab, e->slab_bytes) != cudaSuccess) e->slab = nullptr;
   if (!e->slab) return bad(fail(e, ASR_E_NOMEM, "allocation of %zu bytes failed", e->slab_bytes));
 
-  std::vector<void*> host_keep;
+  // The first failing runtime call of the repack is kept and reported.
+  cudaError_t cerr = cudaSuccess;
+  std::string cwhat;
+  auto note = [&](cudaError_t r, const std::string& what) {
+    if (r != cudaSuccess && cerr == cudaSuccess) {
+      cerr = r;
+      cwhat = what;
+    }
+  };
+  auto cuda_fail = [&](const char* what) {
+    if (cerr != cudaSuccess) return bad(fail(e, ASR_E_CUDA, "%s failed: %s", cwhat.c_str(), cudaGetErrorString(cerr)));
+    return bad(fail(e, ASR_E_CUDA, "%s", what));
+  };
   auto up_f32 = [&](const std::vector<float>& v) -> float* {
     float* p = static_cast<float*>(slab_take(e, v.size() * 4));
-    if (p) cudaMemcpy(p, v.data(), v.size() * 4, cudaMemcpyHostToDevice);
+    if (p) note(cudaMemcpy(p, v.data(), v.size() * 4, cudaMemcpyHostToDevice), "cudaMemcpy (fp32 upload)");
     return p;
   };
   auto up_bf16 = [&](const std::vector<float>& v) -> bf16* {
     std::vector<uint16_t> h(v.size());
     for (size_t i = 0; i < v.size(); ++i) h[i] = f2bf(v[i]);
     bf16* p = static_cast<bf16*>(slab_take(e, h.size() * 2));
-    if (p) cudaMemcpy(p, h.data(), h.size() * 2, cudaMemcpyHostToDevice);
+    if (p) note(cudaMemcpy(p, h.data(), h.size() * 2, cudaMemcpyHostToDevice), "cudaMemcpy (bf16 upload)");
     return p;
   };
   int wi = 0;
   auto next = [&]() {
     const WSpec& s = specs[wi];
-    return fetch(weights[wi++], numel(s), g->dtype);
+    std::vector<float> v;
+    cudaError_t r = cudaSuccess;
+    if (!fetch(weights[wi], numel(s), g->dtype, &v, &r)) note(r, "cudaMemcpy of weight " + s.name);
+    ++wi;
+    return v;
   };
   auto gemm_w = [&](GemmB& gb, const std::vector<float>& v, int N, int K) -> bool {
     gb.ptr = up_bf16(v);
     gb.N = N;
     gb.K = K;
-    return gb.ptr && make_weight_maps(gb);
+    return cerr == cudaSuccess && gb.ptr && make_weight_maps(gb);
   };
-  cudaStreamSynchronize(st);
+  note(cudaStreamSynchronize(st), "cudaStreamSynchronize");
   if (g->stem == ASR_STEM_CONV2D_CHUNKED) {
     const int f3 = (int)conv_len(conv_len(conv_len(g->n_mels, 3, 2, 1), 3, 2, 1), 3, 2, 1);
     auto w1 = next();  // [C][kh*3+kw] -> rows of 16
     std::vector<float> r1((size_t)C * 16, 0.0f);
     for (int o = 0; o < C; ++o)
       for (int k = 0; k < 9; ++k) r1[(size_t)o * 16 + k] = w1[(size_t)o * 9 + k];
-    if (!gemm_w(e->c1, r1, C, 16)) return bad(fail(e, ASR_E_CUDA, "conv1 weight upload / TMA map failed"));
+    if (!gemm_w(e->c1, r1, C, 16)) return cuda_fail("conv1 weight upload / TMA map failed");
     e->c1b = up_f32(next());
     // Conv-box mode needs F_out | 128 (a 128-row tile = whole output rows).
     const int f1 = (int)conv_len(g->n_mels, 3, 2, 1), f2 = (int)conv_len(f1, 3, 2, 1);
@@ -480,7 +463,7 @@ asr_status asr_enc_create(const asr_geometry* g, const void* const* weights, int
           for (int kh = 0; kh < 3; ++kh)
             for (int kw = 0; kw < 3; ++kw)
               r[(size_t)o * 9 * cp + (kw * 3 + kh) * cp + c] = w[(((size_t)o * C + c) * 3 + kh) * 3 + kw];
-      if (!gemm_w(layer == 0 ? e->c2 : e->c3, r, C, 9 * cp)) return bad(fail(e, ASR_E_CUDA, "conv weight upload / TMA map failed"));
+      if (!gemm_w(layer == 0 ? e->c2 : e->c3, r, C, 9 * cp)) return cuda_fail("conv weight upload / TMA map failed");
       auto b = next();
       (layer == 0 ? e->c2b : e->c3b) = up_f32(b);
     }
@@ -489,7 +472,7 @@ asr_status asr_enc_create(const asr_geometry* g, const void* const* weights, int
     for (int o = 0; o < d; ++o)
       for (int c = 0; c < C; ++c)
         for (int f = 0; f < f3; ++f) r[(size_t)o * C * f3 + f * C + c] = wo[(size_t)o * C * f3 + c * f3 + f];
-    if (!gemm_w(e->cout, r, d, C * f3)) return bad(fail(e, ASR_E_CUDA, "conv_out upload / TMA map failed"));
+    if (!gemm_w(e->cout, r, d, C * f3)) return cuda_fail("conv_out upload / TMA map failed");
   } else {
     // Conv1D stem: always conv-box mode (F_out = 1, 128 output frames per tile).
     e->box2 = e->box3 = true;
@@ -500,14 +483,14 @@ asr_status asr_enc_create(const asr_geometry* g, const void* const* weights, int
     for (int o = 0; o < d; ++o)
       for (int c = 0; c < M; ++c)
         for (int k = 0; k < 3; ++k) r1[(size_t)o * 3 * mp + k * mp + c] = w1[((size_t)o * M + c) * 3 + k];
-    if (!gemm_w(e->c2, r1, d, 3 * mp)) return bad(fail(e, ASR_E_CUDA, "conv1 upload failed"));
+    if (!gemm_w(e->c2, r1, d, 3 * mp)) return cuda_fail("conv1 upload failed");
     e->c2b = up_f32(next());
     auto w2 = next();
     std::vector<float> r2((size_t)d * 3 * dp, 0.0f);
     for (int o = 0; o < d; ++o)
       for (int c = 0; c < d; ++c)
         for (int k = 0; k < 3; ++k) r2[(size_t)o * 3 * dp + k * dp + c] = w2[((size_t)o * d + c) * 3 + k];
-    if (!gemm_w(e->c3, r2, d, 3 * dp)) return bad(fail(e, ASR_E_CUDA, "conv2 upload failed"));
+    if (!gemm_w(e->c3, r2, d, 3 * dp)) return cuda_fail("conv2 upload failed");
     e->c3b = up_f32(next());
   }
   e->layers.resize(L);
@@ -522,23 +505,23 @@ asr_status asr_enc_create(const asr_geometry* g, const void* const* weights, int
       wqkv.insert(wqkv.end(), w.begin(), w.end());
       bqkv.insert(bqkv.end(), b.begin(), b.end());
     }
-    if (!gemm_w(lw.qkv, wqkv, 3 * d, d)) return bad(fail(e, ASR_E_CUDA, "qkv upload failed"));
+    if (!gemm_w(lw.qkv, wqkv, 3 * d, d)) return cuda_fail("qkv upload failed");
     lw.bqkv = up_f32(bqkv);
-    if (!gemm_w(lw.o, next(), d, d)) return bad(fail(e, ASR_E_CUDA, "o upload failed"));
+    if (!gemm_w(lw.o, next(), d, d)) return cuda_fail("o upload failed");
     lw.bo = up_f32(next());
     lw.ln2g = up_f32(next());
     lw.ln2b = up_f32(next());
-    if (!gemm_w(lw.fc1, next(), g->d_ffn, d)) return bad(fail(e, ASR_E_CUDA, "fc1 upload failed"));
+    if (!gemm_w(lw.fc1, next(), g->d_ffn, d)) return cuda_fail("fc1 upload failed");
     lw.b1 = up_f32(next());
-    if (!gemm_w(lw.fc2, next(), d, g->d_ffn)) return bad(fail(e, ASR_E_CUDA, "fc2 upload failed"));
+    if (!gemm_w(lw.fc2, next(), d, g->d_ffn)) return cuda_fail("fc2 upload failed");
     lw.b2 = up_f32(next());
   }
   e->lnpg = up_f32(next());
   e->lnpb = up_f32(next());
   if (g->proj1_out) {
-    if (!gemm_w(e->p1, next(), g->proj1_out, d)) return bad(fail(e, ASR_E_CUDA, "proj1 upload failed"));
+    if (!gemm_w(e->p1, next(), g->proj1_out, d)) return cuda_fail("proj1 upload failed");
     e->bp1 = up_f32(next());
-    if (!gemm_w(e->p2, next(), g->proj2_out, g->proj1_out)) return bad(fail(e, ASR_E_CUDA, "proj2 upload failed"));
+    if (!gemm_w(e->p2, next(), g->proj2_out, g->proj1_out)) return cuda_fail("proj2 upload failed");
     e->bp2 = up_f32(next());
   }
   if (g->adapter_hidden) {
@@ -551,22 +534,20 @@ asr_status asr_enc_create(const asr_geometry* g, const void* const* weights, int
         memcpy(&r[((size_t)32 * j + i) * K], &wg[((size_t)16 * j + i) * K], K * 4);
         memcpy(&r[((size_t)32 * j + 16 + i) * K], &wu[((size_t)16 * j + i) * K], K * 4);
       }
-    if (!gemm_w(e->gu, r, 2 * H, K)) return bad(fail(e, ASR_E_CUDA, "adapter gate/up upload failed"));
-    if (!gemm_w(e->down, next(), g->adapter_out, H)) return bad(fail(e, ASR_E_CUDA, "adapter down upload failed"));
+    if (!gemm_w(e->gu, r, 2 * H, K)) return cuda_fail("adapter gate/up upload failed");
+    if (!gemm_w(e->down, next(), g->adapter_out, H)) return cuda_fail("adapter down upload failed");
   }
   e->pe_rows = pe_rows;
   e->pe = up_f32(build_pe(pe_rows, d));
-  MelTables mt;
-  build_mel_tables(g->n_mels, &mt);
   e->mel_tab = static_cast<MelTables*>(slab_take(e, sizeof(MelTables)));
   if (!e->mel_tab) return bad(fail(e, ASR_E_NOMEM, "slab exhausted"));
-  cudaMemcpy(e->mel_tab, &mt, sizeof mt, cudaMemcpyHostToDevice);
+  note(launch_mel_tables(g->n_mels, e->mel_tab, st), "mel table kernel launch");
   e->status = static_cast<int*>(slab_take(e, 256));
   if (!e->status) return bad(fail(e, ASR_E_NOMEM, "slab exhausted"));
-  cudaMemset(e->status, 0, 256);
-  cudaError_t r = cudaDeviceSynchronize();
-  if (r != cudaSuccess) return bad(fail(e, ASR_E_CUDA, "weight repack failed: %s", cudaGetErrorString(r)));
-  if (!e->pe || !e->c2.ptr) return bad(fail(e, ASR_E_NOMEM, "slab exhausted"));
+  note(cudaMemsetAsync(e->status, 0, 256, st), "cudaMemsetAsync (status word)");
+  note(cudaStreamSynchronize(st), "cudaStreamSynchronize");
+  if (cerr != cudaSuccess) return cuda_fail("weight repack");
+  if (!e->pe || !e->c2.ptr || !e->c2b || !e->c3b || !e->lnpg || !e->lnpb) return bad(fail(e, ASR_E_NOMEM, "slab exhausted"));
   *out = e;
   return ASR_OK;
 }
@@ -984,33 +965,22 @@ int asr_enc_last_launches(const asr_enc* e) { return e ? e->launches : -1; }
 
 // ==================================================================== ops
 
-size_t asr_op_log_mel_ws_size(int batch) { return batch > 0 ? align_up((size_t)batch * 4, 256) : 0; }
+// Log-mel workspace: [clip maxima (256-byte aligned)][tables].
+static size_t log_mel_max_bytes(int batch) { return align_up((size_t)batch * 4, 256); }
+size_t asr_op_log_mel_ws_size(int batch) {
+  return batch > 0 ? log_mel_max_bytes(batch) + align_up(sizeof(MelTables), 256) : 0;
+}
 
 asr_status asr_op_log_mel(const float* pcm, int64_t n_samples, int batch, int n_mels, float* mel, void* ws,
                           size_t ws_bytes, void* stream) {
   if (!pcm || !mel || batch <= 0 || n_mels <= 0 || n_mels > 128 || n_samples <= 200 || n_samples % 160)
     return fail(nullptr, ASR_E_INVAL, "log_mel: bad arguments");
   if (!ws || ws_bytes < asr_op_log_mel_ws_size(batch)) return fail(nullptr, ASR_E_WORKSPACE, "log_mel: workspace too small");
-  static std::mutex mu;
-  static std::map<std::pair<int, int>, MelTables*> cache;  // (device, n_mels) -> device tables
-  int dev = 0;
-  cudaGetDevice(&dev);
-  MelTables* tab = nullptr;
-  {
-    std::lock_guard<std::mutex> lk(mu);
-    auto it = cache.find({dev, n_mels});
-    if (it == cache.end()) {
-      MelTables h;
-      build_mel_tables(n_mels, &h);
-      if (cudaMalloc(&tab, sizeof h) != cudaSuccess) return fail(nullptr, ASR_E_NOMEM, "log_mel: table allocation");
-      cudaMemcpy(tab, &h, sizeof h, cudaMemcpyHostToDevice);
-      cache[{dev, n_mels}] = tab;
-    } else {
-      tab = it->second;
-    }
-  }
+  if (reinterpret_cast<uintptr_t>(ws) & 255) return fail(nullptr, ASR_E_WORKSPACE, "log_mel: workspace must be 256-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   unsigned* cm = static_cast<unsigned*>(ws);
+  MelTables* tab = reinterpret_cast<MelTables*>(static_cast<char*>(ws) + log_mel_max_bytes(batch));
+  ASR_CUDA(nullptr, launch_mel_tables(n_mels, tab, st));
   ASR_CUDA(nullptr, cudaMemsetAsync(cm, 0, (size_t)batch * 4, st));
   ASR_CUDA(nullptr, launch_log_mel(pcm, n_samples, batch, n_mels, tab, mel, cm, st));
   ASR_CUDA(nullptr, launch_mel_normalize(mel, cm, (long long)n_mels * (n_samples / 160), batch, mel, st));
@@ -1162,9 +1132,8 @@ asr_status asr_op_log_mel_noalloc(const float* pcm, int64_t n_samples, int batch
     sc = g_noalloc[dev];
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  MelTables h;
-  build_mel_tables(n_mels, &h);
-  ASR_CUDA(nullptr, cudaMemcpyAsync(sc.tables, &h, sizeof h, cudaMemcpyHostToDevice, st));
+  // Tables are rebuilt on the device and the maxima cleared, in stream order.
+  ASR_CUDA(nullptr, launch_mel_tables(n_mels, sc.tables, st));
   ASR_CUDA(nullptr, cudaMemsetAsync(sc.clip_max, 0, (size_t)batch * 4, st));  // the maxima start at zero
   ASR_CUDA(nullptr, launch_log_mel(pcm, n_samples, batch, n_mels, sc.tables, mel, sc.clip_max, st));
   ASR_CUDA(nullptr, launch_mel_normalize(mel, sc.clip_max, (long long)n_mels * (n_samples / 160), batch, mel, st));

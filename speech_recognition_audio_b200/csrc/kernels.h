@@ -26,15 +26,36 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-// Tables of the log-mel kernel, computed on the host in double precision.
+// Tables of the log-mel kernel, built on the device by launch_mel_tables.
+constexpr int kMelMaxWeights = 2048;
 struct MelTables {
   float2 w200[200];   // exp(-2 pi i j / 200)
   float2 w400[201];   // exp(-2 pi i k / 400)
   float hann[400];    // periodic Hann
   int fstart[128], fcount[128], foff[128];
-  float fw[2048];     // non-zero filter weights, filter-major
+  float fw[kMelMaxWeights];  // non-zero filter weights, filter-major
 };
 
+// One clip of a variable-length batch (log-mel view): samples at pcm + s_off,
+// frames = n / 160 at mel + n_mels * f_off ([n_mels][frames]), and the index
+// of its first 32-frame group.
+struct MelClip {
+  long long s_off, n, f_off;
+  int frames, g_off;
+};
+struct MelArgs {
+  const float* pcm;
+  float* mel;                 // raw log10 mel
+  unsigned int* clip_max;     // [batch], order-preserving encoding, zero before the launch
+  int n_mels, batch, n_groups;
+  long long n_samples;        // uniform batches: samples per clip
+  int n_frames;               // uniform batches: frames per clip
+  const MelClip* clips;       // variable-length batches: [batch] (device), else null
+};
+int mel_groups(long long n_frames);  // 32-frame groups of a clip
+
+cudaError_t launch_mel_tables(int n_mels, MelTables* tab, cudaStream_t st);
+cudaError_t launch_log_mel(const MelArgs& args, const MelTables* tab, cudaStream_t st);
 cudaError_t launch_log_mel(const float* pcm, long long n_samples, int batch, int n_mels, const MelTables* tab,
                            float* mel_raw, unsigned int* clip_max, cudaStream_t st);
 cudaError_t launch_mel_normalize(const float* raw, const unsigned int* clip_max, long long per_clip, int batch,

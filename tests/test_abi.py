@@ -94,3 +94,23 @@ def test_null_handle_calls_fail_cleanly():
     sra.lib.asr_enc_destroy(None)
     rc = sra.lib.asr_enc_forward(None, None, 16000, 1, None, None, None, 0, None)
     assert rc == 1
+
+
+def test_documented_limits_are_enforced():
+    # Argument validation only: every call below is rejected on the host
+    # before anything reaches a device.
+    bad = synth.GEOMETRIES["moss"].as_dict()
+    bad.update(d_model=192, n_heads=3)                 # d_model must be a multiple of 128
+    assert sra.lib.asr_enc_weight_count(ctypes.byref(sra.Geometry.of(bad))) == -1
+    big = synth.GEOMETRIES["moss"].as_dict()
+    big.update(d_model=2176, n_heads=34)               # d_model must be <= 2048
+    assert sra.lib.asr_enc_weight_count(ctypes.byref(sra.Geometry.of(big))) == -1
+    # LayerNorm: D a multiple of 128 and at most 2048; NULL operands rejected first.
+    assert sra.lib.asr_op_layer_norm(None, None, None, 4, 1280, 1e-5, None, 0, None) == 1
+    fake = ctypes.c_void_p(256)                        # never dereferenced: the size check fails first
+    for D in (4096, 1000, 2176):
+        assert sra.lib.asr_op_layer_norm(fake, fake, fake, 4, D, 1e-5, fake, 0, None) == 1
+        assert b"layer_norm" in sra.lib.asr_enc_last_error(None)
+    # log-mel: the workspace holds the maxima and the tables
+    assert sra.lib.asr_op_log_mel_ws_size(16) >= 16 * 4 + 14 * 1024
+    assert sra.lib.asr_op_log_mel_ws_size(0) == 0
