@@ -52,7 +52,7 @@ typedef enum {
 
 enum { ASR_STEM_CONV2D_CHUNKED = 0, ASR_STEM_CONV1D = 1 };
 enum { ASR_POS_PER_CHUNK = 0, ASR_POS_GLOBAL = 1 };
-enum { ASR_DTYPE_BF16 = 0, ASR_DTYPE_F32 = 1 };
+enum { ASR_DTYPE_BF16 = 0, ASR_DTYPE_F32 = 1, ASR_DTYPE_F16 = 2 };
 
 /* Encoder geometry.  Field meanings:
  *  stem           ASR_STEM_CONV2D_CHUNKED: 3 x Conv2D k3 s2 p1 (1->C->C->C) + GELU
@@ -202,6 +202,37 @@ asr_status asr_enc_tap(asr_enc* e, int stage, float* dst, size_t dst_bytes, void
 asr_status asr_enc_profile(asr_enc* e, int enable);
 int asr_enc_profile_read(asr_enc* e, int max, const char** names, double* ms, int* launches);
 int asr_enc_last_launches(const asr_enc* e);
+
+/* ---- audio injection --------------------------------------------------------
+ * The LLM input embeddings of a tokenised prompt with the audio spliced in
+ * ("MOSS-Transcribe-preview-2B-GGUF", Architecture table, "Audio injection":
+ * the placeholder positions' token embeddings are replaced by the adapter
+ * output frames; "Prompt": the audio sits between <|audio_start|> and
+ * <|audio_end|> of a ChatML user turn).
+ *  ids          device int32 [n_ids], n_ids >= 1: the prompt's token ids (a
+ *               batch of prompts is passed as one packed sequence).
+ *  placeholder  the id of the audio placeholder token.
+ *  table        device [vocab, dim] token-embedding table of table_dtype
+ *               (ASR_DTYPE_BF16, ASR_DTYPE_F16 or ASR_DTYPE_F32).
+ *  frames       device float32 [n_frames, dim]: adapter output rows (the
+ *               forward's output of each clip, clips in prompt order).
+ *  out          device [n_ids, dim] of out_dtype: row i is frames[r] when
+ *               ids[i] == placeholder, r being the number of placeholders
+ *               before i, else table[ids[i]]; values are converted to
+ *               out_dtype with round-to-nearest-even (same-type rows are
+ *               copied bit for bit).
+ *  ws           device scratch of >= asr_splice_ws_size(n_ids) bytes,
+ *               256-byte aligned; its first int32 is the status word:
+ *               0 ok, 1 an id outside [0, vocab) (that row is zero), 2 the
+ *               placeholder count differs from n_frames (rows without a
+ *               frame are zero).  Asynchronous; asr_splice_check()
+ *               synchronises the stream and turns the word into ASR_OK or
+ *               ASR_E_INVAL. */
+size_t asr_splice_ws_size(int64_t n_ids);
+asr_status asr_splice_embeddings(const int32_t* ids, int64_t n_ids, int32_t placeholder, const void* table,
+                                 int vocab, int table_dtype, const float* frames, int64_t n_frames, int dim,
+                                 void* out, int out_dtype, void* ws, size_t ws_bytes, void* stream);
+asr_status asr_splice_check(const void* ws, void* stream);
 
 /* Message of the last failure on `e` (or process-wide when e is NULL). */
 const char* asr_enc_last_error(const asr_enc* e);

@@ -24,6 +24,8 @@ function.  Pins (in tests/test_oracle_*.py) for each function:
   head, adapter                  float64 torch composition of library ops
   token_count, window_partition  closed forms 13 n/16000 and n/320, and
                                  ceil(T/104) windows per clip
+  splice_embeddings              a hand-written prompt whose spliced rows are
+                                 listed explicitly in the test
 Parity unpinned: the per-chunk position reading (pos_mode 0) and the
 channel-major flatten before conv_out are conventions that only trained
 weights could distinguish; they are fixed by reading, not by a pin.
@@ -40,7 +42,7 @@ __all__ = [
     "mel_filterbank", "log_mel", "conv2d", "conv1d", "gelu", "silu", "layer_norm", "sinusoids",
     "linear", "token_count", "window_partition", "attention_windows", "attention_masked", "window_mask",
     "encoder_layer", "stem_conv2d_chunked", "stem_conv1d", "encode_tokens", "encode_clip", "forward",
-    "as64",
+    "as64", "splice_embeddings",
 ]
 
 SAMPLE_RATE = 16000
@@ -510,3 +512,34 @@ def forward(pcm: np.ndarray, W, geom, taps=None) -> np.ndarray:
         if taps is not None:
             taps.setdefault("clips", []).append(t)
     return np.stack(outs)
+
+
+# --------------------------------------------------------------------------
+# Audio injection.
+# --------------------------------------------------------------------------
+
+def splice_embeddings(ids, placeholder: int, table, frames) -> np.ndarray:
+    """LLM input embeddings of a prompt with the audio spliced in, float64
+    [len(ids), D]: position i takes the next unused adapter frame when its id
+    is the placeholder, else the token's row of the embedding table.
+    [MOSS] Architecture, "Audio injection" row (placeholder positions get
+    their token embedding replaced by the adapter output frames) and
+    "Prompt" row (ChatML framing around the audio).  Raises ValueError when
+    the placeholder count differs from the number of frames or an id is not
+    a row of the table."""
+    ids = [int(i) for i in np.asarray(ids).reshape(-1)]
+    table = as64(table)
+    frames = as64(frames)
+    if sum(1 for i in ids if i == placeholder) != frames.shape[0]:
+        raise ValueError("placeholder count differs from the number of frames")
+    out = np.zeros((len(ids), table.shape[1]), dtype=np.float64)
+    used = 0
+    for pos, tok in enumerate(ids):
+        if tok == placeholder:
+            out[pos] = frames[used]
+            used += 1
+        else:
+            if not 0 <= tok < table.shape[0]:
+                raise ValueError(f"token id {tok} is not a row of the table")
+            out[pos] = table[tok]
+    return out

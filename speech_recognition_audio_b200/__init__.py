@@ -13,6 +13,7 @@ The entry points mirror ``include/asr_enc.h`` and ``include/asr_ops.h``:
   Encoder.sync_status, set_taps, tap       status word and per-stage taps
   log_mel, linear, layer_norm, attention,
   wait_probe                               kernel-level ops
+  splice_embeddings                        asr_splice_embeddings / asr_splice_check
 """
 from __future__ import annotations
 
@@ -20,7 +21,7 @@ import ctypes
 import os
 
 __all__ = ["lib", "LIB_PATH", "AsrError", "Geometry", "tokens", "windows", "weight_names", "Encoder",
-           "log_mel", "linear", "layer_norm", "attention", "gelu", "wait_probe", "TAP_MEL", "TAP_STEM",
+           "log_mel", "linear", "layer_norm", "attention", "gelu", "wait_probe", "splice_embeddings", "TAP_MEL", "TAP_STEM",
            "TAP_LAYER0", "TAP_ENCODER", "TAP_HEAD", "EPI_BF16", "EPI_BF16_GELU", "EPI_F32_RESID",
            "EPI_F32", "EPI_SWIGLU"]
 
@@ -90,6 +91,9 @@ def _load():
         "asr_op_attention": (I, [P, P, I, I, I64, I, P, P, SZ, P]),
         "asr_op_gelu": (I, [P, P, I64, P]),
         "asr_op_wait_probe": (I, [I64, P, P]),
+        "asr_splice_ws_size": (SZ, [I64]),
+        "asr_splice_embeddings": (I, [P, I64, ctypes.c_int32, P, I, I, P, I64, I, P, I, P, SZ, P]),
+        "asr_splice_check": (I, [P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -356,3 +360,28 @@ def wait_probe(limit_ns: int, stream=None) -> int:
     _check(lib.asr_op_wait_probe(int(limit_ns), _ptr(st), _stream(stream)))
     torch.cuda.synchronize()
     return int(st.item())
+
+
+_DTYPE_CODE = {"bfloat16": 0, "float32": 1, "float16": 2}
+
+
+def splice_embeddings(ids, placeholder: int, table, frames, out_dtype=None, stream=None, check: bool = True):
+    """LLM input embeddings with the audio spliced in: ids CUDA int32 [n],
+    table CUDA [vocab, D] (bf16 / f16 / f32), frames CUDA float32 [n_frames, D]
+    -> CUDA [n, D] of out_dtype (default: the table's dtype).  With check the
+    call synchronises and raises on a bad id or a placeholder/frame count
+    mismatch."""
+    import torch
+    out_dtype = out_dtype or table.dtype
+    n = ids.numel()
+    D = table.shape[1]
+    out = torch.empty((n, D), dtype=out_dtype, device=ids.device)
+    ws = torch.empty(int(lib.asr_splice_ws_size(n)), dtype=torch.uint8, device=ids.device)
+    code = lambda t: _DTYPE_CODE[str(t).replace("torch.", "")]
+    st = _stream(stream)
+    _check(lib.asr_splice_embeddings(_ptr(ids), n, int(placeholder), _ptr(table), table.shape[0], code(table.dtype),
+                                     _ptr(frames), frames.shape[0] if frames is not None else 0, D, _ptr(out),
+                                     code(out_dtype), _ptr(ws), ws.numel(), st))
+    if check:
+        _check(lib.asr_splice_check(_ptr(ws), st))
+    return out

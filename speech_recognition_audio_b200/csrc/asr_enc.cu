@@ -1140,6 +1140,36 @@ asr_status asr_op_log_mel_noalloc(const float* pcm, int64_t n_samples, int batch
   return ASR_OK;
 }
 
+size_t asr_splice_ws_size(int64_t n_ids) { return n_ids > 0 ? 256 + align_up((size_t)n_ids * 4, 256) : 0; }
+
+asr_status asr_splice_embeddings(const int32_t* ids, int64_t n_ids, int32_t placeholder, const void* table, int vocab,
+                                 int table_dtype, const float* frames, int64_t n_frames, int dim, void* out,
+                                 int out_dtype, void* ws, size_t ws_bytes, void* stream) {
+  auto dt_ok = [](int d) { return d == ASR_DTYPE_BF16 || d == ASR_DTYPE_F16 || d == ASR_DTYPE_F32; };
+  if (!ids || !table || !out || n_ids <= 0 || vocab <= 0 || dim <= 0 || n_frames < 0 || (n_frames > 0 && !frames) ||
+      !dt_ok(table_dtype) || !dt_ok(out_dtype) || n_ids > 0x7FFFFFFF)
+    return fail(nullptr, ASR_E_INVAL, "splice: bad arguments");
+  if (!ws || ws_bytes < asr_splice_ws_size(n_ids) || (reinterpret_cast<uintptr_t>(ws) & 255))
+    return fail(nullptr, ASR_E_WORKSPACE, "splice: workspace NULL, unaligned or smaller than asr_splice_ws_size()");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* status = static_cast<int*>(ws);
+  int* rank = reinterpret_cast<int*>(static_cast<char*>(ws) + 256);
+  ASR_CUDA(nullptr, cudaMemsetAsync(status, 0, 4, st));
+  ASR_CUDA(nullptr, launch_splice(ids, n_ids, placeholder, table, vocab, table_dtype, frames, n_frames, dim, out,
+                                  out_dtype, rank, status, current_sm_count(), st));
+  return ASR_OK;
+}
+
+asr_status asr_splice_check(const void* ws, void* stream) {
+  if (!ws) return fail(nullptr, ASR_E_INVAL, "splice_check: ws is NULL");
+  ASR_CUDA(nullptr, cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  int s = 0;
+  ASR_CUDA(nullptr, cudaMemcpy(&s, ws, 4, cudaMemcpyDeviceToHost));
+  if (s == SPLICE_E_ID) return fail(nullptr, ASR_E_INVAL, "splice: a token id is outside [0, vocab)");
+  if (s == SPLICE_E_COUNT) return fail(nullptr, ASR_E_INVAL, "splice: the placeholder count differs from the frame count");
+  return ASR_OK;
+}
+
 asr_status asr_op_gelu(const float* x, float* y, int64_t n, void* stream) {
   if (!x || !y || n <= 0) return fail(nullptr, ASR_E_INVAL, "gelu: bad arguments");
   ASR_CUDA(nullptr, launch_gelu(x, y, n, static_cast<cudaStream_t>(stream)));

@@ -27,13 +27,18 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 }
 
 // Tables of the log-mel kernel, built on the device by launch_mel_tables.
-constexpr int kMelMaxWeights = 2048;
+constexpr int kMelMaxWeights = 1024;  // taps of any filterbank of <= 128 filters over 201 bins: <= 2 * 201 + 128
 struct MelTables {
   float2 w200[200];   // exp(-2 pi i j / 200)
   float2 w400[201];   // exp(-2 pi i k / 400)
   float hann[400];    // periodic Hann
   int fstart[128], fcount[128], foff[128];
-  float fw[kMelMaxWeights];  // non-zero filter weights, filter-major
+  float fw[kMelMaxWeights];  // non-zero filter weights, filter-major (an empty filter has one zero tap)
+  // The same taps as (bin | last-tap-of-its-filter << 8 | filter << 9), and
+  // their split over the 8 threads of a frame: thread t takes taps
+  // [tpart[t], tpart[t+1]), whole filters, about equal counts.
+  int tcode[kMelMaxWeights];
+  int tpart[9];
 };
 
 // One clip of a variable-length batch (log-mel view): samples at pcm + s_off,
@@ -80,6 +85,13 @@ cudaError_t launch_attention(const bf16* qkv, const int* cu, int n_seg, int max_
 bool make_tmap_qkv(CUtensorMap* map, const void* qkv, long long T, int H);
 cudaError_t launch_attention_tc(const CUtensorMap& tm_qkv, const bf16* qkv, const int* cu, int n_seg, int H, bf16* out,
                                 int* status, unsigned long long limit_ns, cudaStream_t st);
+
+// Audio-embedding splice (splice.cu).  Element types match ASR_DTYPE_*.
+enum : int { SPLICE_BF16 = 0, SPLICE_F32 = 1, SPLICE_F16 = 2 };
+enum : int { SPLICE_OK = 0, SPLICE_E_ID = 1, SPLICE_E_COUNT = 2 };
+cudaError_t launch_splice(const int* ids, long long n_ids, int placeholder, const void* table, int vocab,
+                          int table_dtype, const float* frames, long long n_frames, int D, void* out, int out_dtype,
+                          int* rank, int* status, int num_sms, cudaStream_t st);
 
 cudaError_t launch_fill_windows(int* cu, int batch, int tokens_per_clip, int window, int n_win_per_clip,
                                 cudaStream_t st);

@@ -25,8 +25,10 @@
 //      X[k] = E + W400^k O and conj X[200-k] = E - W400^k O with
 //      E = (Z[k] + conj Z[200-k]) / 2, O = -i (Z[k] - conj Z[200-k]) / 2;
 //      the 201 powers |X|^2 replace Z in the buffer.
-//   4. Each thread applies 1/8 of the sparse filterbank, takes
-//      log10(max(., 1e-10)), and the block writes the [n_mels][32] tile with
+//   4. The filterbank's taps (filter-major) are split over the octet in
+//      eight runs of whole filters with about equal tap counts; each thread
+//      walks its run with one fixed loop, emitting log10(max(sum, 1e-10))
+//      at each filter's last tap; the block writes the [n_mels][32] tile with
 //      coalesced row stores; the group's maximum goes to its clip with one
 //      atomicMax on an order-preserving integer encoding.
 // Only warp-level synchronisation separates the transform steps; three
@@ -52,8 +54,9 @@ constexpr int SM_TW = SM_FFT + G * NC * 8;                  // float2 [25][8]: W
 constexpr int SM_W25 = SM_TW + 25 * 8 * 8;                  // float2 [25]: W25^j
 constexpr int SM_W400 = SM_W25 + 26 * 8;                    // float2 [201 + 1]
 constexpr int SM_HANN = SM_W400 + 202 * 8;                  // float2 [200]: (w[2m], w[2m+1])
-constexpr int SM_FIDX = SM_HANN + NC * 8;                   // int [3][128]
-constexpr int SM_FW = SM_FIDX + 3 * 128 * 4;                // float [kMelMaxWeights]
+constexpr int SM_TPART = SM_HANN + NC * 8;                  // int [9] (+ pad)
+constexpr int SM_TCODE = SM_TPART + 16 * 4;                 // int [kMelMaxWeights]
+constexpr int SM_FW = SM_TCODE + kMelMaxWeights * 4;        // float [kMelMaxWeights]
 constexpr int SM_RED = SM_FW + kMelMaxWeights * 4;          // float [8]
 constexpr int SM_BYTES = SM_RED + 8 * 4;
 static_assert(128 * STAGE_PITCH <= SPAN_MAX, "the output tile fits in one PCM span buffer");
@@ -147,16 +150,27 @@ __device__ __forceinline__ GroupLoc locate(const MelArgs& a, int g) {
   return L;
 }
 
-// Issue the cp.async copies of group g's reflect-padded PCM span.
+__device__ __forceinline__ void cp_async_16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
+// Issue the cp.async copies of group g's reflect-padded PCM span: 16-byte
+// copies when the span lies inside the clip and is 16-byte aligned (every
+// span is a multiple of 8 samples), else 4-byte copies with the reflection.
 __device__ __forceinline__ void stage_span(const MelArgs& a, int g, float* dst, int tid) {
   const GroupLoc L = locate(a, g);
   const long long base = (long long)L.f0 * HOP - NFFT / 2;
   const int span = (L.nf - 1) * HOP + NFFT;
-  for (int j = tid; j < span; j += THREADS) {
-    long long i = base + j;
-    if (i < 0) i = -i;
-    if (i >= L.n) i = 2 * (L.n - 1) - i;
-    cp_async_4(dst + j, L.x + i);
+  const float* src = L.x + base;
+  if (base >= 0 && base + span <= L.n && (reinterpret_cast<uintptr_t>(src) & 15) == 0) {
+    for (int j = tid; j < span / 4; j += THREADS) cp_async_16(dst + 4 * j, src + 4 * j);
+  } else {
+    for (int j = tid; j < span; j += THREADS) {
+      long long i = base + j;
+      if (i < 0) i = -i;
+      if (i >= L.n) i = 2 * (L.n - 1) - i;
+      cp_async_4(dst + j, L.x + i);
+    }
   }
   cp_async_commit();
 }
@@ -216,15 +230,29 @@ __global__ void __launch_bounds__(256) mel_tables_kernel(int n_mels, MelTables* 
     int off = 0;
     for (int m = 0; m < n_mels; ++m) {
       t->fstart[m] = first[m];
-      t->fcount[m] = min(cnt[m], kMelMaxWeights - off);
+      t->fcount[m] = min(max(cnt[m], 1), kMelMaxWeights - off);  // an empty filter keeps one zero tap
       t->foff[m] = off;
       off += t->fcount[m];
     }
     for (int m = n_mels; m < 128; ++m) t->fstart[m] = t->fcount[m] = t->foff[m] = 0;
+    // thread split: cut at the first filter start at or after each eighth of the taps
+    t->tpart[0] = 0;
+    int m = 0;
+    for (int q = 1; q < 8; ++q) {
+      const int target = (q * off) / 8;
+      while (m < n_mels && t->foff[m] < target) ++m;
+      t->tpart[q] = m < n_mels ? t->foff[m] : off;
+    }
+    t->tpart[8] = off;
   }
   __syncthreads();
-  if (tid < n_mels)
-    for (int j = 0; j < t->fcount[tid]; ++j) t->fw[t->foff[tid] + j] = (float)weight(tid, t->fstart[tid] + j);
+  if (tid < n_mels) {
+    const int st = t->fstart[tid], c = t->fcount[tid], o = t->foff[tid];
+    for (int j = 0; j < c; ++j) {
+      t->fw[o + j] = cnt[tid] ? (float)weight(tid, st + j) : 0.0f;
+      t->tcode[o + j] = (st + j) | ((j == c - 1) << 8) | (tid << 9);
+    }
+  }
 }
 
 // ---------------------------------------------------------------- log-mel
@@ -236,9 +264,8 @@ __global__ void __launch_bounds__(THREADS, 2) log_mel_kernel(const MelArgs a, co
   float2* w25 = reinterpret_cast<float2*>(smem + SM_W25);
   float2* w400 = reinterpret_cast<float2*>(smem + SM_W400);
   float2* hann2 = reinterpret_cast<float2*>(smem + SM_HANN);
-  int* fstart = reinterpret_cast<int*>(smem + SM_FIDX);
-  int* fcount = fstart + 128;
-  int* foff = fstart + 256;
+  int* tpart = reinterpret_cast<int*>(smem + SM_TPART);
+  int* tcode = reinterpret_cast<int*>(smem + SM_TCODE);
   float* fw = reinterpret_cast<float*>(smem + SM_FW);
   float* red = reinterpret_cast<float*>(smem + SM_RED);
 
@@ -256,8 +283,11 @@ __global__ void __launch_bounds__(THREADS, 2) log_mel_kernel(const MelArgs a, co
   for (int i = tid; i < 25; i += THREADS) w25[i] = tab->w200[8 * i];
   for (int i = tid; i < NBIN; i += THREADS) w400[i] = tab->w400[i];
   for (int i = tid; i < NC; i += THREADS) hann2[i] = make_float2(tab->hann[2 * i], tab->hann[2 * i + 1]);
-  for (int i = tid; i < 3 * 128; i += THREADS) fstart[i] = (&tab->fstart[0])[i];
-  for (int i = tid; i < kMelMaxWeights; i += THREADS) fw[i] = tab->fw[i];
+  if (tid < 9) tpart[tid] = tab->tpart[tid];
+  for (int i = tid; i < kMelMaxWeights; i += THREADS) {
+    fw[i] = tab->fw[i];
+    tcode[i] = tab->tcode[i];
+  }
 
   int g = blockIdx.x;
   int buf = 0;
@@ -357,13 +387,20 @@ __global__ void __launch_bounds__(THREADS, 2) log_mel_kernel(const MelArgs a, co
     // ---- filterbank, log10, into the output tile [n_mels][G] (in the PCM span buffer)
     float* tile = cur;
     float lmax = -INFINITY;
-    for (int m = t; m < a.n_mels; m += 8) {
-      const int st = fstart[m], cnt = fcount[m], off = foff[m];
+    {
+      // this thread's share of the taps: whole filters, in order
+      const int j1 = tpart[t + 1];
       float acc = 0.f;
-      for (int j = 0; j < cnt; ++j) acc = fmaf(fw[off + j], pw[st + j], acc);
-      const float l = __log10f(fmaxf(acc, 1e-10f));
-      tile[m * STAGE_PITCH + r] = l;
-      if (r < L.nf) lmax = fmaxf(lmax, l);
+      for (int j = tpart[t]; j < j1; ++j) {
+        const int c = tcode[j];
+        acc = fmaf(fw[j], pw[c & 255], acc);
+        if (c & 256) {
+          const float l = __log10f(fmaxf(acc, 1e-10f));
+          tile[(c >> 9) * STAGE_PITCH + r] = l;
+          if (r < L.nf) lmax = fmaxf(lmax, l);
+          acc = 0.f;
+        }
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
@@ -435,6 +472,9 @@ int mel_groups(long long n_frames) { return static_cast<int>((n_frames + G - 1) 
 cudaError_t launch_log_mel(const MelArgs& args, const MelTables* tab, cudaStream_t st) {
   if (args.n_groups <= 0) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(log_mel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SM_BYTES);
+  // Two blocks per SM need ~213 KB: ask for the whole shared-memory carveout.
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(log_mel_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   const int blocks = std::min(args.n_groups, 2 * sm_count_current());
   return launch_pdl(log_mel_kernel, dim3(blocks), dim3(THREADS), SM_BYTES, st, args, tab);

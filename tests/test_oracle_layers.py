@@ -232,3 +232,20 @@ def test_window_sampling_is_exact():
     cu = oracle.window_partition(g, pcm.shape[0], 1)
     part = oracle.encode_clip(pcm, W, g, windows=[1, 2])
     np.testing.assert_allclose(part, full[cu[1]:cu[3]], rtol=1e-12, atol=1e-12)
+
+
+def test_splice_hand_example():
+    # MOSS card, Architecture "Audio injection": placeholder rows take the
+    # adapter frames in order, every other row its token embedding.
+    P = 9
+    table = np.arange(10 * 3, dtype=np.float64).reshape(10, 3)
+    frames = np.array([[100.0, 101.0, 102.0], [200.0, 201.0, 202.0], [300.0, 301.0, 302.0]])
+    ids = [3, P, P, 1, P, 0]
+    out = oracle.splice_embeddings(ids, P, table, frames)
+    expect = np.array([[9, 10, 11], [100, 101, 102], [200, 201, 202], [3, 4, 5], [300, 301, 302], [0, 1, 2]],
+                      dtype=np.float64)
+    np.testing.assert_array_equal(out, expect)
+    with pytest.raises(ValueError):
+        oracle.splice_embeddings([3, P, 1], P, table, frames)        # 1 placeholder, 3 frames
+    with pytest.raises(ValueError):
+        oracle.splice_embeddings([3, 12, P, P, P], P, table, frames)  # id 12 is not a row
