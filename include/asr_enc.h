@@ -105,11 +105,12 @@ asr_status asr_enc_weight_info(const asr_geometry* g, int i, const char** name, 
 
 /* ---- geometry queries (host only, bit-exact) ----------------------------- */
 
-/* Tokens per clip of n_samples: frames = n_samples/hop (trailing STFT frame
- * dropped); conv2d stem: (frames/chunk_frames) * L3 with L3 the length of a
- * chunk after three k3 s2 p1 convolutions (13 for 100 frames); conv1d stem:
- * frames after k3 s1 p1 then k3 s2 p1 (n/320).  Returns -1 when n_samples is
- * not a whole number of hops (conv2d: of chunks) or the geometry is invalid. */
+/* Tokens per clip of n_samples (> n_fft / 2): frames F = floor(n_samples /
+ * hop) (trailing STFT frame dropped); conv2d stem: the frames are cut into
+ * chunks of chunk_frames, the last one short when F is not a multiple, and a
+ * chunk of L frames gives ceil(ceil(ceil(L / 2) / 2) / 2) tokens (13 for 100);
+ * conv1d stem: frames after k3 s1 p1 then k3 s2 p1 (ceil(F / 2)).  Returns -1
+ * for n_samples <= n_fft / 2 or an invalid geometry. */
 int64_t asr_enc_tokens(const asr_geometry* g, int64_t n_samples);
 
 /* Attention-window partition of a batch of `batch` clips of n_samples each,
@@ -151,8 +152,10 @@ size_t asr_enc_workspace_size(const asr_enc* e, int64_t n_samples, int batch);
 
 /* Run the whole forward on `stream`.
  *  pcm         device float32 [batch, n_samples], row-major.
- *  n_samples   per clip; must be a multiple of 16000 for the conv2d stem and
- *              of 320 for the conv1d stem (ASR_E_UNSUPPORTED otherwise).
+ *  n_samples   per clip, > n_fft / 2.  Conv1d stem: an even number of hops
+ *              (ASR_E_UNSUPPORTED otherwise).  Conv2d stem: any length; a
+ *              clip whose frames are not whole chunks gets a short last
+ *              chunk (see asr_enc_forward_varlen).
  *  out         device float32 [batch, T, D_out], T = asr_enc_tokens(),
  *              D_out = adapter_out, else proj2_out, else d_model.
  *  out_tokens  optional host pointer; receives T.
@@ -163,6 +166,24 @@ size_t asr_enc_workspace_size(const asr_enc* e, int64_t n_samples, int batch);
 asr_status asr_enc_forward(asr_enc* e, const float* pcm, int64_t n_samples, int batch, float* out,
                            int64_t* out_tokens, void* workspace, size_t ws_bytes, void* stream);
 
+/* Variable-length batch (conv2d stem only; ASR_E_UNSUPPORTED otherwise):
+ * clip b has n_samples[b] samples (host int64 array, each > n_fft / 2).
+ *  pcm         device float32, the clips packed back to back (sum of
+ *              n_samples floats).
+ *  out         device float32 [sum of T_b, D_out]: each clip's token rows,
+ *              packed in clip order, T_b = asr_enc_tokens(g, n_samples[b]).
+ *  out_tokens  optional host int64 [batch]; receives T_b.
+ *  workspace   >= asr_enc_workspace_size_varlen() bytes, 256-byte aligned.
+ * Each clip has its own log-mel maximum and attention windows; a clip's
+ * last chunk holds its remaining frames (computed as a zero-padded whole
+ * chunk whose conv outputs past the short chunk's own lengths are zeroed, so
+ * each result equals the short chunk's convolution) and gives fewer tokens,
+ * whose positions restart at 0 like every chunk's.  The mel tap is not
+ * available for these batches. */
+size_t asr_enc_workspace_size_varlen(const asr_enc* e, const int64_t* n_samples, int batch);
+asr_status asr_enc_forward_varlen(asr_enc* e, const float* pcm, const int64_t* n_samples, int batch, float* out,
+                                  int64_t* out_tokens, void* workspace, size_t ws_bytes, void* stream);
+
 /* Same as asr_enc_forward but with HOST buffers: copies pcm (host float32
  * [batch, n_samples]; page-locked for full speed) into the workspace, runs
  * the forward and copies the result back into host `out` ([batch, T,
@@ -170,6 +191,10 @@ asr_status asr_enc_forward(asr_enc* e, const float* pcm, int64_t n_samples, int 
 asr_status asr_enc_forward_host(asr_enc* e, const float* pcm_host, int64_t n_samples, int batch,
                                 float* out_host, int64_t* out_tokens, void* workspace,
                                 size_t ws_bytes, void* stream);
+/* Host-buffer form of asr_enc_forward_varlen (packed host pcm and out). */
+asr_status asr_enc_forward_host_varlen(asr_enc* e, const float* pcm_host, const int64_t* n_samples, int batch,
+                                       float* out_host, int64_t* out_tokens, void* workspace, size_t ws_bytes,
+                                       void* stream);
 
 /* Synchronise the stream of the last forward and read the device status
  * word: ASR_OK, or ASR_E_DEVICE_TIMEOUT if a bounded wait gave up. */

@@ -266,24 +266,30 @@ def _conv_len(n: int, k: int = 3, s: int = 2, p: int = 1) -> int:
 
 
 def token_count(geom, n_samples: int) -> int:
-    """Encoder tokens of one clip of n_samples.
+    """Encoder tokens of one clip of n_samples (> n_fft / 2).
 
-    Mel frames = n_samples / hop ([MOSS] gotchas).  Conv2D stem: each chunk of
-    chunk_frames frames goes through three k3 s2 p1 convolutions along time
-    ([MOSS] Architecture "Conv front-end"; the per-chunk application is the
-    reading of the configured chunk size).  Conv1D stem: k3 s1 p1 then k3 s2 p1
-    ([CW] whisper-small geometry).
+    Mel frames F = floor(n_samples / hop): the centred STFT has 1 + floor(n /
+    hop) frames and the trailing one is dropped ([MOSS] gotchas).  Conv2D
+    stem: the frames are cut into chunks of chunk_frames, the last chunk
+    holding the remaining F mod chunk_frames frames when that is not zero;
+    each chunk goes through three k3 s2 p1 convolutions along time ([MOSS]
+    Architecture "Conv front-end"; the per-chunk application and the short
+    last chunk are the readings of the configured chunk size), so a chunk of
+    L frames gives ceil(ceil(ceil(L/2)/2)/2) tokens (13 for 100).  Conv1D
+    stem: k3 s1 p1 then k3 s2 p1 ([CW] whisper-small geometry).
     """
-    if n_samples % geom.hop:
-        raise ValueError("n_samples must be a multiple of hop")
+    if n_samples <= geom.n_fft // 2:
+        raise ValueError("reflect padding needs more than n_fft/2 samples")
     frames = n_samples // geom.hop
     if geom.stem == 0:
-        if frames % geom.chunk_frames:
-            raise ValueError("whole chunks only")
-        t = geom.chunk_frames
-        for _ in range(3):
-            t = _conv_len(t)
-        return (frames // geom.chunk_frames) * t
+        full, rest = divmod(frames, geom.chunk_frames)
+        total = 0
+        for length in [geom.chunk_frames] * full + ([rest] if rest else []):
+            t = length
+            for _ in range(3):
+                t = _conv_len(t)
+            total += t
+        return total
     return _conv_len(_conv_len(frames, s=1))
 
 

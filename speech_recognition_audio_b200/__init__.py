@@ -10,6 +10,7 @@ The entry points mirror ``include/asr_enc.h`` and ``include/asr_ops.h``:
   tokens, windows, weight_names            geometry queries (host only)
   Encoder(geometry, weights)               asr_enc_create / asr_enc_destroy
   Encoder.forward / forward_host           asr_enc_forward / asr_enc_forward_host
+  Encoder.forward_varlen / forward_host_varlen  variable-length batches
   Encoder.sync_status, set_taps, tap       status word and per-stage taps
   log_mel, linear, layer_norm, attention,
   wait_probe                               kernel-level ops
@@ -73,6 +74,9 @@ def _load():
         "asr_enc_workspace_size": (SZ, [P, I64, I]),
         "asr_enc_forward": (I, [P, P, I64, I, P, ctypes.POINTER(I64), P, SZ, P]),
         "asr_enc_forward_host": (I, [P, P, I64, I, P, ctypes.POINTER(I64), P, SZ, P]),
+        "asr_enc_workspace_size_varlen": (SZ, [P, ctypes.POINTER(I64), I]),
+        "asr_enc_forward_varlen": (I, [P, P, ctypes.POINTER(I64), I, P, ctypes.POINTER(I64), P, SZ, P]),
+        "asr_enc_forward_host_varlen": (I, [P, P, ctypes.POINTER(I64), I, P, ctypes.POINTER(I64), P, SZ, P]),
         "asr_enc_sync_status": (I, [P]),
         "asr_enc_set_taps": (I, [P, ctypes.c_uint]),
         "asr_enc_tap": (I, [P, I, P, SZ, P]),
@@ -274,6 +278,51 @@ class Encoder:
         _check(lib.asr_enc_forward_host(self.handle, _ptr(pcm_host), n, B, _ptr(out_host), ctypes.byref(nt),
                                         _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), self.handle)
         return out_host
+
+    def _ws_varlen(self, ns, workspace):
+        import torch
+        arr = (ctypes.c_int64 * len(ns))(*[int(v) for v in ns])
+        need = int(lib.asr_enc_workspace_size_varlen(self.handle, arr, len(ns)))
+        if need == 0:
+            raise AsrError(2, "unsupported variable-length batch")
+        if workspace is not None:
+            return arr, workspace
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = None
+            self._ws = torch.empty(need, dtype=torch.uint8, device=torch.device("cuda", self.device))
+        return arr, self._ws
+
+    def forward_varlen(self, pcm, n_samples, out=None, workspace=None, stream=None):
+        """Variable-length batch: pcm CUDA float32 [sum n_b] (clips packed),
+        n_samples list of per-clip lengths -> (CUDA float32 [sum T_b, D_out],
+        list of T_b)."""
+        import torch
+        if pcm.dtype != torch.float32 or not pcm.is_cuda or pcm.dim() != 1 or not pcm.is_contiguous():
+            raise ValueError("pcm must be a contiguous 1-D CUDA float32 tensor (clips packed)")
+        if pcm.numel() != sum(int(v) for v in n_samples):
+            raise ValueError("pcm length must equal sum(n_samples)")
+        toks = [self.tokens(v) for v in n_samples]
+        if min(toks) <= 0:
+            raise AsrError(2, "a clip length is not supported by this geometry")
+        if out is None:
+            out = torch.empty((sum(toks), self.d_out), dtype=torch.float32, device=pcm.device)
+        arr, ws = self._ws_varlen(n_samples, workspace)
+        nt = (ctypes.c_int64 * len(n_samples))()
+        _check(lib.asr_enc_forward_varlen(self.handle, _ptr(pcm), arr, len(n_samples), _ptr(out), nt, _ptr(ws),
+                                          ws.numel() * ws.element_size(), _stream(stream)), self.handle)
+        return out, list(nt)
+
+    def forward_host_varlen(self, pcm_host, n_samples, out_host=None, workspace=None, stream=None):
+        """Host form of forward_varlen (synchronous)."""
+        import torch
+        toks = [self.tokens(v) for v in n_samples]
+        if out_host is None:
+            out_host = torch.empty((sum(toks), self.d_out), dtype=torch.float32, pin_memory=pcm_host.is_pinned())
+        arr, ws = self._ws_varlen(n_samples, workspace)
+        nt = (ctypes.c_int64 * len(n_samples))()
+        _check(lib.asr_enc_forward_host_varlen(self.handle, _ptr(pcm_host), arr, len(n_samples), _ptr(out_host), nt,
+                                               _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), self.handle)
+        return out_host, list(nt)
 
     def sync_status(self):
         _check(lib.asr_enc_sync_status(self.handle), self.handle)

@@ -40,7 +40,7 @@ struct LayerW {
 
 struct ActMaps {
   const void* ws = nullptr;
-  int64_t n = 0;
+  int64_t n = 0, T = 0, chunks = 0;
   int batch = 0;
   unsigned taps = 0;
   CUtensorMap h, att, ff, c3, p1, p2, gu;
@@ -56,8 +56,15 @@ struct Plan {
   int64_t n = 0, Tc = 0, T = 0;
   int B = 0, F = 0, nwin_clip = 0, nwin = 0, max_win = 0, chunks = 0;
   int T1 = 0, F1 = 0, T2 = 0, F2 = 0, T3 = 0, F3 = 0;
+  // Variable-length batches (conv2d stem): per-clip layout, padded conv_out
+  // rows (every chunk padded to T3 tokens), total frames and mel groups.
+  bool varlen = false, has_short = false;
+  std::vector<VarClip> clips;
+  int64_t Tpad = 0, n_total = 0, Ftot = 0;
+  int n_groups = 0;
   size_t off_clipmax = 0, off_cu = 0, off_mel = 0, off_a1 = 0, off_c1 = 0, off_c2 = 0, off_c3 = 0, off_melT = 0, off_x = 0,
-         off_h = 0, off_qkv = 0, off_att = 0, off_ff = 0, off_p1 = 0, off_p2 = 0, off_gu = 0, off_pcm = 0, off_out = 0;
+         off_h = 0, off_qkv = 0, off_att = 0, off_ff = 0, off_p1 = 0, off_p2 = 0, off_gu = 0, off_pcm = 0, off_out = 0,
+         off_mclips = 0, off_chunkd = 0, off_xpad = 0;
   size_t off_tap[ASR_TAP_COUNT] = {0, 0, 0, 0, 0};
   size_t tap_bytes[ASR_TAP_COUNT] = {0, 0, 0, 0, 0};
   size_t total = 0;
@@ -159,16 +166,26 @@ int64_t numel(const WSpec& w) {
   return n;
 }
 
-// Tokens per clip, or -1.
+// Tokens of a chunk of L frames after three k3 s2 p1 convolutions.
+int64_t chunk_tokens(int64_t L) { return conv_len(conv_len(conv_len(L, 3, 2, 1), 3, 2, 1), 3, 2, 1); }
+
+// Tokens per clip, or -1.  frames = floor(n / hop) (the trailing STFT frame
+// dropped); the conv2d stem's last chunk may be short.
 int64_t tokens_per_clip(const asr_geometry* g, int64_t n) {
-  if (!geom_valid(g, nullptr) || n <= 0 || n % g->hop) return -1;
+  if (!geom_valid(g, nullptr) || n <= g->n_fft / 2) return -1;
   const int64_t frames = n / g->hop;
   if (g->stem == ASR_STEM_CONV2D_CHUNKED) {
-    if (frames % g->chunk_frames) return -1;
-    const int64_t t3 = conv_len(conv_len(conv_len(g->chunk_frames, 3, 2, 1), 3, 2, 1), 3, 2, 1);
-    return (frames / g->chunk_frames) * t3;
+    const int64_t full = frames / g->chunk_frames, rest = frames % g->chunk_frames;
+    return full * chunk_tokens(g->chunk_frames) + (rest ? chunk_tokens(rest) : 0);
   }
   return conv_len(conv_len(frames, 3, 1, 1), 3, 2, 1);
+}
+
+// A batch the uniform plan handles: whole hops, and for the conv2d stem
+// whole chunks (a short last chunk goes through the variable-length plan).
+bool uniform_ok(const asr_geometry* g, int64_t n) {
+  if (n % g->hop) return false;
+  return g->stem != ASR_STEM_CONV2D_CHUNKED || (n / g->hop) % g->chunk_frames == 0;
 }
 
 // Sinusoidal positions [rows, d]: d/2 frequencies exp(-ln(1e4) i / (d/2 - 1)),
@@ -570,6 +587,8 @@ bool make_plan(const asr_enc* e, int64_t n, int B, Plan* p) {
   p->nwin = p->nwin_clip * B;
   p->max_win = (int)std::min<int64_t>(w, tc);
   const int d = g->d_model;
+  p->Tpad = p->T;
+  p->n_total = n * B;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     off = align_up(off, 1024);
@@ -613,6 +632,104 @@ bool make_plan(const asr_enc* e, int64_t n, int B, Plan* p) {
   p->off_out = take((size_t)p->T * d_out(g) * 4);
   p->total = align_up(off, 1024);
   return true;
+}
+
+// Plan of a variable-length batch of the conv2d stem: clip b has ns[b]
+// samples.  Conv buffers hold every chunk at full size (a short last chunk
+// padded); conv_out writes padded token rows, compacted into the clips'
+// packed rows before the tower.
+bool make_plan_varlen(const asr_enc* e, const int64_t* ns, int B, Plan* p) {
+  const asr_geometry* g = &e->g;
+  if (g->stem != ASR_STEM_CONV2D_CHUNKED || !ns || B <= 0) return false;
+  p->varlen = true;
+  p->B = B;
+  p->n = -1;
+  p->F = 0;
+  p->Tc = 0;
+  const int cf = g->chunk_frames;
+  const int t3 = (int)chunk_tokens(cf);
+  const int w = g->window_tokens;
+  p->T1 = (int)conv_len(cf, 3, 2, 1); p->F1 = (int)conv_len(g->n_mels, 3, 2, 1);
+  p->T2 = (int)conv_len(p->T1, 3, 2, 1); p->F2 = (int)conv_len(p->F1, 3, 2, 1);
+  p->T3 = (int)conv_len(p->T2, 3, 2, 1); p->F3 = (int)conv_len(p->F2, 3, 2, 1);
+  p->clips.assign(B, VarClip{});
+  int64_t s = 0, f = 0, groups = 0, ch = 0, tok = 0, win = 0;
+  int maxseg = 0;
+  p->has_short = false;
+  for (int b = 0; b < B; ++b) {
+    const int64_t n = ns[b];
+    const int64_t tb = tokens_per_clip(g, n);
+    if (tb <= 0) return false;
+    const int64_t F = n / g->hop, K = (F + cf - 1) / cf;
+    const int64_t W = w ? (tb + w - 1) / w : 1;
+    if (F % cf) p->has_short = true;
+    VarClip& v = p->clips[b];
+    v.s_off = s; v.n = n; v.f_off = f; v.frames = (int)F; v.g_off = (int)groups;
+    v.chunk_off = (int)ch; v.chunks = (int)K; v.tok_off = (int)tok; v.tokens = (int)tb;
+    v.win_off = (int)win; v.wins = (int)W;
+    maxseg = std::max<int>(maxseg, (int)(w ? std::min<int64_t>(w, tb) : tb));
+    s += n; f += F; groups += mel_groups(F); ch += K; tok += tb; win += W;
+    if (s > (1LL << 40) || ch * t3 > 0x7FFFFFFFLL / 8 || groups > 0x7FFFFFFF || win > 0x7FFFFFF) return false;
+  }
+  p->n_total = s;
+  p->Ftot = f;
+  p->n_groups = (int)groups;
+  p->chunks = (int)ch;
+  p->Tpad = ch * t3;
+  p->T = tok;
+  p->nwin = (int)win;
+  p->max_win = maxseg;
+  p->nwin_clip = 0;
+  const int d = g->d_model;
+  const size_t C = g->conv_ch;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    off = align_up(off, 1024);
+    size_t r = off;
+    off += bytes;
+    return r;
+  };
+  p->off_clipmax = take((size_t)B * 4);
+  p->off_mclips = take((size_t)B * sizeof(MelClip));
+  p->off_chunkd = take((size_t)p->chunks * sizeof(ChunkDesc));
+  p->off_cu = take((size_t)(p->nwin + 1) * 4);
+  p->off_mel = take((size_t)g->n_mels * p->Ftot * 4);
+  p->off_a1 = take((size_t)p->chunks * p->T1 * p->F1 * 16 * 2);
+  p->off_c1 = take((size_t)p->chunks * p->T1 * p->F1 * C * 2);
+  p->off_c2 = take((size_t)p->chunks * p->T2 * p->F2 * C * 2);
+  p->off_c3 = take((size_t)p->Tpad * p->F3 * C * 2);
+  p->off_xpad = take((size_t)p->Tpad * d * 4);
+  p->off_x = take((size_t)p->T * d * 4);
+  p->off_h = take((size_t)p->T * d * 2);
+  p->off_qkv = take((size_t)p->T * 3 * d * 2);
+  p->off_att = take((size_t)p->T * d * 2);
+  p->off_ff = take((size_t)p->T * g->d_ffn * 2);
+  if (g->proj1_out) {
+    p->off_p1 = take((size_t)p->T * g->proj1_out * 2);
+    p->off_p2 = take((size_t)p->T * g->proj2_out * 2);
+  }
+  if (g->adapter_hidden) p->off_gu = take((size_t)p->T * g->adapter_hidden * 2);
+  p->tap_bytes[ASR_TAP_MEL] = 0;  // the mel tap covers uniform batches only
+  p->tap_bytes[ASR_TAP_STEM] = p->tap_bytes[ASR_TAP_LAYER0] = p->tap_bytes[ASR_TAP_ENCODER] = (size_t)p->T * d * 4;
+  p->tap_bytes[ASR_TAP_HEAD] = g->proj2_out ? (size_t)p->T * g->proj2_out * 4 : 0;
+  for (int t = 0; t < ASR_TAP_COUNT; ++t)
+    if (((e->taps >> t) & 1u) && p->tap_bytes[t]) p->off_tap[t] = take(p->tap_bytes[t]);
+  p->off_pcm = take((size_t)p->n_total * 4);
+  p->off_out = take((size_t)p->T * d_out(g) * 4);
+  p->total = align_up(off, 1024);
+  return true;
+}
+
+// The plan of a batch: per-clip sizes `ns` (variable length), or B clips of
+// n samples (uniform when n is whole chunks, else the variable-length plan
+// with every clip of n samples).
+bool plan_for(const asr_enc* e, const int64_t* ns, int64_t n, int B, Plan* p) {
+  if (ns) return make_plan_varlen(e, ns, B, p);
+  if (B <= 0) return false;
+  if (uniform_ok(&e->g, n)) return make_plan(e, n, B, p);
+  if (e->g.stem != ASR_STEM_CONV2D_CHUNKED) return false;
+  std::vector<int64_t> v(B, n);
+  return make_plan_varlen(e, v.data(), B, p);
 }
 
 asr_status gemm(asr_enc* e, const CUtensorMap* amap, const ConvGather* cg, const GemmB& w, long long M, void* out,
@@ -684,7 +801,7 @@ void prof_end(asr_enc* e, cudaStream_t st) {
 
 asr_status ensure_maps(asr_enc* e, const Plan& p, char* ws) {
   ActMaps& m = e->maps;
-  if (m.ws == ws && m.n == p.n && m.batch == p.B && m.taps == e->taps) return ASR_OK;
+  if (m.ws == ws && m.n == p.n && m.batch == p.B && m.T == p.T && m.chunks == p.chunks && m.taps == e->taps) return ASR_OK;
   const asr_geometry* g = &e->g;
   const int d = g->d_model;
   bool ok = make_tmap_qkv(&m.qkv, ws + p.off_qkv, p.T, g->n_heads) &&
@@ -693,7 +810,7 @@ asr_status ensure_maps(asr_enc* e, const Plan& p, char* ws) {
             make_tmap_bf16(&m.ff, ws + p.off_ff, p.T, g->d_ffn, g->d_ffn, 128);
   if (ok && g->stem == ASR_STEM_CONV2D_CHUNKED) {
     const int C = g->conv_ch;
-    ok = make_tmap_bf16(&m.c3, ws + p.off_c3, p.T, (size_t)p.F3 * C, (size_t)p.F3 * C, 128) &&
+    ok = make_tmap_bf16(&m.c3, ws + p.off_c3, p.Tpad, (size_t)p.F3 * C, (size_t)p.F3 * C, 128) &&
          make_tmap_bf16(&m.a1, ws + p.off_a1, (size_t)p.chunks * p.T1 * p.F1, 16, 16, 128);
     if (ok && e->box2)
       ok = e->phase2 ? make_tmap_convphase(&m.cin2, ws + p.off_c1, C, p.F1 / 2, p.T1 / 2, 4 * p.chunks, p.F2, 128 / p.F2)
@@ -725,6 +842,8 @@ asr_status ensure_maps(asr_enc* e, const Plan& p, char* ws) {
   }
   m.ws = ws;
   m.n = p.n;
+  m.T = p.T;
+  m.chunks = p.chunks;
   m.batch = p.B;
   m.taps = e->taps;
   return ASR_OK;
@@ -749,10 +868,35 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
   e->prof_recs.clear();
   ASR_LAUNCH(e, cudaMemsetAsync(e->status, 0, 4, st));
   ASR_LAUNCH(e, cudaMemsetAsync(clip_max, 0, (size_t)p.B * 4, st));
-  const int w = g->window_tokens ? g->window_tokens : (int)p.Tc;
-  ASR_K(PC_MISC, ASR_LAUNCH(e, launch_fill_windows(cu, p.B, (int)p.Tc, w, p.nwin_clip, st)));
-  ASR_K(PC_MEL, ASR_LAUNCH(e, launch_log_mel(pcm, p.n, p.B, g->n_mels, e->mel_tab, mel, clip_max, st)));
-  if (float* t = tap(ASR_TAP_MEL)) ASR_K(PC_MISC, ASR_LAUNCH(e, launch_mel_normalize(mel, clip_max, (long long)g->n_mels * p.F, p.B, t, st)));
+  MelClip* mclips = reinterpret_cast<MelClip*>(ws + p.off_mclips);
+  ChunkDesc* chunkd = reinterpret_cast<ChunkDesc*>(ws + p.off_chunkd);
+  if (!p.varlen) {
+    const int w = g->window_tokens ? g->window_tokens : (int)p.Tc;
+    ASR_K(PC_MISC, ASR_LAUNCH(e, launch_fill_windows(cu, p.B, (int)p.Tc, w, p.nwin_clip, st)));
+    ASR_K(PC_MEL, ASR_LAUNCH(e, launch_log_mel(pcm, p.n, p.B, g->n_mels, e->mel_tab, mel, clip_max, st)));
+    if (float* t = tap(ASR_TAP_MEL)) ASR_K(PC_MISC, ASR_LAUNCH(e, launch_mel_normalize(mel, clip_max, (long long)g->n_mels * p.F, p.B, t, st)));
+  } else {
+    // per-clip descriptors, chunk descriptors and window offsets, 32 clips a launch
+    const int t3 = p.T3;
+    for (int b0 = 0; b0 < p.B; b0 += kVarClipsPerLaunch) {
+      VarClipBatch vb;
+      vb.first = b0;
+      vb.count = std::min(kVarClipsPerLaunch, p.B - b0);
+      for (int i = 0; i < vb.count; ++i) vb.c[i] = p.clips[b0 + i];
+      const int last = b0 + vb.count == p.B ? 1 : 0;
+      ASR_K(PC_MISC, ASR_LAUNCH(e, launch_varlen_fill(vb, g->chunk_frames, g->window_tokens, t3, mclips, chunkd, cu, last,
+                                                      p.nwin, (int)p.T, st)));
+    }
+    MelArgs ma = {};
+    ma.pcm = pcm;
+    ma.mel = mel;
+    ma.clip_max = clip_max;
+    ma.n_mels = g->n_mels;
+    ma.batch = p.B;
+    ma.n_groups = p.n_groups;
+    ma.clips = mclips;
+    ASR_K(PC_MEL, ASR_LAUNCH(e, launch_log_mel(ma, e->mel_tab, st)));
+  }
 
   if (g->stem == ASR_STEM_CONV2D_CHUNKED) {
     const int C = g->conv_ch;
@@ -760,10 +904,17 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
     bf16* c2 = reinterpret_cast<bf16*>(ws + p.off_c2);
     bf16* c3 = reinterpret_cast<bf16*>(ws + p.off_c3);
     bf16* a1 = reinterpret_cast<bf16*>(ws + p.off_a1);
-    ASR_K(PC_CONV1, ASR_LAUNCH(e, launch_conv1_im2col(mel, clip_max, p.B, g->n_mels, p.F, g->chunk_frames,
-                                                      e->phase2 ? 1 : 0, a1, st)));
+    if (!p.varlen)
+      ASR_K(PC_CONV1, ASR_LAUNCH(e, launch_conv1_im2col(mel, clip_max, p.B, g->n_mels, p.F, g->chunk_frames,
+                                                        e->phase2 ? 1 : 0, a1, st)));
+    else
+      ASR_K(PC_CONV1, ASR_LAUNCH(e, launch_conv1_im2col_varlen(mel, clip_max, p.chunks, g->n_mels, g->chunk_frames,
+                                                               e->phase2 ? 1 : 0, chunkd, mclips, a1, st)));
     ASR_K(PC_CONV1, ASR_TRY(gemm(e, &e->maps.a1, nullptr, e->c1, (long long)p.chunks * p.T1 * p.F1, c1, C, e->c1b,
                                  nullptr, 1, EPI_GELU, st, &e->maps.o_c1)));
+    if (p.has_short)
+      ASR_K(PC_MISC, ASR_LAUNCH(e, launch_mask_short_chunks(c1, chunkd, p.chunks, g->chunk_frames, 1, p.T1, p.F1, C,
+                                                            e->phase2 ? 1 : 0, st)));
     const int CB = (C + 63) / 64;
     if (e->box2) {
       const int TR = 128 / p.F2, tpi = (p.T2 + TR - 1) / TR;
@@ -773,6 +924,9 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
       ConvGather cg2 = {c1, p.T1, p.F1, C, p.T2, p.F2, 2, 2, 3, 3, 1, 1};
       ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, nullptr, &cg2, e->c2, (long long)p.chunks * p.T2 * p.F2, c2, C, e->c2b, nullptr, 1, EPI_GELU, st, &e->maps.o_c2)));
     }
+    if (p.has_short)
+      ASR_K(PC_MISC, ASR_LAUNCH(e, launch_mask_short_chunks(c2, chunkd, p.chunks, g->chunk_frames, 2, p.T2, p.F2, C, 0,
+                                                            st)));
     if (e->box3) {
       const int TR = 128 / p.F3, tpi = (p.T3 + TR - 1) / TR;
       ConvBox b3 = {TR, p.F3, p.T3, tpi, p.chunks * tpi, 2, 2, 1, 1, 3, CB, 0, (C - 64 * (CB - 1) + 15) / 16};
@@ -781,7 +935,13 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
       ConvGather cg3 = {c2, p.T2, p.F2, C, p.T3, p.F3, 2, 2, 3, 3, 1, 1};
       ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, nullptr, &cg3, e->c3, (long long)p.chunks * p.T3 * p.F3, c3, C, e->c3b, nullptr, 1, EPI_GELU, st, &e->maps.o_c3)));
     }
-    ASR_K(PC_GEMM_CONVOUT, ASR_TRY(gemm(e, &e->maps.c3, nullptr, e->cout, p.T, x, d, nullptr, e->pe, p.T3, EPI_OUT_F32 | EPI_PE, st, nullptr)));
+    if (!p.varlen) {
+      ASR_K(PC_GEMM_CONVOUT, ASR_TRY(gemm(e, &e->maps.c3, nullptr, e->cout, p.T, x, d, nullptr, e->pe, p.T3, EPI_OUT_F32 | EPI_PE, st, nullptr)));
+    } else {
+      float* xpad = reinterpret_cast<float*>(ws + p.off_xpad);
+      ASR_K(PC_GEMM_CONVOUT, ASR_TRY(gemm(e, &e->maps.c3, nullptr, e->cout, p.Tpad, xpad, d, nullptr, e->pe, p.T3, EPI_OUT_F32 | EPI_PE, st, nullptr)));
+      ASR_K(PC_MISC, ASR_LAUNCH(e, launch_compact_tokens(xpad, x, chunkd, p.chunks, p.T3, d, st)));
+    }
   } else {
     if (p.Tc > e->pe_rows) return fail(e, ASR_E_UNSUPPORTED, "conv1d stem: %lld positions > %d", (long long)p.Tc, e->pe_rows);
     bf16* melT = reinterpret_cast<bf16*>(ws + p.off_melT);
@@ -838,25 +998,75 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
   return ASR_OK;
 }
 
-asr_status check_forward_args(asr_enc* e, int64_t n, int B, const void* pcm, const void* out, void* ws, size_t ws_bytes,
-                              Plan* p) {
+// Validates a forward of `B` clips, per-clip sizes `ns` (variable length) or
+// n samples each, and builds its plan.
+asr_status check_forward_args(asr_enc* e, const int64_t* ns, int64_t n, int B, const void* pcm, const void* out, void* ws,
+                              size_t ws_bytes, Plan* p) {
   if (!e) return fail(nullptr, ASR_E_INVAL, "handle is NULL");
   if (!pcm || !out) return fail(e, ASR_E_INVAL, "pcm or out is NULL");
   if (B <= 0) return fail(e, ASR_E_INVAL, "batch must be > 0");
-  if (n <= e->g.n_fft / 2) return fail(e, ASR_E_INVAL, "n_samples must exceed n_fft/2 (reflect padding)");
-  if (tokens_per_clip(&e->g, n) <= 0)
-    return fail(e, ASR_E_UNSUPPORTED, e->g.stem == ASR_STEM_CONV2D_CHUNKED
-                                          ? "n_samples must be a whole number of %d-frame chunks"
-                                          : "n_samples must be a multiple of the hop (%d frames ok)",
-                e->g.chunk_frames);
-  if (e->g.stem == ASR_STEM_CONV1D && (n / e->g.hop) % 2)
-    return fail(e, ASR_E_UNSUPPORTED, "conv1d stem: an even number of frames is required");
-  const int64_t T = tokens_per_clip(&e->g, n) * B;
-  if (T > 0x7FFFFFFFLL / 8 || (int64_t)B * n > (1LL << 40)) return fail(e, ASR_E_UNSUPPORTED, "batch too large");
-  if (!make_plan(e, n, B, p)) return fail(e, ASR_E_INVAL, "plan failed");
+  const asr_geometry* g = &e->g;
+  for (int b = 0; b < (ns ? B : 1); ++b) {
+    const int64_t nb = ns ? ns[b] : n;
+    if (nb <= g->n_fft / 2) return fail(e, ASR_E_INVAL, "clip %d: n_samples must exceed n_fft/2 (reflect padding)", b);
+    if (g->stem == ASR_STEM_CONV1D && (nb % g->hop || (nb / g->hop) % 2))
+      return fail(e, ASR_E_UNSUPPORTED, "conv1d stem: n_samples must be an even number of hops (%d samples)", g->hop);
+  }
+  if (ns && g->stem != ASR_STEM_CONV2D_CHUNKED)
+    return fail(e, ASR_E_UNSUPPORTED, "variable-length batches need the chunked conv2d stem");
+  if (!ns) {
+    const int64_t T = tokens_per_clip(g, n) * B;
+    if (T > 0x7FFFFFFFLL / 8 || (int64_t)B * n > (1LL << 40)) return fail(e, ASR_E_UNSUPPORTED, "batch too large");
+  }
+  if (!plan_for(e, ns, n, B, p)) return fail(e, ASR_E_UNSUPPORTED, "batch too large or sizes unsupported");
+  if (p->varlen && ((e->taps >> ASR_TAP_MEL) & 1u))
+    return fail(e, ASR_E_UNSUPPORTED, "the mel tap covers batches of whole chunks only");
   if (!ws || ws_bytes < p->total) return fail(e, ASR_E_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, p->total);
   if (reinterpret_cast<uintptr_t>(ws) & 255) return fail(e, ASR_E_WORKSPACE, "workspace must be 256-byte aligned");
   return ASR_OK;
+}
+
+void report_tokens(const Plan& p, const asr_geometry* g, int64_t n, const int64_t* ns, int64_t* out_tokens) {
+  if (!out_tokens) return;
+  if (ns) {
+    for (int b = 0; b < p.B; ++b) out_tokens[b] = p.clips[b].tokens;
+  } else {
+    *out_tokens = tokens_per_clip(g, n);
+  }
+}
+
+asr_status forward_common(asr_enc* e, const float* pcm, const int64_t* ns, int64_t n, int B, float* out,
+                          int64_t* out_tokens, void* workspace, size_t ws_bytes, void* stream) {
+  Plan p;
+  ASR_TRY(check_forward_args(e, ns, n, B, pcm, out, workspace, ws_bytes, &p));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ASR_TRY(run_forward(e, pcm, p, out, static_cast<char*>(workspace), st));
+  e->last_stream = st;
+  e->have_last = true;
+  e->last_plan = p;
+  e->last_ws = workspace;
+  report_tokens(p, &e->g, n, ns, out_tokens);
+  return ASR_OK;
+}
+
+asr_status forward_host_common(asr_enc* e, const float* pcm_host, const int64_t* ns, int64_t n, int B, float* out_host,
+                               int64_t* out_tokens, void* workspace, size_t ws_bytes, void* stream) {
+  Plan p;
+  ASR_TRY(check_forward_args(e, ns, n, B, pcm_host, out_host, workspace, ws_bytes, &p));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  float* dpcm = reinterpret_cast<float*>(ws + p.off_pcm);
+  ASR_CUDA(e, cudaMemcpyAsync(dpcm, pcm_host, (size_t)p.n_total * 4, cudaMemcpyHostToDevice, st));
+  const size_t out_bytes = (size_t)p.T * d_out(&e->g) * 4;
+  float* dout = reinterpret_cast<float*>(ws + p.off_out);
+  ASR_TRY(run_forward(e, dpcm, p, dout, ws, st));
+  ASR_CUDA(e, cudaMemcpyAsync(out_host, dout, out_bytes, cudaMemcpyDeviceToHost, st));
+  e->last_stream = st;
+  e->have_last = true;
+  e->last_plan = p;
+  e->last_ws = workspace;
+  report_tokens(p, &e->g, n, ns, out_tokens);
+  return asr_enc_sync_status(e);
 }
 
 }  // namespace
@@ -865,22 +1075,25 @@ extern "C" {
 
 size_t asr_enc_workspace_size(const asr_enc* e, int64_t n_samples, int batch) {
   Plan p;
-  if (!e || !make_plan(e, n_samples, batch, &p)) return 0;
+  if (!e || !plan_for(e, nullptr, n_samples, batch, &p)) return 0;
+  return p.total;
+}
+
+size_t asr_enc_workspace_size_varlen(const asr_enc* e, const int64_t* n_samples, int batch) {
+  Plan p;
+  if (!e || !n_samples || !plan_for(e, n_samples, 0, batch, &p)) return 0;
   return p.total;
 }
 
 asr_status asr_enc_forward(asr_enc* e, const float* pcm, int64_t n_samples, int batch, float* out, int64_t* out_tokens,
                            void* workspace, size_t ws_bytes, void* stream) {
-  Plan p;
-  ASR_TRY(check_forward_args(e, n_samples, batch, pcm, out, workspace, ws_bytes, &p));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  ASR_TRY(run_forward(e, pcm, p, out, static_cast<char*>(workspace), st));
-  e->last_stream = st;
-  e->have_last = true;
-  e->last_plan = p;
-  e->last_ws = workspace;
-  if (out_tokens) *out_tokens = p.Tc;
-  return ASR_OK;
+  return forward_common(e, pcm, nullptr, n_samples, batch, out, out_tokens, workspace, ws_bytes, stream);
+}
+
+asr_status asr_enc_forward_varlen(asr_enc* e, const float* pcm, const int64_t* n_samples, int batch, float* out,
+                                  int64_t* out_tokens, void* workspace, size_t ws_bytes, void* stream) {
+  if (!n_samples) return fail(e, ASR_E_INVAL, "n_samples is NULL");
+  return forward_common(e, pcm, n_samples, 0, batch, out, out_tokens, workspace, ws_bytes, stream);
 }
 
 asr_status asr_enc_sync_status(asr_enc* e) {
@@ -895,22 +1108,14 @@ asr_status asr_enc_sync_status(asr_enc* e) {
 
 asr_status asr_enc_forward_host(asr_enc* e, const float* pcm_host, int64_t n_samples, int batch, float* out_host,
                                 int64_t* out_tokens, void* workspace, size_t ws_bytes, void* stream) {
-  Plan p;
-  ASR_TRY(check_forward_args(e, n_samples, batch, pcm_host, out_host, workspace, ws_bytes, &p));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  char* ws = static_cast<char*>(workspace);
-  float* dpcm = reinterpret_cast<float*>(ws + p.off_pcm);
-  ASR_CUDA(e, cudaMemcpyAsync(dpcm, pcm_host, (size_t)batch * n_samples * 4, cudaMemcpyHostToDevice, st));
-  const size_t out_bytes = (size_t)p.T * d_out(&e->g) * 4;
-  float* dout = reinterpret_cast<float*>(ws + p.off_out);
-  ASR_TRY(run_forward(e, dpcm, p, dout, ws, st));
-  ASR_CUDA(e, cudaMemcpyAsync(out_host, dout, out_bytes, cudaMemcpyDeviceToHost, st));
-  e->last_stream = st;
-  e->have_last = true;
-  e->last_plan = p;
-  e->last_ws = workspace;
-  if (out_tokens) *out_tokens = p.Tc;
-  return asr_enc_sync_status(e);
+  return forward_host_common(e, pcm_host, nullptr, n_samples, batch, out_host, out_tokens, workspace, ws_bytes, stream);
+}
+
+asr_status asr_enc_forward_host_varlen(asr_enc* e, const float* pcm_host, const int64_t* n_samples, int batch,
+                                       float* out_host, int64_t* out_tokens, void* workspace, size_t ws_bytes,
+                                       void* stream) {
+  if (!n_samples) return fail(e, ASR_E_INVAL, "n_samples is NULL");
+  return forward_host_common(e, pcm_host, n_samples, 0, batch, out_host, out_tokens, workspace, ws_bytes, stream);
 }
 
 asr_status asr_enc_set_taps(asr_enc* e, unsigned mask) {

@@ -68,6 +68,38 @@ cudaError_t launch_mel_normalize(const float* raw, const unsigned int* clip_max,
 cudaError_t launch_mel_normalize_transpose(const float* raw, const unsigned int* clip_max, int batch, int n_mels,
                                            int n_frames, bf16* out, cudaStream_t st);
 
+// Variable-length batches.  One conv chunk: its clip, its first frame within
+// the clip, its valid frames (chunk_frames except for a clip's last chunk)
+// and the packed token row of its first token.
+struct ChunkDesc {
+  int clip, frame0, nvalid, tok_dst;
+};
+// Per-clip layout of a variable-length batch, computed on the host.
+struct VarClip {
+  long long s_off, n, f_off;          // samples: offset, count; frames: offset
+  int frames, g_off;                   // frames, first 32-frame mel group
+  int chunk_off, chunks;               // conv chunks
+  int tok_off, tokens;                 // packed token rows
+  int win_off, wins;                   // attention windows
+};
+constexpr int kVarClipsPerLaunch = 32;
+struct VarClipBatch {
+  int first, count;
+  VarClip c[kVarClipsPerLaunch];
+};
+// Writes the mel descriptors, the chunk descriptors and the window offsets
+// of the clips in `vb` (one block per clip); with last != 0 also the final
+// window offset cu[n_win] = n_tokens.
+cudaError_t launch_varlen_fill(const VarClipBatch& vb, int chunk_frames, int window, int t3, MelClip* mc,
+                               ChunkDesc* cd, int* cu, int last, int n_win, int n_tokens, cudaStream_t st);
+cudaError_t launch_conv1_im2col_varlen(const float* mel_raw, const unsigned int* clip_max, int n_chunks, int n_mels,
+                                       int chunk_frames, int phase, const ChunkDesc* cd, const MelClip* mc, bf16* a,
+                                       cudaStream_t st);
+cudaError_t launch_mask_short_chunks(bf16* act, const ChunkDesc* cd, int n_chunks, int chunk_frames, int level, int T,
+                                     int F, int C, int phase, cudaStream_t st);
+cudaError_t launch_compact_tokens(const float* xpad, float* x, const ChunkDesc* cd, int n_chunks, int t3, int d,
+                                  cudaStream_t st);
+
 // A operand of the first Conv2D (1 -> C, k3 s2 p1) as a GEMM: per output
 // position of each chunk of chunk_frames frames, its 9 normalised log-mel
 // taps (kh * 3 + kw) as bf16 in a row of 16 (taps 9..15 zero).  Rows

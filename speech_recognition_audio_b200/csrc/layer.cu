@@ -331,6 +331,41 @@ cudaError_t launch_fill_windows(int* cu, int batch, int tokens_per_clip, int win
                     n_win_per_clip);
 }
 
+__global__ void varlen_fill_kernel(const VarClipBatch vb, int chunk_frames, int window, int t3, MelClip* __restrict__ mc,
+                                   ChunkDesc* __restrict__ cd, int* __restrict__ cu, int last, int n_win, int n_tokens) {
+  pdl_wait();
+  pdl_trigger();
+  const VarClip& v = vb.c[blockIdx.x];
+  const int clip = vb.first + blockIdx.x;
+  if (threadIdx.x == 0) {
+    MelClip m;
+    m.s_off = v.s_off;
+    m.n = v.n;
+    m.f_off = v.f_off;
+    m.frames = v.frames;
+    m.g_off = v.g_off;
+    mc[clip] = m;
+  }
+  for (int q = threadIdx.x; q < v.chunks; q += blockDim.x) {
+    ChunkDesc c;
+    c.clip = clip;
+    c.frame0 = q * chunk_frames;
+    c.nvalid = min(chunk_frames, v.frames - q * chunk_frames);
+    c.tok_dst = v.tok_off + q * t3;
+    cd[v.chunk_off + q] = c;
+  }
+  const int w = window ? window : v.tokens;
+  for (int j = threadIdx.x; j < v.wins; j += blockDim.x) cu[v.win_off + j] = v.tok_off + j * w;
+  if (last && blockIdx.x == gridDim.x - 1 && threadIdx.x == 0) cu[n_win] = n_tokens;
+}
+
+cudaError_t launch_varlen_fill(const VarClipBatch& vb, int chunk_frames, int window, int t3, MelClip* mc,
+                               ChunkDesc* cd, int* cu, int last, int n_win, int n_tokens, cudaStream_t st) {
+  if (vb.count <= 0 || vb.count > kVarClipsPerLaunch) return cudaErrorInvalidValue;
+  return launch_pdl(varlen_fill_kernel, dim3(vb.count), dim3(128), 0, st, vb, chunk_frames, window, t3, mc, cd, cu,
+                    last, n_win, n_tokens);
+}
+
 __global__ void bf16_to_f32_kernel(const bf16* __restrict__ in, float* __restrict__ out, long long n) {
   pdl_wait();
   pdl_trigger();

@@ -25,7 +25,8 @@ __global__ void __launch_bounds__(256) conv1_im2col_kernel(const float* __restri
                                                            const unsigned int* __restrict__ clip_max, int n_mels,
                                                            int n_frames, int chunk_frames, int chunks_per_clip,
                                                            int T1, int F1, long long rows, int phase,
-                                                           bf16* __restrict__ a) {
+                                                           const ChunkDesc* __restrict__ cd,
+                                                           const MelClip* __restrict__ mc, bf16* __restrict__ a) {
   pdl_wait();
   pdl_trigger();
   const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
@@ -40,20 +41,34 @@ __global__ void __launch_bounds__(256) conv1_im2col_kernel(const float* __restri
   const long long chunk = phase ? rest / 4 : rest;
   const int t1 = phase ? 2 * t + (plane >> 1) : t;
   const int f1 = phase ? 2 * f + (plane & 1) : f;
-  const int b = static_cast<int>(chunk / chunks_per_clip);
-  const int q = static_cast<int>(chunk - (long long)b * chunks_per_clip);
+  int b, F, valid;
+  const float* src;
+  if (cd) {
+    // variable-length batch: the chunk's clip, first frame and valid frames
+    const ChunkDesc c = cd[chunk];
+    b = c.clip;
+    F = mc[b].frames;
+    valid = c.nvalid;
+    src = mel_raw + (long long)n_mels * mc[b].f_off + c.frame0;
+  } else {
+    b = static_cast<int>(chunk / chunks_per_clip);
+    const int q = static_cast<int>(chunk - (long long)b * chunks_per_clip);
+    F = n_frames;
+    valid = chunk_frames;
+    src = mel_raw + (long long)b * n_mels * n_frames + (long long)q * chunk_frames;
+  }
   const float mfloor = ordered_to_float(clip_max[b]) - 8.0f;
-  const float* src = mel_raw + (long long)b * n_mels * n_frames + (long long)q * chunk_frames;
   float v[16];
 #pragma unroll
   for (int kh = 0; kh < 3; ++kh)
 #pragma unroll
     for (int kw = 0; kw < 3; ++kw) {
-      // tap (kh, kw): frequency 2 f1 + kh - 1, time 2 t1 + kw - 1
+      // tap (kh, kw): frequency 2 f1 + kh - 1, time 2 t1 + kw - 1; frames
+      // past the chunk's valid ones are the convolution's zero padding
       const int m = 2 * f1 + kh - 1, tt = 2 * t1 + kw - 1;
       float x = 0.f;
-      if (m >= 0 && m < n_mels && tt >= 0 && tt < chunk_frames)
-        x = (fmaxf(__ldg(src + (long long)m * n_frames + tt), mfloor) + 4.0f) * 0.25f;
+      if (m >= 0 && m < n_mels && tt >= 0 && tt < valid)
+        x = (fmaxf(__ldg(src + (long long)m * F + tt), mfloor) + 4.0f) * 0.25f;
       v[kh * 3 + kw] = x;
     }
 #pragma unroll
@@ -77,7 +92,95 @@ cudaError_t launch_conv1_im2col(const float* mel_raw, const unsigned int* clip_m
   if (rows == 0) return cudaSuccess;
   const unsigned blocks = static_cast<unsigned>((rows + 255) / 256);
   return launch_pdl(conv1_im2col_kernel, dim3(blocks), dim3(256), 0, st, mel_raw, clip_max, n_mels, n_frames,
-                    chunk_frames, chunks_per_clip, T1, F1, rows, phase ? 1 : 0, a);
+                    chunk_frames, chunks_per_clip, T1, F1, rows, phase ? 1 : 0, (const ChunkDesc*)nullptr,
+                    (const MelClip*)nullptr, a);
+}
+
+cudaError_t launch_conv1_im2col_varlen(const float* mel_raw, const unsigned int* clip_max, int n_chunks, int n_mels,
+                                       int chunk_frames, int phase, const ChunkDesc* cd, const MelClip* mc, bf16* a,
+                                       cudaStream_t st) {
+  const int T1 = (chunk_frames - 1) / 2 + 1, F1 = (n_mels - 1) / 2 + 1;
+  if (phase && (T1 % 2 || F1 % 2)) return cudaErrorInvalidValue;
+  const long long rows = (long long)n_chunks * T1 * F1;
+  if (rows == 0) return cudaSuccess;
+  const unsigned blocks = static_cast<unsigned>((rows + 255) / 256);
+  return launch_pdl(conv1_im2col_kernel, dim3(blocks), dim3(256), 0, st, mel_raw, clip_max, n_mels, 0, chunk_frames,
+                    1, T1, F1, rows, phase ? 1 : 0, cd, mc, a);
+}
+
+// ---------------------------------------------------------- short chunks
+// A chunk with fewer than chunk_frames valid frames is computed in the
+// layout of a whole one.  Its conv1 / conv2 output rows at or past the short
+// chunk's own output length are zeroed, so that the next convolution reads
+// zero padding there exactly as it would at the end of the short input
+// (rows before that length only read valid inputs or that padding).
+// level 1: conv1 output (length ceil(L / 2)), level 2: conv2 output
+// (ceil(ceil(L / 2) / 2)).  One block per chunk; whole chunks return at once.
+__global__ void mask_short_chunks_kernel(bf16* __restrict__ act, const ChunkDesc* __restrict__ cd, int chunk_frames,
+                                         int level, int T, int F, int C, int phase) {
+  pdl_wait();
+  pdl_trigger();
+  const int c = blockIdx.x;
+  const int L = cd[c].nvalid;
+  if (L >= chunk_frames) return;
+  int tv = (L + 1) / 2;
+  if (level == 2) tv = (tv + 1) / 2;
+  if (tv >= T) return;
+  const uint4 z = make_uint4(0, 0, 0, 0);
+  if (!phase) {
+    // rows [tv, T) of the chunk's [T][F][C] block are contiguous
+    uint4* p = reinterpret_cast<uint4*>(act + ((long long)c * T + tv) * F * C);
+    const long long n16 = (long long)(T - tv) * F * C / 8;
+    for (long long j = threadIdx.x; j < n16; j += blockDim.x) p[j] = z;
+  } else {
+    // parity planes [4][T/2][F/2][C]: plane (pt, pf) holds t = 2 th + pt
+    const int TH = T / 2, FH = F / 2;
+    for (int pl = 0; pl < 4; ++pl) {
+      const int pt = pl >> 1;
+      const int th0 = tv - pt <= 0 ? 0 : (tv - pt + 1) / 2;
+      if (th0 >= TH) continue;
+      uint4* p = reinterpret_cast<uint4*>(act + (((long long)c * 4 + pl) * TH + th0) * FH * C);
+      const long long n16 = (long long)(TH - th0) * FH * C / 8;
+      for (long long j = threadIdx.x; j < n16; j += blockDim.x) p[j] = z;
+    }
+  }
+}
+
+cudaError_t launch_mask_short_chunks(bf16* act, const ChunkDesc* cd, int n_chunks, int chunk_frames, int level, int T,
+                                     int F, int C, int phase, cudaStream_t st) {
+  if (n_chunks <= 0) return cudaSuccess;
+  if (C % 8 || (phase && (T % 2 || F % 2))) return cudaErrorInvalidValue;
+  return launch_pdl(mask_short_chunks_kernel, dim3(n_chunks), dim3(256), 0, st, act, cd, chunk_frames, level, T, F, C,
+                    phase);
+}
+
+// Valid tokens of every chunk, from the padded conv_out rows [chunk][t3] to
+// the packed token rows of their clips (one warp per padded row).
+__global__ void compact_tokens_kernel(const float* __restrict__ xpad, float* __restrict__ x,
+                                      const ChunkDesc* __restrict__ cd, long long rows, int t3, int d) {
+  pdl_wait();
+  pdl_trigger();
+  const long long r = blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  const int lane = threadIdx.x & 31;
+  const long long c = r / t3;
+  const int j = static_cast<int>(r - c * t3);
+  const ChunkDesc dsc = cd[c];
+  const int L = dsc.nvalid;
+  const int tv = ((((L + 1) / 2) + 1) / 2 + 1) / 2;  // ceil(ceil(ceil(L / 2) / 2) / 2)
+  if (j >= tv) return;
+  const float4* s = reinterpret_cast<const float4*>(xpad + r * d);
+  float4* o = reinterpret_cast<float4*>(x + (long long)(dsc.tok_dst + j) * d);
+  for (int k = lane; k < d / 4; k += 32) o[k] = s[k];
+}
+
+cudaError_t launch_compact_tokens(const float* xpad, float* x, const ChunkDesc* cd, int n_chunks, int t3, int d,
+                                  cudaStream_t st) {
+  const long long rows = (long long)n_chunks * t3;
+  if (rows <= 0) return cudaSuccess;
+  if (d % 4) return cudaErrorInvalidValue;
+  return launch_pdl(compact_tokens_kernel, dim3(static_cast<unsigned>((rows + 7) / 8)), dim3(256), 0, st, xpad, x, cd,
+                    rows, t3, d);
 }
 
 }  // namespace asr

@@ -42,11 +42,23 @@ def test_tokens_match_oracle(gname, secs):
     assert sra.tokens(g, n) == oracle.token_count(g, n)
 
 
-def test_tokens_reject_partial_chunks():
+@pytest.mark.parametrize("n", [16000 + 160, 16000 + 1, 116800, 192160, 16077, 201, 480000 + 3200])
+def test_tokens_partial_chunks_match_oracle(n):
+    for gname in ("moss", "tiny", "whisper_small"):
+        g = synth.GEOMETRIES[gname]
+        assert sra.tokens(g, n) == oracle.token_count(g, n)
+
+
+def test_tokens_reject_too_short():
+    for gname in ("moss", "whisper_small"):
+        assert sra.tokens(synth.GEOMETRIES[gname], 200) == -1
+        assert sra.tokens(synth.GEOMETRIES[gname], 0) == -1
+
+
+@pytest.mark.parametrize("n", [116800, 192160, 16077])
+def test_windows_partial_chunks_match_oracle(n):
     g = synth.GEOMETRIES["moss"]
-    assert sra.tokens(g, 16000 + 160) == -1
-    assert sra.tokens(g, 16000 + 1) == -1
-    assert sra.tokens(synth.GEOMETRIES["whisper_small"], 16000 + 1) == -1
+    assert sra.windows(g, n, 3) == oracle.window_partition(g, n, 3).tolist()
 
 
 @pytest.mark.parametrize("wname", list(synth.WORKLOADS))

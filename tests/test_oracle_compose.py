@@ -125,6 +125,11 @@ CASES = {
     "conv1d_full": (_geom(stem=1, n_mels=80, pos_mode=1, window_tokens=0, proj1_out=0, proj2_out=0,
                           adapter_hidden=0, adapter_out=0), 2),
     "conv1d_w30": (_geom(stem=1, n_mels=80, pos_mode=1, window_tokens=30), 2),
+    # a short last chunk (730 frames: 7 chunks and 30 frames -> 95 tokens)
+    "conv2d_short_chunk": (_geom(window_tokens=20, n_layers=2), 7.3),
+    # a length that is not a whole number of hops (the extra samples only
+    # enter the last frames through the reflect padding)
+    "conv2d_odd_length": (_geom(window_tokens=26), 3.4567),
 }
 
 
@@ -132,7 +137,7 @@ CASES = {
 def test_encode_clip_from_pcm_matches_torch_composition(case):
     g, secs = CASES[case]
     W = synth.make_weights(g, 31, affine=True, std=0.1)
-    pcm = synth.pcm_clip(16000 * secs, 41)
+    pcm = synth.pcm_clip(int(round(16000 * secs)), 41)
     ref = torch_clip(pcm, W, g)
     full = oracle.encode_clip(pcm, W, g)
     assert full.shape == ref.shape

@@ -77,8 +77,15 @@ def test_token_counts_closed_form():
     w = synth.GEOMETRIES["whisper_small"]
     for sec in (1, 30):
         assert oracle.token_count(w, 16000 * sec) == 16000 * sec // 320
+    # a short last chunk of L frames gives ceil(ceil(ceil(L/2)/2)/2) tokens;
+    # samples past the last whole hop add no frame
+    assert oracle.token_count(g, 16000 + 160) == 13 + 1            # 101 frames
+    assert oracle.token_count(g, 116800) == 7 * 13 + 4             # 730 frames: 30 -> 15 -> 8 -> 4
+    assert oracle.token_count(g, 192160) == 12 * 13 + 1            # 1201 frames
+    assert oracle.token_count(g, 16000 + 159) == 13
+    assert oracle.token_count(w, 16000 + 160) == 51                # 101 frames -> ceil(101 / 2)
     with pytest.raises(ValueError):
-        oracle.token_count(g, 16000 + 160)
+        oracle.token_count(g, 200)                                 # reflect padding needs > 200 samples
 
 
 def test_golden_shape_pins():
