@@ -259,6 +259,41 @@ asr_status asr_splice_embeddings(const int32_t* ids, int64_t n_ids, int32_t plac
                                  void* out, int out_dtype, void* ws, size_t ws_bytes, void* stream);
 asr_status asr_splice_check(const void* ws, void* stream);
 
+/* ---- streaming ---------------------------------------------------------------
+ * Live input, encoded one attention window at a time (the windows are
+ * independent: "MOSS-Transcribe-preview-2B-GGUF", Architecture, "Audio
+ * encoder", windowed block-diagonal attention).  Conv2d stem with
+ * window_tokens a whole number of chunks' tokens only (ASR_E_UNSUPPORTED
+ * otherwise).  Window j covers the stream's mel frames [j WF, (j + 1) WF),
+ * WF = window_tokens / (tokens per chunk) * chunk_frames (800 frames = 8 s for
+ * the 104-token windows of 100-frame chunks).  Its frames are the centred
+ * STFT frames of the whole stream (reflection only at the stream's start and
+ * end), and its log-mel is normalised by the maximum over its own frames --
+ * the offline forward normalises by the clip's maximum instead, which a live
+ * stream cannot know in advance.  A window is encoded as soon as the samples
+ * its last frame reads have arrived ((j + 1) WF - 1) hop + n_fft / 2 samples).
+ *  asr_stream_create: state on the encoder `e` (which must outlive it); its
+ *      sample buffer comes from the encoder's allocator and grows as needed.
+ *  asr_stream_push: appends n device float32 samples (n >= 0), encodes every
+ *      window that became ready and writes their rows, packed in window order,
+ *      to device float32 out [*out_rows, D_out] (out_cap_rows rows
+ *      available; asr_stream_window_tokens() rows per window); the workspace
+ *      must hold asr_stream_workspace_size(e, windows) for the number of
+ *      windows that become ready.  Asynchronous on `stream`; use one stream
+ *      per stream object.
+ *  asr_stream_finish: encodes the remaining frames as a last, possibly
+ *      short window (a short last chunk as in asr_enc_forward_varlen); after
+ *      it the stream takes no more samples.  Needs > n_fft / 2 samples in all. */
+typedef struct asr_stream asr_stream;
+int64_t asr_stream_window_tokens(const asr_enc* e);
+size_t asr_stream_workspace_size(const asr_enc* e, int windows);
+asr_status asr_stream_create(asr_enc* e, asr_stream** out);
+asr_status asr_stream_push(asr_stream* s, const float* pcm, int64_t n, float* out, int64_t out_cap_rows,
+                           int64_t* out_rows, void* ws, size_t ws_bytes, void* stream);
+asr_status asr_stream_finish(asr_stream* s, float* out, int64_t out_cap_rows, int64_t* out_rows, void* ws,
+                             size_t ws_bytes, void* stream);
+void asr_stream_destroy(asr_stream* s);
+
 /* Message of the last failure on `e` (or process-wide when e is NULL). */
 const char* asr_enc_last_error(const asr_enc* e);
 

@@ -26,6 +26,10 @@ function.  Pins (in tests/test_oracle_*.py) for each function:
                                  ceil(T/104) windows per clip
   splice_embeddings              a hand-written prompt whose spliced rows are
                                  listed explicitly in the test
+  encode_stream                  == encode_clip for a stream of one window;
+                                 longer streams vs a float64 torch
+                                 composition (torch.stft, torchaudio
+                                 filterbank, per-window normalisation)
 Parity unpinned: the per-chunk position reading (pos_mode 0) and the
 channel-major flatten before conv_out are conventions that only trained
 weights could distinguish; they are fixed by reading, not by a pin.
@@ -42,7 +46,7 @@ __all__ = [
     "mel_filterbank", "log_mel", "conv2d", "conv1d", "gelu", "silu", "layer_norm", "sinusoids",
     "linear", "token_count", "window_partition", "attention_windows", "attention_masked", "window_mask",
     "encoder_layer", "stem_conv2d_chunked", "stem_conv1d", "encode_tokens", "encode_clip", "forward",
-    "as64", "splice_embeddings",
+    "as64", "splice_embeddings", "encode_stream",
 ]
 
 SAMPLE_RATE = 16000
@@ -505,6 +509,36 @@ def encode_clip(pcm: np.ndarray, W, geom, taps=None, windows=None) -> np.ndarray
     if taps is not None:
         taps["stem"] = x.copy()
     return encode_tokens(x, W, geom, cu_rel, taps)
+
+
+def encode_stream(pcm: np.ndarray, W, geom) -> np.ndarray:
+    """Streaming encoder output of one stream of PCM, [T, D_out].
+
+    The stream is cut into attention windows of window_tokens tokens, i.e.
+    window_tokens / (tokens per chunk) conv chunks of mel frames (800 frames,
+    8 s, for windows of 104 tokens), and each window is encoded on its own
+    ([MOSS] Architecture, "Audio encoder": windowed, block-diagonal attention,
+    so windows are independent once their tokens exist).  Reading for live
+    input: the frames are the centred STFT frames of the whole stream (the
+    stream's own samples on both sides of a window boundary, reflect padding
+    only at the stream's start and end), but each window's log-mel is clamped
+    and scaled with the maximum over that window's frames, since a live stream
+    cannot know the maximum of audio that has not arrived.  The last window
+    may be short (a short last chunk, as for any clip).
+    """
+    t_chunk = token_count(geom, geom.chunk_frames * geom.hop)
+    if geom.stem != 0 or not geom.window_tokens or geom.window_tokens % t_chunk:
+        raise ValueError("streaming needs the chunked stem and windows of whole chunks")
+    wf = geom.window_tokens // t_chunk * geom.chunk_frames
+    p = power_spectrum(pcm, geom.n_fft, geom.hop)                 # [F, n_fft/2 + 1], whole stream
+    lg = np.log10(np.maximum(p @ mel_filterbank(geom.n_fft // 2 + 1, geom.n_mels), 1e-10))
+    outs = []
+    for f0 in range(0, lg.shape[0], wf):
+        w = lg[f0:f0 + wf]
+        w = np.maximum(w, w.max() - 8.0)
+        x = stem_conv2d_chunked(((w + 4.0) / 4.0).T, W, geom)
+        outs.append(encode_tokens(x, W, geom, np.array([0, x.shape[0]], dtype=np.int32)))
+    return np.concatenate(outs, axis=0)
 
 
 def forward(pcm: np.ndarray, W, geom, taps=None) -> np.ndarray:

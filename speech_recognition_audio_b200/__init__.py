@@ -15,13 +15,14 @@ The entry points mirror ``include/asr_enc.h`` and ``include/asr_ops.h``:
   log_mel, linear, layer_norm, attention,
   wait_probe                               kernel-level ops
   splice_embeddings                        asr_splice_embeddings / asr_splice_check
+  Stream(encoder).push / finish            asr_stream_* (live input, window by window)
 """
 from __future__ import annotations
 
 import ctypes
 import os
 
-__all__ = ["lib", "LIB_PATH", "AsrError", "Geometry", "tokens", "windows", "weight_names", "Encoder",
+__all__ = ["lib", "LIB_PATH", "AsrError", "Geometry", "tokens", "windows", "weight_names", "Encoder", "Stream",
            "log_mel", "linear", "layer_norm", "attention", "gelu", "wait_probe", "splice_embeddings", "TAP_MEL", "TAP_STEM",
            "TAP_LAYER0", "TAP_ENCODER", "TAP_HEAD", "EPI_BF16", "EPI_BF16_GELU", "EPI_F32_RESID",
            "EPI_F32", "EPI_SWIGLU"]
@@ -95,6 +96,12 @@ def _load():
         "asr_op_attention": (I, [P, P, I, I, I64, I, P, P, SZ, P]),
         "asr_op_gelu": (I, [P, P, I64, P]),
         "asr_op_wait_probe": (I, [I64, P, P]),
+        "asr_stream_window_tokens": (I64, [P]),
+        "asr_stream_workspace_size": (SZ, [P, I]),
+        "asr_stream_create": (I, [P, ctypes.POINTER(P)]),
+        "asr_stream_push": (I, [P, P, I64, P, I64, ctypes.POINTER(I64), P, SZ, P]),
+        "asr_stream_finish": (I, [P, P, I64, ctypes.POINTER(I64), P, SZ, P]),
+        "asr_stream_destroy": (None, [P]),
         "asr_splice_ws_size": (SZ, [I64]),
         "asr_splice_embeddings": (I, [P, I64, ctypes.c_int32, P, I, I, P, I64, I, P, I, P, SZ, P]),
         "asr_splice_check": (I, [P, P]),
@@ -434,3 +441,74 @@ def splice_embeddings(ids, placeholder: int, table, frames, out_dtype=None, stre
     if check:
         _check(lib.asr_splice_check(_ptr(ws), st))
     return out
+
+
+class Stream:
+    """Live input on an Encoder: push() device float32 samples as they arrive;
+    each call returns the rows of the attention windows that became ready
+    (CUDA float32 [rows, D_out]); finish() returns the rows of the last,
+    possibly short, window.  See asr_enc.h, streaming."""
+
+    def __init__(self, encoder, stream=None):
+        self.enc = encoder
+        self.wtok = int(lib.asr_stream_window_tokens(encoder.handle))
+        if self.wtok <= 0:
+            raise AsrError(2, "streaming needs the chunked conv2d stem and windows of whole chunks")
+        g = encoder.geometry
+        self.win_samples = self.wtok // 13 * g.chunk_frames * g.hop
+        self.half, self.hop = g.n_fft // 2, g.hop
+        h = ctypes.c_void_p()
+        _check(lib.asr_stream_create(encoder.handle, ctypes.byref(h)), encoder.handle)
+        self.handle = h
+        self.total = 0
+        self.done = 0
+        self.stream = stream
+        self._ws = None
+
+    def _ws_for(self, windows):
+        import torch
+        need = int(lib.asr_stream_workspace_size(self.enc.handle, max(windows, 1)))
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = None
+            self._ws = torch.empty(need, dtype=torch.uint8, device=torch.device("cuda", self.enc.device))
+        return self._ws
+
+    def _ready(self, total):
+        k = 0
+        while (self.done + k + 1) * self.win_samples - self.hop + self.half <= total:
+            k += 1
+        return k
+
+    def push(self, pcm):
+        import torch
+        if pcm.dtype != torch.float32 or not pcm.is_cuda or pcm.dim() != 1 or not pcm.is_contiguous():
+            raise ValueError("pcm must be a contiguous 1-D CUDA float32 tensor")
+        k = self._ready(self.total + pcm.numel())
+        out = torch.empty((max(k, 1) * self.wtok, self.enc.d_out), dtype=torch.float32, device=pcm.device)
+        ws = self._ws_for(k)
+        rows = ctypes.c_int64()
+        _check(lib.asr_stream_push(self.handle, _ptr(pcm), pcm.numel(), _ptr(out), out.shape[0], ctypes.byref(rows),
+                                   _ptr(ws), ws.numel(), _stream(self.stream)), self.enc.handle)
+        self.total += pcm.numel()
+        self.done += k
+        return out[: rows.value]
+
+    def finish(self):
+        import torch
+        out = torch.empty((self.wtok, self.enc.d_out), dtype=torch.float32, device=torch.device("cuda", self.enc.device))
+        ws = self._ws_for(1)
+        rows = ctypes.c_int64()
+        _check(lib.asr_stream_finish(self.handle, _ptr(out), out.shape[0], ctypes.byref(rows), _ptr(ws), ws.numel(),
+                                     _stream(self.stream)), self.enc.handle)
+        return out[: rows.value]
+
+    def close(self):
+        if getattr(self, "handle", None):
+            lib.asr_stream_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

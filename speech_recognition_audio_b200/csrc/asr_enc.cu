@@ -171,6 +171,15 @@ int64_t chunk_tokens(int64_t L) { return conv_len(conv_len(conv_len(L, 3, 2, 1),
 
 // Tokens per clip, or -1.  frames = floor(n / hop) (the trailing STFT frame
 // dropped); the conv2d stem's last chunk may be short.
+int64_t tokens_from_frames(const asr_geometry* g, int64_t frames) {
+  if (frames <= 0) return -1;
+  if (g->stem == ASR_STEM_CONV2D_CHUNKED) {
+    const int64_t full = frames / g->chunk_frames, rest = frames % g->chunk_frames;
+    return full * chunk_tokens(g->chunk_frames) + (rest ? chunk_tokens(rest) : 0);
+  }
+  return conv_len(conv_len(frames, 3, 1, 1), 3, 2, 1);
+}
+
 int64_t tokens_per_clip(const asr_geometry* g, int64_t n) {
   if (!geom_valid(g, nullptr) || n <= g->n_fft / 2) return -1;
   const int64_t frames = n / g->hop;
@@ -638,7 +647,11 @@ bool make_plan(const asr_enc* e, int64_t n, int B, Plan* p) {
 // samples.  Conv buffers hold every chunk at full size (a short last chunk
 // padded); conv_out writes padded token rows, compacted into the clips'
 // packed rows before the tower.
-bool make_plan_varlen(const asr_enc* e, const int64_t* ns, int B, Plan* p) {
+//  s_offs, lefts (optional): clip b's samples start at pcm + s_offs[b] with
+//  lefts[b] real samples before them (streamed windows); by default the clips
+//  are packed back to back with no history.
+bool make_plan_varlen(const asr_enc* e, const int64_t* ns, int B, Plan* p, const int64_t* s_offs = nullptr,
+                      const int* lefts = nullptr) {
   const asr_geometry* g = &e->g;
   if (g->stem != ASR_STEM_CONV2D_CHUNKED || !ns || B <= 0) return false;
   p->varlen = true;
@@ -658,13 +671,15 @@ bool make_plan_varlen(const asr_enc* e, const int64_t* ns, int B, Plan* p) {
   p->has_short = false;
   for (int b = 0; b < B; ++b) {
     const int64_t n = ns[b];
-    const int64_t tb = tokens_per_clip(g, n);
+    // a clip with real history before it (a streamed window) needs only one hop
+    const int64_t tb = (lefts && lefts[b] >= g->n_fft / 2) ? tokens_from_frames(g, n / g->hop) : tokens_per_clip(g, n);
     if (tb <= 0) return false;
     const int64_t F = n / g->hop, K = (F + cf - 1) / cf;
     const int64_t W = w ? (tb + w - 1) / w : 1;
     if (F % cf) p->has_short = true;
     VarClip& v = p->clips[b];
-    v.s_off = s; v.n = n; v.f_off = f; v.frames = (int)F; v.g_off = (int)groups;
+    v.s_off = s_offs ? s_offs[b] : s; v.n = n; v.f_off = f; v.frames = (int)F; v.g_off = (int)groups;
+    v.left = lefts ? lefts[b] : 0;
     v.chunk_off = (int)ch; v.chunks = (int)K; v.tok_off = (int)tok; v.tokens = (int)tb;
     v.win_off = (int)win; v.wins = (int)W;
     maxseg = std::max<int>(maxseg, (int)(w ? std::min<int64_t>(w, tb) : tb));
@@ -964,7 +979,8 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
       ASR_K(PC_ATTN, ASR_LAUNCH(e, launch_attention_tc(e->maps.qkv, qkv, cu, p.nwin, g->n_heads, att, e->status,
                                                        kWaitLimitNs, st)));
     else
-      ASR_K(PC_ATTN, ASR_LAUNCH(e, launch_attention(qkv, cu, p.nwin, p.max_win, g->n_heads, att, st)));
+      ASR_K(PC_ATTN, ASR_LAUNCH(e, launch_attention_fa(e->maps.qkv, cu, p.nwin, p.max_win, g->n_heads, att, e->status,
+                                                       kWaitLimitNs, st)));
     ASR_K(PC_GEMM_O, ASR_TRY(gemm(e, &e->maps.att, nullptr, lw.o, p.T, x, d, lw.bo, nullptr, 1, EPI_RESID, st, &e->maps.o_x)));
     ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, lw.ln2g, lw.ln2b, p.T, d, g->ln_eps, h, false, st)));
     ASR_K(PC_GEMM_FC1, ASR_TRY(gemm(e, &e->maps.h, nullptr, lw.fc1, p.T, ff, g->d_ffn, lw.b1, nullptr, 1, EPI_GELU, st, &e->maps.o_ff)));
@@ -1272,15 +1288,15 @@ asr_status asr_op_attention(const void* qkv, const int32_t* cu, int n_seg, int m
     return fail(nullptr, ASR_E_INVAL, "attention: bad arguments");
   if (!ws || ws_bytes < 256) return fail(nullptr, ASR_E_WORKSPACE, "attention: workspace too small");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (max_seg <= 128) {
-    CUtensorMap m;
-    if (!make_tmap_qkv(&m, qkv, T, H)) return fail(nullptr, ASR_E_INVAL, "attention: TMA descriptor encoding failed");
-    ASR_CUDA(nullptr, cudaMemsetAsync(ws, 0, 4, st));
+  CUtensorMap m;
+  if (!make_tmap_qkv(&m, qkv, T, H)) return fail(nullptr, ASR_E_INVAL, "attention: TMA descriptor encoding failed");
+  ASR_CUDA(nullptr, cudaMemsetAsync(ws, 0, 4, st));
+  if (max_seg <= 128)
     ASR_CUDA(nullptr, launch_attention_tc(m, static_cast<const bf16*>(qkv), cu, n_seg, H, static_cast<bf16*>(out),
                                           static_cast<int*>(ws), kWaitLimitNs, st));
-  } else {
-    ASR_CUDA(nullptr, launch_attention(static_cast<const bf16*>(qkv), cu, n_seg, max_seg, H, static_cast<bf16*>(out), st));
-  }
+  else
+    ASR_CUDA(nullptr, launch_attention_fa(m, cu, n_seg, max_seg, H, static_cast<bf16*>(out), static_cast<int*>(ws),
+                                          kWaitLimitNs, st));
   return ASR_OK;
 }
 
@@ -1386,6 +1402,195 @@ asr_status asr_op_wait_probe(int64_t limit_ns, int* status_dev, void* stream) {
     return fail(nullptr, ASR_E_INVAL, "wait_probe: bad arguments (limit 1 ns .. 10 s)");
   ASR_CUDA(nullptr, launch_wait_probe((unsigned long long)limit_ns, status_dev, static_cast<cudaStream_t>(stream)));
   return ASR_OK;
+}
+
+
+}  // extern "C"
+
+// ---- streaming ------------------------------------------------------------
+// A live stream is encoded one attention window at a time (the windows are
+// independent: "MOSS-Transcribe-preview-2B-GGUF", Architecture, "Audio
+// encoder", windowed block-diagonal attention).  Window j covers the stream's
+// mel frames [j WF, (j + 1) WF), WF = window_tokens / tokens-per-chunk *
+// chunk_frames (800 frames, 8 s, for 104-token windows of 100-frame chunks).
+// Its frames are the centred frames of the whole stream (real samples on
+// both sides, reflection only at the stream's start and end), and its log-mel
+// is normalised by the maximum over its own frames, so a window can be
+// encoded as soon as the samples its last frame reads have arrived:
+// ((j + 1) WF - 1) hop + n_fft / 2 of them (128040 for window 0).  Each
+// ready window is one clip of a variable-length forward whose samples start
+// at the window's first frame centre with n_fft / 2 real samples of history
+// before it (none for window 0).
+struct asr_stream {
+  asr_enc* e = nullptr;
+  float* buf[2] = {nullptr, nullptr};
+  size_t cap = 0;            // floats per buffer
+  int cur = 0;
+  int64_t base = 0;          // absolute index of buf[cur][0]
+  int64_t len = 0;           // samples held in buf[cur]
+  int64_t total = 0;         // samples pushed
+  int64_t next_win = 0;      // next window to encode
+  int wf = 0;                // frames per window
+  int64_t wtok = 0;          // tokens of a whole window
+  bool finished = false;
+};
+
+namespace {
+
+void stream_free_bufs(asr_stream* s) {
+  for (float*& b : s->buf) {
+    if (!b) continue;
+    if (s->e->free_fn)
+      s->e->free_fn(s->e->ctx, b);
+    else if (!s->e->alloc)
+      cudaFree(b);
+    b = nullptr;
+  }
+}
+
+void* stream_alloc(asr_enc* e, size_t bytes) {
+  if (e->alloc) return e->alloc(e->ctx, bytes);
+  void* p = nullptr;
+  return cudaMalloc(&p, bytes) == cudaSuccess ? p : nullptr;
+}
+
+// Stream windows j0 .. j0 + k - 1 (k >= 1; `final` = the last one ends the
+// stream) as one variable-length forward writing k windows' rows to `out`.
+asr_status stream_encode(asr_stream* s, int64_t j0, int k, bool final, float* out, int64_t out_cap, int64_t* rows,
+                         void* ws, size_t ws_bytes, cudaStream_t st) {
+  asr_enc* e = s->e;
+  const int hop = e->g.hop, half = e->g.n_fft / 2;
+  std::vector<int64_t> ns(k), offs(k);
+  std::vector<int> lefts(k);
+  for (int i = 0; i < k; ++i) {
+    // the window's first frame is centred on sample `start`; a whole window's
+    // last frame reads up to start + (WF - 1) hop + n_fft / 2 - 1, and that
+    // length gives exactly WF frames (hop <= n_fft / 2 < 2 hop)
+    const int64_t start = (j0 + i) * s->wf * (int64_t)hop;
+    const bool last = final && i == k - 1;
+    ns[i] = last ? s->total - start : (int64_t)(s->wf - 1) * hop + half;
+    offs[i] = start - s->base;
+    lefts[i] = start > 0 ? half : 0;
+  }
+  Plan p;
+  if (!make_plan_varlen(e, ns.data(), k, &p, offs.data(), lefts.data()))
+    return fail(e, ASR_E_UNSUPPORTED, "stream: window plan failed");
+  if (p.T > out_cap) return fail(e, ASR_E_INVAL, "stream: out holds %lld rows, %lld needed", (long long)out_cap, (long long)p.T);
+  if (!ws || ws_bytes < p.total || (reinterpret_cast<uintptr_t>(ws) & 255))
+    return fail(e, ASR_E_WORKSPACE, "stream: workspace %zu bytes < %zu needed (or not 256-byte aligned)", ws_bytes, p.total);
+  ASR_TRY(run_forward(e, s->buf[s->cur], p, out, static_cast<char*>(ws), st));
+  e->last_stream = st;
+  e->have_last = true;
+  e->last_plan = p;
+  e->last_ws = ws;
+  *rows = p.T;
+  return ASR_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t asr_stream_window_tokens(const asr_enc* e) {
+  if (!e || e->g.stem != ASR_STEM_CONV2D_CHUNKED || !e->g.window_tokens) return -1;
+  const int64_t t3 = chunk_tokens(e->g.chunk_frames);
+  return e->g.window_tokens % t3 ? -1 : e->g.window_tokens;
+}
+
+size_t asr_stream_workspace_size(const asr_enc* e, int windows) {
+  if (!e || windows <= 0 || asr_stream_window_tokens(e) <= 0) return 0;
+  const int wf = (int)(e->g.window_tokens / chunk_tokens(e->g.chunk_frames)) * e->g.chunk_frames;
+  const int half = e->g.n_fft / 2;
+  std::vector<int64_t> ns(windows, (int64_t)(wf - 1) * e->g.hop + half), offs(windows, 0);
+  std::vector<int> lefts(windows, half);
+  Plan p;
+  if (!make_plan_varlen(e, ns.data(), windows, &p, offs.data(), lefts.data())) return 0;
+  return p.total;
+}
+
+asr_status asr_stream_create(asr_enc* e, asr_stream** out) {
+  if (!e || !out) return fail(e, ASR_E_INVAL, "stream_create: NULL argument");
+  *out = nullptr;
+  if (asr_stream_window_tokens(e) <= 0)
+    return fail(e, ASR_E_UNSUPPORTED, "streaming needs the chunked conv2d stem and windows of whole chunks");
+  asr_stream* s = new asr_stream();
+  s->e = e;
+  s->wf = (int)(e->g.window_tokens / chunk_tokens(e->g.chunk_frames)) * e->g.chunk_frames;
+  s->wtok = e->g.window_tokens;
+  *out = s;
+  return ASR_OK;
+}
+
+void asr_stream_destroy(asr_stream* s) {
+  if (!s) return;
+  stream_free_bufs(s);
+  delete s;
+}
+
+asr_status asr_stream_push(asr_stream* s, const float* pcm, int64_t n, float* out, int64_t out_cap_rows,
+                           int64_t* out_rows, void* ws, size_t ws_bytes, void* stream) {
+  if (!s || !out_rows || n < 0 || (n > 0 && !pcm)) return fail(s ? s->e : nullptr, ASR_E_INVAL, "stream_push: bad arguments");
+  asr_enc* e = s->e;
+  *out_rows = 0;
+  if (s->finished) return fail(e, ASR_E_INVAL, "stream_push: the stream is finished");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int hop = e->g.hop, half = e->g.n_fft / 2;
+  // room for the new samples (buffers grow through the encoder's allocator)
+  if ((size_t)(s->len + n) > s->cap) {
+    size_t cap = std::max<size_t>(s->cap * 2, (size_t)(s->len + n) + (size_t)s->wf * hop);
+    float* nb[2] = {static_cast<float*>(stream_alloc(e, cap * 4)), static_cast<float*>(stream_alloc(e, cap * 4))};
+    if (!nb[0] || !nb[1]) {
+      for (float* b : nb)
+        if (b) {
+          if (e->free_fn) e->free_fn(e->ctx, b); else if (!e->alloc) cudaFree(b);
+        }
+      return fail(e, ASR_E_NOMEM, "stream_push: buffer allocation of %zu bytes failed", cap * 4);
+    }
+    if (s->len) ASR_CUDA(e, cudaMemcpyAsync(nb[0], s->buf[s->cur], (size_t)s->len * 4, cudaMemcpyDeviceToDevice, st));
+    // the old buffers may still be read by queued work on `stream`
+    ASR_CUDA(e, cudaStreamSynchronize(st));
+    stream_free_bufs(s);
+    s->buf[0] = nb[0];
+    s->buf[1] = nb[1];
+    s->cur = 0;
+    s->cap = cap;
+  }
+  if (n) ASR_CUDA(e, cudaMemcpyAsync(s->buf[s->cur] + s->len, pcm, (size_t)n * 4, cudaMemcpyDeviceToDevice, st));
+  s->len += n;
+  s->total += n;
+  // windows whose last frame's samples have all arrived
+  int64_t k = 0;
+  while ((s->next_win + k + 1) * s->wf * (int64_t)hop - hop + half <= s->total) ++k;
+  if (k == 0) return ASR_OK;
+  ASR_TRY(stream_encode(s, s->next_win, (int)k, false, out, out_cap_rows, out_rows, ws, ws_bytes, st));
+  s->next_win += k;
+  // keep n_fft / 2 samples of history before the next window
+  const int64_t keep = std::max<int64_t>(0, s->next_win * s->wf * (int64_t)hop - half);
+  if (keep > s->base) {
+    const int64_t drop = keep - s->base;
+    const int nxt = s->cur ^ 1;
+    if (s->len - drop > 0)
+      ASR_CUDA(e, cudaMemcpyAsync(s->buf[nxt], s->buf[s->cur] + drop, (size_t)(s->len - drop) * 4,
+                                  cudaMemcpyDeviceToDevice, st));
+    s->cur = nxt;
+    s->len -= drop;
+    s->base = keep;
+  }
+  return ASR_OK;
+}
+
+asr_status asr_stream_finish(asr_stream* s, float* out, int64_t out_cap_rows, int64_t* out_rows, void* ws,
+                             size_t ws_bytes, void* stream) {
+  if (!s || !out_rows) return fail(s ? s->e : nullptr, ASR_E_INVAL, "stream_finish: bad arguments");
+  asr_enc* e = s->e;
+  *out_rows = 0;
+  if (s->finished) return fail(e, ASR_E_INVAL, "stream_finish: the stream is finished");
+  if (s->total <= e->g.n_fft / 2) return fail(e, ASR_E_INVAL, "stream_finish: a stream needs more than n_fft/2 samples");
+  s->finished = true;
+  const int64_t frames_left = s->total / e->g.hop - s->next_win * s->wf;
+  if (frames_left <= 0) return ASR_OK;
+  return stream_encode(s, s->next_win, 1, true, out, out_cap_rows, out_rows, ws, ws_bytes,
+                       static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

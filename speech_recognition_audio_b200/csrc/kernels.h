@@ -43,10 +43,12 @@ struct MelTables {
 
 // One clip of a variable-length batch (log-mel view): samples at pcm + s_off,
 // frames = n / 160 at mel + n_mels * f_off ([n_mels][frames]), and the index
-// of its first 32-frame group.
+// of its first 32-frame group.  `left` samples before pcm + s_off are real
+// audio (a streamed window's history): the centred frames read them instead
+// of reflecting; 0 for a clip that starts there.
 struct MelClip {
   long long s_off, n, f_off;
-  int frames, g_off;
+  int frames, g_off, left;
 };
 struct MelArgs {
   const float* pcm;
@@ -78,6 +80,7 @@ struct ChunkDesc {
 struct VarClip {
   long long s_off, n, f_off;          // samples: offset, count; frames: offset
   int frames, g_off;                   // frames, first 32-frame mel group
+  int left;                            // real samples before s_off (MelClip::left)
   int chunk_off, chunks;               // conv chunks
   int tok_off, tokens;                 // packed token rows
   int win_off, wins;                   // attention windows
@@ -111,11 +114,12 @@ cudaError_t launch_conv1_im2col(const float* mel_raw, const unsigned int* clip_m
 cudaError_t launch_layer_norm(const float* x, const float* g, const float* b, long long M, int D, float eps,
                               void* y, bool out_f32, cudaStream_t st);
 
-cudaError_t launch_attention(const bf16* qkv, const int* cu, int n_seg, int max_seg, int H, bf16* out,
-                             cudaStream_t st);
 // tcgen05 attention for segments of at most 128 tokens (attn_tc.cu).
 bool make_tmap_qkv(CUtensorMap* map, const void* qkv, long long T, int H);
 cudaError_t launch_attention_tc(const CUtensorMap& tm_qkv, const bf16* qkv, const int* cu, int n_seg, int H, bf16* out,
+                                int* status, unsigned long long limit_ns, cudaStream_t st);
+// tcgen05 flash attention for segments of any length (attn_fa.cu).
+cudaError_t launch_attention_fa(const CUtensorMap& tm_qkv, const int* cu, int n_seg, int max_seg, int H, bf16* out,
                                 int* status, unsigned long long limit_ns, cudaStream_t st);
 
 // Audio-embedding splice (splice.cu).  Element types match ASR_DTYPE_*.

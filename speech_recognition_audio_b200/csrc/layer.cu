@@ -1,16 +1,8 @@
-// Per-layer kernels other than the GEMMs: LayerNorm, windowed / full
-// attention, and small helpers.
-//
-// Attention ("MOSS-Transcribe-preview-2B-GGUF", Architecture "Audio encoder":
-// windowed, block-diagonal attention; the whisper-small variant attends over
-// the whole clip): segments are given by cumulative offsets and only a
-// segment's own keys are visited, so the block-diagonal structure costs
-// nothing.  Segments of at most 128 tokens run on the tcgen05 kernel of
-// attn_tc.cu.  Longer ones (the whisper-small variant's 1500-frame clips) run
-// here: QK^T and PV on bf16 tensor cores (mma.sync m16n8k16, fp32
-// accumulate), a flash-style kernel with one block per (64-query tile,
-// segment, head) and an online softmax over 64-key tiles in fp32 registers,
-// keys past the segment end masked to -inf, scale 1/sqrt(64).
+// Per-layer kernels other than the GEMMs and the attention: LayerNorm and
+// small helpers (window offsets, variable-length descriptors, conversions,
+// the device GELU, the bounded-wait probe).  Attention runs on the tcgen05
+// kernels of attn_tc.cu (segments of at most 128 tokens) and attn_fa.cu
+// (longer segments).
 #include "kernels.h"
 
 namespace asr {
@@ -129,186 +121,6 @@ cudaError_t launch_layer_norm(const float* x, const float* g, const float* b, lo
   return out_f32 ? ln_dispatch<true>(D / 128, x, g, b, M, eps, y, st) : ln_dispatch<false>(D / 128, x, g, b, M, eps, y, st);
 }
 
-// ------------------------------------------------------------ attention
-namespace {
-constexpr int BQ = 64, BKV = 64, HD = 64, LDS = HD + 8;
-
-__device__ __forceinline__ void ldsm_x4(uint32_t* r, const void* p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(smem_u32(p)));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t* r, const void* p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(smem_u32(p)));
-}
-__device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-// Copy a 64-row x 64-col bf16 tile (rows >= valid are zero-filled).
-__device__ __forceinline__ void load_tile(bf16* dst, const bf16* src, long long ld, int valid, int tid) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int c = tid + 128 * i;  // 512 chunks of 16 bytes
-    const int r = c >> 3, k = (c & 7) * 8;
-    const bool v = r < valid;
-    cp_async_16_zfill(dst + r * LDS + k, v ? src + r * ld + k : src, v);
-  }
-}
-}  // namespace
-
-__global__ void __launch_bounds__(128) attention_kernel(const bf16* __restrict__ qkv, const int* __restrict__ cu, int H,
-                                                        bf16* __restrict__ out) {
-  __shared__ __align__(16) bf16 Qs[BQ * LDS];
-  __shared__ __align__(16) bf16 Ks[2][BKV * LDS];
-  __shared__ __align__(16) bf16 Vs[2][BKV * LDS];
-  pdl_wait();
-  pdl_trigger();
-  const int seg = blockIdx.y, h = blockIdx.z;
-  const int s0 = cu[seg], L = cu[seg + 1] - s0;
-  const int q0 = blockIdx.x * BQ;
-  if (q0 >= L) return;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const long long ld = 3LL * H * HD;
-  const bf16* qbase = qkv + (long long)(s0 + q0) * ld + h * HD;
-  const bf16* kbase = qkv + (long long)s0 * ld + (H + h) * HD;
-  const bf16* vbase = qkv + (long long)s0 * ld + (2 * H + h) * HD;
-  const int n_kv = (L + BKV - 1) / BKV;
-
-  load_tile(Qs, qbase, ld, L - q0, tid);
-  load_tile(Ks[0], kbase, ld, L, tid);
-  load_tile(Vs[0], vbase, ld, L, tid);
-  cp_async_commit();
-
-  const float sl2 = 0.125f * 1.4426950408889634f;  // (1/sqrt(64)) * log2(e)
-  float o[8][4];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-  float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
-  uint32_t qf[4][4];
-  const int g = lane >> 2, t4 = lane & 3;
-
-  for (int j = 0; j < n_kv; ++j) {
-    const int cur = j & 1;
-    if (j + 1 < n_kv) {
-      load_tile(Ks[cur ^ 1], kbase + (long long)(j + 1) * BKV * ld, ld, L - (j + 1) * BKV, tid);
-      load_tile(Vs[cur ^ 1], vbase + (long long)(j + 1) * BKV * ld, ld, L - (j + 1) * BKV, tid);
-      cp_async_commit();
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    if (j == 0) {
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
-        ldsm_x4(qf[ks], Qs + (warp * 16 + (lane & 15)) * LDS + ks * 16 + (lane >> 4) * 8);
-    }
-    // S = Q K^T for this warp's 16 rows x 64 keys.
-    float s[8][4];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
-    const bf16* Kt = Ks[cur];
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        uint32_t kb[4];
-        ldsm_x4(kb, Kt + (16 * p + (lane & 7) + (lane >> 4) * 8) * LDS + ks * 16 + ((lane >> 3) & 1) * 8);
-        mma_bf16_16816(s[2 * p], qf[ks], kb[0], kb[1]);
-        mma_bf16_16816(s[2 * p + 1], qf[ks], kb[2], kb[3]);
-      }
-    }
-    // Mask keys past the segment end; online softmax (base-2, pre-scaled).
-    const int kv0 = j * BKV;
-    float mnew[2] = {mrow[0], mrow[1]};
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int key = kv0 + nt * 8 + 2 * t4 + (e & 1);
-        float v = s[nt][e] * sl2;
-        if (key >= L) v = -INFINITY;
-        s[nt][e] = v;
-        mnew[e >> 1] = fmaxf(mnew[e >> 1], v);
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      mnew[r] = fmaxf(mnew[r], __shfl_xor_sync(0xffffffffu, mnew[r], 1));
-      mnew[r] = fmaxf(mnew[r], __shfl_xor_sync(0xffffffffu, mnew[r], 2));
-    }
-    float corr[2], psum[2] = {0.f, 0.f};
-#pragma unroll
-    for (int r = 0; r < 2; ++r) corr[r] = exp2f(mrow[r] - mnew[r]);
-    uint32_t pf[4][4];
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      const float p0 = exp2f(s[nt][0] - mnew[0]), p1 = exp2f(s[nt][1] - mnew[0]);
-      const float p2 = exp2f(s[nt][2] - mnew[1]), p3 = exp2f(s[nt][3] - mnew[1]);
-      psum[0] += p0 + p1;
-      psum[1] += p2 + p3;
-      pf[nt >> 1][(nt & 1) * 2 + 0] = pack_bf16(p0, p1);
-      pf[nt >> 1][(nt & 1) * 2 + 1] = pack_bf16(p2, p3);
-    }
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      psum[r] += __shfl_xor_sync(0xffffffffu, psum[r], 1);
-      psum[r] += __shfl_xor_sync(0xffffffffu, psum[r], 2);
-      lrow[r] = lrow[r] * corr[r] + psum[r];
-      mrow[r] = mnew[r];
-    }
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      o[nt][0] *= corr[0]; o[nt][1] *= corr[0];
-      o[nt][2] *= corr[1]; o[nt][3] *= corr[1];
-    }
-    // O += P V
-    const bf16* Vt = Vs[cur];
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      // A fragment of P for keys 16ks..16ks+15: (a0,a1) from n-tile 2ks, (a2,a3) from 2ks+1.
-      uint32_t a[4] = {pf[ks][0], pf[ks][1], pf[ks][2], pf[ks][3]};
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        uint32_t vb[4];
-        ldsm_x4_t(vb, Vt + (16 * ks + (lane & 7) + ((lane >> 3) & 1) * 8) * LDS + 16 * p + (lane >> 4) * 8);
-        mma_bf16_16816(o[2 * p], a, vb[0], vb[1]);
-        mma_bf16_16816(o[2 * p + 1], a, vb[2], vb[3]);
-      }
-    }
-    __syncthreads();
-  }
-  // Normalise and store rows inside the segment.
-  const float inv0 = 1.f / lrow[0], inv1 = 1.f / lrow[1];
-  const int r0 = q0 + warp * 16 + g, r1 = r0 + 8;
-  bf16* ob = out + (long long)s0 * (H * HD) + h * HD;
-#pragma unroll
-  for (int nt = 0; nt < 8; ++nt) {
-    const int col = nt * 8 + 2 * t4;
-    if (r0 < L)
-      *reinterpret_cast<uint32_t*>(ob + (long long)r0 * (H * HD) + col) = pack_bf16(o[nt][0] * inv0, o[nt][1] * inv0);
-    if (r1 < L)
-      *reinterpret_cast<uint32_t*>(ob + (long long)r1 * (H * HD) + col) = pack_bf16(o[nt][2] * inv1, o[nt][3] * inv1);
-  }
-}
-
-cudaError_t launch_attention(const bf16* qkv, const int* cu, int n_seg, int max_seg, int H, bf16* out,
-                             cudaStream_t st) {
-  if (n_seg <= 0 || max_seg <= 0 || H <= 0) return cudaErrorInvalidValue;
-  dim3 grid((max_seg + BQ - 1) / BQ, n_seg, H);
-  return launch_pdl(attention_kernel, grid, dim3(128), 0, st, qkv, cu, H, out);
-}
-
 // ------------------------------------------------------------ helpers
 __global__ void fill_windows_kernel(int* cu, int batch, int tpc, int window, int nw) {
   pdl_wait();
@@ -344,6 +156,7 @@ __global__ void varlen_fill_kernel(const VarClipBatch vb, int chunk_frames, int 
     m.f_off = v.f_off;
     m.frames = v.frames;
     m.g_off = v.g_off;
+    m.left = v.left;
     mc[clip] = m;
   }
   for (int q = threadIdx.x; q < v.chunks; q += blockDim.x) {

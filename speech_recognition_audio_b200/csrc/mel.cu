@@ -120,6 +120,7 @@ struct GroupLoc {
   long long n;          // clip samples
   float* out;           // clip mel [n_mels][F]
   int F, f0, nf, clip;
+  int left;             // real samples before x
 };
 
 __device__ __forceinline__ GroupLoc locate(const MelArgs& a, int g) {
@@ -132,6 +133,7 @@ __device__ __forceinline__ GroupLoc locate(const MelArgs& a, int g) {
     L.n = a.n_samples;
     L.x = a.pcm + (long long)L.clip * a.n_samples;
     L.out = a.mel + (long long)L.clip * a.n_mels * a.n_frames;
+    L.left = 0;
   } else {
     int lo = 0, hi = a.batch - 1;  // last clip whose first group is <= g
     while (lo < hi) {
@@ -145,6 +147,7 @@ __device__ __forceinline__ GroupLoc locate(const MelArgs& a, int g) {
     L.n = c.n;
     L.x = a.pcm + c.s_off;
     L.out = a.mel + (long long)a.n_mels * c.f_off;
+    L.left = c.left;
   }
   L.nf = min(G, L.F - L.f0);
   return L;
@@ -155,20 +158,21 @@ __device__ __forceinline__ void cp_async_16(void* dst, const void* src) {
 }
 
 // Issue the cp.async copies of group g's reflect-padded PCM span: 16-byte
-// copies when the span lies inside the clip and is 16-byte aligned (every
-// span is a multiple of 8 samples), else 4-byte copies with the reflection.
+// copies when the span lies inside the clip (or its real history) and is
+// 16-byte aligned (every span is a multiple of 8 samples), else 4-byte
+// copies with the reflection.
 __device__ __forceinline__ void stage_span(const MelArgs& a, int g, float* dst, int tid) {
   const GroupLoc L = locate(a, g);
   const long long base = (long long)L.f0 * HOP - NFFT / 2;
   const int span = (L.nf - 1) * HOP + NFFT;
   const float* src = L.x + base;
-  if (base >= 0 && base + span <= L.n && (reinterpret_cast<uintptr_t>(src) & 15) == 0) {
+  if (base >= -(long long)L.left && base + span <= L.n && (reinterpret_cast<uintptr_t>(src) & 15) == 0) {
     for (int j = tid; j < span / 4; j += THREADS) cp_async_16(dst + 4 * j, src + 4 * j);
   } else {
     for (int j = tid; j < span; j += THREADS) {
       long long i = base + j;
-      if (i < 0) i = -i;
-      if (i >= L.n) i = 2 * (L.n - 1) - i;
+      if (i < -(long long)L.left) i = -i;      // reflect at the start of the audio
+      if (i >= L.n) i = 2 * (L.n - 1) - i;     // and at its end
       cp_async_4(dst + j, L.x + i);
     }
   }

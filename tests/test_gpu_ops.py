@@ -172,6 +172,39 @@ def test_attention(lens, H):
         np.testing.assert_allclose(got[0], q[0, 2 * d:], atol=1e-2)
 
 
+@pytest.mark.parametrize("lens,H", [([200, 300, 257, 1], 2), ([1500], 3), ([130, 129, 384, 385], 1)])
+def test_attention_long_segments(lens, H):
+    """Segments longer than one 128-key tile run on the flash kernel (online
+    softmax over key tiles, O in tensor memory)."""
+    rng = np.random.default_rng(sum(lens) * 7 + H)
+    T = sum(lens)
+    qkv = _bf16(rng.normal(size=(T, 3 * H * 64)))
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    got = sra.attention(qkv.cuda(), torch.from_numpy(cu).cuda(), H).float().cpu().numpy()
+    q = qkv.float().numpy()
+    d = H * 64
+    ref = oracle.attention_windows(q[:, :d], q[:, d:2 * d], q[:, 2 * d:], cu, H)
+    assert np.abs(got - ref).max() <= 2e-2
+
+
+def test_attention_long_segment_rescale():
+    """Keys whose scores grow tile after tile: the running maximum moves by
+    more than the lazy-rescale threshold several times within a row."""
+    rng = np.random.default_rng(3)
+    H, L = 2, 1000
+    q = rng.normal(size=(L, H * 64)) * 0.6
+    k = rng.normal(size=(L, H * 64)) * 0.6
+    k *= (1.0 + np.arange(L) // 128)[:, None] * 1.5      # scores scale up with the key tile
+    v = rng.normal(size=(L, H * 64))
+    qkv = _bf16(np.concatenate([q, k, v], axis=1))
+    cu = np.array([0, L], dtype=np.int32)
+    got = sra.attention(qkv.cuda(), torch.from_numpy(cu).cuda(), H).float().cpu().numpy()
+    x = qkv.float().numpy()
+    d = H * 64
+    ref = oracle.attention_windows(x[:, :d], x[:, d:2 * d], x[:, 2 * d:], cu, H)
+    assert np.abs(got - ref).max() <= 2e-2
+
+
 # ------------------------------------------------------------------ GELU
 def test_gelu_within_published_bound():
     # The device GELU takes erf from Abramowitz & Stegun 7.1.28 (|error| <= 3e-7),

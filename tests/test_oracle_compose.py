@@ -156,3 +156,42 @@ def test_forward_stacks_independent_clips():
     assert out.shape == (2, 39, g.adapter_out)
     for b in range(2):
         np.testing.assert_allclose(out[b], torch_clip(pcm[b], W, g), rtol=RTOL, atol=ATOL)
+
+
+def _torch_stream(pcm, W, g):
+    """Streaming reference from library routines: torch.stft (centred,
+    reflect, periodic Hann, trailing frame dropped) and the torchaudio Slaney
+    filterbank, each window's log-mel normalised by its own maximum, then the
+    torch stem and tower over the window."""
+    import torchaudio
+    x = _t(pcm)
+    spec = torch.stft(x, 400, 160, window=torch.hann_window(400, periodic=True, dtype=torch.float64),
+                      center=True, pad_mode="reflect", return_complex=True)[:, :-1]
+    fb = torchaudio.functional.melscale_fbanks(201, 0.0, 8000.0, g.n_mels, 16000, norm="slaney",
+                                               mel_scale="slaney").double()
+    lg = torch.log10(torch.clamp((spec.abs() ** 2).T @ fb, min=1e-10))     # [F, M]
+    wf = g.window_tokens // 13 * g.chunk_frames
+    outs = []
+    for f0 in range(0, lg.shape[0], wf):
+        w = lg[f0:f0 + wf]
+        w = torch.maximum(w, w.max() - 8.0)
+        xs = _stem2d(((w + 4.0) / 4.0).T.numpy(), W, g)
+        outs.append(_tower(xs, W, g, _windows(xs.shape[0], 0)))
+    return np.concatenate(outs)
+
+
+def test_encode_stream_one_window_equals_encode_clip():
+    # a stream that fits in one window has the clip's maximum: the offline result
+    g = _geom(window_tokens=26)                     # windows of 2 chunks = 200 frames
+    W = synth.make_weights(g, 33, affine=True, std=0.1)
+    pcm = synth.pcm_clip(31000, 42)                 # 193 frames
+    np.testing.assert_allclose(oracle.encode_stream(pcm, W, g), oracle.encode_clip(pcm, W, g), rtol=1e-12, atol=1e-12)
+
+
+def test_encode_stream_matches_torch_composition():
+    g = _geom(window_tokens=26, n_layers=2)         # windows of 200 frames
+    W = synth.make_weights(g, 34, affine=True, std=0.1)
+    pcm = synth.pcm_clip(16000 * 5 + 1234, 43, speech_like=True)  # 507 frames: windows 200, 200, 107
+    out = oracle.encode_stream(pcm, W, g)
+    assert out.shape[0] == 26 + 26 + 13 + 1
+    np.testing.assert_allclose(out, _torch_stream(pcm, W, g), rtol=RTOL, atol=ATOL)
