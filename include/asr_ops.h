@@ -85,6 +85,19 @@ size_t asr_op_linear_ws_size(void);
 asr_status asr_op_linear(const void* x, const void* w, const float* bias, int64_t M, int N, int K,
                          int epi, int tile_n, void* y, void* ws, size_t ws_bytes, void* stream);
 
+/* The same engine with fp32 operands multiplied as tf32 (tcgen05 kind::tf32:
+ * the tensor cores read each fp32 operand's sign, exponent and top 10
+ * mantissa bits) and fp32 accumulation; the path of geometries with fp32
+ * weights.
+ *  x  device float32 [M, K];  w  device float32 [N, K];  y device float32.
+ *  epi: ASR_EPI_F32 (y = acc + bias), ASR_EPI_BF16_GELU (y = GELU(acc +
+ *  bias), fp32 output), ASR_EPI_F32_RESID (y += acc + bias) or ASR_EPI_SWIGLU
+ *  (y [M, N/2] fp32, rows interleaved as for asr_op_linear).
+ *  tile_n: 0, 256, 128 or 64 (one-SM tiles).  Limits: K % 4 == 0 (16-byte
+ *  rows), N % 16 == 0.  ws: >= 256 bytes (device status word). */
+asr_status asr_op_linear_tf32(const float* x, const float* w, const float* bias, int64_t M, int N, int K, int epi,
+                              int tile_n, float* y, void* ws, size_t ws_bytes, void* stream);
+
 /* LayerNorm over the last axis: y = (x - mean) / sqrt(var + eps) * g + b,
  * x device float32 [M, D], g/b device float32 [D], y device bf16 [M, D]
  * (out_f32 == 0) or float32 (out_f32 != 0).  D must be a multiple of 128 and

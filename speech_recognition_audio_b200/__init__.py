@@ -23,7 +23,7 @@ import ctypes
 import os
 
 __all__ = ["lib", "LIB_PATH", "AsrError", "Geometry", "tokens", "windows", "weight_names", "Encoder", "Stream",
-           "log_mel", "linear", "layer_norm", "attention", "gelu", "wait_probe", "splice_embeddings", "TAP_MEL", "TAP_STEM",
+           "log_mel", "linear", "linear_tf32", "layer_norm", "attention", "gelu", "wait_probe", "splice_embeddings", "TAP_MEL", "TAP_STEM",
            "TAP_LAYER0", "TAP_ENCODER", "TAP_HEAD", "EPI_BF16", "EPI_BF16_GELU", "EPI_F32_RESID",
            "EPI_F32", "EPI_SWIGLU"]
 
@@ -91,6 +91,7 @@ def _load():
         "asr_op_log_mel_noalloc": (I, [P, I64, I, I, P, P]),
         "asr_op_linear_ws_size": (SZ, []),
         "asr_op_linear": (I, [P, P, P, I64, I, I, I, I, P, P, SZ, P]),
+        "asr_op_linear_tf32": (I, [P, P, P, I64, I, I, I, I, P, P, SZ, P]),
         "asr_op_layer_norm": (I, [P, P, P, I64, I, F, P, I, P]),
         "asr_op_attention_ws_size": (SZ, []),
         "asr_op_attention": (I, [P, P, I, I, I64, I, P, P, SZ, P]),
@@ -375,6 +376,22 @@ def linear(x, w, bias=None, epi: int = EPI_BF16, out=None, tile_n: int = 0, stre
     ws = torch.empty(int(lib.asr_op_linear_ws_size()), dtype=torch.uint8, device=x.device)
     _check(lib.asr_op_linear(_ptr(x), _ptr(w), _ptr(bias), M, N, K, epi, int(tile_n), _ptr(out), _ptr(ws),
                              ws.numel(), _stream(stream)))
+    return out
+
+
+def linear_tf32(x, w, bias=None, epi: int = EPI_F32, out=None, tile_n: int = 0, stream=None):
+    """x float32 [M, K], w float32 [N, K] -> epilogue(x w^T + bias) in fp32,
+    multiplied on the tensor cores as tf32 (asr_op_linear_tf32)."""
+    import torch
+    M, K = x.shape
+    N = w.shape[0]
+    if out is None:
+        if epi == EPI_F32_RESID:
+            raise ValueError("EPI_F32_RESID needs `out` (updated in place)")
+        out = torch.empty((M, N // 2 if epi == EPI_SWIGLU else N), dtype=torch.float32, device=x.device)
+    ws = torch.empty(256, dtype=torch.uint8, device=x.device)
+    _check(lib.asr_op_linear_tf32(_ptr(x), _ptr(w), _ptr(bias), M, N, K, epi, int(tile_n), _ptr(out), _ptr(ws),
+                                  ws.numel(), _stream(stream)))
     return out
 
 

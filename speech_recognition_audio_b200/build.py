@@ -20,7 +20,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libasr_enc.so")
 OBJ_DIR = os.path.join(ROOT, "_build")
 
-SOURCES = ["asr_enc.cu", "attn_fa.cu", "attn_tc.cu", "gemm.cu", "layer.cu", "mel.cu", "splice.cu", "stem.cu"]
+SOURCES = ["asr_enc.cu", "attn_f32.cu", "attn_fa.cu", "attn_tc.cu", "gemm.cu", "layer.cu", "mel.cu", "splice.cu", "stem.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-std=c++17", "-O3", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I", INCLUDE]

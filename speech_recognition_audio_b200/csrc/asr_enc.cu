@@ -218,6 +218,10 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct asr_enc {
   asr_geometry g;
+  // Operand kind of every GEMM and element size of the activations between
+  // them: bf16 (bf16 weights), or fp32 with tf32 MMAs (fp32 weights).
+  int kind = KIND_BF16;
+  int es = 2;
   asr_alloc_fn alloc = nullptr;
   asr_free_fn free_fn = nullptr;
   void* ctx = nullptr;
@@ -407,6 +411,9 @@ asr_status asr_enc_create(const asr_geometry* g, const void* const* weights, int
     return bad(fail(e, ASR_E_CUDA, "cudaDeviceGetAttribute failed"));
   if (major != 10) return bad(fail(e, ASR_E_UNSUPPORTED, "this library runs on sm_100 (B200) only; device has sm_%d", major * 10));
 
+  e->kind = g->dtype == ASR_DTYPE_F32 ? KIND_TF32 : KIND_BF16;
+  e->es = e->kind == KIND_TF32 ? 4 : 2;
+  const int rowe = kind_row_elems(e->kind);  // channels per 128-byte row of a conv operand
   const int d = g->d_model, C = g->conv_ch, L = g->n_layers;
   // ---- slab size
   size_t need = 0;
@@ -458,7 +465,11 @@ asr_status asr_enc_create(const asr_geometry* g, const void* const* weights, int
     return v;
   };
   auto gemm_w = [&](GemmB& gb, const std::vector<float>& v, int N, int K) -> bool {
-    gb.ptr = up_bf16(v);
+    gb.kind = e->kind;
+    if (e->kind == KIND_TF32)
+      gb.ptr = up_f32(v);  // fp32 weights stay fp32
+    else
+      gb.ptr = up_bf16(v);
     gb.N = N;
     gb.K = K;
     return cerr == cudaSuccess && gb.ptr && make_weight_maps(gb);
@@ -472,17 +483,20 @@ asr_status asr_enc_create(const asr_geometry* g, const void* const* weights, int
       for (int k = 0; k < 9; ++k) r1[(size_t)o * 16 + k] = w1[(size_t)o * 9 + k];
     if (!gemm_w(e->c1, r1, C, 16)) return cuda_fail("conv1 weight upload / TMA map failed");
     e->c1b = up_f32(next());
-    // Conv-box mode needs F_out | 128 (a 128-row tile = whole output rows).
+    // Conv-box mode needs F_out | 128 (a 128-row tile = whole output rows);
+    // fp32 operands have no gather fallback.
     const int f1 = (int)conv_len(g->n_mels, 3, 2, 1), f2 = (int)conv_len(f1, 3, 2, 1);
     e->box2 = f2 > 0 && 128 % f2 == 0 && (128 / f2) * 2 <= 256 && f2 * 2 <= 256;
     e->box3 = f3 > 0 && 128 % f3 == 0 && (128 / f3) * 2 <= 256 && f3 * 2 <= 256;
     const int t1 = (int)conv_len(g->chunk_frames, 3, 2, 1);
     e->phase2 = e->box2 && t1 % 2 == 0 && f1 % 2 == 0 && f2 == f1 / 2;
+    if (e->kind == KIND_TF32 && !(e->box2 && e->box3))
+      return bad(fail(e, ASR_E_UNSUPPORTED, "fp32 weights need conv outputs whose frequency rows divide 128"));
     for (int layer = 0; layer < 2; ++layer) {
       // [o][c][kh][kw] -> [o][tap = kw*3+kh][c], channels padded to 64 per tap in box mode
       auto w = next();
       const bool box = layer == 0 ? e->box2 : e->box3;
-      const int cp = box ? (C + 63) / 64 * 64 : C;
+      const int cp = box ? (C + rowe - 1) / rowe * rowe : C;
       std::vector<float> r((size_t)C * 9 * cp, 0.0f);
       for (int o = 0; o < C; ++o)
         for (int c = 0; c < C; ++c)
@@ -503,7 +517,7 @@ asr_status asr_enc_create(const asr_geometry* g, const void* const* weights, int
     // Conv1D stem: always conv-box mode (F_out = 1, 128 output frames per tile).
     e->box2 = e->box3 = true;
     const int M = g->n_mels;
-    const int mp = (M + 63) / 64 * 64, dp = (d + 63) / 64 * 64;
+    const int mp = (M + rowe - 1) / rowe * rowe, dp = (d + rowe - 1) / rowe * rowe;
     auto w1 = next();  // [d][c][k] -> [d][k][c] with channels padded to 64
     std::vector<float> r1((size_t)d * 3 * mp, 0.0f);
     for (int o = 0; o < d; ++o)
@@ -583,6 +597,7 @@ asr_status asr_enc_create(const asr_geometry* g, const void* const* weights, int
 namespace {
 
 bool make_plan(const asr_enc* e, int64_t n, int B, Plan* p) {
+  const size_t es = e->es;  // activation element size
   const asr_geometry* g = &e->g;
   const int64_t tc = tokens_per_clip(g, n);
   if (tc <= 0 || B <= 0) return false;
@@ -614,24 +629,24 @@ bool make_plan(const asr_enc* e, int64_t n, int B, Plan* p) {
     p->T2 = (int)conv_len(p->T1, 3, 2, 1); p->F2 = (int)conv_len(p->F1, 3, 2, 1);
     p->T3 = (int)conv_len(p->T2, 3, 2, 1); p->F3 = (int)conv_len(p->F2, 3, 2, 1);
     const size_t C = g->conv_ch;
-    p->off_a1 = take((size_t)p->chunks * p->T1 * p->F1 * 16 * 2);
-    p->off_c1 = take((size_t)p->chunks * p->T1 * p->F1 * C * 2);
-    p->off_c2 = take((size_t)p->chunks * p->T2 * p->F2 * C * 2);
-    p->off_c3 = take((size_t)p->T * p->F3 * C * 2);
+    p->off_a1 = take((size_t)p->chunks * p->T1 * p->F1 * 16 * es);
+    p->off_c1 = take((size_t)p->chunks * p->T1 * p->F1 * C * es);
+    p->off_c2 = take((size_t)p->chunks * p->T2 * p->F2 * C * es);
+    p->off_c3 = take((size_t)p->T * p->F3 * C * es);
   } else {
-    p->off_melT = take((size_t)B * p->F * g->n_mels * 2);
-    p->off_c1 = take((size_t)B * p->F * d * 2);
+    p->off_melT = take((size_t)B * p->F * g->n_mels * es);
+    p->off_c1 = take((size_t)B * p->F * d * es);
   }
   p->off_x = take((size_t)p->T * d * 4);
-  p->off_h = take((size_t)p->T * d * 2);
-  p->off_qkv = take((size_t)p->T * 3 * d * 2);
-  p->off_att = take((size_t)p->T * d * 2);
-  p->off_ff = take((size_t)p->T * g->d_ffn * 2);
+  p->off_h = take((size_t)p->T * d * es);
+  p->off_qkv = take((size_t)p->T * 3 * d * es);
+  p->off_att = take((size_t)p->T * d * es);
+  p->off_ff = take((size_t)p->T * g->d_ffn * es);
   if (g->proj1_out) {
-    p->off_p1 = take((size_t)p->T * g->proj1_out * 2);
-    p->off_p2 = take((size_t)p->T * g->proj2_out * 2);
+    p->off_p1 = take((size_t)p->T * g->proj1_out * es);
+    p->off_p2 = take((size_t)p->T * g->proj2_out * es);
   }
-  if (g->adapter_hidden) p->off_gu = take((size_t)p->T * g->adapter_hidden * 2);
+  if (g->adapter_hidden) p->off_gu = take((size_t)p->T * g->adapter_hidden * es);
   p->tap_bytes[ASR_TAP_MEL] = (size_t)B * g->n_mels * p->F * 4;
   p->tap_bytes[ASR_TAP_STEM] = p->tap_bytes[ASR_TAP_LAYER0] = p->tap_bytes[ASR_TAP_ENCODER] = (size_t)p->T * d * 4;
   p->tap_bytes[ASR_TAP_HEAD] = g->proj2_out ? (size_t)p->T * g->proj2_out * 4 : 0;
@@ -652,6 +667,7 @@ bool make_plan(const asr_enc* e, int64_t n, int B, Plan* p) {
 //  are packed back to back with no history.
 bool make_plan_varlen(const asr_enc* e, const int64_t* ns, int B, Plan* p, const int64_t* s_offs = nullptr,
                       const int* lefts = nullptr) {
+  const size_t es = e->es;  // activation element size
   const asr_geometry* g = &e->g;
   if (g->stem != ASR_STEM_CONV2D_CHUNKED || !ns || B <= 0) return false;
   p->varlen = true;
@@ -709,21 +725,21 @@ bool make_plan_varlen(const asr_enc* e, const int64_t* ns, int B, Plan* p, const
   p->off_chunkd = take((size_t)p->chunks * sizeof(ChunkDesc));
   p->off_cu = take((size_t)(p->nwin + 1) * 4);
   p->off_mel = take((size_t)g->n_mels * p->Ftot * 4);
-  p->off_a1 = take((size_t)p->chunks * p->T1 * p->F1 * 16 * 2);
-  p->off_c1 = take((size_t)p->chunks * p->T1 * p->F1 * C * 2);
-  p->off_c2 = take((size_t)p->chunks * p->T2 * p->F2 * C * 2);
-  p->off_c3 = take((size_t)p->Tpad * p->F3 * C * 2);
+  p->off_a1 = take((size_t)p->chunks * p->T1 * p->F1 * 16 * es);
+  p->off_c1 = take((size_t)p->chunks * p->T1 * p->F1 * C * es);
+  p->off_c2 = take((size_t)p->chunks * p->T2 * p->F2 * C * es);
+  p->off_c3 = take((size_t)p->Tpad * p->F3 * C * es);
   p->off_xpad = take((size_t)p->Tpad * d * 4);
   p->off_x = take((size_t)p->T * d * 4);
-  p->off_h = take((size_t)p->T * d * 2);
-  p->off_qkv = take((size_t)p->T * 3 * d * 2);
-  p->off_att = take((size_t)p->T * d * 2);
-  p->off_ff = take((size_t)p->T * g->d_ffn * 2);
+  p->off_h = take((size_t)p->T * d * es);
+  p->off_qkv = take((size_t)p->T * 3 * d * es);
+  p->off_att = take((size_t)p->T * d * es);
+  p->off_ff = take((size_t)p->T * g->d_ffn * es);
   if (g->proj1_out) {
-    p->off_p1 = take((size_t)p->T * g->proj1_out * 2);
-    p->off_p2 = take((size_t)p->T * g->proj2_out * 2);
+    p->off_p1 = take((size_t)p->T * g->proj1_out * es);
+    p->off_p2 = take((size_t)p->T * g->proj2_out * es);
   }
-  if (g->adapter_hidden) p->off_gu = take((size_t)p->T * g->adapter_hidden * 2);
+  if (g->adapter_hidden) p->off_gu = take((size_t)p->T * g->adapter_hidden * es);
   p->tap_bytes[ASR_TAP_MEL] = 0;  // the mel tap covers uniform batches only
   p->tap_bytes[ASR_TAP_STEM] = p->tap_bytes[ASR_TAP_LAYER0] = p->tap_bytes[ASR_TAP_ENCODER] = (size_t)p->T * d * 4;
   p->tap_bytes[ASR_TAP_HEAD] = g->proj2_out ? (size_t)p->T * g->proj2_out * 4 : 0;
@@ -750,6 +766,8 @@ bool plan_for(const asr_enc* e, const int64_t* ns, int64_t n, int B, Plan* p) {
 asr_status gemm(asr_enc* e, const CUtensorMap* amap, const ConvGather* cg, const GemmB& w, long long M, void* out,
                 long long ldo, const float* bias, const float* pe, int period, int epi, cudaStream_t st,
                 const CUtensorMap* omap, const ConvBox* box = nullptr) {
+  // fp32 operands: every output of the engine is fp32
+  if (e->kind == KIND_TF32 && !(epi & (EPI_OUT_F32 | EPI_RESID))) epi |= EPI_OUT_F32;
   GemmParams p;
   memset(&p, 0, sizeof p);
   p.M = (int)M;
@@ -765,9 +783,11 @@ asr_status gemm(asr_enc* e, const CUtensorMap* amap, const ConvGather* cg, const
   if (box) {
     p.conv_box = 1;
     p.cb = *box;
-    bn = gemm_pick_bn_conv(box->n_sub, w.N, e->num_sms);
+    bn = e->kind == KIND_TF32 ? gemm_pick_bn_tf32(box->n_sub * 128, w.N, e->num_sms)
+                              : gemm_pick_bn_conv(box->n_sub, w.N, e->num_sms);
   } else {
-    bn = gemm_pick_bn((int)M, w.N, e->num_sms, cg != nullptr);
+    bn = e->kind == KIND_TF32 ? gemm_pick_bn_tf32((int)M, w.N, e->num_sms)
+                              : gemm_pick_bn((int)M, w.N, e->num_sms, cg != nullptr);
   }
   cudaError_t r = launch_gemm(amap, w, p, epi, bn, e->num_sms, st, omap);
   if (r != cudaSuccess) return fail(e, ASR_E_CUDA, "gemm launch (N=%d K=%d M=%lld epi=%d bn=%d): %s", w.N, w.K, M, epi, bn, cudaGetErrorString(r));
@@ -818,39 +838,41 @@ asr_status ensure_maps(asr_enc* e, const Plan& p, char* ws) {
   ActMaps& m = e->maps;
   if (m.ws == ws && m.n == p.n && m.batch == p.B && m.T == p.T && m.chunks == p.chunks && m.taps == e->taps) return ASR_OK;
   const asr_geometry* g = &e->g;
-  const int d = g->d_model;
-  bool ok = make_tmap_qkv(&m.qkv, ws + p.off_qkv, p.T, g->n_heads) &&
-            make_tmap_bf16(&m.h, ws + p.off_h, p.T, d, d, 128) &&
-            make_tmap_bf16(&m.att, ws + p.off_att, p.T, d, d, 128) &&
-            make_tmap_bf16(&m.ff, ws + p.off_ff, p.T, g->d_ffn, g->d_ffn, 128);
+  const int d = g->d_model, k = e->kind;
+  const bool f32 = k == KIND_TF32;  // fp32 activations between the GEMMs
+  // (the qkv map feeds the tcgen05 attention, which takes bf16 operands)
+  bool ok = (f32 || make_tmap_qkv(&m.qkv, ws + p.off_qkv, p.T, g->n_heads)) &&
+            make_tmap_act(k, &m.h, ws + p.off_h, p.T, d, d, 128) &&
+            make_tmap_act(k, &m.att, ws + p.off_att, p.T, d, d, 128) &&
+            make_tmap_act(k, &m.ff, ws + p.off_ff, p.T, g->d_ffn, g->d_ffn, 128);
   if (ok && g->stem == ASR_STEM_CONV2D_CHUNKED) {
     const int C = g->conv_ch;
-    ok = make_tmap_bf16(&m.c3, ws + p.off_c3, p.Tpad, (size_t)p.F3 * C, (size_t)p.F3 * C, 128) &&
-         make_tmap_bf16(&m.a1, ws + p.off_a1, (size_t)p.chunks * p.T1 * p.F1, 16, 16, 128);
+    ok = make_tmap_act(k, &m.c3, ws + p.off_c3, p.Tpad, (size_t)p.F3 * C, (size_t)p.F3 * C, 128) &&
+         make_tmap_act(k, &m.a1, ws + p.off_a1, (size_t)p.chunks * p.T1 * p.F1, 16, 16, 128);
     if (ok && e->box2)
-      ok = e->phase2 ? make_tmap_convphase(&m.cin2, ws + p.off_c1, C, p.F1 / 2, p.T1 / 2, 4 * p.chunks, p.F2, 128 / p.F2)
-                     : make_tmap_convbox(&m.cin2, ws + p.off_c1, C, p.F1, p.T1, p.chunks, p.F2, 2, 128 / p.F2, 2);
-    if (ok && e->box3) ok = make_tmap_convbox(&m.cin3, ws + p.off_c2, C, p.F2, p.T2, p.chunks, p.F3, 2, 128 / p.F3, 2);
+      ok = e->phase2 ? make_tmap_convphase(&m.cin2, ws + p.off_c1, C, p.F1 / 2, p.T1 / 2, 4 * p.chunks, p.F2, 128 / p.F2, k)
+                     : make_tmap_convbox(&m.cin2, ws + p.off_c1, C, p.F1, p.T1, p.chunks, p.F2, 2, 128 / p.F2, 2, k);
+    if (ok && e->box3) ok = make_tmap_convbox(&m.cin3, ws + p.off_c2, C, p.F2, p.T2, p.chunks, p.F3, 2, 128 / p.F3, 2, k);
   } else if (ok) {
-    ok = make_tmap_convbox(&m.cin2, ws + p.off_melT, g->n_mels, 1, p.F, p.B, 1, 1, 128, 1) &&
-         make_tmap_convbox(&m.cin3, ws + p.off_c1, d, 1, p.F, p.B, 1, 1, 128, 2);
+    ok = make_tmap_convbox(&m.cin2, ws + p.off_melT, g->n_mels, 1, p.F, p.B, 1, 1, 128, 1, k) &&
+         make_tmap_convbox(&m.cin3, ws + p.off_c1, d, 1, p.F, p.B, 1, 1, 128, 2, k);
   }
   if (ok && g->proj1_out)
-    ok = make_tmap_bf16(&m.p1, ws + p.off_p1, p.T, g->proj1_out, g->proj1_out, 128) &&
-         make_tmap_bf16(&m.p2, ws + p.off_p2, p.T, g->proj2_out, g->proj2_out, 128) &&
-         make_tmap_out(&m.o_p1, ws + p.off_p1, p.T, g->proj1_out, g->proj1_out, false) &&
-         make_tmap_out(&m.o_p2, ws + p.off_p2, p.T, g->proj2_out, g->proj2_out, false);
+    ok = make_tmap_act(k, &m.p1, ws + p.off_p1, p.T, g->proj1_out, g->proj1_out, 128) &&
+         make_tmap_act(k, &m.p2, ws + p.off_p2, p.T, g->proj2_out, g->proj2_out, 128) &&
+         make_tmap_out(&m.o_p1, ws + p.off_p1, p.T, g->proj1_out, g->proj1_out, f32) &&
+         make_tmap_out(&m.o_p2, ws + p.off_p2, p.T, g->proj2_out, g->proj2_out, f32);
   if (ok)
     ok = make_tmap_out(&m.o_x, ws + p.off_x, p.T, d, d, true) &&
-         make_tmap_out(&m.o_qkv, ws + p.off_qkv, p.T, 3 * d, 3 * d, false) &&
-         make_tmap_out(&m.o_ff, ws + p.off_ff, p.T, g->d_ffn, g->d_ffn, false);
+         make_tmap_out(&m.o_qkv, ws + p.off_qkv, p.T, 3 * d, 3 * d, f32) &&
+         make_tmap_out(&m.o_ff, ws + p.off_ff, p.T, g->d_ffn, g->d_ffn, f32);
   if (ok && g->stem == ASR_STEM_CONV2D_CHUNKED)
-    ok = make_tmap_out(&m.o_c1, ws + p.off_c1, (unsigned long long)p.chunks * p.T1 * p.F1, g->conv_ch, g->conv_ch, false) &&
-         make_tmap_out(&m.o_c2, ws + p.off_c2, (unsigned long long)p.chunks * p.T2 * p.F2, g->conv_ch, g->conv_ch, false) &&
-         make_tmap_out(&m.o_c3, ws + p.off_c3, (unsigned long long)p.chunks * p.T3 * p.F3, g->conv_ch, g->conv_ch, false);
+    ok = make_tmap_out(&m.o_c1, ws + p.off_c1, (unsigned long long)p.chunks * p.T1 * p.F1, g->conv_ch, g->conv_ch, f32) &&
+         make_tmap_out(&m.o_c2, ws + p.off_c2, (unsigned long long)p.chunks * p.T2 * p.F2, g->conv_ch, g->conv_ch, f32) &&
+         make_tmap_out(&m.o_c3, ws + p.off_c3, (unsigned long long)p.chunks * p.T3 * p.F3, g->conv_ch, g->conv_ch, f32);
   else if (ok)
-    ok = make_tmap_out(&m.o_c1, ws + p.off_c1, (unsigned long long)p.B * p.F, d, d, false);
-  if (ok && g->adapter_hidden) ok = make_tmap_bf16(&m.gu, ws + p.off_gu, p.T, g->adapter_hidden, g->adapter_hidden, 128);
+    ok = make_tmap_out(&m.o_c1, ws + p.off_c1, (unsigned long long)p.B * p.F, d, d, f32);
+  if (ok && g->adapter_hidden) ok = make_tmap_act(k, &m.gu, ws + p.off_gu, p.T, g->adapter_hidden, g->adapter_hidden, 128);
   if (!ok) {
     m.ws = nullptr;
     return fail(e, ASR_E_CUDA, "TMA descriptor encoding failed (workspace alignment?)");
@@ -872,10 +894,13 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
   int* cu = reinterpret_cast<int*>(ws + p.off_cu);
   float* mel = reinterpret_cast<float*>(ws + p.off_mel);
   float* x = reinterpret_cast<float*>(ws + p.off_x);
-  bf16* h = reinterpret_cast<bf16*>(ws + p.off_h);
-  bf16* qkv = reinterpret_cast<bf16*>(ws + p.off_qkv);
-  bf16* att = reinterpret_cast<bf16*>(ws + p.off_att);
-  bf16* ff = reinterpret_cast<bf16*>(ws + p.off_ff);
+  // activations between the GEMMs: bf16, or fp32 on the tf32 path
+  const bool f32 = e->kind == KIND_TF32;
+  const int RE = kind_row_elems(e->kind), KST = RE / 4;  // conv channel block, MMA step (elements)
+  void* h = ws + p.off_h;
+  void* qkv = ws + p.off_qkv;
+  void* att = ws + p.off_att;
+  void* ff = ws + p.off_ff;
   auto tap = [&](int t) -> float* { return ((e->taps >> t) & 1u) ? reinterpret_cast<float*>(ws + p.off_tap[t]) : nullptr; };
 
   e->launches = 0;
@@ -915,39 +940,40 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
 
   if (g->stem == ASR_STEM_CONV2D_CHUNKED) {
     const int C = g->conv_ch;
-    bf16* c1 = reinterpret_cast<bf16*>(ws + p.off_c1);
-    bf16* c2 = reinterpret_cast<bf16*>(ws + p.off_c2);
-    bf16* c3 = reinterpret_cast<bf16*>(ws + p.off_c3);
-    bf16* a1 = reinterpret_cast<bf16*>(ws + p.off_a1);
+    void* c1 = ws + p.off_c1;
+    void* c2 = ws + p.off_c2;
+    void* c3 = ws + p.off_c3;
+    void* a1 = ws + p.off_a1;
     if (!p.varlen)
       ASR_K(PC_CONV1, ASR_LAUNCH(e, launch_conv1_im2col(mel, clip_max, p.B, g->n_mels, p.F, g->chunk_frames,
-                                                        e->phase2 ? 1 : 0, a1, st)));
+                                                        e->phase2 ? 1 : 0, a1, f32, st)));
     else
       ASR_K(PC_CONV1, ASR_LAUNCH(e, launch_conv1_im2col_varlen(mel, clip_max, p.chunks, g->n_mels, g->chunk_frames,
-                                                               e->phase2 ? 1 : 0, chunkd, mclips, a1, st)));
+                                                               e->phase2 ? 1 : 0, chunkd, mclips, a1, f32, st)));
     ASR_K(PC_CONV1, ASR_TRY(gemm(e, &e->maps.a1, nullptr, e->c1, (long long)p.chunks * p.T1 * p.F1, c1, C, e->c1b,
                                  nullptr, 1, EPI_GELU, st, &e->maps.o_c1)));
     if (p.has_short)
       ASR_K(PC_MISC, ASR_LAUNCH(e, launch_mask_short_chunks(c1, chunkd, p.chunks, g->chunk_frames, 1, p.T1, p.F1, C,
-                                                            e->phase2 ? 1 : 0, st)));
-    const int CB = (C + 63) / 64;
+                                                            e->phase2 ? 1 : 0, e->es, st)));
+    const int CB = (C + RE - 1) / RE;
+    const int k_last = (C - RE * (CB - 1) + KST - 1) / KST;
     if (e->box2) {
       const int TR = 128 / p.F2, tpi = (p.T2 + TR - 1) / TR;
-      ConvBox b2 = {TR, p.F2, p.T2, tpi, p.chunks * tpi, 2, 2, 1, 1, 3, CB, e->phase2 ? 1 : 0, (C - 64 * (CB - 1) + 15) / 16};
+      ConvBox b2 = {TR, p.F2, p.T2, tpi, p.chunks * tpi, 2, 2, 1, 1, 3, CB, e->phase2 ? 1 : 0, k_last};
       ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, &e->maps.cin2, nullptr, e->c2, (long long)p.chunks * p.T2 * p.F2, c2, C, e->c2b, nullptr, 1, EPI_GELU, st, &e->maps.o_c2, &b2)));
     } else {
-      ConvGather cg2 = {c1, p.T1, p.F1, C, p.T2, p.F2, 2, 2, 3, 3, 1, 1};
+      ConvGather cg2 = {static_cast<const bf16*>(c1), p.T1, p.F1, C, p.T2, p.F2, 2, 2, 3, 3, 1, 1};
       ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, nullptr, &cg2, e->c2, (long long)p.chunks * p.T2 * p.F2, c2, C, e->c2b, nullptr, 1, EPI_GELU, st, &e->maps.o_c2)));
     }
     if (p.has_short)
       ASR_K(PC_MISC, ASR_LAUNCH(e, launch_mask_short_chunks(c2, chunkd, p.chunks, g->chunk_frames, 2, p.T2, p.F2, C, 0,
-                                                            st)));
+                                                            e->es, st)));
     if (e->box3) {
       const int TR = 128 / p.F3, tpi = (p.T3 + TR - 1) / TR;
-      ConvBox b3 = {TR, p.F3, p.T3, tpi, p.chunks * tpi, 2, 2, 1, 1, 3, CB, 0, (C - 64 * (CB - 1) + 15) / 16};
+      ConvBox b3 = {TR, p.F3, p.T3, tpi, p.chunks * tpi, 2, 2, 1, 1, 3, CB, 0, k_last};
       ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, &e->maps.cin3, nullptr, e->c3, (long long)p.chunks * p.T3 * p.F3, c3, C, e->c3b, nullptr, 1, EPI_GELU, st, &e->maps.o_c3, &b3)));
     } else {
-      ConvGather cg3 = {c2, p.T2, p.F2, C, p.T3, p.F3, 2, 2, 3, 3, 1, 1};
+      ConvGather cg3 = {static_cast<const bf16*>(c2), p.T2, p.F2, C, p.T3, p.F3, 2, 2, 3, 3, 1, 1};
       ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, nullptr, &cg3, e->c3, (long long)p.chunks * p.T3 * p.F3, c3, C, e->c3b, nullptr, 1, EPI_GELU, st, &e->maps.o_c3)));
     }
     if (!p.varlen) {
@@ -959,30 +985,33 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
     }
   } else {
     if (p.Tc > e->pe_rows) return fail(e, ASR_E_UNSUPPORTED, "conv1d stem: %lld positions > %d", (long long)p.Tc, e->pe_rows);
-    bf16* melT = reinterpret_cast<bf16*>(ws + p.off_melT);
-    bf16* c1 = reinterpret_cast<bf16*>(ws + p.off_c1);
-    ASR_K(PC_MISC, ASR_LAUNCH(e, launch_mel_normalize_transpose(mel, clip_max, p.B, g->n_mels, p.F, melT, st)));
+    void* melT = ws + p.off_melT;
+    void* c1 = ws + p.off_c1;
+    ASR_K(PC_MISC, ASR_LAUNCH(e, launch_mel_normalize_transpose(mel, clip_max, p.B, g->n_mels, p.F, melT, f32, st)));
     const int tpi1 = (p.F + 127) / 128, tpi2 = (int)((p.Tc + 127) / 128);
-    const int CB1 = (g->n_mels + 63) / 64, CBd = (d + 63) / 64;
-    ConvBox b1 = {128, 1, p.F, tpi1, p.B * tpi1, 1, 1, 1, 0, 1, CB1, 0, (g->n_mels - 64 * (CB1 - 1) + 15) / 16};
+    const int CB1 = (g->n_mels + RE - 1) / RE, CBd = (d + RE - 1) / RE;
+    ConvBox b1 = {128, 1, p.F, tpi1, p.B * tpi1, 1, 1, 1, 0, 1, CB1, 0, (g->n_mels - RE * (CB1 - 1) + KST - 1) / KST};
     ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, &e->maps.cin2, nullptr, e->c2, (long long)p.B * p.F, c1, d, e->c2b, nullptr, 1, EPI_GELU, st, &e->maps.o_c1, &b1)));
-    ConvBox b2 = {128, 1, (int)p.Tc, tpi2, p.B * tpi2, 2, 1, 1, 0, 1, CBd, 0, (d - 64 * (CBd - 1) + 15) / 16};
+    ConvBox b2 = {128, 1, (int)p.Tc, tpi2, p.B * tpi2, 2, 1, 1, 0, 1, CBd, 0, (d - RE * (CBd - 1) + KST - 1) / KST};
     ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, &e->maps.cin3, nullptr, e->c3, p.T, x, d, e->c3b, e->pe, (int)p.Tc, EPI_GELU | EPI_OUT_F32 | EPI_PE, st, nullptr, &b2)));
   }
   if (float* t = tap(ASR_TAP_STEM)) ASR_LAUNCH(e, cudaMemcpyAsync(t, x, (size_t)p.T * d * 4, cudaMemcpyDeviceToDevice, st));
 
   for (int l = 0; l < g->n_layers; ++l) {
     const LayerW& lw = e->layers[l];
-    ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, lw.ln1g, lw.ln1b, p.T, d, g->ln_eps, h, false, st)));
+    ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, lw.ln1g, lw.ln1b, p.T, d, g->ln_eps, h, f32, st)));
     ASR_K(PC_GEMM_QKV, ASR_TRY(gemm(e, &e->maps.h, nullptr, lw.qkv, p.T, qkv, 3 * d, lw.bqkv, nullptr, 1, 0, st, &e->maps.o_qkv)));
-    if (p.max_win <= 128)
-      ASR_K(PC_ATTN, ASR_LAUNCH(e, launch_attention_tc(e->maps.qkv, qkv, cu, p.nwin, g->n_heads, att, e->status,
-                                                       kWaitLimitNs, st)));
+    if (f32)
+      ASR_K(PC_ATTN, ASR_LAUNCH(e, launch_attention_f32(static_cast<const float*>(qkv), cu, p.nwin, p.max_win,
+                                                        g->n_heads, static_cast<float*>(att), st)));
+    else if (p.max_win <= 128)
+      ASR_K(PC_ATTN, ASR_LAUNCH(e, launch_attention_tc(e->maps.qkv, static_cast<const bf16*>(qkv), cu, p.nwin, g->n_heads,
+                                                       static_cast<bf16*>(att), e->status, kWaitLimitNs, st)));
     else
-      ASR_K(PC_ATTN, ASR_LAUNCH(e, launch_attention_fa(e->maps.qkv, cu, p.nwin, p.max_win, g->n_heads, att, e->status,
-                                                       kWaitLimitNs, st)));
+      ASR_K(PC_ATTN, ASR_LAUNCH(e, launch_attention_fa(e->maps.qkv, cu, p.nwin, p.max_win, g->n_heads,
+                                                       static_cast<bf16*>(att), e->status, kWaitLimitNs, st)));
     ASR_K(PC_GEMM_O, ASR_TRY(gemm(e, &e->maps.att, nullptr, lw.o, p.T, x, d, lw.bo, nullptr, 1, EPI_RESID, st, &e->maps.o_x)));
-    ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, lw.ln2g, lw.ln2b, p.T, d, g->ln_eps, h, false, st)));
+    ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, lw.ln2g, lw.ln2b, p.T, d, g->ln_eps, h, f32, st)));
     ASR_K(PC_GEMM_FC1, ASR_TRY(gemm(e, &e->maps.h, nullptr, lw.fc1, p.T, ff, g->d_ffn, lw.b1, nullptr, 1, EPI_GELU, st, &e->maps.o_ff)));
     ASR_K(PC_GEMM_FC2, ASR_TRY(gemm(e, &e->maps.ff, nullptr, lw.fc2, p.T, x, d, lw.b2, nullptr, 1, EPI_RESID, st, &e->maps.o_x)));
     if (l == 0)
@@ -994,12 +1023,12 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
     ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, e->lnpg, e->lnpb, p.T, d, g->ln_eps, out, true, st)));
     return ASR_OK;
   }
-  bf16* p1 = reinterpret_cast<bf16*>(ws + p.off_p1);
-  bf16* p2 = reinterpret_cast<bf16*>(ws + p.off_p2);
+  void* p1 = ws + p.off_p1;
+  void* p2 = ws + p.off_p2;
   // Store map of the caller's output (plain stores if it is not 16-byte aligned).
   CUtensorMap o_out_map;
   const CUtensorMap* o_out = make_tmap_out(&o_out_map, out, p.T, d_out(g), d_out(g), true) ? &o_out_map : nullptr;
-  ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, e->lnpg, e->lnpb, p.T, d, g->ln_eps, h, false, st)));
+  ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, e->lnpg, e->lnpb, p.T, d, g->ln_eps, h, f32, st)));
   ASR_K(PC_GEMM_HEAD, ASR_TRY(gemm(e, &e->maps.h, nullptr, e->p1, p.T, p1, g->proj1_out, e->bp1, nullptr, 1, EPI_GELU, st, &e->maps.o_p1)));
   if (!g->adapter_hidden) {
     ASR_K(PC_GEMM_HEAD, ASR_TRY(gemm(e, &e->maps.p1, nullptr, e->p2, p.T, out, g->proj2_out, e->bp2, nullptr, 1, EPI_OUT_F32, st, o_out)));
@@ -1007,8 +1036,13 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
     return ASR_OK;
   }
   ASR_K(PC_GEMM_HEAD, ASR_TRY(gemm(e, &e->maps.p1, nullptr, e->p2, p.T, p2, g->proj2_out, e->bp2, nullptr, 1, 0, st, &e->maps.o_p2)));
-  if (float* t = tap(ASR_TAP_HEAD)) ASR_K(PC_MISC, ASR_LAUNCH(e, launch_bf16_to_f32(p2, t, (long long)p.T * g->proj2_out, st)));
-  bf16* gu = reinterpret_cast<bf16*>(ws + p.off_gu);
+  if (float* t = tap(ASR_TAP_HEAD)) {
+    if (f32)
+      ASR_LAUNCH(e, cudaMemcpyAsync(t, p2, (size_t)p.T * g->proj2_out * 4, cudaMemcpyDeviceToDevice, st));
+    else
+      ASR_K(PC_MISC, ASR_LAUNCH(e, launch_bf16_to_f32(static_cast<const bf16*>(p2), t, (long long)p.T * g->proj2_out, st)));
+  }
+  void* gu = ws + p.off_gu;
   ASR_K(PC_GEMM_ADAPTER, ASR_TRY(gemm(e, &e->maps.p2, nullptr, e->gu, p.T, gu, g->adapter_hidden, nullptr, nullptr, 1, EPI_SWIGLU, st, nullptr)));
   ASR_K(PC_GEMM_ADAPTER, ASR_TRY(gemm(e, &e->maps.gu, nullptr, e->down, p.T, out, g->adapter_out, nullptr, nullptr, 1, EPI_OUT_F32, st, o_out)));
   return ASR_OK;
@@ -1269,6 +1303,51 @@ asr_status asr_op_linear(const void* x, const void* w, const float* bias, int64_
   CUtensorMap omap;
   const bool f32_out = (e_bits & (EPI_OUT_F32 | EPI_RESID)) != 0;
   const bool have_omap = !(e_bits & EPI_SWIGLU) && make_tmap_out(&omap, y, M, N, N, f32_out);
+  ASR_CUDA(nullptr, launch_gemm(&amap, wb, p, e_bits, bn, sms, st, have_omap ? &omap : nullptr));
+  return ASR_OK;
+}
+
+asr_status asr_op_linear_tf32(const float* x, const float* w, const float* bias, int64_t M, int N, int K, int epi,
+                              int tile_n, float* y, void* ws, size_t ws_bytes, void* stream) {
+  if (!x || !w || !y || M <= 0 || N <= 0 || K <= 0 || K % 4 || N % 16)
+    return fail(nullptr, ASR_E_INVAL, "linear_tf32: bad arguments (K %% 4, N %% 16)");
+  if (!ws || ws_bytes < 256) return fail(nullptr, ASR_E_WORKSPACE, "linear_tf32: workspace too small");
+  int e_bits;
+  switch (epi) {
+    case ASR_EPI_F32: e_bits = EPI_OUT_F32; break;
+    case ASR_EPI_BF16_GELU: e_bits = EPI_OUT_F32 | EPI_GELU; break;
+    case ASR_EPI_F32_RESID: e_bits = EPI_RESID; break;
+    case ASR_EPI_SWIGLU:
+      if (N % 32) return fail(nullptr, ASR_E_INVAL, "linear_tf32: SwiGLU needs N %% 32 == 0");
+      e_bits = EPI_OUT_F32 | EPI_SWIGLU;
+      break;
+    default: return fail(nullptr, ASR_E_INVAL, "linear_tf32: unsupported epilogue %d", epi);
+  }
+  if (tile_n && tile_n != 256 && tile_n != 128 && tile_n != 64)
+    return fail(nullptr, ASR_E_INVAL, "linear_tf32: tile_n must be 0, 256, 128 or 64");
+  const int sms = current_sm_count();
+  GemmB wb;
+  wb.ptr = w;
+  wb.N = N;
+  wb.K = K;
+  wb.kind = KIND_TF32;
+  CUtensorMap amap;
+  if (!make_weight_maps(wb) || !make_tmap_f32(&amap, x, M, K, K, 128))
+    return fail(nullptr, ASR_E_INVAL, "linear_tf32: TMA descriptor encoding failed (16-byte alignment?)");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  GemmParams p;
+  memset(&p, 0, sizeof p);
+  p.M = (int)M;
+  p.out = y;
+  p.ldo = (e_bits & EPI_SWIGLU) ? N / 2 : N;
+  p.bias = bias;
+  p.pe_period = 1;
+  p.status = static_cast<int*>(ws);
+  p.limit_ns = kWaitLimitNs;
+  ASR_CUDA(nullptr, cudaMemsetAsync(ws, 0, 4, st));
+  const int bn = tile_n ? tile_n : gemm_pick_bn_tf32((int)M, N, sms);
+  CUtensorMap omap;
+  const bool have_omap = !(e_bits & EPI_SWIGLU) && make_tmap_out(&omap, y, M, N, N, true);
   ASR_CUDA(nullptr, launch_gemm(&amap, wb, p, e_bits, bn, sms, st, have_omap ? &omap : nullptr));
   return ASR_OK;
 }

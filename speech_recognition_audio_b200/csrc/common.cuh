@@ -203,6 +203,28 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Operand kinds of the GEMM engine: bf16 (kind::f16), tf32 (kind::tf32,
+// fp32 operands in memory, the tensor core reading their tf32 part), f16
+// (kind::f16).  A 128-byte swizzled row holds 64 16-bit or 32 fp32 elements,
+// and one MMA step takes 32 bytes of K: 16 or 8 elements.
+enum : int { KIND_BF16 = 0, KIND_TF32 = 1, KIND_F16 = 2 };
+__host__ __device__ constexpr int kind_row_elems(int kind) { return kind == KIND_TF32 ? 32 : 64; }
+// Instruction descriptor of a kind: fp32 D, A and B K-major; A/B format
+// fields (bits 7-9, 10-12): kind::f16 F16 = 0, BF16 = 1; kind::tf32 TF32 = 2.
+__host__ __device__ constexpr uint32_t idesc_kind_f32(int kind, int M, int N) {
+  return (1u << 4) | (kind == KIND_TF32 ? (2u << 7) | (2u << 10) : kind == KIND_F16 ? 0u : (1u << 7) | (1u << 10)) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::tf32 (fp32 operands, fp32 accumulate).
+__device__ __forceinline__ void tc_mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // ---------------------------------------------------------------- math
 // Packed fp32 pair arithmetic (the f32x2 instructions of sm_100): one
 // instruction issues two IEEE fp32 operations with the usual rounding.

@@ -42,6 +42,31 @@ cudaError_t run(const CUtensorMap* a, const CUtensorMap& b, const CUtensorMap& o
   return launch_pdl(k, dim3(grid), dim3(S::THREADS), S::SMEM_BYTES, st, a ? *a : b, b, o, p);
 }
 
+template <int BN, int EPI>
+cudaError_t run_tf32(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& p, int grid,
+                     cudaStream_t st) {
+  using S = GemmShape<BN, stages_for<BN>(), false, KIND_TF32>;
+  auto k = gemm_tf32_tc_kernel<BN, S::STAGES, EPI>;
+  cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_BYTES);
+  if (err != cudaSuccess) return err;
+  return launch_pdl(k, dim3(grid), dim3(S::THREADS), S::SMEM_BYTES, st, a, b, o, p);
+}
+
+// tf32 epilogues: every output is fp32.
+template <int BN>
+cudaError_t run_tf32_epi(int epi, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& p,
+                         int grid, cudaStream_t st) {
+  switch (epi) {
+    case EPI_OUT_F32: return run_tf32<BN, EPI_OUT_F32>(a, b, o, p, grid, st);
+    case EPI_OUT_F32 | EPI_GELU: return run_tf32<BN, EPI_OUT_F32 | EPI_GELU>(a, b, o, p, grid, st);
+    case EPI_RESID: return run_tf32<BN, EPI_RESID>(a, b, o, p, grid, st);
+    case EPI_OUT_F32 | EPI_PE: return run_tf32<BN, EPI_OUT_F32 | EPI_PE>(a, b, o, p, grid, st);
+    case EPI_OUT_F32 | EPI_SWIGLU: return run_tf32<BN, EPI_OUT_F32 | EPI_SWIGLU>(a, b, o, p, grid, st);
+    case EPI_GELU | EPI_OUT_F32 | EPI_PE: return run_tf32<BN, EPI_GELU | EPI_OUT_F32 | EPI_PE>(a, b, o, p, grid, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 template <int BN>
 cudaError_t run_tma(int epi, const CUtensorMap* a, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& p, int grid,
                     cudaStream_t st) {
@@ -181,16 +206,18 @@ bool make_tmap_bf16(CUtensorMap* map, const void* ptr, unsigned long long rows, 
 }
 
 bool make_tmap_convbox(CUtensorMap* map, const void* ptr, int C, int F_in, int T_in, int n_img, int F_out, int sf,
-                       int TR, int st) {
+                       int TR, int st, int kind) {
   EncodeTiledFn fn = encode_fn();
-  if (!fn || !ptr || (reinterpret_cast<uintptr_t>(ptr) & 15) || C % 8 || F_out * sf > 256 || TR * st > 256 ||
+  const cuuint64_t esz = kind == KIND_TF32 ? 4 : 2;
+  if (!fn || !ptr || (reinterpret_cast<uintptr_t>(ptr) & 15) || (C * esz) % 16 || F_out * sf > 256 || TR * st > 256 ||
       F_out * TR != 128 || sf < 1 || sf > 8 || st < 1 || st > 8)
     return false;
   cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)F_in, (cuuint64_t)T_in, (cuuint64_t)n_img};
-  cuuint64_t strides[3] = {(cuuint64_t)C * 2, (cuuint64_t)F_in * C * 2, (cuuint64_t)T_in * F_in * C * 2};
-  cuuint32_t box[4] = {64, (cuuint32_t)(F_out * sf), (cuuint32_t)(TR * st), 1};
+  cuuint64_t strides[3] = {(cuuint64_t)C * esz, (cuuint64_t)F_in * C * esz, (cuuint64_t)T_in * F_in * C * esz};
+  cuuint32_t box[4] = {(cuuint32_t)kind_row_elems(kind), (cuuint32_t)(F_out * sf), (cuuint32_t)(TR * st), 1};
   cuuint32_t es[4] = {1, (cuuint32_t)sf, (cuuint32_t)st, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, es,
+  return fn(map, kind == KIND_TF32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+            const_cast<void*>(ptr), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -211,23 +238,64 @@ bool make_tmap_out(CUtensorMap* map, const void* ptr, unsigned long long rows, u
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool make_tmap_convphase(CUtensorMap* map, const void* ptr, int C, int F_h, int T_h, int n_planes, int F_out, int TR) {
+bool make_tmap_convphase(CUtensorMap* map, const void* ptr, int C, int F_h, int T_h, int n_planes, int F_out, int TR,
+                         int kind) {
   EncodeTiledFn fn = encode_fn();
-  if (!fn || !ptr || (reinterpret_cast<uintptr_t>(ptr) & 15) || C % 8 || F_out > 256 || TR > 256 || F_out * TR != 128)
+  const cuuint64_t esz = kind == KIND_TF32 ? 4 : 2;
+  if (!fn || !ptr || (reinterpret_cast<uintptr_t>(ptr) & 15) || (C * esz) % 16 || F_out > 256 || TR > 256 ||
+      F_out * TR != 128)
     return false;
   cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)F_h, (cuuint64_t)T_h, (cuuint64_t)n_planes};
-  cuuint64_t strides[3] = {(cuuint64_t)C * 2, (cuuint64_t)F_h * C * 2, (cuuint64_t)T_h * F_h * C * 2};
-  cuuint32_t box[4] = {64, (cuuint32_t)F_out, (cuuint32_t)TR, 1};
+  cuuint64_t strides[3] = {(cuuint64_t)C * esz, (cuuint64_t)F_h * C * esz, (cuuint64_t)T_h * F_h * C * esz};
+  cuuint32_t box[4] = {(cuuint32_t)kind_row_elems(kind), (cuuint32_t)F_out, (cuuint32_t)TR, 1};
   cuuint32_t es[4] = {1, 1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, es,
+  return fn(map, kind == KIND_TF32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+            const_cast<void*>(ptr), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_tmap_f32(CUtensorMap* map, const void* ptr, unsigned long long rows, unsigned long long cols,
+                   unsigned long long row_stride_elems, unsigned int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || !ptr || (reinterpret_cast<uintptr_t>(ptr) & 15) || (row_stride_elems * 4) % 16 || rows == 0 ||
+      cols == 0 || box_rows == 0 || box_rows > 256)
+    return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {row_stride_elems * 4};
+  cuuint32_t box[2] = {32, box_rows};  // one 128-byte swizzled row of 32 fp32
+  cuuint32_t es[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tmap_act(int kind, CUtensorMap* map, const void* ptr, unsigned long long rows, unsigned long long cols,
+                   unsigned long long row_stride_elems, unsigned int box_rows) {
+  return kind == KIND_TF32 ? make_tmap_f32(map, ptr, rows, cols, row_stride_elems, box_rows)
+                           : make_tmap_bf16(map, ptr, rows, cols, row_stride_elems, box_rows);
+}
+
 bool make_weight_maps(GemmB& w) {
   for (int i = 0; i < kGemmSlots; ++i)
-    if (!make_tmap_bf16(&w.map[i], w.ptr, w.N, w.K, w.K, kSlotRows[i])) return false;
+    if (!make_tmap_act(w.kind, &w.map[i], w.ptr, w.N, w.K, w.K, kSlotRows[i])) return false;
   return true;
+}
+
+int gemm_pick_bn_tf32(int M, int N, int num_sms) {
+  // one-SM tiles of 256, 128 or 64 columns: fewest waves, then the wider tile
+  if (N <= 64) return 64;
+  int best = 256;
+  long long best_cost = -1;
+  for (int bn : {256, 128}) {
+    const long long tiles = (long long)((M + 127) / 128) * ((N + bn - 1) / bn);
+    const long long cost = (tiles + num_sms - 1) / num_sms * (bn + 32);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = bn;
+    }
+  }
+  return best;
 }
 
 int gemm_pick_bn(int M, int N, int num_sms, bool gather) {
@@ -273,6 +341,7 @@ int gemm_pick_bn_conv(int n_sub, int N, int num_sms) {
 cudaError_t launch_gemm(const CUtensorMap* a_map, const GemmB& w, GemmParams p, int epi, int bn, int num_sms,
                         cudaStream_t st, const CUtensorMap* out_map) {
   p.out_tma = (out_map != nullptr && !(epi & (EPI_PE | EPI_SWIGLU))) ? 1 : 0;
+  if (w.kind == KIND_TF32 && bn < 0) return cudaErrorInvalidValue;  // the CTA-pair kernel takes 16-bit operands
   // Tile order: the tiles running at once share the larger operand, so it
   // crosses from DRAM once and is re-read from L2 (and the TMA latency the
   // stage ring has to cover is the L2's, not the DRAM's).  A (M x K) is the
@@ -308,6 +377,24 @@ cudaError_t launch_gemm(const CUtensorMap* a_map, const GemmB& w, GemmParams p, 
   const int slot = gemm_bn_slot(bn);
   if (slot < 0 || p.M <= 0) return cudaErrorInvalidValue;
   p.sk = 0;  // the one-SM kernel runs whole tiles
+  if (w.kind == KIND_TF32) {
+    if (!a_map) return cudaErrorInvalidValue;  // no gather mode for fp32 operands
+    p.N = w.N;
+    p.K = w.K;
+    p.m_blocks = p.conv_box ? p.cb.n_sub : (p.M + 127) / 128;
+    p.n_blocks = (p.N + bn - 1) / bn;
+    p.k_blocks = (p.K + 31) / 32;
+    p.num_tiles = p.m_blocks * p.n_blocks;
+    const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
+    const CUtensorMap& b = w.map[slot];
+    const CUtensorMap& o = p.out_tma ? *out_map : b;
+    switch (bn) {
+      case 256: return run_tf32_epi<256>(epi, *a_map, b, o, p, grid, st);
+      case 128: return run_tf32_epi<128>(epi, *a_map, b, o, p, grid, st);
+      case 64: return run_tf32_epi<64>(epi, *a_map, b, o, p, grid, st);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   p.N = w.N;
   p.K = w.K;
   p.m_blocks = p.conv_box ? p.cb.n_sub : (p.M + 127) / 128;

@@ -192,7 +192,8 @@ __device__ __forceinline__ void subtile_rows(const GemmParams& p, int u, int& fi
 }
 
 // TMA coordinates of the A tile of sub-tile u at k-block kb (conv-box mode).
-__device__ __forceinline__ void convbox_coords(const GemmParams& p, int u, int kb, int& c0, int& f0, int& t0, int& img) {
+__device__ __forceinline__ void convbox_coords(const GemmParams& p, int u, int kb, int& c0, int& f0, int& t0, int& img,
+                                               int BK = 64) {
   const ConvBox& c = p.cb;
   const int uu = u < c.n_sub ? u : c.n_sub - 1;  // past the end: any valid box, rows are masked
   img = uu / c.tiles_per_img;
@@ -200,7 +201,7 @@ __device__ __forceinline__ void convbox_coords(const GemmParams& p, int u, int k
   const int tap = kb / c.CB;
   const int cbk = kb - tap * c.CB;
   const int dt = tap / c.kf, df = tap - dt * c.kf;
-  c0 = cbk * 64;
+  c0 = cbk * BK;
   if (c.phase) {
     // input index 2 o + d - p lies in plane (d - p) & 1 at o + ((d - p) >> 1)
     const int at = dt - c.pt, af = df - c.pf;
@@ -242,18 +243,21 @@ static constexpr unsigned long long kDrainLimitNs = 200ull * 1000 * 1000;
 // k-block past the end of K (plain mode) or in the last channel block of a
 // tap when the channel count is not a multiple of 64 (conv-box mode), whose
 // zero-padded tail the MMA can skip.
-__device__ __forceinline__ int k16_steps(const GemmParams& p, int kb) {
+// (BK elements per k-block, 4 MMA steps of BK / 4.)
+__device__ __forceinline__ int k16_steps(const GemmParams& p, int kb, int BK = 64) {
   if (p.conv_box) return (kb % p.cb.CB == p.cb.CB - 1) ? p.cb.k16_last : 4;
-  const int rem = p.K - kb * 64;
-  return rem >= 64 ? 4 : (rem + 15) / 16;
+  const int rem = p.K - kb * BK;
+  const int ks = BK / 4;
+  return rem >= BK ? 4 : (rem + ks - 1) / ks;
 }
 
-template <int BN_, int STAGES_, bool GATHER_>
+template <int BN_, int STAGES_, bool GATHER_, int KIND_ = KIND_BF16>
 struct GemmShape {
-  static constexpr int BM = 128, BN = BN_, BK = 64, STAGES = STAGES_;
+  static constexpr int KIND = KIND_;
+  static constexpr int BM = 128, BN = BN_, BK = kind_row_elems(KIND_), STAGES = STAGES_;
   static constexpr bool GATHER = GATHER_;
-  static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int A_BYTES = BM * 128;   // 128-byte rows of BK elements
+  static constexpr int B_BYTES = BN * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int ACC_COLS = (BN + 31) / 32 * 32;
   static constexpr int TMEM_COLS =
@@ -267,6 +271,7 @@ struct GemmShape {
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
   static_assert(2 * ACC_COLS <= 512, "two accumulators must fit in TMEM");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+  static_assert(!(GATHER_ && KIND_ == KIND_TF32), "the cp.async gather stages 16-bit operands");
 };
 
 // Epilogue warps: four per TMEM lane quarter share the accumulator columns
@@ -351,7 +356,7 @@ __device__ __forceinline__ void epilogue_warp(const GemmParams& p, const CUtenso
                                               int mlimit, int n0, int BN, int half, int lane, uint8_t* wbuf,
                                               const float* breg, int kind = PIECE_FULL, int cstride = 64) {
   constexpr bool F32 = (EPI & (EPI_OUT_F32 | EPI_RESID)) != 0;
-  constexpr bool SWI = (EPI & EPI_SWIGLU) != 0;
+  constexpr bool SWI = (EPI & EPI_SWIGLU) != 0;  // with F32: fp32 outputs, stored per row
   constexpr bool TMA_OK = (EPI & (EPI_PE | EPI_SWIGLU)) == 0;
   if (row0 >= mlimit) return;  // no valid row in this quarter (warp-uniform)
   // A 32-row box may be stored whole when all its rows belong to this
@@ -373,6 +378,18 @@ __device__ __forceinline__ void epilogue_warp(const GemmParams& p, const CUtenso
       const float bj = breg[j];
 #pragma unroll
       for (int i = 0; i < 32; ++i) v[i] += __shfl_sync(0xffffffffu, bj, i);
+    }
+    if (SWI && F32) {
+      // gate = columns c..c+15, up = c+16..c+31 -> 16 fp32 outputs of this row
+      const int row = row0 + lane;
+      if (row < mlimit) {
+        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (long long)row * p.ldo + (n >> 1));
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          dst[k] = make_float4(silu(v[4 * k]) * v[16 + 4 * k], silu(v[4 * k + 1]) * v[17 + 4 * k],
+                               silu(v[4 * k + 2]) * v[18 + 4 * k], silu(v[4 * k + 3]) * v[19 + 4 * k]);
+      }
+      continue;
     }
     // The buffer may still be the source of the previous group's bulk store.
     if (lane == 0) bulk_wait_read0();
@@ -480,11 +497,10 @@ __device__ __forceinline__ void epilogue_warp(const GemmParams& p, const CUtenso
   }
 }
 
-template <int BN, int STAGES, bool GATHER, int EPI>
-__global__ void __launch_bounds__(GemmShape<BN, STAGES, GATHER>::THREADS, 1)
-    gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
-  using S = GemmShape<BN, STAGES, GATHER>;
+template <int BN, int STAGES, bool GATHER, int EPI, int KIND>
+__device__ __forceinline__ void gemm_tc_body(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmOut,
+                                             const GemmParams& p) {
+  using S = GemmShape<BN, STAGES, GATHER, KIND>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -551,7 +567,7 @@ __global__ void __launch_bounds__(GemmShape<BN, STAGES, GATHER>::THREADS, 1)
             mbar_arrive_expect_tx(&full[s], S::A_BYTES + S::B_BYTES);
             if (p.conv_box) {
               int c0, f0, t0, img;
-              convbox_coords(p, mb, kb, c0, f0, t0, img);
+              convbox_coords(p, mb, kb, c0, f0, t0, img, S::BK);
               tma_load_4d(sA + s * S::A_BYTES, &tmA, &full[s], c0, f0, t0, img);
             } else {
               tma_load_2d(sA + s * S::A_BYTES, &tmA, &full[s], kb * S::BK, m0);
@@ -586,7 +602,7 @@ __global__ void __launch_bounds__(GemmShape<BN, STAGES, GATHER>::THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(S::BM, BN);
+      const uint32_t idesc = idesc_kind_f32(KIND, S::BM, BN);
       int it = 0, tl = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++tl) {
@@ -611,10 +627,17 @@ __global__ void __launch_bounds__(GemmShape<BN, STAGES, GATHER>::THREADS, 1)
           tc_fence_after();
           const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + s * S::A_BYTES));
           const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + s * S::B_BYTES));
-          const int ks = k16_steps(p, kb);
+          const int ks = k16_steps(p, kb, S::BK);
 #pragma unroll
-          for (int k = 0; k < S::BK / 16; ++k)
-            if (k < ks) tc_mma_bf16(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+          for (int k = 0; k < 4; ++k) {
+            if (k < ks) {
+              // each step: 32 bytes of K (16 bf16 or 8 tf32 elements)
+              if (KIND == KIND_TF32)
+                tc_mma_tf32(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+              else
+                tc_mma_bf16(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+            }
+          }
           tc_commit(&empty[s]);
           ++it;
         }
@@ -718,6 +741,22 @@ __global__ void __launch_bounds__(GemmShape<BN, STAGES, GATHER>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, S::TMEM_COLS);
+}
+
+// bf16 operands (kind::f16).
+template <int BN, int STAGES, bool GATHER, int EPI>
+__global__ void __launch_bounds__(GemmShape<BN, STAGES, GATHER>::THREADS, 1)
+    gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
+  gemm_tc_body<BN, STAGES, GATHER, EPI, KIND_BF16>(tmA, tmB, tmOut, p);
+}
+
+// fp32 operands in memory, multiplied as tf32 (kind::tf32), fp32 accumulate.
+template <int BN, int STAGES, int EPI>
+__global__ void __launch_bounds__(GemmShape<BN, STAGES, false, KIND_TF32>::THREADS, 1)
+    gemm_tf32_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
+  gemm_tc_body<BN, STAGES, false, EPI, KIND_TF32>(tmA, tmB, tmOut, p);
 }
 
 }  // namespace asr

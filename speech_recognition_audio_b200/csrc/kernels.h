@@ -68,7 +68,7 @@ cudaError_t launch_log_mel(const float* pcm, long long n_samples, int batch, int
 cudaError_t launch_mel_normalize(const float* raw, const unsigned int* clip_max, long long per_clip, int batch,
                                  float* out, cudaStream_t st);
 cudaError_t launch_mel_normalize_transpose(const float* raw, const unsigned int* clip_max, int batch, int n_mels,
-                                           int n_frames, bf16* out, cudaStream_t st);
+                                           int n_frames, void* out, bool f32, cudaStream_t st);
 
 // Variable-length batches.  One conv chunk: its clip, its first frame within
 // the clip, its valid frames (chunk_frames except for a clip's last chunk)
@@ -96,10 +96,10 @@ struct VarClipBatch {
 cudaError_t launch_varlen_fill(const VarClipBatch& vb, int chunk_frames, int window, int t3, MelClip* mc,
                                ChunkDesc* cd, int* cu, int last, int n_win, int n_tokens, cudaStream_t st);
 cudaError_t launch_conv1_im2col_varlen(const float* mel_raw, const unsigned int* clip_max, int n_chunks, int n_mels,
-                                       int chunk_frames, int phase, const ChunkDesc* cd, const MelClip* mc, bf16* a,
-                                       cudaStream_t st);
-cudaError_t launch_mask_short_chunks(bf16* act, const ChunkDesc* cd, int n_chunks, int chunk_frames, int level, int T,
-                                     int F, int C, int phase, cudaStream_t st);
+                                       int chunk_frames, int phase, const ChunkDesc* cd, const MelClip* mc, void* a,
+                                       bool f32, cudaStream_t st);
+cudaError_t launch_mask_short_chunks(void* act, const ChunkDesc* cd, int n_chunks, int chunk_frames, int level, int T,
+                                     int F, int C, int phase, int es, cudaStream_t st);
 cudaError_t launch_compact_tokens(const float* xpad, float* x, const ChunkDesc* cd, int n_chunks, int t3, int d,
                                   cudaStream_t st);
 
@@ -109,7 +109,7 @@ cudaError_t launch_compact_tokens(const float* xpad, float* x, const ChunkDesc* 
 // [chunks][T1][F1], or with phase != 0 (T1, F1 even) the parity planes
 // [chunks][t % 2][f % 2][T1 / 2][F1 / 2] read by the phase-mode conv2.
 cudaError_t launch_conv1_im2col(const float* mel_raw, const unsigned int* clip_max, int batch, int n_mels,
-                                int n_frames, int chunk_frames, int phase, bf16* a, cudaStream_t st);
+                                int n_frames, int chunk_frames, int phase, void* a, bool f32, cudaStream_t st);
 
 cudaError_t launch_layer_norm(const float* x, const float* g, const float* b, long long M, int D, float eps,
                               void* y, bool out_f32, cudaStream_t st);
@@ -118,6 +118,9 @@ cudaError_t launch_layer_norm(const float* x, const float* g, const float* b, lo
 bool make_tmap_qkv(CUtensorMap* map, const void* qkv, long long T, int H);
 cudaError_t launch_attention_tc(const CUtensorMap& tm_qkv, const bf16* qkv, const int* cu, int n_seg, int H, bf16* out,
                                 int* status, unsigned long long limit_ns, cudaStream_t st);
+// fp32 attention on the CUDA cores (attn_f32.cu): the fp32-weight path.
+cudaError_t launch_attention_f32(const float* qkv, const int* cu, int n_seg, int max_seg, int H, float* out,
+                                 cudaStream_t st);
 // tcgen05 flash attention for segments of any length (attn_fa.cu).
 cudaError_t launch_attention_fa(const CUtensorMap& tm_qkv, const int* cu, int n_seg, int max_seg, int H, bf16* out,
                                 int* status, unsigned long long limit_ns, cudaStream_t st);
@@ -137,24 +140,35 @@ cudaError_t launch_wait_probe(unsigned long long limit_ns, int* status, cudaStre
 
 // GEMM engine launch (gemm.cu).
 constexpr int kGemmSlots = 6;
-struct GemmB {              // weight operand [N, K] bf16 + its TMA maps
-  const bf16* ptr = nullptr;
+struct GemmB {              // weight operand [N, K] (bf16, or fp32 for KIND_TF32) + its TMA maps
+  const void* ptr = nullptr;
   int N = 0, K = 0;
+  int kind = KIND_BF16;
   CUtensorMap map[kGemmSlots];  // box rows 256, 128, 240, 64, 160, 120 (index by gemm_bn_slot)
 };
 int gemm_bn_slot(int bn);
 bool make_tmap_bf16(CUtensorMap* map, const void* ptr, unsigned long long rows, unsigned long long cols,
                     unsigned long long row_stride_elems, unsigned int box_rows);
+// fp32 activation map (box 32 x box_rows: one 128-byte row per box row).
+bool make_tmap_f32(CUtensorMap* map, const void* ptr, unsigned long long rows, unsigned long long cols,
+                   unsigned long long row_stride_elems, unsigned int box_rows);
+// A-operand map of an activation of the kind's element type.
+bool make_tmap_act(int kind, CUtensorMap* map, const void* ptr, unsigned long long rows, unsigned long long cols,
+                   unsigned long long row_stride_elems, unsigned int box_rows);
 bool make_weight_maps(GemmB& w);
-// 4-D strided-box map over a conv activation [n_img, T_in, F_in, C] (see ConvBox).
+// 4-D strided-box map over a conv activation [n_img, T_in, F_in, C] (see ConvBox),
+// elements of the kind's type (box inner extent: one 128-byte row).
 bool make_tmap_convbox(CUtensorMap* map, const void* ptr, int C, int F_in, int T_in, int n_img, int F_out, int sf,
-                       int TR, int st);
+                       int TR, int st, int kind = KIND_BF16);
 // 4-D dense-box map over a parity-plane activation [n_planes][T_h][F_h][C]
-// (ConvBox phase mode): box {64, F_out, TR, 1}.
-bool make_tmap_convphase(CUtensorMap* map, const void* ptr, int C, int F_h, int T_h, int n_planes, int F_out, int TR);
+// (ConvBox phase mode): box {row elements, F_out, TR, 1}.
+bool make_tmap_convphase(CUtensorMap* map, const void* ptr, int C, int F_h, int T_h, int n_planes, int F_out, int TR,
+                         int kind = KIND_BF16);
 // Picks the tile for an M x N problem on num_sms SMs: a positive width is a
 // one-SM 128 x bn tile, a negative one a CTA-pair 256 x |bn| tile.
 int gemm_pick_bn(int M, int N, int num_sms, bool gather);
+// Tile width for fp32 (tf32) operands: one-SM tiles only.
+int gemm_pick_bn_tf32(int M, int N, int num_sms);
 // Tile choice for a conv-box GEMM with n_sub 128-row sub-tiles.
 int gemm_pick_bn_conv(int n_sub, int N, int num_sms);
 // TMA map of a GEMM output [rows, cols] (row stride in elements), box 32 x 32,

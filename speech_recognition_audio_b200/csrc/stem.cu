@@ -21,12 +21,13 @@
 
 namespace asr {
 
+template <typename OutT>
 __global__ void __launch_bounds__(256) conv1_im2col_kernel(const float* __restrict__ mel_raw,
                                                            const unsigned int* __restrict__ clip_max, int n_mels,
                                                            int n_frames, int chunk_frames, int chunks_per_clip,
                                                            int T1, int F1, long long rows, int phase,
                                                            const ChunkDesc* __restrict__ cd,
-                                                           const MelClip* __restrict__ mc, bf16* __restrict__ a) {
+                                                           const MelClip* __restrict__ mc, OutT* __restrict__ a) {
   pdl_wait();
   pdl_trigger();
   const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
@@ -75,37 +76,51 @@ __global__ void __launch_bounds__(256) conv1_im2col_kernel(const float* __restri
   for (int k = 9; k < 16; ++k) v[k] = 0.f;
   // output row: [chunk][plane][T][F] (plain: [chunk][T1][F1])
   const long long row = (chunk * (phase ? 4 : 1) + plane) * (long long)TP * FP + (long long)t * FP + f;
-  alignas(16) __nv_bfloat162 r[8];
+  if constexpr (sizeof(OutT) == 4) {
+    float4* dst = reinterpret_cast<float4*>(a + row * 16);
 #pragma unroll
-  for (int k = 0; k < 8; ++k) r[k] = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
-  uint4* dst = reinterpret_cast<uint4*>(a + row * 16);
-  dst[0] = *reinterpret_cast<uint4*>(&r[0]);
-  dst[1] = *reinterpret_cast<uint4*>(&r[4]);
+    for (int k = 0; k < 4; ++k) dst[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+  } else {
+    alignas(16) __nv_bfloat162 r[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) r[k] = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+    uint4* dst = reinterpret_cast<uint4*>(a + row * 16);
+    dst[0] = *reinterpret_cast<uint4*>(&r[0]);
+    dst[1] = *reinterpret_cast<uint4*>(&r[4]);
+  }
 }
 
+// a: bf16 rows (f32 == false) or fp32 rows (f32 == true, the fp32-weight path).
 cudaError_t launch_conv1_im2col(const float* mel_raw, const unsigned int* clip_max, int batch, int n_mels,
-                                int n_frames, int chunk_frames, int phase, bf16* a, cudaStream_t st) {
+                                int n_frames, int chunk_frames, int phase, void* a, bool f32, cudaStream_t st) {
   const int T1 = (chunk_frames - 1) / 2 + 1, F1 = (n_mels - 1) / 2 + 1;
   if (phase && (T1 % 2 || F1 % 2)) return cudaErrorInvalidValue;
   const int chunks_per_clip = n_frames / chunk_frames;
   const long long rows = (long long)batch * chunks_per_clip * T1 * F1;
   if (rows == 0) return cudaSuccess;
   const unsigned blocks = static_cast<unsigned>((rows + 255) / 256);
-  return launch_pdl(conv1_im2col_kernel, dim3(blocks), dim3(256), 0, st, mel_raw, clip_max, n_mels, n_frames,
+  if (f32)
+    return launch_pdl(conv1_im2col_kernel<float>, dim3(blocks), dim3(256), 0, st, mel_raw, clip_max, n_mels, n_frames,
+                      chunk_frames, chunks_per_clip, T1, F1, rows, phase ? 1 : 0, (const ChunkDesc*)nullptr,
+                      (const MelClip*)nullptr, static_cast<float*>(a));
+  return launch_pdl(conv1_im2col_kernel<bf16>, dim3(blocks), dim3(256), 0, st, mel_raw, clip_max, n_mels, n_frames,
                     chunk_frames, chunks_per_clip, T1, F1, rows, phase ? 1 : 0, (const ChunkDesc*)nullptr,
-                    (const MelClip*)nullptr, a);
+                    (const MelClip*)nullptr, static_cast<bf16*>(a));
 }
 
 cudaError_t launch_conv1_im2col_varlen(const float* mel_raw, const unsigned int* clip_max, int n_chunks, int n_mels,
-                                       int chunk_frames, int phase, const ChunkDesc* cd, const MelClip* mc, bf16* a,
-                                       cudaStream_t st) {
+                                       int chunk_frames, int phase, const ChunkDesc* cd, const MelClip* mc, void* a,
+                                       bool f32, cudaStream_t st) {
   const int T1 = (chunk_frames - 1) / 2 + 1, F1 = (n_mels - 1) / 2 + 1;
   if (phase && (T1 % 2 || F1 % 2)) return cudaErrorInvalidValue;
   const long long rows = (long long)n_chunks * T1 * F1;
   if (rows == 0) return cudaSuccess;
   const unsigned blocks = static_cast<unsigned>((rows + 255) / 256);
-  return launch_pdl(conv1_im2col_kernel, dim3(blocks), dim3(256), 0, st, mel_raw, clip_max, n_mels, 0, chunk_frames,
-                    1, T1, F1, rows, phase ? 1 : 0, cd, mc, a);
+  if (f32)
+    return launch_pdl(conv1_im2col_kernel<float>, dim3(blocks), dim3(256), 0, st, mel_raw, clip_max, n_mels, 0,
+                      chunk_frames, 1, T1, F1, rows, phase ? 1 : 0, cd, mc, static_cast<float*>(a));
+  return launch_pdl(conv1_im2col_kernel<bf16>, dim3(blocks), dim3(256), 0, st, mel_raw, clip_max, n_mels, 0,
+                    chunk_frames, 1, T1, F1, rows, phase ? 1 : 0, cd, mc, static_cast<bf16*>(a));
 }
 
 // ---------------------------------------------------------- short chunks
@@ -116,8 +131,9 @@ cudaError_t launch_conv1_im2col_varlen(const float* mel_raw, const unsigned int*
 // (rows before that length only read valid inputs or that padding).
 // level 1: conv1 output (length ceil(L / 2)), level 2: conv2 output
 // (ceil(ceil(L / 2) / 2)).  One block per chunk; whole chunks return at once.
-__global__ void mask_short_chunks_kernel(bf16* __restrict__ act, const ChunkDesc* __restrict__ cd, int chunk_frames,
-                                         int level, int T, int F, int C, int phase) {
+// (act: elements of `es` bytes, 2 or 4; C * es a multiple of 16.)
+__global__ void mask_short_chunks_kernel(uint8_t* __restrict__ act, const ChunkDesc* __restrict__ cd, int chunk_frames,
+                                         int level, int T, int F, int C, int phase, int es) {
   pdl_wait();
   pdl_trigger();
   const int c = blockIdx.x;
@@ -129,8 +145,8 @@ __global__ void mask_short_chunks_kernel(bf16* __restrict__ act, const ChunkDesc
   const uint4 z = make_uint4(0, 0, 0, 0);
   if (!phase) {
     // rows [tv, T) of the chunk's [T][F][C] block are contiguous
-    uint4* p = reinterpret_cast<uint4*>(act + ((long long)c * T + tv) * F * C);
-    const long long n16 = (long long)(T - tv) * F * C / 8;
+    uint4* p = reinterpret_cast<uint4*>(act + ((long long)c * T + tv) * F * C * es);
+    const long long n16 = (long long)(T - tv) * F * C * es / 16;
     for (long long j = threadIdx.x; j < n16; j += blockDim.x) p[j] = z;
   } else {
     // parity planes [4][T/2][F/2][C]: plane (pt, pf) holds t = 2 th + pt
@@ -139,19 +155,19 @@ __global__ void mask_short_chunks_kernel(bf16* __restrict__ act, const ChunkDesc
       const int pt = pl >> 1;
       const int th0 = tv - pt <= 0 ? 0 : (tv - pt + 1) / 2;
       if (th0 >= TH) continue;
-      uint4* p = reinterpret_cast<uint4*>(act + (((long long)c * 4 + pl) * TH + th0) * FH * C);
-      const long long n16 = (long long)(TH - th0) * FH * C / 8;
+      uint4* p = reinterpret_cast<uint4*>(act + (((long long)c * 4 + pl) * TH + th0) * FH * C * es);
+      const long long n16 = (long long)(TH - th0) * FH * C * es / 16;
       for (long long j = threadIdx.x; j < n16; j += blockDim.x) p[j] = z;
     }
   }
 }
 
-cudaError_t launch_mask_short_chunks(bf16* act, const ChunkDesc* cd, int n_chunks, int chunk_frames, int level, int T,
-                                     int F, int C, int phase, cudaStream_t st) {
+cudaError_t launch_mask_short_chunks(void* act, const ChunkDesc* cd, int n_chunks, int chunk_frames, int level, int T,
+                                     int F, int C, int phase, int es, cudaStream_t st) {
   if (n_chunks <= 0) return cudaSuccess;
-  if (C % 8 || (phase && (T % 2 || F % 2))) return cudaErrorInvalidValue;
-  return launch_pdl(mask_short_chunks_kernel, dim3(n_chunks), dim3(256), 0, st, act, cd, chunk_frames, level, T, F, C,
-                    phase);
+  if ((C * es) % 16 || (phase && (T % 2 || F % 2))) return cudaErrorInvalidValue;
+  return launch_pdl(mask_short_chunks_kernel, dim3(n_chunks), dim3(256), 0, st, static_cast<uint8_t*>(act), cd,
+                    chunk_frames, level, T, F, C, phase, es);
 }
 
 // Valid tokens of every chunk, from the padded conv_out rows [chunk][t3] to

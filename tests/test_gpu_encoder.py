@@ -68,6 +68,35 @@ def test_tiny_full_with_taps():
     enc.set_taps(0)
 
 
+def test_tiny_fp32_weights_run_tf32_end_to_end():
+    # The tiny geometry's weights are fp32: every GEMM is a kind::tf32 GEMM on
+    # fp32 activations and the attention runs in fp32, so the result sits far
+    # inside the bf16 tolerance tier (tf32 keeps 10 mantissa bits, bf16 7).
+    w = synth.WORKLOADS["tiny_1x1s"]
+    g = synth.GEOMETRIES["tiny"]
+    assert g.dtype == synth.DTYPE_F32
+    enc, W, _ = _encoder("tiny_1x1s", affine=True, seed=78)
+    pcm = np.stack([synth.pcm_clip(32000, 510), synth.pcm_clip(32000, 511)])
+    out = _run(enc, pcm)
+    ref = oracle.forward(pcm, W, g)
+    cmin, rmax = assert_encoder_parity(out, ref, "tiny fp32 weights (tf32)")
+    assert cmin >= 0.99999 and rmax <= 5e-3
+
+
+def test_whisper_style_fp32_geometry():
+    # Conv1D stem, full attention and final LN with fp32 weights (tf32 path).
+    base = synth.GEOMETRIES["whisper_small"].as_dict()
+    base.update(d_model=256, n_heads=4, d_ffn=1024, n_layers=2, dtype=synth.DTYPE_F32)
+    g = synth.Geometry(**base)
+    W = synth.make_weights(g, 79, affine=True)
+    enc = sra.Encoder(g, {k: v.cuda() for k, v in W.items()})
+    pcm = np.stack([synth.pcm_clip(48000, 520), synth.pcm_clip(48000, 521)])
+    out = _run(enc, pcm)
+    assert out.shape == (2, 150, 256)
+    assert_encoder_parity(out, oracle.forward(pcm, W, g), "whisper-style fp32 weights (tf32)")
+    enc.close()
+
+
 def test_affine_biases_small_batch():
     # Non-zero biases and LayerNorm affine parameters exercise every epilogue's
     # bias path and the LN gain/shift; 2 clips x 3 s, windows of 104 > 39 tokens.

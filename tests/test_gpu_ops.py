@@ -118,6 +118,44 @@ def test_linear_epilogues(epi):
         assert np.abs(got - ref).max() <= 2.0 ** -8 * np.abs(ref).max() + 2e-3
 
 
+@pytest.mark.parametrize("M,N,K,tile_n", [(13, 256, 256, 0), (300, 1024, 1024, 0), (777, 480, 4320, 128),
+                                           (129, 512, 64, 64), (1000, 1280, 1280, 256)])
+def test_linear_tf32_matches_oracle(M, N, K, tile_n):
+    """fp32 operands on kind::tf32: every product sees each operand rounded
+    to tf32 (10 explicit mantissa bits), so |error| <= 2^-9 sum |x| |w| plus
+    fp32 accumulation."""
+    rng = np.random.default_rng(M + N + K)
+    x = rng.normal(size=(M, K)).astype(np.float32)
+    w = (rng.normal(size=(N, K)) * 0.05).astype(np.float32)
+    b = rng.normal(size=N).astype(np.float32)
+    xt, wt, bt = (torch.from_numpy(a).cuda() for a in (x, w, b))
+    bound = 2.0 ** -9 * (np.abs(x.astype(np.float64)) @ np.abs(w.astype(np.float64)).T) + 1e-5
+    ref = oracle.linear(x, w, b)
+    y = sra.linear_tf32(xt, wt, bt, sra.EPI_F32, tile_n=tile_n).cpu().numpy()
+    assert (np.abs(y - ref) <= bound).all(), np.abs(y - ref).max()
+    r0 = rng.normal(size=(M, N)).astype(np.float32)
+    out = torch.from_numpy(r0).cuda()
+    sra.linear_tf32(xt, wt, bt, sra.EPI_F32_RESID, out=out, tile_n=tile_n)
+    assert (np.abs(out.cpu().numpy() - (r0 + ref)) <= bound + 1e-5).all()
+    g = sra.linear_tf32(xt, wt, bt, sra.EPI_BF16_GELU, tile_n=tile_n).cpu().numpy()
+    # |GELU'| <= 1.13, plus the device GELU's own error (1e-5 |x| scale)
+    assert (np.abs(g - oracle.gelu(ref)) <= 1.13 * bound + 1e-5 * (1 + np.abs(ref))).all()
+
+
+def test_linear_tf32_swiglu():
+    M, N, K = 333, 1024, 768
+    rng = np.random.default_rng(12)
+    x = rng.normal(size=(M, K)).astype(np.float32)
+    w = (rng.normal(size=(N, K)) * 0.04).astype(np.float32)
+    wg, wu = w[: N // 2], w[N // 2:]
+    wi = np.stack([wg.reshape(-1, 16, K), wu.reshape(-1, 16, K)], 1).reshape(N, K)
+    got = sra.linear_tf32(torch.from_numpy(x).cuda(), torch.from_numpy(np.ascontiguousarray(wi)).cuda(), None,
+                          sra.EPI_SWIGLU).cpu().numpy()
+    ref = oracle.silu(oracle.linear(x, wg)) * oracle.linear(x, wu)
+    assert got.shape == (M, N // 2)
+    assert np.abs(got - ref).max() <= 2e-3 * max(1.0, np.abs(ref).max())
+
+
 # ------------------------------------------------------------------ mel
 @pytest.mark.parametrize("n_mels,secs,batch,speech", [(128, 1, 1, False), (128, 3, 2, False),
                                                       (80, 2, 3, False), (128, 20, 1, True)])
