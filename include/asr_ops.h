@@ -62,7 +62,7 @@ asr_status asr_op_log_mel_noalloc(const float* pcm, int64_t n_samples, int batch
  *  bias  device float32 [N] or NULL.
  *  epi   ASR_EPI_BF16       y bf16 [M, N] = acc + bias
  *        ASR_EPI_BF16_GELU  y bf16 [M, N] = GELU(acc + bias), the GELU of asr_op_gelu
- *                           (erf from Abramowitz & Stegun 7.1.28, |error| <= 3e-7)
+ *                           (tanh form, |error| <= 4.8e-4 + 2.5e-4 |x|)
  *        ASR_EPI_F32_RESID  y f32  [M, N] += acc + bias           (in place)
  *        ASR_EPI_F32        y f32  [M, N] = acc + bias
  *        ASR_EPI_SWIGLU     y bf16 [M, N/2]: W rows interleaved in blocks of
@@ -117,9 +117,11 @@ size_t asr_op_attention_ws_size(void);
 asr_status asr_op_attention(const void* qkv, const int32_t* cu, int n_seg, int max_seg, int64_t T,
                             int H, void* out, void* ws, size_t ws_bytes, void* stream);
 
-/* The GELU every kernel applies (bias-free): y[i] = x[i] Phi(x[i]), with
- * Phi from the Abramowitz & Stegun 7.1.28 approximation of erf (absolute
- * error <= 3e-7; fp32 evaluation adds at most ~6e-6 |x|).  x, y: device float32 [n]. */
+/* The GELU every kernel applies (bias-free): y[i] = GELU(x[i]) in the tanh
+ * form 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))) (Hendrycks & Gimpel),
+ * with tanh from the hardware tanh.approx.f32: |y - x Phi(x)| <= 4.8e-4 (the
+ * form) + 2.5e-4 |x| (the approximate tanh), below the rounding of a bf16
+ * output for |x| >= 0.5.  x, y: device float32 [n]. */
 asr_status asr_op_gelu(const float* x, float* y, int64_t n, void* stream);
 
 /* Bounded-wait self-check: launches one kernel that waits on a shared-memory

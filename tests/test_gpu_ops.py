@@ -138,8 +138,8 @@ def test_linear_tf32_matches_oracle(M, N, K, tile_n):
     sra.linear_tf32(xt, wt, bt, sra.EPI_F32_RESID, out=out, tile_n=tile_n)
     assert (np.abs(out.cpu().numpy() - (r0 + ref)) <= bound + 1e-5).all()
     g = sra.linear_tf32(xt, wt, bt, sra.EPI_BF16_GELU, tile_n=tile_n).cpu().numpy()
-    # |GELU'| <= 1.13, plus the device GELU's own error (1e-5 |x| scale)
-    assert (np.abs(g - oracle.gelu(ref)) <= 1.13 * bound + 1e-5 * (1 + np.abs(ref))).all()
+    # |GELU'| <= 1.13, plus the device GELU's own error (tanh form)
+    assert (np.abs(g - oracle.gelu(ref)) <= 1.13 * bound + 4.8e-4 + 2.6e-4 * np.abs(ref)).all()
 
 
 def test_linear_tf32_swiglu():
@@ -245,17 +245,21 @@ def test_attention_long_segment_rescale():
 
 # ------------------------------------------------------------------ GELU
 def test_gelu_within_published_bound():
-    # The device GELU takes erf from Abramowitz & Stegun 7.1.28 (|error| <= 3e-7),
-    # i.e. |GELU - exact| <= |x| * 0.5 * 3e-7, plus the fp32 evaluation of the
-    # 16th power: <= 111 roundings of 2^-24 relative on h <= 1/2, and the final
-    # rounding of the result.  An odd length sends the last element through the
-    # scalar form, the rest through the packed pair form.
+    # The device GELU is the tanh form 0.5 x (1 + tanh(sqrt(2/pi)(x + 0.044715 x^3)))
+    # (Hendrycks & Gimpel): within 4.8e-4 of the exact x Phi(x) (the form's own
+    # maximum is 4.74e-4, checked on the CPU below), plus 0.5 |x| times the
+    # hardware tanh's relative error (<= 2^-10.98), plus fp32 rounding.  An odd
+    # length sends the last element through the scalar form, the rest through
+    # the packed pair form.
     x = np.concatenate([np.linspace(-12, 12, 2_000_001), [0.0, -0.0, 1e-30, -1e-30, 40.0, -40.0]]).astype(np.float32)
     assert len(x) % 2 == 1
+    xd = x.astype(np.float64)
+    form = 0.5 * xd * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (xd + 0.044715 * xd ** 3)))
+    ref = oracle.gelu(xd)
+    assert np.abs(form - ref).max() <= 4.8e-4
     got = sra.gelu(torch.from_numpy(x).cuda()).cpu().numpy().astype(np.float64)
-    ref = oracle.gelu(x.astype(np.float64))
     err = np.abs(got - ref)
-    bound = (1.5e-7 + 0.5 * 111 * 2.0**-24 + 2.0**-23) * np.abs(x) + 2.0**-23 * np.abs(ref)
+    bound = 4.8e-4 + (0.5 * 2.0 ** -10.98 + 2.0 ** -22) * np.abs(x) + 2.0 ** -22 * np.abs(ref)
     assert (err <= bound).all(), (err.max(), (err / np.maximum(bound, 1e-300)).max())
     assert got[-2] == 40.0 and abs(got[-1]) == 0.0
     assert np.all(np.isfinite(got))
