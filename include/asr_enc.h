@@ -69,7 +69,15 @@ enum { ASR_DTYPE_BF16 = 0, ASR_DTYPE_F32 = 1, ASR_DTYPE_F16 = 2 };
  *  proj1_out, proj2_out        encoder head widths; 0 = absent (final LN only).
  *  adapter_hidden, adapter_out SwiGLU adapter widths; 0 = absent.
  *  ln_eps         LayerNorm epsilon.
- *  dtype          ASR_DTYPE_BF16 (bf16 weights) or ASR_DTYPE_F32 (fp32 weights).
+ *  dtype          the weights' type, which sets the arithmetic of every GEMM:
+ *                 ASR_DTYPE_BF16  bf16 weights, bf16 activations between the
+ *                                 GEMMs, tcgen05 kind::f16, fp32 accumulation;
+ *                 ASR_DTYPE_F16   f16 weights and activations (the F16 variant
+ *                                 of the pages' GGUF builds), kind::f16;
+ *                 ASR_DTYPE_F32   fp32 weights and activations, kind::tf32
+ *                                 GEMMs, attention in fp32 on the CUDA cores.
+ *                 The residual stream, softmax, LayerNorm statistics and the
+ *                 log-mel are fp32 in every case.
  */
 typedef struct {
   int stem;

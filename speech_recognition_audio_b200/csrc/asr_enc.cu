@@ -98,7 +98,7 @@ bool geom_valid(const asr_geometry* g, std::string* why) {
   if (g->adapter_hidden && (g->adapter_hidden % 16 || g->adapter_out % 16)) return fail("adapter widths must be multiples of 16");
   if (g->adapter_hidden && !g->proj1_out) return fail("the adapter needs the head projections");
   if (!(g->ln_eps > 0.f)) return fail("ln_eps must be > 0");
-  if (g->dtype != ASR_DTYPE_BF16 && g->dtype != ASR_DTYPE_F32) return fail("unknown dtype");
+  if (g->dtype != ASR_DTYPE_BF16 && g->dtype != ASR_DTYPE_F32 && g->dtype != ASR_DTYPE_F16) return fail("unknown dtype");
   return true;
 }
 
@@ -282,6 +282,56 @@ void* slab_take(asr_enc* e, size_t bytes) {
   return static_cast<char*>(e->slab) + off;
 }
 
+float bf16_to_float(uint16_t h) {
+  const uint32_t u = static_cast<uint32_t>(h) << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return f;
+}
+
+// IEEE binary16 -> float (exact: every half is a float).
+float f16_to_float(uint16_t h) {
+  const uint32_t sign = static_cast<uint32_t>(h >> 15) << 31;
+  const int ex = (h >> 10) & 31;
+  const uint32_t man = h & 1023;
+  float f;
+  if (ex == 0) {
+    f = std::ldexp(static_cast<float>(man), -24);  // zero or subnormal
+  } else if (ex == 31) {
+    const uint32_t u = 0x7F800000u | (man << 13);  // inf or nan
+    memcpy(&f, &u, 4);
+  } else {
+    const uint32_t u = (static_cast<uint32_t>(ex - 15 + 127) << 23) | (man << 13);
+    memcpy(&f, &u, 4);
+  }
+  if (sign) f = -f;
+  return f;
+}
+
+// float -> IEEE binary16, round to nearest even (values here are weights:
+// finite; overflow saturates to infinity as the rounding rule gives).
+uint16_t float_to_f16(float f) {
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  const uint16_t sign = static_cast<uint16_t>((u >> 16) & 0x8000u);
+  const float a = std::fabs(f);
+  if (!(a == a)) return static_cast<uint16_t>(sign | 0x7E00u);
+  if (a >= 65520.0f) return static_cast<uint16_t>(sign | 0x7C00u);
+  if (a < 6.103515625e-05f) {  // subnormal range: multiples of 2^-24
+    const float q = std::nearbyint(std::ldexp(a, 24));  // default rounding: nearest even
+    return static_cast<uint16_t>(sign | static_cast<uint16_t>(q));
+  }
+  int ex;
+  const float m = std::frexp(a, &ex);                        // a = m 2^ex, m in [0.5, 1)
+  float q = std::nearbyint(std::ldexp(m, 11));                // 11 significant bits
+  if (q >= 2048.0f) {
+    q = 1024.0f;
+    ++ex;
+  }
+  const uint32_t bits = (static_cast<uint32_t>(ex - 1 + 15) << 10) | (static_cast<uint32_t>(q) - 1024u);
+  return static_cast<uint16_t>(sign | bits);
+}
+
 // Copies a weight tensor to the host as float; false if the copy failed.
 bool fetch(const void* dptr, int64_t n, int dtype, std::vector<float>* out, cudaError_t* err) {
   out->assign((size_t)n, 0.0f);
@@ -292,12 +342,7 @@ bool fetch(const void* dptr, int64_t n, int dtype, std::vector<float>* out, cuda
   std::vector<uint16_t> tmp((size_t)n);
   *err = cudaMemcpy(tmp.data(), dptr, n * 2, cudaMemcpyDeviceToHost);
   if (*err != cudaSuccess) return false;
-  for (int64_t i = 0; i < n; ++i) {
-    uint32_t u = static_cast<uint32_t>(tmp[i]) << 16;
-    float f;
-    memcpy(&f, &u, 4);
-    (*out)[i] = f;
-  }
+  for (int64_t i = 0; i < n; ++i) (*out)[i] = dtype == ASR_DTYPE_F16 ? f16_to_float(tmp[i]) : bf16_to_float(tmp[i]);
   return true;
 }
 
@@ -411,7 +456,7 @@ asr_status asr_enc_create(const asr_geometry* g, const void* const* weights, int
     return bad(fail(e, ASR_E_CUDA, "cudaDeviceGetAttribute failed"));
   if (major != 10) return bad(fail(e, ASR_E_UNSUPPORTED, "this library runs on sm_100 (B200) only; device has sm_%d", major * 10));
 
-  e->kind = g->dtype == ASR_DTYPE_F32 ? KIND_TF32 : KIND_BF16;
+  e->kind = g->dtype == ASR_DTYPE_F32 ? KIND_TF32 : g->dtype == ASR_DTYPE_F16 ? KIND_F16 : KIND_BF16;
   e->es = e->kind == KIND_TF32 ? 4 : 2;
   const int rowe = kind_row_elems(e->kind);  // channels per 128-byte row of a conv operand
   const int d = g->d_model, C = g->conv_ch, L = g->n_layers;
@@ -464,10 +509,19 @@ asr_status asr_enc_create(const asr_geometry* g, const void* const* weights, int
     ++wi;
     return v;
   };
+  auto up_f16 = [&](const std::vector<float>& v) -> void* {
+    std::vector<uint16_t> h(v.size());
+    for (size_t i = 0; i < v.size(); ++i) h[i] = float_to_f16(v[i]);
+    void* p = slab_take(e, h.size() * 2);
+    if (p) note(cudaMemcpy(p, h.data(), h.size() * 2, cudaMemcpyHostToDevice), "cudaMemcpy (f16 upload)");
+    return p;
+  };
   auto gemm_w = [&](GemmB& gb, const std::vector<float>& v, int N, int K) -> bool {
     gb.kind = e->kind;
     if (e->kind == KIND_TF32)
       gb.ptr = up_f32(v);  // fp32 weights stay fp32
+    else if (e->kind == KIND_F16)
+      gb.ptr = up_f16(v);  // f16 weights stay f16 (exact round trip)
     else
       gb.ptr = up_bf16(v);
     gb.N = N;
@@ -895,7 +949,7 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
   float* mel = reinterpret_cast<float*>(ws + p.off_mel);
   float* x = reinterpret_cast<float*>(ws + p.off_x);
   // activations between the GEMMs: bf16, or fp32 on the tf32 path
-  const bool f32 = e->kind == KIND_TF32;
+  const bool f32 = e->kind == KIND_TF32, f16 = e->kind == KIND_F16;
   const int RE = kind_row_elems(e->kind), KST = RE / 4;  // conv channel block, MMA step (elements)
   void* h = ws + p.off_h;
   void* qkv = ws + p.off_qkv;
@@ -946,10 +1000,10 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
     void* a1 = ws + p.off_a1;
     if (!p.varlen)
       ASR_K(PC_CONV1, ASR_LAUNCH(e, launch_conv1_im2col(mel, clip_max, p.B, g->n_mels, p.F, g->chunk_frames,
-                                                        e->phase2 ? 1 : 0, a1, f32, st)));
+                                                        e->phase2 ? 1 : 0, a1, e->kind, st)));
     else
       ASR_K(PC_CONV1, ASR_LAUNCH(e, launch_conv1_im2col_varlen(mel, clip_max, p.chunks, g->n_mels, g->chunk_frames,
-                                                               e->phase2 ? 1 : 0, chunkd, mclips, a1, f32, st)));
+                                                               e->phase2 ? 1 : 0, chunkd, mclips, a1, e->kind, st)));
     ASR_K(PC_CONV1, ASR_TRY(gemm(e, &e->maps.a1, nullptr, e->c1, (long long)p.chunks * p.T1 * p.F1, c1, C, e->c1b,
                                  nullptr, 1, EPI_GELU, st, &e->maps.o_c1)));
     if (p.has_short)
@@ -987,7 +1041,7 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
     if (p.Tc > e->pe_rows) return fail(e, ASR_E_UNSUPPORTED, "conv1d stem: %lld positions > %d", (long long)p.Tc, e->pe_rows);
     void* melT = ws + p.off_melT;
     void* c1 = ws + p.off_c1;
-    ASR_K(PC_MISC, ASR_LAUNCH(e, launch_mel_normalize_transpose(mel, clip_max, p.B, g->n_mels, p.F, melT, f32, st)));
+    ASR_K(PC_MISC, ASR_LAUNCH(e, launch_mel_normalize_transpose(mel, clip_max, p.B, g->n_mels, p.F, melT, e->kind, st)));
     const int tpi1 = (p.F + 127) / 128, tpi2 = (int)((p.Tc + 127) / 128);
     const int CB1 = (g->n_mels + RE - 1) / RE, CBd = (d + RE - 1) / RE;
     ConvBox b1 = {128, 1, p.F, tpi1, p.B * tpi1, 1, 1, 1, 0, 1, CB1, 0, (g->n_mels - RE * (CB1 - 1) + KST - 1) / KST};
@@ -999,19 +1053,19 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
 
   for (int l = 0; l < g->n_layers; ++l) {
     const LayerW& lw = e->layers[l];
-    ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, lw.ln1g, lw.ln1b, p.T, d, g->ln_eps, h, f32, st)));
+    ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, lw.ln1g, lw.ln1b, p.T, d, g->ln_eps, h, e->kind, st)));
     ASR_K(PC_GEMM_QKV, ASR_TRY(gemm(e, &e->maps.h, nullptr, lw.qkv, p.T, qkv, 3 * d, lw.bqkv, nullptr, 1, 0, st, &e->maps.o_qkv)));
     if (f32)
       ASR_K(PC_ATTN, ASR_LAUNCH(e, launch_attention_f32(static_cast<const float*>(qkv), cu, p.nwin, p.max_win,
                                                         g->n_heads, static_cast<float*>(att), st)));
     else if (p.max_win <= 128)
-      ASR_K(PC_ATTN, ASR_LAUNCH(e, launch_attention_tc(e->maps.qkv, static_cast<const bf16*>(qkv), cu, p.nwin, g->n_heads,
-                                                       static_cast<bf16*>(att), e->status, kWaitLimitNs, st)));
+      ASR_K(PC_ATTN, ASR_LAUNCH(e, launch_attention_tc(e->maps.qkv, qkv, cu, p.nwin, g->n_heads, att, e->status,
+                                                       kWaitLimitNs, f16, st)));
     else
-      ASR_K(PC_ATTN, ASR_LAUNCH(e, launch_attention_fa(e->maps.qkv, cu, p.nwin, p.max_win, g->n_heads,
-                                                       static_cast<bf16*>(att), e->status, kWaitLimitNs, st)));
+      ASR_K(PC_ATTN, ASR_LAUNCH(e, launch_attention_fa(e->maps.qkv, cu, p.nwin, p.max_win, g->n_heads, att, e->status,
+                                                       kWaitLimitNs, f16, st)));
     ASR_K(PC_GEMM_O, ASR_TRY(gemm(e, &e->maps.att, nullptr, lw.o, p.T, x, d, lw.bo, nullptr, 1, EPI_RESID, st, &e->maps.o_x)));
-    ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, lw.ln2g, lw.ln2b, p.T, d, g->ln_eps, h, f32, st)));
+    ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, lw.ln2g, lw.ln2b, p.T, d, g->ln_eps, h, e->kind, st)));
     ASR_K(PC_GEMM_FC1, ASR_TRY(gemm(e, &e->maps.h, nullptr, lw.fc1, p.T, ff, g->d_ffn, lw.b1, nullptr, 1, EPI_GELU, st, &e->maps.o_ff)));
     ASR_K(PC_GEMM_FC2, ASR_TRY(gemm(e, &e->maps.ff, nullptr, lw.fc2, p.T, x, d, lw.b2, nullptr, 1, EPI_RESID, st, &e->maps.o_x)));
     if (l == 0)
@@ -1020,7 +1074,7 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
   if (float* t = tap(ASR_TAP_ENCODER)) ASR_LAUNCH(e, cudaMemcpyAsync(t, x, (size_t)p.T * d * 4, cudaMemcpyDeviceToDevice, st));
 
   if (!g->proj1_out) {
-    ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, e->lnpg, e->lnpb, p.T, d, g->ln_eps, out, true, st)));
+    ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, e->lnpg, e->lnpb, p.T, d, g->ln_eps, out, KIND_TF32, st)));
     return ASR_OK;
   }
   void* p1 = ws + p.off_p1;
@@ -1028,7 +1082,7 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
   // Store map of the caller's output (plain stores if it is not 16-byte aligned).
   CUtensorMap o_out_map;
   const CUtensorMap* o_out = make_tmap_out(&o_out_map, out, p.T, d_out(g), d_out(g), true) ? &o_out_map : nullptr;
-  ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, e->lnpg, e->lnpb, p.T, d, g->ln_eps, h, f32, st)));
+  ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, e->lnpg, e->lnpb, p.T, d, g->ln_eps, h, e->kind, st)));
   ASR_K(PC_GEMM_HEAD, ASR_TRY(gemm(e, &e->maps.h, nullptr, e->p1, p.T, p1, g->proj1_out, e->bp1, nullptr, 1, EPI_GELU, st, &e->maps.o_p1)));
   if (!g->adapter_hidden) {
     ASR_K(PC_GEMM_HEAD, ASR_TRY(gemm(e, &e->maps.p1, nullptr, e->p2, p.T, out, g->proj2_out, e->bp2, nullptr, 1, EPI_OUT_F32, st, o_out)));
@@ -1040,7 +1094,7 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
     if (f32)
       ASR_LAUNCH(e, cudaMemcpyAsync(t, p2, (size_t)p.T * g->proj2_out * 4, cudaMemcpyDeviceToDevice, st));
     else
-      ASR_K(PC_MISC, ASR_LAUNCH(e, launch_bf16_to_f32(static_cast<const bf16*>(p2), t, (long long)p.T * g->proj2_out, st)));
+      ASR_K(PC_MISC, ASR_LAUNCH(e, launch_bf16_to_f32(p2, t, (long long)p.T * g->proj2_out, f16, st)));
   }
   void* gu = ws + p.off_gu;
   ASR_K(PC_GEMM_ADAPTER, ASR_TRY(gemm(e, &e->maps.p2, nullptr, e->gu, p.T, gu, g->adapter_hidden, nullptr, nullptr, 1, EPI_SWIGLU, st, nullptr)));
@@ -1355,7 +1409,7 @@ asr_status asr_op_linear_tf32(const float* x, const float* w, const float* bias,
 asr_status asr_op_layer_norm(const float* x, const float* g, const float* b, int64_t M, int D, float eps, void* y,
                              int out_f32, void* stream) {
   if (!x || !g || !b || !y || M <= 0 || D % 128 || D > 2048) return fail(nullptr, ASR_E_INVAL, "layer_norm: bad arguments");
-  ASR_CUDA(nullptr, launch_layer_norm(x, g, b, M, D, eps, y, out_f32 != 0, static_cast<cudaStream_t>(stream)));
+  ASR_CUDA(nullptr, launch_layer_norm(x, g, b, M, D, eps, y, out_f32 ? KIND_TF32 : KIND_BF16, static_cast<cudaStream_t>(stream)));
   return ASR_OK;
 }
 
@@ -1371,11 +1425,9 @@ asr_status asr_op_attention(const void* qkv, const int32_t* cu, int n_seg, int m
   if (!make_tmap_qkv(&m, qkv, T, H)) return fail(nullptr, ASR_E_INVAL, "attention: TMA descriptor encoding failed");
   ASR_CUDA(nullptr, cudaMemsetAsync(ws, 0, 4, st));
   if (max_seg <= 128)
-    ASR_CUDA(nullptr, launch_attention_tc(m, static_cast<const bf16*>(qkv), cu, n_seg, H, static_cast<bf16*>(out),
-                                          static_cast<int*>(ws), kWaitLimitNs, st));
+    ASR_CUDA(nullptr, launch_attention_tc(m, qkv, cu, n_seg, H, out, static_cast<int*>(ws), kWaitLimitNs, false, st));
   else
-    ASR_CUDA(nullptr, launch_attention_fa(m, cu, n_seg, max_seg, H, static_cast<bf16*>(out), static_cast<int*>(ws),
-                                          kWaitLimitNs, st));
+    ASR_CUDA(nullptr, launch_attention_fa(m, cu, n_seg, max_seg, H, out, static_cast<int*>(ws), kWaitLimitNs, false, st));
   return ASR_OK;
 }
 

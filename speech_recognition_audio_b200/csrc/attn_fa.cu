@@ -16,9 +16,9 @@
 //           exponentials moves only when a tile's maximum exceeds it by
 //           more than 8 (then O and the row sum are rescaled by
 //           2^(old - new)), so probabilities stay <= 256 and most tiles need
-//           no rescale.  P (bf16) goes to shared memory as the A operand of
-//           the next MMA; at the end each thread divides its O row by its
-//           sum and stores it.
+//           no rescale.  P (bf16 or f16, the operands' type) goes to shared
+//           memory as the A operand of the next MMA; at the end each thread
+//           divides its O row by its sum and stores it.
 // Tensor memory: S in columns 0..127, O in 128..191 (256 allocated: two
 // CTAs per SM).  Shared memory: Q, K, V (16 KB each), P (32 KB).  Every wait
 // is bounded; tensor memory is freed after all MMAs have completed.
@@ -51,6 +51,7 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 }  // namespace
 
+template <int KIND>
 __global__ void __launch_bounds__(FA_THREADS, 2) attention_fa_kernel(const __grid_constant__ CUtensorMap tm_qkv,
                                                                      const int* __restrict__ cu, int H,
                                                                      bf16* __restrict__ out, int* status,
@@ -116,8 +117,8 @@ __global__ void __launch_bounds__(FA_THREADS, 2) attention_fa_kernel(const __gri
     } else if (warp == 5) {
       // ------------------------------------------------ MMA issuer
       if (lane == 0) {
-        const uint32_t idesc_s = idesc_bf16_f32(128, 128);
-        const uint32_t idesc_o = idesc_bf16_f32(128, 64) | (1u << 16);  // B = V, MN-major
+        const uint32_t idesc_s = idesc_kind_f32(KIND, 128, 128);
+        const uint32_t idesc_o = idesc_kind_f32(KIND, 128, 64) | (1u << 16);  // B = V, MN-major
         const uint64_t qd = sw128_kmajor_desc(smem_u32(sm + FA_SQ));
         const uint64_t kd = sw128_kmajor_desc(smem_u32(sm + FA_SK));
         const uint64_t vd = sw128_mnmajor_desc(smem_u32(sm + FA_SV));
@@ -230,11 +231,7 @@ __global__ void __launch_bounds__(FA_THREADS, 2) attention_fa_kernel(const __gri
           uint4* prow = reinterpret_cast<uint4*>(sm + FA_SP + kb * 16384 + row * 128);
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            const float* q = sv + kb * 64 + c * 8;
-            alignas(16) __nv_bfloat162 r[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) r[i] = __floats2bfloat162_rn(q[2 * i], q[2 * i + 1]);
-            prow[c ^ (row & 7)] = *reinterpret_cast<uint4*>(r);
+            prow[c ^ (row & 7)] = pack8_16<KIND>(sv + kb * 64 + c * 8);
           }
         }
         fence_proxy_async_smem();
@@ -255,10 +252,10 @@ __global__ void __launch_bounds__(FA_THREADS, 2) attention_fa_kernel(const __gri
         uint4* dst = reinterpret_cast<uint4*>(out + (long long)(s0 + q0 + row) * (H * 64) + h * 64);
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          alignas(16) __nv_bfloat162 r[4];
+          float t8[8];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) r[i] = __floats2bfloat162_rn(ov[8 * c + 2 * i] * inv, ov[8 * c + 2 * i + 1] * inv);
-          dst[c] = *reinterpret_cast<uint4*>(r);
+          for (int i = 0; i < 8; ++i) t8[i] = ov[8 * c + i] * inv;
+          dst[c] = pack8_16<KIND>(t8);
         }
       }
     }
@@ -269,16 +266,25 @@ __global__ void __launch_bounds__(FA_THREADS, 2) attention_fa_kernel(const __gri
   if (warp == 0) tmem_dealloc(tmem, FA_TMEM_COLS);
 }
 
-cudaError_t launch_attention_fa(const CUtensorMap& tm_qkv, const int* cu, int n_seg, int max_seg, int H, bf16* out,
-                                int* status, unsigned long long limit_ns, cudaStream_t st) {
-  if (n_seg <= 0 || max_seg <= 0 || H <= 0) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(attention_fa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FA_SMEM);
+template <int KIND>
+static cudaError_t launch_fa(const CUtensorMap& tm_qkv, const int* cu, int n_seg, int max_seg, int H, bf16* out,
+                             int* status, unsigned long long limit_ns, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(attention_fa_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, FA_SMEM);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(attention_fa_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+    e = cudaFuncSetAttribute(attention_fa_kernel<KIND>, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   dim3 grid((max_seg + 127) / 128, n_seg, H);
-  return launch_pdl(attention_fa_kernel, grid, dim3(FA_THREADS), FA_SMEM, st, tm_qkv, cu, H, out, status, limit_ns);
+  return launch_pdl(attention_fa_kernel<KIND>, grid, dim3(FA_THREADS), FA_SMEM, st, tm_qkv, cu, H, out, status, limit_ns);
+}
+
+// out: bf16, or f16 with f16 != 0.
+cudaError_t launch_attention_fa(const CUtensorMap& tm_qkv, const int* cu, int n_seg, int max_seg, int H, void* out,
+                                int* status, unsigned long long limit_ns, bool f16, cudaStream_t st) {
+  if (n_seg <= 0 || max_seg <= 0 || H <= 0) return cudaErrorInvalidValue;
+  bf16* o = static_cast<bf16*>(out);
+  return f16 ? launch_fa<KIND_F16>(tm_qkv, cu, n_seg, max_seg, H, o, status, limit_ns, st)
+             : launch_fa<KIND_BF16>(tm_qkv, cu, n_seg, max_seg, H, o, status, limit_ns, st);
 }
 
 }  // namespace asr

@@ -12,8 +12,8 @@
 //   - S = Q K^T: tcgen05.mma M=128 N=128 K=64 into tensor memory;
 //   - each thread owns one query row: tcgen05.ld of its 128 scores, scale
 //     1/8, mask keys >= L, max, exp2 (over the 16-key chunks below L), sum;
-//     P (bf16) is written row-major, swizzled, over the Q and K tiles as the
-//     A operand of the next MMA;
+//     P (bf16, or f16 for f16 operands) is written row-major, swizzled, over
+//     the Q and K tiles as the A operand of the next MMA;
 //   - O = P V: tcgen05.mma M=128 N=64 K=128 into S's tensor-memory columns;
 //   48 KB of shared memory and 128 TMEM columns per block: 4 blocks per SM.
 //   - each thread scales its output row by 1 / sum and stores 128 bytes.
@@ -31,6 +31,7 @@ constexpr int AT_SMEM = 1024 + 49152 + 64;  // tiles + barriers + TMEM slot
 constexpr int AT_TMEM_COLS = 128;           // S (128 columns), then O (64) in the same columns
 }  // namespace
 
+template <int KIND>
 __global__ void __launch_bounds__(AT_THREADS) attention_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv,
                                                                    const bf16* __restrict__ qkv,
                                                                    const int* __restrict__ cu, int H,
@@ -77,7 +78,7 @@ __global__ void __launch_bounds__(AT_THREADS) attention_tc_kernel(const __grid_c
     ok = mbar_wait_bounded(bar_qk, 0, limit_ns, status, DEV_TIMEOUT_MMA);
     if (ok) {
       tc_fence_after();
-      const uint32_t idesc = idesc_bf16_f32(128, 128);
+      const uint32_t idesc = idesc_kind_f32(KIND, 128, 128);
       const uint64_t ad = sw128_kmajor_desc(smem_u32(sm + SQ)), bd = sw128_kmajor_desc(smem_u32(sm + SK));
 #pragma unroll
       for (int k = 0; k < 4; ++k) tc_mma_bf16(tmem, ad + 2 * k, bd + 2 * k, idesc, k > 0 ? 1u : 0u);
@@ -128,11 +129,7 @@ __global__ void __launch_bounds__(AT_THREADS) attention_tc_kernel(const __grid_c
       uint4* prow = reinterpret_cast<uint4*>(sm + SP + kb * 16384 + row * 128);
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        const float* q = sv + kb * 64 + c * 8;
-        alignas(16) __nv_bfloat162 r[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) r[i] = __floats2bfloat162_rn(q[2 * i], q[2 * i + 1]);
-        prow[c ^ (row & 7)] = *reinterpret_cast<uint4*>(r);
+        prow[c ^ (row & 7)] = pack8_16<KIND>(sv + kb * 64 + c * 8);
       }
     }
   }
@@ -145,7 +142,7 @@ __global__ void __launch_bounds__(AT_THREADS) attention_tc_kernel(const __grid_c
     if (ok) {
       // B = V stored keys x dims (dims contiguous): MN-major, 128-byte swizzle,
       // 8-key groups 1024 bytes apart; each K=16 step advances 16 keys (2048 B).
-      const uint32_t idesc = idesc_bf16_f32(128, 64) | (1u << 16);
+      const uint32_t idesc = idesc_kind_f32(KIND, 128, 64) | (1u << 16);
       const uint64_t bd0 = sw128_mnmajor_desc(smem_u32(sm + SV));
 #pragma unroll
       for (int kb = 0; kb < 2; ++kb) {
@@ -170,10 +167,10 @@ __global__ void __launch_bounds__(AT_THREADS) attention_tc_kernel(const __grid_c
       uint4* dst = reinterpret_cast<uint4*>(out + (long long)(s0 + row) * (H * 64) + h * 64);
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        alignas(16) __nv_bfloat162 r[4];
+        float t8[8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) r[i] = __floats2bfloat162_rn(ov[8 * c + 2 * i] * rsum, ov[8 * c + 2 * i + 1] * rsum);
-        dst[c] = *reinterpret_cast<uint4*>(r);
+        for (int i = 0; i < 8; ++i) t8[i] = ov[8 * c + i] * rsum;
+        dst[c] = pack8_16<KIND>(t8);
       }
     }
   }
@@ -190,17 +187,27 @@ bool make_tmap_qkv(CUtensorMap* map, const void* qkv, long long T, int H) {
   return make_tmap_bf16(map, qkv, (unsigned long long)T, 3ULL * H * 64, 3ULL * H * 64, 128);
 }
 
-cudaError_t launch_attention_tc(const CUtensorMap& tm_qkv, const bf16* qkv, const int* cu, int n_seg, int H, bf16* out,
-                                int* status, unsigned long long limit_ns, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM);
+template <int KIND>
+static cudaError_t launch_tc(const CUtensorMap& tm_qkv, const bf16* qkv, const int* cu, int n_seg, int H, bf16* out,
+                             int* status, unsigned long long limit_ns, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(attention_tc_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM);
   // Ask for the whole shared-memory carveout: without it the driver picked a
   // 164 KB configuration (3 blocks per SM, 2.7 waves for 1200 blocks).
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+    e = cudaFuncSetAttribute(attention_tc_kernel<KIND>, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
-  return launch_pdl(attention_tc_kernel, dim3(n_seg, H), dim3(AT_THREADS), AT_SMEM, st, tm_qkv, qkv, cu, H, out, status,
-                    limit_ns);
+  return launch_pdl(attention_tc_kernel<KIND>, dim3(n_seg, H), dim3(AT_THREADS), AT_SMEM, st, tm_qkv, qkv, cu, H, out,
+                    status, limit_ns);
+}
+
+// qkv / out: bf16, or f16 with f16 != 0 (the bytes pass through TMA as they are).
+cudaError_t launch_attention_tc(const CUtensorMap& tm_qkv, const void* qkv, const int* cu, int n_seg, int H, void* out,
+                                int* status, unsigned long long limit_ns, bool f16, cudaStream_t st) {
+  const bf16* q = static_cast<const bf16*>(qkv);
+  bf16* o = static_cast<bf16*>(out);
+  return f16 ? launch_tc<KIND_F16>(tm_qkv, q, cu, n_seg, H, o, status, limit_ns, st)
+             : launch_tc<KIND_BF16>(tm_qkv, q, cu, n_seg, H, o, status, limit_ns, st);
 }
 
 }  // namespace asr

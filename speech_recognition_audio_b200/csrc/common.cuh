@@ -215,6 +215,25 @@ __host__ __device__ constexpr uint32_t idesc_kind_f32(int kind, int M, int N) {
   return (1u << 4) | (kind == KIND_TF32 ? (2u << 7) | (2u << 10) : kind == KIND_F16 ? 0u : (1u << 7) | (1u << 10)) |
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
+// Two fp32 values rounded to nearest-even into a packed pair of the kind's
+// 16-bit type (f16 for KIND_F16, else bf16), low half first.
+template <int KIND>
+__device__ __forceinline__ uint32_t pack2_16(float a, float b) {
+  if constexpr (KIND == KIND_F16) {
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+  } else {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+}
+// Eight fp32 values as one 16-byte chunk of the kind's 16-bit type.
+template <int KIND>
+__device__ __forceinline__ uint4 pack8_16(const float* v) {
+  return make_uint4(pack2_16<KIND>(v[0], v[1]), pack2_16<KIND>(v[2], v[3]), pack2_16<KIND>(v[4], v[5]),
+                    pack2_16<KIND>(v[6], v[7]));
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T, kind::tf32 (fp32 operands, fp32 accumulate).
 __device__ __forceinline__ void tc_mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                             uint32_t accumulate) {

@@ -33,10 +33,14 @@ constexpr int stages_for() {
   return BN >= 192 ? 4 : (BN > 128 ? 5 : (BN == 128 ? 6 : 8));
 }
 
-template <int BN, bool G, int EPI>
+template <int BN, bool G, int EPI, int KIND>
 cudaError_t run(const CUtensorMap* a, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& p, int grid, cudaStream_t st) {
   using S = GemmShape<BN, stages_for<BN>(), G>;
-  auto k = gemm_bf16_tc_kernel<BN, S::STAGES, G, EPI>;
+  void (*k)(CUtensorMap, CUtensorMap, CUtensorMap, GemmParams);
+  if constexpr (KIND == KIND_F16)
+    k = gemm_f16_tc_kernel<BN, S::STAGES, G, EPI>;
+  else
+    k = gemm_bf16_tc_kernel<BN, S::STAGES, G, EPI>;
   cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_BYTES);
   if (err != cudaSuccess) return err;
   return launch_pdl(k, dim3(grid), dim3(S::THREADS), S::SMEM_BYTES, st, a ? *a : b, b, o, p);
@@ -67,44 +71,49 @@ cudaError_t run_tf32_epi(int epi, const CUtensorMap& a, const CUtensorMap& b, co
   }
 }
 
-template <int BN>
+template <int BN, int KIND>
 cudaError_t run_tma(int epi, const CUtensorMap* a, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& p, int grid,
                     cudaStream_t st) {
   switch (epi) {
-    case 0: return run<BN, false, 0>(a, b, o, p, grid, st);
-    case EPI_GELU: return run<BN, false, EPI_GELU>(a, b, o, p, grid, st);
-    case EPI_OUT_F32: return run<BN, false, EPI_OUT_F32>(a, b, o, p, grid, st);
-    case EPI_RESID: return run<BN, false, EPI_RESID>(a, b, o, p, grid, st);
-    case EPI_OUT_F32 | EPI_PE: return run<BN, false, EPI_OUT_F32 | EPI_PE>(a, b, o, p, grid, st);
-    case EPI_SWIGLU: return run<BN, false, EPI_SWIGLU>(a, b, o, p, grid, st);
-    case EPI_GELU | EPI_OUT_F32 | EPI_PE: return run<BN, false, EPI_GELU | EPI_OUT_F32 | EPI_PE>(a, b, o, p, grid, st);
+    case 0: return run<BN, false, 0, KIND>(a, b, o, p, grid, st);
+    case EPI_GELU: return run<BN, false, EPI_GELU, KIND>(a, b, o, p, grid, st);
+    case EPI_OUT_F32: return run<BN, false, EPI_OUT_F32, KIND>(a, b, o, p, grid, st);
+    case EPI_RESID: return run<BN, false, EPI_RESID, KIND>(a, b, o, p, grid, st);
+    case EPI_OUT_F32 | EPI_PE: return run<BN, false, EPI_OUT_F32 | EPI_PE, KIND>(a, b, o, p, grid, st);
+    case EPI_SWIGLU: return run<BN, false, EPI_SWIGLU, KIND>(a, b, o, p, grid, st);
+    case EPI_GELU | EPI_OUT_F32 | EPI_PE: return run<BN, false, EPI_GELU | EPI_OUT_F32 | EPI_PE, KIND>(a, b, o, p, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
 // 240-wide tiles only serve the convolutions (N = 480).
+template <int KIND>
 cudaError_t run_tma240(int epi, const CUtensorMap* a, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& p, int grid,
                        cudaStream_t st) {
   switch (epi) {
-    case EPI_GELU: return run<240, false, EPI_GELU>(a, b, o, p, grid, st);
-    case EPI_GELU | EPI_OUT_F32 | EPI_PE: return run<240, false, EPI_GELU | EPI_OUT_F32 | EPI_PE>(a, b, o, p, grid, st);
+    case EPI_GELU: return run<240, false, EPI_GELU, KIND>(a, b, o, p, grid, st);
+    case EPI_GELU | EPI_OUT_F32 | EPI_PE: return run<240, false, EPI_GELU | EPI_OUT_F32 | EPI_PE, KIND>(a, b, o, p, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <int BN>
+template <int BN, int KIND>
 cudaError_t run_gather(int epi, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& p, int grid, cudaStream_t st) {
   switch (epi) {
-    case EPI_GELU: return run<BN, true, EPI_GELU>(nullptr, b, o, p, grid, st);
-    case EPI_GELU | EPI_OUT_F32 | EPI_PE: return run<BN, true, EPI_GELU | EPI_OUT_F32 | EPI_PE>(nullptr, b, o, p, grid, st);
+    case EPI_GELU: return run<BN, true, EPI_GELU, KIND>(nullptr, b, o, p, grid, st);
+    case EPI_GELU | EPI_OUT_F32 | EPI_PE: return run<BN, true, EPI_GELU | EPI_OUT_F32 | EPI_PE, KIND>(nullptr, b, o, p, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, int KIND>
 cudaError_t run2(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& p, int grid, cudaStream_t st) {
   using S = Gemm2Shape<BN, (BN >= 192 ? 6 : 8), gemm2_epi_warps<EPI>()>;
-  auto k = gemm_bf16_tc2_kernel<BN, S::STAGES, EPI>;
+  void (*k)(CUtensorMap, CUtensorMap, CUtensorMap, GemmParams);
+  if constexpr (KIND == KIND_F16)
+    k = gemm_f16_tc2_kernel<BN, S::STAGES, EPI>;
+  else
+    k = gemm_bf16_tc2_kernel<BN, S::STAGES, EPI>;
   cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_BYTES);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
@@ -124,26 +133,27 @@ cudaError_t run2(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& 
   return cudaLaunchKernelEx(&cfg, k, a, b, o, p);
 }
 
-template <int BN>
+template <int BN, int KIND>
 cudaError_t run2_epi(int epi, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& p, int grid,
                      cudaStream_t st) {
   switch (epi) {
-    case 0: return run2<BN, 0>(a, b, o, p, grid, st);
-    case EPI_GELU: return run2<BN, EPI_GELU>(a, b, o, p, grid, st);
-    case EPI_OUT_F32: return run2<BN, EPI_OUT_F32>(a, b, o, p, grid, st);
-    case EPI_RESID: return run2<BN, EPI_RESID>(a, b, o, p, grid, st);
-    case EPI_OUT_F32 | EPI_PE: return run2<BN, EPI_OUT_F32 | EPI_PE>(a, b, o, p, grid, st);
-    case EPI_SWIGLU: return run2<BN, EPI_SWIGLU>(a, b, o, p, grid, st);
-    case EPI_GELU | EPI_OUT_F32 | EPI_PE: return run2<BN, EPI_GELU | EPI_OUT_F32 | EPI_PE>(a, b, o, p, grid, st);
+    case 0: return run2<BN, 0, KIND>(a, b, o, p, grid, st);
+    case EPI_GELU: return run2<BN, EPI_GELU, KIND>(a, b, o, p, grid, st);
+    case EPI_OUT_F32: return run2<BN, EPI_OUT_F32, KIND>(a, b, o, p, grid, st);
+    case EPI_RESID: return run2<BN, EPI_RESID, KIND>(a, b, o, p, grid, st);
+    case EPI_OUT_F32 | EPI_PE: return run2<BN, EPI_OUT_F32 | EPI_PE, KIND>(a, b, o, p, grid, st);
+    case EPI_SWIGLU: return run2<BN, EPI_SWIGLU, KIND>(a, b, o, p, grid, st);
+    case EPI_GELU | EPI_OUT_F32 | EPI_PE: return run2<BN, EPI_GELU | EPI_OUT_F32 | EPI_PE, KIND>(a, b, o, p, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
+template <int KIND>
 cudaError_t run2_240(int epi, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& p, int grid,
                      cudaStream_t st) {
   switch (epi) {
-    case EPI_GELU: return run2<240, EPI_GELU>(a, b, o, p, grid, st);
-    case EPI_GELU | EPI_OUT_F32 | EPI_PE: return run2<240, EPI_GELU | EPI_OUT_F32 | EPI_PE>(a, b, o, p, grid, st);
+    case EPI_GELU: return run2<240, EPI_GELU, KIND>(a, b, o, p, grid, st);
+    case EPI_GELU | EPI_OUT_F32 | EPI_PE: return run2<240, EPI_GELU | EPI_OUT_F32 | EPI_PE, KIND>(a, b, o, p, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -338,10 +348,10 @@ int gemm_pick_bn_conv(int n_sub, int N, int num_sms) {
   return (w2 * 93 <= w1 * 100) ? -bn : bn;
 }
 
-cudaError_t launch_gemm(const CUtensorMap* a_map, const GemmB& w, GemmParams p, int epi, int bn, int num_sms,
-                        cudaStream_t st, const CUtensorMap* out_map) {
+template <int KIND>
+cudaError_t launch16(const CUtensorMap* a_map, const GemmB& w, GemmParams p, int epi, int bn, int num_sms,
+                     cudaStream_t st, const CUtensorMap* out_map) {
   p.out_tma = (out_map != nullptr && !(epi & (EPI_PE | EPI_SWIGLU))) ? 1 : 0;
-  if (w.kind == KIND_TF32 && bn < 0) return cudaErrorInvalidValue;  // the CTA-pair kernel takes 16-bit operands
   // Tile order: the tiles running at once share the larger operand, so it
   // crosses from DRAM once and is re-read from L2 (and the TMA latency the
   // stage ring has to cover is the L2's, not the DRAM's).  A (M x K) is the
@@ -369,32 +379,14 @@ cudaError_t launch_gemm(const CUtensorMap* a_map, const GemmB& w, GemmParams p, 
             p.num_tiles % pairs != 0)
                ? 1
                : 0;
-    if (w2 == 240) return run2_240(epi, *a_map, w.map[slot2], p.out_tma ? *out_map : w.map[slot2], p, grid, st);
+    if (w2 == 240) return run2_240<KIND>(epi, *a_map, w.map[slot2], p.out_tma ? *out_map : w.map[slot2], p, grid, st);
     const CUtensorMap& o2 = p.out_tma ? *out_map : w.map[slot2];
-    return w2 == 256 ? run2_epi<256>(epi, *a_map, w.map[slot2], o2, p, grid, st)
-                     : run2_epi<128>(epi, *a_map, w.map[slot2], o2, p, grid, st);
+    return w2 == 256 ? run2_epi<256, KIND>(epi, *a_map, w.map[slot2], o2, p, grid, st)
+                     : run2_epi<128, KIND>(epi, *a_map, w.map[slot2], o2, p, grid, st);
   }
   const int slot = gemm_bn_slot(bn);
   if (slot < 0 || p.M <= 0) return cudaErrorInvalidValue;
   p.sk = 0;  // the one-SM kernel runs whole tiles
-  if (w.kind == KIND_TF32) {
-    if (!a_map) return cudaErrorInvalidValue;  // no gather mode for fp32 operands
-    p.N = w.N;
-    p.K = w.K;
-    p.m_blocks = p.conv_box ? p.cb.n_sub : (p.M + 127) / 128;
-    p.n_blocks = (p.N + bn - 1) / bn;
-    p.k_blocks = (p.K + 31) / 32;
-    p.num_tiles = p.m_blocks * p.n_blocks;
-    const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
-    const CUtensorMap& b = w.map[slot];
-    const CUtensorMap& o = p.out_tma ? *out_map : b;
-    switch (bn) {
-      case 256: return run_tf32_epi<256>(epi, *a_map, b, o, p, grid, st);
-      case 128: return run_tf32_epi<128>(epi, *a_map, b, o, p, grid, st);
-      case 64: return run_tf32_epi<64>(epi, *a_map, b, o, p, grid, st);
-      default: return cudaErrorInvalidValue;
-    }
-  }
   p.N = w.N;
   p.K = w.K;
   p.m_blocks = p.conv_box ? p.cb.n_sub : (p.M + 127) / 128;
@@ -407,19 +399,47 @@ cudaError_t launch_gemm(const CUtensorMap* a_map, const GemmB& w, GemmParams p, 
   const bool gather = (a_map == nullptr);
   if (gather) {
     switch (bn) {
-      case 256: return run_gather<256>(epi, b, o, p, grid, st);
-      case 240: return run_gather<240>(epi, b, o, p, grid, st);
-      case 128: return run_gather<128>(epi, b, o, p, grid, st);
-      case 64: return run_gather<64>(epi, b, o, p, grid, st);
+      case 256: return run_gather<256, KIND>(epi, b, o, p, grid, st);
+      case 240: return run_gather<240, KIND>(epi, b, o, p, grid, st);
+      case 128: return run_gather<128, KIND>(epi, b, o, p, grid, st);
+      case 64: return run_gather<64, KIND>(epi, b, o, p, grid, st);
       default: return cudaErrorInvalidValue;
     }
   }
   switch (bn) {
-    case 256: return run_tma<256>(epi, a_map, b, o, p, grid, st);
-    case 240: return run_tma240(epi, a_map, b, o, p, grid, st);
-    case 160: return run_tma<160>(epi, a_map, b, o, p, grid, st);
-    case 128: return run_tma<128>(epi, a_map, b, o, p, grid, st);
-    case 64: return run_tma<64>(epi, a_map, b, o, p, grid, st);
+    case 256: return run_tma<256, KIND>(epi, a_map, b, o, p, grid, st);
+    case 240: return run_tma240<KIND>(epi, a_map, b, o, p, grid, st);
+    case 160: return run_tma<160, KIND>(epi, a_map, b, o, p, grid, st);
+    case 128: return run_tma<128, KIND>(epi, a_map, b, o, p, grid, st);
+    case 64: return run_tma<64, KIND>(epi, a_map, b, o, p, grid, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_gemm(const CUtensorMap* a_map, const GemmB& w, GemmParams p, int epi, int bn, int num_sms,
+                        cudaStream_t st, const CUtensorMap* out_map) {
+  if (w.kind == KIND_BF16) return launch16<KIND_BF16>(a_map, w, p, epi, bn, num_sms, st, out_map);
+  if (w.kind == KIND_F16) return launch16<KIND_F16>(a_map, w, p, epi, bn, num_sms, st, out_map);
+  // fp32 operands: one-SM tiles only (the CTA-pair kernel takes 16-bit
+  // operands), no gather mode
+  p.out_tma = (out_map != nullptr && !(epi & (EPI_PE | EPI_SWIGLU))) ? 1 : 0;
+  p.n_fast = (p.conv_box || p.M > w.N) ? 1 : 0;
+  const int slot = gemm_bn_slot(bn);
+  if (bn < 0 || slot < 0 || p.M <= 0 || !a_map) return cudaErrorInvalidValue;
+  p.sk = 0;
+  p.N = w.N;
+  p.K = w.K;
+  p.m_blocks = p.conv_box ? p.cb.n_sub : (p.M + 127) / 128;
+  p.n_blocks = (p.N + bn - 1) / bn;
+  p.k_blocks = (p.K + 31) / 32;
+  p.num_tiles = p.m_blocks * p.n_blocks;
+  const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
+  const CUtensorMap& b = w.map[slot];
+  const CUtensorMap& o = p.out_tma ? *out_map : b;
+  switch (bn) {
+    case 256: return run_tf32_epi<256>(epi, *a_map, b, o, p, grid, st);
+    case 128: return run_tf32_epi<128>(epi, *a_map, b, o, p, grid, st);
+    case 64: return run_tf32_epi<64>(epi, *a_map, b, o, p, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }

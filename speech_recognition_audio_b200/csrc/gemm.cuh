@@ -351,7 +351,7 @@ __device__ __forceinline__ void load_bias(const GemmParams& p, int n0, int BN, i
 //   Stream-K pieces (residual epilogue only): PIECE_PARTIAL adds its raw
 //     accumulator (no bias) to the residual stream; the caller orders the
 //     owner's update after it.
-template <int EPI>
+template <int EPI, int KIND = KIND_BF16>
 __device__ __forceinline__ void epilogue_warp(const GemmParams& p, const CUtensorMap* tm_out, uint32_t tb, int row0,
                                               int mlimit, int n0, int BN, int half, int lane, uint8_t* wbuf,
                                               const float* breg, int kind = PIECE_FULL, int cstride = 64) {
@@ -399,13 +399,13 @@ __device__ __forceinline__ void epilogue_warp(const GemmParams& p, const CUtenso
       uint4* row = reinterpret_cast<uint4*>(wbuf + lane * 64);
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
-        alignas(16) __nv_bfloat162 r[4];
+        uint32_t r[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int jj = 8 * k + 2 * i;
-          r[i] = __floats2bfloat162_rn(silu(v[jj]) * v[16 + jj], silu(v[jj + 1]) * v[17 + jj]);
+          r[i] = pack2_16<KIND>(silu(v[jj]) * v[16 + jj], silu(v[jj + 1]) * v[17 + jj]);
         }
-        row[k ^ ((lane >> 1) & 3)] = *reinterpret_cast<uint4*>(r);
+        row[k ^ ((lane >> 1) & 3)] = make_uint4(r[0], r[1], r[2], r[3]);
       }
     } else {
       if (EPI & EPI_GELU) {
@@ -423,12 +423,7 @@ __device__ __forceinline__ void epilogue_warp(const GemmParams& p, const CUtenso
       } else {
         uint4* row = reinterpret_cast<uint4*>(wbuf + lane * 64);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          alignas(16) __nv_bfloat162 r[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) r[i] = __floats2bfloat162_rn(v[8 * k + 2 * i], v[8 * k + 2 * i + 1]);
-          row[k ^ ((lane >> 1) & 3)] = *reinterpret_cast<uint4*>(r);
-        }
+        for (int k = 0; k < 4; ++k) row[k ^ ((lane >> 1) & 3)] = pack8_16<KIND>(v + 8 * k);
       }
     }
     if (use_tma) {
@@ -668,7 +663,7 @@ __device__ __forceinline__ void gemm_tc_body(const CUtensorMap& tmA, const CUten
       int r_first, r_last;
       subtile_rows(p, mb, r_first, r_last);
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + a * S::ACC_COLS;
-      epilogue_warp<EPI>(p, &tmOut, tb, r_first + 32 * q, r_last, n0, BN, half, lane, sEpi + (warp - 2) * 4096, breg);
+      epilogue_warp<EPI, KIND>(p, &tmOut, tb, r_first + 32 * q, r_last, n0, BN, half, lane, sEpi + (warp - 2) * 4096, breg);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[a]);
@@ -749,6 +744,14 @@ __global__ void __launch_bounds__(GemmShape<BN, STAGES, GATHER>::THREADS, 1)
     gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
   gemm_tc_body<BN, STAGES, GATHER, EPI, KIND_BF16>(tmA, tmB, tmOut, p);
+}
+
+// f16 operands (kind::f16).
+template <int BN, int STAGES, bool GATHER, int EPI>
+__global__ void __launch_bounds__(GemmShape<BN, STAGES, GATHER>::THREADS, 1)
+    gemm_f16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                       const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
+  gemm_tc_body<BN, STAGES, GATHER, EPI, KIND_F16>(tmA, tmB, tmOut, p);
 }
 
 // fp32 operands in memory, multiplied as tf32 (kind::tf32), fp32 accumulate.

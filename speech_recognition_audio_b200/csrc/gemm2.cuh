@@ -121,10 +121,9 @@ constexpr int gemm2_epi_warps() {
   return EPI == EPI_GELU ? 16 : 8;
 }
 
-template <int BN, int STAGES, int EPI>
-__global__ void __launch_bounds__(Gemm2Shape<BN, STAGES, gemm2_epi_warps<EPI>()>::THREADS, 1)
-    gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                         const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
+template <int BN, int STAGES, int EPI, int KIND>
+__device__ __forceinline__ void gemm_tc2_body(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmOut,
+                                              const GemmParams& p) {
   using S = Gemm2Shape<BN, STAGES, gemm2_epi_warps<EPI>()>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -218,7 +217,7 @@ __global__ void __launch_bounds__(Gemm2Shape<BN, STAGES, gemm2_epi_warps<EPI>()>
     }
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
-      const uint32_t idesc = idesc_bf16_f32(S::BM, BN);
+      const uint32_t idesc = idesc_kind_f32(KIND, S::BM, BN);
       int it = 0, tl = 0;
       bool ok = true;
       PieceIter pi(p, pair, n_pairs);
@@ -294,8 +293,8 @@ __global__ void __launch_bounds__(Gemm2Shape<BN, STAGES, gemm2_epi_warps<EPI>()>
         have = __shfl_sync(0xffffffffu, have, 0);
       }
       if (have)
-        epilogue_warp<EPI>(p, &tmOut, tb, r_first + 32 * q, r_last, n0, BN, half, lane, sEpi + ew * S::WBUF, breg, kind,
-                           S::CSTRIDE);
+        epilogue_warp<EPI, KIND>(p, &tmOut, tb, r_first + 32 * q, r_last, n0, BN, half, lane, sEpi + ew * S::WBUF, breg,
+                                 kind, S::CSTRIDE);
       tc_fence_before();
       __syncwarp();
       if (kind == PIECE_PARTIAL && lane == 0) {
@@ -314,6 +313,20 @@ __global__ void __launch_bounds__(Gemm2Shape<BN, STAGES, gemm2_epi_warps<EPI>()>
   cluster_sync();  // the pair's MMAs are drained before either CTA frees TMEM
   tc_fence_after();
   if (warp == 1) tmem_dealloc_pair(tmem_base, S::TMEM_COLS);
+}
+
+// bf16 and f16 operands (kind::f16), CTA pairs.
+template <int BN, int STAGES, int EPI>
+__global__ void __launch_bounds__(Gemm2Shape<BN, STAGES, gemm2_epi_warps<EPI>()>::THREADS, 1)
+    gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                         const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
+  gemm_tc2_body<BN, STAGES, EPI, KIND_BF16>(tmA, tmB, tmOut, p);
+}
+template <int BN, int STAGES, int EPI>
+__global__ void __launch_bounds__(Gemm2Shape<BN, STAGES, gemm2_epi_warps<EPI>()>::THREADS, 1)
+    gemm_f16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
+  gemm_tc2_body<BN, STAGES, EPI, KIND_F16>(tmA, tmB, tmOut, p);
 }
 
 }  // namespace asr

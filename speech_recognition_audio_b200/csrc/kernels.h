@@ -68,7 +68,7 @@ cudaError_t launch_log_mel(const float* pcm, long long n_samples, int batch, int
 cudaError_t launch_mel_normalize(const float* raw, const unsigned int* clip_max, long long per_clip, int batch,
                                  float* out, cudaStream_t st);
 cudaError_t launch_mel_normalize_transpose(const float* raw, const unsigned int* clip_max, int batch, int n_mels,
-                                           int n_frames, void* out, bool f32, cudaStream_t st);
+                                           int n_frames, void* out, int kind, cudaStream_t st);
 
 // Variable-length batches.  One conv chunk: its clip, its first frame within
 // the clip, its valid frames (chunk_frames except for a clip's last chunk)
@@ -97,7 +97,7 @@ cudaError_t launch_varlen_fill(const VarClipBatch& vb, int chunk_frames, int win
                                ChunkDesc* cd, int* cu, int last, int n_win, int n_tokens, cudaStream_t st);
 cudaError_t launch_conv1_im2col_varlen(const float* mel_raw, const unsigned int* clip_max, int n_chunks, int n_mels,
                                        int chunk_frames, int phase, const ChunkDesc* cd, const MelClip* mc, void* a,
-                                       bool f32, cudaStream_t st);
+                                       int kind, cudaStream_t st);
 cudaError_t launch_mask_short_chunks(void* act, const ChunkDesc* cd, int n_chunks, int chunk_frames, int level, int T,
                                      int F, int C, int phase, int es, cudaStream_t st);
 cudaError_t launch_compact_tokens(const float* xpad, float* x, const ChunkDesc* cd, int n_chunks, int t3, int d,
@@ -108,22 +108,24 @@ cudaError_t launch_compact_tokens(const float* xpad, float* x, const ChunkDesc* 
 // taps (kh * 3 + kw) as bf16 in a row of 16 (taps 9..15 zero).  Rows
 // [chunks][T1][F1], or with phase != 0 (T1, F1 even) the parity planes
 // [chunks][t % 2][f % 2][T1 / 2][F1 / 2] read by the phase-mode conv2.
+// a: rows of the kind's element type (bf16, f16, or fp32 for KIND_TF32).
 cudaError_t launch_conv1_im2col(const float* mel_raw, const unsigned int* clip_max, int batch, int n_mels,
-                                int n_frames, int chunk_frames, int phase, void* a, bool f32, cudaStream_t st);
+                                int n_frames, int chunk_frames, int phase, void* a, int kind, cudaStream_t st);
 
+// y: bf16 (out_kind KIND_BF16), fp32 (KIND_TF32) or f16 (KIND_F16).
 cudaError_t launch_layer_norm(const float* x, const float* g, const float* b, long long M, int D, float eps,
-                              void* y, bool out_f32, cudaStream_t st);
+                              void* y, int out_kind, cudaStream_t st);
 
 // tcgen05 attention for segments of at most 128 tokens (attn_tc.cu).
 bool make_tmap_qkv(CUtensorMap* map, const void* qkv, long long T, int H);
-cudaError_t launch_attention_tc(const CUtensorMap& tm_qkv, const bf16* qkv, const int* cu, int n_seg, int H, bf16* out,
-                                int* status, unsigned long long limit_ns, cudaStream_t st);
+cudaError_t launch_attention_tc(const CUtensorMap& tm_qkv, const void* qkv, const int* cu, int n_seg, int H, void* out,
+                                int* status, unsigned long long limit_ns, bool f16, cudaStream_t st);
 // fp32 attention on the CUDA cores (attn_f32.cu): the fp32-weight path.
 cudaError_t launch_attention_f32(const float* qkv, const int* cu, int n_seg, int max_seg, int H, float* out,
                                  cudaStream_t st);
 // tcgen05 flash attention for segments of any length (attn_fa.cu).
-cudaError_t launch_attention_fa(const CUtensorMap& tm_qkv, const int* cu, int n_seg, int max_seg, int H, bf16* out,
-                                int* status, unsigned long long limit_ns, cudaStream_t st);
+cudaError_t launch_attention_fa(const CUtensorMap& tm_qkv, const int* cu, int n_seg, int max_seg, int H, void* out,
+                                int* status, unsigned long long limit_ns, bool f16, cudaStream_t st);
 
 // Audio-embedding splice (splice.cu).  Element types match ASR_DTYPE_*.
 enum : int { SPLICE_BF16 = 0, SPLICE_F32 = 1, SPLICE_F16 = 2 };
@@ -134,7 +136,8 @@ cudaError_t launch_splice(const int* ids, long long n_ids, int placeholder, cons
 
 cudaError_t launch_fill_windows(int* cu, int batch, int tokens_per_clip, int window, int n_win_per_clip,
                                 cudaStream_t st);
-cudaError_t launch_bf16_to_f32(const bf16* in, float* out, long long n, cudaStream_t st);
+// 16-bit (bf16, or f16 with f16 != 0) to fp32.
+cudaError_t launch_bf16_to_f32(const void* in, float* out, long long n, bool f16, cudaStream_t st);
 cudaError_t launch_gelu(const float* x, float* y, long long n, cudaStream_t st);
 cudaError_t launch_wait_probe(unsigned long long limit_ns, int* status, cudaStream_t st);
 

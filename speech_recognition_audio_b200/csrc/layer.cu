@@ -26,7 +26,7 @@ __device__ __forceinline__ float4 ldg_f4_nomerge(const float4* p) {
   return v;
 }
 
-template <int V, bool OUT_F32>
+template <int V, int OUT>
 __global__ void __launch_bounds__(256, 6) layer_norm_kernel(const float* __restrict__ x, const float* __restrict__ g,
                                                             const float* __restrict__ b, long long M, float eps,
                                                             void* __restrict__ y) {
@@ -82,27 +82,24 @@ __global__ void __launch_bounds__(256, 6) layer_norm_kernel(const float* __restr
       const float o1 = (v[u].y - mean) * rstd * gg.y + bv.y;
       const float o2 = (v[u].z - mean) * rstd * gg.z + bv.z;
       const float o3 = (v[u].w - mean) * rstd * gg.w + bv.w;
-      if (OUT_F32) {
+      if (OUT == KIND_TF32) {
         reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + row * D)[c4] = make_float4(o0, o1, o2, o3);
       } else {
-        __nv_bfloat162 p0 = __floats2bfloat162_rn(o0, o1), p1 = __floats2bfloat162_rn(o2, o3);
-        uint2 w2;
-        w2.x = *reinterpret_cast<uint32_t*>(&p0);
-        w2.y = *reinterpret_cast<uint32_t*>(&p1);
+        const uint2 w2 = make_uint2(pack2_16<OUT>(o0, o1), pack2_16<OUT>(o2, o3));
         reinterpret_cast<uint2*>(reinterpret_cast<bf16*>(y) + row * D)[c4] = w2;
       }
     }
   }
 }
 
-template <bool F32>
+template <int OUT>
 static cudaError_t ln_dispatch(int V, const float* x, const float* g, const float* b, long long M, float eps, void* y,
                                cudaStream_t st) {
   const unsigned blocks = static_cast<unsigned>((M + 7) / 8);
   switch (V) {
 #define ASR_LN_CASE(n) \
   case n: {                                                                                  \
-    cudaError_t e_ = launch_pdl(layer_norm_kernel<n, F32>, dim3(blocks), dim3(256), 0, st, x, g, b, M, eps, y); \
+    cudaError_t e_ = launch_pdl(layer_norm_kernel<n, OUT>, dim3(blocks), dim3(256), 0, st, x, g, b, M, eps, y); \
     if (e_ != cudaSuccess) return e_;                                                        \
     break;                                                                                   \
   }
@@ -116,9 +113,13 @@ static cudaError_t ln_dispatch(int V, const float* x, const float* g, const floa
 }
 
 cudaError_t launch_layer_norm(const float* x, const float* g, const float* b, long long M, int D, float eps, void* y,
-                              bool out_f32, cudaStream_t st) {
+                              int out_kind, cudaStream_t st) {
   if (D % 128 || D > 2048 || M <= 0) return cudaErrorInvalidValue;
-  return out_f32 ? ln_dispatch<true>(D / 128, x, g, b, M, eps, y, st) : ln_dispatch<false>(D / 128, x, g, b, M, eps, y, st);
+  switch (out_kind) {
+    case KIND_TF32: return ln_dispatch<KIND_TF32>(D / 128, x, g, b, M, eps, y, st);
+    case KIND_F16: return ln_dispatch<KIND_F16>(D / 128, x, g, b, M, eps, y, st);
+    default: return ln_dispatch<KIND_BF16>(D / 128, x, g, b, M, eps, y, st);
+  }
 }
 
 // ------------------------------------------------------------ helpers
@@ -179,16 +180,17 @@ cudaError_t launch_varlen_fill(const VarClipBatch& vb, int chunk_frames, int win
                     last, n_win, n_tokens);
 }
 
-__global__ void bf16_to_f32_kernel(const bf16* __restrict__ in, float* __restrict__ out, long long n) {
+__global__ void bf16_to_f32_kernel(const uint16_t* __restrict__ in, float* __restrict__ out, long long n, int f16) {
   pdl_wait();
   pdl_trigger();
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
-    out[i] = __bfloat162float(in[i]);
+    out[i] = f16 ? __half2float(__ushort_as_half(in[i])) : __bfloat162float(__ushort_as_bfloat16(in[i]));
 }
 
-cudaError_t launch_bf16_to_f32(const bf16* in, float* out, long long n, cudaStream_t st) {
+cudaError_t launch_bf16_to_f32(const void* in, float* out, long long n, bool f16, cudaStream_t st) {
   const int blocks = static_cast<int>(std::min<long long>((n + 255) / 256, 148LL * 32));
-  return launch_pdl(bf16_to_f32_kernel, dim3(blocks), dim3(256), 0, st, in, out, n);
+  return launch_pdl(bf16_to_f32_kernel, dim3(blocks), dim3(256), 0, st, static_cast<const uint16_t*>(in), out, n,
+                    f16 ? 1 : 0);
 }
 
 __global__ void gelu_kernel(const float* __restrict__ x, float* __restrict__ y, long long n) {

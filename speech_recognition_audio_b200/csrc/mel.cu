@@ -438,9 +438,9 @@ __global__ void mel_normalize_kernel(const float* __restrict__ raw, const unsign
 
 // Normalise and transpose to time-major bf16 [B, F, n_mels] (input of the
 // Conv1D stem's implicit GEMM).
-template <typename OutT>
+template <int OUTK>
 __global__ void mel_normalize_transpose_kernel(const float* __restrict__ raw, const unsigned int* __restrict__ clip_max,
-                                               int n_mels, int n_frames, OutT* __restrict__ out) {
+                                               int n_mels, int n_frames, void* __restrict__ out) {
   __shared__ float tile[32][33];
   pdl_wait();
   pdl_trigger();
@@ -453,14 +453,18 @@ __global__ void mel_normalize_transpose_kernel(const float* __restrict__ raw, co
     if (m < n_mels && f < n_frames) tile[j][threadIdx.x] = (fmaxf(src[(long long)m * n_frames + f], mx) + 4.0f) * 0.25f;
   }
   __syncthreads();
-  OutT* dst = out + (long long)b * n_frames * n_mels;
+  const long long base = (long long)b * n_frames * n_mels;
   for (int j = threadIdx.y; j < 32; j += blockDim.y) {
     const int f = f0 + j, m = m0 + threadIdx.x;
     if (m < n_mels && f < n_frames) {
-      if constexpr (sizeof(OutT) == 4)
-        dst[(long long)f * n_mels + m] = tile[threadIdx.x][j];
+      const long long i = base + (long long)f * n_mels + m;
+      const float v = tile[threadIdx.x][j];
+      if constexpr (OUTK == KIND_TF32)
+        static_cast<float*>(out)[i] = v;
+      else if constexpr (OUTK == KIND_F16)
+        static_cast<__half*>(out)[i] = __float2half_rn(v);
       else
-        dst[(long long)f * n_mels + m] = __float2bfloat16_rn(tile[threadIdx.x][j]);
+        static_cast<bf16*>(out)[i] = __float2bfloat16_rn(v);
     }
   }
 }
@@ -513,13 +517,19 @@ cudaError_t launch_mel_normalize(const float* raw, const unsigned int* clip_max,
 }
 
 cudaError_t launch_mel_normalize_transpose(const float* raw, const unsigned int* clip_max, int batch, int n_mels,
-                                           int n_frames, void* out, bool f32, cudaStream_t st) {
+                                           int n_frames, void* out, int kind, cudaStream_t st) {
   dim3 grid((n_frames + 31) / 32, (n_mels + 31) / 32, batch);
-  if (f32)
-    return launch_pdl(mel_normalize_transpose_kernel<float>, grid, dim3(32, 8), 0, st, raw, clip_max, n_mels, n_frames,
-                      static_cast<float*>(out));
-  return launch_pdl(mel_normalize_transpose_kernel<bf16>, grid, dim3(32, 8), 0, st, raw, clip_max, n_mels, n_frames,
-                    static_cast<bf16*>(out));
+  switch (kind) {
+    case KIND_TF32:
+      return launch_pdl(mel_normalize_transpose_kernel<KIND_TF32>, grid, dim3(32, 8), 0, st, raw, clip_max, n_mels,
+                        n_frames, out);
+    case KIND_F16:
+      return launch_pdl(mel_normalize_transpose_kernel<KIND_F16>, grid, dim3(32, 8), 0, st, raw, clip_max, n_mels,
+                        n_frames, out);
+    default:
+      return launch_pdl(mel_normalize_transpose_kernel<KIND_BF16>, grid, dim3(32, 8), 0, st, raw, clip_max, n_mels,
+                        n_frames, out);
+  }
 }
 
 }  // namespace asr

@@ -21,13 +21,13 @@
 
 namespace asr {
 
-template <typename OutT>
+template <int OUTK>
 __global__ void __launch_bounds__(256) conv1_im2col_kernel(const float* __restrict__ mel_raw,
                                                            const unsigned int* __restrict__ clip_max, int n_mels,
                                                            int n_frames, int chunk_frames, int chunks_per_clip,
                                                            int T1, int F1, long long rows, int phase,
                                                            const ChunkDesc* __restrict__ cd,
-                                                           const MelClip* __restrict__ mc, OutT* __restrict__ a) {
+                                                           const MelClip* __restrict__ mc, void* __restrict__ a_out) {
   pdl_wait();
   pdl_trigger();
   const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
@@ -76,51 +76,59 @@ __global__ void __launch_bounds__(256) conv1_im2col_kernel(const float* __restri
   for (int k = 9; k < 16; ++k) v[k] = 0.f;
   // output row: [chunk][plane][T][F] (plain: [chunk][T1][F1])
   const long long row = (chunk * (phase ? 4 : 1) + plane) * (long long)TP * FP + (long long)t * FP + f;
-  if constexpr (sizeof(OutT) == 4) {
-    float4* dst = reinterpret_cast<float4*>(a + row * 16);
+  if constexpr (OUTK == KIND_TF32) {
+    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a_out) + row * 16);
 #pragma unroll
     for (int k = 0; k < 4; ++k) dst[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
   } else {
-    alignas(16) __nv_bfloat162 r[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) r[k] = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
-    uint4* dst = reinterpret_cast<uint4*>(a + row * 16);
-    dst[0] = *reinterpret_cast<uint4*>(&r[0]);
-    dst[1] = *reinterpret_cast<uint4*>(&r[4]);
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a_out) + row * 16);
+    dst[0] = pack8_16<OUTK>(v);
+    dst[1] = pack8_16<OUTK>(v + 8);
   }
 }
 
-// a: bf16 rows (f32 == false) or fp32 rows (f32 == true, the fp32-weight path).
+// a: rows of the kind's element type (bf16, f16, or fp32 for KIND_TF32).
+template <int OUTK>
+static cudaError_t im2col_launch(const float* mel_raw, const unsigned int* clip_max, int n_mels, int n_frames,
+                                 int chunk_frames, int chunks_per_clip, int T1, int F1, long long rows, int phase,
+                                 const ChunkDesc* cd, const MelClip* mc, void* a, cudaStream_t st) {
+  const unsigned blocks = static_cast<unsigned>((rows + 255) / 256);
+  return launch_pdl(conv1_im2col_kernel<OUTK>, dim3(blocks), dim3(256), 0, st, mel_raw, clip_max, n_mels, n_frames,
+                    chunk_frames, chunks_per_clip, T1, F1, rows, phase, cd, mc, a);
+}
+
+static cudaError_t im2col_kind(int kind, const float* mel_raw, const unsigned int* clip_max, int n_mels, int n_frames,
+                               int chunk_frames, int chunks_per_clip, int T1, int F1, long long rows, int phase,
+                               const ChunkDesc* cd, const MelClip* mc, void* a, cudaStream_t st) {
+  switch (kind) {
+    case KIND_TF32: return im2col_launch<KIND_TF32>(mel_raw, clip_max, n_mels, n_frames, chunk_frames, chunks_per_clip,
+                                                    T1, F1, rows, phase, cd, mc, a, st);
+    case KIND_F16: return im2col_launch<KIND_F16>(mel_raw, clip_max, n_mels, n_frames, chunk_frames, chunks_per_clip,
+                                                  T1, F1, rows, phase, cd, mc, a, st);
+    default: return im2col_launch<KIND_BF16>(mel_raw, clip_max, n_mels, n_frames, chunk_frames, chunks_per_clip, T1,
+                                             F1, rows, phase, cd, mc, a, st);
+  }
+}
+
 cudaError_t launch_conv1_im2col(const float* mel_raw, const unsigned int* clip_max, int batch, int n_mels,
-                                int n_frames, int chunk_frames, int phase, void* a, bool f32, cudaStream_t st) {
+                                int n_frames, int chunk_frames, int phase, void* a, int kind, cudaStream_t st) {
   const int T1 = (chunk_frames - 1) / 2 + 1, F1 = (n_mels - 1) / 2 + 1;
   if (phase && (T1 % 2 || F1 % 2)) return cudaErrorInvalidValue;
   const int chunks_per_clip = n_frames / chunk_frames;
   const long long rows = (long long)batch * chunks_per_clip * T1 * F1;
   if (rows == 0) return cudaSuccess;
-  const unsigned blocks = static_cast<unsigned>((rows + 255) / 256);
-  if (f32)
-    return launch_pdl(conv1_im2col_kernel<float>, dim3(blocks), dim3(256), 0, st, mel_raw, clip_max, n_mels, n_frames,
-                      chunk_frames, chunks_per_clip, T1, F1, rows, phase ? 1 : 0, (const ChunkDesc*)nullptr,
-                      (const MelClip*)nullptr, static_cast<float*>(a));
-  return launch_pdl(conv1_im2col_kernel<bf16>, dim3(blocks), dim3(256), 0, st, mel_raw, clip_max, n_mels, n_frames,
-                    chunk_frames, chunks_per_clip, T1, F1, rows, phase ? 1 : 0, (const ChunkDesc*)nullptr,
-                    (const MelClip*)nullptr, static_cast<bf16*>(a));
+  return im2col_kind(kind, mel_raw, clip_max, n_mels, n_frames, chunk_frames, chunks_per_clip, T1, F1, rows,
+                     phase ? 1 : 0, nullptr, nullptr, a, st);
 }
 
 cudaError_t launch_conv1_im2col_varlen(const float* mel_raw, const unsigned int* clip_max, int n_chunks, int n_mels,
                                        int chunk_frames, int phase, const ChunkDesc* cd, const MelClip* mc, void* a,
-                                       bool f32, cudaStream_t st) {
+                                       int kind, cudaStream_t st) {
   const int T1 = (chunk_frames - 1) / 2 + 1, F1 = (n_mels - 1) / 2 + 1;
   if (phase && (T1 % 2 || F1 % 2)) return cudaErrorInvalidValue;
   const long long rows = (long long)n_chunks * T1 * F1;
   if (rows == 0) return cudaSuccess;
-  const unsigned blocks = static_cast<unsigned>((rows + 255) / 256);
-  if (f32)
-    return launch_pdl(conv1_im2col_kernel<float>, dim3(blocks), dim3(256), 0, st, mel_raw, clip_max, n_mels, 0,
-                      chunk_frames, 1, T1, F1, rows, phase ? 1 : 0, cd, mc, static_cast<float*>(a));
-  return launch_pdl(conv1_im2col_kernel<bf16>, dim3(blocks), dim3(256), 0, st, mel_raw, clip_max, n_mels, 0,
-                    chunk_frames, 1, T1, F1, rows, phase ? 1 : 0, cd, mc, static_cast<bf16*>(a));
+  return im2col_kind(kind, mel_raw, clip_max, n_mels, 0, chunk_frames, 1, T1, F1, rows, phase ? 1 : 0, cd, mc, a, st);
 }
 
 // ---------------------------------------------------------- short chunks

@@ -43,6 +43,7 @@ POS_GLOBAL = 1
 
 DTYPE_BF16 = 0
 DTYPE_F32 = 1
+DTYPE_F16 = 2
 
 
 @dataclass(frozen=True)
@@ -217,11 +218,11 @@ def make_weights(g: Geometry, seed: int, affine: bool = False, std: float = 0.02
     LayerNorms are identity (gain 1, shift 0).  With ``affine`` the biases are
     N(0, 0.02), LayerNorm gains 1 + N(0, 0.1) and shifts N(0, 0.02), drawn in
     the same stream, so that every bias and LayerNorm path carries signal.
-    Values are rounded once to the geometry's dtype (bf16 or fp32); both the
-    oracle and the CUDA path consume exactly these rounded values.
+    Values are rounded once to the geometry's dtype (bf16, f16 or fp32); both
+    the oracle and the CUDA path consume exactly these rounded values.
     """
     gen = torch.Generator().manual_seed(seed)
-    dt = torch.bfloat16 if g.dtype == DTYPE_BF16 else torch.float32
+    dt = {DTYPE_BF16: torch.bfloat16, DTYPE_F16: torch.float16}.get(g.dtype, torch.float32)
     out = {}
     for name, shape, kind in weight_specs(g):
         if kind == "w":

@@ -97,6 +97,35 @@ def test_whisper_style_fp32_geometry():
     enc.close()
 
 
+def test_tiny_f16_weights():
+    # f16 weights and activations between the GEMMs (kind::f16 with f16 operands).
+    base = synth.GEOMETRIES["tiny"].as_dict()
+    base.update(dtype=synth.DTYPE_F16)
+    g = synth.Geometry(**base)
+    W = synth.make_weights(g, 80, affine=True)
+    assert W["conv1.w"].dtype == torch.float16
+    enc = sra.Encoder(g, {k: v.cuda() for k, v in W.items()})
+    pcm = np.stack([synth.pcm_clip(48000, 530), synth.pcm_clip(48000, 531)])
+    out = _run(enc, pcm)
+    assert_encoder_parity(out, oracle.forward(pcm, W, g), "tiny f16 weights")
+    enc.close()
+
+
+def test_moss_1x30s_f16_weights():
+    # The MOSS tower with the F16 weights the pages' GGUF builds keep for the
+    # encoder and adapter; 10 s keep the float64 oracle short.
+    base = synth.GEOMETRIES["moss"].as_dict()
+    base.update(dtype=synth.DTYPE_F16)
+    g = synth.Geometry(**base)
+    W = synth.make_weights(g, 1241)
+    enc = sra.Encoder(g, {k: v.cuda() for k, v in W.items()})
+    pcm = synth.pcm_clip(160000, 540)[None]
+    out = _run(enc, pcm)
+    assert out.shape == (1, 130, 2048)
+    assert_encoder_parity(out, oracle.forward(pcm, W, g), "moss 1x10s f16 weights")
+    enc.close()
+
+
 def test_affine_biases_small_batch():
     # Non-zero biases and LayerNorm affine parameters exercise every epilogue's
     # bias path and the LN gain/shift; 2 clips x 3 s, windows of 104 > 39 tokens.
