@@ -286,6 +286,27 @@ def run_kernel(args, w, g):
         pcm = torch.from_numpy(synth.pcm_batch(w)).to(dev)
         run = lambda: sra.log_mel(pcm, g.n_mels)
         flops, unit = 4 * pcm.numel() + 4 * w.batch * g.n_mels * (w.n_samples // g.hop), "bytes"
+    elif args.kernel == "layer_norm":
+        x = (torch.randn(T, d, generator=gen) * 3).to(dev)
+        gam, bet = torch.ones(d, device=dev), torch.zeros(d, device=dev)
+        run = lambda: sra.layer_norm(x, gam, bet)
+        flops, unit = T * d * (4 + 2), "bytes"
+    elif args.kernel == "attention":
+        import ctypes
+        qkv = (torch.randn(T, 3 * d, generator=gen)).to(torch.bfloat16).to(dev)
+        cu_h = sra.windows(g, w.n_samples, w.batch)
+        cu = torch.tensor(cu_h, dtype=torch.int32, device=dev)
+        att = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+        aws = torch.zeros(256, dtype=torch.uint8, device=dev)
+        mx = max(b - a for a, b in zip(cu_h[:-1], cu_h[1:]))
+        st = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+        run = lambda: sra.lib.asr_op_attention(ctypes.c_void_p(qkv.data_ptr()), ctypes.c_void_p(cu.data_ptr()),
+                                               len(cu_h) - 1, mx, T, g.n_heads, ctypes.c_void_p(att.data_ptr()),
+                                               ctypes.c_void_p(aws.data_ptr()), 256, st)
+        wt = g.window_tokens if g.window_tokens else T // w.batch
+        tc = T // w.batch
+        flops = sum(4 * min(wt, tc - a) ** 2 * d for a in range(0, tc, wt)) * w.batch
+        unit = "flop"
     else:
         N, K, epi = {"gemm_fc1": (f, d, sra.EPI_BF16_GELU), "gemm_fc2": (d, f, sra.EPI_F32_RESID),
                      "gemm_qkv": (3 * d, d, sra.EPI_BF16), "gemm_o": (d, d, sra.EPI_F32_RESID)}[args.kernel]
@@ -320,7 +341,8 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-steps", type=int, default=3)
-    ap.add_argument("--kernel", default=None, choices=["gemm_fc1", "gemm_fc2", "gemm_qkv", "gemm_o", "log_mel"],
+    ap.add_argument("--kernel", default=None, choices=["gemm_fc1", "gemm_fc2", "gemm_qkv", "gemm_o", "log_mel", "layer_norm",
+                                                       "attention"],
                     help="run one op of the workload's shape through the C ABI (for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -464,6 +464,15 @@ asr_status asr_enc_create(const asr_geometry* g, const void* const* weights, int
   size_t need = 0;
   auto acc = [&](size_t bytes) { need = align_up(need, 1024) + bytes; };
   for (auto& w : specs) acc((size_t)numel(w) * 4);  // generous: every tensor at 4 bytes/element
+  // conv kernels are repacked with their input channels padded to a whole
+  // 128-byte row per tap (up to 63 extra channels), at up to 4 bytes each
+  if (g->stem == ASR_STEM_CONV2D_CHUNKED) {
+    acc((size_t)C * 9 * 64 * 4);
+    acc((size_t)C * 9 * 64 * 4);
+  } else {
+    acc((size_t)d * 3 * 64 * 4);
+    acc((size_t)d * 3 * 64 * 4);
+  }
   const int pe_rows = g->stem == ASR_STEM_CONV2D_CHUNKED
                           ? (int)conv_len(conv_len(conv_len(g->chunk_frames, 3, 2, 1), 3, 2, 1), 3, 2, 1)
                           : 1500;

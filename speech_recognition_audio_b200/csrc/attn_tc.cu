@@ -10,14 +10,12 @@
 //   - V comes by TMA too (keys x dims) and serves as the MN-major B operand
 //     of P V (rows past the segment meet zero probabilities);
 //   - S = Q K^T: tcgen05.mma M=128 N=128 K=64 into tensor memory;
-//   - each thread owns one query row: a first pass over its scores in
-//     tensor memory finds the maximum over keys < L, a second pass takes
-//     exp2((s - max) / 8 log2 e) over the 16-key chunks below L and the sum;
+//   - each thread owns one query row: tcgen05.ld of its 128 scores, scale
+//     1/8, mask keys >= L, max, exp2 (over the 16-key chunks below L), sum;
 //     P (bf16, or f16 for f16 operands) is written row-major, swizzled, over
 //     the Q and K tiles as the A operand of the next MMA;
 //   - O = P V: tcgen05.mma M=128 N=64 K=128 into S's tensor-memory columns;
-//   48 KB of shared memory, 128 TMEM columns and <= 128 registers a thread
-//   per block: 4 blocks per SM.
+//   48 KB of shared memory and 128 TMEM columns per block: 4 blocks per SM.
 //   - each thread scales its output row by 1 / sum and stores 128 bytes.
 // Every barrier wait is bounded (status word); tensor memory is freed after
 // all MMAs have completed.
@@ -34,7 +32,7 @@ constexpr int AT_TMEM_COLS = 128;           // S (128 columns), then O (64) in t
 }  // namespace
 
 template <int KIND>
-__global__ void __launch_bounds__(AT_THREADS, 4) attention_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv,
+__global__ void __launch_bounds__(AT_THREADS) attention_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv,
                                                                    const bf16* __restrict__ qkv,
                                                                    const int* __restrict__ cu, int H,
                                                                    bf16* __restrict__ out, int* status,
@@ -87,57 +85,53 @@ __global__ void __launch_bounds__(AT_THREADS, 4) attention_tc_kernel(const __gri
     }
     tc_commit(bar_s);
   }
-  // softmax of this thread's row, in two passes over tensor memory (16 keys
-  // at a time, so a thread holds 16 scores, not 128: four blocks fit an SM)
+  // softmax of this thread's row
   float rsum = 1.f;
   {
     const bool got = mbar_wait_bounded(bar_s, 0, limit_ns, status, DEV_TIMEOUT_EPILOGUE);
     tc_fence_after();
     const int row = warp * 32 + lane;
     const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    float sv[128];
+#pragma unroll
+    for (int c = 0; c < 128; c += 16) tmem_ld16(taddr + c, sv + c);
+    tmem_ld_wait();
     const float sl2 = 0.125f * 1.4426950408889634f;
-    // pass 1: the row maximum over the segment's keys (uniform branches: L is the block's)
     float mx = -INFINITY;
 #pragma unroll
-    for (int c = 0; c < 128; c += 16) {
-      if (c < L) {
-        float v[16];
-        tmem_ld16(taddr + c, v);
-        tmem_ld_wait();
+    for (int j = 0; j < 128; ++j) {
+      sv[j] = (j < L && got) ? sv[j] * sl2 : -INFINITY;
+      mx = fmaxf(mx, sv[j]);
+    }
+    if (mx == -INFINITY) mx = 0.f;  // only when the wait failed
+    float s = 0.f;
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          if (c + j < L) mx = fmaxf(mx, v[j]);
+    for (int c = 0; c < 128; c += 16) {
+      if (c < L) {  // uniform: 16-key chunks wholly past the segment stay zero
+#pragma unroll
+        for (int j = c; j < c + 16; ++j) {
+          sv[j] = exp2f(sv[j] - mx);
+          s += sv[j];
+        }
+      } else {
+#pragma unroll
+        for (int j = c; j < c + 16; ++j) sv[j] = 0.f;
       }
     }
-    mx = got ? mx * sl2 : 0.f;  // the scale is positive: max(s) * scale = max(s * scale)
+    rsum = s > 0.f ? 1.f / s : 0.f;
     // P overwrites Q and K: every thread has passed bar_s, so the MMA that
     // read them is complete.
     __syncthreads();
     fence_proxy_async_smem();
-    // pass 2: exponentials, the sum, and P in two 64-key blocks, 16-byte
-    // chunks swizzled by (row & 7); keys past the segment are zero
-    float s = 0.f;
+    // P row into two 64-key blocks, 16-byte chunks swizzled by (row & 7)
 #pragma unroll
-    for (int c = 0; c < 128; c += 16) {
-      float v[16];
-      if (c < L && got) {
-        tmem_ld16(taddr + c, v);
-        tmem_ld_wait();
+    for (int kb = 0; kb < 2; ++kb) {
+      uint4* prow = reinterpret_cast<uint4*>(sm + SP + kb * 16384 + row * 128);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          v[j] = (c + j < L) ? exp2f(fmaf(v[j], sl2, -mx)) : 0.f;
-          s += v[j];
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = 0.f;
+      for (int c = 0; c < 8; ++c) {
+        prow[c ^ (row & 7)] = pack8_16<KIND>(sv + kb * 64 + c * 8);
       }
-      uint4* prow = reinterpret_cast<uint4*>(sm + SP + (c / 64) * 16384 + row * 128);
-      const int cc = (c % 64) / 8;
-      prow[cc ^ (row & 7)] = pack8_16<KIND>(v);
-      prow[(cc + 1) ^ (row & 7)] = pack8_16<KIND>(v + 8);
     }
-    rsum = s > 0.f ? 1.f / s : 0.f;
   }
   fence_proxy_async_smem();
   tc_fence_before();

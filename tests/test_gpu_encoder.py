@@ -191,11 +191,17 @@ def test_host_forward_matches_device_forward():
 
 
 def test_forward_rejects_bad_sizes():
+    import ctypes
     enc, W, g = _encoder("tiny_1x1s")
-    pcm = torch.zeros((1, 16000 + 160), device="cuda")
+    pcm = torch.zeros((1, 200), device="cuda")    # reflect padding needs more than n_fft/2 samples
     with pytest.raises(sra.AsrError) as ei:
         enc.forward(pcm)
     assert ei.value.code == 2
+    out = torch.empty((1, 1, g.adapter_out), device="cuda")
+    ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
+    rc = sra.lib.asr_enc_forward(enc.handle, ctypes.c_void_p(pcm.data_ptr()), 200, 1, ctypes.c_void_p(out.data_ptr()),
+                                 None, ctypes.c_void_p(ws.data_ptr()), ws.numel(), None)
+    assert rc == 1
     pcm = torch.zeros((1, 16000), device="cuda")
     small = torch.empty(1024, dtype=torch.uint8, device="cuda")
     with pytest.raises(sra.AsrError) as ei:
