@@ -180,13 +180,22 @@ __global__ void __launch_bounds__(FA_THREADS, 2) attention_fa_kernel(const __gri
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar[B_SFREE]);
         const int kv = min(128, L - j * 128);  // valid keys in this tile (>= 1)
-        float mt = -INFINITY;
+        // tile maximum of the raw scores (four chains; only a partial last
+        // tile needs the per-key mask); the scale is positive, so
+        // max(s) * scale = max(s * scale)
+        float m8[4];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          sv[c] = (c < kv && ok) ? sv[c] * sl2 : -INFINITY;
-          mt = fmaxf(mt, sv[c]);
+        for (int i = 0; i < 4; ++i) m8[i] = -INFINITY;
+        if (kv == 128) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c) m8[c & 3] = fmaxf(m8[c & 3], sv[c]);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c < kv) m8[c & 3] = fmaxf(m8[c & 3], sv[c]);
         }
-        if (mt == -INFINITY) mt = 0.f;  // only after a failed wait
+        float mt = fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3]));
+        mt = ok ? mt * sl2 : 0.f;
         // P_j may overwrite P_{j-1} and O may be rescaled once O_{j-1} is complete
         if (j > 0) ok = mbar_wait_bounded(&bar[B_OD], (j - 1) & 1, limit_ns, status, DEV_TIMEOUT_EPILOGUE) && ok;
         tc_fence_after();
@@ -194,7 +203,7 @@ __global__ void __launch_bounds__(FA_THREADS, 2) attention_fa_kernel(const __gri
         if (j == 0) {
           m_used = mt;
         } else if (__any_sync(0xffffffffu, grow)) {
-          const float corr = grow ? exp2f(m_used - mt) : 1.0f;
+          const float corr = grow ? ex2_approx(m_used - mt) : 1.0f;
           if (grow) {
             m_used = mt;
             lsum *= corr;
@@ -210,21 +219,25 @@ __global__ void __launch_bounds__(FA_THREADS, 2) attention_fa_kernel(const __gri
           }
           tmem_st_wait();
         }
-        float s = 0.f;
+        // p = 2^((s - m) / 8 log2 e) as one FMA into ex2.approx
+        const float nm = -m_used;
+        float s8[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) s8[i] = 0.f;
 #pragma unroll
         for (int c = 0; c < 128; c += 16) {
-          if (c < kv) {  // uniform: 16-key chunks wholly past the segment stay zero
+          if (c < kv && ok) {  // uniform: 16-key chunks wholly past the segment stay zero
 #pragma unroll
             for (int i = c; i < c + 16; ++i) {
-              sv[i] = exp2f(sv[i] - m_used);
-              s += sv[i];
+              sv[i] = (i < kv) ? ex2_approx(fmaf(sv[i], sl2, nm)) : 0.f;
+              s8[i & 3] += sv[i];
             }
           } else {
 #pragma unroll
             for (int i = c; i < c + 16; ++i) sv[i] = 0.f;
           }
         }
-        lsum += s;
+        lsum += (s8[0] + s8[1]) + (s8[2] + s8[3]);
         // P row into two 64-key halves, 16-byte chunks swizzled by (row & 7)
 #pragma unroll
         for (int kb = 0; kb < 2; ++kb) {

@@ -10,8 +10,10 @@
 //   - V comes by TMA too (keys x dims) and serves as the MN-major B operand
 //     of P V (rows past the segment meet zero probabilities);
 //   - S = Q K^T: tcgen05.mma M=128 N=128 K=64 into tensor memory;
-//   - each thread owns one query row: tcgen05.ld of its 128 scores, scale
-//     1/8, mask keys >= L, max, exp2 (over the 16-key chunks below L), sum;
+//   - each thread owns one query row: tcgen05.ld of its 128 scores, the
+//     maximum over keys < L, then exp2 of (s - max) / 8 log2 e as one FMA
+//     into ex2.approx (over the 16-key chunks below L) and the sum, both
+//     in four independent chains;
 //     P (bf16, or f16 for f16 operands) is written row-major, swizzled, over
 //     the Q and K tiles as the A operand of the next MMA;
 //   - O = P V: tcgen05.mma M=128 N=64 K=128 into S's tensor-memory columns;
@@ -32,7 +34,7 @@ constexpr int AT_TMEM_COLS = 128;           // S (128 columns), then O (64) in t
 }  // namespace
 
 template <int KIND>
-__global__ void __launch_bounds__(AT_THREADS) attention_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv,
+__global__ void __launch_bounds__(AT_THREADS, 3) attention_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv,
                                                                    const bf16* __restrict__ qkv,
                                                                    const int* __restrict__ cu, int H,
                                                                    bf16* __restrict__ out, int* status,
@@ -97,27 +99,43 @@ __global__ void __launch_bounds__(AT_THREADS) attention_tc_kernel(const __grid_c
     for (int c = 0; c < 128; c += 16) tmem_ld16(taddr + c, sv + c);
     tmem_ld_wait();
     const float sl2 = 0.125f * 1.4426950408889634f;
-    float mx = -INFINITY;
+    // row maximum over keys < L (four independent chains; only the 16-key
+    // chunk that holds L needs a per-key mask)
+    float m8[4];
 #pragma unroll
-    for (int j = 0; j < 128; ++j) {
-      sv[j] = (j < L && got) ? sv[j] * sl2 : -INFINITY;
-      mx = fmaxf(mx, sv[j]);
-    }
-    if (mx == -INFINITY) mx = 0.f;  // only when the wait failed
-    float s = 0.f;
+    for (int i = 0; i < 4; ++i) m8[i] = -INFINITY;
 #pragma unroll
     for (int c = 0; c < 128; c += 16) {
-      if (c < L) {  // uniform: 16-key chunks wholly past the segment stay zero
+      if (c + 16 <= L) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) m8[j & 3] = fmaxf(m8[j & 3], sv[c + j]);
+      } else if (c < L) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (c + j < L) m8[j & 3] = fmaxf(m8[j & 3], sv[c + j]);
+      }
+    }
+    float mx = fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3]));
+    // exp2((s - max) / 8 log2 e) as one FMA into ex2; the scale is positive,
+    // so max(s) * scale = max(s * scale)
+    const float nm = got ? -mx * sl2 : 0.f;
+    float s8[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) s8[i] = 0.f;
+#pragma unroll
+    for (int c = 0; c < 128; c += 16) {
+      if (c < L && got) {  // uniform: 16-key chunks wholly past the segment stay zero
 #pragma unroll
         for (int j = c; j < c + 16; ++j) {
-          sv[j] = exp2f(sv[j] - mx);
-          s += sv[j];
+          sv[j] = (j < L) ? ex2_approx(fmaf(sv[j], sl2, nm)) : 0.f;
+          s8[j & 3] += sv[j];
         }
       } else {
 #pragma unroll
         for (int j = c; j < c + 16; ++j) sv[j] = 0.f;
       }
     }
+    const float s = (s8[0] + s8[1]) + (s8[2] + s8[3]);
     rsum = s > 0.f ? 1.f / s : 0.f;
     // P overwrites Q and K: every thread has passed bar_s, so the MMA that
     // read them is complete.

@@ -289,6 +289,13 @@ __device__ __forceinline__ float tanh_approx(float x) {
   asm("tanh.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
   return r;
 }
+// 2^x from the hardware ex2.approx.ftz.f32 (relative error ~2^-22; inputs
+// below the normal range give 0, -inf gives 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
 namespace gelu_tanh {
 constexpr float k0 = 0.7978845608028654f;               // sqrt(2 / pi)
 constexpr float k1 = 0.7978845608028654f * 0.044715f;   // sqrt(2 / pi) * 0.044715

@@ -314,6 +314,8 @@ __device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, const 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Shared-memory sources of this thread's bulk stores may be overwritten.
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// All but the most recent of this thread's bulk stores have read their source.
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 // This thread's bulk stores have completed (written to global memory).
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
@@ -351,10 +353,15 @@ __device__ __forceinline__ void load_bias(const GemmParams& p, int n0, int BN, i
 //   Stream-K pieces (residual epilogue only): PIECE_PARTIAL adds its raw
 //     accumulator (no bias) to the residual stream; the caller orders the
 //     owner's update after it.
-template <int EPI, int KIND = KIND_BF16>
+//   Staging: NBUF buffers of BUFB bytes per warp, used in turn (gcount
+//     counts the warp's groups across tiles), so with two a group's smem
+//     writes overlap the previous group's store and two stores per warp are
+//     in flight.
+template <int EPI, int KIND = KIND_BF16, int NBUF = 1, int BUFB = 4096>
 __device__ __forceinline__ void epilogue_warp(const GemmParams& p, const CUtensorMap* tm_out, uint32_t tb, int row0,
-                                              int mlimit, int n0, int BN, int half, int lane, uint8_t* wbuf,
-                                              const float* breg, int kind = PIECE_FULL, int cstride = 64) {
+                                              int mlimit, int n0, int BN, int half, int lane, uint8_t* wbase,
+                                              const float* breg, int kind = PIECE_FULL, int cstride = 64,
+                                              int* gcount = nullptr) {
   constexpr bool F32 = (EPI & (EPI_OUT_F32 | EPI_RESID)) != 0;
   constexpr bool SWI = (EPI & EPI_SWIGLU) != 0;  // with F32: fp32 outputs, stored per row
   constexpr bool TMA_OK = (EPI & (EPI_PE | EPI_SWIGLU)) == 0;
@@ -391,8 +398,19 @@ __device__ __forceinline__ void epilogue_warp(const GemmParams& p, const CUtenso
       }
       continue;
     }
-    // The buffer may still be the source of the previous group's bulk store.
-    if (lane == 0) bulk_wait_read0();
+    // This group's buffer, which may still be the source of the bulk store
+    // issued from it NBUF groups ago.
+    uint8_t* wbuf = wbase;
+    if (NBUF == 2) {
+      wbuf += (*gcount & 1) * BUFB;
+      ++*gcount;
+    }
+    if (lane == 0) {
+      if (NBUF == 2)
+        bulk_wait_read1();
+      else
+        bulk_wait_read0();
+    }
     __syncwarp();
     if (SWI) {
       // gate = columns c..c+15, up = c+16..c+31 -> 16 bf16 outputs (2 chunks).

@@ -91,7 +91,8 @@ __device__ __forceinline__ void tc_commit_pair_mc(uint64_t* bar, uint16_t mask) 
 }
 
 // EPIW_: epilogue warps, 8 or 16 (16 only for bf16 outputs, whose 32 x 32
-// staging box takes 2 KB, so the staging area stays 32 KB).
+// staging box takes 2 KB); each warp stages its groups in two buffers, so
+// the staging area is 64 KB.
 template <int BN_, int STAGES_, int EPIW_ = 8>
 struct Gemm2Shape {
   static constexpr int BM = 256, BN = BN_, BK = 64, STAGES = STAGES_;
@@ -103,7 +104,9 @@ struct Gemm2Shape {
   static constexpr int TMEM_COLS = 2 * ACC_COLS <= 64 ? 64 : 2 * ACC_COLS <= 128 ? 128 : 2 * ACC_COLS <= 256 ? 256 : 512;
   static constexpr int EPI_WARPS = EPIW_;
   static constexpr int THREADS = 32 * (2 + EPI_WARPS);
-  static constexpr int WBUF = EPI_WARPS == 16 ? 2048 : 4096;  // staging bytes per epilogue warp
+  static constexpr int BOXB = EPI_WARPS == 16 ? 2048 : 4096;  // one 32 x 32 output box (bf16 / fp32)
+  static constexpr int NBUF = 2;                              // staging buffers per epilogue warp
+  static constexpr int WBUF = NBUF * BOXB;                    // staging bytes per epilogue warp
   static constexpr int CSTRIDE = 32 * (EPI_WARPS / 4);       // column stride of a warp's groups
   static constexpr int EPI_BUF_BYTES = EPI_WARPS * WBUF;
   static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5) + 16;
@@ -261,7 +264,7 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap& tmA, const CUte
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
     const int rank_rows = static_cast<int>(rank) * 128;
     const int ew = warp - 2;
-    int tl = 0;
+    int tl = 0, groups = 0;
     PieceIter pi(p, pair, n_pairs);
     int t, kb0, kb1;
     for (; pi.next(p, t, kb0, kb1); ++tl) {
@@ -293,8 +296,8 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap& tmA, const CUte
         have = __shfl_sync(0xffffffffu, have, 0);
       }
       if (have)
-        epilogue_warp<EPI, KIND>(p, &tmOut, tb, r_first + 32 * q, r_last, n0, BN, half, lane, sEpi + ew * S::WBUF, breg,
-                                 kind, S::CSTRIDE);
+        epilogue_warp<EPI, KIND, S::NBUF, S::BOXB>(p, &tmOut, tb, r_first + 32 * q, r_last, n0, BN, half, lane,
+                                                   sEpi + ew * S::WBUF, breg, kind, S::CSTRIDE, &groups);
       tc_fence_before();
       __syncwarp();
       if (kind == PIECE_PARTIAL && lane == 0) {

@@ -8,55 +8,38 @@
 namespace asr {
 
 // ------------------------------------------------------------ LayerNorm
-// One warp per row, V float4 per lane (D = 128 V).  The statistics take one
-// pass over the row in shifted form: with K = x[row][0],
+// One warp per row, V float4 per lane (D = 128 V), the whole row held in
+// registers: every load of the row is issued at once (one memory round trip
+// per row), then the statistics, then the normalised row is written from the
+// registers.  The statistics take one pass in shifted form: with
+// K = x[row][0],
 //   mean = K + S1 / D,  var = S2 / D - (S1 / D)^2,
 //   S1 = sum (x - K),   S2 = sum (x - K)^2,
 // which keeps the cancellation at the scale of the row's spread (|x - K|
-// is a few standard deviations), not of its mean.  The second pass re-reads
-// the row (L1 / L2 hits) to normalise and store, so no thread holds a whole
-// row and every row of a 6240 x 1280 residual stream is in flight at once
-// (one wave of warps instead of two).
-
-// Read-only 16-byte load that the compiler may not merge with another load
-// of the same address (the second pass must re-read, not keep the row).
-__device__ __forceinline__ float4 ldg_f4_nomerge(const float4* p) {
-  float4 v;
-  asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(p));
-  return v;
-}
+// is a few standard deviations), not of its mean.  Four rows per 128-thread
+// block.
 
 template <int V, int OUT>
-__global__ void __launch_bounds__(256, 6) layer_norm_kernel(const float* __restrict__ x, const float* __restrict__ g,
-                                                            const float* __restrict__ b, long long M, float eps,
-                                                            void* __restrict__ y) {
+__global__ void __launch_bounds__(128) layer_norm_kernel(const float* __restrict__ x, const float* __restrict__ g,
+                                                         const float* __restrict__ b, long long M, float eps,
+                                                         void* __restrict__ y) {
   pdl_wait();
   pdl_trigger();
-  const long long row = blockIdx.x * 8LL + (threadIdx.x >> 5);
+  const long long row = blockIdx.x * 4LL + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= M) return;
   constexpr int D = V * 128;
-  // 16-byte loads in flight per lane: the statistics pass keeps up to 5 in
-  // flight (the row arrives in two round trips), the normalising pass 2
-  // (its re-reads hit L1, and it also holds gamma and beta).
-  constexpr int U1 = V % 5 == 0 ? 5 : (V % 4 == 0 ? 4 : (V % 3 == 0 ? 3 : (V % 2 == 0 ? 2 : 1)));
-  constexpr int U = V % 2 == 0 ? 2 : 1;
-  // (at most 6 blocks of 256 threads per SM fit 42 registers per thread:
-  // 48 row-warps per SM, 7104 rows in flight on 148 SMs)
   const float4* xr = reinterpret_cast<const float4*>(x + row * D);
-  const float K = __ldg(x + row * D);
+  float4 v[V];
+#pragma unroll
+  for (int i = 0; i < V; ++i) v[i] = __ldg(xr + lane + 32 * i);
+  const float K = __shfl_sync(0xffffffffu, v[0].x, 0);  // x[row][0]
   float s1 = 0.f, s2 = 0.f;
-#pragma unroll 1
-  for (int i0 = 0; i0 < V; i0 += U1) {
-    float4 v[U1];
 #pragma unroll
-    for (int u = 0; u < U1; ++u) v[u] = ldg_f4_nomerge(xr + lane + 32 * (i0 + u));
-#pragma unroll
-    for (int u = 0; u < U1; ++u) {
-      const float a = v[u].x - K, bb = v[u].y - K, c = v[u].z - K, d = v[u].w - K;
-      s1 += (a + bb) + (c + d);
-      s2 += (a * a + bb * bb) + (c * c + d * d);
-    }
+  for (int i = 0; i < V; ++i) {
+    const float a = v[i].x - K, bb = v[i].y - K, c = v[i].z - K, d = v[i].w - K;
+    s1 += (a + bb) + (c + d);
+    s2 += (a * a + bb * bb) + (c * c + d * d);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -69,25 +52,19 @@ __global__ void __launch_bounds__(256, 6) layer_norm_kernel(const float* __restr
   const float rstd = rsqrtf(var + eps);
   const float4* g4 = reinterpret_cast<const float4*>(g);
   const float4* b4 = reinterpret_cast<const float4*>(b);
-#pragma unroll 1
-  for (int i0 = 0; i0 < V; i0 += U) {
-    float4 v[U];
 #pragma unroll
-    for (int u = 0; u < U; ++u) v[u] = ldg_f4_nomerge(xr + lane + 32 * (i0 + u));
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int c4 = lane + 32 * (i0 + u);
-      const float4 gg = __ldg(g4 + c4), bv = __ldg(b4 + c4);
-      const float o0 = (v[u].x - mean) * rstd * gg.x + bv.x;
-      const float o1 = (v[u].y - mean) * rstd * gg.y + bv.y;
-      const float o2 = (v[u].z - mean) * rstd * gg.z + bv.z;
-      const float o3 = (v[u].w - mean) * rstd * gg.w + bv.w;
-      if (OUT == KIND_TF32) {
-        reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + row * D)[c4] = make_float4(o0, o1, o2, o3);
-      } else {
-        const uint2 w2 = make_uint2(pack2_16<OUT>(o0, o1), pack2_16<OUT>(o2, o3));
-        reinterpret_cast<uint2*>(reinterpret_cast<bf16*>(y) + row * D)[c4] = w2;
-      }
+  for (int i = 0; i < V; ++i) {
+    const int c4 = lane + 32 * i;
+    const float4 gg = __ldg(g4 + c4), bv = __ldg(b4 + c4);
+    const float o0 = (v[i].x - mean) * rstd * gg.x + bv.x;
+    const float o1 = (v[i].y - mean) * rstd * gg.y + bv.y;
+    const float o2 = (v[i].z - mean) * rstd * gg.z + bv.z;
+    const float o3 = (v[i].w - mean) * rstd * gg.w + bv.w;
+    if (OUT == KIND_TF32) {
+      reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + row * D)[c4] = make_float4(o0, o1, o2, o3);
+    } else {
+      const uint2 w2 = make_uint2(pack2_16<OUT>(o0, o1), pack2_16<OUT>(o2, o3));
+      reinterpret_cast<uint2*>(reinterpret_cast<bf16*>(y) + row * D)[c4] = w2;
     }
   }
 }
@@ -95,11 +72,11 @@ __global__ void __launch_bounds__(256, 6) layer_norm_kernel(const float* __restr
 template <int OUT>
 static cudaError_t ln_dispatch(int V, const float* x, const float* g, const float* b, long long M, float eps, void* y,
                                cudaStream_t st) {
-  const unsigned blocks = static_cast<unsigned>((M + 7) / 8);
+  const unsigned blocks = static_cast<unsigned>((M + 3) / 4);
   switch (V) {
 #define ASR_LN_CASE(n) \
   case n: {                                                                                  \
-    cudaError_t e_ = launch_pdl(layer_norm_kernel<n, OUT>, dim3(blocks), dim3(256), 0, st, x, g, b, M, eps, y); \
+    cudaError_t e_ = launch_pdl(layer_norm_kernel<n, OUT>, dim3(blocks), dim3(128), 0, st, x, g, b, M, eps, y); \
     if (e_ != cudaSuccess) return e_;                                                        \
     break;                                                                                   \
   }
