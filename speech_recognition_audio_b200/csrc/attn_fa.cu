@@ -4,39 +4,46 @@
 // encoder frames per 30 s window), and any segment longer than the 128
 // tokens the one-tile kernel of attn_tc.cu takes.
 //
-// One CTA per (128-query tile, segment, head), 6 warps:
-//   warp 4  TMA producer: Q once, then K_j and V_j (128 keys x 64 dims, one
-//           buffer each) as soon as the previous tile's MMA has read them;
-//   warp 5  MMA issuer: S = Q K_j^T (M=128, N=128, K=64) into tensor memory,
-//           issued for tile j+1 while the softmax of tile j runs, then
+// One CTA per (128-query tile, segment, head), 10 warps:
+//   warp 8  TMA producer: Q once, then K_j (two buffers, so K_{j+1} arrives
+//           while tile j is in flight) and V_j (one buffer, loaded once the
+//           previous tile's P V has read it);
+//   warp 9  MMA issuer: S = Q K_j^T (M=128, N=128, K=64) into tensor memory,
+//           issued for tile j+1 as soon as the softmax has read S_j, then
 //           O += P_j V_j (M=128, N=64, K=128) with O kept in tensor memory;
-//   warps 0-3  softmax, one query row per thread: load the row of S, mask
-//           keys past the segment, online softmax in base 2 with the scale
-//           1/sqrt(64) folded in.  The running maximum used for the
-//           exponentials moves only when a tile's maximum exceeds it by
-//           more than 8 (then O and the row sum are rescaled by
-//           2^(old - new)), so probabilities stay <= 256 and most tiles need
-//           no rescale.  P (bf16 or f16, the operands' type) goes to shared
-//           memory as the A operand of the next MMA; at the end each thread
-//           divides its O row by its sum and stores it.
+//   warps 0-7  softmax: warps w and w+4 share the 32 query rows of TMEM lane
+//           quarter w % 4 and take keys [64 h, 64 h + 64) of every tile and
+//           O columns [32 h, 32 h + 32), h = w / 4; the two halves of a row
+//           exchange their maxima and, at the end, their sums through shared
+//           memory at a named barrier of the warp pair.  Online softmax in
+//           base 2 with the scale 1/sqrt(64) folded into one FMA into
+//           ex2.approx; the running maximum used for the exponentials moves
+//           only when a tile's maximum exceeds it by more than 8 (then O and
+//           the row sums are rescaled by 2^(old - new)), so probabilities
+//           stay <= 256 and most tiles need no rescale.  P (bf16 or f16, the
+//           operands' type) goes to shared memory as the A operand of the
+//           next MMA; at the end each thread divides its 32 O columns by the
+//           row sum and stores them.
 // Tensor memory: S in columns 0..127, O in 128..191 (256 allocated: two
-// CTAs per SM).  Shared memory: Q, K, V (16 KB each), P (32 KB).  Every wait
-// is bounded; tensor memory is freed after all MMAs have completed.
+// CTAs per SM).  Shared memory: Q (16 KB), K (2 x 16 KB), V (16 KB), P
+// (32 KB).  Every wait is bounded; tensor memory is freed after all MMAs
+// have completed.
 #include "kernels.h"
 
 namespace asr {
 
 namespace {
-constexpr int FA_THREADS = 192;
-constexpr int FA_SQ = 0, FA_SK = 16384, FA_SV = 32768, FA_SP = 49152;  // P: two 64-key halves of 16 KB
-constexpr int FA_TILES = 81920;
-constexpr int FA_BARS = FA_TILES;                                    // 10 barriers + TMEM slot
-constexpr int FA_SMEM = 1024 + FA_TILES + 128;
+constexpr int FA_THREADS = 320;
+constexpr int FA_SQ = 0, FA_SK = 16384, FA_SV = 49152, FA_SP = 65536;  // K: two buffers; P: two 64-key halves
+constexpr int FA_TILES = 98304;
+constexpr int FA_RED = FA_TILES;                 // float [2 tiles][2 halves][128 rows] row maxima, then sums
+constexpr int FA_BARS = FA_RED + 2 * 2 * 128 * 4;
+constexpr int FA_SMEM = 1024 + FA_BARS + 256;
 constexpr int FA_TMEM_COLS = 256;
 constexpr int FA_O_COL = 128;
 constexpr float FA_RESCALE_LOG2 = 8.0f;
 
-enum { B_Q = 0, B_KF, B_KE, B_VF, B_VE, B_SF, B_SFREE, B_PF, B_OD, B_DRAIN, B_COUNT };
+enum { B_Q = 0, B_KF0, B_KF1, B_KE0, B_KE1, B_VF, B_VE, B_SF, B_SFREE, B_PF, B_OD, B_DRAIN, B_COUNT };
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
   asm volatile(
@@ -49,6 +56,8 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
       : "memory");
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// Named barrier of the two softmax warps of one TMEM lane quarter (ids 1-4).
+__device__ __forceinline__ void pair_sync(int q) { asm volatile("bar.sync %0, 64;" ::"r"(1 + q) : "memory"); }
 }  // namespace
 
 template <int KIND>
@@ -58,22 +67,14 @@ __global__ void __launch_bounds__(FA_THREADS, 2) attention_fa_kernel(const __gri
                                                                      unsigned long long limit_ns) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* red = reinterpret_cast<float*>(sm + FA_RED);
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + FA_BARS);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + B_COUNT);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qt = blockIdx.x, seg = blockIdx.y, h = blockIdx.z;
 
   if (tid == 0) {
-    mbar_init(&bar[B_Q], 1);
-    mbar_init(&bar[B_KF], 1);
-    mbar_init(&bar[B_KE], 1);
-    mbar_init(&bar[B_VF], 1);
-    mbar_init(&bar[B_VE], 1);
-    mbar_init(&bar[B_SF], 1);
-    mbar_init(&bar[B_SFREE], 4);
-    mbar_init(&bar[B_PF], 4);
-    mbar_init(&bar[B_OD], 1);
-    mbar_init(&bar[B_DRAIN], 1);
+    for (int i = 0; i < B_COUNT; ++i) mbar_init(&bar[i], (i == B_SFREE || i == B_PF) ? 8 : 1);
     fence_mbar_init();
     tma_prefetch_desc(&tm_qkv);
   }
@@ -92,7 +93,7 @@ __global__ void __launch_bounds__(FA_THREADS, 2) attention_fa_kernel(const __gri
   const int q0 = qt * 128;
   const int nk = (L + 127) / 128;
   if (q0 < L) {
-    if (warp == 4) {
+    if (warp == 8) {
       // ------------------------------------------------ TMA producer
       if (lane == 0) {
         bool ok = true;
@@ -100,10 +101,15 @@ __global__ void __launch_bounds__(FA_THREADS, 2) attention_fa_kernel(const __gri
         mbar_arrive_expect_tx(&bar[B_Q], 16384);
         tma_load_2d(sm + FA_SQ, &tm_qkv, &bar[B_Q], h * 64, s0 + q0);
         for (int j = 0; j < nk && ok; ++j) {
-          if (j > 0 && !(ok = mbar_wait_bounded(&bar[B_KE], (j - 1) & 1, limit_ns, status, DEV_TIMEOUT_PRODUCER))) break;
-          mbar_arrive_expect_tx(&bar[B_KF], 16384);
-          tma_load_2d(sm + FA_SK, &tm_qkv, &bar[B_KF], (H + h) * 64, s0 + j * 128);
+          const int kb = j & 1;
+          // K_j into buffer j % 2 once S_{j-2} has read it
+          if (j >= 2 && !(ok = mbar_wait_bounded(&bar[B_KE0 + kb], ((j >> 1) - 1) & 1, limit_ns, status,
+                                                 DEV_TIMEOUT_PRODUCER)))
+            break;
+          mbar_arrive_expect_tx(&bar[B_KF0 + kb], 16384);
+          tma_load_2d(sm + FA_SK + kb * 16384, &tm_qkv, &bar[B_KF0 + kb], (H + h) * 64, s0 + j * 128);
           ++issued_k;
+          // V_j once P_{j-1} V_{j-1} has read V_{j-1}
           if (j > 0 && !(ok = mbar_wait_bounded(&bar[B_VE], (j - 1) & 1, limit_ns, status, DEV_TIMEOUT_PRODUCER))) break;
           mbar_arrive_expect_tx(&bar[B_VF], 16384);
           tma_load_2d(sm + FA_SV, &tm_qkv, &bar[B_VF], (2 * H + h) * 64, s0 + j * 128);
@@ -111,37 +117,35 @@ __global__ void __launch_bounds__(FA_THREADS, 2) attention_fa_kernel(const __gri
         }
         // every issued load lands before the CTA exits
         mbar_wait_bounded(&bar[B_Q], 0, kDrainLimitNs, nullptr, 0);
-        if (issued_k) mbar_wait_bounded(&bar[B_KF], (issued_k - 1) & 1, kDrainLimitNs, nullptr, 0);
+        for (int j = issued_k - 2 < 0 ? 0 : issued_k - 2; j < issued_k; ++j)
+          mbar_wait_bounded(&bar[B_KF0 + (j & 1)], (j >> 1) & 1, kDrainLimitNs, nullptr, 0);
         if (issued_v) mbar_wait_bounded(&bar[B_VF], (issued_v - 1) & 1, kDrainLimitNs, nullptr, 0);
       }
-    } else if (warp == 5) {
+    } else if (warp == 9) {
       // ------------------------------------------------ MMA issuer
       if (lane == 0) {
         const uint32_t idesc_s = idesc_kind_f32(KIND, 128, 128);
         const uint32_t idesc_o = idesc_kind_f32(KIND, 128, 64) | (1u << 16);  // B = V, MN-major
         const uint64_t qd = sw128_kmajor_desc(smem_u32(sm + FA_SQ));
-        const uint64_t kd = sw128_kmajor_desc(smem_u32(sm + FA_SK));
         const uint64_t vd = sw128_mnmajor_desc(smem_u32(sm + FA_SV));
-        bool ok = mbar_wait_bounded(&bar[B_Q], 0, limit_ns, status, DEV_TIMEOUT_MMA) &&
-                  mbar_wait_bounded(&bar[B_KF], 0, limit_ns, status, DEV_TIMEOUT_MMA);
-        if (ok) {
+        auto issue_s = [&](int j) {
+          const uint64_t kd = sw128_kmajor_desc(smem_u32(sm + FA_SK + (j & 1) * 16384));
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < 4; ++k) tc_mma_bf16(tmem, qd + 2 * k, kd + 2 * k, idesc_s, k > 0 ? 1u : 0u);
           tc_commit(&bar[B_SF]);
-          tc_commit(&bar[B_KE]);
-        }
+          tc_commit(&bar[B_KE0 + (j & 1)]);
+        };
+        bool ok = mbar_wait_bounded(&bar[B_Q], 0, limit_ns, status, DEV_TIMEOUT_MMA) &&
+                  mbar_wait_bounded(&bar[B_KF0], 0, limit_ns, status, DEV_TIMEOUT_MMA);
+        if (ok) issue_s(0);
         for (int j = 0; j < nk && ok; ++j) {
           if (j + 1 < nk) {
             // S for the next tile once its K has landed and the softmax has read S_j
-            ok = mbar_wait_bounded(&bar[B_KF], (j + 1) & 1, limit_ns, status, DEV_TIMEOUT_MMA) &&
+            ok = mbar_wait_bounded(&bar[B_KF0 + ((j + 1) & 1)], ((j + 1) >> 1) & 1, limit_ns, status, DEV_TIMEOUT_MMA) &&
                  mbar_wait_bounded(&bar[B_SFREE], j & 1, limit_ns, status, DEV_TIMEOUT_MMA);
             if (!ok) break;
-            tc_fence_after();
-#pragma unroll
-            for (int k = 0; k < 4; ++k) tc_mma_bf16(tmem, qd + 2 * k, kd + 2 * k, idesc_s, k > 0 ? 1u : 0u);
-            tc_commit(&bar[B_SF]);
-            tc_commit(&bar[B_KE]);
+            issue_s(j + 1);
           }
           ok = mbar_wait_bounded(&bar[B_PF], j & 1, limit_ns, status, DEV_TIMEOUT_MMA) &&
                mbar_wait_bounded(&bar[B_VF], j & 1, limit_ns, status, DEV_TIMEOUT_MMA);
@@ -163,108 +167,107 @@ __global__ void __launch_bounds__(FA_THREADS, 2) attention_fa_kernel(const __gri
         mbar_wait_bounded(&bar[B_DRAIN], 0, kDrainLimitNs, nullptr, 0);
       }
     } else {
-      // ------------------------------------------------ softmax (warps 0-3)
-      const int row = warp * 32 + lane;
-      const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+      // ------------------------------------------------ softmax (warps 0-7)
+      const int q = warp & 3, hh = warp >> 2;            // lane quarter, key / O-column half
+      const int row = q * 32 + lane;
+      const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
       const float sl2 = 0.125f * 1.4426950408889634f;  // (1 / sqrt(64)) log2(e)
       float m_used = -INFINITY, lsum = 0.f;
       bool ok = true;
+      // Every tile runs through both pair barriers even after a failed wait
+      // (ok stays false and later waits are skipped), so the two warps of a
+      // pair always meet the same number of barriers.
       for (int j = 0; j < nk; ++j) {
-        ok = mbar_wait_bounded(&bar[B_SF], j & 1, limit_ns, status, DEV_TIMEOUT_EPILOGUE);
+        ok = __all_sync(0xffffffffu, ok && mbar_wait_bounded(&bar[B_SF], j & 1, limit_ns, status, DEV_TIMEOUT_EPILOGUE));
         tc_fence_after();
-        float sv[128];
+        float sv[64];
 #pragma unroll
-        for (int c = 0; c < 128; c += 16) tmem_ld16(trow + c, sv + c);
+        for (int c = 0; c < 64; c += 16) tmem_ld16(trow + hh * 64 + c, sv + c);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar[B_SFREE]);
-        const int kv = min(128, L - j * 128);  // valid keys in this tile (>= 1)
-        // tile maximum of the raw scores (four chains; only a partial last
-        // tile needs the per-key mask); the scale is positive, so
-        // max(s) * scale = max(s * scale)
-        float m8[4];
+        const int kv = min(128, L - j * 128) - hh * 64;  // valid keys of this half (may be <= 0)
+        // half-row maximum of the raw scores (four chains; only a partial
+        // half needs the per-key mask)
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        if (kv >= 64) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) m8[i] = -INFINITY;
-        if (kv == 128) {
-#pragma unroll
-          for (int c = 0; c < 128; ++c) m8[c & 3] = fmaxf(m8[c & 3], sv[c]);
+          for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], sv[c]);
         } else {
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (c < kv) m8[c & 3] = fmaxf(m8[c & 3], sv[c]);
+          for (int c = 0; c < 64; ++c)
+            if (c < kv) m4[c & 3] = fmaxf(m4[c & 3], sv[c]);
         }
-        float mt = fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3]));
+        float* rbuf = red + (j & 1) * 256;
+        rbuf[hh * 128 + row] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        pair_sync(q);
+        // the scale is positive: max(s) * scale = max(s * scale)
+        float mt = fmaxf(rbuf[row], rbuf[128 + row]);
         mt = ok ? mt * sl2 : 0.f;
-        // P_j may overwrite P_{j-1} and O may be rescaled once O_{j-1} is complete
-        if (j > 0) ok = mbar_wait_bounded(&bar[B_OD], (j - 1) & 1, limit_ns, status, DEV_TIMEOUT_EPILOGUE) && ok;
-        tc_fence_after();
-        const bool grow = mt > m_used + FA_RESCALE_LOG2;
-        if (j == 0) {
-          m_used = mt;
-        } else if (__any_sync(0xffffffffu, grow)) {
-          const float corr = grow ? ex2_approx(m_used - mt) : 1.0f;
-          if (grow) {
-            m_used = mt;
-            lsum *= corr;
-          }
-#pragma unroll
-          for (int c = 0; c < 64; c += 16) {
-            float ov[16];
-            tmem_ld16(trow + FA_O_COL + c, ov);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) ov[i] *= corr;
-            tmem_st16(trow + FA_O_COL + c, ov);
-          }
-          tmem_st_wait();
-        }
-        // p = 2^((s - m) / 8 log2 e) as one FMA into ex2.approx
+        const bool grow = j > 0 && mt > m_used + FA_RESCALE_LOG2;
+        const float corr = grow ? ex2_approx(m_used - mt) : 1.0f;
+        if (j == 0 || grow) m_used = mt;
+        // p = 2^((s - m) / 8 log2 e) as one FMA into ex2.approx, while the
+        // previous tile's P V may still run
         const float nm = -m_used;
-        float s8[4];
+        float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) s8[i] = 0.f;
-#pragma unroll
-        for (int c = 0; c < 128; c += 16) {
+        for (int c = 0; c < 64; c += 16) {
           if (c < kv && ok) {  // uniform: 16-key chunks wholly past the segment stay zero
 #pragma unroll
             for (int i = c; i < c + 16; ++i) {
               sv[i] = (i < kv) ? ex2_approx(fmaf(sv[i], sl2, nm)) : 0.f;
-              s8[i & 3] += sv[i];
+              s4[i & 3] += sv[i];
             }
           } else {
 #pragma unroll
             for (int i = c; i < c + 16; ++i) sv[i] = 0.f;
           }
         }
-        lsum += (s8[0] + s8[1]) + (s8[2] + s8[3]);
-        // P row into two 64-key halves, 16-byte chunks swizzled by (row & 7)
+        lsum = lsum * corr + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+        // P_j may overwrite P_{j-1} and O may be rescaled once O_{j-1} is complete
+        if (j > 0) ok = __all_sync(0xffffffffu, ok && mbar_wait_bounded(&bar[B_OD], (j - 1) & 1, limit_ns, status,
+                                                                        DEV_TIMEOUT_EPILOGUE));
+        tc_fence_after();
+        // this half's 64 keys of the P row: one 128-byte row of P block hh,
+        // 16-byte chunks swizzled by (row & 7)
+        uint4* prow = reinterpret_cast<uint4*>(sm + FA_SP + hh * 16384 + row * 128);
 #pragma unroll
-        for (int kb = 0; kb < 2; ++kb) {
-          uint4* prow = reinterpret_cast<uint4*>(sm + FA_SP + kb * 16384 + row * 128);
+        for (int c = 0; c < 8; ++c) prow[c ^ (row & 7)] = pack8_16<KIND>(sv + c * 8);
+        if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            prow[c ^ (row & 7)] = pack8_16<KIND>(sv + kb * 64 + c * 8);
+          for (int c = 0; c < 32; c += 16) {
+            float ov[16];
+            tmem_ld16(trow + FA_O_COL + hh * 32 + c, ov);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) ov[i] *= corr;
+            tmem_st16(trow + FA_O_COL + hh * 32 + c, ov);
           }
+          tmem_st_wait();
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar[B_PF]);
-        if (!ok) break;
       }
-      // epilogue: O / sum
+      // epilogue: the row sum from both halves, then this half's O columns / sum
       const bool got = ok && mbar_wait_bounded(&bar[B_OD], (nk - 1) & 1, limit_ns, status, DEV_TIMEOUT_EPILOGUE);
       tc_fence_after();
-      float ov[64];
+      float* sbuf = red + (nk & 1) * 256;  // the buffer the last tile did not use
+      sbuf[hh * 128 + row] = lsum;
+      pair_sync(q);
+      const float tot = sbuf[row] + sbuf[128 + row];
+      float ov[32];
 #pragma unroll
-      for (int c = 0; c < 64; c += 16) tmem_ld16(trow + FA_O_COL + c, ov + c);
+      for (int c = 0; c < 32; c += 16) tmem_ld16(trow + FA_O_COL + hh * 32 + c, ov + c);
       tmem_ld_wait();
-      const float inv = (got && lsum > 0.f) ? 1.0f / lsum : 0.f;
+      const float inv = (got && tot > 0.f) ? 1.0f / tot : 0.f;
       if (q0 + row < L) {
-        uint4* dst = reinterpret_cast<uint4*>(out + (long long)(s0 + q0 + row) * (H * 64) + h * 64);
+        uint4* dst = reinterpret_cast<uint4*>(out + (long long)(s0 + q0 + row) * (H * 64) + h * 64 + hh * 32);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < 4; ++c) {
           float t8[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) t8[i] = ov[8 * c + i] * inv;

@@ -108,7 +108,7 @@ cudaError_t run_gather(int epi, const CUtensorMap& b, const CUtensorMap& o, cons
 
 template <int BN, int EPI, int KIND>
 cudaError_t run2(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& p, int grid, cudaStream_t st) {
-  using S = Gemm2Shape<BN, (BN >= 192 ? 5 : 6), gemm2_epi_warps<EPI>()>;
+  using S = Gemm2Shape<BN, 6, gemm2_epi_warps<EPI>(), gemm2_nbuf<BN>()>;
   void (*k)(CUtensorMap, CUtensorMap, CUtensorMap, GemmParams);
   if constexpr (KIND == KIND_F16)
     k = gemm_f16_tc2_kernel<BN, S::STAGES, EPI>;
@@ -169,8 +169,8 @@ int resident_pairs(int num_sms) {
   cudaGetDevice(&dev);
   std::lock_guard<std::mutex> lock(mu);
   if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
-  using S = Gemm2Shape<256, 5>;
-  auto k = gemm_bf16_tc2_kernel<256, 5, EPI_RESID>;
+  using S = Gemm2Shape<256, 6, gemm2_epi_warps<EPI_RESID>(), gemm2_nbuf<256>()>;
+  auto k = gemm_bf16_tc2_kernel<256, 6, EPI_RESID>;
   int n = 0;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_BYTES) == cudaSuccess) {
     cudaLaunchConfig_t cfg = {};

@@ -91,9 +91,10 @@ __device__ __forceinline__ void tc_commit_pair_mc(uint64_t* bar, uint16_t mask) 
 }
 
 // EPIW_: epilogue warps, 8 or 16 (16 only for bf16 outputs, whose 32 x 32
-// staging box takes 2 KB); each warp stages its groups in two buffers, so
-// the staging area is 64 KB.
-template <int BN_, int STAGES_, int EPIW_ = 8>
+// staging box takes 2 KB); NBUF_: staging buffers per epilogue warp, used in
+// turn (two let a warp fill the next box while the previous TMA store still
+// reads its buffer).  The staging area is 32 KB per buffer.
+template <int BN_, int STAGES_, int EPIW_ = 8, int NBUF_ = 1>
 struct Gemm2Shape {
   static constexpr int BM = 256, BN = BN_, BK = 64, STAGES = STAGES_;
   static constexpr int A_BYTES = 128 * BK * 2;        // this CTA's half of A
@@ -105,7 +106,7 @@ struct Gemm2Shape {
   static constexpr int EPI_WARPS = EPIW_;
   static constexpr int THREADS = 32 * (2 + EPI_WARPS);
   static constexpr int BOXB = EPI_WARPS == 16 ? 2048 : 4096;  // one 32 x 32 output box (bf16 / fp32)
-  static constexpr int NBUF = 2;                              // staging buffers per epilogue warp
+  static constexpr int NBUF = NBUF_;                          // staging buffers per epilogue warp
   static constexpr int WBUF = NBUF * BOXB;                    // staging bytes per epilogue warp
   static constexpr int CSTRIDE = 32 * (EPI_WARPS / 4);       // column stride of a warp's groups
   static constexpr int EPI_BUF_BYTES = EPI_WARPS * WBUF;
@@ -115,6 +116,15 @@ struct Gemm2Shape {
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
   static_assert(EPI_WARPS == 8 || EPI_WARPS == 16, "two or four column parts per lane quarter");
 };
+
+// Staging buffers per epilogue warp: tiles of 192 columns and more keep six
+// 32 KB pipeline stages with one buffer (measured: a second buffer at the
+// cost of a stage made the residual GEMMs 2-6 % slower and the others no
+// faster); narrower tiles have room for both.
+template <int BN>
+constexpr int gemm2_nbuf() {
+  return BN >= 192 ? 1 : 2;
+}
 
 // Epilogue warps of an instance: 16 for the bias + GELU bf16 epilogue (the
 // GELU's arithmetic is the epilogue's cost; with 8 warps it is latency-bound,
@@ -127,7 +137,7 @@ constexpr int gemm2_epi_warps() {
 template <int BN, int STAGES, int EPI, int KIND>
 __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmOut,
                                               const GemmParams& p) {
-  using S = Gemm2Shape<BN, STAGES, gemm2_epi_warps<EPI>()>;
+  using S = Gemm2Shape<BN, STAGES, gemm2_epi_warps<EPI>(), gemm2_nbuf<BN>()>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -320,13 +330,13 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap& tmA, const CUte
 
 // bf16 and f16 operands (kind::f16), CTA pairs.
 template <int BN, int STAGES, int EPI>
-__global__ void __launch_bounds__(Gemm2Shape<BN, STAGES, gemm2_epi_warps<EPI>()>::THREADS, 1)
+__global__ void __launch_bounds__(Gemm2Shape<BN, STAGES, gemm2_epi_warps<EPI>(), gemm2_nbuf<BN>()>::THREADS, 1)
     gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
   gemm_tc2_body<BN, STAGES, EPI, KIND_BF16>(tmA, tmB, tmOut, p);
 }
 template <int BN, int STAGES, int EPI>
-__global__ void __launch_bounds__(Gemm2Shape<BN, STAGES, gemm2_epi_warps<EPI>()>::THREADS, 1)
+__global__ void __launch_bounds__(Gemm2Shape<BN, STAGES, gemm2_epi_warps<EPI>(), gemm2_nbuf<BN>()>::THREADS, 1)
     gemm_f16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
   gemm_tc2_body<BN, STAGES, EPI, KIND_F16>(tmA, tmB, tmOut, p);
