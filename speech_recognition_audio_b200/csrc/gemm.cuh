@@ -94,6 +94,12 @@ struct GemmParams {
   // element sees the same additions in the same order on every run.
   int sk;
   int* sk_flags;          // [pairs][2 CTAs][8 warps], zero before the launch
+  int k_full;             // 1 = every k-block holds four whole MMA steps (set by the launcher)
+};
+
+template <bool B>
+struct BoolTag {
+  static constexpr bool value = B;
 };
 
 // Kinds of work piece: a whole tile, the trailing k-blocks of a split tile
@@ -627,33 +633,50 @@ __device__ __forceinline__ void gemm_tc_body(const CUtensorMap& tmA, const CUten
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + a * S::ACC_COLS;
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1;
-          if (!mbar_wait_bounded(&full[s], ph, p.limit_ns, p.status, DEV_TIMEOUT_MMA)) {
-            ok = false;
-            break;
-          }
-          // cp.async wrote the A tile through the generic proxy; order those
-          // writes (observed through the barrier) before the MMA's reads.
-          if (GATHER) fence_proxy_async_smem();
-          tc_fence_after();
-          const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + s * S::A_BYTES));
-          const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + s * S::B_BYTES));
-          const int ks = k16_steps(p, kb, S::BK);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            if (k < ks) {
-              // each step: 32 bytes of K (16 bf16 or 8 tf32 elements)
-              if (KIND == KIND_TF32)
-                tc_mma_tf32(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
-              else
-                tc_mma_bf16(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+        // The k-loop in two versions: every k-block whole (four MMA steps
+        // issued as one sequence, no per-block test: a test in the loop
+        // measured about 8 % of the MMA rate), or with partial k-blocks.
+        auto kloop = [&](auto full_tag) {
+          constexpr bool FULL = decltype(full_tag)::value;
+          for (int kb = 0; kb < p.k_blocks; ++kb) {
+            const int s = it % STAGES;
+            const uint32_t ph = (it / STAGES) & 1;
+            if (!mbar_wait_bounded(&full[s], ph, p.limit_ns, p.status, DEV_TIMEOUT_MMA)) {
+              ok = false;
+              break;
             }
+            // cp.async wrote the A tile through the generic proxy; order those
+            // writes (observed through the barrier) before the MMA's reads.
+            if (GATHER) fence_proxy_async_smem();
+            tc_fence_after();
+            const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + s * S::A_BYTES));
+            const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + s * S::B_BYTES));
+            // each step: 32 bytes of K (16 bf16 or 8 tf32 elements)
+            if (FULL) {
+              if (KIND == KIND_TF32)
+                tc_mma4_tf32(d_tmem, ad, bd, idesc, kb > 0 ? 1u : 0u);
+              else
+                tc_mma4_bf16(d_tmem, ad, bd, idesc, kb > 0 ? 1u : 0u);
+            } else {
+              const int ks = k16_steps(p, kb, S::BK);
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                if (k < ks) {
+                  if (KIND == KIND_TF32)
+                    tc_mma_tf32(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                  else
+                    tc_mma_bf16(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                }
+              }
+            }
+            tc_commit(&empty[s]);
+            ++it;
           }
-          tc_commit(&empty[s]);
-          ++it;
-        }
+        };
+        if (p.k_full)
+          kloop(BoolTag<true>{});
+        else
+          kloop(BoolTag<false>{});
         if (!ok) break;
         tc_commit(&tfull[a]);
       }

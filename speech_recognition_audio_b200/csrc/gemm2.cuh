@@ -80,6 +80,20 @@ __device__ __forceinline__ void tc_mma_bf16_pair(uint32_t d_tmem, uint64_t adesc
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// The four K = 16 steps of a 64-element k-block as one sequence (see
+// tc_mma4_bf16), CTA-pair form.
+__device__ __forceinline__ void tc_mma4_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                  uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %5, %6, %3, 1;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %7, %8, %3, 1;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %9, %10, %3, 1;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "l"(adesc + 2), "l"(bdesc + 2), "l"(adesc + 4),
+      "l"(bdesc + 4), "l"(adesc + 6), "l"(bdesc + 6)
+      : "memory");
+}
 // Arrive (once each) on the barrier at the same offset in every CTA of `mask`
 // when the pair's previously issued MMAs complete.
 __device__ __forceinline__ void tc_commit_pair_mc(uint64_t* bar, uint16_t mask) {
@@ -244,23 +258,36 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap& tmA, const CUte
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + a * S::ACC_COLS;
-        for (int kb = kb0; kb < kb1; ++kb) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1;
-          if (!mbar_wait_bounded(&full[s], ph, p.limit_ns, p.status, DEV_TIMEOUT_MMA)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + s * S::A_BYTES));
-          const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + s * S::B_BYTES));
-          const int ks = k16_steps(p, kb);
+        // Two versions of the k-loop (see the one-SM kernel): whole k-blocks
+        // only, or with partial ones.
+        auto kloop = [&](auto full_tag) {
+          constexpr bool FULL = decltype(full_tag)::value;
+          for (int kb = kb0; kb < kb1; ++kb) {
+            const int s = it % STAGES;
+            const uint32_t ph = (it / STAGES) & 1;
+            if (!mbar_wait_bounded(&full[s], ph, p.limit_ns, p.status, DEV_TIMEOUT_MMA)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + s * S::A_BYTES));
+            const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + s * S::B_BYTES));
+            if (FULL) {
+              tc_mma4_bf16_pair(d_tmem, ad, bd, idesc, kb > kb0 ? 1u : 0u);
+            } else {
+              const int ks = k16_steps(p, kb);
 #pragma unroll
-          for (int k = 0; k < S::BK / 16; ++k)
-            if (k < ks) tc_mma_bf16_pair(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
-          tc_commit_pair_mc(&empty[s], 0x3);
-          ++it;
-        }
+              for (int k = 0; k < S::BK / 16; ++k)
+                if (k < ks) tc_mma_bf16_pair(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+            }
+            tc_commit_pair_mc(&empty[s], 0x3);
+            ++it;
+          }
+        };
+        if (p.k_full)
+          kloop(BoolTag<true>{});
+        else
+          kloop(BoolTag<false>{});
         if (!ok) break;
         tc_commit_pair_mc(&tfull[a], 0x3);
       }
