@@ -211,21 +211,35 @@ __global__ void __launch_bounds__(FA_THREADS, 2) attention_fa_kernel(const __gri
         // p = 2^((s - m) / 8 log2 e) as one FMA into ex2.approx, while the
         // previous tile's P V may still run
         const float nm = -m_used;
-        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+        // whole 16-key chunks as packed pair FMAs and packed sums; per-key
+        // masks only in the chunk that holds the segment's end; chunks past
+        // it stay zero (uniform tests)
+        const float2 sl2v = make_float2(sl2, sl2), nmv = make_float2(nm, nm);
+        float2 s2[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) s2[i] = make_float2(0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < 64; c += 16) {
-          if (c < kv && ok) {  // uniform: 16-key chunks wholly past the segment stay zero
+          if (c + 16 <= kv && ok) {
+#pragma unroll
+            for (int i = c; i < c + 16; i += 2) {
+              const float2 a = fma2(make_float2(sv[i], sv[i + 1]), sl2v, nmv);
+              sv[i] = ex2_approx(a.x);
+              sv[i + 1] = ex2_approx(a.y);
+              s2[(i >> 1) & 3] = add2(s2[(i >> 1) & 3], make_float2(sv[i], sv[i + 1]));
+            }
+          } else if (c < kv && ok) {
 #pragma unroll
             for (int i = c; i < c + 16; ++i) {
               sv[i] = (i < kv) ? ex2_approx(fmaf(sv[i], sl2, nm)) : 0.f;
-              s4[i & 3] += sv[i];
+              s2[(i >> 1) & 3].x += sv[i];
             }
           } else {
 #pragma unroll
             for (int i = c; i < c + 16; ++i) sv[i] = 0.f;
           }
         }
-        lsum = lsum * corr + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+        lsum = lsum * corr + (((s2[0].x + s2[0].y) + (s2[1].x + s2[1].y)) + ((s2[2].x + s2[2].y) + (s2[3].x + s2[3].y)));
         // P_j may overwrite P_{j-1} and O may be rescaled once O_{j-1} is complete
         if (j > 0) ok = __all_sync(0xffffffffu, ok && mbar_wait_bounded(&bar[B_OD], (j - 1) & 1, limit_ns, status,
                                                                         DEV_TIMEOUT_EPILOGUE));

@@ -12,8 +12,9 @@
 //   - S = Q K^T: tcgen05.mma M=128 N=128 K=64 into tensor memory;
 //   - each thread owns one query row: tcgen05.ld of its 128 scores, the
 //     maximum over keys < L, then exp2 of (s - max) / 8 log2 e as one FMA
-//     into ex2.approx (over the 16-key chunks below L) and the sum, both
-//     in four independent chains;
+//     into ex2.approx (packed pair FMAs over whole 16-key chunks, per-key
+//     masks only in the chunk that holds L) and the sum, in independent
+//     chains;
 //     P (bf16, or f16 for f16 operands) is written row-major, swizzled, over
 //     the Q and K tiles as the A operand of the next MMA;
 //   - O = P V: tcgen05.mma M=128 N=64 K=128 into S's tensor-memory columns;
@@ -119,23 +120,35 @@ __global__ void __launch_bounds__(AT_THREADS, 3) attention_tc_kernel(const __gri
     // exp2((s - max) / 8 log2 e) as one FMA into ex2; the scale is positive,
     // so max(s) * scale = max(s * scale)
     const float nm = got ? -mx * sl2 : 0.f;
-    float s8[4];
+    // whole 16-key chunks: the argument as a packed pair FMA, the sum in
+    // four packed chains; the chunk that holds L masks per key; chunks past
+    // the segment stay zero (all tests are uniform across the block)
+    const float2 sl2v = make_float2(sl2, sl2), nmv = make_float2(nm, nm);
+    float2 s2[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) s8[i] = 0.f;
+    for (int i = 0; i < 4; ++i) s2[i] = make_float2(0.f, 0.f);
 #pragma unroll
     for (int c = 0; c < 128; c += 16) {
-      if (c < L && got) {  // uniform: 16-key chunks wholly past the segment stay zero
+      if (c + 16 <= L && got) {
+#pragma unroll
+        for (int j = c; j < c + 16; j += 2) {
+          const float2 a = fma2(make_float2(sv[j], sv[j + 1]), sl2v, nmv);
+          sv[j] = ex2_approx(a.x);
+          sv[j + 1] = ex2_approx(a.y);
+          s2[(j >> 1) & 3] = add2(s2[(j >> 1) & 3], make_float2(sv[j], sv[j + 1]));
+        }
+      } else if (c < L && got) {
 #pragma unroll
         for (int j = c; j < c + 16; ++j) {
           sv[j] = (j < L) ? ex2_approx(fmaf(sv[j], sl2, nm)) : 0.f;
-          s8[j & 3] += sv[j];
+          s2[(j >> 1) & 3].x += sv[j];
         }
       } else {
 #pragma unroll
         for (int j = c; j < c + 16; ++j) sv[j] = 0.f;
       }
     }
-    const float s = (s8[0] + s8[1]) + (s8[2] + s8[3]);
+    const float s = ((s2[0].x + s2[0].y) + (s2[1].x + s2[1].y)) + ((s2[2].x + s2[2].y) + (s2[3].x + s2[3].y));
     rsum = s > 0.f ? 1.f / s : 0.f;
     // P overwrites Q and K: every thread has passed bar_s, so the MMA that
     // read them is complete.

@@ -352,7 +352,12 @@ template <int KIND>
 cudaError_t launch16(const CUtensorMap* a_map, const GemmB& w, GemmParams p, int epi, int bn, int num_sms,
                      cudaStream_t st, const CUtensorMap* out_map) {
   p.out_tma = (out_map != nullptr && !(epi & (EPI_PE | EPI_SWIGLU))) ? 1 : 0;
-  p.k_full = (p.conv_box ? p.cb.k16_last == 4 : w.K % 64 == 0) ? 1 : 0;
+  // Whole four-step k-blocks everywhere when A and B both come by TMA: the
+  // steps past K (or past a tap's channels) multiply the zeros that the TMA
+  // fills outside the tensors and that pad the conv weights, and issuing
+  // them costs less than a test per k-block.  The cp.async gather leaves
+  // those bytes unwritten, so it keeps the partial steps.
+  p.k_full = a_map != nullptr ? 1 : 0;
   // Tile order: the tiles running at once share the larger operand, so it
   // crosses from DRAM once and is re-read from L2 (and the TMA latency the
   // stage ring has to cover is the L2's, not the DRAM's).  A (M x K) is the
@@ -425,7 +430,7 @@ cudaError_t launch_gemm(const CUtensorMap* a_map, const GemmB& w, GemmParams p, 
   // operands), no gather mode
   p.out_tma = (out_map != nullptr && !(epi & (EPI_PE | EPI_SWIGLU))) ? 1 : 0;
   p.n_fast = (p.conv_box || p.M > w.N) ? 1 : 0;
-  p.k_full = (p.conv_box ? p.cb.k16_last == 4 : w.K % 32 == 0) ? 1 : 0;
+  p.k_full = 1;  // A and B by TMA (see launch16)
   const int slot = gemm_bn_slot(bn);
   if (bn < 0 || slot < 0 || p.M <= 0 || !a_map) return cudaErrorInvalidValue;
   p.sk = 0;

@@ -16,77 +16,120 @@ namespace asr {
 //   mean = K + S1 / D,  var = S2 / D - (S1 / D)^2,
 //   S1 = sum (x - K),   S2 = sum (x - K)^2,
 // which keeps the cancellation at the scale of the row's spread (|x - K|
-// is a few standard deviations), not of its mean.  Four rows per 128-thread
-// block.
+// is a few standard deviations), not of its mean.
+// The grid is one wave of resident blocks (four warps each); a warp takes
+// rows gw, gw + W, ... and copies its next row into its shared-memory
+// buffer (cp.async) while it normalises the current one, so rows past the
+// first wave do not pay a second memory round trip.  Gamma and beta are
+// staged in shared memory once per block, before the dependency wait (they
+// are weights, not the previous kernel's output).
 
 template <int V, int OUT>
 __global__ void __launch_bounds__(128) layer_norm_kernel(const float* __restrict__ x, const float* __restrict__ g,
                                                          const float* __restrict__ b, long long M, float eps,
                                                          void* __restrict__ y) {
+  constexpr int D = V * 128;
+  extern __shared__ float4 ln_smem[];
+  float4* g4 = ln_smem;                 // [D / 4]
+  float4* b4 = ln_smem + D / 4;         // [D / 4]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float4* buf = ln_smem + 2 * (D / 4) + warp * (D / 4);  // this warp's row buffer
+  for (int i = threadIdx.x; i < D / 4; i += 128) {
+    g4[i] = __ldg(reinterpret_cast<const float4*>(g) + i);
+    b4[i] = __ldg(reinterpret_cast<const float4*>(b) + i);
+  }
+  __syncthreads();
   pdl_wait();
   pdl_trigger();
-  const long long row = blockIdx.x * 4LL + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= M) return;
-  constexpr int D = V * 128;
-  const float4* xr = reinterpret_cast<const float4*>(x + row * D);
-  float4 v[V];
+  const long long W = gridDim.x * 4LL;
+  long long row = blockIdx.x * 4LL + warp;
+  auto fetch = [&](long long r) {
+    const float4* xr = reinterpret_cast<const float4*>(x + r * D);
 #pragma unroll
-  for (int i = 0; i < V; ++i) v[i] = __ldg(xr + lane + 32 * i);
-  const float K = __shfl_sync(0xffffffffu, v[0].x, 0);  // x[row][0]
-  float s1 = 0.f, s2 = 0.f;
+    for (int i = 0; i < V; ++i) cp_async_16_zfill(buf + lane + 32 * i, xr + lane + 32 * i, true);
+    cp_async_commit();
+  };
+  if (row < M) fetch(row);
+  for (; row < M; row += W) {
+    // each lane reads back exactly the 16-byte chunks it copied
+    cp_async_wait<0>();
+    float4 v[V];
 #pragma unroll
-  for (int i = 0; i < V; ++i) {
-    const float a = v[i].x - K, bb = v[i].y - K, c = v[i].z - K, d = v[i].w - K;
-    s1 += (a + bb) + (c + d);
-    s2 += (a * a + bb * bb) + (c * c + d * d);
-  }
+    for (int i = 0; i < V; ++i) v[i] = buf[lane + 32 * i];
+    if (row + W < M) fetch(row + W);
+    const float K = __shfl_sync(0xffffffffu, v[0].x, 0);  // x[row][0]
+    float s1 = 0.f, s2 = 0.f;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    s1 += __shfl_xor_sync(0xffffffffu, s1, o);
-    s2 += __shfl_xor_sync(0xffffffffu, s2, o);
-  }
-  const float m1 = s1 * (1.0f / D);
-  const float mean = K + m1;
-  const float var = fmaxf(s2 * (1.0f / D) - m1 * m1, 0.0f);
-  const float rstd = rsqrtf(var + eps);
-  const float4* g4 = reinterpret_cast<const float4*>(g);
-  const float4* b4 = reinterpret_cast<const float4*>(b);
+    for (int i = 0; i < V; ++i) {
+      const float a = v[i].x - K, bb = v[i].y - K, c = v[i].z - K, d = v[i].w - K;
+      s1 += (a + bb) + (c + d);
+      s2 += (a * a + bb * bb) + (c * c + d * d);
+    }
 #pragma unroll
-  for (int i = 0; i < V; ++i) {
-    const int c4 = lane + 32 * i;
-    const float4 gg = __ldg(g4 + c4), bv = __ldg(b4 + c4);
-    const float o0 = (v[i].x - mean) * rstd * gg.x + bv.x;
-    const float o1 = (v[i].y - mean) * rstd * gg.y + bv.y;
-    const float o2 = (v[i].z - mean) * rstd * gg.z + bv.z;
-    const float o3 = (v[i].w - mean) * rstd * gg.w + bv.w;
-    if (OUT == KIND_TF32) {
-      reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + row * D)[c4] = make_float4(o0, o1, o2, o3);
-    } else {
-      const uint2 w2 = make_uint2(pack2_16<OUT>(o0, o1), pack2_16<OUT>(o2, o3));
-      reinterpret_cast<uint2*>(reinterpret_cast<bf16*>(y) + row * D)[c4] = w2;
+    for (int o = 16; o > 0; o >>= 1) {
+      s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+      s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+    }
+    const float m1 = s1 * (1.0f / D);
+    const float mean = K + m1;
+    const float var = fmaxf(s2 * (1.0f / D) - m1 * m1, 0.0f);
+    const float rstd = rsqrtf(var + eps);
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+      const int c4 = lane + 32 * i;
+      const float4 gg = g4[c4], bv = b4[c4];
+      const float o0 = (v[i].x - mean) * rstd * gg.x + bv.x;
+      const float o1 = (v[i].y - mean) * rstd * gg.y + bv.y;
+      const float o2 = (v[i].z - mean) * rstd * gg.z + bv.z;
+      const float o3 = (v[i].w - mean) * rstd * gg.w + bv.w;
+      if (OUT == KIND_TF32) {
+        reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + row * D)[c4] = make_float4(o0, o1, o2, o3);
+      } else {
+        const uint2 w2 = make_uint2(pack2_16<OUT>(o0, o1), pack2_16<OUT>(o2, o3));
+        reinterpret_cast<uint2*>(reinterpret_cast<bf16*>(y) + row * D)[c4] = w2;
+      }
     }
   }
+}
+
+template <int V, int OUT>
+static cudaError_t ln_launch(const float* x, const float* g, const float* b, long long M, float eps, void* y,
+                             cudaStream_t st) {
+  constexpr int SMEM = (2 + 4) * V * 128 * 4;  // gamma, beta, four row buffers
+  static int per_sm[64] = {0};                  // resident blocks per SM, per device
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (per_sm[dev] == 0) {
+    cudaError_t e = cudaFuncSetAttribute(layer_norm_kernel<V, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(layer_norm_kernel<V, OUT>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared);
+    int n = 0;
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, layer_norm_kernel<V, OUT>, 128, SMEM);
+    if (e != cudaSuccess) return e;
+    per_sm[dev] = n > 0 ? n : 1;
+  }
+  int sms = 0;
+  cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const long long need = (M + 3) / 4;
+  const long long wave = (long long)sms * per_sm[dev];
+  const unsigned blocks = static_cast<unsigned>(need < wave ? need : wave);
+  return launch_pdl(layer_norm_kernel<V, OUT>, dim3(blocks), dim3(128), SMEM, st, x, g, b, M, eps, y);
 }
 
 template <int OUT>
 static cudaError_t ln_dispatch(int V, const float* x, const float* g, const float* b, long long M, float eps, void* y,
                                cudaStream_t st) {
-  const unsigned blocks = static_cast<unsigned>((M + 3) / 4);
   switch (V) {
 #define ASR_LN_CASE(n) \
-  case n: {                                                                                  \
-    cudaError_t e_ = launch_pdl(layer_norm_kernel<n, OUT>, dim3(blocks), dim3(128), 0, st, x, g, b, M, eps, y); \
-    if (e_ != cudaSuccess) return e_;                                                        \
-    break;                                                                                   \
-  }
+  case n: return ln_launch<n, OUT>(x, g, b, M, eps, y, st);
     ASR_LN_CASE(1) ASR_LN_CASE(2) ASR_LN_CASE(3) ASR_LN_CASE(4) ASR_LN_CASE(5) ASR_LN_CASE(6) ASR_LN_CASE(7)
     ASR_LN_CASE(8) ASR_LN_CASE(9) ASR_LN_CASE(10) ASR_LN_CASE(11) ASR_LN_CASE(12) ASR_LN_CASE(13)
     ASR_LN_CASE(14) ASR_LN_CASE(15) ASR_LN_CASE(16)
 #undef ASR_LN_CASE
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_layer_norm(const float* x, const float* g, const float* b, long long M, int D, float eps, void* y,
