@@ -56,6 +56,10 @@ struct Plan {
   int64_t n = 0, Tc = 0, T = 0;
   int B = 0, F = 0, nwin_clip = 0, nwin = 0, max_win = 0, chunks = 0;
   int T1 = 0, F1 = 0, T2 = 0, F2 = 0, T3 = 0, F3 = 0;
+  // conv1 / conv2 output rows (positions) and, in the packed layout, the
+  // per-chunk row stride S2 = T2 + 1 of the conv1 planes and of conv2's output
+  int S2 = 0;
+  int64_t rows1 = 0, rows2 = 0;
   // Variable-length batches (conv2d stem): per-clip layout, padded conv_out
   // rows (every chunk padded to T3 tokens), total frames and mel groups.
   bool varlen = false, has_short = false;
@@ -169,6 +173,15 @@ int64_t numel(const WSpec& w) {
 // Tokens of a chunk of L frames after three k3 s2 p1 convolutions.
 int64_t chunk_tokens(int64_t L) { return conv_len(conv_len(conv_len(L, 3, 2, 1), 3, 2, 1), 3, 2, 1); }
 
+// Output rows of conv1 and conv2 (conv2d stem): [chunk][T][F] each, or in the
+// packed layout the four conv1 parity planes [plane][chunk][S2][F1 / 2] and
+// conv2's [chunk][S2][F2], S2 = T2 + 1 (one zero row per chunk).
+void set_stem_rows(bool packed, Plan* p) {
+  p->S2 = packed ? p->T2 + 1 : 0;
+  p->rows1 = packed ? 4LL * p->chunks * p->S2 * (p->F1 / 2) : (int64_t)p->chunks * p->T1 * p->F1;
+  p->rows2 = (int64_t)p->chunks * (packed ? p->S2 : p->T2) * p->F2;
+}
+
 // Tokens per clip, or -1.  frames = floor(n / hop) (the trailing STFT frame
 // dropped); the conv2d stem's last chunk may be short.
 int64_t tokens_from_frames(const asr_geometry* g, int64_t frames) {
@@ -234,6 +247,12 @@ struct asr_enc {
   GemmB c1, c2, c3, cout;  // conv stem GEMMs (conv1: [C][16] taps kh*3+kw, 9..15 zero)
   bool box2 = false, box3 = false;  // conv GEMMs read A as strided TMA boxes (else cp.async gather)
   bool phase2 = false;              // conv1 writes parity planes, conv2 reads dense boxes
+  // Packed stem layout (parity planes, odd conv2 length per chunk): the
+  // chunks follow each other along time with one zero row after each (conv1
+  // planes and conv2 output alike), so the stride-2 convolutions read the
+  // neighbour chunk's zero row as their padding and conv2 / conv3 tiles run
+  // across chunk boundaries (no partly empty tiles).
+  bool packed = false;
   float* pe = nullptr;
   int pe_rows = 0;
   std::vector<LayerW> layers;
@@ -553,6 +572,8 @@ asr_status asr_enc_create(const asr_geometry* g, const void* const* weights, int
     e->box3 = f3 > 0 && 128 % f3 == 0 && (128 / f3) * 2 <= 256 && f3 * 2 <= 256;
     const int t1 = (int)conv_len(g->chunk_frames, 3, 2, 1);
     e->phase2 = e->box2 && t1 % 2 == 0 && f1 % 2 == 0 && f2 == f1 / 2;
+    const int t2 = (int)conv_len(t1, 3, 2, 1);
+    e->packed = e->phase2 && e->box3 && t2 % 2 == 1;
     if (e->kind == KIND_TF32 && !(e->box2 && e->box3))
       return bad(fail(e, ASR_E_UNSUPPORTED, "fp32 weights need conv outputs whose frequency rows divide 128"));
     for (int layer = 0; layer < 2; ++layer) {
@@ -692,9 +713,10 @@ bool make_plan(const asr_enc* e, int64_t n, int B, Plan* p) {
     p->T2 = (int)conv_len(p->T1, 3, 2, 1); p->F2 = (int)conv_len(p->F1, 3, 2, 1);
     p->T3 = (int)conv_len(p->T2, 3, 2, 1); p->F3 = (int)conv_len(p->F2, 3, 2, 1);
     const size_t C = g->conv_ch;
-    p->off_a1 = take((size_t)p->chunks * p->T1 * p->F1 * 16 * es);
-    p->off_c1 = take((size_t)p->chunks * p->T1 * p->F1 * C * es);
-    p->off_c2 = take((size_t)p->chunks * p->T2 * p->F2 * C * es);
+    set_stem_rows(e->packed, p);
+    p->off_a1 = take((size_t)p->rows1 * 16 * es);
+    p->off_c1 = take((size_t)p->rows1 * C * es);
+    p->off_c2 = take((size_t)p->rows2 * C * es);
     p->off_c3 = take((size_t)p->T * p->F3 * C * es);
   } else {
     p->off_melT = take((size_t)B * p->F * g->n_mels * es);
@@ -788,9 +810,10 @@ bool make_plan_varlen(const asr_enc* e, const int64_t* ns, int B, Plan* p, const
   p->off_chunkd = take((size_t)p->chunks * sizeof(ChunkDesc));
   p->off_cu = take((size_t)(p->nwin + 1) * 4);
   p->off_mel = take((size_t)g->n_mels * p->Ftot * 4);
-  p->off_a1 = take((size_t)p->chunks * p->T1 * p->F1 * 16 * es);
-  p->off_c1 = take((size_t)p->chunks * p->T1 * p->F1 * C * es);
-  p->off_c2 = take((size_t)p->chunks * p->T2 * p->F2 * C * es);
+  set_stem_rows(e->packed, p);
+  p->off_a1 = take((size_t)p->rows1 * 16 * es);
+  p->off_c1 = take((size_t)p->rows1 * C * es);
+  p->off_c2 = take((size_t)p->rows2 * C * es);
   p->off_c3 = take((size_t)p->Tpad * p->F3 * C * es);
   p->off_xpad = take((size_t)p->Tpad * d * 4);
   p->off_x = take((size_t)p->T * d * 4);
@@ -828,7 +851,7 @@ bool plan_for(const asr_enc* e, const int64_t* ns, int64_t n, int B, Plan* p) {
 
 asr_status gemm(asr_enc* e, const CUtensorMap* amap, const ConvGather* cg, const GemmB& w, long long M, void* out,
                 long long ldo, const float* bias, const float* pe, int period, int epi, cudaStream_t st,
-                const CUtensorMap* omap, const ConvBox* box = nullptr) {
+                const CUtensorMap* omap, const ConvBox* box = nullptr, int zero_period = 0, int zero_from = 0) {
   // fp32 operands: every output of the engine is fp32
   if (e->kind == KIND_TF32 && !(epi & (EPI_OUT_F32 | EPI_RESID))) epi |= EPI_OUT_F32;
   GemmParams p;
@@ -842,6 +865,8 @@ asr_status gemm(asr_enc* e, const CUtensorMap* amap, const ConvGather* cg, const
   if (cg) p.g = *cg;
   p.status = e->status;
   p.limit_ns = kWaitLimitNs;
+  p.zero_period = zero_period;
+  p.zero_from = zero_from;
   int bn;
   if (box) {
     p.conv_box = 1;
@@ -911,11 +936,15 @@ asr_status ensure_maps(asr_enc* e, const Plan& p, char* ws) {
   if (ok && g->stem == ASR_STEM_CONV2D_CHUNKED) {
     const int C = g->conv_ch;
     ok = make_tmap_act(k, &m.c3, ws + p.off_c3, p.Tpad, (size_t)p.F3 * C, (size_t)p.F3 * C, 128) &&
-         make_tmap_act(k, &m.a1, ws + p.off_a1, (size_t)p.chunks * p.T1 * p.F1, 16, 16, 128);
+         make_tmap_act(k, &m.a1, ws + p.off_a1, (size_t)p.rows1, 16, 16, 128);
+    // packed: one image of chunks x S2 rows (planes: [4][chunks * S2][F1 / 2][C])
     if (ok && e->box2)
-      ok = e->phase2 ? make_tmap_convphase(&m.cin2, ws + p.off_c1, C, p.F1 / 2, p.T1 / 2, 4 * p.chunks, p.F2, 128 / p.F2, k)
-                     : make_tmap_convbox(&m.cin2, ws + p.off_c1, C, p.F1, p.T1, p.chunks, p.F2, 2, 128 / p.F2, 2, k);
-    if (ok && e->box3) ok = make_tmap_convbox(&m.cin3, ws + p.off_c2, C, p.F2, p.T2, p.chunks, p.F3, 2, 128 / p.F3, 2, k);
+      ok = e->packed   ? make_tmap_convphase(&m.cin2, ws + p.off_c1, C, p.F1 / 2, p.chunks * p.S2, 4, p.F2, 128 / p.F2, k)
+           : e->phase2 ? make_tmap_convphase(&m.cin2, ws + p.off_c1, C, p.F1 / 2, p.T1 / 2, 4 * p.chunks, p.F2, 128 / p.F2, k)
+                       : make_tmap_convbox(&m.cin2, ws + p.off_c1, C, p.F1, p.T1, p.chunks, p.F2, 2, 128 / p.F2, 2, k);
+    if (ok && e->box3)
+      ok = e->packed ? make_tmap_convbox(&m.cin3, ws + p.off_c2, C, p.F2, p.chunks * p.S2, 1, p.F3, 2, 128 / p.F3, 2, k)
+                     : make_tmap_convbox(&m.cin3, ws + p.off_c2, C, p.F2, p.T2, p.chunks, p.F3, 2, 128 / p.F3, 2, k);
   } else if (ok) {
     ok = make_tmap_convbox(&m.cin2, ws + p.off_melT, g->n_mels, 1, p.F, p.B, 1, 1, 128, 1, k) &&
          make_tmap_convbox(&m.cin3, ws + p.off_c1, d, 1, p.F, p.B, 1, 1, 128, 2, k);
@@ -930,8 +959,8 @@ asr_status ensure_maps(asr_enc* e, const Plan& p, char* ws) {
          make_tmap_out(&m.o_qkv, ws + p.off_qkv, p.T, 3 * d, 3 * d, f32) &&
          make_tmap_out(&m.o_ff, ws + p.off_ff, p.T, g->d_ffn, g->d_ffn, f32);
   if (ok && g->stem == ASR_STEM_CONV2D_CHUNKED)
-    ok = make_tmap_out(&m.o_c1, ws + p.off_c1, (unsigned long long)p.chunks * p.T1 * p.F1, g->conv_ch, g->conv_ch, f32) &&
-         make_tmap_out(&m.o_c2, ws + p.off_c2, (unsigned long long)p.chunks * p.T2 * p.F2, g->conv_ch, g->conv_ch, f32) &&
+    ok = make_tmap_out(&m.o_c1, ws + p.off_c1, (unsigned long long)p.rows1, g->conv_ch, g->conv_ch, f32) &&
+         make_tmap_out(&m.o_c2, ws + p.off_c2, (unsigned long long)p.rows2, g->conv_ch, g->conv_ch, f32) &&
          make_tmap_out(&m.o_c3, ws + p.off_c3, (unsigned long long)p.chunks * p.T3 * p.F3, g->conv_ch, g->conv_ch, f32);
   else if (ok)
     ok = make_tmap_out(&m.o_c1, ws + p.off_c1, (unsigned long long)p.B * p.F, d, d, f32);
@@ -1007,33 +1036,42 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
     void* c2 = ws + p.off_c2;
     void* c3 = ws + p.off_c3;
     void* a1 = ws + p.off_a1;
+    // row layout of conv1's output: 0 plain, 1 parity planes per chunk, 2 packed
+    const int lay1 = e->packed ? 2 : (e->phase2 ? 1 : 0);
     if (!p.varlen)
-      ASR_K(PC_CONV1, ASR_LAUNCH(e, launch_conv1_im2col(mel, clip_max, p.B, g->n_mels, p.F, g->chunk_frames,
-                                                        e->phase2 ? 1 : 0, a1, e->kind, st)));
+      ASR_K(PC_CONV1, ASR_LAUNCH(e, launch_conv1_im2col(mel, clip_max, p.B, g->n_mels, p.F, g->chunk_frames, lay1, a1,
+                                                        e->kind, st)));
     else
-      ASR_K(PC_CONV1, ASR_LAUNCH(e, launch_conv1_im2col_varlen(mel, clip_max, p.chunks, g->n_mels, g->chunk_frames,
-                                                               e->phase2 ? 1 : 0, chunkd, mclips, a1, e->kind, st)));
-    ASR_K(PC_CONV1, ASR_TRY(gemm(e, &e->maps.a1, nullptr, e->c1, (long long)p.chunks * p.T1 * p.F1, c1, C, e->c1b,
-                                 nullptr, 1, EPI_GELU, st, &e->maps.o_c1)));
+      ASR_K(PC_CONV1, ASR_LAUNCH(e, launch_conv1_im2col_varlen(mel, clip_max, p.chunks, g->n_mels, g->chunk_frames, lay1,
+                                                               chunkd, mclips, a1, e->kind, st)));
+    // packed: the zero row j = S2 - 1 of every chunk in every plane stays zero
+    const int fh = p.F1 / 2;
+    ASR_K(PC_CONV1, ASR_TRY(gemm(e, &e->maps.a1, nullptr, e->c1, p.rows1, c1, C, e->c1b, nullptr, 1, EPI_GELU, st,
+                                 &e->maps.o_c1, nullptr, e->packed ? p.S2 * fh : 0, e->packed ? (p.S2 - 1) * fh : 0)));
     if (p.has_short)
-      ASR_K(PC_MISC, ASR_LAUNCH(e, launch_mask_short_chunks(c1, chunkd, p.chunks, g->chunk_frames, 1, p.T1, p.F1, C,
-                                                            e->phase2 ? 1 : 0, e->es, st)));
+      ASR_K(PC_MISC, ASR_LAUNCH(e, launch_mask_short_chunks(c1, chunkd, p.chunks, g->chunk_frames, 1, p.T1, p.F1, C, lay1,
+                                                            p.S2, e->es, st)));
     const int CB = (C + RE - 1) / RE;
     const int k_last = (C - RE * (CB - 1) + KST - 1) / KST;
     if (e->box2) {
-      const int TR = 128 / p.F2, tpi = (p.T2 + TR - 1) / TR;
-      ConvBox b2 = {TR, p.F2, p.T2, tpi, p.chunks * tpi, 2, 2, 1, 1, 3, CB, e->phase2 ? 1 : 0, k_last};
-      ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, &e->maps.cin2, nullptr, e->c2, (long long)p.chunks * p.T2 * p.F2, c2, C, e->c2b, nullptr, 1, EPI_GELU, st, &e->maps.o_c2, &b2)));
+      // packed: one image of chunks x S2 output rows, the last row of every
+      // chunk written as zeros (conv3's padding)
+      const int TR = 128 / p.F2, To = e->packed ? p.chunks * p.S2 : p.T2, tpi = (To + TR - 1) / TR;
+      ConvBox b2 = {TR, p.F2, To, tpi, e->packed ? tpi : p.chunks * tpi, 2, 2, 1, 1, 3, CB, e->phase2 ? 1 : 0, k_last};
+      ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, &e->maps.cin2, nullptr, e->c2, p.rows2, c2, C, e->c2b, nullptr, 1, EPI_GELU, st,
+                                       &e->maps.o_c2, &b2, e->packed ? p.S2 * p.F2 : 0, e->packed ? p.T2 * p.F2 : 0)));
     } else {
       ConvGather cg2 = {static_cast<const bf16*>(c1), p.T1, p.F1, C, p.T2, p.F2, 2, 2, 3, 3, 1, 1};
       ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, nullptr, &cg2, e->c2, (long long)p.chunks * p.T2 * p.F2, c2, C, e->c2b, nullptr, 1, EPI_GELU, st, &e->maps.o_c2)));
     }
     if (p.has_short)
-      ASR_K(PC_MISC, ASR_LAUNCH(e, launch_mask_short_chunks(c2, chunkd, p.chunks, g->chunk_frames, 2, p.T2, p.F2, C, 0,
-                                                            e->es, st)));
+      ASR_K(PC_MISC, ASR_LAUNCH(e, launch_mask_short_chunks(c2, chunkd, p.chunks, g->chunk_frames, 2, p.T2, p.F2, C,
+                                                            e->packed ? 2 : 0, p.S2, e->es, st)));
     if (e->box3) {
-      const int TR = 128 / p.F3, tpi = (p.T3 + TR - 1) / TR;
-      ConvBox b3 = {TR, p.F3, p.T3, tpi, p.chunks * tpi, 2, 2, 1, 1, 3, CB, 0, k_last};
+      // packed: conv3 output row o = 13 c + t reads conv2 rows 26 c + 2 t - 1 ..
+      // + 1 of the one image, whose zero rows are the chunks' padding
+      const int TR = 128 / p.F3, To = e->packed ? p.chunks * p.T3 : p.T3, tpi = (To + TR - 1) / TR;
+      ConvBox b3 = {TR, p.F3, To, tpi, e->packed ? tpi : p.chunks * tpi, 2, 2, 1, 1, 3, CB, 0, k_last};
       ASR_K(PC_GEMM_CONV, ASR_TRY(gemm(e, &e->maps.cin3, nullptr, e->c3, (long long)p.chunks * p.T3 * p.F3, c3, C, e->c3b, nullptr, 1, EPI_GELU, st, &e->maps.o_c3, &b3)));
     } else {
       ConvGather cg3 = {static_cast<const bf16*>(c2), p.T2, p.F2, C, p.T3, p.F3, 2, 2, 3, 3, 1, 1};

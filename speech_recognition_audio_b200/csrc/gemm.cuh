@@ -95,6 +95,9 @@ struct GemmParams {
   int sk;
   int* sk_flags;          // [pairs][2 CTAs][8 warps], zero before the launch
   int k_full;             // 1 = every k-block holds four whole MMA steps (set by the launcher)
+  // Output rows r with r % zero_period >= zero_from are written as zeros
+  // (the padding rows of a packed convolution layout); zero_period 0 = none.
+  int zero_period, zero_from;
 };
 
 template <bool B>
@@ -391,6 +394,10 @@ __device__ __forceinline__ void epilogue_warp(const GemmParams& p, const CUtenso
       const float bj = breg[j];
 #pragma unroll
       for (int i = 0; i < 32; ++i) v[i] += __shfl_sync(0xffffffffu, bj, i);
+    }
+    if (p.zero_period && (row0 + lane) % p.zero_period >= p.zero_from) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = 0.f;  // GELU(0) = 0: the row stays zero
     }
     if (SWI && F32) {
       // gate = columns c..c+15, up = c+16..c+31 -> 16 fp32 outputs of this row

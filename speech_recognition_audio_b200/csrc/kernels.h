@@ -98,16 +98,21 @@ cudaError_t launch_varlen_fill(const VarClipBatch& vb, int chunk_frames, int win
 cudaError_t launch_conv1_im2col_varlen(const float* mel_raw, const unsigned int* clip_max, int n_chunks, int n_mels,
                                        int chunk_frames, int phase, const ChunkDesc* cd, const MelClip* mc, void* a,
                                        int kind, cudaStream_t st);
+// layout: 0 [chunk][T][F], 1 parity planes per chunk, 2 packed (S2 rows per
+// chunk: conv1 planes [4][chunk][S2][F / 2] at level 1, conv2 [chunk][S2][F]
+// at level 2).
 cudaError_t launch_mask_short_chunks(void* act, const ChunkDesc* cd, int n_chunks, int chunk_frames, int level, int T,
-                                     int F, int C, int phase, int es, cudaStream_t st);
+                                     int F, int C, int layout, int S2, int es, cudaStream_t st);
 cudaError_t launch_compact_tokens(const float* xpad, float* x, const ChunkDesc* cd, int n_chunks, int t3, int d,
                                   cudaStream_t st);
 
 // A operand of the first Conv2D (1 -> C, k3 s2 p1) as a GEMM: per output
 // position of each chunk of chunk_frames frames, its 9 normalised log-mel
 // taps (kh * 3 + kw) as bf16 in a row of 16 (taps 9..15 zero).  Rows
-// [chunks][T1][F1], or with phase != 0 (T1, F1 even) the parity planes
-// [chunks][t % 2][f % 2][T1 / 2][F1 / 2] read by the phase-mode conv2.
+// (phase = layout): 0 [chunks][T1][F1]; 1 (T1, F1 even) the parity planes
+// [chunks][t % 2][f % 2][T1 / 2][F1 / 2] read by the phase-mode conv2;
+// 2 the packed planes [t % 2][f % 2][chunks][T1 / 2 + 1][F1 / 2], whose last
+// row per chunk is zero.
 // a: rows of the kind's element type (bf16, f16, or fp32 for KIND_TF32).
 cudaError_t launch_conv1_im2col(const float* mel_raw, const unsigned int* clip_max, int batch, int n_mels,
                                 int n_frames, int chunk_frames, int phase, void* a, int kind, cudaStream_t st);

@@ -11,10 +11,13 @@
 // maximum - 8, then (x + 4) / 4; zero outside the chunk), as bf16, in rows
 // of 16.
 //
-// Row order: plain [chunk][T1][F1], or (phase mode, T1 and F1 even) the
+// Row order (layout): 0 plain [chunk][T1][F1]; 1 (T1 and F1 even) the
 // chunk's four parity planes [chunk][t % 2][f % 2][T1 / 2][F1 / 2], so the
 // GEMM's output rows land in the layout the stride-2 conv2 reads as dense
-// TMA boxes.  Threads run along time within a plane row so that the mel
+// TMA boxes; 2 (packed) the planes over all chunks,
+// [t % 2][f % 2][chunk][S2][F1 / 2] with S2 = T1 / 2 + 1: the last row of
+// every chunk is a zero row (A row zero here; the GEMM writes its output
+// row as zero).  Threads run along time within a plane row so that the mel
 // reads (frames contiguous) are coalesced; each thread writes one 32-byte
 // row.
 #include "kernels.h"
@@ -26,20 +29,43 @@ __global__ void __launch_bounds__(256) conv1_im2col_kernel(const float* __restri
                                                            const unsigned int* __restrict__ clip_max, int n_mels,
                                                            int n_frames, int chunk_frames, int chunks_per_clip,
                                                            int T1, int F1, long long rows, int phase,
-                                                           const ChunkDesc* __restrict__ cd,
+                                                           long long n_chunks, const ChunkDesc* __restrict__ cd,
                                                            const MelClip* __restrict__ mc, void* __restrict__ a_out) {
   pdl_wait();
   pdl_trigger();
   const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
   if (i >= rows) return;
-  // thread index -> (chunk, plane, f, t) with t fastest
-  const int TP = phase ? T1 / 2 : T1, FP = phase ? F1 / 2 : F1;
-  const int t = static_cast<int>(i % TP);
-  long long rest = i / TP;
+  // thread index -> (chunk, plane, f, t) with t fastest (t < TS; t = TP is
+  // the packed layout's zero row)
+  const int TP = phase ? T1 / 2 : T1, FP = phase ? F1 / 2 : F1, TS = phase == 2 ? TP + 1 : TP;
+  const int t = static_cast<int>(i % TS);
+  long long rest = i / TS;
   const int f = static_cast<int>(rest % FP);
   rest /= FP;
-  const int plane = phase ? static_cast<int>(rest % 4) : 0;
-  const long long chunk = phase ? rest / 4 : rest;
+  int plane;
+  long long chunk;
+  if (phase == 2) {
+    chunk = rest % n_chunks;
+    plane = static_cast<int>(rest / n_chunks);
+  } else {
+    plane = phase ? static_cast<int>(rest % 4) : 0;
+    chunk = phase ? rest / 4 : rest;
+  }
+  // output row: [chunk][plane][T][F] (plain: [chunk][T1][F1]; packed:
+  // [plane][chunk][S2][F])
+  const long long row = phase == 2 ? ((plane * n_chunks + chunk) * (long long)TS + t) * FP + f
+                                   : (chunk * (phase ? 4 : 1) + plane) * (long long)TP * FP + (long long)t * FP + f;
+  if (t >= TP) {
+    if constexpr (OUTK == KIND_TF32) {
+      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a_out) + row * 16);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) dst[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    } else {
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a_out) + row * 16);
+      dst[0] = dst[1] = make_uint4(0, 0, 0, 0);
+    }
+    return;
+  }
   const int t1 = phase ? 2 * t + (plane >> 1) : t;
   const int f1 = phase ? 2 * f + (plane & 1) : f;
   int b, F, valid;
@@ -74,8 +100,6 @@ __global__ void __launch_bounds__(256) conv1_im2col_kernel(const float* __restri
     }
 #pragma unroll
   for (int k = 9; k < 16; ++k) v[k] = 0.f;
-  // output row: [chunk][plane][T][F] (plain: [chunk][T1][F1])
-  const long long row = (chunk * (phase ? 4 : 1) + plane) * (long long)TP * FP + (long long)t * FP + f;
   if constexpr (OUTK == KIND_TF32) {
     float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a_out) + row * 16);
 #pragma unroll
@@ -91,44 +115,50 @@ __global__ void __launch_bounds__(256) conv1_im2col_kernel(const float* __restri
 template <int OUTK>
 static cudaError_t im2col_launch(const float* mel_raw, const unsigned int* clip_max, int n_mels, int n_frames,
                                  int chunk_frames, int chunks_per_clip, int T1, int F1, long long rows, int phase,
-                                 const ChunkDesc* cd, const MelClip* mc, void* a, cudaStream_t st) {
+                                 long long n_chunks, const ChunkDesc* cd, const MelClip* mc, void* a, cudaStream_t st) {
   const unsigned blocks = static_cast<unsigned>((rows + 255) / 256);
   return launch_pdl(conv1_im2col_kernel<OUTK>, dim3(blocks), dim3(256), 0, st, mel_raw, clip_max, n_mels, n_frames,
-                    chunk_frames, chunks_per_clip, T1, F1, rows, phase, cd, mc, a);
+                    chunk_frames, chunks_per_clip, T1, F1, rows, phase, n_chunks, cd, mc, a);
 }
 
 static cudaError_t im2col_kind(int kind, const float* mel_raw, const unsigned int* clip_max, int n_mels, int n_frames,
                                int chunk_frames, int chunks_per_clip, int T1, int F1, long long rows, int phase,
-                               const ChunkDesc* cd, const MelClip* mc, void* a, cudaStream_t st) {
+                               long long n_chunks, const ChunkDesc* cd, const MelClip* mc, void* a, cudaStream_t st) {
   switch (kind) {
     case KIND_TF32: return im2col_launch<KIND_TF32>(mel_raw, clip_max, n_mels, n_frames, chunk_frames, chunks_per_clip,
-                                                    T1, F1, rows, phase, cd, mc, a, st);
+                                                    T1, F1, rows, phase, n_chunks, cd, mc, a, st);
     case KIND_F16: return im2col_launch<KIND_F16>(mel_raw, clip_max, n_mels, n_frames, chunk_frames, chunks_per_clip,
-                                                  T1, F1, rows, phase, cd, mc, a, st);
+                                                  T1, F1, rows, phase, n_chunks, cd, mc, a, st);
     default: return im2col_launch<KIND_BF16>(mel_raw, clip_max, n_mels, n_frames, chunk_frames, chunks_per_clip, T1,
-                                             F1, rows, phase, cd, mc, a, st);
+                                             F1, rows, phase, n_chunks, cd, mc, a, st);
   }
+}
+
+// Rows of the A operand (= conv1 output positions) in a layout.
+static long long im2col_rows(long long chunks, int T1, int F1, int phase) {
+  return phase == 2 ? 4LL * chunks * (T1 / 2 + 1) * (F1 / 2) : chunks * T1 * F1;
 }
 
 cudaError_t launch_conv1_im2col(const float* mel_raw, const unsigned int* clip_max, int batch, int n_mels,
                                 int n_frames, int chunk_frames, int phase, void* a, int kind, cudaStream_t st) {
   const int T1 = (chunk_frames - 1) / 2 + 1, F1 = (n_mels - 1) / 2 + 1;
-  if (phase && (T1 % 2 || F1 % 2)) return cudaErrorInvalidValue;
+  if (phase < 0 || phase > 2 || (phase && (T1 % 2 || F1 % 2))) return cudaErrorInvalidValue;
   const int chunks_per_clip = n_frames / chunk_frames;
-  const long long rows = (long long)batch * chunks_per_clip * T1 * F1;
+  const long long chunks = (long long)batch * chunks_per_clip;
+  const long long rows = im2col_rows(chunks, T1, F1, phase);
   if (rows == 0) return cudaSuccess;
-  return im2col_kind(kind, mel_raw, clip_max, n_mels, n_frames, chunk_frames, chunks_per_clip, T1, F1, rows,
-                     phase ? 1 : 0, nullptr, nullptr, a, st);
+  return im2col_kind(kind, mel_raw, clip_max, n_mels, n_frames, chunk_frames, chunks_per_clip, T1, F1, rows, phase,
+                     chunks, nullptr, nullptr, a, st);
 }
 
 cudaError_t launch_conv1_im2col_varlen(const float* mel_raw, const unsigned int* clip_max, int n_chunks, int n_mels,
                                        int chunk_frames, int phase, const ChunkDesc* cd, const MelClip* mc, void* a,
                                        int kind, cudaStream_t st) {
   const int T1 = (chunk_frames - 1) / 2 + 1, F1 = (n_mels - 1) / 2 + 1;
-  if (phase && (T1 % 2 || F1 % 2)) return cudaErrorInvalidValue;
-  const long long rows = (long long)n_chunks * T1 * F1;
+  if (phase < 0 || phase > 2 || (phase && (T1 % 2 || F1 % 2))) return cudaErrorInvalidValue;
+  const long long rows = im2col_rows(n_chunks, T1, F1, phase);
   if (rows == 0) return cudaSuccess;
-  return im2col_kind(kind, mel_raw, clip_max, n_mels, 0, chunk_frames, 1, T1, F1, rows, phase ? 1 : 0, cd, mc, a, st);
+  return im2col_kind(kind, mel_raw, clip_max, n_mels, 0, chunk_frames, 1, T1, F1, rows, phase, n_chunks, cd, mc, a, st);
 }
 
 // ---------------------------------------------------------- short chunks
@@ -141,7 +171,7 @@ cudaError_t launch_conv1_im2col_varlen(const float* mel_raw, const unsigned int*
 // (ceil(ceil(L / 2) / 2)).  One block per chunk; whole chunks return at once.
 // (act: elements of `es` bytes, 2 or 4; C * es a multiple of 16.)
 __global__ void mask_short_chunks_kernel(uint8_t* __restrict__ act, const ChunkDesc* __restrict__ cd, int chunk_frames,
-                                         int level, int T, int F, int C, int phase, int es) {
+                                         int level, int T, int F, int C, int layout, int S2, int n_chunks, int es) {
   pdl_wait();
   pdl_trigger();
   const int c = blockIdx.x;
@@ -151,19 +181,23 @@ __global__ void mask_short_chunks_kernel(uint8_t* __restrict__ act, const ChunkD
   if (level == 2) tv = (tv + 1) / 2;
   if (tv >= T) return;
   const uint4 z = make_uint4(0, 0, 0, 0);
-  if (!phase) {
-    // rows [tv, T) of the chunk's [T][F][C] block are contiguous
-    uint4* p = reinterpret_cast<uint4*>(act + ((long long)c * T + tv) * F * C * es);
+  if (layout == 0 || (layout == 2 && level == 2)) {
+    // rows [tv, T) of the chunk's [T][F][C] block are contiguous (packed
+    // conv2 output: the chunk's block starts at row c * S2)
+    const long long r0 = (layout == 2 ? (long long)c * S2 : (long long)c * T) + tv;
+    uint4* p = reinterpret_cast<uint4*>(act + r0 * F * C * es);
     const long long n16 = (long long)(T - tv) * F * C * es / 16;
     for (long long j = threadIdx.x; j < n16; j += blockDim.x) p[j] = z;
   } else {
-    // parity planes [4][T/2][F/2][C]: plane (pt, pf) holds t = 2 th + pt
+    // parity planes: plane (pt, pf) holds t = 2 th + pt, TH = T / 2 rows of
+    // the chunk, [chunk][4][TH] (layout 1) or [4][chunk][S2] (layout 2)
     const int TH = T / 2, FH = F / 2;
     for (int pl = 0; pl < 4; ++pl) {
       const int pt = pl >> 1;
       const int th0 = tv - pt <= 0 ? 0 : (tv - pt + 1) / 2;
       if (th0 >= TH) continue;
-      uint4* p = reinterpret_cast<uint4*>(act + (((long long)c * 4 + pl) * TH + th0) * FH * C * es);
+      const long long r0 = layout == 2 ? ((long long)pl * n_chunks + c) * S2 + th0 : ((long long)c * 4 + pl) * TH + th0;
+      uint4* p = reinterpret_cast<uint4*>(act + r0 * FH * C * es);
       const long long n16 = (long long)(TH - th0) * FH * C * es / 16;
       for (long long j = threadIdx.x; j < n16; j += blockDim.x) p[j] = z;
     }
@@ -171,11 +205,13 @@ __global__ void mask_short_chunks_kernel(uint8_t* __restrict__ act, const ChunkD
 }
 
 cudaError_t launch_mask_short_chunks(void* act, const ChunkDesc* cd, int n_chunks, int chunk_frames, int level, int T,
-                                     int F, int C, int phase, int es, cudaStream_t st) {
+                                     int F, int C, int layout, int S2, int es, cudaStream_t st) {
   if (n_chunks <= 0) return cudaSuccess;
-  if ((C * es) % 16 || (phase && (T % 2 || F % 2))) return cudaErrorInvalidValue;
+  if ((C * es) % 16 || layout < 0 || layout > 2 || (layout == 1 && (T % 2 || F % 2)) ||
+      (layout == 2 && level == 1 && (T % 2 || F % 2 || S2 != T / 2 + 1)) || (layout == 2 && level == 2 && S2 != T + 1))
+    return cudaErrorInvalidValue;
   return launch_pdl(mask_short_chunks_kernel, dim3(n_chunks), dim3(256), 0, st, static_cast<uint8_t*>(act), cd,
-                    chunk_frames, level, T, F, C, phase, es);
+                    chunk_frames, level, T, F, C, layout, S2, n_chunks, es);
 }
 
 // Valid tokens of every chunk, from the padded conv_out rows [chunk][t3] to
