@@ -5,9 +5,9 @@
 // tokens the one-tile kernel of attn_tc.cu takes.
 //
 // One CTA per (128-query tile, segment, head), 10 warps:
-//   warp 8  TMA producer: Q once, then K_j (two buffers, so K_{j+1} arrives
-//           while tile j is in flight) and V_j (one buffer, loaded once the
-//           previous tile's P V has read it);
+//   warp 8  TMA producer: Q once, then K_j (one buffer, reloaded once S_j
+//           has read it) and V_j (two buffers, so V_{j+1} arrives while the
+//           softmax and P V of tile j run);
 //   warp 9  MMA issuer: S = Q K_j^T (M=128, N=128, K=64) into tensor memory,
 //           issued for tile j+1 as soon as the softmax has read S_j, then
 //           O += P_j V_j (M=128, N=64, K=128) with O kept in tensor memory;
@@ -25,7 +25,7 @@
 //           next MMA; at the end each thread divides its 32 O columns by the
 //           row sum and stores them.
 // Tensor memory: S in columns 0..127, O in 128..191 (256 allocated: two
-// CTAs per SM).  Shared memory: Q (16 KB), K (2 x 16 KB), V (16 KB), P
+// CTAs per SM).  Shared memory: Q (16 KB), K (16 KB), V (2 x 16 KB), P
 // (32 KB).  Every wait is bounded; tensor memory is freed after all MMAs
 // have completed.
 #include "kernels.h"
@@ -34,8 +34,13 @@ namespace asr {
 
 namespace {
 constexpr int FA_THREADS = 320;
-constexpr int FA_SQ = 0, FA_SK = 16384, FA_SV = 49152, FA_SP = 65536;  // K: two buffers; P: two 64-key halves
-constexpr int FA_TILES = 98304;
+// K and V ring slots (16 KB each): V double-buffered (measured 504 against
+// 535 us per whisper-small launch with K double-buffered instead; both
+// double-buffered do not fit two CTAs per SM, and one CTA per SM, or two
+// query tiles per CTA sharing the rings, measured slower)
+constexpr int FA_KB = 1, FA_VB = 2;
+constexpr int FA_SQ = 0, FA_SK = 16384, FA_SV = FA_SK + FA_KB * 16384, FA_SP = FA_SV + FA_VB * 16384;  // P: two 64-key halves
+constexpr int FA_TILES = FA_SP + 32768;
 constexpr int FA_RED = FA_TILES;                 // float [2 tiles][2 halves][128 rows] row maxima, then sums
 constexpr int FA_BARS = FA_RED + 2 * 2 * 128 * 4;
 constexpr int FA_SMEM = 1024 + FA_BARS + 256;
@@ -43,7 +48,8 @@ constexpr int FA_TMEM_COLS = 256;
 constexpr int FA_O_COL = 128;
 constexpr float FA_RESCALE_LOG2 = 8.0f;
 
-enum { B_Q = 0, B_KF0, B_KF1, B_KE0, B_KE1, B_VF, B_VE, B_SF, B_SFREE, B_PF, B_OD, B_DRAIN, B_COUNT };
+enum { B_Q = 0, B_KF0, B_KF1, B_KE0, B_KE1, B_VF0, B_VF1, B_VE0, B_VE1, B_SF, B_SFREE, B_PF, B_OD, B_DRAIN, B_COUNT };
+static_assert(FA_KB <= 2 && FA_VB <= 2, "barrier table");
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
   asm volatile(
@@ -101,25 +107,29 @@ __global__ void __launch_bounds__(FA_THREADS, 2) attention_fa_kernel(const __gri
         mbar_arrive_expect_tx(&bar[B_Q], 16384);
         tma_load_2d(sm + FA_SQ, &tm_qkv, &bar[B_Q], h * 64, s0 + q0);
         for (int j = 0; j < nk && ok; ++j) {
-          const int kb = j & 1;
-          // K_j into buffer j % 2 once S_{j-2} has read it
-          if (j >= 2 && !(ok = mbar_wait_bounded(&bar[B_KE0 + kb], ((j >> 1) - 1) & 1, limit_ns, status,
-                                                 DEV_TIMEOUT_PRODUCER)))
+          // K_j into ring slot j % KB once S_{j-KB} has read it
+          const int kb = j % FA_KB;
+          if (j >= FA_KB && !(ok = mbar_wait_bounded(&bar[B_KE0 + kb], (j / FA_KB - 1) & 1, limit_ns, status,
+                                                     DEV_TIMEOUT_PRODUCER)))
             break;
           mbar_arrive_expect_tx(&bar[B_KF0 + kb], 16384);
           tma_load_2d(sm + FA_SK + kb * 16384, &tm_qkv, &bar[B_KF0 + kb], (H + h) * 64, s0 + j * 128);
           ++issued_k;
-          // V_j once P_{j-1} V_{j-1} has read V_{j-1}
-          if (j > 0 && !(ok = mbar_wait_bounded(&bar[B_VE], (j - 1) & 1, limit_ns, status, DEV_TIMEOUT_PRODUCER))) break;
-          mbar_arrive_expect_tx(&bar[B_VF], 16384);
-          tma_load_2d(sm + FA_SV, &tm_qkv, &bar[B_VF], (2 * H + h) * 64, s0 + j * 128);
+          // V_j into ring slot j % VB once P_{j-VB} V_{j-VB} has read it
+          const int vb = j % FA_VB;
+          if (j >= FA_VB && !(ok = mbar_wait_bounded(&bar[B_VE0 + vb], (j / FA_VB - 1) & 1, limit_ns, status,
+                                                     DEV_TIMEOUT_PRODUCER)))
+            break;
+          mbar_arrive_expect_tx(&bar[B_VF0 + vb], 16384);
+          tma_load_2d(sm + FA_SV + vb * 16384, &tm_qkv, &bar[B_VF0 + vb], (2 * H + h) * 64, s0 + j * 128);
           ++issued_v;
         }
         // every issued load lands before the CTA exits
         mbar_wait_bounded(&bar[B_Q], 0, kDrainLimitNs, nullptr, 0);
-        for (int j = issued_k - 2 < 0 ? 0 : issued_k - 2; j < issued_k; ++j)
-          mbar_wait_bounded(&bar[B_KF0 + (j & 1)], (j >> 1) & 1, kDrainLimitNs, nullptr, 0);
-        if (issued_v) mbar_wait_bounded(&bar[B_VF], (issued_v - 1) & 1, kDrainLimitNs, nullptr, 0);
+        for (int j = issued_k - FA_KB < 0 ? 0 : issued_k - FA_KB; j < issued_k; ++j)
+          mbar_wait_bounded(&bar[B_KF0 + j % FA_KB], (j / FA_KB) & 1, kDrainLimitNs, nullptr, 0);
+        for (int j = issued_v - FA_VB < 0 ? 0 : issued_v - FA_VB; j < issued_v; ++j)
+          mbar_wait_bounded(&bar[B_VF0 + j % FA_VB], (j / FA_VB) & 1, kDrainLimitNs, nullptr, 0);
       }
     } else if (warp == 9) {
       // ------------------------------------------------ MMA issuer
@@ -127,14 +137,13 @@ __global__ void __launch_bounds__(FA_THREADS, 2) attention_fa_kernel(const __gri
         const uint32_t idesc_s = idesc_kind_f32(KIND, 128, 128);
         const uint32_t idesc_o = idesc_kind_f32(KIND, 128, 64) | (1u << 16);  // B = V, MN-major
         const uint64_t qd = sw128_kmajor_desc(smem_u32(sm + FA_SQ));
-        const uint64_t vd = sw128_mnmajor_desc(smem_u32(sm + FA_SV));
         auto issue_s = [&](int j) {
-          const uint64_t kd = sw128_kmajor_desc(smem_u32(sm + FA_SK + (j & 1) * 16384));
+          const uint64_t kd = sw128_kmajor_desc(smem_u32(sm + FA_SK + (j % FA_KB) * 16384));
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < 4; ++k) tc_mma_bf16(tmem, qd + 2 * k, kd + 2 * k, idesc_s, k > 0 ? 1u : 0u);
           tc_commit(&bar[B_SF]);
-          tc_commit(&bar[B_KE0 + (j & 1)]);
+          tc_commit(&bar[B_KE0 + j % FA_KB]);
         };
         bool ok = mbar_wait_bounded(&bar[B_Q], 0, limit_ns, status, DEV_TIMEOUT_MMA) &&
                   mbar_wait_bounded(&bar[B_KF0], 0, limit_ns, status, DEV_TIMEOUT_MMA);
@@ -142,15 +151,16 @@ __global__ void __launch_bounds__(FA_THREADS, 2) attention_fa_kernel(const __gri
         for (int j = 0; j < nk && ok; ++j) {
           if (j + 1 < nk) {
             // S for the next tile once its K has landed and the softmax has read S_j
-            ok = mbar_wait_bounded(&bar[B_KF0 + ((j + 1) & 1)], ((j + 1) >> 1) & 1, limit_ns, status, DEV_TIMEOUT_MMA) &&
+            ok = mbar_wait_bounded(&bar[B_KF0 + (j + 1) % FA_KB], ((j + 1) / FA_KB) & 1, limit_ns, status, DEV_TIMEOUT_MMA) &&
                  mbar_wait_bounded(&bar[B_SFREE], j & 1, limit_ns, status, DEV_TIMEOUT_MMA);
             if (!ok) break;
             issue_s(j + 1);
           }
           ok = mbar_wait_bounded(&bar[B_PF], j & 1, limit_ns, status, DEV_TIMEOUT_MMA) &&
-               mbar_wait_bounded(&bar[B_VF], j & 1, limit_ns, status, DEV_TIMEOUT_MMA);
+               mbar_wait_bounded(&bar[B_VF0 + j % FA_VB], (j / FA_VB) & 1, limit_ns, status, DEV_TIMEOUT_MMA);
           if (!ok) break;
           tc_fence_after();
+          const uint64_t vd = sw128_mnmajor_desc(smem_u32(sm + FA_SV + (j % FA_VB) * 16384));
 #pragma unroll
           for (int kb = 0; kb < 2; ++kb) {
             const uint64_t pd = sw128_kmajor_desc(smem_u32(sm + FA_SP + kb * 16384));
@@ -160,7 +170,7 @@ __global__ void __launch_bounds__(FA_THREADS, 2) attention_fa_kernel(const __gri
                           (j > 0 || kb > 0 || k > 0) ? 1u : 0u);
           }
           tc_commit(&bar[B_OD]);
-          tc_commit(&bar[B_VE]);
+          tc_commit(&bar[B_VE0 + j % FA_VB]);
         }
         // all issued MMAs complete before tensor memory is released
         tc_commit(&bar[B_DRAIN]);
