@@ -224,6 +224,23 @@ enum { ASR_TAP_MEL = 0, ASR_TAP_STEM = 1, ASR_TAP_LAYER0 = 2, ASR_TAP_ENCODER = 
 asr_status asr_enc_set_taps(asr_enc* e, unsigned mask);
 asr_status asr_enc_tap(asr_enc* e, int stage, float* dst, size_t dst_bytes, void* stream);
 
+/* ---- CUDA-graph replay -------------------------------------------------------
+ * A uniform forward (asr_enc_forward / asr_enc_forward_host) is recorded as a
+ * CUDA graph on the encoder's own stream the first time a given set of
+ * (pcm, out, workspace) pointers, n_samples, batch and tap mask is seen, and
+ * the graph is launched on the caller's stream then and on every later call
+ * with the same set (one launch instead of one per kernel; results are
+ * bit-identical to the direct launches).  A new set records a new graph and
+ * drops the old one.  Variable-length batches, profiling, and a caller whose
+ * stream is itself being captured launch the kernels directly.  If recording
+ * fails the encoder falls back to direct launches for good.  The data behind
+ * the pointers may change between calls; the pointers may not be freed while
+ * the encoder may still replay a graph that uses them (a later call with other
+ * pointers, asr_enc_set_graphs(e, 0) or asr_enc_destroy releases it).
+ * asr_enc_set_graphs(e, 0) turns recording off (and drops the graph); 1 turns
+ * it back on.  Default: on. */
+asr_status asr_enc_set_graphs(asr_enc* e, int enable);
+
 /* ---- kernel timing (profiling) --------------------------------------------
  * asr_enc_profile(e, 1) makes every later forward bracket each of its kernel
  * launches with CUDA events on the forward's stream (small extra cost; do not

@@ -83,6 +83,7 @@ def _load():
         "asr_enc_tap": (I, [P, I, P, SZ, P]),
         "asr_enc_last_error": (ctypes.c_char_p, [P]),
         "asr_enc_profile": (I, [P, I]),
+        "asr_enc_set_graphs": (I, [P, I]),
         "asr_enc_profile_read": (I, [P, I, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_double),
                                      ctypes.POINTER(I)]),
         "asr_enc_last_launches": (I, [P]),
@@ -334,6 +335,10 @@ class Encoder:
 
     def sync_status(self):
         _check(lib.asr_enc_sync_status(self.handle), self.handle)
+
+    def set_graphs(self, enable: bool):
+        """Record uniform forwards as CUDA graphs and replay them (default on)."""
+        _check(lib.asr_enc_set_graphs(self.handle, 1 if enable else 0), self.handle)
 
     def set_taps(self, mask: int):
         _check(lib.asr_enc_set_taps(self.handle, int(mask)), self.handle)

@@ -262,6 +262,25 @@ struct asr_enc {
   int* status = nullptr;
   unsigned taps = 0;
   cudaStream_t last_stream = nullptr;
+  // The last uniform forward recorded as a CUDA graph (keyed on its
+  // pointers and shape) and replayed while the key matches: one launch
+  // instead of ~240, programmatic (PDL) edges kept.  `graphs` off after a
+  // failed capture or by asr_enc_set_graphs.
+  struct GraphKey {
+    const float* pcm = nullptr;
+    float* out = nullptr;
+    void* ws = nullptr;
+    int64_t n = 0;
+    int B = 0;
+    unsigned taps = 0;
+    bool operator==(const GraphKey& o) const {
+      return pcm == o.pcm && out == o.out && ws == o.ws && n == o.n && B == o.B && taps == o.taps;
+    }
+  } gkey;
+  cudaGraphExec_t gexec = nullptr;
+  int glaunches = 0;
+  cudaStream_t cap_st = nullptr;
+  bool graphs = true;
   bool have_last = false;
   Plan last_plan;
   void* last_ws = nullptr;
@@ -433,6 +452,8 @@ const char* asr_enc_last_error(const asr_enc* e) {
 
 void asr_enc_destroy(asr_enc* e) {
   if (!e) return;
+  if (e->gexec) cudaGraphExecDestroy(e->gexec);
+  if (e->cap_st) cudaStreamDestroy(e->cap_st);
   for (cudaEvent_t ev : e->ev_pool) cudaEventDestroy(ev);
   if (e->slab) {
     if (e->free_fn)
@@ -1186,12 +1207,63 @@ void report_tokens(const Plan& p, const asr_geometry* g, int64_t n, const int64_
   }
 }
 
+// A uniform forward through the graph cache: replay when the pointers and
+// shape match the recorded forward, else record it (stream capture on the
+// encoder's own stream) and launch the new graph on `st`.  Variable-length
+// batches, profiling and a failed capture take the direct path.
+asr_status run_forward_cached(asr_enc* e, const float* pcm, const Plan& p, float* out, char* ws, cudaStream_t st) {
+  // a caller recording its own graph on `st` records the kernels directly
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) {
+    (void)cudaGetLastError();
+    cs = cudaStreamCaptureStatusActive;
+  }
+  if (!e->graphs || e->prof || p.varlen || cs != cudaStreamCaptureStatusNone) return run_forward(e, pcm, p, out, ws, st);
+  asr_enc::GraphKey key;
+  key.pcm = pcm;
+  key.out = out;
+  key.ws = ws;
+  key.n = p.n;
+  key.B = p.B;
+  key.taps = e->taps;
+  if (!e->gexec || !(key == e->gkey)) {
+    if (e->gexec) {
+      cudaGraphExecDestroy(e->gexec);
+      e->gexec = nullptr;
+    }
+    if (!e->cap_st && cudaStreamCreateWithFlags(&e->cap_st, cudaStreamNonBlocking) != cudaSuccess) {
+      e->cap_st = nullptr;
+      e->graphs = false;
+      (void)cudaGetLastError();
+      return run_forward(e, pcm, p, out, ws, st);
+    }
+    cudaGraph_t graph = nullptr;
+    bool ok = cudaStreamBeginCapture(e->cap_st, cudaStreamCaptureModeThreadLocal) == cudaSuccess;
+    const asr_status r = ok ? run_forward(e, pcm, p, out, ws, e->cap_st) : ASR_E_CUDA;
+    if (ok) ok = cudaStreamEndCapture(e->cap_st, &graph) == cudaSuccess && r == ASR_OK;
+    if (ok) ok = cudaGraphInstantiate(&e->gexec, graph, 0) == cudaSuccess;
+    if (graph) cudaGraphDestroy(graph);
+    if (!ok) {
+      if (e->gexec) cudaGraphExecDestroy(e->gexec);
+      e->gexec = nullptr;
+      e->graphs = false;
+      (void)cudaGetLastError();
+      return run_forward(e, pcm, p, out, ws, st);
+    }
+    e->gkey = key;
+    e->glaunches = e->launches;
+  }
+  ASR_CUDA(e, cudaGraphLaunch(e->gexec, st));
+  e->launches = e->glaunches;
+  return ASR_OK;
+}
+
 asr_status forward_common(asr_enc* e, const float* pcm, const int64_t* ns, int64_t n, int B, float* out,
                           int64_t* out_tokens, void* workspace, size_t ws_bytes, void* stream) {
   Plan p;
   ASR_TRY(check_forward_args(e, ns, n, B, pcm, out, workspace, ws_bytes, &p));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  ASR_TRY(run_forward(e, pcm, p, out, static_cast<char*>(workspace), st));
+  ASR_TRY(run_forward_cached(e, pcm, p, out, static_cast<char*>(workspace), st));
   e->last_stream = st;
   e->have_last = true;
   e->last_plan = p;
@@ -1210,7 +1282,7 @@ asr_status forward_host_common(asr_enc* e, const float* pcm_host, const int64_t*
   ASR_CUDA(e, cudaMemcpyAsync(dpcm, pcm_host, (size_t)p.n_total * 4, cudaMemcpyHostToDevice, st));
   const size_t out_bytes = (size_t)p.T * d_out(&e->g) * 4;
   float* dout = reinterpret_cast<float*>(ws + p.off_out);
-  ASR_TRY(run_forward(e, dpcm, p, dout, ws, st));
+  ASR_TRY(run_forward_cached(e, dpcm, p, dout, ws, st));
   ASR_CUDA(e, cudaMemcpyAsync(out_host, dout, out_bytes, cudaMemcpyDeviceToHost, st));
   e->last_stream = st;
   e->have_last = true;
@@ -1285,6 +1357,16 @@ asr_status asr_enc_tap(asr_enc* e, int stage, float* dst, size_t dst_bytes, void
   if (!dst || dst_bytes < bytes) return fail(e, ASR_E_INVAL, "tap needs %zu bytes", bytes);
   ASR_CUDA(e, cudaMemcpyAsync(dst, static_cast<char*>(e->last_ws) + e->last_plan.off_tap[stage], bytes,
                               cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream)));
+  return ASR_OK;
+}
+
+asr_status asr_enc_set_graphs(asr_enc* e, int enable) {
+  if (!e) return fail(nullptr, ASR_E_INVAL, "handle is NULL");
+  e->graphs = enable != 0;
+  if (!e->graphs && e->gexec) {
+    cudaGraphExecDestroy(e->gexec);
+    e->gexec = nullptr;
+  }
   return ASR_OK;
 }
 
