@@ -68,7 +68,7 @@ struct Plan {
   int n_groups = 0;
   size_t off_clipmax = 0, off_cu = 0, off_mel = 0, off_a1 = 0, off_c1 = 0, off_c2 = 0, off_c3 = 0, off_melT = 0, off_x = 0,
          off_h = 0, off_qkv = 0, off_att = 0, off_ff = 0, off_p1 = 0, off_p2 = 0, off_gu = 0, off_pcm = 0, off_out = 0,
-         off_mclips = 0, off_chunkd = 0, off_xpad = 0;
+         off_mclips = 0, off_chunkd = 0, off_xpad = 0, off_skflags = 0;
   size_t off_tap[ASR_TAP_COUNT] = {0, 0, 0, 0, 0};
   size_t tap_bytes[ASR_TAP_COUNT] = {0, 0, 0, 0, 0};
   size_t total = 0;
@@ -172,6 +172,11 @@ int64_t numel(const WSpec& w) {
 
 // Tokens of a chunk of L frames after three k3 s2 p1 convolutions.
 int64_t chunk_tokens(int64_t L) { return conv_len(conv_len(conv_len(L, 3, 2, 1), 3, 2, 1), 3, 2, 1); }
+
+// Stream-K flags of the residual GEMMs (one per CTA-pair slot, CTA and
+// epilogue warp); zeroed at the start of every forward, each cleared again by
+// the tile owner that consumed it.
+size_t sk_flags_bytes(const asr_enc* e);
 
 // Output rows of conv1 and conv2 (conv2d stem): [chunk][T][F] each, or in the
 // packed layout the four conv1 parity planes [plane][chunk][S2][F1 / 2] and
@@ -701,6 +706,8 @@ asr_status asr_enc_create(const asr_geometry* g, const void* const* weights, int
 
 namespace {
 
+size_t sk_flags_bytes(const asr_enc* e) { return ((size_t)e->num_sms * 8 * 4 + 255) / 256 * 256; }
+
 bool make_plan(const asr_enc* e, int64_t n, int B, Plan* p) {
   const size_t es = e->es;  // activation element size
   const asr_geometry* g = &e->g;
@@ -760,6 +767,7 @@ bool make_plan(const asr_enc* e, int64_t n, int B, Plan* p) {
     if ((e->taps >> t) & 1u) p->off_tap[t] = take(p->tap_bytes[t]);
   p->off_pcm = take((size_t)B * n * 4);
   p->off_out = take((size_t)p->T * d_out(g) * 4);
+  p->off_skflags = take(sk_flags_bytes(e));
   p->total = align_up(off, 1024);
   return true;
 }
@@ -854,6 +862,7 @@ bool make_plan_varlen(const asr_enc* e, const int64_t* ns, int B, Plan* p, const
     if (((e->taps >> t) & 1u) && p->tap_bytes[t]) p->off_tap[t] = take(p->tap_bytes[t]);
   p->off_pcm = take((size_t)p->n_total * 4);
   p->off_out = take((size_t)p->T * d_out(g) * 4);
+  p->off_skflags = take(sk_flags_bytes(e));
   p->total = align_up(off, 1024);
   return true;
 }
@@ -872,7 +881,8 @@ bool plan_for(const asr_enc* e, const int64_t* ns, int64_t n, int B, Plan* p) {
 
 asr_status gemm(asr_enc* e, const CUtensorMap* amap, const ConvGather* cg, const GemmB& w, long long M, void* out,
                 long long ldo, const float* bias, const float* pe, int period, int epi, cudaStream_t st,
-                const CUtensorMap* omap, const ConvBox* box = nullptr, int zero_period = 0, int zero_from = 0) {
+                const CUtensorMap* omap, const ConvBox* box = nullptr, int zero_period = 0, int zero_from = 0,
+                int* sk_flags = nullptr) {
   // fp32 operands: every output of the engine is fp32
   if (e->kind == KIND_TF32 && !(epi & (EPI_OUT_F32 | EPI_RESID))) epi |= EPI_OUT_F32;
   GemmParams p;
@@ -888,6 +898,7 @@ asr_status gemm(asr_enc* e, const CUtensorMap* amap, const ConvGather* cg, const
   p.limit_ns = kWaitLimitNs;
   p.zero_period = zero_period;
   p.zero_from = zero_from;
+  p.sk_flags = sk_flags;  // stream-K allowed (residual epilogue, the launcher decides)
   int bn;
   if (box) {
     p.conv_box = 1;
@@ -1021,6 +1032,8 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
   e->prof_recs.clear();
   ASR_LAUNCH(e, cudaMemsetAsync(e->status, 0, 4, st));
   ASR_LAUNCH(e, cudaMemsetAsync(clip_max, 0, (size_t)p.B * 4, st));
+  int* skf = reinterpret_cast<int*>(ws + p.off_skflags);
+  ASR_LAUNCH(e, cudaMemsetAsync(skf, 0, sk_flags_bytes(e), st));
   MelClip* mclips = reinterpret_cast<MelClip*>(ws + p.off_mclips);
   ChunkDesc* chunkd = reinterpret_cast<ChunkDesc*>(ws + p.off_chunkd);
   if (!p.varlen) {
@@ -1132,10 +1145,12 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
     else
       ASR_K(PC_ATTN, ASR_LAUNCH(e, launch_attention_fa(e->maps.qkv, cu, p.nwin, p.max_win, g->n_heads, att, e->status,
                                                        kWaitLimitNs, f16, st)));
-    ASR_K(PC_GEMM_O, ASR_TRY(gemm(e, &e->maps.att, nullptr, lw.o, p.T, x, d, lw.bo, nullptr, 1, EPI_RESID, st, &e->maps.o_x)));
+    ASR_K(PC_GEMM_O, ASR_TRY(gemm(e, &e->maps.att, nullptr, lw.o, p.T, x, d, lw.bo, nullptr, 1, EPI_RESID, st, &e->maps.o_x,
+                                  nullptr, 0, 0, skf)));
     ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, lw.ln2g, lw.ln2b, p.T, d, g->ln_eps, h, e->kind, st)));
     ASR_K(PC_GEMM_FC1, ASR_TRY(gemm(e, &e->maps.h, nullptr, lw.fc1, p.T, ff, g->d_ffn, lw.b1, nullptr, 1, EPI_GELU, st, &e->maps.o_ff)));
-    ASR_K(PC_GEMM_FC2, ASR_TRY(gemm(e, &e->maps.ff, nullptr, lw.fc2, p.T, x, d, lw.b2, nullptr, 1, EPI_RESID, st, &e->maps.o_x)));
+    ASR_K(PC_GEMM_FC2, ASR_TRY(gemm(e, &e->maps.ff, nullptr, lw.fc2, p.T, x, d, lw.b2, nullptr, 1, EPI_RESID, st, &e->maps.o_x,
+                                    nullptr, 0, 0, skf)));
     if (l == 0)
       if (float* t = tap(ASR_TAP_LAYER0)) ASR_LAUNCH(e, cudaMemcpyAsync(t, x, (size_t)p.T * d * 4, cudaMemcpyDeviceToDevice, st));
   }

@@ -162,6 +162,11 @@ cudaError_t run2_240(int epi, const CUtensorMap& a, const CUtensorMap& b, const 
 // into 74 clusters of two, and stream-K needs every pair of its grid
 // resident (an owner waits for the next pair's first piece).  Queried once
 // per device for the largest pair configuration (one CTA per SM).
+// Stream-K only from 40 k-blocks: in the 16 x 30 s forward it takes fc2
+// (80 k-blocks) from 2.45 to 2.39 ms per step, and at 20 it would also take
+// the out-projection, which it slows (1.00 to 1.10 ms).
+constexpr int kStreamKMinKBlocks = 40;
+
 int resident_pairs(int num_sms) {
   static std::mutex mu;
   static int cache[64] = {0};
@@ -381,7 +386,7 @@ cudaError_t launch16(const CUtensorMap* a_map, const GemmB& w, GemmParams p, int
     // (>= 40 k-blocks) for a split piece to outlast an epilogue (about 3 us):
     // with short K the extra epilogues of the split tiles cost more than the
     // balanced last wave saves.
-    p.sk = (p.sk_flags && epi == EPI_RESID && !p.conv_box && p.k_blocks >= 40 && p.num_tiles > pairs &&
+    p.sk = (p.sk_flags && epi == EPI_RESID && !p.conv_box && p.k_blocks >= kStreamKMinKBlocks && p.num_tiles > pairs &&
             p.num_tiles % pairs != 0)
                ? 1
                : 0;

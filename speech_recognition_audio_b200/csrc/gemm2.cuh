@@ -329,6 +329,9 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap& tmA, const CUte
         if (lane == 0) {
           have = flag_wait_bounded(flag, p.limit_ns, p.status, DEV_TIMEOUT_EPILOGUE);
           fence_proxy_async_global();  // the bulk reduces below come after the trailing piece's
+          // one split per flag and launch: clear it for the next launch (which
+          // starts after this grid has completed)
+          if (have) *flag = 0;
         }
         have = __shfl_sync(0xffffffffu, have, 0);
       }
