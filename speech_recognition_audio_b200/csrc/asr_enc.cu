@@ -50,6 +50,25 @@ struct ActMaps {
   // Store maps of the GEMM outputs (32 x 32 boxes): residual stream, QKV,
   // FFN hidden, head, adapter hidden, conv outputs.
   CUtensorMap o_x, o_qkv, o_ff, o_p1, o_p2, o_c2, o_c3, o_c1;
+  // 3-D companions of the plain activation maps (boxes of 128 rows x two
+  // 64-column k-blocks, 16-bit kinds with K a multiple of 128): with one, the
+  // CTA-pair GEMM loads two k-blocks of A per TMA copy.
+  static constexpr int kMax3 = 8;
+  const CUtensorMap* src3[kMax3] = {};
+  CUtensorMap map3[kMax3];
+  int n3 = 0;
+  bool add3(const CUtensorMap* m2, const void* ptr, unsigned long long rows, unsigned long long cols, int kind) {
+    if (n3 >= kMax3) return false;
+    if (kind == KIND_TF32 || cols % 128) return true;  // no companion: the 2-D path
+    if (!make_tmap_3d16(&map3[n3], ptr, rows, cols, cols, 128, kind)) return false;
+    src3[n3++] = m2;
+    return true;
+  }
+  const CUtensorMap* companion3(const CUtensorMap* m2) const {
+    for (int i = 0; i < n3; ++i)
+      if (src3[i] == m2) return &map3[i];
+    return nullptr;
+  }
 };
 
 struct Plan {
@@ -900,6 +919,7 @@ asr_status gemm(asr_enc* e, const CUtensorMap* amap, const ConvGather* cg, const
   p.zero_from = zero_from;
   p.sk_flags = sk_flags;  // stream-K allowed (residual epilogue, the launcher decides)
   int bn;
+  const CUtensorMap* amap3 = box ? nullptr : e->maps.companion3(amap);
   if (box) {
     p.conv_box = 1;
     p.cb = *box;
@@ -909,7 +929,7 @@ asr_status gemm(asr_enc* e, const CUtensorMap* amap, const ConvGather* cg, const
     bn = e->kind == KIND_TF32 ? gemm_pick_bn_tf32((int)M, w.N, e->num_sms)
                               : gemm_pick_bn((int)M, w.N, e->num_sms, cg != nullptr);
   }
-  cudaError_t r = launch_gemm(amap, w, p, epi, bn, e->num_sms, st, omap);
+  cudaError_t r = launch_gemm(amap, w, p, epi, bn, e->num_sms, st, omap, amap3);
   if (r != cudaSuccess) return fail(e, ASR_E_CUDA, "gemm launch (N=%d K=%d M=%lld epi=%d bn=%d): %s", w.N, w.K, M, epi, bn, cudaGetErrorString(r));
   return ASR_OK;
 }
@@ -997,6 +1017,15 @@ asr_status ensure_maps(asr_enc* e, const Plan& p, char* ws) {
   else if (ok)
     ok = make_tmap_out(&m.o_c1, ws + p.off_c1, (unsigned long long)p.B * p.F, d, d, f32);
   if (ok && g->adapter_hidden) ok = make_tmap_act(k, &m.gu, ws + p.off_gu, p.T, g->adapter_hidden, g->adapter_hidden, 128);
+  m.n3 = 0;
+  if (ok)
+    ok = m.add3(&m.h, ws + p.off_h, p.T, d, k) && m.add3(&m.att, ws + p.off_att, p.T, d, k) &&
+         m.add3(&m.ff, ws + p.off_ff, p.T, g->d_ffn, k);
+  if (ok && g->stem == ASR_STEM_CONV2D_CHUNKED)
+    ok = m.add3(&m.c3, ws + p.off_c3, p.Tpad, (unsigned long long)p.F3 * g->conv_ch, k);
+  if (ok && g->proj1_out)
+    ok = m.add3(&m.p1, ws + p.off_p1, p.T, g->proj1_out, k) && m.add3(&m.p2, ws + p.off_p2, p.T, g->proj2_out, k);
+  if (ok && g->adapter_hidden) ok = m.add3(&m.gu, ws + p.off_gu, p.T, g->adapter_hidden, k);
   if (!ok) {
     m.ws = nullptr;
     return fail(e, ASR_E_CUDA, "TMA descriptor encoding failed (workspace alignment?)");
@@ -1498,10 +1527,11 @@ asr_status asr_op_linear(const void* x, const void* w, const float* bias, int64_
     return fail(nullptr, ASR_E_INVAL, "linear: tile_n must be 0, 256, 160, 128, 64, -256 or -128");
   if (tile_n == 160 && N % 160) return fail(nullptr, ASR_E_INVAL, "linear: tile_n 160 needs N %% 160 == 0");
   const int bn = tile_n ? tile_n : gemm_pick_bn((int)M, N, sms, false);
-  CUtensorMap omap;
+  CUtensorMap omap, amap3;
   const bool f32_out = (e_bits & (EPI_OUT_F32 | EPI_RESID)) != 0;
   const bool have_omap = !(e_bits & EPI_SWIGLU) && make_tmap_out(&omap, y, M, N, N, f32_out);
-  ASR_CUDA(nullptr, launch_gemm(&amap, wb, p, e_bits, bn, sms, st, have_omap ? &omap : nullptr));
+  const bool have_a3 = K % 128 == 0 && make_tmap_3d16(&amap3, x, M, K, K, 128, KIND_BF16);
+  ASR_CUDA(nullptr, launch_gemm(&amap, wb, p, e_bits, bn, sms, st, have_omap ? &omap : nullptr, have_a3 ? &amap3 : nullptr));
   return ASR_OK;
 }
 

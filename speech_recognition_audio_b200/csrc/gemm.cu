@@ -106,14 +106,16 @@ cudaError_t run_gather(int epi, const CUtensorMap& b, const CUtensorMap& o, cons
   }
 }
 
-template <int BN, int EPI, int KIND>
+// KP = 2: stages of two k-blocks (3-D maps), three of them in the same
+// shared memory as six single-k-block stages.
+template <int BN, int EPI, int KIND, int KP = 1>
 cudaError_t run2(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& p, int grid, cudaStream_t st) {
-  using S = Gemm2Shape<BN, 6, gemm2_epi_warps<EPI>(), gemm2_nbuf<BN>()>;
+  using S = Gemm2Shape<BN, KP == 2 ? 3 : 6, gemm2_epi_warps<EPI>(), gemm2_nbuf<BN>(), KP>;
   void (*k)(CUtensorMap, CUtensorMap, CUtensorMap, GemmParams);
   if constexpr (KIND == KIND_F16)
-    k = gemm_f16_tc2_kernel<BN, S::STAGES, EPI>;
+    k = gemm_f16_tc2_kernel<BN, S::STAGES, EPI, KP>;
   else
-    k = gemm_bf16_tc2_kernel<BN, S::STAGES, EPI>;
+    k = gemm_bf16_tc2_kernel<BN, S::STAGES, EPI, KP>;
   cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_BYTES);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
@@ -144,6 +146,20 @@ cudaError_t run2_epi(int epi, const CUtensorMap& a, const CUtensorMap& b, const 
     case EPI_OUT_F32 | EPI_PE: return run2<BN, EPI_OUT_F32 | EPI_PE, KIND>(a, b, o, p, grid, st);
     case EPI_SWIGLU: return run2<BN, EPI_SWIGLU, KIND>(a, b, o, p, grid, st);
     case EPI_GELU | EPI_OUT_F32 | EPI_PE: return run2<BN, EPI_GELU | EPI_OUT_F32 | EPI_PE, KIND>(a, b, o, p, grid, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+// 256-wide pair tiles with two-k-block stages (plain A, K % 128 == 0).
+template <int KIND>
+cudaError_t run2_kp2(int epi, const CUtensorMap& a3, const CUtensorMap& b3, const CUtensorMap& o, const GemmParams& p,
+                     int grid, cudaStream_t st) {
+  switch (epi) {
+    case 0: return run2<256, 0, KIND, 2>(a3, b3, o, p, grid, st);
+    case EPI_GELU: return run2<256, EPI_GELU, KIND, 2>(a3, b3, o, p, grid, st);
+    case EPI_OUT_F32: return run2<256, EPI_OUT_F32, KIND, 2>(a3, b3, o, p, grid, st);
+    case EPI_RESID: return run2<256, EPI_RESID, KIND, 2>(a3, b3, o, p, grid, st);
+    case EPI_OUT_F32 | EPI_PE: return run2<256, EPI_OUT_F32 | EPI_PE, KIND, 2>(a3, b3, o, p, grid, st);
+    case EPI_SWIGLU: return run2<256, EPI_SWIGLU, KIND, 2>(a3, b3, o, p, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -291,7 +307,23 @@ bool make_tmap_act(int kind, CUtensorMap* map, const void* ptr, unsigned long lo
                            : make_tmap_bf16(map, ptr, rows, cols, row_stride_elems, box_rows);
 }
 
+bool make_tmap_3d16(CUtensorMap* map, const void* ptr, unsigned long long rows, unsigned long long cols,
+                    unsigned long long row_stride_elems, unsigned int box_rows, int kind) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || !ptr || kind == KIND_TF32 || (reinterpret_cast<uintptr_t>(ptr) & 15) || (row_stride_elems * 2) % 16 ||
+      rows == 0 || cols % 128 || box_rows == 0 || box_rows > 256)
+    return false;
+  cuuint64_t dims[3] = {64, rows, cols / 64};
+  cuuint64_t strides[2] = {row_stride_elems * 2, 128};
+  cuuint32_t box[3] = {64, box_rows, 2};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(map, kind == KIND_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+            const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_weight_maps(GemmB& w) {
+  w.has3 = w.kind != KIND_TF32 && w.K % 128 == 0 && make_tmap_3d16(&w.map3, w.ptr, w.N, w.K, w.K, 128, w.kind);
   for (int i = 0; i < kGemmSlots; ++i)
     if (!make_tmap_act(w.kind, &w.map[i], w.ptr, w.N, w.K, w.K, kSlotRows[i])) return false;
   return true;
@@ -355,7 +387,7 @@ int gemm_pick_bn_conv(int n_sub, int N, int num_sms) {
 
 template <int KIND>
 cudaError_t launch16(const CUtensorMap* a_map, const GemmB& w, GemmParams p, int epi, int bn, int num_sms,
-                     cudaStream_t st, const CUtensorMap* out_map) {
+                     cudaStream_t st, const CUtensorMap* out_map, const CUtensorMap* a_map3) {
   p.out_tma = (out_map != nullptr && !(epi & (EPI_PE | EPI_SWIGLU))) ? 1 : 0;
   // Whole four-step k-blocks everywhere when A and B both come by TMA: the
   // steps past K (or past a tap's channels) multiply the zeros that the TMA
@@ -377,7 +409,12 @@ cudaError_t launch16(const CUtensorMap* a_map, const GemmB& w, GemmParams p, int
     p.K = w.K;
     p.m_blocks = p.conv_box ? (p.cb.n_sub + 1) / 2 : (p.M + 255) / 256;
     p.n_blocks = (p.N + w2 - 1) / w2;
-    p.k_blocks = (p.K + 63) / 64;
+    // Two k-blocks per stage (3-D copies) for plain 256-wide tiles when the
+    // caller gave the 3-D map of A and K is a whole number of stages.
+    const bool kp2 = a_map3 && w.has3 && w2 == 256 && !p.conv_box && p.K % 128 == 0 &&
+                     (epi == 0 || epi == EPI_GELU || epi == EPI_OUT_F32 || epi == EPI_RESID ||
+                      epi == (EPI_OUT_F32 | EPI_PE) || epi == EPI_SWIGLU);
+    p.k_blocks = kp2 ? p.K / 128 : (p.K + 63) / 64;
     p.num_tiles = p.m_blocks * p.n_blocks;
     const int pairs = std::min(p.num_tiles, resident_pairs(num_sms));
     const int grid = 2 * pairs;
@@ -385,11 +422,13 @@ cudaError_t launch16(const CUtensorMap* a_map, const GemmB& w, GemmParams p, int
     // add, whole tiles would leave a ragged last wave, and K is long enough
     // (>= 40 k-blocks) for a split piece to outlast an epilogue (about 3 us):
     // with short K the extra epilogues of the split tiles cost more than the
-    // balanced last wave saves.
-    p.sk = (p.sk_flags && epi == EPI_RESID && !p.conv_box && p.k_blocks >= kStreamKMinKBlocks && p.num_tiles > pairs &&
-            p.num_tiles % pairs != 0)
+    // balanced last wave saves.  (Its units are stages.)
+    p.sk = (p.sk_flags && epi == EPI_RESID && !p.conv_box && (p.K + 63) / 64 >= kStreamKMinKBlocks &&
+            p.num_tiles > pairs && p.num_tiles % pairs != 0)
                ? 1
                : 0;
+    if (kp2)
+      return run2_kp2<KIND>(epi, *a_map3, w.map3, p.out_tma ? *out_map : w.map3, p, grid, st);
     if (w2 == 240) return run2_240<KIND>(epi, *a_map, w.map[slot2], p.out_tma ? *out_map : w.map[slot2], p, grid, st);
     const CUtensorMap& o2 = p.out_tma ? *out_map : w.map[slot2];
     return w2 == 256 ? run2_epi<256, KIND>(epi, *a_map, w.map[slot2], o2, p, grid, st)
@@ -428,9 +467,9 @@ cudaError_t launch16(const CUtensorMap* a_map, const GemmB& w, GemmParams p, int
 }
 
 cudaError_t launch_gemm(const CUtensorMap* a_map, const GemmB& w, GemmParams p, int epi, int bn, int num_sms,
-                        cudaStream_t st, const CUtensorMap* out_map) {
-  if (w.kind == KIND_BF16) return launch16<KIND_BF16>(a_map, w, p, epi, bn, num_sms, st, out_map);
-  if (w.kind == KIND_F16) return launch16<KIND_F16>(a_map, w, p, epi, bn, num_sms, st, out_map);
+                        cudaStream_t st, const CUtensorMap* out_map, const CUtensorMap* a_map3) {
+  if (w.kind == KIND_BF16) return launch16<KIND_BF16>(a_map, w, p, epi, bn, num_sms, st, out_map, a_map3);
+  if (w.kind == KIND_F16) return launch16<KIND_F16>(a_map, w, p, epi, bn, num_sms, st, out_map, a_map3);
   // fp32 operands: one-SM tiles only (the CTA-pair kernel takes 16-bit
   // operands), no gather mode
   p.out_tma = (out_map != nullptr && !(epi & (EPI_PE | EPI_SWIGLU))) ? 1 : 0;

@@ -61,6 +61,17 @@ __device__ __forceinline__ void tma_load_4d_pair(void* dst, const CUtensorMap* m
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
 }
+// 3-D box {64 elements, rows, 2 k-blocks} of a [rows][K] matrix viewed as
+// {64, rows, K / 64}: two 64-element k-blocks of `rows` rows in one copy,
+// landing as two consecutive canonical 128-byte-row tiles.
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster_addr, int c0,
+                                                 int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
+      "[%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
                "r"(ncols)
@@ -108,11 +119,15 @@ __device__ __forceinline__ void tc_commit_pair_mc(uint64_t* bar, uint16_t mask) 
 // staging box takes 2 KB); NBUF_: staging buffers per epilogue warp, used in
 // turn (two let a warp fill the next box while the previous TMA store still
 // reads its buffer).  The staging area is 32 KB per buffer.
-template <int BN_, int STAGES_, int EPIW_ = 8, int NBUF_ = 1>
+// KP_: 64-element k-blocks per pipeline stage.  With 2 each operand's stage
+// comes in one 3-D copy (the per-copy cost of the TMA, not its bytes, bounds
+// 128-row boxes: 0.27 us per k-block with one copy per k-block and operand,
+// 0.19 us with one per two, measured without MMAs).
+template <int BN_, int STAGES_, int EPIW_ = 8, int NBUF_ = 1, int KP_ = 1>
 struct Gemm2Shape {
-  static constexpr int BM = 256, BN = BN_, BK = 64, STAGES = STAGES_;
-  static constexpr int A_BYTES = 128 * BK * 2;        // this CTA's half of A
-  static constexpr int B_BYTES = (BN / 2) * BK * 2;   // this CTA's half of B
+  static constexpr int BM = 256, BN = BN_, BK = 64, STAGES = STAGES_, KP = KP_;
+  static constexpr int A_BYTES = 128 * BK * 2 * KP;        // this CTA's half of A
+  static constexpr int B_BYTES = (BN / 2) * BK * 2 * KP;   // this CTA's half of B
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TX_BYTES = 2 * STAGE_BYTES;    // both CTAs, counted on the leader
   static constexpr int ACC_COLS = (BN + 31) / 32 * 32;
@@ -148,10 +163,11 @@ constexpr int gemm2_epi_warps() {
   return EPI == EPI_GELU ? 16 : 8;
 }
 
-template <int BN, int STAGES, int EPI, int KIND>
+template <int BN, int STAGES, int EPI, int KIND, int KP = 1>
 __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmOut,
                                               const GemmParams& p) {
-  using S = Gemm2Shape<BN, STAGES, gemm2_epi_warps<EPI>(), gemm2_nbuf<BN>()>;
+  // KP == 2: tmA / tmB are 3-D maps, p.k_blocks counts two-k-block stages
+  using S = Gemm2Shape<BN, STAGES, gemm2_epi_warps<EPI>(), gemm2_nbuf<BN>(), KP>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -221,14 +237,19 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap& tmA, const CUte
           }
           if (rank == 0) mbar_arrive_expect_tx(&full[s], S::TX_BYTES);
           const uint32_t fb = full_leader0 + 8u * s;
-          if (p.conv_box) {
-            int c0, f0, t0, img;
-            convbox_coords(p, u, kb, c0, f0, t0, img);
-            tma_load_4d_pair(sA + s * S::A_BYTES, &tmA, fb, c0, f0, t0, img);
+          if constexpr (KP == 2) {
+            tma_load_3d_pair(sA + s * S::A_BYTES, &tmA, fb, 0, m0, 2 * kb);
+            tma_load_3d_pair(sB + s * S::B_BYTES, &tmB, fb, 0, n0, 2 * kb);
           } else {
-            tma_load_2d_pair(sA + s * S::A_BYTES, &tmA, fb, kb * S::BK, m0);
+            if (p.conv_box) {
+              int c0, f0, t0, img;
+              convbox_coords(p, u, kb, c0, f0, t0, img);
+              tma_load_4d_pair(sA + s * S::A_BYTES, &tmA, fb, c0, f0, t0, img);
+            } else {
+              tma_load_2d_pair(sA + s * S::A_BYTES, &tmA, fb, kb * S::BK, m0);
+            }
+            tma_load_2d_pair(sB + s * S::B_BYTES, &tmB, fb, kb * S::BK, n0);
           }
-          tma_load_2d_pair(sB + s * S::B_BYTES, &tmB, fb, kb * S::BK, n0);
           ++it;
         }
       }
@@ -273,7 +294,11 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap& tmA, const CUte
             const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + s * S::A_BYTES));
             const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + s * S::B_BYTES));
             if (FULL) {
-              tc_mma4_bf16_pair(d_tmem, ad, bd, idesc, kb > kb0 ? 1u : 0u);
+              // k-block j of the stage: A tile at +16 KB j, B tile at +(BN/2) x 128 B j
+#pragma unroll
+              for (int j = 0; j < KP; ++j)
+                tc_mma4_bf16_pair(d_tmem, ad + (uint64_t)(j * (128 * 128 >> 4)), bd + (uint64_t)(j * ((BN / 2) * 128 >> 4)),
+                                  idesc, (kb > kb0 || j > 0) ? 1u : 0u);
             } else {
               const int ks = k16_steps(p, kb);
 #pragma unroll
@@ -359,17 +384,17 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap& tmA, const CUte
 }
 
 // bf16 and f16 operands (kind::f16), CTA pairs.
-template <int BN, int STAGES, int EPI>
-__global__ void __launch_bounds__(Gemm2Shape<BN, STAGES, gemm2_epi_warps<EPI>(), gemm2_nbuf<BN>()>::THREADS, 1)
+template <int BN, int STAGES, int EPI, int KP = 1>
+__global__ void __launch_bounds__(Gemm2Shape<BN, STAGES, gemm2_epi_warps<EPI>(), gemm2_nbuf<BN>(), KP>::THREADS, 1)
     gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
-  gemm_tc2_body<BN, STAGES, EPI, KIND_BF16>(tmA, tmB, tmOut, p);
+  gemm_tc2_body<BN, STAGES, EPI, KIND_BF16, KP>(tmA, tmB, tmOut, p);
 }
-template <int BN, int STAGES, int EPI>
-__global__ void __launch_bounds__(Gemm2Shape<BN, STAGES, gemm2_epi_warps<EPI>(), gemm2_nbuf<BN>()>::THREADS, 1)
+template <int BN, int STAGES, int EPI, int KP = 1>
+__global__ void __launch_bounds__(Gemm2Shape<BN, STAGES, gemm2_epi_warps<EPI>(), gemm2_nbuf<BN>(), KP>::THREADS, 1)
     gemm_f16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
-  gemm_tc2_body<BN, STAGES, EPI, KIND_F16>(tmA, tmB, tmOut, p);
+  gemm_tc2_body<BN, STAGES, EPI, KIND_F16, KP>(tmA, tmB, tmOut, p);
 }
 
 }  // namespace asr

@@ -153,7 +153,14 @@ struct GemmB {              // weight operand [N, K] (bf16, or fp32 for KIND_TF3
   int N = 0, K = 0;
   int kind = KIND_BF16;
   CUtensorMap map[kGemmSlots];  // box rows 256, 128, 240, 64, 160, 120 (index by gemm_bn_slot)
+  CUtensorMap map3;             // 3-D {64, N, K / 64} view, box {64, 128, 2} (16-bit kinds, K % 128 == 0)
+  bool has3 = false;
 };
+// 3-D view {64 elements, rows, cols / 64} of a row-major 16-bit [rows][cols]
+// matrix with a box of two 64-element k-blocks of box_rows rows (the A and B
+// stages of the CTA-pair kernel's two-k-block pipeline); cols % 128 == 0.
+bool make_tmap_3d16(CUtensorMap* map, const void* ptr, unsigned long long rows, unsigned long long cols,
+                    unsigned long long row_stride_elems, unsigned int box_rows, int kind);
 int gemm_bn_slot(int bn);
 bool make_tmap_bf16(CUtensorMap* map, const void* ptr, unsigned long long rows, unsigned long long cols,
                     unsigned long long row_stride_elems, unsigned int box_rows);
@@ -186,7 +193,9 @@ bool make_tmap_out(CUtensorMap* map, const void* ptr, unsigned long long rows, u
 // a_map: TMA map of A (box 128 x 64), or null with p.g set for the implicit-GEMM mode.
 // out_map: store map of the output (make_tmap_out), or null for plain stores;
 // ignored for the position and SwiGLU epilogues.
+// a_map3: 3-D map of A (make_tmap_3d16, box rows 128) or null; with it, plain
+// 256-wide CTA-pair launches run two k-blocks per pipeline stage.
 cudaError_t launch_gemm(const CUtensorMap* a_map, const GemmB& w, GemmParams p, int epi, int bn, int num_sms,
-                        cudaStream_t st, const CUtensorMap* out_map);
+                        cudaStream_t st, const CUtensorMap* out_map, const CUtensorMap* a_map3 = nullptr);
 
 }  // namespace asr
