@@ -241,6 +241,27 @@ asr_status asr_enc_tap(asr_enc* e, int stage, float* dst, size_t dst_bytes, void
  * it back on.  Default: on. */
 asr_status asr_enc_set_graphs(asr_enc* e, int enable);
 
+/* ---- LayerNorm epilogue ------------------------------------------------------
+ * With 16-bit weights whose shapes allow it (d_model and d_ffn multiples of
+ * 128, d_model a multiple of 32), the fc2 GEMM of every block also computes
+ * the LayerNorm that reads its residual update ("Audio encoder": pre-norm
+ * blocks, each sub-layer's input is the LayerNorm of the residual stream):
+ * the next block's first LayerNorm, or the head's LayerNorm after the last
+ * block when there is a projection head.  The GEMM's epilogue adds its tile
+ * to the fp32 residual stream, publishes the rows' partial mean / sum of
+ * squared deviations, waits (bounded) for the other tiles of the same rows,
+ * and writes the normalised 16-bit rows; the separate LayerNorm launch goes
+ * away.  (The attention out-projection keeps its separate LayerNorm: with
+ * K = d_model its mainloop is shorter than that epilogue.)  The residual
+ * stream is computed with the same additions as the unfused path; the
+ * LayerNorm outputs differ by the summation order of the statistics (well
+ * inside the encoder's tolerance), and so does everything downstream.
+ * asr_enc_set_ln_fusion(e, 0) turns it off (the separate LayerNorm kernels
+ * run instead; drops a recorded graph), 1 back on (default: on).
+ * asr_enc_ln_fusion reports whether forwards use it (*active = 1) or not. */
+asr_status asr_enc_set_ln_fusion(asr_enc* e, int enable);
+asr_status asr_enc_ln_fusion(const asr_enc* e, int* active);
+
 /* ---- kernel timing (profiling) --------------------------------------------
  * asr_enc_profile(e, 1) makes every later forward bracket each of its kernel
  * launches with CUDA events on the forward's stream (small extra cost; do not

@@ -85,6 +85,29 @@ size_t asr_op_linear_ws_size(void);
 asr_status asr_op_linear(const void* x, const void* w, const float* bias, int64_t M, int N, int K,
                          int epi, int tile_n, void* y, void* ws, size_t ws_bytes, void* stream);
 
+/* Residual dense layer and the LayerNorm of the updated rows in one launch
+ * of the CTA-pair engine (the epilogue of the encoder's out-projection and
+ * fc2; "Audio encoder": pre-norm blocks):
+ *   y[M, N] += X W^T + bias                                  (f32, in place)
+ *   h[M, N]  = (y - mean) / sqrt(var + eps) * gamma + beta   (bf16; mean and
+ *              biased variance over each updated row of y)
+ * The update of y is computed exactly as by ASR_EPI_F32_RESID (same adds in
+ * the same order); the statistics combine per-tile partial means and sums of
+ * squared deviations (Chan, Golub and LeVeque's pairwise update).
+ *  x bf16 [M, K] row-major;  w bf16 [N, K];  bias, gamma, beta f32 [N].
+ *  Limits: M >= 1, K % 128 == 0, N % 32 == 0, ceil(N / 256) <= the CTA pairs
+ *  the device can hold at once (74 on a B200), 16-byte aligned pointers.
+ *  ws: device scratch of at least asr_op_linear_resid_ln_ws_size(M, N)
+ *  bytes (status word, one counter per 32 rows, and per row two 16-byte
+ *  partial statistics per 256 columns); the call clears what it needs with
+ *  a memset on `stream`.  ASR_E_UNSUPPORTED when the shape is outside the
+ *  limits; a statistics wait that runs out (bounded, seconds) is reported by
+ *  the status word like the engine's other waits. */
+size_t asr_op_linear_resid_ln_ws_size(int64_t M, int N);
+asr_status asr_op_linear_resid_ln(const void* x, const void* w, const float* bias, const float* gamma,
+                                  const float* beta, float eps, int64_t M, int N, int K, float* y, void* h,
+                                  void* ws, size_t ws_bytes, void* stream);
+
 /* The same engine with fp32 operands multiplied as tf32 (tcgen05 kind::tf32:
  * the tensor cores read each fp32 operand's sign, exponent and top 10
  * mantissa bits) and fp32 accumulation; the path of geometries with fp32

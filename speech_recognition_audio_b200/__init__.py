@@ -84,6 +84,8 @@ def _load():
         "asr_enc_last_error": (ctypes.c_char_p, [P]),
         "asr_enc_profile": (I, [P, I]),
         "asr_enc_set_graphs": (I, [P, I]),
+        "asr_enc_set_ln_fusion": (I, [P, I]),
+        "asr_enc_ln_fusion": (I, [P, ctypes.POINTER(I)]),
         "asr_enc_profile_read": (I, [P, I, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_double),
                                      ctypes.POINTER(I)]),
         "asr_enc_last_launches": (I, [P]),
@@ -93,6 +95,8 @@ def _load():
         "asr_op_linear_ws_size": (SZ, []),
         "asr_op_linear": (I, [P, P, P, I64, I, I, I, I, P, P, SZ, P]),
         "asr_op_linear_tf32": (I, [P, P, P, I64, I, I, I, I, P, P, SZ, P]),
+        "asr_op_linear_resid_ln_ws_size": (SZ, [I64, I]),
+        "asr_op_linear_resid_ln": (I, [P, P, P, P, P, ctypes.c_float, I64, I, I, P, P, P, SZ, P]),
         "asr_op_layer_norm": (I, [P, P, P, I64, I, F, P, I, P]),
         "asr_op_attention_ws_size": (SZ, []),
         "asr_op_attention": (I, [P, P, I, I, I64, I, P, P, SZ, P]),
@@ -340,6 +344,16 @@ class Encoder:
         """Record uniform forwards as CUDA graphs and replay them (default on)."""
         _check(lib.asr_enc_set_graphs(self.handle, 1 if enable else 0), self.handle)
 
+    def set_ln_fusion(self, enable: bool):
+        """LayerNorms computed by the residual GEMMs' epilogues (default on where supported)."""
+        _check(lib.asr_enc_set_ln_fusion(self.handle, 1 if enable else 0), self.handle)
+
+    def ln_fusion(self) -> bool:
+        """Whether forwards compute the LayerNorms in the residual GEMMs' epilogues."""
+        v = ctypes.c_int(0)
+        _check(lib.asr_enc_ln_fusion(self.handle, ctypes.byref(v)), self.handle)
+        return bool(v.value)
+
     def set_taps(self, mask: int):
         _check(lib.asr_enc_set_taps(self.handle, int(mask)), self.handle)
         self.taps = int(mask)
@@ -382,6 +396,20 @@ def linear(x, w, bias=None, epi: int = EPI_BF16, out=None, tile_n: int = 0, stre
     _check(lib.asr_op_linear(_ptr(x), _ptr(w), _ptr(bias), M, N, K, epi, int(tile_n), _ptr(out), _ptr(ws),
                              ws.numel(), _stream(stream)))
     return out
+
+
+def linear_resid_ln(x, w, bias, gamma, beta, y, eps: float = 1e-5, h=None, stream=None):
+    """y f32 [M, N] += x w^T + bias (in place), then h bf16 [M, N] = LayerNorm(y) * gamma + beta, in one
+    launch (asr_op_linear_resid_ln).  Returns h."""
+    import torch
+    M, K = x.shape
+    N = w.shape[0]
+    if h is None:
+        h = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    ws = torch.empty(int(lib.asr_op_linear_resid_ln_ws_size(M, N)), dtype=torch.uint8, device=x.device)
+    _check(lib.asr_op_linear_resid_ln(_ptr(x), _ptr(w), _ptr(bias), _ptr(gamma), _ptr(beta), float(eps), M, N, K,
+                                      _ptr(y), _ptr(h), _ptr(ws), ws.numel(), _stream(stream)))
+    return h
 
 
 def linear_tf32(x, w, bias=None, epi: int = EPI_F32, out=None, tile_n: int = 0, stream=None):

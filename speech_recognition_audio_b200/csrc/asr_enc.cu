@@ -11,6 +11,7 @@
 // exports instead / Results): log-mel -> transpose -> conv1 (k3 s1) + GELU ->
 // conv2 (k3 s2) + GELU + global positions -> 12 layers with full attention
 // -> final LayerNorm.
+#include <climits>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -87,7 +88,7 @@ struct Plan {
   int n_groups = 0;
   size_t off_clipmax = 0, off_cu = 0, off_mel = 0, off_a1 = 0, off_c1 = 0, off_c2 = 0, off_c3 = 0, off_melT = 0, off_x = 0,
          off_h = 0, off_qkv = 0, off_att = 0, off_ff = 0, off_p1 = 0, off_p2 = 0, off_gu = 0, off_pcm = 0, off_out = 0,
-         off_mclips = 0, off_chunkd = 0, off_xpad = 0, off_skflags = 0;
+         off_mclips = 0, off_chunkd = 0, off_xpad = 0, off_skflags = 0, off_lncnt = 0, off_lnpart = 0;
   size_t off_tap[ASR_TAP_COUNT] = {0, 0, 0, 0, 0};
   size_t tap_bytes[ASR_TAP_COUNT] = {0, 0, 0, 0, 0};
   size_t total = 0;
@@ -196,6 +197,8 @@ int64_t chunk_tokens(int64_t L) { return conv_len(conv_len(conv_len(L, 3, 2, 1),
 // epilogue warp); zeroed at the start of every forward, each cleared again by
 // the tile owner that consumed it.
 size_t sk_flags_bytes(const asr_enc* e);
+size_t ln_count_bytes(int64_t T);
+int ln_parts(const asr_enc* e);
 
 // Output rows of conv1 and conv2 (conv2d stem): [chunk][T][F] each, or in the
 // packed layout the four conv1 parity planes [plane][chunk][S2][F1 / 2] and
@@ -277,6 +280,10 @@ struct asr_enc {
   // neighbour chunk's zero row as their padding and conv2 / conv3 tiles run
   // across chunk boundaries (no partly empty tiles).
   bool packed = false;
+  // fc2 of every block also writes the next LayerNorm's output (EPI_LN):
+  // possible for 16-bit weights of suitable shape (ln_fuse), on unless
+  // asr_enc_set_ln_fusion turned it off.
+  bool ln_fuse = false, ln_fuse_on = true;
   float* pe = nullptr;
   int pe_rows = 0;
   std::vector<LayerW> layers;
@@ -687,6 +694,8 @@ asr_status asr_enc_create(const asr_geometry* g, const void* const* weights, int
   }
   e->lnpg = up_f32(next());
   e->lnpb = up_f32(next());
+  e->ln_fuse = L > 0 && e->kind != KIND_TF32 && gemm_ln_supported(e->layers[0].o, e->num_sms) &&
+               gemm_ln_supported(e->layers[0].fc2, e->num_sms);
   if (g->proj1_out) {
     if (!gemm_w(e->p1, next(), g->proj1_out, d)) return cuda_fail("proj1 upload failed");
     e->bp1 = up_f32(next());
@@ -726,6 +735,10 @@ asr_status asr_enc_create(const asr_geometry* g, const void* const* weights, int
 namespace {
 
 size_t sk_flags_bytes(const asr_enc* e) { return ((size_t)e->num_sms * 8 * 4 + 255) / 256 * 256; }
+// LayerNorm epilogue: one arrival counter per 32 rows, and per row two
+// partial statistics (16 bytes each) per 256-column n-tile.
+size_t ln_count_bytes(int64_t T) { return ((size_t)(T + 31) / 32 * 4 + 255) / 256 * 256; }
+int ln_parts(const asr_enc* e) { return 2 * ((e->g.d_model + 255) / 256); }
 
 bool make_plan(const asr_enc* e, int64_t n, int B, Plan* p) {
   const size_t es = e->es;  // activation element size
@@ -787,6 +800,10 @@ bool make_plan(const asr_enc* e, int64_t n, int B, Plan* p) {
   p->off_pcm = take((size_t)B * n * 4);
   p->off_out = take((size_t)p->T * d_out(g) * 4);
   p->off_skflags = take(sk_flags_bytes(e));
+  if (e->ln_fuse) {
+    p->off_lncnt = take(ln_count_bytes(p->T));
+    p->off_lnpart = take((size_t)p->T * ln_parts(e) * 16);
+  }
   p->total = align_up(off, 1024);
   return true;
 }
@@ -882,6 +899,10 @@ bool make_plan_varlen(const asr_enc* e, const int64_t* ns, int B, Plan* p, const
   p->off_pcm = take((size_t)p->n_total * 4);
   p->off_out = take((size_t)p->T * d_out(g) * 4);
   p->off_skflags = take(sk_flags_bytes(e));
+  if (e->ln_fuse) {
+    p->off_lncnt = take(ln_count_bytes(p->T));
+    p->off_lnpart = take((size_t)p->T * ln_parts(e) * 16);
+  }
   p->total = align_up(off, 1024);
   return true;
 }
@@ -901,7 +922,11 @@ bool plan_for(const asr_enc* e, const int64_t* ns, int64_t n, int B, Plan* p) {
 asr_status gemm(asr_enc* e, const CUtensorMap* amap, const ConvGather* cg, const GemmB& w, long long M, void* out,
                 long long ldo, const float* bias, const float* pe, int period, int epi, cudaStream_t st,
                 const CUtensorMap* omap, const ConvBox* box = nullptr, int zero_period = 0, int zero_from = 0,
-                int* sk_flags = nullptr) {
+                int* sk_flags = nullptr, const float* ln_g = nullptr, const float* ln_b = nullptr,
+                const Plan* plan = nullptr, char* ws = nullptr, int ln_epoch = 0) {
+  // ln_g / ln_b: residual update followed by the LayerNorm (gamma, beta) of
+  // the updated rows into h (EPI_LN; the plan and workspace give its buffers,
+  // ln_epoch counts the earlier such launches of the forward)
   // fp32 operands: every output of the engine is fp32
   if (e->kind == KIND_TF32 && !(epi & (EPI_OUT_F32 | EPI_RESID))) epi |= EPI_OUT_F32;
   GemmParams p;
@@ -918,6 +943,17 @@ asr_status gemm(asr_enc* e, const CUtensorMap* amap, const ConvGather* cg, const
   p.zero_period = zero_period;
   p.zero_from = zero_from;
   p.sk_flags = sk_flags;  // stream-K allowed (residual epilogue, the launcher decides)
+  if (ln_g) {
+    epi |= EPI_LN;
+    p.sk_flags = nullptr;
+    p.ln_gamma = ln_g;
+    p.ln_beta = ln_b;
+    p.ln_eps = e->g.ln_eps;
+    p.ln_count = reinterpret_cast<int*>(ws + plan->off_lncnt);
+    p.ln_part = reinterpret_cast<float*>(ws + plan->off_lnpart);
+    p.ln_h = ws + plan->off_h;
+    p.ln_epoch = ln_epoch;
+  }
   int bn;
   const CUtensorMap* amap3 = box ? nullptr : e->maps.companion3(amap);
   if (box) {
@@ -1063,6 +1099,10 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
   ASR_LAUNCH(e, cudaMemsetAsync(clip_max, 0, (size_t)p.B * 4, st));
   int* skf = reinterpret_cast<int*>(ws + p.off_skflags);
   ASR_LAUNCH(e, cudaMemsetAsync(skf, 0, sk_flags_bytes(e), st));
+  // LayerNorm epilogue of fc2 (16-bit tower): the next block's LN1, or the
+  // head's LayerNorm
+  const bool lnf = e->ln_fuse && e->ln_fuse_on && !f32;
+  if (lnf) ASR_LAUNCH(e, cudaMemsetAsync(ws + p.off_lncnt, 0, ln_count_bytes(p.T), st));
   MelClip* mclips = reinterpret_cast<MelClip*>(ws + p.off_mclips);
   ChunkDesc* chunkd = reinterpret_cast<ChunkDesc*>(ws + p.off_chunkd);
   if (!p.varlen) {
@@ -1163,7 +1203,7 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
 
   for (int l = 0; l < g->n_layers; ++l) {
     const LayerW& lw = e->layers[l];
-    ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, lw.ln1g, lw.ln1b, p.T, d, g->ln_eps, h, e->kind, st)));
+    if (l == 0 || !lnf) ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, lw.ln1g, lw.ln1b, p.T, d, g->ln_eps, h, e->kind, st)));
     ASR_K(PC_GEMM_QKV, ASR_TRY(gemm(e, &e->maps.h, nullptr, lw.qkv, p.T, qkv, 3 * d, lw.bqkv, nullptr, 1, 0, st, &e->maps.o_qkv)));
     if (f32)
       ASR_K(PC_ATTN, ASR_LAUNCH(e, launch_attention_f32(static_cast<const float*>(qkv), cu, p.nwin, p.max_win,
@@ -1174,12 +1214,19 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
     else
       ASR_K(PC_ATTN, ASR_LAUNCH(e, launch_attention_fa(e->maps.qkv, cu, p.nwin, p.max_win, g->n_heads, att, e->status,
                                                        kWaitLimitNs, f16, st)));
-    ASR_K(PC_GEMM_O, ASR_TRY(gemm(e, &e->maps.att, nullptr, lw.o, p.T, x, d, lw.bo, nullptr, 1, EPI_RESID, st, &e->maps.o_x,
-                                  nullptr, 0, 0, skf)));
+    // The out-projection keeps the separate LayerNorm: its K = d_model
+    // mainloop is shorter than the LayerNorm epilogue, which would then
+    // stall the tensor cores (measured slower than the two launches).
+    ASR_K(PC_GEMM_O, ASR_TRY(gemm(e, &e->maps.att, nullptr, lw.o, p.T, x, d, lw.bo, nullptr, 1, EPI_RESID, st,
+                                  &e->maps.o_x, nullptr, 0, 0, skf)));
     ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, lw.ln2g, lw.ln2b, p.T, d, g->ln_eps, h, e->kind, st)));
     ASR_K(PC_GEMM_FC1, ASR_TRY(gemm(e, &e->maps.h, nullptr, lw.fc1, p.T, ff, g->d_ffn, lw.b1, nullptr, 1, EPI_GELU, st, &e->maps.o_ff)));
+    // the LayerNorm that reads this update: the next layer's LN1, or the head's
+    const bool last = l + 1 == g->n_layers;
+    const float* nlg = !lnf ? nullptr : !last ? e->layers[l + 1].ln1g : g->proj1_out ? e->lnpg : nullptr;
+    const float* nlb = !lnf ? nullptr : !last ? e->layers[l + 1].ln1b : e->lnpb;
     ASR_K(PC_GEMM_FC2, ASR_TRY(gemm(e, &e->maps.ff, nullptr, lw.fc2, p.T, x, d, lw.b2, nullptr, 1, EPI_RESID, st, &e->maps.o_x,
-                                    nullptr, 0, 0, skf)));
+                                    nullptr, 0, 0, nlg ? nullptr : skf, nlg, nlb, &p, ws, l)));
     if (l == 0)
       if (float* t = tap(ASR_TAP_LAYER0)) ASR_LAUNCH(e, cudaMemcpyAsync(t, x, (size_t)p.T * d * 4, cudaMemcpyDeviceToDevice, st));
   }
@@ -1194,7 +1241,7 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
   // Store map of the caller's output (plain stores if it is not 16-byte aligned).
   CUtensorMap o_out_map;
   const CUtensorMap* o_out = make_tmap_out(&o_out_map, out, p.T, d_out(g), d_out(g), true) ? &o_out_map : nullptr;
-  ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, e->lnpg, e->lnpb, p.T, d, g->ln_eps, h, e->kind, st)));
+  if (!lnf) ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, e->lnpg, e->lnpb, p.T, d, g->ln_eps, h, e->kind, st)));
   ASR_K(PC_GEMM_HEAD, ASR_TRY(gemm(e, &e->maps.h, nullptr, e->p1, p.T, p1, g->proj1_out, e->bp1, nullptr, 1, EPI_GELU, st, &e->maps.o_p1)));
   if (!g->adapter_hidden) {
     ASR_K(PC_GEMM_HEAD, ASR_TRY(gemm(e, &e->maps.p1, nullptr, e->p2, p.T, out, g->proj2_out, e->bp2, nullptr, 1, EPI_OUT_F32, st, o_out)));
@@ -1414,6 +1461,22 @@ asr_status asr_enc_set_graphs(asr_enc* e, int enable) {
   return ASR_OK;
 }
 
+asr_status asr_enc_set_ln_fusion(asr_enc* e, int enable) {
+  if (!e) return fail(nullptr, ASR_E_INVAL, "handle is NULL");
+  e->ln_fuse_on = enable != 0;
+  if (e->gexec) {  // the recorded forward has the other kernel sequence
+    cudaGraphExecDestroy(e->gexec);
+    e->gexec = nullptr;
+  }
+  return ASR_OK;
+}
+
+asr_status asr_enc_ln_fusion(const asr_enc* e, int* active) {
+  if (!e || !active) return fail(nullptr, ASR_E_INVAL, "handle or output is NULL");
+  *active = (e->ln_fuse && e->ln_fuse_on) ? 1 : 0;
+  return ASR_OK;
+}
+
 asr_status asr_enc_profile(asr_enc* e, int enable) {
   if (!e) return fail(nullptr, ASR_E_INVAL, "handle is NULL");
   e->prof = enable != 0;
@@ -1532,6 +1595,56 @@ asr_status asr_op_linear(const void* x, const void* w, const float* bias, int64_
   const bool have_omap = !(e_bits & EPI_SWIGLU) && make_tmap_out(&omap, y, M, N, N, f32_out);
   const bool have_a3 = K % 128 == 0 && make_tmap_3d16(&amap3, x, M, K, K, 128, KIND_BF16);
   ASR_CUDA(nullptr, launch_gemm(&amap, wb, p, e_bits, bn, sms, st, have_omap ? &omap : nullptr, have_a3 ? &amap3 : nullptr));
+  return ASR_OK;
+}
+
+size_t asr_op_linear_resid_ln_ws_size(int64_t M, int N) {
+  if (M <= 0 || N <= 0) return 0;
+  const size_t cnt = ((size_t)(M + 31) / 32 * 4 + 255) / 256 * 256;
+  return 256 + cnt + (size_t)M * 2 * ((N + 255) / 256) * 16;
+}
+
+asr_status asr_op_linear_resid_ln(const void* x, const void* w, const float* bias, const float* gamma,
+                                  const float* beta, float eps, int64_t M, int N, int K, float* y, void* h,
+                                  void* ws, size_t ws_bytes, void* stream) {
+  if (!x || !w || !y || !h || !gamma || !beta || M <= 0 || N <= 0 || K <= 0 || !(eps > 0.f) || M > INT_MAX)
+    return fail(nullptr, ASR_E_INVAL, "linear_resid_ln: bad arguments");
+  if (K % 128 || N % 32) return fail(nullptr, ASR_E_UNSUPPORTED, "linear_resid_ln: needs K %% 128 == 0 and N %% 32 == 0");
+  if (!ws || ws_bytes < asr_op_linear_resid_ln_ws_size(M, N))
+    return fail(nullptr, ASR_E_WORKSPACE, "linear_resid_ln: workspace too small");
+  const int sms = current_sm_count();
+  GemmB wb;
+  wb.ptr = static_cast<const bf16*>(w);
+  wb.N = N;
+  wb.K = K;
+  CUtensorMap amap, amap3;
+  if ((reinterpret_cast<uintptr_t>(y) | reinterpret_cast<uintptr_t>(h) | reinterpret_cast<uintptr_t>(gamma) |
+       reinterpret_cast<uintptr_t>(beta)) & 15)
+    return fail(nullptr, ASR_E_INVAL, "linear_resid_ln: y, h, gamma and beta must be 16-byte aligned");
+  if (!make_weight_maps(wb) || !make_tmap_bf16(&amap, x, M, K, K, 128) ||
+      !make_tmap_3d16(&amap3, x, M, K, K, 128, KIND_BF16))
+    return fail(nullptr, ASR_E_INVAL, "linear_resid_ln: TMA descriptor encoding failed (16-byte alignment?)");
+  if (!gemm_ln_supported(wb, sms)) return fail(nullptr, ASR_E_UNSUPPORTED, "linear_resid_ln: N = %d too wide", N);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t cnt = ((size_t)(M + 31) / 32 * 4 + 255) / 256 * 256;
+  ASR_CUDA(nullptr, cudaMemsetAsync(ws, 0, 256 + cnt, st));
+  GemmParams p;
+  memset(&p, 0, sizeof p);
+  p.M = (int)M;
+  p.out = y;
+  p.ldo = N;
+  p.bias = bias;
+  p.pe_period = 1;
+  p.status = static_cast<int*>(ws);
+  p.limit_ns = kWaitLimitNs;
+  p.ln_gamma = gamma;
+  p.ln_beta = beta;
+  p.ln_eps = eps;
+  p.ln_count = reinterpret_cast<int*>(static_cast<char*>(ws) + 256);
+  p.ln_part = reinterpret_cast<float*>(static_cast<char*>(ws) + 256 + cnt);
+  p.ln_h = h;
+  p.ln_epoch = 0;  // counters cleared above
+  ASR_CUDA(nullptr, launch_gemm(&amap, wb, p, EPI_RESID | EPI_LN, -256, sms, st, nullptr, &amap3));
   return ASR_OK;
 }
 

@@ -163,6 +163,10 @@ cudaError_t run2_kp2(int epi, const CUtensorMap& a3, const CUtensorMap& b3, cons
     default: return cudaErrorInvalidValue;
   }
 }
+template <int KIND>
+cudaError_t run2_kp2_ln(const CUtensorMap& a3, const CUtensorMap& b3, const GemmParams& p, int grid, cudaStream_t st) {
+  return run2<256, EPI_RESID | EPI_LN, KIND, 2>(a3, b3, b3, p, grid, st);
+}
 
 template <int KIND>
 cudaError_t run2_240(int epi, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& p, int grid,
@@ -389,6 +393,30 @@ template <int KIND>
 cudaError_t launch16(const CUtensorMap* a_map, const GemmB& w, GemmParams p, int epi, int bn, int num_sms,
                      cudaStream_t st, const CUtensorMap* out_map, const CUtensorMap* a_map3) {
   p.out_tma = (out_map != nullptr && !(epi & (EPI_PE | EPI_SWIGLU))) ? 1 : 0;
+  if (epi & EPI_LN) {
+    // Residual + LayerNorm: 256-wide pair tiles with two-k-block stages,
+    // whole tiles in n-fast order (the epilogue waits on the row block's
+    // other n-tiles), N a multiple of 32, and at least as many resident
+    // pairs as n-tiles per row block.  Both outputs by plain stores.
+    const int n_blocks = (w.N + 255) / 256;
+    if (epi != (EPI_RESID | EPI_LN) || !a_map || !a_map3 || !w.has3 || p.conv_box || w.K % 128 || w.N % 32 ||
+        p.ldo % 8 || !p.ln_gamma || !p.ln_beta || !p.ln_count || !p.ln_part || !p.ln_h || p.M <= 0 ||
+        resident_pairs(num_sms) < n_blocks)
+      return cudaErrorInvalidValue;
+    p.out_tma = 0;
+    p.k_full = 1;
+    p.n_fast = 1;
+    p.sk = 0;
+    p.N = w.N;
+    p.K = w.K;
+    p.m_blocks = (p.M + 255) / 256;
+    p.n_blocks = n_blocks;
+    p.k_blocks = p.K / 128;
+    p.num_tiles = p.m_blocks * p.n_blocks;
+    p.ln_parts = 2 * n_blocks;  // two epilogue warps per lane quarter and n-tile
+    const int grid = 2 * std::min(p.num_tiles, resident_pairs(num_sms));
+    return run2_kp2_ln<KIND>(*a_map3, w.map3, p, grid, st);
+  }
   // Whole four-step k-blocks everywhere when A and B both come by TMA: the
   // steps past K (or past a tap's channels) multiply the zeros that the TMA
   // fills outside the tensors and that pad the conv weights, and issuing
@@ -466,12 +494,18 @@ cudaError_t launch16(const CUtensorMap* a_map, const GemmB& w, GemmParams p, int
   }
 }
 
+bool gemm_ln_supported(const GemmB& w, int num_sms) {
+  return w.kind != KIND_TF32 && w.has3 && w.K % 128 == 0 && w.N % 32 == 0 && w.N > 0 &&
+         resident_pairs(num_sms) >= (w.N + 255) / 256;
+}
+
 cudaError_t launch_gemm(const CUtensorMap* a_map, const GemmB& w, GemmParams p, int epi, int bn, int num_sms,
                         cudaStream_t st, const CUtensorMap* out_map, const CUtensorMap* a_map3) {
   if (w.kind == KIND_BF16) return launch16<KIND_BF16>(a_map, w, p, epi, bn, num_sms, st, out_map, a_map3);
   if (w.kind == KIND_F16) return launch16<KIND_F16>(a_map, w, p, epi, bn, num_sms, st, out_map, a_map3);
   // fp32 operands: one-SM tiles only (the CTA-pair kernel takes 16-bit
-  // operands), no gather mode
+  // operands), no gather mode, no LayerNorm epilogue
+  if (epi & EPI_LN) return cudaErrorInvalidValue;
   p.out_tma = (out_map != nullptr && !(epi & (EPI_PE | EPI_SWIGLU))) ? 1 : 0;
   p.n_fast = (p.conv_box || p.M > w.N) ? 1 : 0;
   p.k_full = 1;  // A and B by TMA (see launch16)

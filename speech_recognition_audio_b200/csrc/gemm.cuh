@@ -38,7 +38,9 @@
 
 namespace asr {
 
-enum : int { EPI_GELU = 1, EPI_OUT_F32 = 2, EPI_RESID = 4, EPI_PE = 8, EPI_SWIGLU = 16 };
+// EPI_LN (with EPI_RESID, CTA-pair tiles): the residual update is followed
+// by the LayerNorm of the updated rows, written as a second 16-bit output.
+enum : int { EPI_GELU = 1, EPI_OUT_F32 = 2, EPI_RESID = 4, EPI_PE = 8, EPI_SWIGLU = 16, EPI_LN = 32 };
 
 struct ConvGather {
   const bf16* x;  // activation [n_img, T_in, F_in, C] (C innermost)
@@ -98,6 +100,21 @@ struct GemmParams {
   // Output rows r with r % zero_period >= zero_from are written as zeros
   // (the padding rows of a packed convolution layout); zero_period 0 = none.
   int zero_period, zero_from;
+  // Residual + LayerNorm epilogue (EPI_LN): gamma, beta [N] and epsilon of
+  // the norm, its 16-bit output ln_h [M][ldo]; ln_part holds ln_parts
+  // partial statistics {count, mean, M2, 0} per row, [part][M] (one per
+  // epilogue warp and n-tile covering the row), ln_count one arrival counter
+  // per 32-row group: zero before the first launch on the buffer, each
+  // launch adds ln_parts to every group's count, and ln_epoch is the number
+  // of launches on the buffer before this one.
+  const float* ln_gamma;
+  const float* ln_beta;
+  float ln_eps;
+  int ln_parts;
+  int* ln_count;
+  float* ln_part;
+  void* ln_h;
+  int ln_epoch;
 };
 
 template <bool B>
@@ -178,6 +195,36 @@ static __device__ __noinline__ bool flag_wait_bounded(const int* flag, uint64_t 
       if (status && *reinterpret_cast<volatile int*>(status) != 0) return false;
     }
   }
+}
+
+// Wait (one thread) until *count >= target, for at most limit_ns; gives up
+// early when the status word already holds an error.
+static __device__ __noinline__ bool count_wait_bounded(const int* count, int target, uint64_t limit_ns, int* status,
+                                                       int code) {
+  if (ld_acquire_gpu(count) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 0;; ++it) {
+    __nanosleep(32);
+    if (ld_acquire_gpu(count) >= target) return true;
+    if ((it & 15) == 15) {
+      if (globaltimer_ns() - t0 > limit_ns) {
+        if (status) atomicCAS(status, 0, code);
+        return false;
+      }
+      if (status && *reinterpret_cast<volatile int*>(status) != 0) return false;
+    }
+  }
+}
+__device__ __forceinline__ void red_add_release_gpu(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ float4 ld_relaxed_gpu_f4(const float* p) {
+  float4 v;
+  asm volatile("ld.relaxed.gpu.global.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(p)
+               : "memory");
+  return v;
 }
 
 // Output rows covered by 128-row sub-tile u: [first, last) (conv-box mode

@@ -163,6 +163,205 @@ constexpr int gemm2_epi_warps() {
   return EPI == EPI_GELU ? 16 : 8;
 }
 
+// Residual + LayerNorm epilogue (EPI_RESID | EPI_LN; whole tiles of plain
+// GEMMs, BN = 256, N a multiple of 32, the n-tiles of a row block back to
+// back).
+//
+// One warp: 32 rows (one per lane) over the four 32-column groups
+// c = 32 half + 64 j of the accumulator, with a 4 KB shared buffer in which
+// 32 x 32 blocks are transposed between the row-per-lane layout of tensor
+// memory and coalesced global accesses (8 lanes per 128-byte row segment of
+// fp32, 4 per 64-byte segment of 16-bit values; 16-byte chunks XOR-swizzled
+// by row, which keeps both access patterns free of bank conflicts).
+//   pass 1, per group: the old residual block (loaded two groups ahead, the
+//     first two before the accumulator is ready) is transposed into the
+//     lanes; each lane forms x_new = x + (acc + bias) for its row (the
+//     additions of the plain residual epilogue, so the stream is the same
+//     bit for bit), writes it back into tensor memory and accumulates
+//     shifted sums (shift = the row's first value here);
+//   publish: the warp's partial statistics {count, mean, M2} of each row go
+//     to p.ln_part [part][row], then one release reduction-add (lane 0, after
+//     the warp barrier) on the 32-row group's counter;
+//   x pass: x_new from tensor memory, transposed, stored (coalesced) into
+//     the residual stream, while the other tiles of the rows publish;
+//   wait (bounded) until every warp of every n-tile covering these rows has
+//     added to the counter: it then holds (p.ln_epoch + 1) * p.ln_parts;
+//   merge: each lane folds its row's partials in one pass with the pairwise
+//     update of Chan, Golub and LeVeque (mean and M2 of a union from those
+//     of its parts), var = M2 / N;
+//   pass 3: h = (x_new - mean) / sqrt(var + eps) * gamma + beta from tensor
+//     memory, in 16 bits, transposed and stored (coalesced) into p.ln_h.
+// No wait cycle: under the persistent whole-tile schedule a tile's epilogue
+// waits only on the other n-tiles of its row block, whose indices are within
+// n_blocks of its own; each of those is processed by a resident pair after a
+// tile at least n_pairs (>= n_blocks) lower, and every warp publishes
+// before it waits.
+constexpr int kLnGroups = 4;  // 32-column groups of a warp (BN = 256, two warps per lane quarter)
+
+// Old residual block of rows row0.. (< mlimit) and columns n..n+31 in the
+// coalesced layout: lane l holds row row0 + l / 8 + 4 i, columns n + 4 (l % 8).
+__device__ __forceinline__ void ln_load_x(const GemmParams& p, int row0, int mlimit, int n, int lane, float4* pre) {
+  const float* base = reinterpret_cast<const float*>(p.out) + n + 4 * (lane & 7);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int row = row0 + (lane >> 3) + 4 * i;
+    pre[i] = row < mlimit ? *reinterpret_cast<const float4*>(base + (long long)row * p.ldo) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+template <int KIND>
+__device__ __forceinline__ void epilogue_warp_resid_ln(const GemmParams& p, uint32_t tb, int row0, int mlimit, int n0,
+                                                       int half, int lane, uint8_t* wbuf, int part,
+                                                       float4 (&pre)[2][8]) {
+  if (row0 >= mlimit) return;  // no valid row: nobody waits on this group (warp-uniform)
+  const int row = row0 + lane;
+  const bool valid = row < mlimit;
+  float4* wrow = reinterpret_cast<float4*>(wbuf + lane * 128);  // this lane's fp32 row of the block
+  float K = 0.f;
+  float2 s1 = make_float2(0.f, 0.f), s2 = make_float2(0.f, 0.f);
+  int cnt = 0;
+#pragma unroll
+  for (int j = 0; j < kLnGroups; ++j) {
+    const int n = n0 + half * 32 + 64 * j;
+    if (n >= p.N) break;  // warp-uniform
+    float v[32];
+    tmem_ld16(tb + n - n0, v);
+    tmem_ld16(tb + n - n0 + 16, v + 16);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = (lane >> 3) + 4 * i;
+      reinterpret_cast<float4*>(wbuf + r * 128)[(lane & 7) ^ (r & 7)] = pre[j & 1][i];
+    }
+    if (j + 2 < kLnGroups && n + 128 < p.N) ln_load_x(p, row0, mlimit, n + 128, lane, pre[j & 1]);
+    __syncwarp();
+    tmem_ld_wait();
+    const float4* b4 = p.bias ? reinterpret_cast<const float4*>(p.bias + n) : nullptr;  // same address in every lane
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float4 o = wrow[k ^ (lane & 7)];
+      const float4 bq = b4 ? __ldg(b4 + k) : make_float4(0.f, 0.f, 0.f, 0.f);
+      // x_new = x + (acc + bias), the plain residual epilogue's additions
+      const float2 lo = add2(make_float2(o.x, o.y), add2(make_float2(v[4 * k], v[4 * k + 1]), make_float2(bq.x, bq.y)));
+      const float2 hi =
+          add2(make_float2(o.z, o.w), add2(make_float2(v[4 * k + 2], v[4 * k + 3]), make_float2(bq.z, bq.w)));
+      v[4 * k] = lo.x;
+      v[4 * k + 1] = lo.y;
+      v[4 * k + 2] = hi.x;
+      v[4 * k + 3] = hi.y;
+    }
+    __syncwarp();  // the block is read before the next group overwrites it
+    if (j == 0) K = v[0];
+    const float2 nk = make_float2(-K, -K);
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      const float2 dv = add2(make_float2(v[i], v[i + 1]), nk);
+      s1 = add2(s1, dv);
+      s2 = fma2(dv, dv, s2);
+    }
+    cnt += 32;
+    tmem_st16(tb + n - n0, v);
+    tmem_st16(tb + n - n0 + 16, v + 16);
+  }
+  // publish this warp's partial statistics of its rows
+  {
+    const float inv = cnt ? 1.0f / static_cast<float>(cnt) : 0.f;
+    const float t1 = s1.x + s1.y, t2 = s2.x + s2.y;
+    const float mu = K + t1 * inv;
+    const float m2 = fmaxf(t2 - t1 * t1 * inv, 0.f);
+    if (valid)
+      *reinterpret_cast<float4*>(p.ln_part + ((long long)part * p.M + row) * 4) =
+          make_float4(static_cast<float>(cnt), mu, m2, 0.f);
+  }
+  __syncwarp();  // orders the lanes' partials before lane 0's release
+  int* counter = p.ln_count + row0 / 32;
+  if (lane == 0) red_add_release_gpu(counter, 1);
+  tmem_st_wait();
+  // x pass: the updated rows into the residual stream
+  float* xo = reinterpret_cast<float*>(p.out) + 4 * (lane & 7);
+#pragma unroll
+  for (int j = 0; j < kLnGroups; ++j) {
+    const int n = n0 + half * 32 + 64 * j;
+    if (n >= p.N) break;
+    float v[32];
+    tmem_ld16(tb + n - n0, v);
+    tmem_ld16(tb + n - n0 + 16, v + 16);
+    tmem_ld_wait();
+#pragma unroll
+    for (int k = 0; k < 8; ++k) wrow[k ^ (lane & 7)] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = (lane >> 3) + 4 * i;
+      const float4 o = reinterpret_cast<const float4*>(wbuf + r * 128)[(lane & 7) ^ (r & 7)];
+      if (row0 + r < mlimit) *reinterpret_cast<float4*>(xo + (long long)(row0 + r) * p.ldo + n) = o;
+    }
+    __syncwarp();
+  }
+  // every warp of this launch covering these rows has added once: the
+  // counter (zero before the forward) reaches (epoch + 1) * parts
+  if (lane == 0) count_wait_bounded(counter, (p.ln_epoch + 1) * p.ln_parts, p.limit_ns, p.status, DEV_TIMEOUT_EPILOGUE);
+  __syncwarp();
+  (void)ld_acquire_gpu(counter);  // every lane: the partials below come after the arrivals
+  float mean = 0.f, rstd = 0.f;
+  if (valid) {
+    const float4* pr = reinterpret_cast<const float4*>(p.ln_part) + row;
+    float nt = 0.f, m2 = 0.f;
+    for (int i0 = 0; i0 < p.ln_parts; i0 += 8) {
+      float4 q[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) q[i] = i0 + i < p.ln_parts ? __ldcg(pr + (long long)(i0 + i) * p.M) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (q[i].x > 0.f) {
+          const float nn = nt + q[i].x;
+          const float dm = q[i].y - mean;
+          const float wb = __fdividef(q[i].x, nn);
+          mean = fmaf(dm, wb, mean);
+          m2 += q[i].z + dm * dm * nt * wb;
+          nt = nn;
+        }
+    }
+    rstd = rsqrtf(fmaxf(m2 / nt, 0.f) + p.ln_eps);
+  }
+  // pass 3: the normalised rows, 16-bit (64-byte row segments in the buffer)
+  uint16_t* ho = reinterpret_cast<uint16_t*>(p.ln_h) + 8 * (lane & 3);
+  const float2 nm = make_float2(-mean, -mean), rs = make_float2(rstd, rstd);
+#pragma unroll
+  for (int j = 0; j < kLnGroups; ++j) {
+    const int n = n0 + half * 32 + 64 * j;
+    if (n >= p.N) break;
+    float v[32];
+    tmem_ld16(tb + n - n0, v);
+    tmem_ld16(tb + n - n0 + 16, v + 16);
+    tmem_ld_wait();
+    const float4* g4 = reinterpret_cast<const float4*>(p.ln_gamma + n);
+    const float4* b4 = reinterpret_cast<const float4*>(p.ln_beta + n);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float4 g = __ldg(g4 + k), b = __ldg(b4 + k);
+      const float2 lo = fma2(add2(make_float2(v[4 * k], v[4 * k + 1]), nm), mul2(rs, make_float2(g.x, g.y)),
+                             make_float2(b.x, b.y));
+      const float2 hi = fma2(add2(make_float2(v[4 * k + 2], v[4 * k + 3]), nm), mul2(rs, make_float2(g.z, g.w)),
+                             make_float2(b.z, b.w));
+      v[4 * k] = lo.x;
+      v[4 * k + 1] = lo.y;
+      v[4 * k + 2] = hi.x;
+      v[4 * k + 3] = hi.y;
+    }
+    uint4* hrow = reinterpret_cast<uint4*>(wbuf + lane * 64);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) hrow[k ^ ((lane >> 1) & 3)] = pack8_16<KIND>(v + 8 * k);
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = (lane >> 2) + 8 * i;
+      const uint4 o = reinterpret_cast<const uint4*>(wbuf + r * 64)[(lane & 3) ^ ((r >> 1) & 3)];
+      if (row0 + r < mlimit) *reinterpret_cast<uint4*>(ho + (long long)(row0 + r) * p.ldo + n) = o;
+    }
+    __syncwarp();
+  }
+}
+
 template <int BN, int STAGES, int EPI, int KIND, int KP = 1>
 __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmOut,
                                               const GemmParams& p) {
@@ -340,10 +539,17 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap& tmA, const CUte
         epilogue_prefetch_l2(p, t, half, q, lane, BN, S::BM, rank_rows, S::CSTRIDE);
       float breg[4];
       load_bias(p, n0, BN, half, lane, breg, S::CSTRIDE);
-      if (!mbar_wait_bounded(&tfull[a], aph, p.limit_ns, p.status, DEV_TIMEOUT_EPILOGUE)) break;
-      tc_fence_after();
       int r_first, r_last;
       subtile_rows(p, 2 * mb + static_cast<int>(rank), r_first, r_last);
+      float4 pre[2][(EPI & EPI_LN) ? 8 : 1];  // LayerNorm epilogue: the first two groups' old rows
+      if constexpr ((EPI & EPI_LN) != 0) {
+        static_assert(BN == 256 && S::EPI_WARPS == 8, "LayerNorm epilogue: four groups per warp");
+        const int row0 = r_first + 32 * q;
+        for (int j = 0; j < 2; ++j)
+          if (row0 < r_last && n0 + half * 32 + 64 * j < p.N) ln_load_x(p, row0, r_last, n0 + half * 32 + 64 * j, lane, pre[j]);
+      }
+      if (!mbar_wait_bounded(&tfull[a], aph, p.limit_ns, p.status, DEV_TIMEOUT_EPILOGUE)) break;
+      tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + a * S::ACC_COLS;
       // Flag of this warp's rows and columns: the trailing piece of a split
       // tile is the first piece of the next pair, so it uses that pair's slot.
@@ -360,7 +566,10 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap& tmA, const CUte
         }
         have = __shfl_sync(0xffffffffu, have, 0);
       }
-      if (have)
+      if constexpr ((EPI & EPI_LN) != 0)
+        epilogue_warp_resid_ln<KIND>(p, tb, r_first + 32 * q, r_last, n0, half, lane, sEpi + ew * S::WBUF,
+                                     nb * 2 + half, pre);
+      else if (have)
         epilogue_warp<EPI, KIND, S::NBUF, S::BOXB>(p, &tmOut, tb, r_first + 32 * q, r_last, n0, BN, half, lane,
                                                    sEpi + ew * S::WBUF, breg, kind, S::CSTRIDE, &groups);
       tc_fence_before();

@@ -195,7 +195,14 @@ bool make_tmap_out(CUtensorMap* map, const void* ptr, unsigned long long rows, u
 // ignored for the position and SwiGLU epilogues.
 // a_map3: 3-D map of A (make_tmap_3d16, box rows 128) or null; with it, plain
 // 256-wide CTA-pair launches run two k-blocks per pipeline stage.
+// epi = EPI_RESID | EPI_LN (16-bit kinds; needs a_map3 and p.ln_* set,
+// p.ldo % 8 == 0): the residual update and the LayerNorm of the updated
+// rows into p.ln_h; the launch runs whole 256 x 256 pair tiles (bn and
+// out_map ignored).  cudaErrorInvalidValue when the shape does not allow it.
 cudaError_t launch_gemm(const CUtensorMap* a_map, const GemmB& w, GemmParams p, int epi, int bn, int num_sms,
                         cudaStream_t st, const CUtensorMap* out_map, const CUtensorMap* a_map3 = nullptr);
+// Whether launch_gemm takes EPI_RESID | EPI_LN for this weight (16-bit
+// kind, K % 128 == 0, N % 32 == 0, enough resident CTA pairs).
+bool gemm_ln_supported(const GemmB& w, int num_sms);
 
 }  // namespace asr

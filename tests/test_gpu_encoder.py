@@ -182,6 +182,44 @@ def test_whisper_small_32x30s_sampled():
     _sampled("whisper_small_32x30s", [(0, None), (31, None)])
 
 
+@pytest.mark.parametrize("wname", ["moss_1x30s", "tiny_f16"])
+def test_ln_fusion_matches_separate_layernorms(wname):
+    """16-bit encoders compute each block's first LayerNorm (and the head's)
+    in the previous fc2's epilogue; with that turned off the separate
+    LayerNorm kernels run.  Both match the oracle, and they agree closely
+    with each other (they differ only by the order in which the row
+    statistics are summed)."""
+    if wname == "tiny_f16":
+        base = synth.GEOMETRIES["tiny"].as_dict()
+        base.update(dtype=synth.DTYPE_F16)
+        g = synth.Geometry(**base)
+        W = synth.make_weights(g, 81, affine=True)
+        enc = sra.Encoder(g, {k: v.cuda() for k, v in W.items()})
+        pcm = np.stack([synth.pcm_clip(48000, 532), synth.pcm_clip(48000, 533)])
+    else:
+        enc, W, g = _encoder(wname)
+        pcm = synth.pcm_batch(synth.WORKLOADS[wname])
+    assert enc.ln_fusion()
+    fused = _run(enc, pcm)
+    enc.set_ln_fusion(False)
+    assert not enc.ln_fusion()
+    plain = _run(enc, pcm)
+    enc.set_ln_fusion(True)
+    again = _run(enc, pcm)
+    np.testing.assert_array_equal(fused, again)
+    ref = oracle.forward(pcm, W, g)
+    assert_encoder_parity(fused, ref, f"{wname} LayerNorm epilogue")
+    assert_encoder_parity(plain, ref, f"{wname} separate LayerNorms")
+    rel = np.linalg.norm(fused - plain) / np.linalg.norm(plain)
+    print(f"[parity] {wname} fused vs separate LayerNorm rel L2 {rel:.2e}")
+    assert rel < 1e-2
+
+
+def test_fp32_weights_keep_separate_layernorms():
+    enc, W, g = _encoder("tiny_1x1s")
+    assert not enc.ln_fusion()
+
+
 def test_host_forward_matches_device_forward():
     enc, W, g = _encoder("tiny_1x1s")
     pcm = np.stack([synth.pcm_clip(32000, 900 + b) for b in range(3)])

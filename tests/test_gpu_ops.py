@@ -87,6 +87,57 @@ def test_linear_stream_k(M, N, K, epi):
     assert np.array_equal(runs[0], runs[1])
 
 
+@pytest.mark.parametrize("M,N,K,shift", [(6240, 1280, 1280, 0.0), (6240, 1280, 5120, 0.0), (333, 768, 3072, 0.0),
+                                         (1, 256, 128, 0.0), (300, 1280, 256, 50.0), (77, 32, 128, 0.0),
+                                         (500, 96, 256, -3.0), (1000, 1312, 128, 0.0), (48000, 768, 128, 0.0)])
+def test_linear_resid_ln(M, N, K, shift):
+    """Residual GEMM + LayerNorm of the updated rows in one launch: y against
+    the oracle's r0 + x w^T + b (and bit for bit against the plain residual
+    epilogue where that runs whole tiles, K < 40 k-blocks), h against the
+    oracle's LayerNorm of it.  Ragged M (partial 32-row groups and 256-row
+    tiles), N with a partial last n-tile (96, 1312: halves of warps with 32 or
+    no valid columns), a single row, rows with a large common offset (the
+    statistics' cancellation), and 188 row blocks (more tiles than pairs)."""
+    rng = np.random.default_rng(M + 3 * N + K)
+    x = _bf16(rng.normal(size=(M, K)))
+    w = _bf16(rng.normal(size=(N, K)) * 0.04)
+    b = torch.from_numpy(rng.normal(size=N).astype(np.float32) * 0.1)
+    g = torch.from_numpy((1 + 0.1 * rng.normal(size=N)).astype(np.float32))
+    be = torch.from_numpy((0.05 * rng.normal(size=N)).astype(np.float32))
+    r0 = (rng.normal(size=(M, N)) + shift).astype(np.float32)
+    xc, wc, bc = x.cuda(), w.cuda(), b.cuda()
+    y = torch.from_numpy(r0).cuda()
+    h = sra.linear_resid_ln(xc, wc, bc, g.cuda(), be.cuda(), y, eps=1e-5)
+    y2 = torch.from_numpy(r0).cuda()
+    h2 = sra.linear_resid_ln(xc, wc, bc, g.cuda(), be.cuda(), y2, eps=1e-5)
+    torch.cuda.synchronize()
+    yr = r0.astype(np.float64) + oracle.linear(x.float().numpy(), w, b.numpy())
+    hr = oracle.layer_norm(yr, g.numpy(), be.numpy(), 1e-5)
+    got_y, got_h = y.cpu().numpy(), h.float().cpu().numpy()
+    np.testing.assert_allclose(got_y, yr, rtol=1e-5, atol=2e-4 * np.sqrt(K / 64) * 0.8)
+    err = np.abs(got_h - hr)
+    tol = 2.0 ** -8 * np.abs(hr) + 2e-3
+    assert (err <= tol).all(), f"h max err {err.max()} at {np.unravel_index(err.argmax(), err.shape)}"
+    assert np.array_equal(got_y, y2.cpu().numpy()) and np.array_equal(got_h, h2.float().cpu().numpy())
+    if K < 40 * 64:
+        y3 = torch.from_numpy(r0).cuda()
+        sra.linear(xc, wc, bc, sra.EPI_F32_RESID, out=y3, tile_n=-256)
+        assert np.array_equal(got_y, y3.cpu().numpy())
+
+
+def test_linear_resid_ln_rejects_unsupported_shapes():
+    x = torch.zeros((64, 96), dtype=torch.bfloat16, device="cuda")       # K % 128 != 0
+    w = torch.zeros((256, 96), dtype=torch.bfloat16, device="cuda")
+    v = torch.zeros(256, device="cuda")
+    y = torch.zeros((64, 256), device="cuda")
+    with pytest.raises(sra.AsrError):
+        sra.linear_resid_ln(x, w, v, v, v, y)
+    x = torch.zeros((64, 128), dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros((48, 128), dtype=torch.bfloat16, device="cuda")      # N % 32 != 0
+    with pytest.raises(sra.AsrError):
+        sra.linear_resid_ln(x, w, v[:48], v[:48], v[:48], y[:, :48].contiguous())
+
+
 @pytest.mark.parametrize("epi", ["gelu", "f32", "resid", "swiglu"])
 def test_linear_epilogues(epi):
     M, N, K = 333, 1024, 768
