@@ -39,10 +39,11 @@ def test_linear_bf16_bias(M, N, K):
 
 
 @pytest.mark.parametrize("tile_n", [256, 160, 128, 64, -256, -128])
-@pytest.mark.parametrize("M,N,K", [(6240, 1280, 1280), (300, 480, 4320), (257, 2560, 96)])
+@pytest.mark.parametrize("M,N,K", [(6240, 1280, 1280), (300, 480, 4320), (257, 2560, 96), (20000, 480, 16)])
 def test_linear_tile_modes(tile_n, M, N, K):
     """Every tile shape of the engine (one SM 128 x tile_n, or a CTA pair
-    256 x -tile_n) gives the same result, including ragged M and N tails."""
+    256 x -tile_n) gives the same result, including ragged M and N tails
+    and a single partial k-block (K = 16, as in conv1)."""
     if tile_n == 160 and N % 160:
         pytest.skip("160-wide tiles need N % 160 == 0")
     rng = np.random.default_rng(M + N + K + tile_n)
