@@ -425,6 +425,9 @@ __device__ __forceinline__ void epilogue_warp(const GemmParams& p, const CUtenso
   // A 32-row box may be stored whole when all its rows belong to this
   // sub-tile, or when the rows past the end lie past M (the TMA clips them).
   const bool rows_ok = TMA_OK && p.out_tma && (mlimit - row0 >= 32 || mlimit >= p.M);
+  // 16-byte aligned bias: vector loads of each group's biases (else the
+  // per-lane values loaded before the accumulator wait, broadcast by shuffle)
+  const bool bias_vec = (reinterpret_cast<uintptr_t>(p.bias) & 15) == 0;
   int j = 0;
 #pragma unroll 1
   for (int c = half * 32; c < BN; c += cstride, ++j) {
@@ -438,9 +441,26 @@ __device__ __forceinline__ void epilogue_warp(const GemmParams& p, const CUtenso
     tmem_ld_wait();
     // ---- phase A
     if (p.bias && kind != PIECE_PARTIAL) {
-      const float bj = breg[j];
+      if (bias_vec) {
+        // the group's biases: the same address in every lane (broadcast loads)
+        const float4* b4 = reinterpret_cast<const float4*>(p.bias + n);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] += __shfl_sync(0xffffffffu, bj, i);
+        for (int k = 0; k < 8; ++k) {
+          if (4 * k < w) {
+            const float4 b = __ldg(b4 + k);
+            const float2 lo = add2(make_float2(v[4 * k], v[4 * k + 1]), make_float2(b.x, b.y));
+            const float2 hi = add2(make_float2(v[4 * k + 2], v[4 * k + 3]), make_float2(b.z, b.w));
+            v[4 * k] = lo.x;
+            v[4 * k + 1] = lo.y;
+            v[4 * k + 2] = hi.x;
+            v[4 * k + 3] = hi.y;
+          }
+        }
+      } else {
+        const float bj = breg[j];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] += __shfl_sync(0xffffffffu, bj, i);
+      }
     }
     if (p.zero_period && (row0 + lane) % p.zero_period >= p.zero_from) {
 #pragma unroll
