@@ -428,6 +428,8 @@ __device__ __forceinline__ void epilogue_warp(const GemmParams& p, const CUtenso
   // 16-byte aligned bias: vector loads of each group's biases (else the
   // per-lane values loaded before the accumulator wait, broadcast by shuffle)
   const bool bias_vec = (reinterpret_cast<uintptr_t>(p.bias) & 15) == 0;
+  // this lane's row is a zero (padding) row of a packed convolution layout
+  const bool zero_row = p.zero_period && (row0 + lane) % p.zero_period >= p.zero_from;
   int j = 0;
 #pragma unroll 1
   for (int c = half * 32; c < BN; c += cstride, ++j) {
@@ -436,8 +438,10 @@ __device__ __forceinline__ void epilogue_warp(const GemmParams& p, const CUtenso
     const int w = (BN - c < 32 || p.N - n < 32) ? 16 : 32;  // valid columns in this group (N % 16 == 0)
     const bool use_tma = rows_ok && BN - c >= 32;
     float v[32];
-    tmem_ld16(tb + c, v);
-    if (BN - c >= 32) tmem_ld16(tb + c + 16, v + 16);
+    if (BN - c >= 32)
+      tmem_ld32(tb + c, v);
+    else
+      tmem_ld16(tb + c, v);
     tmem_ld_wait();
     // ---- phase A
     if (p.bias && kind != PIECE_PARTIAL) {
@@ -462,7 +466,7 @@ __device__ __forceinline__ void epilogue_warp(const GemmParams& p, const CUtenso
         for (int i = 0; i < 32; ++i) v[i] += __shfl_sync(0xffffffffu, bj, i);
       }
     }
-    if (p.zero_period && (row0 + lane) % p.zero_period >= p.zero_from) {
+    if (zero_row) {
 #pragma unroll
       for (int i = 0; i < 32; ++i) v[i] = 0.f;  // GELU(0) = 0: the row stays zero
     }
