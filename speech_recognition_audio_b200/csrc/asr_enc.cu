@@ -51,6 +51,11 @@ struct ActMaps {
   // Store maps of the GEMM outputs (32 x 32 boxes): residual stream, QKV,
   // FFN hidden, head, adapter hidden, conv outputs.
   CUtensorMap o_x, o_qkv, o_ff, o_p1, o_p2, o_c2, o_c3, o_c1;
+  // QKV split (16-bit, T not a multiple of 256): rows [0, qkv_main) on
+  // CTA-pair tiles, the last T - qkv_main on one-SM tiles (A and output maps
+  // of those rows), concurrently on the encoder's side stream
+  int64_t qkv_main = 0;
+  CUtensorMap h_tail, o_qkv_tail;
   // 3-D companions of the plain activation maps (boxes of 128 rows x two
   // 64-column k-blocks, 16-bit kinds with K a multiple of 128): with one, the
   // CTA-pair GEMM loads two k-blocks of A per TMA copy.
@@ -311,6 +316,9 @@ struct asr_enc {
   cudaGraphExec_t gexec = nullptr;
   int glaunches = 0;
   cudaStream_t cap_st = nullptr;
+  // side stream and fork / join events of the split QKV projection
+  cudaStream_t aux_st = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
   bool graphs = true;
   bool have_last = false;
   Plan last_plan;
@@ -485,6 +493,9 @@ void asr_enc_destroy(asr_enc* e) {
   if (!e) return;
   if (e->gexec) cudaGraphExecDestroy(e->gexec);
   if (e->cap_st) cudaStreamDestroy(e->cap_st);
+  if (e->aux_st) cudaStreamDestroy(e->aux_st);
+  if (e->ev_fork) cudaEventDestroy(e->ev_fork);
+  if (e->ev_join) cudaEventDestroy(e->ev_join);
   for (cudaEvent_t ev : e->ev_pool) cudaEventDestroy(ev);
   if (e->slab) {
     if (e->free_fn)
@@ -923,7 +934,7 @@ asr_status gemm(asr_enc* e, const CUtensorMap* amap, const ConvGather* cg, const
                 long long ldo, const float* bias, const float* pe, int period, int epi, cudaStream_t st,
                 const CUtensorMap* omap, const ConvBox* box = nullptr, int zero_period = 0, int zero_from = 0,
                 int* sk_flags = nullptr, const float* ln_g = nullptr, const float* ln_b = nullptr,
-                const Plan* plan = nullptr, char* ws = nullptr, int ln_epoch = 0) {
+                const Plan* plan = nullptr, char* ws = nullptr, int ln_epoch = 0, int force_bn = 0) {
   // ln_g / ln_b: residual update followed by the LayerNorm (gamma, beta) of
   // the updated rows into h (EPI_LN; the plan and workspace give its buffers,
   // ln_epoch counts the earlier such launches of the forward)
@@ -965,6 +976,7 @@ asr_status gemm(asr_enc* e, const CUtensorMap* amap, const ConvGather* cg, const
     bn = e->kind == KIND_TF32 ? gemm_pick_bn_tf32((int)M, w.N, e->num_sms)
                               : gemm_pick_bn((int)M, w.N, e->num_sms, cg != nullptr);
   }
+  if (force_bn) bn = force_bn;
   cudaError_t r = launch_gemm(amap, w, p, epi, bn, e->num_sms, st, omap, amap3);
   if (r != cudaSuccess) return fail(e, ASR_E_CUDA, "gemm launch (N=%d K=%d M=%lld epi=%d bn=%d): %s", w.N, w.K, M, epi, bn, cudaGetErrorString(r));
   return ASR_OK;
@@ -1053,6 +1065,16 @@ asr_status ensure_maps(asr_enc* e, const Plan& p, char* ws) {
   else if (ok)
     ok = make_tmap_out(&m.o_c1, ws + p.off_c1, (unsigned long long)p.B * p.F, d, d, f32);
   if (ok && g->adapter_hidden) ok = make_tmap_act(k, &m.gu, ws + p.off_gu, p.T, g->adapter_hidden, g->adapter_hidden, 128);
+  // QKV split: the CTA-pair launch takes whole 256-row blocks; with T % 256
+  // rows left over (the 16 x 30 s batch: 6240 = 24 x 256 + 96) it would run
+  // one more wave of tiles a third full, which the one-SM tail launch replaces
+  m.qkv_main = 0;
+  if (ok && !f32 && p.T > 256 && p.T % 256 && d % 128 == 0) {
+    const int64_t mm = p.T / 256 * 256;
+    ok = make_tmap_act(k, &m.h_tail, ws + p.off_h + (size_t)mm * d * e->es, p.T - mm, d, d, 128) &&
+         make_tmap_out(&m.o_qkv_tail, ws + p.off_qkv + (size_t)mm * 3 * d * e->es, p.T - mm, 3 * d, 3 * d, false);
+    if (ok) m.qkv_main = mm;
+  }
   m.n3 = 0;
   if (ok)
     ok = m.add3(&m.h, ws + p.off_h, p.T, d, k) && m.add3(&m.att, ws + p.off_att, p.T, d, k) &&
@@ -1097,6 +1119,12 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
   e->prof_recs.clear();
   ASR_LAUNCH(e, cudaMemsetAsync(e->status, 0, 4, st));
   ASR_LAUNCH(e, cudaMemsetAsync(clip_max, 0, (size_t)p.B * 4, st));
+  if (e->maps.qkv_main && !e->aux_st) {
+    if (cudaStreamCreateWithFlags(&e->aux_st, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&e->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&e->ev_join, cudaEventDisableTiming) != cudaSuccess)
+      return fail(e, ASR_E_CUDA, "side stream / events for the split QKV projection");
+  }
   int* skf = reinterpret_cast<int*>(ws + p.off_skflags);
   ASR_LAUNCH(e, cudaMemsetAsync(skf, 0, sk_flags_bytes(e), st));
   // LayerNorm epilogue of fc2 (16-bit tower): the next block's LN1, or the
@@ -1204,7 +1232,25 @@ asr_status run_forward(asr_enc* e, const float* pcm, const Plan& p, float* out, 
   for (int l = 0; l < g->n_layers; ++l) {
     const LayerW& lw = e->layers[l];
     if (l == 0 || !lnf) ASR_K(PC_LN, ASR_LAUNCH(e, launch_layer_norm(x, lw.ln1g, lw.ln1b, p.T, d, g->ln_eps, h, e->kind, st)));
-    ASR_K(PC_GEMM_QKV, ASR_TRY(gemm(e, &e->maps.h, nullptr, lw.qkv, p.T, qkv, 3 * d, lw.bqkv, nullptr, 1, 0, st, &e->maps.o_qkv)));
+    if (e->maps.qkv_main) {
+      // rows [0, main) on CTA-pair tiles; the last T % 256 rows on one-SM
+      // tiles on the side stream, whose CTAs take the SMs that the pair
+      // launch leaves idle in its last wave; joined before the attention
+      const int64_t mm = e->maps.qkv_main;
+      void* qkv_tail = static_cast<char*>(qkv) + (size_t)mm * 3 * d * e->es;
+      prof_begin(e, PC_GEMM_QKV, st);
+      ASR_LAUNCH(e, cudaEventRecord(e->ev_fork, st));
+      ASR_TRY(gemm(e, &e->maps.h, nullptr, lw.qkv, mm, qkv, 3 * d, lw.bqkv, nullptr, 1, 0, st, &e->maps.o_qkv));
+      ASR_LAUNCH(e, cudaStreamWaitEvent(e->aux_st, e->ev_fork, 0));
+      ++e->launches;
+      ASR_TRY(gemm(e, &e->maps.h_tail, nullptr, lw.qkv, p.T - mm, qkv_tail, 3 * d, lw.bqkv, nullptr, 1, 0, e->aux_st,
+                   &e->maps.o_qkv_tail, nullptr, 0, 0, nullptr, nullptr, nullptr, nullptr, nullptr, 0, 256));
+      ASR_LAUNCH(e, cudaEventRecord(e->ev_join, e->aux_st));
+      ASR_LAUNCH(e, cudaStreamWaitEvent(st, e->ev_join, 0));
+      prof_end(e, st);
+    } else {
+      ASR_K(PC_GEMM_QKV, ASR_TRY(gemm(e, &e->maps.h, nullptr, lw.qkv, p.T, qkv, 3 * d, lw.bqkv, nullptr, 1, 0, st, &e->maps.o_qkv)));
+    }
     if (f32)
       ASR_K(PC_ATTN, ASR_LAUNCH(e, launch_attention_f32(static_cast<const float*>(qkv), cu, p.nwin, p.max_win,
                                                         g->n_heads, static_cast<float*>(att), st)));
