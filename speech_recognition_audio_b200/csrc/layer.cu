@@ -92,9 +92,97 @@ __global__ void __launch_bounds__(128) layer_norm_kernel(const float* __restrict
   }
 }
 
+// Single-wave form, for row counts that fit the SMs at once (at d = 1280
+// up to 44 rows per SM: four blocks of 11 warps, 220 KB of row buffers):
+// one row per warp, copied into the warp's shared-memory buffer (cp.async)
+// and read from there twice, statistics then output, so a thread holds none
+// of the row across the two passes; every row's load is in flight at once
+// instead of the two rounds of the register form.  Same arithmetic, in the
+// same order, as layer_norm_kernel.
+constexpr int kLnWaveWarps = 11;
+template <int V, int OUT>
+__global__ void __launch_bounds__(32 * kLnWaveWarps, 4) layer_norm_wave_kernel(const float* __restrict__ x, const float* __restrict__ g,
+                                                              const float* __restrict__ b, long long M, float eps,
+                                                              void* __restrict__ y) {
+  constexpr int D = V * 128;
+  extern __shared__ float4 ln_smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float4* buf = ln_smem + warp * (D / 4);
+  const long long row = (long long)blockIdx.x * kLnWaveWarps + warp;
+  pdl_wait();
+  pdl_trigger();
+  if (row >= M) return;
+  const float4* xr = reinterpret_cast<const float4*>(x + row * D);
+#pragma unroll
+  for (int i = 0; i < V; ++i) cp_async_16_zfill(buf + lane + 32 * i, xr + lane + 32 * i, true);
+  cp_async_commit();
+  cp_async_wait<0>();
+  // each lane reads back exactly the 16-byte chunks it copied
+  const float K = __shfl_sync(0xffffffffu, buf[lane].x, 0);  // x[row][0]
+  float s1 = 0.f, s2 = 0.f;
+#pragma unroll 2
+  for (int i = 0; i < V; ++i) {
+    const float4 v = buf[lane + 32 * i];
+    const float a = v.x - K, bb = v.y - K, c = v.z - K, d = v.w - K;
+    s1 += (a + bb) + (c + d);
+    s2 += (a * a + bb * bb) + (c * c + d * d);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+    s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+  }
+  const float m1 = s1 * (1.0f / D);
+  const float mean = K + m1;
+  const float var = fmaxf(s2 * (1.0f / D) - m1 * m1, 0.0f);
+  const float rstd = rsqrtf(var + eps);
+#pragma unroll 2
+  for (int i = 0; i < V; ++i) {
+    const int c4 = lane + 32 * i;
+    const float4 v = buf[c4];
+    const float4 gg = __ldg(reinterpret_cast<const float4*>(g) + c4), bv = __ldg(reinterpret_cast<const float4*>(b) + c4);
+    const float o0 = (v.x - mean) * rstd * gg.x + bv.x;
+    const float o1 = (v.y - mean) * rstd * gg.y + bv.y;
+    const float o2 = (v.z - mean) * rstd * gg.z + bv.z;
+    const float o3 = (v.w - mean) * rstd * gg.w + bv.w;
+    if (OUT == KIND_TF32) {
+      reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + row * D)[c4] = make_float4(o0, o1, o2, o3);
+    } else {
+      const uint2 w2 = make_uint2(pack2_16<OUT>(o0, o1), pack2_16<OUT>(o2, o3));
+      reinterpret_cast<uint2*>(reinterpret_cast<bf16*>(y) + row * D)[c4] = w2;
+    }
+  }
+}
+
 template <int V, int OUT>
 static cudaError_t ln_launch(const float* x, const float* g, const float* b, long long M, float eps, void* y,
                              cudaStream_t st) {
+  {
+    // single-wave form when every row fits in flight at once
+    constexpr int WSMEM = kLnWaveWarps * V * 128 * 4;  // one row buffer per warp
+    static int wave_per_sm[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (wave_per_sm[dev] == 0) {
+      cudaError_t e =
+          cudaFuncSetAttribute(layer_norm_wave_kernel<V, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize, WSMEM);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(layer_norm_wave_kernel<V, OUT>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+      int n = 0;
+      if (e == cudaSuccess)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, layer_norm_wave_kernel<V, OUT>, 32 * kLnWaveWarps, WSMEM);
+      if (e != cudaSuccess) return e;
+      wave_per_sm[dev] = n > 0 ? n : -1;
+    }
+    int sms = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const long long need = (M + kLnWaveWarps - 1) / kLnWaveWarps;
+    if (wave_per_sm[dev] > 0 && need <= (long long)sms * wave_per_sm[dev])
+      return launch_pdl(layer_norm_wave_kernel<V, OUT>, dim3(static_cast<unsigned>(need)), dim3(32 * kLnWaveWarps),
+                        WSMEM, st, x, g, b, M, eps, y);
+  }
   constexpr int SMEM = (2 + 4) * V * 128 * 4;  // gamma, beta, four row buffers
   static int per_sm[64] = {0};                  // resident blocks per SM, per device
   int dev = 0;

@@ -229,7 +229,7 @@ def test_log_mel_ragged_frames():
 
 
 # ------------------------------------------------------------------ LN
-@pytest.mark.parametrize("M,D", [(1, 256), (77, 768), (6240, 1280), (5, 2048)])
+@pytest.mark.parametrize("M,D", [(1, 256), (77, 768), (6240, 1280), (5, 2048), (48000, 768), (20000, 1280)])
 def test_layer_norm(M, D):
     rng = np.random.default_rng(D + M)
     x = (rng.normal(size=(M, D)) * 3 + 0.5).astype(np.float32)
@@ -241,6 +241,22 @@ def test_layer_norm(M, D):
                          out_f32=True)
     np.testing.assert_allclose(y32.cpu().numpy(), ref, rtol=1e-4, atol=1e-4)
     assert np.abs(y16.float().cpu().numpy() - ref).max() <= 2.0 ** -8 * np.abs(ref).max()
+
+
+def test_layer_norm_forms_agree():
+    """Row counts that fit the SMs at once run the single-wave form (rows
+    staged in shared memory), larger ones the register form with prefetch:
+    the same arithmetic in the same order, so a row normalises to the same
+    bits in both."""
+    rng = np.random.default_rng(4)
+    D = 1280
+    big = torch.from_numpy((rng.normal(size=(40000, D)) * 2 + 0.3).astype(np.float32)).cuda()
+    g = torch.from_numpy((1 + 0.1 * rng.normal(size=D)).astype(np.float32)).cuda()
+    b = torch.from_numpy((0.02 * rng.normal(size=D)).astype(np.float32)).cuda()
+    small = big[:6240].contiguous()
+    y_big = sra.layer_norm(big, g, b)
+    y_small = sra.layer_norm(small, g, b)
+    assert torch.equal(y_big[:6240], y_small)
 
 
 # ------------------------------------------------------------------ attention
