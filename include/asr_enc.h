@@ -256,8 +256,10 @@ asr_status asr_enc_set_graphs(asr_enc* e, int enable);
  * stream is computed with the same additions as the unfused path; the
  * LayerNorm outputs differ by the summation order of the statistics (well
  * inside the encoder's tolerance), and so does everything downstream.
- * asr_enc_set_ln_fusion(e, 0) turns it off (the separate LayerNorm kernels
- * run instead; drops a recorded graph), 1 back on (default: on).
+ * asr_enc_set_ln_fusion(e, 1) turns it on, 0 off (the separate LayerNorm
+ * kernels run; either call drops a recorded graph).  Default: off — on one
+ * B200 the separate single-wave LayerNorm launches make the 16 x 30 s
+ * forward about 0.17 ms faster than the fused epilogue.
  * asr_enc_ln_fusion reports whether forwards use it (*active = 1) or not. */
 asr_status asr_enc_set_ln_fusion(asr_enc* e, int enable);
 asr_status asr_enc_ln_fusion(const asr_enc* e, int* active);

@@ -345,7 +345,7 @@ class Encoder:
         _check(lib.asr_enc_set_graphs(self.handle, 1 if enable else 0), self.handle)
 
     def set_ln_fusion(self, enable: bool):
-        """LayerNorms computed by the residual GEMMs' epilogues (default on where supported)."""
+        """Next-block LayerNorm computed in fc2's epilogue (default off; see asr_enc.h)."""
         _check(lib.asr_enc_set_ln_fusion(self.handle, 1 if enable else 0), self.handle)
 
     def ln_fusion(self) -> bool:

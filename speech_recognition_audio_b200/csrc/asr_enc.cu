@@ -286,9 +286,10 @@ struct asr_enc {
   // across chunk boundaries (no partly empty tiles).
   bool packed = false;
   // fc2 of every block also writes the next LayerNorm's output (EPI_LN):
-  // possible for 16-bit weights of suitable shape (ln_fuse), on unless
-  // asr_enc_set_ln_fusion turned it off.
-  bool ln_fuse = false, ln_fuse_on = true;
+  // possible for 16-bit weights of suitable shape (ln_fuse), used when
+  // asr_enc_set_ln_fusion turned it on (off by default: with the single-wave
+  // LayerNorm kernel the separate launches are faster).
+  bool ln_fuse = false, ln_fuse_on = false;
   float* pe = nullptr;
   int pe_rows = 0;
   std::vector<LayerW> layers;

@@ -184,11 +184,11 @@ def test_whisper_small_32x30s_sampled():
 
 @pytest.mark.parametrize("wname", ["moss_1x30s", "tiny_f16"])
 def test_ln_fusion_matches_separate_layernorms(wname):
-    """16-bit encoders compute each block's first LayerNorm (and the head's)
-    in the previous fc2's epilogue; with that turned off the separate
-    LayerNorm kernels run.  Both match the oracle, and they agree closely
-    with each other (they differ only by the order in which the row
-    statistics are summed)."""
+    """16-bit encoders can compute each block's first LayerNorm (and the
+    head's) in the previous fc2's epilogue (asr_enc_set_ln_fusion; off by
+    default, when the separate LayerNorm kernels run).  Both match the
+    oracle, and they agree closely with each other (they differ only by the
+    order in which the row statistics are summed)."""
     if wname == "tiny_f16":
         base = synth.GEOMETRIES["tiny"].as_dict()
         base.update(dtype=synth.DTYPE_F16)
@@ -199,6 +199,8 @@ def test_ln_fusion_matches_separate_layernorms(wname):
     else:
         enc, W, g = _encoder(wname)
         pcm = synth.pcm_batch(synth.WORKLOADS[wname])
+    assert not enc.ln_fusion()
+    enc.set_ln_fusion(True)
     assert enc.ln_fusion()
     fused = _run(enc, pcm)
     enc.set_ln_fusion(False)
@@ -206,6 +208,7 @@ def test_ln_fusion_matches_separate_layernorms(wname):
     plain = _run(enc, pcm)
     enc.set_ln_fusion(True)
     again = _run(enc, pcm)
+    enc.set_ln_fusion(False)
     np.testing.assert_array_equal(fused, again)
     ref = oracle.forward(pcm, W, g)
     assert_encoder_parity(fused, ref, f"{wname} LayerNorm epilogue")
@@ -217,7 +220,9 @@ def test_ln_fusion_matches_separate_layernorms(wname):
 
 def test_fp32_weights_keep_separate_layernorms():
     enc, W, g = _encoder("tiny_1x1s")
-    assert not enc.ln_fusion()
+    enc.set_ln_fusion(True)
+    assert not enc.ln_fusion()  # kind::tf32 has no LayerNorm epilogue
+    enc.set_ln_fusion(False)
 
 
 def test_host_forward_matches_device_forward():
