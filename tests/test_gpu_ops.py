@@ -278,6 +278,30 @@ def test_attention(lens, H):
         np.testing.assert_allclose(got[0], q[0, 2 * d:], atol=1e-2)
 
 
+@pytest.mark.parametrize("case", ["windows_16x30s", "ragged"])
+def test_attention_many_items_per_block(case):
+    """Many more (segment, head) blocks than fit on the GPU at once: the
+    16 x 30 s window layout (64 windows x 20 heads, several waves of blocks)
+    and a ragged mix of 150 segments of 1..128 tokens, element by element
+    against the oracle, and the same bits from a second call."""
+    rng = np.random.default_rng(11 if case == "ragged" else 12)
+    if case == "ragged":
+        lens, H = [int(v) for v in rng.integers(1, 129, size=150)], 7
+    else:
+        lens, H = [104, 104, 104, 78] * 16, 20
+    T = sum(lens)
+    qkv = _bf16(rng.normal(size=(T, 3 * H * 64)))
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    got = sra.attention(qkv.cuda(), torch.from_numpy(cu).cuda(), H).float().cpu().numpy()
+    q = qkv.float().numpy()
+    d = H * 64
+    ref = oracle.attention_windows(q[:, :d], q[:, d:2 * d], q[:, 2 * d:], cu, H)
+    assert np.abs(got - ref).max() <= 2e-2
+    # a second call on the same inputs gives the same bits
+    again = sra.attention(qkv.cuda(), torch.from_numpy(cu).cuda(), H).float().cpu().numpy()
+    assert np.array_equal(got, again)
+
+
 @pytest.mark.parametrize("lens,H", [([200, 300, 257, 1], 2), ([1500], 3), ([130, 129, 384, 385], 1)])
 def test_attention_long_segments(lens, H):
     """Segments longer than one 128-key tile run on the flash kernel (online
