@@ -149,9 +149,9 @@ def test_moss_1x30s_full():
     assert_encoder_parity(out, ref, "moss 1x30s")
 
 
-def _sampled(wname, picks):
+def _sampled(wname, picks, affine=False, seed=None):
     w = synth.WORKLOADS[wname]
-    enc, W, g = _encoder(wname)
+    enc, W, g = _encoder(wname, affine=affine, seed=seed)
     pcm = synth.pcm_batch(w)
     enc.set_taps(1 << sra.TAP_MEL)
     out = _run(enc, pcm)
@@ -180,6 +180,15 @@ def test_moss_1x600s_sampled():
 
 def test_whisper_small_32x30s_sampled():
     _sampled("whisper_small_32x30s", [(0, None), (31, None)])
+
+
+@pytest.mark.parametrize("wname,picks", [("moss_16x30s", [(2, 1), (13, 3)]), ("whisper_small_32x30s", [(5, None)])])
+def test_affine_biases_full_size_sampled(wname, picks):
+    """Non-zero biases and LayerNorm gains and shifts at full size, in the
+    benchmark's launch configuration: the CTA-pair tiles, the conv-box stem
+    GEMMs, the split QKV projection, stream-K fc2 (d = 1280) and the flash
+    attention path (whisper-small) all carry bias signal end to end."""
+    _sampled(wname, picks, affine=True, seed=91)
 
 
 @pytest.mark.parametrize("wname", ["moss_1x30s", "tiny_f16"])
