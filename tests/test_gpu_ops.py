@@ -302,6 +302,31 @@ def test_attention_many_items_per_block(case):
     assert np.array_equal(got, again)
 
 
+def test_attention_large_orthogonal_rows():
+    """Head 0 has query and key rows of norm 300 along different axes, so
+    their scores come only from small components and sit far below the
+    product of the norms (a softmax shifted by a norm bound instead of the
+    row maximum would underflow here).  Head 1 is ordinary; both are
+    compared with the oracle element by element."""
+    rng = np.random.default_rng(21)
+    H, lens = 2, [104, 104, 57, 1]
+    T, d = sum(lens), 2 * 64
+    q = rng.normal(size=(T, d)) * 0.6
+    k = rng.normal(size=(T, d)) * 0.6
+    q[:, :64] *= 0.05
+    k[:, :64] *= 0.05
+    q[:, 0] = 300.0
+    k[:, 1] = 300.0
+    v = rng.normal(size=(T, d))
+    qkv = _bf16(np.concatenate([q, k, v], axis=1))
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    got = sra.attention(qkv.cuda(), torch.from_numpy(cu).cuda(), H).float().cpu().numpy()
+    x = qkv.float().numpy()
+    ref = oracle.attention_windows(x[:, :d], x[:, d:2 * d], x[:, 2 * d:], cu, H)
+    assert np.isfinite(got).all()
+    assert np.abs(got - ref).max() <= 2e-2
+
+
 @pytest.mark.parametrize("lens,H", [([200, 300, 257, 1], 2), ([1500], 3), ([130, 129, 384, 385], 1)])
 def test_attention_long_segments(lens, H):
     """Segments longer than one 128-key tile run on the flash kernel (online
